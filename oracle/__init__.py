@@ -1,0 +1,189 @@
+"""GSA oracle — TEST INFRASTRUCTURE ONLY.
+
+Python marshalling around ``gsa_oracle.c`` (plain C, fp64).  Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package; the CUDA library and its binding never do.
+
+Inputs are numpy arrays in their storage type (fp32, or bf16 bit patterns in
+uint16); the C code widens each element exactly to double.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gsa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+F32, BF16, F64 = 0, 1, 2
+ALL_GISTS, SELECTED_PAIRS = 0, 1
+_DT = {"f32": F32, "bf16": BF16, "f64": F64}
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` (gcc -O2, IEEE fp64, OpenMP over rows)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    L = ctypes.CDLL(_LIB)
+    i, i64, d, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+    sig = {
+        "oracle_gist_scores": [i, i, i, i, i, i, vp, vp, vp],
+        "oracle_topk": [i, i, i, vp, vp],
+        "oracle_topk_gap": [i, i, i, vp, vp],
+        "oracle_score_error_bound": [i, i, i, i, i, i, vp, vp, vp],
+        "oracle_decode": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
+        "oracle_unfold_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 9,
+        "oracle_hier_decode": [i, i, i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12,
+        "oracle_gist_mask": [i64, i64, i],
+        "oracle_prefill_pair_count": [i, i],
+        "oracle_prefill_rows": [i, i, i, i, i, i, d, i, vp, vp, vp, i64, vp, vp],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = None
+    L.oracle_gist_mask.restype = i
+    L.oracle_prefill_pair_count.restype = i64
+    _lib = L
+    return L
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert isinstance(a, np.ndarray) and a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data
+
+
+def _dtcode(a: np.ndarray) -> int:
+    if a.dtype == np.float64:
+        return F64
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    raise TypeError(a.dtype)
+
+
+# --- step 1: routing scores -------------------------------------------------
+def gist_scores(q: np.ndarray, k_gist: np.ndarray) -> np.ndarray:
+    """q [B,Hq,d], k_gist [B,Hkv,N,d] -> s [B,Hkv,N] fp64."""
+    B, Hq, d = q.shape
+    _, Hkv, N, _ = k_gist.shape
+    s = np.empty((B, Hkv, N), np.float64)
+    _load().oracle_gist_scores(B, Hq, Hkv, d, N, _dtcode(q), _p(q), _p(k_gist), _p(s))
+    return s
+
+
+# --- step 2: selection ------------------------------------------------------
+def topk(scores: np.ndarray, k: int) -> np.ndarray:
+    """scores [..., N] fp64 -> idx [..., k] int32, ascending; ties -> lowest index."""
+    s = np.ascontiguousarray(scores, np.float64)
+    N = s.shape[-1]
+    rows = int(np.prod(s.shape[:-1])) if s.ndim > 1 else 1
+    idx = np.empty(s.shape[:-1] + (k,), np.int32)
+    _load().oracle_topk(rows, N, k, _p(s), _p(idx))
+    return idx
+
+
+def topk_gap(scores: np.ndarray, k: int) -> np.ndarray:
+    s = np.ascontiguousarray(scores, np.float64)
+    N = s.shape[-1]
+    rows = int(np.prod(s.shape[:-1])) if s.ndim > 1 else 1
+    gap = np.empty(s.shape[:-1], np.float64)
+    _load().oracle_topk_gap(rows, N, k, _p(s), _p(gap))
+    return gap
+
+
+def score_error_bound(q: np.ndarray, k_gist: np.ndarray) -> np.ndarray:
+    """Per (b, hk): bound on |fp32 score - exact score| for any summation order."""
+    B, Hq, d = q.shape
+    _, Hkv, N, _ = k_gist.shape
+    eps = np.empty((B, Hkv), np.float64)
+    _load().oracle_score_error_bound(B, Hq, Hkv, d, N, _dtcode(q), _p(q), _p(k_gist), _p(eps))
+    return eps
+
+
+# --- steps 1-4: decode --------------------------------------------------------
+def decode(t: dict, top_k: int, mode: int = ALL_GISTS, scale: float = 0.0):
+    """Flat decode step.  t: q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail.
+    Returns (scores [B,Hkv,N], idx [B,Hkv,k], out [B,Hq,d]) in fp64 / int32."""
+    q, kg = t["q"], t["k_gist"]
+    B, Hq, d = q.shape
+    _, Hkv, N, c, _ = t["k_raw"].shape
+    W = t["k_tail"].shape[2]
+    s = np.empty((B, Hkv, N), np.float64)
+    idx = np.empty((B, Hkv, top_k), np.int32)
+    out = np.empty((B, Hq, d), np.float64)
+    _load().oracle_decode(B, Hq, Hkv, d, N, c, top_k, W, mode, scale, _dtcode(q), _p(q), _p(kg),
+                          _p(t["v_gist"]), _p(t["k_raw"]), _p(t["v_raw"]), _p(t["k_tail"]),
+                          _p(t["v_tail"]), _p(s), _p(idx), _p(out))
+    return s, idx, out
+
+
+def unfold_attn(t: dict, idx: np.ndarray, mode: int = ALL_GISTS, scale: float = 0.0) -> np.ndarray:
+    q = t["q"]
+    B, Hq, d = q.shape
+    _, Hkv, N, c, _ = t["k_raw"].shape
+    W = t["k_tail"].shape[2]
+    k = idx.shape[-1]
+    idx = np.ascontiguousarray(idx, np.int32)
+    out = np.empty((B, Hq, d), np.float64)
+    _load().oracle_unfold_attn(B, Hq, Hkv, d, N, c, k, W, mode, scale, _dtcode(q), _p(q),
+                               _p(t["k_gist"]), _p(t["v_gist"]), _p(t["k_raw"]), _p(t["v_raw"]),
+                               _p(t["k_tail"]), _p(t["v_tail"]), _p(idx), _p(out))
+    return out
+
+
+def hier_decode(t: dict, group: int, top_k2: int, top_k1: int, scale: float = 0.0):
+    """t: q, k_g2, v_g2, k_g1, v_g1, k_raw, v_raw, k_tail, v_tail.
+    Returns (idx2 [B,Hkv,k2], idx1 [B,Hkv,k1], out [B,Hq,d])."""
+    q = t["q"]
+    B, Hq, d = q.shape
+    _, Hkv, N1, c, _ = t["k_raw"].shape
+    n_l2 = t["k_g2"].shape[2]
+    W = t["k_tail"].shape[2]
+    idx2 = np.empty((B, Hkv, top_k2), np.int32)
+    idx1 = np.empty((B, Hkv, top_k1), np.int32)
+    out = np.empty((B, Hq, d), np.float64)
+    _load().oracle_hier_decode(B, Hq, Hkv, d, N1, c, top_k1, W, n_l2, group, top_k2, scale,
+                               _dtcode(q), _p(q), _p(t["k_g2"]), _p(t["v_g2"]), _p(t["k_g1"]),
+                               _p(t["v_g1"]), _p(t["k_raw"]), _p(t["v_raw"]), _p(t["k_tail"]),
+                               _p(t["v_tail"]), _p(idx2), _p(idx1), _p(out))
+    return idx2, idx1, out
+
+
+# --- prefill ------------------------------------------------------------------
+def gist_mask(p: int, t: int, chunk: int) -> bool:
+    return bool(_load().oracle_gist_mask(p, t, chunk))
+
+
+def prefill_pair_count(n_chunks: int, chunk: int) -> int:
+    return int(_load().oracle_prefill_pair_count(n_chunks, chunk))
+
+
+def prefill_rows(t: dict, n_chunks: int, chunk: int, rows: np.ndarray, scale: float = 0.0) -> np.ndarray:
+    """rows: int64 [n, 3] of (b, h, p).  Returns [n, d] fp64."""
+    q, k, v = t["q"], t["k"], t["v"]
+    B, Hq, P, d = q.shape
+    Hkv = k.shape[1]
+    assert P == n_chunks * (chunk + 1)
+    rows = np.ascontiguousarray(rows, np.int64)
+    out = np.empty((rows.shape[0], d), np.float64)
+    _load().oracle_prefill_rows(B, Hq, Hkv, d, n_chunks, chunk, scale, _dtcode(q), _p(q), _p(k),
+                                _p(v), rows.shape[0], _p(rows), _p(out))
+    return out

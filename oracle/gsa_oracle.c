@@ -1,0 +1,377 @@
+/*
+ * GSA oracle — TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, fp64 CPU restatement of what the Gist Sparse Attention (GSA)
+ * decode path and the gist-causal prefill compute.  Only the tests, the smoke
+ * check and the bench's CPU-baseline leg call it; the CUDA library never links
+ * or calls it and shares no code with it.
+ *
+ * Sources (pages about "Forget, Then Recall: Learnable Compression and
+ * Selective Unfolding via Gist Sparse Attention", Mao, Li & Fox):
+ *   [EN-2]   gist.science explainer (EN), section 2 "Methodology: Gist Sparse
+ *            Attention" — interleaved gist tokens, gist as routing signals,
+ *            selective unfolding, hybrid attention, hierarchical extension;
+ *   [DE-M]   gist.science explainer (DE), section "Methodik";
+ *   [SL-6]   Taki-lab slide deck (docswell), page 6 "GSA とは" — query scores
+ *            every gist, takes top-k, restores the chunks with their gists;
+ *   [SL-7]   slide deck, page 7 "Gist token" — gist causal mask example;
+ *   [SL-9]   slide deck, page 9 "Training, Stage 1" — the suffix sees gists only;
+ *   [SL-10]  slide deck, page 10 "Training, Stage 2" — top-k worked example;
+ *   [SL-11]  slide deck, page 11 "Hierarchical Gist-of-Gist Compression";
+ *   [SL-17]  slide deck, page 17 "Selective Rules Comparison" — SR-only,
+ *            AG+SR, SG+SR.
+ *
+ * Every floating-point value is widened exactly to double before use; all
+ * arithmetic is in double.  Softmax is the two-pass textbook form.
+ * Parity status of each function is stated beside it; all are pinned by the
+ * CPU tests (worked examples, closed forms, brute force, library routines).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
+enum { OR_ALL_GISTS = 0, OR_SELECTED_PAIRS = 1 };
+
+/* Exact widening of one stored element to double. */
+static double ld(const void* p, int dt, int64_t i) {
+    if (dt == OR_F64) return ((const double*)p)[i];
+    if (dt == OR_F32) return (double)((const float*)p)[i];
+    uint32_t u = (uint32_t)((const uint16_t*)p)[i] << 16; /* bf16 bits */
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+static double default_scale(double scale, int d) { return scale > 0 ? scale : 1.0 / sqrt((double)d); }
+
+/* ------------------------------------------------------------------------ */
+/* Step 1 — routing score of every gist.  [EN-2] "Gist as Routing Signals":   */
+/* the decoding query is scored against every gist token; [DE-M] "Relevanz-  */
+/* Scoring": by dot product with the gist key.  Under grouped-query sharing   */
+/* the G query heads of one KV head share one selection, so the score of     */
+/* gist j for KV head hk is the sum over the group of the raw logits:        */
+/*        s[b,hk,j] = sum_{h in group(hk)} sum_i q[b,h,i] * Kg[b,hk,j,i].    */
+/* (No softmax scale: a positive scale does not change the ranking.)         */
+/* ------------------------------------------------------------------------ */
+static double gist_score(int Hq, int Hkv, int d, int N, int dt, const void* q, const void* kg,
+                         int b, int hk, int j) {
+    int G = Hq / Hkv;
+    double acc = 0.0;
+    for (int g = 0; g < G; ++g) {
+        int h = hk * G + g;
+        for (int i = 0; i < d; ++i)
+            acc += ld(q, dt, ((int64_t)b * Hq + h) * d + i) *
+                   ld(kg, dt, (((int64_t)b * Hkv + hk) * N + j) * d + i);
+    }
+    return acc;
+}
+
+void oracle_gist_scores(int B, int Hq, int Hkv, int d, int N, int dt, const void* q, const void* kg,
+                        double* s) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk)
+            for (int j = 0; j < N; ++j)
+                s[((int64_t)b * Hkv + hk) * N + j] = gist_score(Hq, Hkv, d, N, dt, q, kg, b, hk, j);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 2 — top-k chunk selection.  [EN-2] "Selective Unfolding": the k most  */
+/* relevant chunks by score; [SL-10] scores 0.1/0.8/0.7/0.2, k=2 -> g2, g3.   */
+/* Ties go to the lowest index; the result is listed in ascending order.     */
+/* Implementation: sort every (score, index) pair by score descending, index  */
+/* ascending; keep the first k; sort those indices ascending.  NaN ranks     */
+/* below every number.                                                       */
+/* ------------------------------------------------------------------------ */
+typedef struct { double s; int32_t j; } scored_t;
+
+static int by_score_desc_then_index(const void* a, const void* b) {
+    const scored_t* x = (const scored_t*)a;
+    const scored_t* y = (const scored_t*)b;
+    int xn = isnan(x->s), yn = isnan(y->s);
+    if (xn != yn) return xn ? 1 : -1;
+    if (!xn && x->s != y->s) return x->s > y->s ? -1 : 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+static int by_index(const void* a, const void* b) {
+    int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+    return (x > y) - (x < y);
+}
+
+/* Top-k of n scores whose positions are idx_of[0..n) (NULL: 0..n-1). */
+static void topk_list(int n, const double* s, const int32_t* idx_of, int k, int32_t* out) {
+    scored_t* all = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n > 0 ? n : 1));
+    for (int t = 0; t < n; ++t) {
+        all[t].s = s[t];
+        all[t].j = idx_of ? idx_of[t] : t;
+    }
+    qsort(all, (size_t)n, sizeof(scored_t), by_score_desc_then_index);
+    for (int t = 0; t < k; ++t) out[t] = all[t].j;
+    qsort(out, (size_t)k, sizeof(int32_t), by_index);
+    free(all);
+}
+
+void oracle_topk(int rows, int N, int k, const double* s, int32_t* idx) {
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) topk_list(N, s + (int64_t)r * N, NULL, k, idx + (int64_t)r * k);
+}
+
+/* Selection margin of one row: the gap between the k-th and (k+1)-th largest */
+/* score (INFINITY when k = 0 or k = n).  Test helper for the decidability     */
+/* rule on selected indices.                                                  */
+void oracle_topk_gap(int rows, int N, int k, const double* s, double* gap) {
+    for (int r = 0; r < rows; ++r) {
+        if (k <= 0 || k >= N) { gap[r] = INFINITY; continue; }
+        scored_t* all = (scored_t*)malloc(sizeof(scored_t) * (size_t)N);
+        for (int t = 0; t < N; ++t) { all[t].s = s[(int64_t)r * N + t]; all[t].j = t; }
+        qsort(all, (size_t)N, sizeof(scored_t), by_score_desc_then_index);
+        gap[r] = all[k - 1].s - all[k].s;
+        free(all);
+    }
+}
+
+/* Rounding-error bound of an fp32 evaluation of each score, any summation   */
+/* order (Higham, "Accuracy and Stability of Numerical Algorithms", 2nd ed., */
+/* eq. 3.5, inner products):  |fl(s) - s| <= gamma_n * sum |q_i k_i|,        */
+/* gamma_n = n u / (1 - n u), u = 2^-24, n = G*d products summed.  Per row,  */
+/* the maximum over the row's gists.                                         */
+void oracle_score_error_bound(int B, int Hq, int Hkv, int d, int N, int dt, const void* q,
+                              const void* kg, double* eps_row) {
+    int G = Hq / Hkv;
+    double u = ldexp(1.0, -24), n = (double)G * d;
+    double gamma = n * u / (1.0 - n * u);
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk) {
+            double worst = 0.0;
+            for (int j = 0; j < N; ++j) {
+                double acc = 0.0;
+                for (int g = 0; g < G; ++g)
+                    for (int i = 0; i < d; ++i)
+                        acc += fabs(ld(q, dt, ((int64_t)b * Hq + hk * G + g) * d + i) *
+                                    ld(kg, dt, (((int64_t)b * Hkv + hk) * N + j) * d + i));
+                if (acc > worst) worst = acc;
+            }
+            eps_row[(int64_t)b * Hkv + hk] = gamma * worst;
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Steps 3-4 — hybrid attention over the assembled context.                  */
+/* A context is a list of keys, each a (K row, V row) pair in some tensor.   */
+/* For each query head h of the group: l_x = scale * q_h . K_x,              */
+/* p_x = exp(l_x - max l) / sum exp(l - max l), out_h = sum_x p_x V_x.       */
+/* ------------------------------------------------------------------------ */
+typedef struct { const void* k; const void* v; int64_t off; } key_ref;
+
+static void attend(int d, int dt, double scale, const void* q, int64_t q_off, int nkeys,
+                   const key_ref* keys, double* out) {
+    double* logit = (double*)malloc(sizeof(double) * (size_t)(nkeys > 0 ? nkeys : 1));
+    double mx = -INFINITY;
+    for (int x = 0; x < nkeys; ++x) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += ld(q, dt, q_off + i) * ld(keys[x].k, dt, keys[x].off + i);
+        logit[x] = scale * acc;
+        if (logit[x] > mx) mx = logit[x];
+    }
+    double z = 0.0;
+    for (int x = 0; x < nkeys; ++x) { logit[x] = exp(logit[x] - mx); z += logit[x]; }
+    for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int x = 0; x < nkeys; ++x) acc += logit[x] * ld(keys[x].v, dt, keys[x].off + i);
+        out[i] = nkeys > 0 ? acc / z : NAN;
+    }
+    free(logit);
+}
+
+/* Context of one (b, hk) for flat decode.
+ * [EN-2] "Hybrid Attention": k raw chunks + their gist tokens + the gist
+ * tokens of unselected chunks  -> ALL_GISTS = every gist once, plus the raw
+ * tokens of the selected chunks ([SL-17] "AG+SR").
+ * [SL-6] / [SL-17] "SG+SR": only the selected chunks' gists and raw tokens
+ * -> SELECTED_PAIRS.
+ * In both modes the W uncompressed tail tokens after the last chunk are
+ * always attended ([SL-9]: the generation suffix attends directly).          */
+static int flat_context(int Hkv, int d, int N, int c, int W, int mode, int b, int hk, int k,
+                        const int32_t* sel, const void* kg, const void* vg, const void* kraw,
+                        const void* vraw, const void* ktail, const void* vtail, key_ref* keys) {
+    int n = 0;
+    int64_t row = (int64_t)b * Hkv + hk;
+    if (mode == OR_ALL_GISTS) {
+        for (int j = 0; j < N; ++j) keys[n++] = (key_ref){kg, vg, (row * N + j) * d};
+    } else {
+        for (int t = 0; t < k; ++t) keys[n++] = (key_ref){kg, vg, (row * N + sel[t]) * d};
+    }
+    for (int t = 0; t < k; ++t)
+        for (int u = 0; u < c; ++u)
+            keys[n++] = (key_ref){kraw, vraw, ((row * N + sel[t]) * c + u) * d};
+    for (int u = 0; u < W; ++u) keys[n++] = (key_ref){ktail, vtail, (row * W + u) * d};
+    return n;
+}
+
+/* Full flat decode step: scores (step 1), selection (step 2), hybrid
+ * attention (steps 3-4).  Outputs: scores [B*Hkv*N] (may be NULL), selected
+ * indices [B*Hkv*k] ascending, out [B*Hq*d].                                */
+void oracle_decode(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode, double scale,
+                   int dt, const void* q, const void* kg, const void* vg, const void* kraw,
+                   const void* vraw, const void* ktail, const void* vtail, double* scores_out,
+                   int32_t* idx_out, double* out) {
+    int G = Hq / Hkv;
+    double sc = default_scale(scale, d);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk) {
+            int64_t row = (int64_t)b * Hkv + hk;
+            double* s = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+            for (int j = 0; j < N; ++j) s[j] = gist_score(Hq, Hkv, d, N, dt, q, kg, b, hk, j);
+            if (scores_out)
+                for (int j = 0; j < N; ++j) scores_out[row * N + j] = s[j];
+            int32_t* sel = idx_out + row * k;
+            topk_list(N, s, NULL, k, sel);
+            key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(N + (int64_t)k * c + W + 1));
+            int nk = flat_context(Hkv, d, N, c, W, mode, b, hk, k, sel, kg, vg, kraw, vraw, ktail,
+                                  vtail, keys);
+            for (int g = 0; g < G; ++g) {
+                int h = hk * G + g;
+                attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
+                       out + ((int64_t)b * Hq + h) * d);
+            }
+            free(keys);
+            free(s);
+        }
+}
+
+/* Hybrid attention alone, for a given selection idx [B*Hkv*k] (the unfolding
+ * + attention step without routing).                                         */
+void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode,
+                        double scale, int dt, const void* q, const void* kg, const void* vg,
+                        const void* kraw, const void* vraw, const void* ktail, const void* vtail,
+                        const int32_t* idx, double* out) {
+    int G = Hq / Hkv;
+    double sc = default_scale(scale, d);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk) {
+            int64_t row = (int64_t)b * Hkv + hk;
+            key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(N + (int64_t)k * c + W + 1));
+            int nk = flat_context(Hkv, d, N, c, W, mode, b, hk, k, idx + row * k, kg, vg, kraw, vraw,
+                                  ktail, vtail, keys);
+            for (int g = 0; g < G; ++g) {
+                int h = hk * G + g;
+                attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
+                       out + ((int64_t)b * Hq + h) * d);
+            }
+            free(keys);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Hierarchical gist-of-gist decode (H-GSA).  [EN-2] "Hierarchical Extension"*/
+/* and [DE-M] "Erweiterung": gists are grouped, a meta-gist summarises each  */
+/* group; decoding scores the meta-gists, selects segments, scores the gists */
+/* inside the selected segments, then unfolds raw tokens.  [SL-11]: groups  */
+/* of consecutive gists (g1..g10 -> G1, ...).                                */
+/*   level 2: s2[J] over all n_l2 meta-gists -> S2 = top-k2;                  */
+/*   candidates: level-1 gists j with floor(j / group) in S2, ascending;      */
+/*   level 1: s1[j] over the candidates -> S1 = top-k1 among them;            */
+/*   context: every meta-gist, every candidate gist, raw tokens of S1, tail.  */
+/* ------------------------------------------------------------------------ */
+void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, int W, int n_l2,
+                        int group, int k2, double scale, int dt, const void* q, const void* kg2,
+                        const void* vg2, const void* kg1, const void* vg1, const void* kraw,
+                        const void* vraw, const void* ktail, const void* vtail, int32_t* idx2_out,
+                        int32_t* idx1_out, double* out) {
+    int G = Hq / Hkv;
+    double sc = default_scale(scale, d);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk) {
+            int64_t row = (int64_t)b * Hkv + hk;
+            double* s2 = (double*)malloc(sizeof(double) * (size_t)n_l2);
+            for (int J = 0; J < n_l2; ++J) s2[J] = gist_score(Hq, Hkv, d, n_l2, dt, q, kg2, b, hk, J);
+            int32_t* S2 = idx2_out + row * k2;
+            topk_list(n_l2, s2, NULL, k2, S2);
+
+            int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * (size_t)k2 * group + 1);
+            int nc = 0;
+            for (int t = 0; t < k2; ++t)
+                for (int u = 0; u < group; ++u) {
+                    int j = S2[t] * group + u;
+                    if (j < N1) cand[nc++] = j;
+                }
+            double* s1 = (double*)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
+            for (int t = 0; t < nc; ++t) s1[t] = gist_score(Hq, Hkv, d, N1, dt, q, kg1, b, hk, cand[t]);
+            int32_t* S1 = idx1_out + row * k1;
+            topk_list(nc, s1, cand, k1, S1);
+
+            key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(n_l2 + nc + (int64_t)k1 * c + W + 1));
+            int nk = 0;
+            for (int J = 0; J < n_l2; ++J) keys[nk++] = (key_ref){kg2, vg2, (row * n_l2 + J) * d};
+            for (int t = 0; t < nc; ++t) keys[nk++] = (key_ref){kg1, vg1, (row * N1 + cand[t]) * d};
+            for (int t = 0; t < k1; ++t)
+                for (int u = 0; u < c; ++u)
+                    keys[nk++] = (key_ref){kraw, vraw, ((row * N1 + S1[t]) * c + u) * d};
+            for (int u = 0; u < W; ++u) keys[nk++] = (key_ref){ktail, vtail, (row * W + u) * d};
+            for (int g = 0; g < G; ++g) {
+                int h = hk * G + g;
+                attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
+                       out + ((int64_t)b * Hq + h) * d);
+            }
+            free(keys);
+            free(s1);
+            free(cand);
+            free(s2);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gist-causal prefill.  [EN-2] "Interleaved Gist Tokens": the sequence is   */
+/* cut into chunks of c tokens and a gist token follows every chunk; a       */
+/* gist attends only to its own chunk and to earlier gists.  [SL-7]:         */
+/* g1 -> x1,x2; g2 -> g1,x3,x4; g3 -> g1,g2,x5,(x6),g3.  [SL-9]: a token that */
+/* follows compressed context sees the gists, not the earlier raw tokens.     */
+/* Positions p = 0..N(c+1)-1: chunk(p) = p / (c+1); p is a gist iff          */
+/* p mod (c+1) == c.  Query p may attend key t iff t <= p and                */
+/*   (t is a gist of an earlier chunk) or (t == p) or                         */
+/*   (t is a raw token of p's own chunk).                                    */
+/* ------------------------------------------------------------------------ */
+int oracle_gist_mask(int64_t p, int64_t t, int c) {
+    if (t > p) return 0;
+    if (t == p) return 1;
+    int64_t cp = p / (c + 1), ct = t / (c + 1);
+    int t_gist = (t % (c + 1)) == c;
+    if (t_gist) return ct < cp;
+    return ct == cp;
+}
+
+/* Brute-force count of allowed (query, key) pairs in one sequence. */
+int64_t oracle_prefill_pair_count(int N, int c) {
+    int64_t P = (int64_t)N * (c + 1), n = 0;
+    for (int64_t p = 0; p < P; ++p)
+        for (int64_t t = 0; t <= p; ++t) n += oracle_gist_mask(p, t, c);
+    return n;
+}
+
+/* Prefill output of the listed query rows.  rows: n_rows triples (b, h, p);
+ * out: n_rows * d.  q [B][Hq][P][d], k, v [B][Hkv][P][d].                     */
+void oracle_prefill_rows(int B, int Hq, int Hkv, int d, int N, int c, double scale, int dt,
+                         const void* q, const void* k, const void* v, int64_t n_rows,
+                         const int64_t* rows, double* out) {
+    int G = Hq / Hkv;
+    int64_t P = (int64_t)N * (c + 1);
+    double sc = default_scale(scale, d);
+    (void)B;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t b = rows[3 * r], h = rows[3 * r + 1], p = rows[3 * r + 2];
+        int64_t hk = h / G;
+        key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(p + 1));
+        int nk = 0;
+        for (int64_t t = 0; t <= p; ++t)
+            if (oracle_gist_mask(p, t, c)) keys[nk++] = (key_ref){k, v, ((b * Hkv + hk) * P + t) * d};
+        attend(d, dt, sc, q, ((b * Hq + h) * P + p) * d, nk, keys, out + r * d);
+        free(keys);
+    }
+}

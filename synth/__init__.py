@@ -1,0 +1,319 @@
+"""Seeded synthetic inputs for the GSA decode / prefill workloads.
+
+This package only produces numbers: standard normals from a counter-based
+generator (``synth.c``), needle planting along a query direction, and the
+workload shape table.  It holds none of the attention method's arithmetic and
+is imported by both sides of every parity check (the CUDA library's callers
+and the oracle's callers), so the two see byte-identical inputs.
+
+Storage conventions (host numpy arrays):
+  * fp32 tensors are ``numpy.float32``;
+  * bf16 tensors are ``numpy.uint16`` holding the bf16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field, replace
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "synth.c")
+_LIB = os.path.join(_HERE, "libsynth.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``libsynth.so`` next to its source (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        u64, i64, vp = ctypes.c_uint64, ctypes.c_int64, ctypes.c_void_p
+        lib.synth_u64.restype = u64
+        lib.synth_u64.argtypes = [u64, u64, u64]
+        for name in ("synth_normal_f64", "synth_normal_f32", "synth_normal_bf16"):
+            f = getattr(lib, name)
+            f.restype = None
+            f.argtypes = [u64, u64, u64, i64, vp]
+        for name in ("synth_round_f32", "synth_round_bf16"):
+            f = getattr(lib, name)
+            f.restype = None
+            f.argtypes = [vp, i64, vp]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def normal(seed: int, stream: int, shape, dtype: str, offset: int = 0) -> np.ndarray:
+    """Standard normals for (seed, stream), element i of the flattened shape
+    taking counter ``offset + i``.  dtype: 'f64' | 'f32' | 'bf16'."""
+    lib = _load()
+    n = int(np.prod(shape)) if len(shape) else 1
+    if dtype == "f64":
+        out = np.empty(shape, np.float64)
+        lib.synth_normal_f64(seed, stream, offset, n, _ptr(out))
+    elif dtype == "f32":
+        out = np.empty(shape, np.float32)
+        lib.synth_normal_f32(seed, stream, offset, n, _ptr(out))
+    elif dtype == "bf16":
+        out = np.empty(shape, np.uint16)
+        lib.synth_normal_bf16(seed, stream, offset, n, _ptr(out))
+    else:
+        raise ValueError(dtype)
+    return out
+
+
+def u64(seed: int, stream: int, i: int) -> int:
+    return int(_load().synth_u64(seed, stream, i))
+
+
+def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round fp64 values to the storage dtype (fp32 RNE; bf16 RNE via fp32)."""
+    x = np.ascontiguousarray(x, np.float64)
+    lib = _load()
+    if dtype == "f32":
+        out = np.empty(x.shape, np.float32)
+        lib.synth_round_f32(_ptr(x), x.size, _ptr(out))
+    elif dtype == "bf16":
+        out = np.empty(x.shape, np.uint16)
+        lib.synth_round_bf16(_ptr(x), x.size, _ptr(out))
+    else:
+        raise ValueError(dtype)
+    return out
+
+
+def widen(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact widening of stored values to fp64 (bf16 bits -> fp32 -> fp64)."""
+    if dtype == "bf16":
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Workload shapes
+# ---------------------------------------------------------------------------
+ALL_GISTS, SELECTED_PAIRS = 0, 1
+
+# stream ids, one per generated tensor
+S_Q, S_KG, S_VG, S_KR, S_VR, S_KT, S_VT, S_NEEDLE_IDX, S_NEEDLE_NOISE = range(1, 10)
+S_KG2, S_VG2, S_NEEDLE2_NOISE = 10, 11, 12
+S_PQ, S_PK, S_PV = 20, 21, 22
+
+
+@dataclass(frozen=True)
+class DecodeShape:
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    n_chunks: int          # N gists, one per chunk
+    chunk: int             # c raw tokens per chunk
+    top_k: int
+    tail_len: int          # W uncompressed local tokens after the chunks
+    dtype: str = "bf16"    # 'f32' | 'bf16'
+    mode: int = ALL_GISTS
+    n_needles: int = 0
+    needle_alpha: float = 3.0
+    scale: float = 0.0     # <= 0: 1/sqrt(head_dim)
+
+    @property
+    def group(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    @property
+    def rows(self) -> int:
+        return self.batch * self.n_kv_heads
+
+
+@dataclass(frozen=True)
+class HierShape:
+    l1: DecodeShape        # level-1 gists, raw chunks, tail; l1.top_k = k1
+    n_l2: int              # level-2 (meta) gists
+    group: int             # level-1 gists per level-2 gist
+    top_k2: int
+
+
+@dataclass(frozen=True)
+class PrefillShape:
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    n_chunks: int
+    chunk: int
+    dtype: str = "bf16"
+    scale: float = 0.0
+
+    @property
+    def positions(self) -> int:
+        return self.n_chunks * (self.chunk + 1)
+
+
+# The five workloads (shapes, dtypes, needles).
+WORKLOADS = {
+    "tiny_f32": DecodeShape(1, 4, 1, 64, 128, 16, 4, 16, "f32", ALL_GISTS, n_needles=4),
+    "llama8b_decode": DecodeShape(8, 32, 8, 128, 2048, 16, 16, 64, "bf16", ALL_GISTS, n_needles=16),
+    # compression-ratio sweep: 131072 raw tokens, k*c = 2048 unfolded tokens
+    "sweep_c8_all": DecodeShape(4, 32, 8, 128, 16384, 8, 256, 128, "bf16", ALL_GISTS, n_needles=256),
+    "sweep_c16_all": DecodeShape(4, 32, 8, 128, 8192, 16, 128, 128, "bf16", ALL_GISTS, n_needles=128),
+    "sweep_c32_all": DecodeShape(4, 32, 8, 128, 4096, 32, 64, 128, "bf16", ALL_GISTS, n_needles=64),
+    "sweep_c8_pairs": DecodeShape(4, 32, 8, 128, 16384, 8, 256, 128, "bf16", SELECTED_PAIRS, n_needles=256),
+    "sweep_c16_pairs": DecodeShape(4, 32, 8, 128, 8192, 16, 128, 128, "bf16", SELECTED_PAIRS, n_needles=128),
+    "sweep_c32_pairs": DecodeShape(4, 32, 8, 128, 4096, 32, 64, 128, "bf16", SELECTED_PAIRS, n_needles=64),
+    "hier_1m": HierShape(DecodeShape(1, 32, 8, 128, 65536, 16, 8, 128, "bf16", ALL_GISTS, n_needles=8),
+                         n_l2=4096, group=16, top_k2=8),
+    "gist_prefill": PrefillShape(2, 32, 8, 128, 1024, 16, "bf16"),
+}
+
+# workload -> index in the published config list (seeds 20260422 + 100*cfg + rep)
+CONFIG_INDEX = {"tiny_f32": 1, "llama8b_decode": 2, "sweep_c8_all": 3, "sweep_c16_all": 3,
+                "sweep_c32_all": 3, "sweep_c8_pairs": 3, "sweep_c16_pairs": 3,
+                "sweep_c32_pairs": 3, "hier_1m": 4, "gist_prefill": 5}
+
+
+def seed_for(workload: str, rep: int = 0) -> int:
+    return 20260422 + 100 * CONFIG_INDEX[workload] + rep
+
+
+def _distinct_draws(seed: int, stream: int, base: int, count: int, modulus: int) -> list:
+    """`count` distinct values in [0, modulus) from successive draws."""
+    assert count <= modulus
+    out, seen, i = [], set(), 0
+    while len(out) < count:
+        v = u64(seed, stream, base + i) % modulus
+        i += 1
+        if v not in seen:
+            seen.add(v)
+            out.append(v)
+    return out
+
+
+def _needle_keys(q_wide: np.ndarray, b: int, hk: int, G: int, alpha: float, noise: np.ndarray) -> np.ndarray:
+    """alpha * qbar/|qbar| + 0.1 * noise, qbar = sum of the group's query heads."""
+    qbar = q_wide[b, hk * G:(hk + 1) * G, :].sum(axis=0)
+    return alpha * qbar / np.linalg.norm(qbar) + 0.1 * noise
+
+
+@dataclass
+class DecodeInputs:
+    shape: DecodeShape
+    q: np.ndarray
+    k_gist: np.ndarray
+    v_gist: np.ndarray
+    k_raw: np.ndarray
+    v_raw: np.ndarray
+    k_tail: np.ndarray
+    v_tail: np.ndarray
+    needles: np.ndarray = field(default=None)   # [rows, n_needles] chunk ids
+
+    def tensors(self):
+        return dict(q=self.q, k_gist=self.k_gist, v_gist=self.v_gist, k_raw=self.k_raw,
+                    v_raw=self.v_raw, k_tail=self.k_tail, v_tail=self.v_tail)
+
+
+def decode_inputs(s: DecodeShape, seed: int) -> DecodeInputs:
+    B, Hq, Hkv, d, N, c, W = s.batch, s.n_q_heads, s.n_kv_heads, s.head_dim, s.n_chunks, s.chunk, s.tail_len
+    dt = s.dtype
+    q = normal(seed, S_Q, (B, Hq, d), dt)
+    kg = normal(seed, S_KG, (B, Hkv, N, d), dt)
+    vg = normal(seed, S_VG, (B, Hkv, N, d), dt)
+    kr = normal(seed, S_KR, (B, Hkv, N, c, d), dt)
+    vr = normal(seed, S_VR, (B, Hkv, N, c, d), dt)
+    kt = normal(seed, S_KT, (B, Hkv, W, d), dt)
+    vt = normal(seed, S_VT, (B, Hkv, W, d), dt)
+    needles = np.zeros((B * Hkv, s.n_needles), np.int64)
+    if s.n_needles:
+        qw = widen(q, dt)
+        G = s.group
+        for b in range(B):
+            for hk in range(Hkv):
+                row = b * Hkv + hk
+                ids = _distinct_draws(seed, S_NEEDLE_IDX, row * 1_000_003, s.n_needles, N)
+                needles[row] = ids
+                noise = normal(seed, S_NEEDLE_NOISE, (s.n_needles, d), "f64",
+                               offset=row * s.n_needles * d)
+                for t, j in enumerate(ids):
+                    kg[b, hk, j] = round_to(_needle_keys(qw, b, hk, G, s.needle_alpha, noise[t]), dt)
+    return DecodeInputs(s, q, kg, vg, kr, vr, kt, vt, needles)
+
+
+@dataclass
+class HierInputs:
+    shape: HierShape
+    q: np.ndarray
+    k_g2: np.ndarray
+    v_g2: np.ndarray
+    k_g1: np.ndarray
+    v_g1: np.ndarray
+    k_raw: np.ndarray
+    v_raw: np.ndarray
+    k_tail: np.ndarray
+    v_tail: np.ndarray
+    needles: np.ndarray = field(default=None)
+
+    def tensors(self):
+        return dict(q=self.q, k_g2=self.k_g2, v_g2=self.v_g2, k_g1=self.k_g1, v_g1=self.v_g1,
+                    k_raw=self.k_raw, v_raw=self.v_raw, k_tail=self.k_tail, v_tail=self.v_tail)
+
+
+def hier_inputs(h: HierShape, seed: int) -> HierInputs:
+    """Level-1 tensors as for flat decode (without needles), plus level-2 gists.
+    Needles go into distinct level-2 groups: one level-1 chunk per needle group
+    gets the needle key, and so does that group's level-2 gist."""
+    s = h.l1
+    base = decode_inputs(replace(s, n_needles=0), seed)
+    B, Hkv, d, dt = s.batch, s.n_kv_heads, s.head_dim, s.dtype
+    kg2 = normal(seed, S_KG2, (B, Hkv, h.n_l2, d), dt)
+    vg2 = normal(seed, S_VG2, (B, Hkv, h.n_l2, d), dt)
+    needles = np.zeros((B * Hkv, s.n_needles), np.int64)
+    if s.n_needles:
+        qw = widen(base.q, dt)
+        G = s.group
+        for b in range(B):
+            for hk in range(Hkv):
+                row = b * Hkv + hk
+                groups = _distinct_draws(seed, S_NEEDLE_IDX, row * 1_000_003, s.n_needles, h.n_l2)
+                noise1 = normal(seed, S_NEEDLE_NOISE, (s.n_needles, d), "f64", offset=row * s.n_needles * d)
+                noise2 = normal(seed, S_NEEDLE2_NOISE, (s.n_needles, d), "f64", offset=row * s.n_needles * d)
+                for t, g in enumerate(groups):
+                    lo = g * h.group
+                    width = min(h.group, s.n_chunks - lo)
+                    j = lo + u64(seed, S_NEEDLE_IDX, 7_777_777 + row * 1_000_003 + t) % width
+                    needles[row, t] = j
+                    base.k_gist[b, hk, j] = round_to(_needle_keys(qw, b, hk, G, s.needle_alpha, noise1[t]), dt)
+                    kg2[b, hk, g] = round_to(_needle_keys(qw, b, hk, G, s.needle_alpha, noise2[t]), dt)
+    return HierInputs(h, base.q, kg2, vg2, base.k_gist, base.v_gist, base.k_raw, base.v_raw,
+                      base.k_tail, base.v_tail, needles)
+
+
+@dataclass
+class PrefillInputs:
+    shape: PrefillShape
+    q: np.ndarray   # [B, Hq, P, d]
+    k: np.ndarray   # [B, Hkv, P, d]
+    v: np.ndarray
+
+    def tensors(self):
+        return dict(q=self.q, k=self.k, v=self.v)
+
+
+def prefill_inputs(p: PrefillShape, seed: int) -> PrefillInputs:
+    P = p.positions
+    q = normal(seed, S_PQ, (p.batch, p.n_q_heads, P, p.head_dim), p.dtype)
+    k = normal(seed, S_PK, (p.batch, p.n_kv_heads, P, p.head_dim), p.dtype)
+    v = normal(seed, S_PV, (p.batch, p.n_kv_heads, P, p.head_dim), p.dtype)
+    return PrefillInputs(p, q, k, v)

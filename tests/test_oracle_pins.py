@@ -1,0 +1,349 @@
+"""Pins for the fp64 oracle: worked examples printed on the pages, closed
+forms, brute force and library routines (torch SDPA in fp64, numpy sorts).
+
+None of these retypes the oracle's own formulas: attention is checked against
+``torch.nn.functional.scaled_dot_product_attention`` over an explicitly
+assembled key list or a boolean mask, selection against ``numpy.lexsort``,
+scores against one-hot closed forms, the prefill mask against the slide's
+table and a pair-count closed form.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import DecodeShape, HierShape, ALL_GISTS, SELECTED_PAIRS
+
+
+def sdpa(qv, K, V, scale, mask=None, causal=False):
+    """Library attention in fp64: qv [..., L, d], K/V [..., S, d]."""
+    q = torch.as_tensor(qv, dtype=torch.float64)
+    k = torch.as_tensor(K, dtype=torch.float64)
+    v = torch.as_tensor(V, dtype=torch.float64)
+    m = None if mask is None else torch.as_tensor(mask, dtype=torch.bool)
+    return torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, attn_mask=m, is_causal=causal, scale=scale).numpy()
+
+
+def small_shape(**kw):
+    base = dict(batch=2, n_q_heads=4, n_kv_heads=2, head_dim=8, n_chunks=6, chunk=3, top_k=2,
+                tail_len=2, dtype="f32", mode=ALL_GISTS)
+    base.update(kw)
+    return DecodeShape(**base)
+
+
+# ---------------------------------------------------------------- scores ----
+def test_score_one_hot_queries_pick_gist_columns():
+    """q_h = e_{i_h}: the group score of gist j is the sum of Kg[j, i_h] over
+    the group's heads; heads of the other KV head do not contribute."""
+    B, Hq, Hkv, d, N = 1, 4, 2, 8, 5
+    kg = synth.normal(11, 1, (B, Hkv, N, d), "f64")
+    q = np.zeros((B, Hq, d))
+    cols = [1, 6, 3, 0]             # head h -> one-hot column; heads 0,1 -> kv 0; 2,3 -> kv 1
+    for h, i in enumerate(cols):
+        q[0, h, i] = 1.0
+    s = oracle.gist_scores(q, kg)
+    np.testing.assert_array_equal(s[0, 0], kg[0, 0, :, 1] + kg[0, 0, :, 6])
+    np.testing.assert_array_equal(s[0, 1], kg[0, 1, :, 3] + kg[0, 1, :, 0])
+
+
+def test_score_error_bound_covers_fp32_evaluation():
+    """Higham's inner-product bound holds for a float32 evaluation of the same sum."""
+    sh = small_shape(head_dim=64, n_chunks=40)
+    x = synth.decode_inputs(sh, 5)
+    s = oracle.gist_scores(x.q, x.k_gist)
+    eps = oracle.score_error_bound(x.q, x.k_gist)
+    G = sh.group
+    for b in range(sh.batch):
+        for hk in range(sh.n_kv_heads):
+            q32 = x.q[b, hk * G:(hk + 1) * G].astype(np.float32)
+            for j in range(sh.n_chunks):
+                acc = np.float32(0)
+                for g in range(G):
+                    for i in range(sh.head_dim):
+                        acc = np.float32(acc + np.float32(q32[g, i] * x.k_gist[b, hk, j, i]))
+                assert abs(float(acc) - s[b, hk, j]) <= eps[b, hk]
+
+
+# ------------------------------------------------------------- selection ----
+def test_topk_worked_example(golden):
+    rows = dict(r.split(None, 1) for r in golden("topk_slide10.txt"))
+    scores = np.array([float(v) for v in rows["scores"].split()])
+    k = int(rows["k"])
+    want = [int(v) for v in rows["selected"].split()]
+    assert oracle.topk(scores[None], k)[0].tolist() == want
+
+
+@pytest.mark.parametrize("N,k,seed", [(1, 1, 0), (7, 3, 1), (50, 10, 2), (64, 64, 3), (200, 17, 4)])
+def test_topk_matches_lexsort_with_ties(N, k, seed):
+    rng = np.random.default_rng(seed)
+    s = rng.integers(-3, 4, size=(5, N)).astype(np.float64)   # many exact ties
+    got = oracle.topk(s, k)
+    for r in range(5):
+        order = np.lexsort((np.arange(N), -s[r]))               # score desc, index asc
+        want = np.sort(order[:k])
+        assert got[r].tolist() == want.tolist()
+
+
+def test_topk_invariants_and_nan():
+    rng = np.random.default_rng(9)
+    s = rng.standard_normal((3, 100))
+    s[1, [5, 50]] = np.nan
+    idx = oracle.topk(s, 98)
+    for r in range(3):
+        assert len(set(idx[r].tolist())) == 98 and np.all(np.diff(idx[r]) > 0)
+        assert idx[r].min() >= 0 and idx[r].max() < 100
+    assert 5 not in idx[1] and 50 not in idx[1]
+    assert oracle.topk(s, 100)[0].tolist() == list(range(100))
+
+
+def test_topk_gap():
+    s = np.array([[0.1, 0.8, 0.7, 0.2]])
+    assert oracle.topk_gap(s, 2)[0] == pytest.approx(0.5)
+    assert math.isinf(oracle.topk_gap(s, 4)[0])
+
+
+# -------------------------------------------------------------- attention ---
+def _all_keys(x, b, hk):
+    """[all gists, all raw tokens chunk by chunk, tail] for one (b, hk), fp64."""
+    dt = x.shape.dtype
+    N, c, d = x.shape.n_chunks, x.shape.chunk, x.shape.head_dim
+    K = np.concatenate([synth.widen(x.k_gist[b, hk], dt), synth.widen(x.k_raw[b, hk], dt).reshape(N * c, d),
+                        synth.widen(x.k_tail[b, hk], dt)])
+    V = np.concatenate([synth.widen(x.v_gist[b, hk], dt), synth.widen(x.v_raw[b, hk], dt).reshape(N * c, d),
+                        synth.widen(x.v_tail[b, hk], dt)])
+    return K, V
+
+
+@pytest.mark.parametrize("mode", [ALL_GISTS, SELECTED_PAIRS])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_full_selection_is_full_attention(mode, dtype):
+    """k = N: both modes reduce to softmax attention over every gist, every raw
+    token and the tail."""
+    sh = small_shape(top_k=6, mode=mode, dtype=dtype)
+    x = synth.decode_inputs(sh, 21)
+    _, idx, out = oracle.decode(x.tensors(), sh.top_k, mode)
+    assert (idx == np.arange(6)).all()
+    G = sh.group
+    for b in range(sh.batch):
+        for hk in range(sh.n_kv_heads):
+            K, V = _all_keys(x, b, hk)
+            qv = synth.widen(x.q[b, hk * G:(hk + 1) * G], dtype)
+            np.testing.assert_allclose(out[b, hk * G:(hk + 1) * G], sdpa(qv, K, V, 1 / math.sqrt(8)),
+                                       rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", [ALL_GISTS, SELECTED_PAIRS])
+def test_partial_selection_is_masked_attention(mode):
+    """k < N: the gathered context equals full attention under a boolean mask
+    that keeps the selected chunks' raw tokens (and, for SELECTED_PAIRS, only
+    the selected gists); the selection itself equals a lexsort top-k."""
+    sh = small_shape(n_chunks=9, chunk=4, top_k=3, tail_len=3, mode=mode)
+    x = synth.decode_inputs(sh, 33)
+    s, idx, out = oracle.decode(x.tensors(), sh.top_k, mode, scale=0.3)
+    N, c, G = sh.n_chunks, sh.chunk, sh.group
+    for b in range(sh.batch):
+        for hk in range(sh.n_kv_heads):
+            order = np.lexsort((np.arange(N), -s[b, hk]))
+            assert idx[b, hk].tolist() == sorted(order[:3].tolist())
+            sel = np.zeros(N, bool)
+            sel[idx[b, hk]] = True
+            gist_keep = np.ones(N, bool) if mode == ALL_GISTS else sel
+            mask = np.concatenate([gist_keep, np.repeat(sel, c), np.ones(sh.tail_len, bool)])
+            K, V = _all_keys(x, b, hk)
+            qv = synth.widen(x.q[b, hk * G:(hk + 1) * G], "f32")
+            want = sdpa(qv, K, V, 0.3, mask=np.broadcast_to(mask, (G, mask.size)))
+            np.testing.assert_allclose(out[b, hk * G:(hk + 1) * G], want, rtol=0, atol=1e-12)
+
+
+def test_unfold_attn_equals_decode_for_same_selection():
+    sh = small_shape()
+    x = synth.decode_inputs(sh, 41)
+    for mode in (ALL_GISTS, SELECTED_PAIRS):
+        _, idx, out = oracle.decode(x.tensors(), sh.top_k, mode)
+        np.testing.assert_array_equal(oracle.unfold_attn(x.tensors(), idx, mode), out)
+
+
+def test_empty_selection_is_tail_attention_and_single_key_returns_value():
+    sh = small_shape(top_k=0, mode=SELECTED_PAIRS, tail_len=5)
+    x = synth.decode_inputs(sh, 43)
+    _, _, out = oracle.decode(x.tensors(), 0, SELECTED_PAIRS)
+    G = sh.group
+    for b in range(sh.batch):
+        for hk in range(sh.n_kv_heads):
+            want = sdpa(x.q[b, hk * G:(hk + 1) * G].astype(np.float64), x.k_tail[b, hk].astype(np.float64),
+                        x.v_tail[b, hk].astype(np.float64), 1 / math.sqrt(8))
+            np.testing.assert_allclose(out[b, hk * G:(hk + 1) * G], want, rtol=0, atol=1e-12)
+    sh1 = small_shape(top_k=0, mode=SELECTED_PAIRS, tail_len=1)
+    x1 = synth.decode_inputs(sh1, 44)
+    _, _, out1 = oracle.decode(x1.tensors(), 0, SELECTED_PAIRS)
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_array_equal(out1[b, h], x1.v_tail[b, h // 2, 0].astype(np.float64))
+
+
+def test_weights_sum_to_one():
+    sh = small_shape(n_chunks=12, top_k=4)
+    x = synth.decode_inputs(sh, 47)
+    t = x.tensors()
+    for name in ("v_gist", "v_raw", "v_tail"):
+        t[name] = np.ones_like(t[name])
+    for mode in (ALL_GISTS, SELECTED_PAIRS):
+        _, _, out = oracle.decode(t, sh.top_k, mode)
+        np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-14)
+
+
+def test_strong_needles_are_always_selected():
+    """needle gist key = alpha * qbar/|qbar| + noise with alpha = 3*sqrt(d):
+    every planted needle chunk is in the selected set (k = #needles)."""
+    sh = DecodeShape(2, 8, 2, 64, 300, 4, 6, 4, "bf16", ALL_GISTS, n_needles=6, needle_alpha=3 * 8.0)
+    x = synth.decode_inputs(sh, 51)
+    _, idx, _ = oracle.decode(x.tensors(), sh.top_k)
+    for r in range(sh.rows):
+        assert sorted(x.needles[r].tolist()) == idx.reshape(sh.rows, -1)[r].tolist()
+
+
+# -------------------------------------------------------------- hierarchy ---
+def _hier_small(n1=40, group=4, c=2, k2=3, k1=4, W=2, seed=61, d=8):
+    n2 = -(-n1 // group)
+    h = HierShape(DecodeShape(1, 4, 2, d, n1, c, k1, W, "f32", ALL_GISTS), n_l2=n2, group=group, top_k2=k2)
+    return h, synth.hier_inputs(h, seed)
+
+
+def test_hier_full_level2_selection_equals_flat_selection():
+    """k2 = n_l2: every level-1 gist is a candidate, so the level-1 selection
+    equals flat top-k1, and the context is every meta-gist + every gist + raw
+    of the selection + tail."""
+    h, x = _hier_small(n1=39, group=4, k2=10)
+    t = x.tensors()
+    idx2, idx1, out = oracle.hier_decode(t, h.group, h.top_k2, h.l1.top_k)
+    assert idx2[0, 0].tolist() == list(range(10))
+    flat_s = oracle.gist_scores(x.q, x.k_g1)
+    np.testing.assert_array_equal(idx1, oracle.topk(flat_s, h.l1.top_k))
+    G, c, d = 2, h.l1.chunk, h.l1.head_dim
+    for hk in range(2):
+        sel = idx1[0, hk]
+        K = np.concatenate([x.k_g2[0, hk], x.k_g1[0, hk], x.k_raw[0, hk][sel].reshape(-1, d), x.k_tail[0, hk]])
+        V = np.concatenate([x.v_g2[0, hk], x.v_g1[0, hk], x.v_raw[0, hk][sel].reshape(-1, d), x.v_tail[0, hk]])
+        want = sdpa(x.q[0, hk * G:(hk + 1) * G].astype(np.float64), K.astype(np.float64), V.astype(np.float64),
+                    1 / math.sqrt(d))
+        np.testing.assert_allclose(out[0, hk * G:(hk + 1) * G], want, rtol=0, atol=1e-12)
+
+
+def test_hier_slide11_parent_child_mapping(golden):
+    """Slide 11: 100 raw tokens per gist, 10 gists per meta-gist.  Forcing the
+    level-2 selection to G2 makes the candidates exactly g11..g20."""
+    rows = dict(r.split(None, 1) for r in golden("hierarchy_slide11.txt"))
+    c, n1, group = int(rows["chunk"]), int(rows["n_gists"]), int(rows["group"])
+    lo, hi = (int(v) for v in rows["G2_children_range0"].split())
+    assert int(rows["n_meta"]) == n1 // group
+    d = 4
+    h = HierShape(DecodeShape(1, 1, 1, d, n1, c, 3, 1, "f32", ALL_GISTS), n_l2=n1 // group, group=group, top_k2=1)
+    x = synth.hier_inputs(h, 71)
+    x.q[...] = np.float32([1.0, 0.5, -0.25, 0.125])
+    x.k_g2[0, 0, 1] = np.float32(50.0) * x.q[0, 0]          # G2 (0-based 1) dominates level 2
+    idx2, idx1, out = oracle.hier_decode(x.tensors(), group, 1, 3)
+    assert idx2[0, 0].tolist() == [1]
+    assert all(lo <= j < hi for j in idx1[0, 0])
+    s1 = oracle.gist_scores(x.q, x.k_g1)[0, 0, lo:hi]
+    assert idx1[0, 0].tolist() == sorted((lo + np.lexsort((np.arange(10), -s1))[:3]).tolist())
+    sel = idx1[0, 0]
+    K = np.concatenate([x.k_g2[0, 0], x.k_g1[0, 0, lo:hi], x.k_raw[0, 0][sel].reshape(-1, d), x.k_tail[0, 0]])
+    V = np.concatenate([x.v_g2[0, 0], x.v_g1[0, 0, lo:hi], x.v_raw[0, 0][sel].reshape(-1, d), x.v_tail[0, 0]])
+    want = sdpa(x.q[0].astype(np.float64), K.astype(np.float64), V.astype(np.float64), 0.5)
+    np.testing.assert_allclose(out[0], want, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- prefill ---
+def _slide7_names(c=2, n=3):
+    names = []
+    for j in range(n):
+        names += [f"x{j * c + u + 1}" for u in range(c)] + [f"g{j + 1}"]
+    return names
+
+
+def test_mask_matches_slide7_table(golden):
+    names = _slide7_names()
+    pos = {nm: p for p, nm in enumerate(names)}
+    for line in golden("gist_mask_slide7.txt"):
+        kind, rest = line.split(None, 1)
+        qn, keys = rest.split(":")
+        allowed = set(keys.split())
+        p = pos[qn]
+        got = {names[t] for t in range(len(names)) if oracle.gist_mask(p, t, 2)}
+        assert got == allowed, (kind, qn, got, allowed)
+
+
+def test_mask_layout_slide3(golden):
+    rows = dict(r.split() for r in golden("layout_slide3.txt"))
+    c = int(rows["chunk"])
+    g1, t17, g2, t33 = (int(rows[k]) for k in ("gist1", "token17", "gist2", "token33"))
+    assert [t for t in range(g1 + 1) if oracle.gist_mask(g1, t, c)] == list(range(int(rows["token1"]), int(rows["token16"]) + 1)) + [g1]
+    assert [t for t in range(t17 + 1) if oracle.gist_mask(t17, t, c)] == [g1, t17]
+    assert [t for t in range(g2 + 1) if oracle.gist_mask(g2, t, c)] == [g1] + list(range(t17, int(rows["token32"]) + 1)) + [g2]
+    assert [t for t in range(t33 + 1) if oracle.gist_mask(t33, t, c)] == [g1, g2, t33]
+    assert oracle.gist_mask(int(rows["gist3"]), g2, c)
+
+
+def _pairs_closed_form(N, c):
+    """gist->earlier gists + gist->self + gist->own raw + raw->earlier gists + raw->own-chunk causal."""
+    return N * (N - 1) // 2 + N + N * c + c * N * (N - 1) // 2 + N * c * (c + 1) // 2
+
+
+@pytest.mark.parametrize("N,c", [(1, 1), (1, 5), (3, 2), (4, 1), (7, 3), (12, 16)])
+def test_pair_count_closed_form_small(N, c):
+    assert oracle.prefill_pair_count(N, c) == _pairs_closed_form(N, c)
+
+
+def test_pair_count_full_prefill_size():
+    assert _pairs_closed_form(1024, 16) == 9_060_864
+    assert oracle.prefill_pair_count(1024, 16) == 9_060_864
+
+
+def test_mask_c1_closed_form():
+    """c = 1: x_j (p = 2j) sees g_i for i < j and itself; g_j (p = 2j+1) sees g_i
+    for i < j, x_j and itself."""
+    N = 6
+    for p in range(2 * N):
+        j = p // 2
+        want = {2 * i + 1 for i in range(j)} | {p}
+        if p % 2 == 1:
+            want |= {2 * j}
+        assert {t for t in range(2 * N) if oracle.gist_mask(p, t, 1)} == want
+
+
+def test_prefill_single_chunk_is_causal_attention():
+    """N = 1: the mask is the plain causal mask over the c + 1 positions."""
+    p = synth.PrefillShape(1, 2, 1, 8, 1, 6, "f32")
+    x = synth.prefill_inputs(p, 81)
+    P = p.positions
+    rows = np.array([(0, h, t) for h in range(2) for t in range(P)], np.int64)
+    out = oracle.prefill_rows(x.tensors(), 1, 6, rows).reshape(2, P, 8)
+    k = np.repeat(x.k.astype(np.float64), 2, axis=1)[0]
+    v = np.repeat(x.v.astype(np.float64), 2, axis=1)[0]
+    want = sdpa(x.q[0].astype(np.float64), k, v, 1 / math.sqrt(8), causal=True)
+    np.testing.assert_allclose(out, want, rtol=0, atol=1e-12)
+
+
+def test_prefill_matches_sdpa_under_slide7_mask(golden):
+    """Masked library attention with the slide-7 table (c = 2, three chunks),
+    grouped-query heads: head h reads KV head h // (Hq / Hkv)."""
+    names = _slide7_names()
+    pos = {nm: p for p, nm in enumerate(names)}
+    P = len(names)
+    M = np.zeros((P, P), bool)
+    for line in golden("gist_mask_slide7.txt"):
+        qn, keys = line.split(None, 1)[1].split(":")
+        for kn in keys.split():
+            M[pos[qn], pos[kn]] = True
+    p = synth.PrefillShape(1, 4, 2, 8, 3, 2, "bf16")
+    x = synth.prefill_inputs(p, 91)
+    rows = np.array([(0, h, t) for h in range(4) for t in range(P)], np.int64)
+    out = oracle.prefill_rows(x.tensors(), 3, 2, rows, scale=0.2).reshape(4, P, 8)
+    k = np.repeat(synth.widen(x.k, "bf16"), 2, axis=1)[0]
+    v = np.repeat(synth.widen(x.v, "bf16"), 2, axis=1)[0]
+    want = sdpa(synth.widen(x.q, "bf16")[0], k, v, 0.2, mask=np.broadcast_to(M, (4, P, P)))
+    np.testing.assert_allclose(out, want, rtol=0, atol=1e-12)

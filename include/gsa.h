@@ -1,0 +1,185 @@
+/*
+ * gsa.h — C ABI of libgsa.so: the decode-time hot path of Gist Sparse
+ * Attention (GSA) and its gist-causal prefill, for NVIDIA B200 (sm_100a).
+ *
+ * Method: "Forget, Then Recall: Learnable Compression and Selective Unfolding
+ * via Gist Sparse Attention" (Mao, Li, Fox).  Citations below name the page
+ * and the section that define each operation:
+ *   [EN-2]  gist.science explainer (EN), section 2 "Methodology: Gist Sparse
+ *           Attention" (interleaved gist tokens; gist as routing signals;
+ *           selective unfolding; hybrid attention; hierarchical extension);
+ *   [DE-M]  gist.science explainer (DE), section "Methodik";
+ *   [SL-n]  Taki-lab slide deck (docswell), page n: 6 "GSA とは", 7 "Gist
+ *           token", 9/10 "Training", 11 "H-GSA", 17 "Selective Rules
+ *           Comparison".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major, caller-owned DEVICE pointers (16-byte
+ *    aligned).  Shapes use B batch, Hq query heads, Hkv KV heads
+ *    (G = Hq / Hkv query heads share one KV head: head h reads KV head h / G),
+ *    d head_dim, N chunks (= gists), c raw tokens per chunk, k top-k,
+ *    W uncompressed tail tokens:
+ *        q        [B][Hq][d]
+ *        k_gist,  v_gist  [B][Hkv][N][d]        one gist K/V per chunk
+ *        k_raw,   v_raw   [B][Hkv][N][c][d]     raw K/V, chunk-major
+ *        k_tail,  v_tail  [B][Hkv][W][d]        tokens after the last chunk
+ *        scores   [B][Hkv][N]  fp32              routing scores
+ *        idx      [B][Hkv][k]  int32             selected chunks, ascending
+ *        out      [B][Hq][d]   same dtype as q
+ *  - Element type: GSA_F32 or GSA_BF16 for q and every K/V tensor alike;
+ *    all accumulation is fp32; the output is rounded once (RNE).
+ *  - The library allocates nothing and keeps no state between calls.  Work is
+ *    enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *    runs asynchronously; no entry point synchronises.
+ *  - Workspace: entry points that take `ws` need a device buffer of at least
+ *    the size the matching gsa_*_workspace_size() returns, 256-byte aligned.
+ *    It must be ZERO-FILLED ONCE after allocation (e.g. cudaMemset); each call
+ *    that completes leaves its counter words zero again.  One workspace serves
+ *    one call at a time: calls that overlap on the GPU must use separate
+ *    workspaces.
+ *  - Errors: arguments are checked on the host before anything is enqueued;
+ *    a failing check returns an error code and enqueues nothing.  A CUDA
+ *    launch failure returns GSA_ERR_CUDA.  Nothing is printed, no exception
+ *    crosses the ABI.  Device-side anomalies (an out-of-range chunk index
+ *    passed to gsa_unfold_attn, an expired bounded wait) never fault: the
+ *    kernel skips the access and ORs a flag into the workspace error word,
+ *    which gsa_workspace_error() reads back.
+ */
+#ifndef GSA_H_
+#define GSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GSA_OK = 0,
+    GSA_ERR_ARG = 1,        /* null pointer, k/W/chunk out of range, empty context, bad mode */
+    GSA_ERR_SHAPE = 2,      /* head_dim not 64/128, Hq % Hkv != 0, G not in {1,2,4,8}, size overflow */
+    GSA_ERR_DTYPE = 3,      /* dtype not supported by this entry point */
+    GSA_ERR_ALIGN = 4,      /* a tensor pointer is not 16-byte aligned */
+    GSA_ERR_WORKSPACE = 5,  /* ws is NULL, too small or not 256-byte aligned */
+    GSA_ERR_CUDA = 6,       /* a CUDA call or launch failed */
+    GSA_ERR_TIMEOUT = 7     /* device-side bounded wait expired (workspace error word) */
+} gsa_status;
+
+typedef enum { GSA_F32 = 0, GSA_BF16 = 1 } gsa_dtype;
+
+/* Context rule of the hybrid attention.
+ * GSA_ALL_GISTS      every gist once + raw tokens of the k selected chunks +
+ *                    tail ([EN-2] "Hybrid Attention"; [SL-17] "AG+SR").
+ * GSA_SELECTED_PAIRS gists and raw tokens of the k selected chunks only +
+ *                    tail ([SL-6]; [SL-17] "SG+SR").                       */
+typedef enum { GSA_ALL_GISTS = 0, GSA_SELECTED_PAIRS = 1 } gsa_mode;
+
+typedef struct {
+    int32_t batch, n_q_heads, n_kv_heads, head_dim;
+    int32_t n_chunks;   /* N >= 0 */
+    int32_t chunk;      /* c >= 1 */
+    int32_t top_k;      /* 0 <= k <= N */
+    int32_t tail_len;   /* W >= 0 */
+    gsa_dtype dtype;
+    gsa_mode mode;
+    float scale;        /* softmax scale; <= 0 selects 1/sqrt(head_dim) */
+} gsa_decode_desc;
+
+/* Two-level gist-of-gist hierarchy ([EN-2] "Hierarchical Extension (H-GSA)";
+ * [DE-M] "Erweiterung"; [SL-11]).  l1 describes the level-1 gists, raw chunks
+ * and tail (l1.top_k = k1, l1.mode must be GSA_ALL_GISTS); level-2 gist J
+ * summarises level-1 gists [J*group, (J+1)*group). n_l2 = ceil(N / group).  */
+typedef struct {
+    gsa_decode_desc l1;
+    int32_t n_l2, group, top_k2;
+} gsa_hier_desc;
+
+/* Gist-causal prefill over P = N*(c+1) interleaved positions (a gist after
+ * every chunk of c raw tokens). */
+typedef struct {
+    int32_t batch, n_q_heads, n_kv_heads, head_dim, n_chunks, chunk;
+    gsa_dtype dtype;    /* GSA_BF16 only */
+    float scale;        /* <= 0 selects 1/sqrt(head_dim) */
+} gsa_prefill_desc;
+
+/* Bytes of workspace gsa_unfold_attn / gsa_decode_step need for `desc`
+ * (0 if the descriptor is invalid). */
+size_t gsa_decode_workspace_size(const gsa_decode_desc* desc);
+/* Bytes of workspace gsa_hier_decode needs (0 if invalid). */
+size_t gsa_hier_workspace_size(const gsa_hier_desc* desc);
+
+/* Routing scores ([EN-2] "Gist as Routing Signals"; [DE-M]
+ * "Relevanz-Scoring"): the decoding query is scored against every gist key
+ * by dot product; the G query heads of a KV head share one selection, so
+ *     scores[b][hk][j] = sum_{h in group(hk)} q[b][h] . k_gist[b][hk][j]
+ * (fp32 accumulation, no softmax scale).  Reads q, k_gist; writes scores.  */
+gsa_status gsa_score(const gsa_decode_desc* desc, const void* q, const void* k_gist, float* scores,
+                     void* stream);
+
+/* Top-k chunk selection ([EN-2] "Selective Unfolding"; [SL-10] worked
+ * example 0.1/0.8/0.7/0.2, k=2 -> g2, g3): per (b, hk) the k indices with the
+ * largest scores; equal scores go to the lower index; -0 equals +0; NaN ranks
+ * below every number.  Output ascending.  Reads scores [B][Hkv][N]; writes
+ * idx [B][Hkv][k].                                                         */
+gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* idx, void* stream);
+
+/* Selective unfolding + hybrid attention ([EN-2] "Selective Unfolding",
+ * "Hybrid Attention"; [DE-M] "Selektive Entfaltung", "Hybride Attention";
+ * [SL-17]).  For every query head h of KV head hk the softmax of
+ * scale * q_h . K over the context of desc->mode, times V, where the selected
+ * chunks are idx[b][hk][0..k) (distinct, in [0, N); an index out of range is
+ * skipped and flagged).  lse (nullable) [B][Hq] receives the natural-log
+ * sum of exp(scale * q.K) over the context.                               */
+gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist,
+                           const void* v_gist, const void* k_raw, const void* v_raw,
+                           const void* k_tail, const void* v_tail, const int32_t* idx, void* out,
+                           float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* One full decode step: gsa_score -> gsa_topk -> gsa_unfold_attn in one
+ * fused pass (gist keys are read once; in GSA_ALL_GISTS mode the same pass
+ * accumulates the attention over all gists).  idx_out and scores_out are
+ * nullable: when given they receive the selection and the routing scores.  */
+gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const void* k_gist,
+                           const void* v_gist, const void* k_raw, const void* v_raw,
+                           const void* k_tail, const void* v_tail, int32_t* idx_out,
+                           float* scores_out, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Hierarchical decode: level-2 scores over every meta-gist -> top-k2 groups;
+ * level-1 scores over the gists of those groups -> top-k1 chunks among them;
+ * attention over every meta-gist, every gist of the selected groups, the raw
+ * tokens of the k1 chunks and the tail.
+ *   k_g2, v_g2 [B][Hkv][n_l2][d]; k_g1, v_g1 [B][Hkv][N][d]; raw and tail as
+ *   above; idx2_out [B][Hkv][k2] and idx1_out [B][Hkv][k1] (nullable),
+ *   ascending.                                                              */
+gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void* k_g2,
+                           const void* v_g2, const void* k_g1, const void* v_g1,
+                           const void* k_raw, const void* v_raw, const void* k_tail,
+                           const void* v_tail, int32_t* idx2_out, int32_t* idx1_out, void* out,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Gist-causal prefill ([EN-2] "Interleaved Gist Tokens"; [SL-7] gist causal
+ * mask g1 -> x1,x2; g2 -> g1,x3,x4; g3 -> g1,g2,x5,x6,g3; [SL-9]).  Position p
+ * is in chunk p / (c+1) and is a gist iff p % (c+1) == c.  Query p attends key
+ * t <= p iff t == p, or t is a gist of an earlier chunk, or t is a raw token
+ * of p's own chunk.
+ *   q, out [B][Hq][P][d]; k, v [B][Hkv][P][d], bf16; lse (nullable)
+ *   [B][Hq][P] fp32 natural-log sum of exp over the allowed keys.          */
+gsa_status gsa_gist_prefill(const gsa_prefill_desc* desc, const void* q, const void* k,
+                            const void* v, void* out, float* lse, void* stream);
+
+/* Reads (synchronously, on `stream`) the workspace error word: 0, or an OR of
+ * GSA_WS_ERR_* flags; returns GSA_ERR_TIMEOUT if a bounded wait expired,
+ * GSA_ERR_ARG if an index was out of range, else GSA_OK.  flags_out nullable. */
+#define GSA_WS_ERR_TIMEOUT 1u
+#define GSA_WS_ERR_INDEX 2u
+gsa_status gsa_workspace_error(const void* ws, uint32_t* flags_out, void* stream);
+
+/* Static description of a status code. */
+const char* gsa_status_string(gsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GSA_H_ */

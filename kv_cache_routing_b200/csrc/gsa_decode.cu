@@ -1,0 +1,779 @@
+// Flat GSA decode on B200: routing scores, top-k, selective unfolding and the
+// hybrid attention, as two kernels chained by programmatic dependent launch.
+//
+//   gist pass   grid (S_A splits, B*Hkv rows).  Streams the split's gist keys
+//               (and, in ALL_GISTS mode, gist values) once through a TMA ring.
+//               Writes the routing score of every gist, accumulates the
+//               attention of the G heads over these gists, keeps the split's
+//               local top-k, and the row's last CTA (atomic ticket) merges the
+//               local candidates into the row's exact top-k.
+//   unfold pass grid (S_B splits, rows).  After the gist pass completes, bulk-
+//               copies the selected chunks' raw K/V (and, in SELECTED_PAIRS
+//               mode, the selected gists) plus the tail, attends over them, and
+//               the row's last CTA merges every partial (log-sum-exp) into out.
+//
+// Method: gist.science explainer (EN), section 2 "Methodology": gist as
+// routing signals, selective unfolding, hybrid attention; Taki-lab slides
+// page 6 (score every gist, take top-k, restore chunks with their gists) and
+// page 17 (AG+SR / SG+SR context rules).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "gsa_attn.cuh"
+#include "gsa_plan.h"
+
+namespace gsa {
+
+__device__ uint32_t g_err_sink;   // error word for entry points without a workspace
+
+// ------------------------------------------------------------------ params --
+struct PassParams {
+    int rows, Hkv, N, C, K, W, mode;
+    float c2;                         // softmax scale * log2(e)
+    const uint8_t* q;                 // [B][Hq][d]
+    const uint8_t* kg;                // [rows][N][d]
+    const uint8_t* vg;
+    const uint8_t* kr;                // [rows][N][c][d]
+    const uint8_t* vr;
+    const uint8_t* kt;                // [rows][W][d]
+    const uint8_t* vt;
+    const int32_t* idx_in;            // selection read by the unfold pass
+    float* scores;                    // [rows][N]
+    int32_t* idx_out;                 // [rows][K] written by the gist pass
+    uint8_t* out;                     // [B][Hq][d]
+    float* lse;                       // [B][Hq] or null
+    uint32_t* err;
+    uint32_t* cntA;
+    uint32_t* cntB;
+    uint32_t* cand_key;               // [rows][candA]
+    int32_t* cand_idx;
+    float* partA;                     // [rows][SA][G][d]
+    float* mlA;                       // [rows][SA][G][2]
+    float* partB;
+    float* mlB;
+    int SA, tprA;                     // gist pass: splits, stages per row
+    int SB, tprB, KB, U;              // unfold pass: splits, stages, keys per row, keys per unit
+    int64_t candA;
+    int do_score, do_attn, do_topk;   // gist pass work
+    int local_topk;                   // 1: per-split candidates then merge; 0: last CTA selects from all scores
+    int merge_a;                      // unfold pass merges the gist-pass partials
+    // gist-pass source: the virtual gist list of a row has Nv entries.  Flat:
+    // entry v is gist v.  Gathered (parent_idx != null): entry v is gist
+    // parent_idx[row][v / group] * group + v % group (children of selected
+    // parent groups, ascending); entries past the row's valid count are empty.
+    int Nv;
+    const int32_t* parent_idx;        // [rows][parent_k]
+    int parent_k, group;
+    int slot_base, slot_stride;       // gist-pass partial slots: [rows][slot_stride], this pass at slot_base + s
+};
+
+// --------------------------------------------------------- shared memory --
+template <typename T, int D, int G, int NS>
+struct Smem {
+    using C = Cfg<T, D, G>;
+    alignas(128) uint8_t stage[NS][2][STAGE_TENSOR_BYTES];  // [slot][K|V]
+    uint64_t full[NS];
+    uint64_t empty[NS];
+    WarpScratch<G, C::TW> warp[NCW];
+    uint32_t topk[256 + 8 + NTHREADS / 32 + 8];
+    int flag;
+};
+
+// Combine area inside the (then idle) stage ring.
+template <int D, int G>
+struct CombineView {
+    float* cm;   // [NCW][G]
+    float* cl;   // [NCW][G]
+    float* co;   // [NCW][G][D]
+    __device__ CombineView(uint8_t* base) {
+        co = reinterpret_cast<float*>(base);
+        cm = co + NCW * G * D;
+        cl = cm + NCW * G;
+    }
+};
+
+// Gist-pass split s of a row covers stages [s*tpr/S, (s+1)*tpr/S).
+__device__ __forceinline__ void split_range(int s, int S, int tpr, int& t0, int& t1) {
+    t0 = (int)((int64_t)s * tpr / S);
+    t1 = (int)((int64_t)(s + 1) * tpr / S);
+}
+
+// ============================================================ gist pass ====
+// Physical gist index of virtual entry v of a row.
+__device__ __forceinline__ int gist_of(const PassParams& p, int row, int v) {
+    if (p.parent_idx == nullptr) return v;
+    const int u = v / p.group;
+    return __ldcg(p.parent_idx + (size_t)row * p.parent_k + u) * p.group + (v - u * p.group);
+}
+
+// Valid entries of a row's virtual gist list.
+__device__ __forceinline__ int valid_entries(const PassParams& p, int row) {
+    if (p.parent_idx == nullptr) return p.Nv;
+    if (p.parent_k == 0) return 0;
+    const int last = __ldcg(p.parent_idx + (size_t)row * p.parent_k + p.parent_k - 1);
+    return (p.parent_k - 1) * p.group + min(p.group, p.N - last * p.group);
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_constant__ PassParams p) {
+    using C = Cfg<T, D, G>;
+    constexpr int NS = 3;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    auto& sm = *reinterpret_cast<Smem<T, D, G, NS>*>(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int s = blockIdx.x, row = blockIdx.y;
+    const int b = row / p.Hkv, hk = row % p.Hkv;
+    const bool attn = p.do_attn != 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], NCW);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();                 // previous grid on the stream (parent selection, workspace reuse)
+    pdl_launch_dependents();
+
+    int t0, t1;
+    split_range(s, p.SA, p.tprA, t0, t1);
+    const int nvalid = valid_entries(p, row);
+    const int j0 = t0 * C::TILE;
+    const int j1 = min(t1 * C::TILE, nvalid);
+    const int ntiles = j1 > j0 ? (j1 - j0 + C::TILE - 1) / C::TILE : 0;
+    const size_t gist_row = (size_t)row * p.N;      // physical gist rows of this (b, hk)
+    const size_t score_row = (size_t)row * p.Nv;     // virtual score entries
+
+    if (warp == NCW) {
+        // ------------------------------------------------------- producer --
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            for (int t = 0; t < ntiles; ++t) {
+                const int slot = t % NS;
+                if (t >= NS && !mbar_wait(&sm.empty[slot], ((t / NS) - 1) & 1, p.err)) break;
+                const int g0 = j0 + t * C::TILE;
+                const int nk = min(C::TILE, j1 - g0);
+                const uint32_t bytes = (uint32_t)nk * C::ROWB;
+                mbar_arrive_expect_tx(&sm.full[slot], attn ? 2 * bytes : bytes);
+                uint8_t* dk = sm.stage[slot][0];
+                uint8_t* dv = sm.stage[slot][1];
+                for (int v = g0; v < g0 + nk;) {
+                    int run = g0 + nk - v;
+                    if (p.parent_idx != nullptr) run = min(run, p.group - v % p.group);
+                    const int j = gist_of(p, row, v);
+                    const size_t o = (gist_row + j) * C::ROWB;
+                    bulk_g2s(dk, p.kg + o, (uint32_t)run * C::ROWB, &sm.full[slot], pol);
+                    if (attn) bulk_g2s(dv, p.vg + o, (uint32_t)run * C::ROWB, &sm.full[slot], pol);
+                    dk += run * C::ROWB;
+                    dv += run * C::ROWB;
+                    v += run;
+                }
+            }
+            // drain: the last use of every slot must have landed before exit
+            for (int t = max(0, ntiles - NS); t < ntiles; ++t) mbar_wait(&sm.full[t % NS], (t / NS) & 1, p.err);
+        }
+    } else {
+        // ------------------------------------------------------ consumers --
+        WarpAttn<T, D, G> wa;
+        wa.load_q(reinterpret_cast<const T*>(p.q + ((size_t)b * p.Hkv * G + (size_t)hk * G) * C::ROWB), lane);
+        auto& ws = sm.warp[warp];
+        for (int t = 0; t < ntiles; ++t) {
+            const int slot = t % NS;
+            if (!mbar_wait(&sm.full[slot], (t / NS) & 1, p.err)) break;
+            const int g0 = j0 + t * C::TILE;
+            const int nk = min(C::TILE, j1 - g0);
+            const int nv = min(C::TW, nk - warp * C::TW);
+            if (nv > 0) {
+                const uint8_t* kt = sm.stage[slot][0] + warp * C::TW * C::ROWB;
+                wa.qk(kt, ws, lane);
+                if (p.do_score) {
+                    const float sc = wa.score(ws, lane);
+                    if (lane < nv) p.scores[score_row + g0 + warp * C::TW + lane] = sc;
+                }
+                if (attn) wa.softmax_pv(sm.stage[slot][1] + warp * C::TW * C::ROWB, ws, nv, p.c2, lane);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[slot]);
+        }
+        if (attn) {
+            // all consumers are past their last stage read once this barrier passes
+            asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+            CombineView<D, G> cv(&sm.stage[0][0][0]);
+            wa.finish(cv.cm + warp * G, cv.cl + warp * G, cv.co + warp * G * D, lane);
+        }
+    }
+    __syncthreads();
+
+    if (attn) {
+        CombineView<D, G> cv(&sm.stage[0][0][0]);
+        const size_t slot = (size_t)row * p.slot_stride + p.slot_base + s;
+        cta_combine<D, G>(cv.cm, cv.cl, cv.co, p.partA + slot * G * D, p.mlA + slot * G * 2);
+    }
+    if (!p.do_topk) return;
+
+    if (p.local_topk) {
+        // --------------------------------------- local top-k of this split --
+        __syncthreads();   // scores of this split written by this CTA are visible
+        int64_t off = 0;   // candidates of earlier splits
+        for (int s2 = 0; s2 < s; ++s2) {
+            int a0, a1;
+            split_range(s2, p.SA, p.tprA, a0, a1);
+            const int len = min(a1 * C::TILE, p.Nv) - a0 * C::TILE;
+            off += min(p.K, len);
+        }
+        const float* sc = p.scores + score_row + j0;
+        uint32_t* ck = p.cand_key + (size_t)row * p.candA + off;
+        int32_t* ci = p.cand_idx + (size_t)row * p.candA + off;
+        block_topk<NTHREADS>(
+            j1 - j0, p.K, [&](int i) { return order_key(sc[i]); },
+            [&](int r, int i) {
+                ck[r] = order_key(sc[i]);
+                ci[r] = j0 + i;
+            },
+            sm.topk);
+    }
+    // ---------------------------------- row ticket: last CTA selects top-k --
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t ticket = atomicAdd(&p.cntA[row], 1u);
+        sm.flag = (ticket == (uint32_t)p.SA - 1);
+    }
+    __syncthreads();
+    if (!sm.flag) return;
+    __threadfence();
+    int32_t* out = p.idx_out + (size_t)row * p.K;
+    if (p.local_topk) {
+        const uint32_t* ck = p.cand_key + (size_t)row * p.candA;
+        const int32_t* ci = p.cand_idx + (size_t)row * p.candA;
+        block_topk<NTHREADS>(
+            (int)p.candA, p.K, [&](int i) { return __ldcg(ck + i); },
+            [&](int r, int i) { out[r] = gist_of(p, row, __ldcg(ci + i)); }, sm.topk);
+    } else {
+        const float* sc = p.scores + score_row;
+        block_topk<NTHREADS>(
+            nvalid, p.K, [&](int i) { return order_key(__ldcg(sc + i)); },
+            [&](int r, int i) { out[r] = gist_of(p, row, i); }, sm.topk);
+    }
+    if (threadIdx.x == 0) p.cntA[row] = 0;   // leave the ticket zero for the next pass
+}
+
+// ========================================================== unfold pass ====
+// Unfolded keys of a row, in order: for each selected chunk u (idx order) its
+// c raw tokens (then its gist in SELECTED_PAIRS mode), then the W tail tokens.
+template <int ROWB>
+__device__ __forceinline__ void unfold_issue(const PassParams& p, int row, int x, int xe, uint8_t* dk,
+                                             uint8_t* dv, uint64_t* bar, uint64_t pol) {
+    const int kU = p.K * p.U;
+    while (x < xe) {
+        const uint8_t *sk, *sv;
+        int run;
+        if (x < kU) {
+            const int u = x / p.U, r = x % p.U;
+            int j = __ldcg(p.idx_in + (size_t)row * p.K + u);
+            if (j < 0 || j >= p.N) {
+                atomicOr(p.err, kErrIndex);
+                j = j < 0 ? 0 : p.N - 1;
+            }
+            if (r < p.C) {
+                run = min(p.C - r, xe - x);
+                const size_t o = (((size_t)row * p.N + j) * p.C + r) * ROWB;
+                sk = p.kr + o;
+                sv = p.vr + o;
+            } else {
+                run = 1;
+                const size_t o = ((size_t)row * p.N + j) * ROWB;
+                sk = p.kg + o;
+                sv = p.vg + o;
+            }
+        } else {
+            const int tt = x - kU;
+            run = min(p.W - tt, xe - x);
+            const size_t o = ((size_t)row * p.W + tt) * ROWB;
+            sk = p.kt + o;
+            sv = p.vt + o;
+        }
+        bulk_g2s(dk, sk, (uint32_t)run * ROWB, bar, pol);
+        bulk_g2s(dv, sv, (uint32_t)run * ROWB, bar, pol);
+        dk += run * ROWB;
+        dv += run * ROWB;
+        x += run;
+    }
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(NTHREADS, 3) unfold_pass_kernel(const __grid_constant__ PassParams p) {
+    using C = Cfg<T, D, G>;
+    constexpr int NS = 2;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    auto& sm = *reinterpret_cast<Smem<T, D, G, NS>*>(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int s = blockIdx.x, row = blockIdx.y;
+    const int b = row / p.Hkv, hk = row % p.Hkv;
+    int t0, t1;
+    split_range(s, p.SB, p.tprB, t0, t1);
+    const int x0 = t0 * C::TILE;
+    const int x1 = min(t1 * C::TILE, p.KB);
+    const int ntiles = t1 - t0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], NCW);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();                 // the gist pass (selection, partials) is complete
+    pdl_launch_dependents();
+
+    if (warp == NCW) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            for (int t = 0; t < ntiles; ++t) {
+                const int slot = t % NS;
+                if (t >= NS && !mbar_wait(&sm.empty[slot], ((t / NS) - 1) & 1, p.err)) break;
+                const int xa = x0 + t * C::TILE;
+                const int nk = min(C::TILE, x1 - xa);
+                mbar_arrive_expect_tx(&sm.full[slot], 2u * nk * C::ROWB);
+                unfold_issue<C::ROWB>(p, row, xa, xa + nk, sm.stage[slot][0], sm.stage[slot][1], &sm.full[slot],
+                                      pol);
+            }
+            for (int t = max(0, ntiles - NS); t < ntiles; ++t) mbar_wait(&sm.full[t % NS], (t / NS) & 1, p.err);
+        }
+    } else {
+        WarpAttn<T, D, G> wa;
+        wa.load_q(reinterpret_cast<const T*>(p.q + ((size_t)b * p.Hkv * G + (size_t)hk * G) * C::ROWB), lane);
+        auto& ws = sm.warp[warp];
+        for (int t = 0; t < ntiles; ++t) {
+            const int slot = t % NS;
+            if (!mbar_wait(&sm.full[slot], (t / NS) & 1, p.err)) break;
+            const int xa = x0 + t * C::TILE;
+            const int nk = min(C::TILE, x1 - xa);
+            const int nv = min(C::TW, nk - warp * C::TW);
+            if (nv > 0) {
+                wa.qk(sm.stage[slot][0] + warp * C::TW * C::ROWB, ws, lane);
+                wa.softmax_pv(sm.stage[slot][1] + warp * C::TW * C::ROWB, ws, nv, p.c2, lane);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[slot]);
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+        CombineView<D, G> cv(&sm.stage[0][0][0]);
+        wa.finish(cv.cm + warp * G, cv.cl + warp * G, cv.co + warp * G * D, lane);
+    }
+    __syncthreads();
+    {
+        CombineView<D, G> cv(&sm.stage[0][0][0]);
+        const size_t slot = (size_t)row * p.SB + s;
+        cta_combine<D, G>(cv.cm, cv.cl, cv.co, p.partB + slot * G * D, p.mlB + slot * G * 2);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t ticket = atomicAdd(&p.cntB[row], 1u);
+        sm.flag = (ticket == (uint32_t)p.SB - 1);
+    }
+    __syncthreads();
+    if (!sm.flag) return;
+    __threadfence();
+
+    // ------------------------------------- final log-sum-exp merge of a row --
+    const int na = p.merge_a ? p.slot_stride : 0;
+    const int nslots = na + p.SB;
+    float* wgt = reinterpret_cast<float*>(&sm.stage[0][0][0]);   // [nslots][G]
+    float* fin = wgt + nslots * G;                                // [G][2]: M, L
+    auto ml_of = [&](int sl, int h, int which) -> float {
+        return sl < na ? __ldcg(p.mlA + (((size_t)row * p.slot_stride + sl) * G + h) * 2 + which)
+                       : __ldcg(p.mlB + (((size_t)row * p.SB + (sl - na)) * G + h) * 2 + which);
+    };
+    for (int h = warp; h < G; h += NCW + 1) {
+        float M = kNegInf;
+        for (int sl = lane; sl < nslots; sl += 32) M = fmaxf(M, ml_of(sl, h, 0));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+        float L = 0.f;
+        for (int sl = lane; sl < nslots; sl += 32) {
+            const float m = ml_of(sl, h, 0);
+            const float w = (m == kNegInf) ? 0.f : exp2f(m - M);
+            wgt[sl * G + h] = w;
+            L += ml_of(sl, h, 1) * w;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+        if (lane == 0) {
+            fin[h * 2 + 0] = M;
+            fin[h * 2 + 1] = L;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * D; i += NTHREADS) {
+        const int h = i / D, e = i % D;
+        float acc = 0.f;
+        for (int sl = 0; sl < nslots; ++sl) {
+            const float w = wgt[sl * G + h];
+            const float v = sl < na ? __ldcg(p.partA + (((size_t)row * p.slot_stride + sl) * G + h) * D + e)
+                                    : __ldcg(p.partB + (((size_t)row * p.SB + (sl - na)) * G + h) * D + e);
+            acc = fmaf(w, v, acc);
+        }
+        const float r = acc / fin[h * 2 + 1];
+        const size_t oi = ((size_t)b * p.Hkv * G + (size_t)hk * G + h) * D + e;
+        if constexpr (sizeof(T) == 4) {
+            reinterpret_cast<float*>(p.out)[oi] = r;
+        } else {
+            reinterpret_cast<uint16_t*>(p.out)[oi] = f32_to_bf16_rne(r);
+        }
+    }
+    if (p.lse != nullptr && threadIdx.x < G) {
+        const int h = threadIdx.x;
+        p.lse[(size_t)b * p.Hkv * G + (size_t)hk * G + h] = (fin[h * 2] + log2f(fin[h * 2 + 1])) * 0.69314718055994531f;
+    }
+    if (threadIdx.x == 0) p.cntB[row] = 0;
+}
+
+// =============================================================== top-k =====
+// Standalone selection: one CTA per row over the row's N scores.
+__global__ void __launch_bounds__(NTHREADS) topk_kernel(const float* __restrict__ scores, int N, int K,
+                                                        int32_t* __restrict__ idx) {
+    __shared__ uint32_t sh[256 + 8 + NTHREADS / 32 + 8];
+    const int row = blockIdx.x;
+    const float* sc = scores + (size_t)row * N;
+    int32_t* out = idx + (size_t)row * K;
+    pdl_wait();
+    block_topk<NTHREADS>(
+        N, K, [&](int i) { return order_key(sc[i]); }, [&](int r, int i) { out[r] = i; }, sh);
+}
+
+// ============================================================ host side ====
+template <typename T, int D, int G>
+size_t gist_smem() {
+    return sizeof(Smem<T, D, G, 3>);
+}
+template <typename T, int D, int G>
+size_t unfold_smem() {
+    return sizeof(Smem<T, D, G, 2>);
+}
+
+static cudaError_t launch(const void* fn, dim3 grid, size_t smem, cudaStream_t st, const PassParams& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {const_cast<PassParams*>(&p)};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+template <typename T, int D, int G>
+struct Launcher {
+    static void set_attrs() {
+        static bool done = false;
+        if (!done) {
+            cudaFuncSetAttribute(gist_pass_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gist_smem<T, D, G>());
+            cudaFuncSetAttribute(unfold_pass_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)unfold_smem<T, D, G>());
+            done = true;
+        }
+    }
+    static cudaError_t gist(const PassParams& p, cudaStream_t st) {
+        set_attrs();
+        if (p.SA <= 0) return cudaSuccess;
+        return launch((const void*)gist_pass_kernel<T, D, G>, dim3(p.SA, p.rows), gist_smem<T, D, G>(), st, p);
+    }
+    static cudaError_t unfold(const PassParams& p, cudaStream_t st) {
+        set_attrs();
+        return launch((const void*)unfold_pass_kernel<T, D, G>, dim3(p.SB, p.rows), unfold_smem<T, D, G>(), st, p);
+    }
+};
+
+struct Kernels {
+    cudaError_t (*gist)(const PassParams&, cudaStream_t);
+    cudaError_t (*unfold)(const PassParams&, cudaStream_t);
+};
+
+template <typename T, int D>
+static Kernels pick_g(int G) {
+    switch (G) {
+        case 1: return {Launcher<T, D, 1>::gist, Launcher<T, D, 1>::unfold};
+        case 2: return {Launcher<T, D, 2>::gist, Launcher<T, D, 2>::unfold};
+        case 4: return {Launcher<T, D, 4>::gist, Launcher<T, D, 4>::unfold};
+        default: return {Launcher<T, D, 8>::gist, Launcher<T, D, 8>::unfold};
+    }
+}
+
+static Kernels pick_kernels(int dtype, int D, int G) {
+    if (dtype == GSA_F32) return D == 64 ? pick_g<float, 64>(G) : pick_g<float, 128>(G);
+    return D == 64 ? pick_g<bf16_t, 64>(G) : pick_g<bf16_t, 128>(G);
+}
+
+static cudaError_t run_passes(const PassParams& p, int dtype, int D, int G, bool gist, bool unfold,
+                              cudaStream_t st) {
+    Kernels k = pick_kernels(dtype, D, G);
+    cudaError_t e = cudaSuccess;
+    if (gist && (e = k.gist(p, st)) != cudaSuccess) return e;
+    if (unfold) e = k.unfold(p, st);
+    return e;
+}
+
+// Fill PassParams from a validated descriptor and plan.
+static PassParams make_params(const DecodePlan& pl, const gsa_decode_desc& d, const void* q, const void* kg,
+                              const void* vg, const void* kr, const void* vr, const void* kt, const void* vt,
+                              void* ws) {
+    PassParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.rows = pl.rows;
+    p.Hkv = d.n_kv_heads;
+    p.N = d.n_chunks;
+    p.C = d.chunk;
+    p.K = d.top_k;
+    p.W = d.tail_len;
+    p.mode = d.mode;
+    const double scale = d.scale > 0 ? (double)d.scale : 1.0 / std::sqrt((double)d.head_dim);
+    p.c2 = (float)(scale * 1.4426950408889634);
+    p.q = static_cast<const uint8_t*>(q);
+    p.kg = static_cast<const uint8_t*>(kg);
+    p.vg = static_cast<const uint8_t*>(vg);
+    p.kr = static_cast<const uint8_t*>(kr);
+    p.vr = static_cast<const uint8_t*>(vr);
+    p.kt = static_cast<const uint8_t*>(kt);
+    p.vt = static_cast<const uint8_t*>(vt);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    if (w != nullptr) {
+        p.err = reinterpret_cast<uint32_t*>(w + pl.off_err);
+        p.cntA = reinterpret_cast<uint32_t*>(w + pl.off_cnt);
+        p.cntB = p.cntA + pl.rows;
+        p.scores = reinterpret_cast<float*>(w + pl.off_scores);
+        p.cand_key = reinterpret_cast<uint32_t*>(w + pl.off_cand_key);
+        p.cand_idx = reinterpret_cast<int32_t*>(w + pl.off_cand_idx);
+        p.idx_out = reinterpret_cast<int32_t*>(w + pl.off_idx);
+        p.partA = reinterpret_cast<float*>(w + pl.off_partA);
+        p.mlA = reinterpret_cast<float*>(w + pl.off_mlA);
+        p.partB = reinterpret_cast<float*>(w + pl.off_partB);
+        p.mlB = reinterpret_cast<float*>(w + pl.off_mlB);
+    }
+    p.SA = pl.SA;
+    p.tprA = pl.tprA;
+    p.SB = pl.SB;
+    p.tprB = pl.tprB;
+    p.KB = pl.KB;
+    p.U = pl.U;
+    p.candA = pl.candA;
+    p.local_topk = 1;
+    p.Nv = d.n_chunks;
+    p.slot_base = 0;
+    p.slot_stride = pl.SA;
+    return p;
+}
+
+}  // namespace gsa
+
+// ================================================================ C ABI ====
+using namespace gsa;
+
+extern "C" {
+
+size_t gsa_decode_workspace_size(const gsa_decode_desc* desc) {
+    if (validate_decode(desc) != GSA_OK) return 0;
+    return make_decode_plan(*desc).total;
+}
+
+gsa_status gsa_score(const gsa_decode_desc* desc, const void* q, const void* k_gist, float* scores,
+                     void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if (!q || (desc->n_chunks > 0 && (!k_gist || !scores))) return GSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k_gist) || !aligned16(scores)) return GSA_ERR_ALIGN;
+    if (desc->n_chunks == 0) return GSA_OK;
+    DecodePlan pl = make_decode_plan(*desc);
+    PassParams p = make_params(pl, *desc, q, k_gist, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+    uint32_t* sink = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&sink), g_err_sink) != cudaSuccess) return GSA_ERR_CUDA;
+    p.err = sink;
+    p.scores = scores;
+    p.do_score = 1;
+    cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, desc->n_q_heads / desc->n_kv_heads, true, false,
+                               static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* idx, void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if (desc->top_k == 0) return GSA_OK;
+    if (!scores || !idx) return GSA_ERR_ARG;
+    if (!aligned16(scores) || !aligned16(idx)) return GSA_ERR_ALIGN;
+    const int rows = desc->batch * desc->n_kv_heads;
+    topk_kernel<<<rows, NTHREADS, 0, static_cast<cudaStream_t>(stream)>>>(scores, desc->n_chunks, desc->top_k,
+                                                                         idx);
+    return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+static gsa_status check_tensors(const gsa_decode_desc* d, const void* q, const void* kg, const void* vg,
+                                const void* kr, const void* vr, const void* kt, const void* vt, const void* out) {
+    const bool gists_needed = d->n_chunks > 0;
+    const bool raw_needed = d->top_k > 0;
+    const bool tail_needed = d->tail_len > 0;
+    if (!q || !out) return GSA_ERR_ARG;
+    if (gists_needed && (!kg || (d->mode == GSA_ALL_GISTS && !vg))) return GSA_ERR_ARG;
+    if (raw_needed && (!kr || !vr || (d->mode == GSA_SELECTED_PAIRS && (!kg || !vg)))) return GSA_ERR_ARG;
+    if (tail_needed && (!kt || !vt)) return GSA_ERR_ARG;
+    const void* all[] = {q, kg, vg, kr, vr, kt, vt, out};
+    for (const void* x : all)
+        if (!aligned16(x)) return GSA_ERR_ALIGN;
+    return GSA_OK;
+}
+
+static gsa_status check_ws(const DecodePlan& pl, const void* ws, size_t ws_bytes) {
+    if (!ws || ws_bytes < pl.total) return GSA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return GSA_ERR_WORKSPACE;
+    return GSA_OK;
+}
+
+gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+                           const void* k_raw, const void* v_raw, const void* k_tail, const void* v_tail,
+                           const int32_t* idx, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
+    if (desc->top_k > 0 && (!idx || !aligned16(idx))) return idx ? GSA_ERR_ALIGN : GSA_ERR_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GSA_ERR_ALIGN;
+    DecodePlan pl = make_decode_plan(*desc);
+    if ((st = check_ws(pl, ws, ws_bytes)) != GSA_OK) return st;
+    PassParams p = make_params(pl, *desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ws);
+    p.idx_in = idx;
+    p.out = static_cast<uint8_t*>(out);
+    p.lse = lse;
+    p.do_attn = (desc->mode == GSA_ALL_GISTS);
+    p.merge_a = p.do_attn && desc->n_chunks > 0;
+    cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, desc->n_q_heads / desc->n_kv_heads, p.merge_a != 0,
+                               true, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+                           const void* k_raw, const void* v_raw, const void* k_tail, const void* v_tail,
+                           int32_t* idx_out, float* scores_out, void* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
+    if (!aligned16(idx_out) || !aligned16(scores_out)) return GSA_ERR_ALIGN;
+    DecodePlan pl = make_decode_plan(*desc);
+    if ((st = check_ws(pl, ws, ws_bytes)) != GSA_OK) return st;
+    PassParams p = make_params(pl, *desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ws);
+    if (scores_out) p.scores = scores_out;
+    if (idx_out) p.idx_out = idx_out;
+    p.idx_in = p.idx_out;
+    p.out = static_cast<uint8_t*>(out);
+    p.do_score = 1;
+    p.do_topk = 1;
+    p.do_attn = (desc->mode == GSA_ALL_GISTS);
+    p.merge_a = p.do_attn && desc->n_chunks > 0;
+    cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, desc->n_q_heads / desc->n_kv_heads,
+                               desc->n_chunks > 0, true, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+
+// Hierarchical decode ([EN-2] "Hierarchical Extension (H-GSA)"; slide page 11):
+// gist pass over the level-2 gists (scores, attention, top-k2), gist pass over
+// the children of the selected groups (scores, attention, top-k1), unfold pass
+// over the raw tokens of the k1 chunks and the tail, merging all partials.
+size_t gsa_hier_workspace_size(const gsa_hier_desc* desc) {
+    if (validate_hier(desc) != GSA_OK) return 0;
+    return make_hier_plan(*desc).total;
+}
+
+gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void* k_g2, const void* v_g2,
+                           const void* k_g1, const void* v_g1, const void* k_raw, const void* v_raw,
+                           const void* k_tail, const void* v_tail, int32_t* idx2_out, int32_t* idx1_out, void* out,
+                           void* ws, size_t ws_bytes, void* stream) {
+    gsa_status st = validate_hier(desc);
+    if (st != GSA_OK) return st;
+    const gsa_decode_desc& d = desc->l1;
+    if (!q || !k_g2 || !v_g2 || !k_g1 || !v_g1 || !out) return GSA_ERR_ARG;
+    if (d.top_k > 0 && (!k_raw || !v_raw)) return GSA_ERR_ARG;
+    if (d.tail_len > 0 && (!k_tail || !v_tail)) return GSA_ERR_ARG;
+    const void* all[] = {q, k_g2, v_g2, k_g1, v_g1, k_raw, v_raw, k_tail, v_tail, idx2_out, idx1_out, out};
+    for (const void* x : all)
+        if (!aligned16(x)) return GSA_ERR_ALIGN;
+    const HierPlan hp = make_hier_plan(*desc);
+    if (!ws || ws_bytes < hp.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSA_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    const int G = d.n_q_heads / d.n_kv_heads;
+    int32_t* idx2 = idx2_out ? idx2_out : reinterpret_cast<int32_t*>(w + hp.off_idx2);
+    int32_t* idx1 = idx1_out ? idx1_out : reinterpret_cast<int32_t*>(w + hp.off_idx1);
+
+    // pass 1: level-2 gists, flat
+    PassParams p = make_params(hp.l2, hp.l2desc, q, k_g2, v_g2, nullptr, nullptr, nullptr, nullptr, ws);
+    p.cntA = reinterpret_cast<uint32_t*>(w + hp.l2.off_cnt);
+    p.scores = reinterpret_cast<float*>(w + hp.off_scores2);
+    p.cand_key = reinterpret_cast<uint32_t*>(w + hp.off_cand_key);
+    p.cand_idx = reinterpret_cast<int32_t*>(w + hp.off_cand_idx);
+    p.idx_out = idx2;
+    p.partA = reinterpret_cast<float*>(w + hp.off_partA);
+    p.mlA = reinterpret_cast<float*>(w + hp.off_mlA);
+    p.slot_base = 0;
+    p.slot_stride = hp.SA2 + hp.SA1;
+    p.do_score = p.do_attn = p.do_topk = 1;
+    Kernels kern = pick_kernels(d.dtype, d.head_dim, G);
+    if (kern.gist(p, strm) != cudaSuccess) return GSA_ERR_CUDA;
+
+    // pass 2: children of the selected level-2 groups
+    PassParams c = p;
+    c.N = d.n_chunks;
+    c.K = d.top_k;
+    c.kg = static_cast<const uint8_t*>(k_g1);
+    c.vg = static_cast<const uint8_t*>(v_g1);
+    c.Nv = hp.Nv1;
+    c.parent_idx = idx2;
+    c.parent_k = desc->top_k2;
+    c.group = desc->group;
+    c.SA = hp.SA1;
+    c.tprA = hp.tprA1;
+    c.scores = reinterpret_cast<float*>(w + hp.off_scores1);
+    c.idx_out = idx1;
+    c.local_topk = 0;
+    c.slot_base = hp.SA2;
+    if (kern.gist(c, strm) != cudaSuccess) return GSA_ERR_CUDA;
+
+    // pass 3: raw tokens of the selected level-1 chunks + tail, final merge
+    PassParams u = make_params(hp.l1, d, q, k_g1, v_g1, k_raw, v_raw, k_tail, v_tail, ws);
+    u.cntB = reinterpret_cast<uint32_t*>(w + hp.l2.off_cnt) + hp.l2.rows;
+    u.partA = p.partA;
+    u.mlA = p.mlA;
+    u.partB = reinterpret_cast<float*>(w + hp.off_partB);
+    u.mlB = reinterpret_cast<float*>(w + hp.off_mlB);
+    u.idx_in = idx1;
+    u.out = static_cast<uint8_t*>(out);
+    u.merge_a = 1;
+    u.slot_stride = hp.SA2 + hp.SA1;
+    if (kern.unfold(u, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    return GSA_OK;
+}
+
+gsa_status gsa_workspace_error(const void* ws, uint32_t* flags_out, void* stream) {
+    if (!ws) return GSA_ERR_WORKSPACE;
+    uint32_t f = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&f, static_cast<const uint8_t*>(ws) + kWsErrOffset, 4, cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return GSA_ERR_CUDA;
+    if (flags_out) *flags_out = f;
+    if (f & kErrTimeout) return GSA_ERR_TIMEOUT;
+    if (f & kErrIndex) return GSA_ERR_ARG;
+    return GSA_OK;
+}
+
+}  // extern "C"

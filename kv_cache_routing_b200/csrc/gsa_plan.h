@@ -1,0 +1,170 @@
+// Host-side descriptor validation and launch plans (split counts, workspace
+// layout).  Every quantity is a function of the descriptor alone, so results
+// are bit-identical for a given descriptor on any device.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "gsa.h"
+
+namespace gsa {
+
+constexpr size_t kWsErrOffset = 0;          // u32 error word
+constexpr size_t kWsCntOffset = 64;         // u32 tickets [2][rows]
+constexpr int kTargetGistCtas = 296;        // 2 resident gist-pass CTAs per SM on 148 SMs
+constexpr int kTargetUnfoldCtas = 444;      // 3 resident unfold-pass CTAs per SM
+constexpr int kMaxSplits = 256;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline int elem_bytes(int dtype) { return dtype == GSA_F32 ? 4 : 2; }
+// keys per pipeline stage (one 16 KiB stage per tensor)
+inline int stage_keys(int dtype, int head_dim) { return 16384 / (head_dim * elem_bytes(dtype)); }
+
+inline gsa_status validate_decode(const gsa_decode_desc* d) {
+    if (!d) return GSA_ERR_ARG;
+    if (d->dtype != GSA_F32 && d->dtype != GSA_BF16) return GSA_ERR_DTYPE;
+    if (d->mode != GSA_ALL_GISTS && d->mode != GSA_SELECTED_PAIRS) return GSA_ERR_ARG;
+    if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1) return GSA_ERR_SHAPE;
+    if (d->n_q_heads % d->n_kv_heads != 0) return GSA_ERR_SHAPE;
+    const int G = d->n_q_heads / d->n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return GSA_ERR_SHAPE;
+    if (d->head_dim != 64 && d->head_dim != 128) return GSA_ERR_SHAPE;
+    if (d->n_chunks < 0 || d->chunk < 1 || d->tail_len < 0) return GSA_ERR_ARG;
+    if (d->top_k < 0 || d->top_k > d->n_chunks) return GSA_ERR_ARG;
+    const int64_t rows = (int64_t)d->batch * d->n_kv_heads;
+    const int64_t unit = (int64_t)d->chunk + (d->mode == GSA_SELECTED_PAIRS ? 1 : 0);
+    const int64_t kb = (int64_t)d->top_k * unit + d->tail_len;
+    // element counts must fit the kernels' 32-bit per-row key arithmetic
+    if (kb > INT32_MAX / 2 || (int64_t)d->n_chunks * d->chunk > INT32_MAX / 2) return GSA_ERR_SHAPE;
+    if (rows > 65535) return GSA_ERR_SHAPE;   // grid.y
+    const int64_t ctx = (d->mode == GSA_ALL_GISTS ? d->n_chunks : 0) + kb;
+    if (ctx <= 0) return GSA_ERR_ARG;         // empty attention context
+    return GSA_OK;
+}
+
+struct DecodePlan {
+    int rows, G, tile;
+    int SA, tprA;          // gist pass
+    int SB, tprB, KB, U;   // unfold pass
+    int64_t candA;         // candidates per row
+    size_t off_err, off_cnt, off_scores, off_cand_key, off_cand_idx, off_idx;
+    size_t off_partA, off_mlA, off_partB, off_mlB, total;
+};
+
+inline int split_len(int s, int S, int tpr, int tile, int n) {
+    const int t0 = (int)((int64_t)s * tpr / S), t1 = (int)((int64_t)(s + 1) * tpr / S);
+    return std::min(t1 * tile, n) - t0 * tile;
+}
+
+inline DecodePlan make_decode_plan(const gsa_decode_desc& d) {
+    DecodePlan p{};
+    p.rows = d.batch * d.n_kv_heads;
+    p.G = d.n_q_heads / d.n_kv_heads;
+    p.tile = stage_keys(d.dtype, d.head_dim);
+    const int N = d.n_chunks;
+    p.tprA = (N + p.tile - 1) / p.tile;
+    p.SA = p.tprA == 0 ? 0 : std::min({p.tprA, std::max(1, kTargetGistCtas / p.rows), kMaxSplits});
+    p.U = d.chunk + (d.mode == GSA_SELECTED_PAIRS ? 1 : 0);
+    p.KB = d.top_k * p.U + d.tail_len;
+    p.tprB = (p.KB + p.tile - 1) / p.tile;
+    p.SB = std::max(1, std::min({p.tprB, std::max(1, kTargetUnfoldCtas / p.rows), kMaxSplits}));
+    p.candA = 0;
+    for (int s = 0; s < p.SA; ++s) p.candA += std::min(d.top_k, split_len(s, p.SA, p.tprA, p.tile, N));
+    const size_t rows = (size_t)p.rows;
+    size_t o = 0;
+    p.off_err = kWsErrOffset;
+    p.off_cnt = kWsCntOffset;
+    o = round256(kWsCntOffset + 2 * rows * 4);
+    p.off_scores = o;
+    o = round256(o + rows * (size_t)N * 4);
+    p.off_cand_key = o;
+    o = round256(o + rows * (size_t)p.candA * 4);
+    p.off_cand_idx = o;
+    o = round256(o + rows * (size_t)p.candA * 4);
+    p.off_idx = o;
+    o = round256(o + rows * (size_t)d.top_k * 4);
+    p.off_partA = o;
+    o = round256(o + rows * (size_t)p.SA * p.G * d.head_dim * 4);
+    p.off_mlA = o;
+    o = round256(o + rows * (size_t)p.SA * p.G * 2 * 4);
+    p.off_partB = o;
+    o = round256(o + rows * (size_t)p.SB * p.G * d.head_dim * 4);
+    p.off_mlB = o;
+    o = round256(o + rows * (size_t)p.SB * p.G * 2 * 4);
+    p.total = o;
+    return p;
+}
+
+}  // namespace gsa
+
+namespace gsa {
+
+inline gsa_status validate_hier(const gsa_hier_desc* h) {
+    if (!h) return GSA_ERR_ARG;
+    gsa_status st = validate_decode(&h->l1);
+    if (st != GSA_OK) return st;
+    const gsa_decode_desc& d = h->l1;
+    if (d.mode != GSA_ALL_GISTS) return GSA_ERR_ARG;
+    if (h->group < 1 || d.n_chunks < 1) return GSA_ERR_ARG;
+    if (h->n_l2 != (d.n_chunks + h->group - 1) / h->group) return GSA_ERR_SHAPE;
+    if (h->top_k2 < 1 || h->top_k2 > h->n_l2) return GSA_ERR_ARG;
+    if ((int64_t)h->top_k2 * h->group > INT32_MAX / 2) return GSA_ERR_SHAPE;
+    // k1 must not exceed the fewest candidates the level-2 selection can yield
+    const int64_t last = d.n_chunks - (int64_t)(h->n_l2 - 1) * h->group;
+    if (d.top_k > (int64_t)(h->top_k2 - 1) * h->group + last) return GSA_ERR_ARG;
+    return GSA_OK;
+}
+
+struct HierPlan {
+    gsa_decode_desc l2desc;   // level-2 pass as a flat descriptor (N = n_l2, k = k2)
+    DecodePlan l2, l1;        // l2: pass 1; l1: unfold pass of the level-1 descriptor
+    int Nv1, tprA1, SA1, SA2;
+    size_t off_scores2, off_scores1, off_cand_key, off_cand_idx, off_idx2, off_idx1;
+    size_t off_partA, off_mlA, off_partB, off_mlB, total;
+};
+
+inline HierPlan make_hier_plan(const gsa_hier_desc& h) {
+    HierPlan p{};
+    const gsa_decode_desc& d = h.l1;
+    p.l2desc = d;
+    p.l2desc.n_chunks = h.n_l2;
+    p.l2desc.top_k = h.top_k2;
+    p.l2 = make_decode_plan(p.l2desc);
+    p.l1 = make_decode_plan(d);
+    p.SA2 = p.l2.SA;
+    p.Nv1 = h.top_k2 * h.group;
+    p.tprA1 = (p.Nv1 + p.l1.tile - 1) / p.l1.tile;
+    p.SA1 = std::min({p.tprA1, std::max(1, kTargetGistCtas / p.l1.rows), kMaxSplits});
+    const size_t rows = (size_t)p.l1.rows;
+    const int G = p.l1.G, D = d.head_dim;
+    size_t o = round256(kWsCntOffset + 2 * rows * 4);
+    p.off_scores2 = o;
+    o = round256(o + rows * (size_t)h.n_l2 * 4);
+    p.off_scores1 = o;
+    o = round256(o + rows * (size_t)p.Nv1 * 4);
+    p.off_cand_key = o;
+    o = round256(o + rows * (size_t)p.l2.candA * 4);
+    p.off_cand_idx = o;
+    o = round256(o + rows * (size_t)p.l2.candA * 4);
+    p.off_idx2 = o;
+    o = round256(o + rows * (size_t)h.top_k2 * 4);
+    p.off_idx1 = o;
+    o = round256(o + rows * (size_t)d.top_k * 4);
+    p.off_partA = o;
+    o = round256(o + rows * (size_t)(p.SA2 + p.SA1) * G * D * 4);
+    p.off_mlA = o;
+    o = round256(o + rows * (size_t)(p.SA2 + p.SA1) * G * 2 * 4);
+    p.off_partB = o;
+    o = round256(o + rows * (size_t)p.l1.SB * G * D * 4);
+    p.off_mlB = o;
+    o = round256(o + rows * (size_t)p.l1.SB * G * 2 * 4);
+    p.total = o;
+    return p;
+}
+
+}  // namespace gsa

@@ -46,7 +46,7 @@ def _load():
         "oracle_topk_gap": [i, i, i, vp, vp],
         "oracle_score_error_bound": [i, i, i, i, i, i, vp, vp, vp],
         "oracle_decode": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
-        "oracle_unfold_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 9,
+        "oracle_unfold_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
         "oracle_hier_decode": [i, i, i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12,
         "oracle_gist_mask": [i64, i64, i],
         "oracle_prefill_pair_count": [i, i],
@@ -135,7 +135,8 @@ def decode(t: dict, top_k: int, mode: int = ALL_GISTS, scale: float = 0.0):
     return s, idx, out
 
 
-def unfold_attn(t: dict, idx: np.ndarray, mode: int = ALL_GISTS, scale: float = 0.0) -> np.ndarray:
+def unfold_attn(t: dict, idx: np.ndarray, mode: int = ALL_GISTS, scale: float = 0.0, with_lse: bool = False):
+    """Hybrid attention for a given selection; returns out [B,Hq,d] (and lse [B,Hq])."""
     q = t["q"]
     B, Hq, d = q.shape
     _, Hkv, N, c, _ = t["k_raw"].shape
@@ -143,10 +144,11 @@ def unfold_attn(t: dict, idx: np.ndarray, mode: int = ALL_GISTS, scale: float = 
     k = idx.shape[-1]
     idx = np.ascontiguousarray(idx, np.int32)
     out = np.empty((B, Hq, d), np.float64)
+    lse = np.empty((B, Hq), np.float64)
     _load().oracle_unfold_attn(B, Hq, Hkv, d, N, c, k, W, mode, scale, _dtcode(q), _p(q),
                                _p(t["k_gist"]), _p(t["v_gist"]), _p(t["k_raw"]), _p(t["v_raw"]),
-                               _p(t["k_tail"]), _p(t["v_tail"]), _p(idx), _p(out))
-    return out
+                               _p(t["k_tail"]), _p(t["v_tail"]), _p(idx), _p(out), _p(lse))
+    return (out, lse) if with_lse else out
 
 
 def hier_decode(t: dict, group: int, top_k2: int, top_k1: int, scale: float = 0.0):

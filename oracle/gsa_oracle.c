@@ -167,7 +167,7 @@ void oracle_score_error_bound(int B, int Hq, int Hkv, int d, int N, int dt, cons
 typedef struct { const void* k; const void* v; int64_t off; } key_ref;
 
 static void attend(int d, int dt, double scale, const void* q, int64_t q_off, int nkeys,
-                   const key_ref* keys, double* out) {
+                   const key_ref* keys, double* out, double* lse) {
     double* logit = (double*)malloc(sizeof(double) * (size_t)(nkeys > 0 ? nkeys : 1));
     double mx = -INFINITY;
     for (int x = 0; x < nkeys; ++x) {
@@ -183,6 +183,7 @@ static void attend(int d, int dt, double scale, const void* q, int64_t q_off, in
         for (int x = 0; x < nkeys; ++x) acc += logit[x] * ld(keys[x].v, dt, keys[x].off + i);
         out[i] = nkeys > 0 ? acc / z : NAN;
     }
+    if (lse) *lse = nkeys > 0 ? mx + log(z) : NAN;   /* log of sum_x exp(l_x) */
     free(logit);
 }
 
@@ -236,7 +237,7 @@ void oracle_decode(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, in
             for (int g = 0; g < G; ++g) {
                 int h = hk * G + g;
                 attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
-                       out + ((int64_t)b * Hq + h) * d);
+                       out + ((int64_t)b * Hq + h) * d, NULL);
             }
             free(keys);
             free(s);
@@ -244,11 +245,12 @@ void oracle_decode(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, in
 }
 
 /* Hybrid attention alone, for a given selection idx [B*Hkv*k] (the unfolding
- * + attention step without routing).                                         */
+ * + attention step without routing).  lse (may be NULL) [B*Hq] receives the
+ * natural log of sum_x exp(scale * q_h . K_x) over the context.              */
 void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode,
                         double scale, int dt, const void* q, const void* kg, const void* vg,
                         const void* kraw, const void* vraw, const void* ktail, const void* vtail,
-                        const int32_t* idx, double* out) {
+                        const int32_t* idx, double* out, double* lse) {
     int G = Hq / Hkv;
     double sc = default_scale(scale, d);
 #pragma omp parallel for collapse(2) schedule(dynamic)
@@ -261,7 +263,7 @@ void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int 
             for (int g = 0; g < G; ++g) {
                 int h = hk * G + g;
                 attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
-                       out + ((int64_t)b * Hq + h) * d);
+                       out + ((int64_t)b * Hq + h) * d, lse ? lse + (int64_t)b * Hq + h : NULL);
             }
             free(keys);
         }
@@ -317,7 +319,7 @@ void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, in
             for (int g = 0; g < G; ++g) {
                 int h = hk * G + g;
                 attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
-                       out + ((int64_t)b * Hq + h) * d);
+                       out + ((int64_t)b * Hq + h) * d, NULL);
             }
             free(keys);
             free(s1);
@@ -371,7 +373,7 @@ void oracle_prefill_rows(int B, int Hq, int Hkv, int d, int N, int c, double sca
         int nk = 0;
         for (int64_t t = 0; t <= p; ++t)
             if (oracle_gist_mask(p, t, c)) keys[nk++] = (key_ref){k, v, ((b * Hkv + hk) * P + t) * d};
-        attend(d, dt, sc, q, ((b * Hq + h) * P + p) * d, nk, keys, out + r * d);
+        attend(d, dt, sc, q, ((b * Hq + h) * P + p) * d, nk, keys, out + r * d, NULL);
         free(keys);
     }
 }

@@ -1,0 +1,103 @@
+"""CPU-side checks of the C-ABI library: it loads without a GPU, exports every
+function the header declares, and rejects bad arguments on the host before
+touching the device (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kv_cache_routing_b200 as gsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "gsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gsa_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    declared = _header_functions()
+    assert set(declared) == set(gsa.EXPORTS)
+    L = ctypes.CDLL(gsa.LIB_PATH)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code in range(8):
+        assert gsa.status_string(code).startswith("GSA_")
+    assert "unknown" in gsa.status_string(99)
+
+
+def _desc(**kw):
+    base = dict(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, n_chunks=100, chunk=16, top_k=4, tail_len=8,
+                dtype=gsa.GSA_BF16, mode=gsa.GSA_ALL_GISTS, scale=0.0)
+    base.update(kw)
+    return gsa.decode_desc(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), gsa.GSA_ERR_SHAPE),
+    (dict(n_q_heads=6), gsa.GSA_ERR_SHAPE),
+    (dict(n_q_heads=24, n_kv_heads=2), gsa.GSA_ERR_SHAPE),    # G = 12
+    (dict(top_k=101), gsa.GSA_ERR_ARG),
+    (dict(top_k=-1), gsa.GSA_ERR_ARG),
+    (dict(chunk=0), gsa.GSA_ERR_ARG),
+    (dict(tail_len=-3), gsa.GSA_ERR_ARG),
+    (dict(dtype=7), gsa.GSA_ERR_DTYPE),
+    (dict(mode=5), gsa.GSA_ERR_ARG),
+    (dict(mode=gsa.GSA_SELECTED_PAIRS, top_k=0, tail_len=0), gsa.GSA_ERR_ARG),   # empty context
+    (dict(batch=0), gsa.GSA_ERR_SHAPE),
+])
+def test_descriptor_validation(kw, code):
+    d = _desc(**kw)
+    assert gsa.gsa_decode_workspace_size(d) == 0
+    with pytest.raises(gsa.GsaError) as e:
+        gsa.gsa_score(d, 1 << 20, 1 << 21, 1 << 22, stream=0)
+    assert e.value.status == code
+
+
+def test_pointer_and_workspace_checks_happen_before_launch():
+    d = _desc()
+    n = gsa.gsa_decode_workspace_size(d)
+    assert n > 0 and n % 256 == 0
+    A = 1 << 20
+    ptrs = [A * (i + 1) for i in range(7)]
+    with pytest.raises(gsa.GsaError) as e:      # misaligned q
+        gsa.gsa_decode_step(d, ptrs[0] + 4, *ptrs[1:], None, None, A * 9, A * 10, stream=0, ws_bytes=n)
+    assert e.value.status == gsa.GSA_ERR_ALIGN
+    with pytest.raises(gsa.GsaError) as e:      # missing workspace
+        gsa.gsa_decode_step(d, *ptrs, None, None, A * 9, None, stream=0, ws_bytes=0)
+    assert e.value.status == gsa.GSA_ERR_WORKSPACE
+    with pytest.raises(gsa.GsaError) as e:      # workspace too small
+        gsa.gsa_decode_step(d, *ptrs, None, None, A * 9, A * 10, stream=0, ws_bytes=n - 256)
+    assert e.value.status == gsa.GSA_ERR_WORKSPACE
+    with pytest.raises(gsa.GsaError) as e:      # workspace not 256-byte aligned
+        gsa.gsa_decode_step(d, *ptrs, None, None, A * 9, A * 10 + 16, stream=0, ws_bytes=n)
+    assert e.value.status == gsa.GSA_ERR_WORKSPACE
+    with pytest.raises(gsa.GsaError) as e:      # null output
+        gsa.gsa_decode_step(d, *ptrs, None, None, None, A * 10, stream=0, ws_bytes=n)
+    assert e.value.status == gsa.GSA_ERR_ARG
+
+
+def test_hier_validation():
+    l1 = _desc(n_chunks=160, top_k=8)
+    ok = gsa.hier_desc(l1, 10, 16, 2)
+    assert gsa.gsa_hier_workspace_size(ok) > 0
+    assert gsa.gsa_hier_workspace_size(gsa.hier_desc(l1, 11, 16, 2)) == 0       # n_l2 != ceil(N/group)
+    assert gsa.gsa_hier_workspace_size(gsa.hier_desc(l1, 10, 16, 0)) == 0       # k2 = 0
+    assert gsa.gsa_hier_workspace_size(gsa.hier_desc(_desc(n_chunks=160, top_k=40), 10, 16, 2)) == 0  # k1 > cands
+    assert gsa.gsa_hier_workspace_size(gsa.hier_desc(_desc(n_chunks=160, mode=gsa.GSA_SELECTED_PAIRS), 10, 16, 2)) == 0
+
+
+def test_prefill_validation():
+    with pytest.raises(gsa.GsaError) as e:
+        gsa.gsa_gist_prefill(gsa.prefill_desc(1, 8, 2, 128, 4, 16, gsa.GSA_F32), 1 << 20, 1 << 21, 1 << 22,
+                             1 << 23, stream=0)
+    assert e.value.status == gsa.GSA_ERR_DTYPE
+    with pytest.raises(gsa.GsaError) as e:
+        gsa.gsa_gist_prefill(gsa.prefill_desc(1, 8, 2, 96, 4, 16), 1 << 20, 1 << 21, 1 << 22, 1 << 23, stream=0)
+    assert e.value.status == gsa.GSA_ERR_SHAPE

@@ -1,0 +1,196 @@
+"""GPU parity of the flat decode path (libgsa.so through the C-ABI binding)
+against the fp64 oracle on identical seeded inputs."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_routing_b200 as gsa
+import oracle
+import synth
+from synth import ALL_GISTS, SELECTED_PAIRS, DecodeShape
+
+from gsa_check import (check_out, check_selection, desc_of, dev, gpu_decode_step, host, tdtype, upload,
+                       workspace)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_and_check(s: DecodeShape, seed: int, label: str):
+    x = synth.decode_inputs(s, seed)
+    t = x.tensors()
+    s_ex, idx_ex, out_ex = oracle.decode(t, s.top_k, s.mode, s.scale)
+    idx, sc, out = gpu_decode_step(s, upload(x))
+    eps = oracle.score_error_bound(x.q, x.k_gist) if s.n_chunks else np.zeros(s.rows)
+    if s.n_chunks:
+        assert np.max(np.abs(sc - s_ex) - eps[..., None]) <= 0, f"{label}: score outside fp32 bound"
+    und = check_selection(idx, s_ex, eps, s.top_k, label) if s.top_k else 0
+    if und == 0:
+        check_out(out, out_ex, s.dtype, label)
+    else:
+        # where the GPU's valid selection differs, compare against the oracle's
+        # attention over the GPU's own selection
+        check_out(out, oracle.unfold_attn(t, idx.astype(np.int32), s.mode, s.scale), s.dtype, label)
+    return und
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "llama8b_decode"])
+def test_decode_configs_full(name):
+    s = synth.WORKLOADS[name]
+    und = _run_and_check(s, synth.seed_for(name), name)
+    assert und == 0, f"{name}: {und} undecidable rows (needle margin expected to decide every row)"
+
+
+@pytest.mark.parametrize("name", ["sweep_c8_all", "sweep_c16_all", "sweep_c32_all",
+                                  "sweep_c8_pairs", "sweep_c16_pairs", "sweep_c32_pairs"])
+def test_decode_compression_sweep_full(name):
+    s = synth.WORKLOADS[name]
+    _run_and_check(s, synth.seed_for(name), name)
+
+
+EDGE = {
+    # ragged: N not a multiple of the stage, odd chunk, odd tail
+    "ragged": DecodeShape(2, 8, 2, 128, 1000, 3, 7, 5, "bf16", ALL_GISTS, n_needles=7),
+    "ragged_pairs": DecodeShape(2, 8, 2, 128, 1000, 3, 7, 5, "bf16", SELECTED_PAIRS, n_needles=7),
+    "k_equals_n": DecodeShape(1, 4, 1, 64, 37, 4, 37, 3, "f32", ALL_GISTS),
+    "k_zero_all": DecodeShape(2, 4, 2, 64, 50, 4, 0, 9, "f32", ALL_GISTS),
+    "k_zero_no_tail": DecodeShape(1, 4, 2, 128, 300, 16, 0, 0, "bf16", ALL_GISTS),
+    "pairs_tail_only": DecodeShape(1, 4, 1, 128, 40, 8, 0, 33, "bf16", SELECTED_PAIRS),
+    "no_gists": DecodeShape(2, 4, 2, 64, 0, 16, 0, 20, "f32", ALL_GISTS),
+    "no_tail": DecodeShape(1, 8, 2, 128, 777, 16, 9, 0, "bf16", ALL_GISTS, n_needles=9),
+    "g1": DecodeShape(2, 4, 4, 128, 600, 16, 5, 16, "bf16", ALL_GISTS, n_needles=5),
+    "g2_f32_d128": DecodeShape(1, 4, 2, 128, 300, 8, 6, 10, "f32", SELECTED_PAIRS, n_needles=6),
+    "g8": DecodeShape(1, 16, 2, 128, 700, 16, 6, 32, "bf16", ALL_GISTS, n_needles=6),
+    "bf16_d64": DecodeShape(3, 12, 3, 64, 900, 16, 8, 24, "bf16", ALL_GISTS, n_needles=8),
+    "chunk1": DecodeShape(1, 4, 1, 128, 513, 1, 40, 7, "bf16", SELECTED_PAIRS, n_needles=40),
+    "chunk64": DecodeShape(1, 4, 1, 128, 100, 64, 5, 64, "bf16", ALL_GISTS, n_needles=5),
+    "many_rows": DecodeShape(40, 16, 8, 64, 64, 16, 4, 16, "bf16", ALL_GISTS, n_needles=4),
+    "custom_scale": dataclasses.replace(DecodeShape(1, 8, 2, 128, 256, 16, 8, 16, "f32", ALL_GISTS,
+                                                    n_needles=8), scale=0.05),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_decode_edge_cases(name):
+    _run_and_check(EDGE[name], 1000 + sorted(EDGE).index(name), name)
+
+
+def test_exact_ties_go_to_lowest_index():
+    """All gist keys identical -> every score ties -> selection = 0..k-1."""
+    s = DecodeShape(2, 8, 2, 128, 700, 4, 9, 4, "bf16", ALL_GISTS)
+    x = synth.decode_inputs(s, 77)
+    x.k_gist[...] = x.k_gist[:, :, :1, :]
+    idx, sc, _ = gpu_decode_step(s, upload(x))
+    assert (idx == np.arange(9)).all()
+    assert np.all(sc == sc[..., :1])
+
+
+def test_strong_needles_always_selected():
+    s = DecodeShape(4, 32, 8, 128, 4096, 16, 16, 64, "bf16", ALL_GISTS, n_needles=16,
+                    needle_alpha=3 * np.sqrt(128))
+    x = synth.decode_inputs(s, 78)
+    idx, _, _ = gpu_decode_step(s, upload(x))
+    for r in range(s.rows):
+        assert idx.reshape(s.rows, -1)[r].tolist() == sorted(x.needles[r].tolist())
+
+
+def test_repeat_calls_are_bitwise_identical_and_leave_workspace_clean():
+    s = synth.WORKLOADS["llama8b_decode"]
+    x = synth.decode_inputs(dataclasses.replace(s, batch=2), 79)
+    s2 = dataclasses.replace(s, batch=2)
+    d = upload(x)
+    ws = workspace(gsa.gsa_decode_workspace_size(desc_of(s2)))
+    a = gpu_decode_step(s2, d, ws)
+    b = gpu_decode_step(s2, d, ws)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+    desc = desc_of(s2)
+    # tickets are back to zero: bytes [64, 64 + 8*rows) of the workspace
+    assert int(ws[64:64 + 8 * s2.rows].sum().item()) == 0
+
+
+def test_standalone_score_topk_unfold_match_oracle():
+    s = DecodeShape(2, 16, 4, 128, 1500, 16, 12, 40, "bf16", ALL_GISTS, n_needles=12)
+    x = synth.decode_inputs(s, 80)
+    t = x.tensors()
+    d = upload(x)
+    desc = desc_of(s)
+    sc = torch.empty((2, 4, 1500), dtype=torch.float32, device="cuda")
+    gsa.gsa_score(desc, d["q"], d["k_gist"], sc)
+    s_ex = oracle.gist_scores(x.q, x.k_gist)
+    eps = oracle.score_error_bound(x.q, x.k_gist)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(sc.cpu().numpy() - s_ex) - eps[..., None]) <= 0
+    # top-k of the GPU's own fp32 scores is integer work: bit-exact vs a lexsort
+    idx = torch.empty((2, 4, 12), dtype=torch.int32, device="cuda")
+    gsa.gsa_topk(desc, sc, idx)
+    s32 = sc.cpu().numpy().reshape(8, 1500)
+    want = np.stack([np.sort(np.lexsort((np.arange(1500), -s32[r]))[:12]) for r in range(8)])
+    np.testing.assert_array_equal(idx.cpu().numpy().reshape(8, 12), want)
+    # unfold + attention for a given selection, both modes, with lse
+    idx_ex = oracle.topk(s_ex, 12)
+    for mode in (ALL_GISTS, SELECTED_PAIRS):
+        sm = dataclasses.replace(s, mode=mode)
+        dm = desc_of(sm)
+        ws = workspace(gsa.gsa_decode_workspace_size(dm))
+        out = torch.empty((2, 16, 128), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((2, 16), dtype=torch.float32, device="cuda")
+        gsa.gsa_unfold_attn(dm, d["q"], d["k_gist"], d["v_gist"], d["k_raw"], d["v_raw"], d["k_tail"],
+                            d["v_tail"], dev(idx_ex), out, lse, ws)
+        o_ex, l_ex = oracle.unfold_attn(t, idx_ex, mode, with_lse=True)
+        check_out(host(out), o_ex, "bf16", f"unfold mode {mode}")
+        assert np.max(np.abs(lse.cpu().numpy() - l_ex)) < 1e-3
+
+
+def test_topk_nan_and_signed_zero():
+    """NaN ranks lowest, -0 equals +0 (lower index wins the tie)."""
+    desc = gsa.decode_desc(1, 1, 1, 64, 8, 1, 3, 0, gsa.GSA_F32)
+    s = torch.tensor([[[float("nan"), -0.0, 0.0, -1.0, float("nan"), -2.0, 0.0, -0.5]]], device="cuda")
+    idx = torch.empty((1, 1, 3), dtype=torch.int32, device="cuda")
+    gsa.gsa_topk(desc, s, idx)
+    assert idx.cpu().tolist() == [[[1, 2, 6]]]
+    desc5 = gsa.decode_desc(1, 1, 1, 64, 8, 1, 7, 0, gsa.GSA_F32)
+    idx5 = torch.empty((1, 1, 7), dtype=torch.int32, device="cuda")
+    gsa.gsa_topk(desc5, s, idx5)
+    assert idx5.cpu().tolist() == [[[0, 1, 2, 3, 5, 6, 7]]]
+
+
+def test_out_of_range_index_is_flagged_not_faulted():
+    s = DecodeShape(1, 4, 1, 128, 64, 16, 2, 4, "bf16", SELECTED_PAIRS)
+    x = synth.decode_inputs(s, 81)
+    d = upload(x)
+    desc = desc_of(s)
+    ws = workspace(gsa.gsa_decode_workspace_size(desc))
+    out = torch.empty((1, 4, 128), dtype=torch.bfloat16, device="cuda")
+    bad = torch.tensor([[[3, 64]]], dtype=torch.int32, device="cuda")
+    gsa.gsa_unfold_attn(desc, d["q"], d["k_gist"], d["v_gist"], d["k_raw"], d["v_raw"], d["k_tail"], d["v_tail"],
+                        bad, out, None, ws)
+    torch.cuda.synchronize()
+    assert gsa.gsa_workspace_error(ws) & gsa.GSA_WS_ERR_INDEX
+
+
+def test_cuda_graph_capture_replays_identically():
+    s = dataclasses.replace(synth.WORKLOADS["llama8b_decode"], batch=2)
+    x = synth.decode_inputs(s, 82)
+    d = upload(x)
+    desc = desc_of(s)
+    ws = workspace(gsa.gsa_decode_workspace_size(desc))
+    idx = torch.empty((2, 8, 16), dtype=torch.int32, device="cuda")
+    out = torch.empty((2, 32, 128), dtype=torch.bfloat16, device="cuda")
+    gsa.gsa_decode_step(desc, d["q"], d["k_gist"], d["v_gist"], d["k_raw"], d["v_raw"], d["k_tail"], d["v_tail"],
+                        idx, None, out, ws)
+    torch.cuda.synchronize()
+    ref = (idx.clone(), out.clone())
+    g = torch.cuda.CUDAGraph()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            gsa.gsa_decode_step(desc, d["q"], d["k_gist"], d["v_gist"], d["k_raw"], d["v_raw"], d["k_tail"],
+                                d["v_tail"], idx, None, out, ws, stream=stream)
+    idx.zero_()
+    out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ref[0]) and torch.equal(out, ref[1])

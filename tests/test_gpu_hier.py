@@ -1,0 +1,68 @@
+"""GPU parity of the hierarchical (gist-of-gist) decode against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_routing_b200 as gsa
+import oracle
+import synth
+from synth import DecodeShape, HierShape
+
+from gsa_check import check_out, check_selection, desc_of, host, tdtype, upload, workspace
+
+pytestmark = pytest.mark.gpu
+
+
+def run_hier(h: HierShape, seed: int, label: str):
+    s = h.l1
+    x = synth.hier_inputs(h, seed)
+    t = x.tensors()
+    idx2_ex, idx1_ex, out_ex = oracle.hier_decode(t, h.group, h.top_k2, s.top_k, s.scale)
+    d = upload(x)
+    hd = gsa.hier_desc(desc_of(s), h.n_l2, h.group, h.top_k2)
+    ws = workspace(gsa.gsa_hier_workspace_size(hd))
+    B, Hkv = s.batch, s.n_kv_heads
+    idx2 = torch.full((B, Hkv, h.top_k2), -1, dtype=torch.int32, device="cuda")
+    idx1 = torch.full((B, Hkv, max(1, s.top_k)), -1, dtype=torch.int32, device="cuda")
+    out = torch.empty((B, s.n_q_heads, s.head_dim), dtype=tdtype(s.dtype), device="cuda")
+    gsa.gsa_hier_decode(hd, d["q"], d["k_g2"], d["v_g2"], d["k_g1"], d["v_g1"], d["k_raw"], d["v_raw"],
+                        d["k_tail"], d["v_tail"], idx2, idx1, out, ws)
+    torch.cuda.synchronize()
+    assert gsa.gsa_workspace_error(ws) == 0
+    # level 2: decidability rule on the meta-gist scores
+    s2 = oracle.gist_scores(x.q, x.k_g2)
+    eps2 = oracle.score_error_bound(x.q, x.k_g2)
+    und = check_selection(idx2.cpu().numpy(), s2, eps2, h.top_k2, f"{label} level 2")
+    assert und == 0, f"{label}: undecidable level-2 rows"
+    # level 1: scores of the candidates (children of the selected groups); others -inf
+    s1 = oracle.gist_scores(x.q, x.k_g1)
+    masked = np.full_like(s1, -np.inf)
+    for b in range(B):
+        for hk in range(Hkv):
+            for g in idx2_ex[b, hk]:
+                lo, hi = g * h.group, min((g + 1) * h.group, s.n_chunks)
+                masked[b, hk, lo:hi] = s1[b, hk, lo:hi]
+    eps1 = oracle.score_error_bound(x.q, x.k_g1)
+    und = check_selection(idx1[..., :s.top_k].cpu().numpy(), masked, eps1, s.top_k, f"{label} level 1")
+    assert und == 0, f"{label}: undecidable level-1 rows"
+    return check_out(host(out), out_ex, s.dtype, label)
+
+
+def test_hier_one_million_tokens():
+    name = "hier_1m"
+    h = synth.WORKLOADS[name]
+    run_hier(h, synth.seed_for(name), name)
+
+
+@pytest.mark.parametrize("case", [
+    # ragged last group (N1 = 1000 -> 63 groups of 16, the last of 8), selected by a needle
+    HierShape(DecodeShape(2, 8, 2, 128, 1000, 16, 6, 20, "bf16", n_needles=6, needle_alpha=40.0), 63, 16, 6),
+    # k2 = n_l2: every gist is a candidate
+    HierShape(DecodeShape(1, 4, 1, 64, 96, 4, 5, 8, "f32", n_needles=5, needle_alpha=30.0), 6, 16, 6),
+    # group 1: level 2 mirrors level 1
+    HierShape(DecodeShape(1, 8, 2, 128, 200, 8, 4, 0, "bf16", n_needles=4, needle_alpha=40.0), 200, 1, 10),
+    # many candidates, small chunks, G = 8
+    HierShape(DecodeShape(1, 16, 2, 128, 4096, 2, 32, 64, "bf16", n_needles=32, needle_alpha=40.0), 128, 32, 32),
+])
+def test_hier_edge_cases(case):
+    run_hier(case, 500 + case.n_l2, f"hier n_l2={case.n_l2}")

@@ -159,6 +159,25 @@ def test_partial_selection_is_masked_attention(mode):
             np.testing.assert_allclose(out[b, hk * G:(hk + 1) * G], want, rtol=0, atol=1e-12)
 
 
+def test_unfold_attn_lse_is_library_logsumexp():
+    """lse output = torch.logsumexp of the scaled logits over the assembled context."""
+    sh = small_shape(n_chunks=7, top_k=3, tail_len=4)
+    x = synth.decode_inputs(sh, 45)
+    for mode in (ALL_GISTS, SELECTED_PAIRS):
+        _, idx, _ = oracle.decode(x.tensors(), sh.top_k, mode, scale=0.7)
+        _, lse = oracle.unfold_attn(x.tensors(), idx, mode, scale=0.7, with_lse=True)
+        G, c = sh.group, sh.chunk
+        for b in range(sh.batch):
+            for hk in range(sh.n_kv_heads):
+                sel = idx[b, hk]
+                gl = np.arange(sh.n_chunks) if mode == ALL_GISTS else sel
+                K = np.concatenate([x.k_gist[b, hk][gl], x.k_raw[b, hk][sel].reshape(-1, sh.head_dim),
+                                    x.k_tail[b, hk]]).astype(np.float64)
+                for g in range(G):
+                    logits = 0.7 * torch.from_numpy(K) @ torch.from_numpy(x.q[b, hk * G + g].astype(np.float64))
+                    assert lse[b, hk * G + g] == pytest.approx(torch.logsumexp(logits, 0).item(), abs=1e-12)
+
+
 def test_unfold_attn_equals_decode_for_same_selection():
     sh = small_shape()
     x = synth.decode_inputs(sh, 41)

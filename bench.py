@@ -162,6 +162,8 @@ def run_ours(args, world, rank, local):
     l2 = dev_props.L2_cache_size
     nbytes_step = algorithmic_bytes(s)
     L = max(2, -(-4 * l2 // nbytes_step))                 # replicas: touched bytes per rotation >= 4 x L2
+    if args.replicas:
+        L = args.replicas
     x = synth.decode_inputs(s, synth.seed_for(args.workload) + 17 * rank)
     base = {k: dev(v) for k, v in x.tensors().items()}
     reps = []
@@ -342,6 +344,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="layer replicas to rotate over (default: enough to exceed 4x L2); 1 for profiling captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -47,7 +47,7 @@ def _load():
         "oracle_score_error_bound": [i, i, i, i, i, i, vp, vp, vp],
         "oracle_decode": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
         "oracle_unfold_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
-        "oracle_hier_decode": [i, i, i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12,
+        "oracle_hier_decode": [i, i, i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12 + [i],
         "oracle_gist_mask": [i64, i64, i],
         "oracle_prefill_pair_count": [i, i],
         "oracle_prefill_rows": [i, i, i, i, i, i, d, i, vp, vp, vp, i64, vp, vp],
@@ -151,21 +151,26 @@ def unfold_attn(t: dict, idx: np.ndarray, mode: int = ALL_GISTS, scale: float = 
     return (out, lse) if with_lse else out
 
 
-def hier_decode(t: dict, group: int, top_k2: int, top_k1: int, scale: float = 0.0):
+def hier_decode(t: dict, group: int, top_k2: int, top_k1: int, scale: float = 0.0, given=None):
     """t: q, k_g2, v_g2, k_g1, v_g1, k_raw, v_raw, k_tail, v_tail.
-    Returns (idx2 [B,Hkv,k2], idx1 [B,Hkv,k1], out [B,Hq,d])."""
+    Returns (idx2 [B,Hkv,k2], idx1 [B,Hkv,k1], out [B,Hq,d]).  given=(idx2, idx1)
+    evaluates the attention for that selection instead of selecting."""
     q = t["q"]
     B, Hq, d = q.shape
     _, Hkv, N1, c, _ = t["k_raw"].shape
     n_l2 = t["k_g2"].shape[2]
     W = t["k_tail"].shape[2]
-    idx2 = np.empty((B, Hkv, top_k2), np.int32)
-    idx1 = np.empty((B, Hkv, top_k1), np.int32)
+    if given is None:
+        idx2 = np.empty((B, Hkv, top_k2), np.int32)
+        idx1 = np.empty((B, Hkv, top_k1), np.int32)
+    else:
+        idx2 = np.ascontiguousarray(given[0], np.int32).copy()
+        idx1 = np.ascontiguousarray(given[1], np.int32).copy()
     out = np.empty((B, Hq, d), np.float64)
     _load().oracle_hier_decode(B, Hq, Hkv, d, N1, c, top_k1, W, n_l2, group, top_k2, scale,
                                _dtcode(q), _p(q), _p(t["k_g2"]), _p(t["v_g2"]), _p(t["k_g1"]),
                                _p(t["v_g1"]), _p(t["k_raw"]), _p(t["v_raw"]), _p(t["k_tail"]),
-                               _p(t["v_tail"]), _p(idx2), _p(idx1), _p(out))
+                               _p(t["v_tail"]), _p(idx2), _p(idx1), _p(out), 0 if given is None else 1)
     return idx2, idx1, out
 
 

@@ -279,12 +279,15 @@ void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int 
 /*   candidates: level-1 gists j with floor(j / group) in S2, ascending;      */
 /*   level 1: s1[j] over the candidates -> S1 = top-k1 among them;            */
 /*   context: every meta-gist, every candidate gist, raw tokens of S1, tail.  */
+/* With given != 0, idx2_out / idx1_out are inputs: the attention is evaluated */
+/* for that selection (a test helper for rows whose selection is not decided  */
+/* at fp32 precision).                                                        */
 /* ------------------------------------------------------------------------ */
 void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, int W, int n_l2,
                         int group, int k2, double scale, int dt, const void* q, const void* kg2,
                         const void* vg2, const void* kg1, const void* vg1, const void* kraw,
                         const void* vraw, const void* ktail, const void* vtail, int32_t* idx2_out,
-                        int32_t* idx1_out, double* out) {
+                        int32_t* idx1_out, double* out, int given) {
     int G = Hq / Hkv;
     double sc = default_scale(scale, d);
 #pragma omp parallel for collapse(2) schedule(dynamic)
@@ -294,7 +297,7 @@ void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, in
             double* s2 = (double*)malloc(sizeof(double) * (size_t)n_l2);
             for (int J = 0; J < n_l2; ++J) s2[J] = gist_score(Hq, Hkv, d, n_l2, dt, q, kg2, b, hk, J);
             int32_t* S2 = idx2_out + row * k2;
-            topk_list(n_l2, s2, NULL, k2, S2);
+            if (!given) topk_list(n_l2, s2, NULL, k2, S2);
 
             int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * (size_t)k2 * group + 1);
             int nc = 0;
@@ -306,7 +309,7 @@ void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, in
             double* s1 = (double*)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
             for (int t = 0; t < nc; ++t) s1[t] = gist_score(Hq, Hkv, d, N1, dt, q, kg1, b, hk, cand[t]);
             int32_t* S1 = idx1_out + row * k1;
-            topk_list(nc, s1, cand, k1, S1);
+            if (!given) topk_list(nc, s1, cand, k1, S1);
 
             key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(n_l2 + nc + (int64_t)k1 * c + W + 1));
             int nk = 0;

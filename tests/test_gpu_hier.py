@@ -32,8 +32,10 @@ def run_hier(h: HierShape, seed: int, label: str):
     # level 2: decidability rule on the meta-gist scores
     s2 = oracle.gist_scores(x.q, x.k_g2)
     eps2 = oracle.score_error_bound(x.q, x.k_g2)
-    und = check_selection(idx2.cpu().numpy(), s2, eps2, h.top_k2, f"{label} level 2")
-    assert und == 0, f"{label}: undecidable level-2 rows"
+    g2 = idx2.cpu().numpy()
+    und2 = check_selection(g2, s2, eps2, h.top_k2, f"{label} level 2")
+    if und2:
+        idx2_ex = g2   # level 1 is judged on the candidates of the GPU's (valid) level-2 set
     # level 1: scores of the candidates (children of the selected groups); others -inf
     s1 = oracle.gist_scores(x.q, x.k_g1)
     masked = np.full_like(s1, -np.inf)
@@ -43,8 +45,13 @@ def run_hier(h: HierShape, seed: int, label: str):
                 lo, hi = g * h.group, min((g + 1) * h.group, s.n_chunks)
                 masked[b, hk, lo:hi] = s1[b, hk, lo:hi]
     eps1 = oracle.score_error_bound(x.q, x.k_g1)
-    und = check_selection(idx1[..., :s.top_k].cpu().numpy(), masked, eps1, s.top_k, f"{label} level 1")
-    assert und == 0, f"{label}: undecidable level-1 rows"
+    g1 = idx1[..., :s.top_k].cpu().numpy()
+    und1 = check_selection(g1, masked, eps1, s.top_k, f"{label} level 1")
+    if und2 or und1:
+        # the literal 3-sigma needles leave some rows undecidable at fp32: judge
+        # the output against the oracle's attention over the GPU's valid selection
+        _, _, out_ex = oracle.hier_decode(t, h.group, h.top_k2, s.top_k, s.scale, given=(g2, g1))
+    print(f"{label}: undecidable rows level 2 {und2}, level 1 {und1}")
     return check_out(host(out), out_ex, s.dtype, label)
 
 

@@ -366,3 +366,12 @@ def test_prefill_matches_sdpa_under_slide7_mask(golden):
     v = np.repeat(synth.widen(x.v, "bf16"), 2, axis=1)[0]
     want = sdpa(synth.widen(x.q, "bf16")[0], k, v, 0.2, mask=np.broadcast_to(M, (4, P, P)))
     np.testing.assert_allclose(out, want, rtol=0, atol=1e-12)
+
+
+def test_hier_given_selection_reproduces_own_selection():
+    """Evaluating the attention for the oracle's own selection gives the same output."""
+    h, x = _hier_small(n1=41, group=4, k2=3, k1=5)
+    t = x.tensors()
+    idx2, idx1, out = oracle.hier_decode(t, h.group, h.top_k2, h.l1.top_k)
+    _, _, out2 = oracle.hier_decode(t, h.group, h.top_k2, h.l1.top_k, given=(idx2, idx1))
+    np.testing.assert_array_equal(out, out2)

@@ -117,7 +117,9 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup(gpus: int):
+def dist_setup(gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun env).  Only the barrier and the timing
+    reduction use the process group; the data path has no collective."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -126,20 +128,30 @@ def dist_setup(gpus: int):
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return world, rank, local
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank value (device time) over all ranks."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(steps_per_rank: int, world: int, ms_max: float) -> float:
+    """Steps of all ranks divided by the slowest rank's time (weak scaling)."""
+    return world * steps_per_rank / (ms_max / 1e3)
 
 
 def barrier(world: int):
@@ -241,7 +253,7 @@ def run_ours(args, world, rank, local):
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
 
     per_step_ms = ms_max / args.steps
-    steps_per_s = world * args.steps / (ms_max / 1e3)
+    steps_per_s = whole_job_rate(args.steps, world, ms_max)
     gbs = nbytes_step / (per_step_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
     line = {
@@ -269,7 +281,7 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "kernel": "gsa_decode_step (gist pass + unfold pass, one step)",
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                      "peak_kind": peak_kind, "traffic": None},
-        "e2e": {"value": round(world * args.steps / (e2e_ms / 1e3), 2), "unit": "steps/s",
+        "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()
                 + idx_host.numel() * idx_host.element_size()},

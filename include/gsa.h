@@ -43,8 +43,8 @@
  *    launch failure returns GSA_ERR_CUDA.  Nothing is printed, no exception
  *    crosses the ABI.  Device-side anomalies (an out-of-range chunk index
  *    passed to gsa_unfold_attn, an expired bounded wait) never fault: the
- *    kernel skips the access and ORs a flag into the workspace error word,
- *    which gsa_workspace_error() reads back.
+ *    kernel clamps the index into range (or abandons the wait) and ORs a flag
+ *    into the workspace error word, which gsa_workspace_error() reads back.
  */
 #ifndef GSA_H_
 #define GSA_H_
@@ -130,7 +130,7 @@ gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* i
  * [SL-17]).  For every query head h of KV head hk the softmax of
  * scale * q_h . K over the context of desc->mode, times V, where the selected
  * chunks are idx[b][hk][0..k) (distinct, in [0, N); an index out of range is
- * skipped and flagged).  lse (nullable) [B][Hq] receives the natural-log
+ * clamped into range and flagged).  lse (nullable) [B][Hq] receives the natural-log
  * sum of exp(scale * q.K) over the context.                               */
 gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist,
                            const void* v_gist, const void* k_raw, const void* v_raw,

@@ -169,6 +169,30 @@ gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void*
 gsa_status gsa_gist_prefill(const gsa_prefill_desc* desc, const void* q, const void* k,
                             const void* v, void* out, float* lse, void* stream);
 
+/* gsa_decode_step without a caller-provided workspace.  No counterpart in the
+ * paper: this is a deployment convenience.  Some callers cannot allocate
+ * device memory at the point where they run a decode step — for instance
+ * plugin or engine code whose enqueue path is forbidden to allocate, or a
+ * server that plans all of its device memory up front and hands out no
+ * per-call buffers.  This entry point allocates nothing: it uses a scratch
+ * array of 8 MiB that is part of the library's device image (every GPU that
+ * loads the library holds it until the process exits).
+ *  - Arguments, layouts and results are those of gsa_decode_step.
+ *  - Descriptors whose workspace (gsa_decode_workspace_size) exceeds 8 MiB
+ *    are rejected with GSA_ERR_WORKSPACE.
+ *  - The first call on a device looks up the array's device address for that
+ *    device; make that first call before any stream capture on the device.
+ *  - Each call clears the scratch words that must start at zero
+ *    (cudaMemsetAsync on `stream`), then runs the decode step in it.
+ *  - All calls share the one array: calls whose work overlaps on the GPU
+ *    (different streams, or different host threads) race and corrupt each
+ *    other's results.  Serialise them on one stream.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.           */
+gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, const void* k_gist,
+                                   const void* v_gist, const void* k_raw, const void* v_raw,
+                                   const void* k_tail, const void* v_tail, int32_t* idx_out,
+                                   float* scores_out, void* out, void* stream);
+
 /* Reads (synchronously, on `stream`) the workspace error word: 0, or an OR of
  * GSA_WS_ERR_* flags; returns GSA_ERR_TIMEOUT if a bounded wait expired,
  * GSA_ERR_ARG if an index was out of range, else GSA_OK.  flags_out nullable. */

@@ -23,7 +23,7 @@ GSA_WS_ERR_TIMEOUT, GSA_WS_ERR_INDEX = 1, 2
 # Every function the C header declares (checked by the tests).
 EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", "gsa_topk",
            "gsa_unfold_attn", "gsa_decode_step", "gsa_hier_decode", "gsa_gist_prefill",
-           "gsa_workspace_error", "gsa_status_string")
+           "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc")
 
 
 class GsaError(RuntimeError):
@@ -64,6 +64,7 @@ def _signatures():
         "gsa_topk": (st, [pd, vp, vp, vp]),
         "gsa_unfold_attn": (st, [pd] + [vp] * 10 + [vp, sz, vp]),
         "gsa_decode_step": (st, [pd] + [vp] * 11 + [sz, vp]),
+        "gsa_decode_step_noalloc": (st, [pd] + [vp] * 10 + [vp]),
         "gsa_hier_decode": (st, [ph] + [vp] * 13 + [sz, vp]),
         "gsa_gist_prefill": (st, [pp, vp, vp, vp, vp, vp, vp]),
         "gsa_workspace_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
@@ -175,6 +176,15 @@ def gsa_decode_step(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_o
     _check(lib().gsa_decode_step(ctypes.byref(desc), _ptr(q), _ptr(k_gist), _ptr(v_gist), _ptr(k_raw),
                                  _ptr(v_raw), _ptr(k_tail), _ptr(v_tail), _ptr(idx_out), _ptr(scores_out),
                                  _ptr(out), _ptr(ws), nb, _stream(stream)), "gsa_decode_step")
+
+
+def gsa_decode_step_noalloc(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, scores_out, out,
+                            stream=None):
+    """gsa_decode_step for callers that cannot allocate: the scratch is a fixed
+    8 MiB device array inside the library (see include/gsa.h)."""
+    _check(lib().gsa_decode_step_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k_gist), _ptr(v_gist), _ptr(k_raw),
+                                         _ptr(v_raw), _ptr(k_tail), _ptr(v_tail), _ptr(idx_out), _ptr(scores_out),
+                                         _ptr(out), _stream(stream)), "gsa_decode_step_noalloc")
 
 
 def gsa_hier_decode(desc, q, k_g2, v_g2, k_g1, v_g1, k_raw, v_raw, k_tail, v_tail, idx2_out, idx1_out, out,

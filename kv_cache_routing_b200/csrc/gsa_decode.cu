@@ -20,6 +20,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "gsa_attn.cuh"
 #include "gsa_plan.h"
@@ -760,6 +761,50 @@ gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void*
     u.slot_stride = hp.SA2 + hp.SA1;
     if (kern.unfold(u, strm) != cudaSuccess) return GSA_ERR_CUDA;
     return GSA_OK;
+}
+
+// ------------------------------------------------ no-allocation variant ----
+// Scratch for gsa_decode_step_noalloc: a fixed device array that lives as long
+// as the library is loaded, so that callers who may not allocate device memory
+// can still run a decode step.  Its size is the largest workspace the variant
+// accepts.
+constexpr size_t kStaticWsBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+
+// Device address of g_static_ws on each device, resolved once per device with
+// that device current.  (In host code the symbol itself is only a stand-in.)
+static void* static_ws_address(int device) {
+    static std::mutex mu;
+    static void* addr[128] = {};
+    if (device < 0 || device >= 128) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[device] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess) return nullptr;
+        addr[device] = p;
+    }
+    return addr[device];
+}
+
+gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, const void* k_gist,
+                                   const void* v_gist, const void* k_raw, const void* v_raw, const void* k_tail,
+                                   const void* v_tail, int32_t* idx_out, float* scores_out, void* out,
+                                   void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
+    if (!aligned16(idx_out) || !aligned16(scores_out)) return GSA_ERR_ALIGN;
+    const DecodePlan pl = make_decode_plan(*desc);
+    if (pl.total > kStaticWsBytes) return GSA_ERR_WORKSPACE;
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess) return GSA_ERR_CUDA;
+    void* ws = static_ws_address(device);
+    if (ws == nullptr) return GSA_ERR_CUDA;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    // the error word and the tickets must start at zero
+    if (cudaMemsetAsync(ws, 0, pl.off_scores, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    return gsa_decode_step(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, scores_out, out, ws,
+                           pl.total, stream);
 }
 
 gsa_status gsa_workspace_error(const void* ws, uint32_t* flags_out, void* stream) {

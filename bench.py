@@ -188,6 +188,7 @@ def run_ours(args, world, rank, local):
         reps.append(t)
     desc = desc_of(s)
     wsz = gsa.gsa_decode_workspace_size(desc)
+    launches = gsa.gsa_decode_launch_count(desc)
     outs = [torch.empty((s.batch, s.n_q_heads, s.head_dim), dtype=tdtype(s.dtype), device="cuda") for _ in range(L)]
     idxs = [torch.empty((s.batch, s.n_kv_heads, s.top_k), dtype=torch.int32, device="cuda") for _ in range(L)]
     ws = torch.zeros(wsz, dtype=torch.uint8, device="cuda")
@@ -278,14 +279,14 @@ def run_ours(args, world, rank, local):
                          f"(L2 {l2 / 1e6:.0f} MB)"},
         "head_steps_per_s": round(steps_per_s * s.batch * s.n_q_heads, 1),
         "algorithmic_bytes_per_step": nbytes_step,
-        "roofline": {"bound": "hbm", "kernel": "gsa_decode_step (gist pass + unfold pass, one step)",
+        "roofline": {"bound": "hbm", "kernel": f"gsa_decode_step ({launches} launches per step, one step)",
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                      "peak_kind": peak_kind, "traffic": None},
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()
                 + idx_host.numel() * idx_host.element_size()},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

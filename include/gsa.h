@@ -193,6 +193,11 @@ gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, c
                                    const void* k_tail, const void* v_tail, int32_t* idx_out,
                                    float* scores_out, void* out, void* stream);
 
+/* Number of kernel launches one gsa_decode_step call with this descriptor
+ * enqueues (for launch accounting and graph sizing); -1 if the descriptor is
+ * invalid.  Host only, enqueues nothing. */
+int gsa_decode_launch_count(const gsa_decode_desc* desc);
+
 /* Reads (synchronously, on `stream`) the workspace error word: 0, or an OR of
  * GSA_WS_ERR_* flags; returns GSA_ERR_TIMEOUT if a bounded wait expired,
  * GSA_ERR_ARG if an index was out of range, else GSA_OK.  flags_out nullable. */

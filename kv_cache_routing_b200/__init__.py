@@ -23,7 +23,7 @@ GSA_WS_ERR_TIMEOUT, GSA_WS_ERR_INDEX = 1, 2
 # Every function the C header declares (checked by the tests).
 EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", "gsa_topk",
            "gsa_unfold_attn", "gsa_decode_step", "gsa_hier_decode", "gsa_gist_prefill",
-           "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc")
+           "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count")
 
 
 class GsaError(RuntimeError):
@@ -69,6 +69,7 @@ def _signatures():
         "gsa_gist_prefill": (st, [pp, vp, vp, vp, vp, vp, vp]),
         "gsa_workspace_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
         "gsa_status_string": (ctypes.c_char_p, [st]),
+        "gsa_decode_launch_count": (ctypes.c_int, [pd]),
     }
 
 
@@ -198,6 +199,14 @@ def gsa_hier_decode(desc, q, k_g2, v_g2, k_g1, v_g1, k_raw, v_raw, k_tail, v_tai
 def gsa_gist_prefill(desc, q, k, v, out, lse=None, stream=None):
     _check(lib().gsa_gist_prefill(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                   _stream(stream)), "gsa_gist_prefill")
+
+
+def gsa_decode_launch_count(desc) -> int:
+    """Kernel launches one gsa_decode_step with `desc` enqueues."""
+    n = lib().gsa_decode_launch_count(ctypes.byref(desc))
+    if n < 0:
+        raise GsaError(1, "gsa_decode_launch_count")
+    return int(n)
 
 
 def gsa_workspace_error(ws, stream=None) -> int:

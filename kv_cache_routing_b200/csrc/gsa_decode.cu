@@ -23,6 +23,7 @@
 #include <mutex>
 
 #include "gsa_attn.cuh"
+#include "gsa_fused.h"
 #include "gsa_plan.h"
 
 namespace gsa {
@@ -575,6 +576,12 @@ static PassParams make_params(const DecodePlan& pl, const gsa_decode_desc& d, co
     return p;
 }
 
+// Workspace bytes of a flat decode descriptor on the path it will take.
+static size_t decode_ws_bytes(const gsa_decode_desc& d) {
+    return fused_supported(d) ? std::max(make_fused_plan(d).total, make_fused_plan(d, true).total)
+                              : make_decode_plan(d).total;
+}
+
 }  // namespace gsa
 
 // ================================================================ C ABI ====
@@ -584,7 +591,7 @@ extern "C" {
 
 size_t gsa_decode_workspace_size(const gsa_decode_desc* desc) {
     if (validate_decode(desc) != GSA_OK) return 0;
-    return make_decode_plan(*desc).total;
+    return decode_ws_bytes(*desc);
 }
 
 gsa_status gsa_score(const gsa_decode_desc* desc, const void* q, const void* k_gist, float* scores,
@@ -633,8 +640,8 @@ static gsa_status check_tensors(const gsa_decode_desc* d, const void* q, const v
     return GSA_OK;
 }
 
-static gsa_status check_ws(const DecodePlan& pl, const void* ws, size_t ws_bytes) {
-    if (!ws || ws_bytes < pl.total) return GSA_ERR_WORKSPACE;
+static gsa_status check_ws(size_t need, const void* ws, size_t ws_bytes) {
+    if (!ws || ws_bytes < need) return GSA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return GSA_ERR_WORKSPACE;
     return GSA_OK;
 }
@@ -647,8 +654,11 @@ gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const voi
     if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
     if (desc->top_k > 0 && (!idx || !aligned16(idx))) return idx ? GSA_ERR_ALIGN : GSA_ERR_ARG;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GSA_ERR_ALIGN;
+    if ((st = check_ws(decode_ws_bytes(*desc), ws, ws_bytes)) != GSA_OK) return st;
+    if (fused_supported(*desc))
+        return fused_launch(*desc, make_fused_plan(*desc, true), q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx,
+                            nullptr, nullptr, out, lse, ws, static_cast<cudaStream_t>(stream));
     DecodePlan pl = make_decode_plan(*desc);
-    if ((st = check_ws(pl, ws, ws_bytes)) != GSA_OK) return st;
     PassParams p = make_params(pl, *desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ws);
     p.idx_in = idx;
     p.out = static_cast<uint8_t*>(out);
@@ -668,8 +678,11 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
     if (st != GSA_OK) return st;
     if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
     if (!aligned16(idx_out) || !aligned16(scores_out)) return GSA_ERR_ALIGN;
+    if ((st = check_ws(decode_ws_bytes(*desc), ws, ws_bytes)) != GSA_OK) return st;
+    if (fused_supported(*desc))
+        return fused_launch(*desc, make_fused_plan(*desc), q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, nullptr,
+                            idx_out, scores_out, out, nullptr, ws, static_cast<cudaStream_t>(stream));
     DecodePlan pl = make_decode_plan(*desc);
-    if ((st = check_ws(pl, ws, ws_bytes)) != GSA_OK) return st;
     PassParams p = make_params(pl, *desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ws);
     if (scores_out) p.scores = scores_out;
     if (idx_out) p.idx_out = idx_out;
@@ -794,17 +807,24 @@ gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, c
     if (st != GSA_OK) return st;
     if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
     if (!aligned16(idx_out) || !aligned16(scores_out)) return GSA_ERR_ALIGN;
-    const DecodePlan pl = make_decode_plan(*desc);
-    if (pl.total > kStaticWsBytes) return GSA_ERR_WORKSPACE;
+    const size_t need = decode_ws_bytes(*desc);
+    if (need > kStaticWsBytes) return GSA_ERR_WORKSPACE;
     int device = 0;
     if (cudaGetDevice(&device) != cudaSuccess) return GSA_ERR_CUDA;
     void* ws = static_ws_address(device);
     if (ws == nullptr) return GSA_ERR_CUDA;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
-    // the error word and the tickets must start at zero
-    if (cudaMemsetAsync(ws, 0, pl.off_scores, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    // the error word and the tickets (the words before the first data region) must start at zero
+    const size_t head = fused_supported(*desc) ? make_fused_plan(*desc).off_scores : make_decode_plan(*desc).off_scores;
+    if (cudaMemsetAsync(ws, 0, head, strm) != cudaSuccess) return GSA_ERR_CUDA;
     return gsa_decode_step(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, scores_out, out, ws,
-                           pl.total, stream);
+                           need, stream);
+}
+
+int gsa_decode_launch_count(const gsa_decode_desc* desc) {
+    if (validate_decode(desc) != GSA_OK) return -1;
+    if (fused_supported(*desc)) return make_fused_plan(*desc).grid > 0 ? 2 : 1;
+    return (desc->n_chunks > 0 ? 1 : 0) + 1;
 }
 
 gsa_status gsa_workspace_error(const void* ws, uint32_t* flags_out, void* stream) {

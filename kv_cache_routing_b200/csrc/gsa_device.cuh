@@ -14,9 +14,8 @@ namespace gsa {
 
 constexpr uint32_t kErrTimeout = 1u;   // matches GSA_WS_ERR_TIMEOUT
 constexpr uint32_t kErrIndex = 2u;     // matches GSA_WS_ERR_INDEX
-// try_wait suspends the thread for a hardware-chosen interval per probe; this
-// many probes bound one wait to well under a few seconds.
-constexpr uint32_t kSpinLimit = 1u << 22;
+// A bounded wait gives up after this many nanoseconds of %globaltimer time.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -43,23 +42,36 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
+    // the suspend-time hint (ns) lets the thread sleep until the phase
+    // completes instead of spinning on the issue slots
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
         : "memory");
     return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete; gives up after kSpinLimit
-// probes, ORs kErrTimeout into *err and returns false.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of `bar` to complete; after kWaitLimitNs it gives
+// up, ORs kErrTimeout into *err and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    atomicOr(err, kErrTimeout);
-    return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, kErrTimeout);
+            return false;
+        }
+    }
+    return true;
 }
 
 // ------------------------------------------------------------- bulk copies --
@@ -199,9 +211,17 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += NT) hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += NT) {
-            uint32_t u = key(i);
-            if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+        // warp-aggregated histogram: float keys crowd a few bins in the high
+        // digits, so lanes with the same bin add once per warp instruction
+        for (int i0 = tid - (tid & 31); i0 < n; i0 += NT) {
+            const int i = i0 + (tid & 31);
+            uint32_t bin = 0xFFFFFFFFu;
+            if (i < n) {
+                const uint32_t u = key(i);
+                if ((u & pmask) == prefix) bin = (u >> shift) & 255u;
+            }
+            const uint32_t same = __match_any_sync(0xFFFFFFFFu, bin);
+            if (bin != 0xFFFFFFFFu && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
         }
         __syncthreads();
         if (tid < 32) {
@@ -260,6 +280,272 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
         else if (u == T) { take = e < kk; ++e; }
         if (take) emit(static_cast<int>(r++), i);
     }
+}
+
+
+// ------------------------------------------------- shared-memory top-k --
+// Exact top-k of n orderable keys held in shared memory (keys[i] for
+// position i): the k largest keys, equal keys taken lowest position first.
+// Writes the k selected positions to out[0..k) in ascending order.
+// Radix select, 8 bits per digit, compacting the candidates after every
+// digit (keys above the threshold digit are selected at once, keys on it
+// stay candidates), so only the first digit reads all n keys; the selection
+// is kept as a bitmap and emitted in position order by a popcount prefix.
+// Scratch `w` (shared): >= 256 + 16 + 2*NT/32 + (n+31)/32 * 2 + 2*n words
+// (histogram, control, scan, two bitmaps, two candidate lists).
+// All NT threads of the block call it.
+template <int NT>
+__device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint32_t* w) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = NT / 32;
+    if (k <= 0 || n <= 0) return;
+    if (k >= n) {
+        for (int i = tid; i < n; i += NT) out[i] = i;
+        return;
+    }
+    const int nw = (n + 31) >> 5;
+    uint32_t* hist = w;                   // 256
+    uint32_t* ctl = w + 256;              // [0] digit, [1] above, [2] next count, [3] done flag
+    uint32_t* scan = ctl + 16;            // 2 * NW
+    uint32_t* sel = scan + 2 * NW;        // nw words: selected positions
+    uint32_t* tie = sel + nw;             // nw words: candidates left after the last digit
+    uint32_t* cand = tie + nw;            // candidate positions (unordered), read list
+    uint32_t* next = cand + n;            // write list; the two swap after every digit
+    for (int i = tid; i < nw; i += NT) {
+        sel[i] = 0;
+        tie[i] = 0;
+    }
+    uint32_t kk = (uint32_t)k;
+    int m = n;                            // candidates: all positions on the first digit
+    bool all = true;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += NT) hist[i] = 0;
+        if (tid == 0) ctl[2] = 0;
+        __syncthreads();
+        for (int i0 = tid - lane; i0 < m; i0 += NT) {
+            const int i = i0 + lane;
+            uint32_t bin = 0xFFFFFFFFu;
+            if (i < m) bin = (keys[all ? i : cand[i]] >> shift) & 255u;
+            const uint32_t same = __match_any_sync(0xFFFFFFFFu, bin);
+            if (bin != 0xFFFFFFFFu && lane == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns bins 255-8l .. 248-8l (descending)
+            uint32_t cnt[8], tot = 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                cnt[t] = hist[255 - 8 * lane - t];
+                tot += cnt[t];
+            }
+            uint32_t incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            uint32_t above = incl - tot;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                if (above < kk && above + cnt[t] >= kk) {
+                    ctl[0] = 255u - 8u * lane - t;
+                    ctl[1] = above;
+                }
+                above += cnt[t];
+            }
+        }
+        __syncthreads();
+        const uint32_t D = ctl[0], above = ctl[1];
+        const bool last = shift == 0;
+        // keys above the threshold digit are selected; keys on it stay
+        // candidates (warp-aggregated: one atomic per warp and predicate)
+        for (int i0 = tid - lane; i0 < m; i0 += NT) {
+            const int i = i0 + lane;
+            int pos = 0;
+            uint32_t dg = 0;
+            if (i < m) {
+                pos = all ? i : (int)cand[i];
+                dg = (keys[pos] >> shift) & 255u;
+            }
+            const bool up = i < m && dg > D, eq = i < m && dg == D;
+            const uint32_t mup = __ballot_sync(0xFFFFFFFFu, up);
+            const uint32_t meq = __ballot_sync(0xFFFFFFFFu, eq);
+            if (all) {
+                // positions i0..i0+31 are exactly one bitmap word (i0 is a multiple of 32)
+                if (lane == 0) {
+                    if (mup) sel[i0 >> 5] |= mup;
+                    if (last && meq) tie[i0 >> 5] |= meq;
+                }
+            } else {
+                if (up) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+                if (last && eq) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+            }
+            if (!last && meq) {
+                uint32_t base = 0;
+                if (lane == 0) base = atomicAdd(&ctl[2], (uint32_t)__popc(meq));
+                base = __shfl_sync(0xFFFFFFFFu, base, 0);
+                if (eq) next[base + __popc(meq & ((1u << lane) - 1u))] = (uint32_t)pos;
+            }
+        }
+        __syncthreads();
+        kk -= above;
+        m = (int)ctl[2];
+        all = false;
+        {
+            uint32_t* t = cand;
+            cand = next;
+            next = t;
+        }
+        __syncthreads();
+        if (!last && (uint32_t)m == kk) {
+            // every remaining candidate is selected
+            for (int i = tid; i < m; i += NT) atomicOr(&sel[cand[i] >> 5], 1u << (cand[i] & 31));
+            kk = 0;
+            __syncthreads();
+            break;
+        }
+    }
+    // equal keys on the threshold: the kk lowest positions (tie bitmap in position order)
+    if (kk > 0) {
+        uint32_t c = 0;
+        const int per = (nw + NT - 1) / NT, lo = tid * per, hi = min(nw, lo + per);
+        for (int i = lo; i < hi; ++i) c += __popc(tie[i]);
+        uint32_t tot;
+        uint32_t before = block_exclusive_scan<NT>(c, scan, &tot);
+        for (int i = lo; i < hi; ++i) {
+            uint32_t bits = tie[i];
+            while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1;
+                if (before < kk) atomicOr(&sel[i], 1u << b);
+                ++before;
+            }
+        }
+        __syncthreads();
+    }
+    // emit the selection in ascending position order
+    {
+        uint32_t c = 0;
+        const int per = (nw + NT - 1) / NT, lo = tid * per, hi = min(nw, lo + per);
+        for (int i = lo; i < hi; ++i) c += __popc(sel[i]);
+        uint32_t tot;
+        uint32_t r = block_exclusive_scan<NT>(c, scan, &tot);
+        for (int i = lo; i < hi; ++i) {
+            uint32_t bits = sel[i];
+            while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1;
+                out[r++] = i * 32 + b;
+            }
+        }
+    }
+}
+
+
+// --------------------------------------------------- threshold top-k --
+// Exact top-k for k <= 32 of n <= NT * M keys held in shared memory (keys[i]
+// for position i): the k largest keys, equal keys taken lowest position
+// first; out[0..k) receives the positions in ascending order.
+//  1. Thread t holds the block of positions [t*m, t*m + m), m = ceil(n / NT).
+//  2. In each warp, the k-th largest of the 32 lane maxima bounds the k-th
+//     largest key of the whole set from below (k distinct keys reach it), so
+//     the largest such bound over the warps, tau, does as well.
+//  3. The keys >= tau (k of them at least, and rarely many more) are compacted
+//     in position order; each counts the candidates ahead of it (a larger key,
+//     or the same key at a lower position), and those with fewer than k ahead
+//     are written out in position order.
+// Returns false without writing anything when more than NT keys reach tau
+// (a flood of equal keys): the caller then runs a general selection.
+// Scratch `w` (shared): >= 2 * NT + 2 * (NT / 32) + 8 words.
+// All NT threads call it; it ends with the block synchronised.
+template <int NT, int M>
+__device__ bool threshold_topk(const uint32_t* keys, int n, int k, int32_t* out, uint32_t* w) {
+    constexpr int NW = NT / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m = (n + NT - 1) / NT;
+    const int lo = tid * m;
+    const int mine = max(0, min(m, n - lo));
+    uint32_t key[M];
+    uint32_t tmax = 0u;
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        key[i] = i < mine ? keys[lo + i] : 0u;
+        tmax = max(tmax, key[i]);
+    }
+    // rank of this lane's maximum in its warp (equal values ordered by lane):
+    // the lane of rank k-1 holds the warp's bound (a lane without keys offers
+    // 0, the smallest key, which can only weaken the bound)
+    int ahead = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const uint32_t v = __shfl_sync(0xFFFFFFFFu, tmax, j);
+        ahead += (v > tmax || (v == tmax && j < lane)) ? 1 : 0;
+    }
+    const uint32_t at = __ballot_sync(0xFFFFFFFFu, ahead == k - 1);
+    const uint32_t tau_w = __shfl_sync(0xFFFFFFFFu, tmax, __ffs(at) - 1);
+    if (lane == 0) w[warp] = tau_w;
+    __syncthreads();
+    uint32_t tau = w[0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) tau = max(tau, w[i]);
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < M; ++i) c += (i < mine && key[i] >= tau) ? 1u : 0u;
+    uint32_t total;
+    uint32_t off = block_exclusive_scan<NT>(c, w + NW, &total);
+    if (total > (uint32_t)NT) return false;       // the same on every thread
+    uint32_t* ckey = w + 2 * NW + 8;   // 16-byte aligned when w is
+    uint32_t* cpos = ckey + NT;
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+        if (i < mine && key[i] >= tau) {
+            ckey[off] = key[i];
+            cpos[off] = (uint32_t)(lo + i);
+            ++off;
+        }
+    // pad the list to a multiple of 4 with key 0: a pad is never ahead of a
+    // candidate (it is not larger, and an equal one sits at a higher index)
+    if ((uint32_t)tid < ((total + 3u) & ~3u) - total) ckey[total + tid] = 0u;
+    __syncthreads();
+    uint32_t sel = 0, pos = 0;
+    if ((uint32_t)tid < total) {
+        const uint32_t mk = ckey[tid];
+        int a = 0;
+        const uint4* c4 = reinterpret_cast<const uint4*>(ckey);
+        for (int j = 0; j < (int)(total + 3u) / 4; ++j) {
+            const uint4 v = c4[j];
+            const int jb = 4 * j;
+            a += (v.x > mk || (v.x == mk && jb + 0 < tid)) ? 1 : 0;
+            a += (v.y > mk || (v.y == mk && jb + 1 < tid)) ? 1 : 0;
+            a += (v.z > mk || (v.z == mk && jb + 2 < tid)) ? 1 : 0;
+            a += (v.w > mk || (v.w == mk && jb + 3 < tid)) ? 1 : 0;
+        }
+        sel = a < k ? 1u : 0u;
+        pos = cpos[tid];
+    }
+    uint32_t nsel;
+    const uint32_t r = block_exclusive_scan<NT>(sel, w + NW, &nsel);
+    if (sel) out[r] = (int32_t)pos;
+    __syncthreads();
+    return true;
+}
+
+// ----------------------------------------------------- per-thread copies --
+// 16-byte global -> shared copy that bypasses L1 (cp.async, tracked per thread).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// Zero 16 bytes of shared memory through the same path (source size 0 reads nothing).
+__device__ __forceinline__ void cp_async16_zero(void* dst, const void* any_global) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 0;" ::"r"(smem_u32(dst)), "l"(any_global) : "memory");
+}
+// One arrival on `bar` once every cp.async this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// `count` arrivals on `bar` at once.
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 
 }  // namespace gsa

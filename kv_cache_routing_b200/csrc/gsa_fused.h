@@ -1,0 +1,64 @@
+// Host interface of the fused tensor-core decode step (bf16, head_dim 128).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "gsa_plan.h"
+
+namespace gsa {
+
+constexpr int kFusedCtas = 148;   // one persistent CTA per B200 SM (work split is fixed by this, not the device)
+constexpr int kSelCap = 2048;     // largest top_k of the tensor-core path (selection kept in shared memory)
+constexpr int kMaxTpc = 8;        // largest number of gathered tiles one phase-B CTA takes
+
+struct FusedPlan {
+    int rows, G, tg, tt, upr, grid;   // phase A: units per row, Stream-K grid
+    int T;                            // phase A: units in all
+    int maxs;                         // phase A: most CTAs meeting one row (its partial slots)
+    int nrows_g, nbt, tpc, cb, grid_b;   // phase B: gathered rows / tiles per row, tiles per CTA, CTAs per row, grid
+    int slot_stride;                  // maxs + cb
+    int sel_direct;                   // phase B selects from the scores (else from phase-A candidates)
+    size_t off_scores, off_cand_key, off_cand_idx, off_idx, off_part, off_ml, total;
+};
+
+namespace fused {
+struct Params {
+    CUtensorMap tm_kg, tm_vg;      // gists  [rows][N][d], box {64, 128, 1}
+    CUtensorMap tm_kt, tm_vt;      // tail   [rows][W][d], box {64, 128, 1}
+    const uint16_t* q;             // [B][Hq][d]
+    const uint8_t* kr;             // raw K/V and gist K/V base pointers (gathered tiles)
+    const uint8_t* vr;
+    const uint8_t* kgp;
+    const uint8_t* vgp;
+    uint16_t* out;                 // [B][Hq][d]
+    float* lse;                    // [B][Hq] or null
+    float* scores;                 // [rows][N]
+    int32_t* idx;                  // [rows][K]: written by the selection, or given
+    uint32_t* err;
+    uint32_t* cnt;                 // [rows] phase-B tickets
+    uint32_t* cand_key;            // [rows][N] local top-k candidates (orderable score keys)
+    int32_t* cand_idx;             // [rows][N] their gist indices
+    float* part;                   // [rows][slot_stride][G][d]
+    float* ml;                     // [rows][slot_stride][G][4]: (m, l, unused, unused)
+    int rows, Hkv, G, N, NA, C, K, W, mode;
+    int tg, upr, grid, slot_stride, maxs;
+    int nrows_g, nbt, tpc, cb;
+    int phase;                     // 0: phase A (launch 1), 1: phase B (launch 2)
+    int T;                         // phase-A units in all
+    float c2;
+    int do_score, do_topk, do_attn_gists, sel_direct;
+};
+}  // namespace fused
+
+bool fused_supported(const gsa_decode_desc& d);
+// given: the selection is supplied (gsa_unfold_attn), so nothing is scored.
+FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given = false);
+// Enqueue the fused decode step.  idx_given != null: attend over that
+// selection (no scores, no selection); else select and write idx_out (or the
+// workspace copy) and scores_out (or the workspace copy).
+gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void* q, const void* kg, const void* vg,
+                        const void* kr, const void* vr, const void* kt, const void* vt, const int32_t* idx_given,
+                        int32_t* idx_out, float* scores_out, void* out, float* lse, void* ws, cudaStream_t st);
+
+}  // namespace gsa

@@ -44,6 +44,9 @@ constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, 0, 0);   // Q (K-major) x 
 constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, 128, 0, 1);  // P (K-major) x V (MN-major)
 constexpr float kRescaleLog2 = 8.f;
 
+// Error word of the prefill's bounded waits (the prefill takes no workspace).
+__device__ uint32_t g_prefill_err;
+
 struct PrefillParams {
     CUtensorMap tm_q;    // [B*Hq][P][d]
     CUtensorMap tm_k;    // [B*Hkv][P][d]
@@ -108,7 +111,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
     tc::fence_after();
     const uint32_t tmem = bars.tmem;
     const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
-    uint32_t err_dummy = 0;   // waits below are bounded; a timeout abandons the tile
+    uint32_t* err = &g_prefill_err;   // waits below are bounded; a timeout abandons the tile
 
     if (warp == 4) {
         if (lane == 0) {
@@ -144,18 +147,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
             tc::tma_load_3d(base + SM_Q, &p.tm_q, 0, p0, bh, &bars.q_full);
             tc::tma_load_3d(base + SM_Q + 16384, &p.tm_q, 64, p0, bh, &bars.q_full);
             for (int i = 0; i < min(2, n_kv); ++i) load_kv(i, i);
-            bool ok = mbar_wait(&bars.q_full, 0, &err_dummy) && mbar_wait(&bars.kv_full[0], 0, &err_dummy);
+            bool ok = mbar_wait(&bars.q_full, 0, err) && mbar_wait(&bars.kv_full[0], 0, err);
             tc::fence_after();
             if (ok) issue_s(0);
             for (int i = 0; ok && i < n_kv; ++i) {
                 if (i + 1 < n_kv) {
-                    ok = mbar_wait(&bars.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1, &err_dummy) &&
-                         mbar_wait(&bars.s_free, i & 1, &err_dummy);
+                    ok = mbar_wait(&bars.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1, err) &&
+                         mbar_wait(&bars.s_free, i & 1, err);
                     tc::fence_after();
                     if (!ok) break;
                     issue_s(i + 1);
                 }
-                if (!mbar_wait(&bars.p_full[i & 1], (i >> 1) & 1, &err_dummy)) break;
+                if (!mbar_wait(&bars.p_full[i & 1], (i >> 1) & 1, err)) break;
                 tc::fence_after();
                 const uint32_t pb = sbase + SM_P + (i & 1) * 32768;
                 const uint32_t vs = sbase + SM_KV + (i & 1) * 65536 + 32768;
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
                 tc::commit(&bars.o_done[i & 1]);
                 tc::commit(&bars.kv_empty[i & 1]);
                 if (i + 2 < n_kv) {
-                    if (!mbar_wait(&bars.kv_empty[i & 1], (i >> 1) & 1, &err_dummy)) break;
+                    if (!mbar_wait(&bars.kv_empty[i & 1], (i >> 1) & 1, err)) break;
                     load_kv(i + 2, i & 1);
                 }
             }
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
         float m_run = -INFINITY, l_run = 0.f;
         float s[128];
         for (int i = 0; i < n_kv; ++i) {
-            if (!mbar_wait(&bars.s_full, i & 1, &err_dummy)) break;
+            if (!mbar_wait(&bars.s_full, i & 1, err)) break;
             tc::fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
             const float alpha = need ? exp2f(m_run - m_new) : 1.f;
             if (__any_sync(0xFFFFFFFFu, need) && i > 0) {
                 // O holds P.V of tiles < i: wait for the last of them, then rescale
-                mbar_wait(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &err_dummy);
+                mbar_wait(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1, err);
                 tc::fence_after();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
             }
             m_run = m_new;
             // the P buffer of this tile was last read by the P.V MMA of tile i-2
-            if (i >= 2) mbar_wait(&bars.o_done[i & 1], ((i - 2) >> 1) & 1, &err_dummy);
+            if (i >= 2) mbar_wait(&bars.o_done[i & 1], ((i - 2) >> 1) & 1, err);
             uint8_t* prow = base + SM_P + (i & 1) * 32768 + r * 128;
             float sum = 0.f;
 #pragma unroll
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
             mbar_arrive(&bars.p_full[i & 1]);
         }
         // ------------------------------------------------------ epilogue ----
-        mbar_wait(&bars.o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, &err_dummy);
+        mbar_wait(&bars.o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, err);
         tc::fence_after();
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         uint16_t* orow = p.out + ((size_t)bh * p.P + qp) * PF_D;

@@ -63,6 +63,34 @@ def peaks():
     return 6650.0, "fallback"
 
 
+KERNEL_SOURCES = ("gsa_fused.cu", "gsa_fused.h", "gsa_device.cuh", "gsa_tc.cuh")
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the decode step from a committed ncu summary
+    under profiles/, or None when none covers this workload or the kernel
+    sources have changed since the counters were taken."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "kv_cache_routing_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        kv = {}
+        for line in open(path):
+            if ":" in line and not line.startswith(("#", "|", "-", " ")):
+                k, _, v = line.partition(":")
+                kv[k.strip()] = v.strip()
+        if kv.get("workload") == workload and kv.get("sources_sha256") == digest:
+            try:
+                return int(kv["dram_bytes_per_step"]) / int(kv["launches_per_step"])
+            except (KeyError, ValueError):
+                return None
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
 
@@ -279,9 +307,13 @@ def run_ours(args, world, rank, local):
                          f"(L2 {l2 / 1e6:.0f} MB)"},
         "head_steps_per_s": round(steps_per_s * s.batch * s.n_q_heads, 1),
         "algorithmic_bytes_per_step": nbytes_step,
-        "roofline": {"bound": "hbm", "kernel": f"gsa_decode_step ({launches} launches per step, one step)",
+        "roofline": {"bound": "hbm",
+                     "kernel": f"gsa_decode_step: {launches} launches per step of one kernel "
+                               f"(per launch: half the step's algorithmic bytes in half the step's time)",
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-                     "peak_kind": peak_kind, "traffic": None},
+                     "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": nbytes_step / launches,
+                     "traffic": measured_traffic(args.workload)},
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()

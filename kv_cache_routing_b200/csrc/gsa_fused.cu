@@ -166,9 +166,7 @@ struct Ctx {
     int warp, lane;
     // role counters (each role keeps its own copy; all roles see the same unit sequence)
     int tiles, segs, atiles;
-    // MMA role: previous attention tile waiting for its P.V
-    int prev_valid, prev_stage, prev_pj, prev_obuf, prev_first;
-    int first_attn;
+    int first_attn;   // MMA role: the next attention tile starts its segment
     // softmax role: running state of the current segment
     float m_run[16];
     float l_part[16];
@@ -216,61 +214,93 @@ __device__ __forceinline__ void produce(const Params& p, Ctx& cx, const Unit& u)
 }
 
 // ----------------------------------------------------------------- MMA --
-__device__ __forceinline__ void issue_pv(const Params& p, Ctx& cx) {
-    const int pj = cx.prev_pj;
-    const int pb = pj & 1;
-    cx.prev_valid = 0;
-    if (!mbar_wait(&cx.bars->p_full[pb], (pj >> 1) & 1, p.err)) return;
-    tc::fence_after();
-    const uint32_t vs = cx.sbase + SM_STAGE + cx.prev_stage * STAGE_BYTES + KV_BYTES;
-    const uint32_t pt = cx.sbase + SM_P + pb * 4096;
-    const uint32_t dO = cx.tmem + 32 + cx.prev_obuf * 16;
+// The MMA thread runs an event loop over its units: it issues a unit's S
+// product as soon as the unit's data, a free S buffer and (for a new segment)
+// its Q are there, and a pending P.V as soon as its P is there, whichever
+// comes first.  A stage is thus released right after its own P.V, not after
+// the next unit's data has arrived.
+struct PendingPV {
+    int stage, obuf, first, pj;
+};
+
+__device__ __forceinline__ void issue_pv(Ctx& cx, const PendingPV& r) {
+    const uint32_t vs = cx.sbase + SM_STAGE + r.stage * STAGE_BYTES + KV_BYTES;
+    const uint32_t pt = cx.sbase + SM_P + (r.pj & 1) * 4096;
+    const uint32_t dO = cx.tmem + 32 + r.obuf * 16;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
         tc::mma_bf16(dO, tc::sdesc_sw128(vs + kk * 2048, 16384, 1024),
                      tc::sdesc_sw128(pt + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), IDESC_PV,
-                     (cx.prev_first && kk == 0) ? 0u : 1u);
+                     (r.first && kk == 0) ? 0u : 1u);
     }
-    tc::commit(&cx.bars->o_done[pb]);
-    tc::commit(&cx.bars->empty[cx.prev_stage]);
+    tc::commit(&cx.bars->o_done[r.pj & 1]);
+    tc::commit(&cx.bars->empty[r.stage]);
 }
 
-__device__ __forceinline__ void mma_tile(const Params& p, Ctx& cx, const Unit& u, bool new_seg) {
-    const int gi = cx.tiles;
-    const int stage = gi % NS, sb = gi & 1;
-    cx.tiles = gi + 1;
-    if (new_seg) {
-        if (!mbar_wait(&cx.bars->q_ready[cx.segs & 1], (cx.segs >> 1) & 1, p.err)) return;
-        cx.segs++;
-        cx.first_attn = 1;
-    }
-    bool ok = mbar_wait(&cx.bars->full[stage], (gi / NS) & 1, p.err);
-    if (ok && gi >= 2) ok = mbar_wait(&cx.bars->s_free[sb], ((gi - 2) >> 1) & 1, p.err);
-    if (!ok) return;
-    tc::fence_after();
-    if (u.kind == 2) tc::fence_async_smem();   // cp.async (generic proxy) writes -> tensor core reads
-    const uint32_t ks = cx.sbase + SM_STAGE + stage * STAGE_BYTES;
-    const uint32_t qb = cx.sbase + SM_Q + ((cx.segs - 1) & 1) * 4096;
-    const uint32_t dS = cx.tmem + sb * 16;
+__device__ __forceinline__ void mma_loop(const Params& p, Ctx& cx, int u0, int row, int n) {
+    PendingPV ring[4];
+    int head = 0, tail = 0;   // pending P.V products [head, tail)
+    int next = 0;             // next unit whose S product is due
+    int prev_row = -1;
+    uint64_t t_last = global_ns();
+    while (next < n || head != tail) {
+        bool prog = false;
+        if (next < n && tail - head < 4) {
+            const Unit u = unit_at(p, u0, row, next);
+            const bool ns = u.row != prev_row;
+            const int gi = cx.tiles, stage = gi % NS, sb = gi & 1;
+            const bool ready = (!ns || mbar_test(&cx.bars->q_ready[cx.segs & 1], (cx.segs >> 1) & 1)) &&
+                               mbar_test(&cx.bars->full[stage], (gi / NS) & 1) &&
+                               (gi < 2 || mbar_test(&cx.bars->s_free[sb], ((gi - 2) >> 1) & 1));
+            if (ready) {
+                tc::fence_after();
+                if (ns) {
+                    cx.segs++;
+                    cx.first_attn = 1;
+                }
+                cx.tiles = gi + 1;
+                if (u.kind == 2) tc::fence_async_smem();   // cp.async (generic proxy) writes -> tensor core reads
+                const uint32_t ks = cx.sbase + SM_STAGE + stage * STAGE_BYTES;
+                const uint32_t qb = cx.sbase + SM_Q + ((cx.segs - 1) & 1) * 4096;
+                const uint32_t dS = cx.tmem + sb * 16;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
-        const uint32_t qa = (kk >> 2) * 2048 + (kk & 3) * 32;
-        tc::mma_bf16(dS, tc::sdesc_sw128(ks + ka, 16, 1024), tc::sdesc_sw128(qb + qa, 16, 1024), IDESC_S,
-                     kk > 0 ? 1u : 0u);
-    }
-    tc::commit(&cx.bars->s_full[sb]);
-    if (!u.attn) tc::commit(&cx.bars->empty[stage]);
-    // P.V of the previous attention tile (one tile behind, so S of this tile overlaps its softmax)
-    if (cx.prev_valid) issue_pv(p, cx);
-    if (u.attn) {
-        cx.prev_valid = 1;
-        cx.prev_stage = stage;
-        cx.prev_pj = cx.atiles;
-        cx.prev_obuf = (cx.segs - 1) & 1;
-        cx.prev_first = cx.first_attn;
-        cx.first_attn = 0;
-        cx.atiles++;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint32_t qa = (kk >> 2) * 2048 + (kk & 3) * 32;
+                    tc::mma_bf16(dS, tc::sdesc_sw128(ks + ka, 16, 1024), tc::sdesc_sw128(qb + qa, 16, 1024), IDESC_S,
+                                 kk > 0 ? 1u : 0u);
+                }
+                tc::commit(&cx.bars->s_full[sb]);
+                if (!u.attn) tc::commit(&cx.bars->empty[stage]);
+                if (u.attn) {
+                    ring[tail & 3] = PendingPV{stage, (cx.segs - 1) & 1, cx.first_attn, cx.atiles};
+                    ++tail;
+                    cx.first_attn = 0;
+                    cx.atiles++;
+                }
+                prev_row = u.row;
+                ++next;
+                prog = true;
+            }
+        }
+        if (head != tail) {
+            const PendingPV& r = ring[head & 3];
+            if (mbar_test(&cx.bars->p_full[r.pj & 1], (r.pj >> 1) & 1)) {
+                tc::fence_after();
+                issue_pv(cx, r);
+                ++head;
+                prog = true;
+            }
+        }
+        if (prog) {
+            t_last = global_ns();
+        } else {
+            __nanosleep(20);   // leave the issue slots to the softmax warp sharing this scheduler
+            if (global_ns() - t_last > kWaitLimitNs) {
+                atomicOr(p.err, kErrTimeout);
+                return;
+            }
+        }
     }
 }
 
@@ -453,15 +483,7 @@ __device__ __forceinline__ void run_pipeline(const Params& p, Ctx& cx, int u0, i
     if (cx.warp == 4) {
         for (int i = 0; i < n; ++i) produce(p, cx, unit_at(p, u0, row, i));
     } else if (cx.warp == 5) {
-        if (cx.lane == 0) {
-            int prev_row = -1;
-            for (int i = 0; i < n; ++i) {
-                const Unit u = unit_at(p, u0, row, i);
-                mma_tile(p, cx, u, u.row != prev_row);
-                prev_row = u.row;
-            }
-            if (cx.prev_valid) issue_pv(p, cx);
-        }
+        if (cx.lane == 0) mma_loop(p, cx, u0, row, n);
     } else {
         int prev_row = -1;
         for (int i = 0; i < n; ++i) {
@@ -703,16 +725,16 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
     cx.warp = threadIdx.x >> 5;
     cx.lane = threadIdx.x & 31;
     cx.tiles = cx.segs = cx.atiles = 0;
-    cx.prev_valid = 0;
     cx.had_attn = 0;
     cx.first_attn = 1;
     cx.cur_row = -1;
     cx.cur_slot = 0;
     cx.gtiles = 0;
 
-    // zero the operand buffers once: stale rows of gathered tiles must be finite,
-    // and the Q / P^T rows of heads >= G must be zero
-    for (uint32_t o = threadIdx.x * 16; o < SM_WMAX; o += NT * 16)
+    // the Q and P^T rows of heads >= G must be zero (K/V stages need no
+    // clearing: TMA zero-fills past a row's end, and a gathered tile zeroes
+    // the V rows it leaves empty)
+    for (uint32_t o = SM_Q + threadIdx.x * 16; o < SM_WMAX; o += NT * 16)
         *reinterpret_cast<uint4*>(cx.base + o) = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         Bars* b = cx.bars;

@@ -21,6 +21,11 @@ by the slowest rank's time.
 
 --impl reference times the CPU oracle (fp64, OpenMP over rows) on the host
 cores on a bounded sample of the same workload.
+
+Other workloads: --workload NAME for every decode shape of synth.WORKLOADS
+(the sweeps), hier_1m (two-level descent, steps/s against the HBM roofline)
+and gist_prefill (the gist-causal prefill, algorithmic TFLOP/s against the
+bf16 tensor roofline).
 """
 from __future__ import annotations
 
@@ -61,6 +66,44 @@ def peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """Measured bf16 dense TFLOP/s, sustained (a kernel timed back to back for a
+    long stretch runs under the power cap), else the recipe's fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["bf16_tflops_sustained"]), "measured (sustained)"
+    return 1400.0, "fallback (sustained)"
+
+
+PREFILL_METRIC = "gist-causal prefill: algorithmic TFLOP/s (4 d per allowed query-key pair) and % of bf16 tensor peak"
+HIER_METRIC = "GSA hierarchical decode steps/sec and achieved HBM GB/s as % of B200 peak"
+
+
+def prefill_pairs(n_chunks: int, chunk: int) -> int:
+    """Allowed (query, key) pairs of one (sequence, head) under the gist mask:
+    a gist sees the earlier gists, itself and its chunk's raw tokens; raw token
+    i of a chunk sees the earlier gists and raw tokens 0..i of its chunk."""
+    n, c = n_chunks, chunk
+    earlier = n * (n - 1) // 2
+    return earlier + n + n * c + c * earlier + n * c * (c + 1) // 2
+
+
+def prefill_row_pairs(pos: int, chunk: int) -> int:
+    j, i = divmod(pos, chunk + 1)
+    return j + (chunk + 1 if i == chunk else i + 1)
+
+
+def hier_bytes(h) -> int:
+    """Bytes a hierarchical step must move: q, every level-2 gist K and V, the
+    K and V of the selected groups' level-1 gists, the raw K/V of the k1
+    chunks, the tail K/V, out."""
+    s = h.l1
+    row = s.head_dim * (4 if s.dtype == "f32" else 2)
+    per_kv = 2 * h.n_l2 * row + 2 * h.top_k2 * h.group * row + 2 * s.top_k * s.chunk * row + 2 * s.tail_len * row
+    return s.rows * per_kv + 2 * s.batch * s.n_q_heads * row
 
 
 KERNEL_SOURCES = ("gsa_fused.cu", "gsa_fused.h", "gsa_device.cuh", "gsa_tc.cuh")
@@ -328,6 +371,218 @@ def run_ours(args, world, rank, local):
     del g
 
 
+# ------------------------------------------------------------- prefill ----
+def run_prefill(args, world, rank, local):
+    """The gist-causal prefill: K launches back to back (each reads its q, k,
+    v, together far larger than L2), timed with CUDA events on the stream."""
+    import torch
+
+    import kv_cache_routing_b200 as gsa
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from gsa_check import dev
+
+    p = synth.WORKLOADS[args.workload]
+    torch.cuda.set_device(local)
+    x = synth.prefill_inputs(p, synth.seed_for(args.workload) + 17 * rank)
+    d = {k: dev(v) for k, v in x.tensors().items()}
+    P = p.positions
+    desc = gsa.prefill_desc(p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.n_chunks, p.chunk, gsa.GSA_BF16,
+                            p.scale)
+    out = torch.empty((p.batch, p.n_q_heads, P, p.head_dim), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.Stream()
+    step = lambda: gsa.gsa_gist_prefill(desc, d["q"], d["k"], d["v"], out, None, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+        stream.synchronize()
+        barrier(world)
+    ms_max = max_over_ranks(e0.elapsed_time(e1), world)
+    flops = 4.0 * p.head_dim * prefill_pairs(p.n_chunks, p.chunk) * p.batch * p.n_q_heads
+    per_ms = ms_max / args.steps
+    tflops = world * flops / (per_ms / 1e3) / 1e12
+    # e2e: q, k, v from pinned host memory, out back, every step
+    hq = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in d.items()}
+    for k in d:
+        hq[k].copy_(d[k].cpu())
+    ho = torch.empty_like(out, device="cpu").pin_memory()
+    steps_e2e = max(1, min(args.steps, 5))
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(steps_e2e):
+            for k in d:
+                d[k].copy_(hq[k], non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+            stream.synchronize()
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world) / steps_e2e
+    peak, peak_kind = tensor_peak()
+    line = {
+        "metric": PREFILL_METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": p.batch, "n_q_heads": p.n_q_heads,
+                   "n_kv_heads": p.n_kv_heads, "head_dim": p.head_dim, "n_chunks": p.n_chunks, "chunk": p.chunk,
+                   "positions": P, "parallelism": f"replicas x{world}",
+                   "l2": f"q, k, v of {sum(v.numel() * v.element_size() for v in d.values()) / 1e6:.0f} MB "
+                         f"per step (L2 {torch.cuda.get_device_properties(local).L2_cache_size / 1e6:.0f} MB)"},
+        "algorithmic_flop_per_step": flops,
+        "roofline": {"bound": "tensor", "kernel": "gist_prefill_kernel (one launch per step)",
+                     "achieved": round(tflops / world, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tflops / world / peak, 4), "peak_kind": peak_kind, "traffic": None},
+        "e2e": {"value": round(world * flops / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in d.values()),
+                "d2h_bytes_per_step": out.numel() * out.element_size()},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(p, x, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_prefill(p, x, budget_s: float):
+    """The fp64 oracle on random query rows until the time budget is spent,
+    in the metric's unit (algorithmic FLOP of the rows done / time)."""
+    import oracle
+    rng = np.random.default_rng(7)
+    t = x.tensors()
+    P = p.positions
+    done_flop, n, t0 = 0.0, 0, time.perf_counter()
+    while True:
+        rows = np.stack([rng.integers(p.batch, size=64), rng.integers(p.n_q_heads, size=64),
+                         rng.integers(P, size=64)], axis=1).astype(np.int64)
+        oracle.prefill_rows(t, p.n_chunks, p.chunk, rows, p.scale)
+        done_flop += sum(4.0 * p.head_dim * prefill_row_pairs(int(r[2]), p.chunk) for r in rows)
+        n += len(rows)
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(done_flop / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} random query rows of the workload, fp64, {el:.1f} s"}
+
+
+# -------------------------------------------------------- hierarchical ----
+def run_hier(args, world, rank, local):
+    """The two-level descent: K steps captured as one graph rotating over L
+    replicas (own level-2 gists and query each; level-1 gists and raw chunks
+    shared, distinct queries select distinct children) so that the bytes a
+    rotation touches exceed 4x L2."""
+    import torch
+
+    import kv_cache_routing_b200 as gsa
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from gsa_check import desc_of, dev, tdtype
+
+    h = synth.WORKLOADS[args.workload]
+    s = h.l1
+    torch.cuda.set_device(local)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    nbytes = hier_bytes(h)
+    L = max(2, -(-4 * l2 // nbytes)) if not args.replicas else args.replicas
+    seed = synth.seed_for(args.workload) + 17 * rank
+    x = synth.hier_inputs(h, seed)
+    base = {k: dev(v) for k, v in x.tensors().items()}
+    reps = []
+    for r in range(L):
+        t = dict(base)
+        if r:
+            t["q"] = dev(synth.normal(seed + 1000 * r, synth.S_Q, x.q.shape, s.dtype))
+            t["k_g2"] = base["k_g2"].clone()
+            t["v_g2"] = base["v_g2"].clone()
+        reps.append(t)
+    hd = gsa.hier_desc(desc_of(s), h.n_l2, h.group, h.top_k2)
+    ws = torch.zeros(max(256, gsa.gsa_hier_workspace_size(hd)), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((s.batch, s.n_q_heads, s.head_dim), dtype=tdtype(s.dtype), device="cuda") for _ in range(L)]
+    i2 = torch.empty((s.batch, s.n_kv_heads, h.top_k2), dtype=torch.int32, device="cuda")
+    i1 = torch.empty((s.batch, s.n_kv_heads, s.top_k), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(i, st):
+        t = reps[i % L]
+        gsa.gsa_hier_decode(hd, t["q"], t["k_g2"], t["v_g2"], t["k_g1"], t["v_g1"], t["k_raw"], t["v_raw"],
+                            t["k_tail"], t["v_tail"], i2, i1, outs[i % L], ws, stream=st)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(args.steps):
+                step(i, stream)
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        barrier(world)
+    ms_max = max_over_ranks(e0.elapsed_time(e1), world)
+    per_ms = ms_max / args.steps
+    gbs = nbytes / (per_ms / 1e3) / 1e9
+    qh = torch.empty_like(reps[0]["q"], device="cpu").pin_memory()
+    qh.copy_(reps[0]["q"].cpu())
+    oh = torch.empty_like(outs[0], device="cpu").pin_memory()
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for i in range(args.steps):
+            reps[i % L]["q"].copy_(qh, non_blocking=True)
+            step(i, stream)
+            oh.copy_(outs[i % L], non_blocking=True)
+            stream.synchronize()
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+    peak, peak_kind = peaks()
+    line = {
+        "metric": HIER_METRIC, "value": round(whole_job_rate(args.steps, world, ms_max), 2), "unit": "steps/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+        "config": {"workload": args.workload, "batch": s.batch, "n_q_heads": s.n_q_heads,
+                   "n_kv_heads": s.n_kv_heads, "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk,
+                   "chunk": s.chunk, "n_l2": h.n_l2, "group": h.group, "top_k2": h.top_k2, "top_k1": s.top_k,
+                   "tail": s.tail_len, "parallelism": f"replicas x{world}",
+                   "l2": f"rotating {L} replicas (own level-2 gists and query), {L * nbytes / 1e6:.0f} MB touched "
+                         f"per rotation (L2 {l2 / 1e6:.0f} MB)"},
+        "algorithmic_bytes_per_step": nbytes,
+        "roofline": {"bound": "hbm", "kernel": f"gsa_hier_decode (whole step)", "achieved": round(gbs, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
+                     "traffic": None},
+        "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
+                "h2d_bytes_per_step": qh.numel() * qh.element_size(),
+                "d2h_bytes_per_step": oh.numel() * oh.element_size()},
+        "gpu_launches": 3 * args.steps,   # level-2 gist pass, level-1 gist pass, unfold pass
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+
+
 # ------------------------------------------------------------ CPU oracle ----
 def cpu_baseline(s, x, budget_s: float):
     """The fp64 oracle, as it stands, on the host cores: whole decode steps of
@@ -384,8 +639,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="llama8b_decode",
-                    choices=[k for k, v in synth.WORKLOADS.items() if isinstance(v, synth.DecodeShape)])
+    ap.add_argument("--workload", default="llama8b_decode", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -395,13 +649,21 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
+        if not isinstance(synth.WORKLOADS[args.workload], synth.DecodeShape):
+            ap.error("--impl reference times the decode workloads")
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, world, rank)
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_ours(args, world, rank, local)
+        w = synth.WORKLOADS[args.workload]
+        if isinstance(w, synth.PrefillShape):
+            run_prefill(args, world, rank, local)
+        elif isinstance(w, synth.HierShape):
+            run_hier(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -18,13 +18,18 @@
 // So the work is ~ (earlier gists + 128) per 119 queries instead of the full
 // causal triangle.
 //
-// Per CTA (one query tile of one head): warp 4 allocates TMEM, issues the
-// TMA loads and the MMAs from one thread; warps 0-3 own one query row each
-// (TMEM lane = row) and run the online softmax.  S = Q.K^T lands in TMEM
-// columns [0,128), O accumulates in columns [128,256).  K/V tiles are double
-// buffered, P (bf16, written by the softmax warps in the MMA's swizzled
-// K-major layout) is double buffered, and O is rescaled lazily: only when a
-// row's running maximum grows by more than 2^8.
+// Per CTA: one query tile of TWO query heads of the same KV head (grouped-
+// query attention), which see the same keys under the same mask, so every
+// K/V tile is loaded once for both.  Warps 0-3 run the online softmax of head
+// A, warps 4-7 that of head B (thread = query row = TMEM lane), warp 8 issues
+// the TMA loads and warp 9 the MMAs from one thread.  TMEM (512 columns): S_A
+// [0,128), S_B [128,256), O_A [256,384), O_B [384,512); each head's P (bf16,
+// two per column) overwrites the first 64 columns of its S once read and is
+// the A operand of its P.V product straight from TMEM.  The tensor core
+// alternates between the heads (S_A, S_B, P.V_A, S_A', P.V_B, S_B', ...), so
+// one head's softmax overlaps the other head's products.  K/V tiles are double
+// buffered; O is rescaled lazily (only when a row's running maximum grows by
+// more than 2^8).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -38,10 +43,10 @@
 
 namespace gsa {
 
-constexpr int PF_THREADS = 160;
+constexpr int PF_THREADS = 320;
 constexpr int PF_D = 128;
 constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
-constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, 128, 0, 1);  // P (K-major) x V (MN-major)
+constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, 128, 0, 1);  // P (TMEM, K-major) x V (MN-major)
 constexpr float kRescaleLog2 = 8.f;
 
 // Error word of the prefill's bounded waits (the prefill takes no workspace).
@@ -55,23 +60,23 @@ struct PrefillParams {
     CUtensorMap tm_vg;
     uint16_t* out;       // [B*Hq][P][d] bf16
     float* lse;          // [B*Hq][P] or null
-    int BH, Hq, G, N, C, P, QC, n_qt;
+    int B, Hq, Hkv, G, NPAIR, N, C, P, QC, n_qt;
     float c2;            // scale * log2(e)
 };
 
 // shared-memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t SM_Q = 0;                  // 32 KiB
-constexpr uint32_t SM_KV = 32768;             // 2 stages x (K 32 KiB + V 32 KiB)
-constexpr uint32_t SM_P = SM_KV + 2 * 65536;  // 2 x 32 KiB
-constexpr uint32_t SM_BAR = SM_P + 2 * 32768; // barriers and the TMEM address
+constexpr uint32_t SM_Q = 0;                  // 2 heads x 32 KiB
+constexpr uint32_t SM_KV = 65536;             // 2 stages x (K 32 KiB + V 32 KiB)
+constexpr uint32_t SM_BAR = SM_KV + 2 * 65536; // barriers and the TMEM address
 constexpr uint32_t PF_SMEM = SM_BAR + 256 + 1024;
 
 struct PfBars {
-    uint64_t q_full, kv_full[2], kv_empty[2], s_full, s_free, p_full[2], o_done[2];
+    uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done[2];
     uint32_t tmem;
 };
 
-__global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __grid_constant__ PrefillParams p) {
+// 168 registers a thread: three warps of 10 share each scheduler's 16K registers
+__global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -79,11 +84,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
     PfBars& bars = *reinterpret_cast<PfBars*>(base + SM_BAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // work item: heaviest query tiles first; then (batch, kv head, head pair)
+    const int nw = p.B * p.Hkv * p.NPAIR;
     const int bid = blockIdx.x;
-    const int bh = bid % p.BH;
-    const int t = p.n_qt - 1 - bid / p.BH;          // heaviest query tiles first
-    const int b = bh / p.Hq, h = bh % p.Hq;
-    const int bkv = b * (p.Hq / p.G) + h / p.G;
+    const int wi = bid % nw;
+    const int t = p.n_qt - 1 - bid / nw;
+    const int hp = wi % p.NPAIR, bkv = wi / p.NPAIR;   // bkv = b * Hkv + kv head
+    const int b = bkv / p.Hkv, hkv = bkv % p.Hkv;
+    const int hA = hkv * p.G + 2 * hp;
+    const bool hasB = 2 * hp + 1 < p.G;
+    const int bhA = b * p.Hq + hA;
     const int j0 = t * p.QC;
     const int p0 = j0 * (p.C + 1);
     const int j_last = min(j0 + p.QC, p.N) - 1;      // last chunk of the tile
@@ -95,204 +105,214 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.kv_full[i], 1);
             mbar_init(&bars.kv_empty[i], 1);
+            mbar_init(&bars.s_full[i], 1);
             mbar_init(&bars.p_full[i], 128);
             mbar_init(&bars.o_done[i], 1);
         }
-        mbar_init(&bars.s_full, 1);
-        mbar_init(&bars.s_free, 128);
         fence_mbar_init();
     }
-    if (warp == 4) {
-        tc::tmem_alloc(&bars.tmem, 256);
+    if (warp == 9) {
+        tc::tmem_alloc(&bars.tmem, 512);
         tc::tmem_relinquish();
     }
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = bars.tmem;
-    const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
     uint32_t* err = &g_prefill_err;   // waits below are bounded; a timeout abandons the tile
 
-    if (warp == 4) {
+    if (warp == 8) {
         if (lane == 0) {
-            // ---------------------------------------------- TMA + MMA issue --
-            auto load_kv = [&](int i, int s) {
+            // --------------------------------------------------- TMA loads --
+            mbar_arrive_expect_tx(&bars.q_full, hasB ? 65536 : 32768);
+            tc::tma_load_3d(base + SM_Q, &p.tm_q, 0, p0, bhA, &bars.q_full);
+            tc::tma_load_3d(base + SM_Q + 16384, &p.tm_q, 64, p0, bhA, &bars.q_full);
+            if (hasB) {
+                tc::tma_load_3d(base + SM_Q + 32768, &p.tm_q, 0, p0, bhA + 1, &bars.q_full);
+                tc::tma_load_3d(base + SM_Q + 49152, &p.tm_q, 64, p0, bhA + 1, &bars.q_full);
+            }
+            for (int i = 0; i < n_kv; ++i) {
+                const int s = i & 1;
+                if (i >= 2 && !mbar_wait(&bars.kv_empty[s], ((i - 2) >> 1) & 1, err)) break;
                 uint8_t* ks = base + SM_KV + s * 65536;
                 uint8_t* vs = ks + 32768;
                 mbar_arrive_expect_tx(&bars.kv_full[s], 65536);
-                if (i < n_gt) {
-                    const int g0 = i * 128;
-                    tc::tma_load_3d(ks, &p.tm_kg, 0, g0, bkv, &bars.kv_full[s]);
-                    tc::tma_load_3d(ks + 16384, &p.tm_kg, 64, g0, bkv, &bars.kv_full[s]);
-                    tc::tma_load_3d(vs, &p.tm_vg, 0, g0, bkv, &bars.kv_full[s]);
-                    tc::tma_load_3d(vs + 16384, &p.tm_vg, 64, g0, bkv, &bars.kv_full[s]);
-                } else {
-                    tc::tma_load_3d(ks, &p.tm_k, 0, p0, bkv, &bars.kv_full[s]);
-                    tc::tma_load_3d(ks + 16384, &p.tm_k, 64, p0, bkv, &bars.kv_full[s]);
-                    tc::tma_load_3d(vs, &p.tm_v, 0, p0, bkv, &bars.kv_full[s]);
-                    tc::tma_load_3d(vs + 16384, &p.tm_v, 64, p0, bkv, &bars.kv_full[s]);
-                }
-            };
-            auto issue_s = [&](int i) {
+                const CUtensorMap* mk = i < n_gt ? &p.tm_kg : &p.tm_k;
+                const CUtensorMap* mv = i < n_gt ? &p.tm_vg : &p.tm_v;
+                const int y = i < n_gt ? i * 128 : p0;
+                tc::tma_load_3d(ks, mk, 0, y, bkv, &bars.kv_full[s]);
+                tc::tma_load_3d(ks + 16384, mk, 64, y, bkv, &bars.kv_full[s]);
+                tc::tma_load_3d(vs, mv, 0, y, bkv, &bars.kv_full[s]);
+                tc::tma_load_3d(vs + 16384, mv, 64, y, bkv, &bars.kv_full[s]);
+            }
+        }
+    } else if (warp == 9) {
+        if (lane == 0) {
+            // ----------------------------------------------------- MMA issue --
+            // S_h = Q_h . K^T into TMEM columns 128 h; P_h . V into 256 + 128 h
+            auto issue_s = [&](int h, int i) {
                 const uint32_t ks = sbase + SM_KV + (i & 1) * 65536;
+                const uint32_t qs = sbase + SM_Q + h * 32768;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    tc::mma_bf16(tmem_s, tc::sdesc_sw128(sbase + SM_Q + off, 16, 1024),
+                    tc::mma_bf16(tmem + h * 128, tc::sdesc_sw128(qs + off, 16, 1024),
                                  tc::sdesc_sw128(ks + off, 16, 1024), IDESC_S, kk > 0);
                 }
-                tc::commit(&bars.s_full);
+                tc::commit(&bars.s_full[h]);
             };
-            mbar_arrive_expect_tx(&bars.q_full, 32768);
-            tc::tma_load_3d(base + SM_Q, &p.tm_q, 0, p0, bh, &bars.q_full);
-            tc::tma_load_3d(base + SM_Q + 16384, &p.tm_q, 64, p0, bh, &bars.q_full);
-            for (int i = 0; i < min(2, n_kv); ++i) load_kv(i, i);
-            bool ok = mbar_wait(&bars.q_full, 0, err) && mbar_wait(&bars.kv_full[0], 0, err);
-            tc::fence_after();
-            if (ok) issue_s(0);
-            for (int i = 0; ok && i < n_kv; ++i) {
-                if (i + 1 < n_kv) {
-                    ok = mbar_wait(&bars.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1, err) &&
-                         mbar_wait(&bars.s_free, i & 1, err);
-                    tc::fence_after();
-                    if (!ok) break;
-                    issue_s(i + 1);
-                }
-                if (!mbar_wait(&bars.p_full[i & 1], (i >> 1) & 1, err)) break;
-                tc::fence_after();
-                const uint32_t pb = sbase + SM_P + (i & 1) * 32768;
+            auto issue_pv = [&](int h, int i) {
                 const uint32_t vs = sbase + SM_KV + (i & 1) * 65536 + 32768;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    tc::mma_bf16(tmem_o, tc::sdesc_sw128(pb + aoff, 16, 1024),
-                                 tc::sdesc_sw128(vs + kk * 2048, 16384, 1024), IDESC_PV, (i > 0 || kk > 0));
-                }
-                tc::commit(&bars.o_done[i & 1]);
-                tc::commit(&bars.kv_empty[i & 1]);
-                if (i + 2 < n_kv) {
-                    if (!mbar_wait(&bars.kv_empty[i & 1], (i >> 1) & 1, err)) break;
-                    load_kv(i + 2, i & 1);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8,
+                                    tc::sdesc_sw128(vs + kk * 2048, 16384, 1024), IDESC_PV, (i > 0 || kk > 0));
+                tc::commit(&bars.o_done[h]);
+            };
+            bool ok = mbar_wait(&bars.q_full, 0, err) && mbar_wait(&bars.kv_full[0], 0, err);
+            tc::fence_after();
+            if (ok) {
+                issue_s(0, 0);
+                if (hasB) issue_s(1, 0);
+            }
+            for (int i = 0; ok && i < n_kv; ++i) {
+                const bool more = i + 1 < n_kv;
+                for (int h = 0; ok && h < (hasB ? 2 : 1); ++h) {
+                    // P_h of tile i (which also means S_h of tile i has been read)
+                    ok = mbar_wait(&bars.p_full[h], i & 1, err);
+                    if (!ok) break;
+                    tc::fence_after();
+                    issue_pv(h, i);
+                    if (h == (hasB ? 1 : 0)) tc::commit(&bars.kv_empty[i & 1]);
+                    if (more) {
+                        if (h == 0) {
+                            ok = mbar_wait(&bars.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1, err);
+                            if (!ok) break;
+                            tc::fence_after();
+                        }
+                        issue_s(h, i + 1);
+                    }
                 }
             }
         }
     } else {
         // ------------------------------------------------ softmax warps ----
-        const int r = threadIdx.x;                       // query row = TMEM lane
-        const int qp = p0 + r;
-        const bool valid = r < p.QC * (p.C + 1) && qp < p.P;
-        const int jq = valid ? j0 + r / (p.C + 1) : -1;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        float m_run = -INFINITY, l_run = 0.f;
-        float s[128];
-        for (int i = 0; i < n_kv; ++i) {
-            if (!mbar_wait(&bars.s_full, i & 1, err)) break;
-            tc::fence_after();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t u[32];
-                tc::ld32(tmem_s + lane_off + c * 32, u);
-                tc::wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) s[c * 32 + j] = __uint_as_float(u[j]);
-            }
-            tc::fence_before();
-            mbar_arrive(&bars.s_free);
-            // allowed key columns [lo, hi] of this row in this tile
-            int lo, hi;
-            if (i < n_gt) {
-                lo = 0;
-                hi = valid ? min(127, jq - i * 128 - 1) : -1;
-            } else {
-                lo = valid ? jq * (p.C + 1) - p0 : 1;
-                hi = valid ? r : 0;
-            }
-            float mt = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 128; ++j) {
-                s[j] = (j >= lo && j <= hi) ? s[j] * p.c2 : -INFINITY;
-                mt = fmaxf(mt, s[j]);
-            }
-            bool need = false;
-            float m_new = m_run;
-            if (mt > -INFINITY) {
-                if (m_run == -INFINITY) {
-                    m_new = mt;
-                } else if (mt > m_run + kRescaleLog2) {
-                    m_new = mt;
-                    need = true;
-                }
-            }
-            const float alpha = need ? exp2f(m_run - m_new) : 1.f;
-            if (__any_sync(0xFFFFFFFFu, need) && i > 0) {
-                // O holds P.V of tiles < i: wait for the last of them, then rescale
-                mbar_wait(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1, err);
+        const int h = warp >> 2;                         // 0: head A, 1: head B
+        if (h == 0 || hasB) {
+            const int r = threadIdx.x & 127;             // query row = TMEM lane
+            const int qp = p0 + r;
+            const bool valid = r < p.QC * (p.C + 1) && qp < p.P;
+            const int jq = valid ? j0 + r / (p.C + 1) : -1;
+            const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+            const uint32_t ts = tmem + h * 128 + lane_off, to = tmem + 256 + h * 128 + lane_off;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int i = 0; i < n_kv; ++i) {
+                if (!mbar_wait(&bars.s_full[h], i & 1, err)) break;
                 tc::fence_after();
+                // allowed key columns [lo, hi] of this row in this tile
+                int lo, hi;
+                if (i < n_gt) {
+                    lo = 0;
+                    hi = valid ? min(127, jq - i * 128 - 1) : -1;
+                } else {
+                    lo = valid ? jq * (p.C + 1) - p0 : 1;
+                    hi = valid ? r : 0;
+                }
+                // pass 1: the row maximum (S stays in TMEM)
+                float mt = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t u[32];
-                    tc::ld32(tmem_o + lane_off + c * 32, u);
+                    tc::ld32(ts + c * 32, u);
                     tc::wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
-                    tc::st32(tmem_o + lane_off + c * 32, u);
+                    for (int j = 0; j < 32; ++j)
+                        if (c * 32 + j >= lo && c * 32 + j <= hi) mt = fmaxf(mt, __uint_as_float(u[j]) * p.c2);
                 }
+                bool need = false;
+                float m_new = m_run;
+                if (mt > -INFINITY) {
+                    if (m_run == -INFINITY) {
+                        m_new = mt;
+                    } else if (mt > m_run + kRescaleLog2) {
+                        m_new = mt;
+                        need = true;
+                    }
+                }
+                const float alpha = need ? exp2f(m_run - m_new) : 1.f;
+                if (__any_sync(0xFFFFFFFFu, need) && i > 0) {
+                    // O holds P.V of tiles < i: wait for the last of them, then rescale
+                    mbar_wait(&bars.o_done[h], (i - 1) & 1, err);
+                    tc::fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t u[16];
+                        tc::ld16(to + c * 16, u);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
+                        tc::st16(to + c * 16, u);
+                    }
+                }
+                m_run = m_new;
+                // pass 2: P (bf16 pairs) over the first 64 columns of S, in key
+                // order, so every column it overwrites has been read already; the
+                // P.V of the previous tile finished before this S was written
+                float sum = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t u[32];
+                    tc::ld32(ts + c * 32, u);
+                    tc::wait_ld();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = c * 32 + 2 * e;
+                        const bool oa = j >= lo && j <= hi, ob = j + 1 >= lo && j + 1 <= hi;
+                        const float a = oa ? exp2f(__uint_as_float(u[2 * e]) * p.c2 - m_run) : 0.f;
+                        const float bb = ob ? exp2f(__uint_as_float(u[2 * e + 1]) * p.c2 - m_run) : 0.f;
+                        sum += a + bb;
+                        w[e] = tc::pack_bf16x2(a, bb);
+                    }
+                    tc::st16(ts + c * 16, w);
+                }
+                l_run = l_run * alpha + sum;
                 tc::wait_st();
+                tc::fence_before();
+                mbar_arrive(&bars.p_full[h]);
             }
-            m_run = m_new;
-            // the P buffer of this tile was last read by the P.V MMA of tile i-2
-            if (i >= 2) mbar_wait(&bars.o_done[i & 1], ((i - 2) >> 1) & 1, err);
-            uint8_t* prow = base + SM_P + (i & 1) * 32768 + r * 128;
-            float sum = 0.f;
+            // -------------------------------------------------- epilogue ----
+            mbar_wait(&bars.o_done[h], (n_kv - 1) & 1, err);
+            tc::fence_after();
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const int bh = bhA + h;
+            uint16_t* orow = p.out + ((size_t)bh * p.P + qp) * PF_D;
 #pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16) {
-                uint32_t w[4];
+            for (int c = 0; c < 4; ++c) {
+                uint32_t u[32];
+                tc::ld32(to + c * 32, u);
+                tc::wait_ld();
+                if (valid) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = c16 * 8 + 2 * e;
-                    const float a = (m_run == -INFINITY) ? 0.f : exp2f(s[j] - m_run);
-                    const float bb = (m_run == -INFINITY) ? 0.f : exp2f(s[j + 1] - m_run);
-                    sum += a + bb;
-                    w[e] = tc::pack_bf16x2(a, bb);
-                }
-                const int kb = c16 >> 3, ch = c16 & 7;
-                *reinterpret_cast<uint4*>(prow + kb * 16384 + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            l_run = l_run * alpha + sum;
-            tc::fence_async_smem();
-            tc::fence_before();
-            mbar_arrive(&bars.p_full[i & 1]);
-        }
-        // ------------------------------------------------------ epilogue ----
-        mbar_wait(&bars.o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, err);
-        tc::fence_after();
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        uint16_t* orow = p.out + ((size_t)bh * p.P + qp) * PF_D;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t u[32];
-            tc::ld32(tmem_o + lane_off + c * 32, u);
-            tc::wait_ld();
-            if (valid) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    uint4 v;
-                    v.x = tc::pack_bf16x2(__uint_as_float(u[j]) * inv, __uint_as_float(u[j + 1]) * inv);
-                    v.y = tc::pack_bf16x2(__uint_as_float(u[j + 2]) * inv, __uint_as_float(u[j + 3]) * inv);
-                    v.z = tc::pack_bf16x2(__uint_as_float(u[j + 4]) * inv, __uint_as_float(u[j + 5]) * inv);
-                    v.w = tc::pack_bf16x2(__uint_as_float(u[j + 6]) * inv, __uint_as_float(u[j + 7]) * inv);
-                    *reinterpret_cast<uint4*>(orow + c * 32 + j) = v;
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 v;
+                        v.x = tc::pack_bf16x2(__uint_as_float(u[j]) * inv, __uint_as_float(u[j + 1]) * inv);
+                        v.y = tc::pack_bf16x2(__uint_as_float(u[j + 2]) * inv, __uint_as_float(u[j + 3]) * inv);
+                        v.z = tc::pack_bf16x2(__uint_as_float(u[j + 4]) * inv, __uint_as_float(u[j + 5]) * inv);
+                        v.w = tc::pack_bf16x2(__uint_as_float(u[j + 6]) * inv, __uint_as_float(u[j + 7]) * inv);
+                        *reinterpret_cast<uint4*>(orow + c * 32 + j) = v;
+                    }
                 }
             }
+            if (valid && p.lse != nullptr)
+                p.lse[(size_t)bh * p.P + qp] = (m_run + log2f(l_run)) * 0.69314718055994531f;
         }
-        if (valid && p.lse != nullptr)
-            p.lse[(size_t)bh * p.P + qp] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 9) {
         tc::fence_after();
-        tc::tmem_dealloc(tmem, 256);
+        tc::tmem_dealloc(tmem, 512);
     }
 }
 
@@ -365,9 +385,11 @@ extern "C" gsa_status gsa_gist_prefill(const gsa_prefill_desc* desc, const void*
     if (!ok) return GSA_ERR_CUDA;
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
-    p.BH = B * Hq;
+    p.B = B;
     p.Hq = Hq;
+    p.Hkv = Hkv;
     p.G = Hq / Hkv;
+    p.NPAIR = (p.G + 1) / 2;
     p.N = N;
     p.C = C;
     p.P = (int)P;
@@ -382,7 +404,7 @@ extern "C" gsa_status gsa_gist_prefill(const gsa_prefill_desc* desc, const void*
             return GSA_ERR_CUDA;
         attr = true;
     }
-    const unsigned grid = (unsigned)p.n_qt * (unsigned)p.BH;
+    const unsigned grid = (unsigned)p.n_qt * (unsigned)(B * Hkv * p.NPAIR);
     gist_prefill_kernel<<<grid, PF_THREADS, PF_SMEM, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }

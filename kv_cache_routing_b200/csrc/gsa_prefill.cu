@@ -64,6 +64,37 @@ struct PrefillParams {
     float c2;            // scale * log2(e)
 };
 
+// 2^x on the special-function unit (ex2.approx.ftz: -inf -> +0), a
+// three-input maximum, and packed two-wide fp32 arithmetic (sm_100).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unf2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // shared-memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t SM_Q = 0;                  // 2 heads x 32 KiB
 constexpr uint32_t SM_KV = 65536;             // 2 stages x (K 32 KiB + V 32 KiB)
@@ -218,17 +249,33 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
                     lo = valid ? jq * (p.C + 1) - p0 : 1;
                     hi = valid ? r : 0;
                 }
-                // pass 1: the row maximum (S stays in TMEM)
+                // pass 1: the row maximum (S stays in TMEM); the scale is applied
+                // to the maximum (it is positive), and a warp whose rows all see
+                // the whole tile takes the unmasked path (warp-uniform: the
+                // tcgen05.ld inside is .sync.aligned)
+                const bool full = __all_sync(0xFFFFFFFFu, lo == 0 && hi >= 127);
                 float mt = -INFINITY;
+                if (full) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t u[32];
-                    tc::ld32(ts + c * 32, u);
-                    tc::wait_ld();
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t u[32];
+                        tc::ld32(ts + c * 32, u);
+                        tc::wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c * 32 + j >= lo && c * 32 + j <= hi) mt = fmaxf(mt, __uint_as_float(u[j]) * p.c2);
+                        for (int j = 0; j < 32; j += 2) mt = max3(mt, __uint_as_float(u[j]), __uint_as_float(u[j + 1]));
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t u[32];
+                        tc::ld32(ts + c * 32, u);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (c * 32 + j >= lo && c * 32 + j <= hi) mt = fmaxf(mt, __uint_as_float(u[j]));
+                    }
                 }
+                mt *= p.c2;
                 bool need = false;
                 float m_new = m_run;
                 if (mt > -INFINITY) {
@@ -258,7 +305,9 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
                 // pass 2: P (bf16 pairs) over the first 64 columns of S, in key
                 // order, so every column it overwrites has been read already; the
                 // P.V of the previous tile finished before this S was written
-                float sum = 0.f;
+                // x * c2 - m in pairs (fma.f32x2), 2^x on the SFU, pair sums (add.f32x2)
+                const uint64_t c22 = f2(p.c2, p.c2), nm2 = f2(-m_run, -m_run);
+                uint64_t acc2 = f2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t u[32];
@@ -268,14 +317,21 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const int j = c * 32 + 2 * e;
-                        const bool oa = j >= lo && j <= hi, ob = j + 1 >= lo && j + 1 <= hi;
-                        const float a = oa ? exp2f(__uint_as_float(u[2 * e]) * p.c2 - m_run) : 0.f;
-                        const float bb = ob ? exp2f(__uint_as_float(u[2 * e + 1]) * p.c2 - m_run) : 0.f;
-                        sum += a + bb;
+                        float xa, xb;
+                        unf2(ffma2(f2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), c22, nm2), xa, xb);
+                        if (!full) {
+                            xa = (j >= lo && j <= hi) ? xa : -INFINITY;
+                            xb = (j + 1 >= lo && j + 1 <= hi) ? xb : -INFINITY;
+                        }
+                        const float a = ex2(xa), bb = ex2(xb);
+                        acc2 = fadd2(acc2, f2(a, bb));
                         w[e] = tc::pack_bf16x2(a, bb);
                     }
                     tc::st16(ts + c * 16, w);
                 }
+                float sa, sb;
+                unf2(acc2, sa, sb);
+                const float sum = m_run == -INFINITY ? 0.f : sa + sb;
                 l_run = l_run * alpha + sum;
                 tc::wait_st();
                 tc::fence_before();

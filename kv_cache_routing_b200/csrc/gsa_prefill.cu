@@ -256,14 +256,25 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
                 const bool full = __all_sync(0xFFFFFFFFu, lo == 0 && hi >= 127);
                 float mt = -INFINITY;
                 if (full) {
+                    // two 32-column loads in flight, four independent max chains
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t u[32];
+                    for (int c = 0; c < 4; c += 2) {
+                        uint32_t u[32], v[32];
                         tc::ld32(ts + c * 32, u);
+                        tc::ld32(ts + c * 32 + 32, v);
                         tc::wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) mt = max3(mt, __uint_as_float(u[j]), __uint_as_float(u[j + 1]));
+                        for (int j = 0; j < 32; j += 4) {
+                            m4[(j >> 2) & 3] = max3(m4[(j >> 2) & 3], __uint_as_float(u[j]), __uint_as_float(u[j + 1]));
+                            m4[((j >> 2) + 1) & 3] =
+                                max3(m4[((j >> 2) + 1) & 3], __uint_as_float(u[j + 2]), __uint_as_float(u[j + 3]));
+                            m4[((j >> 2) + 2) & 3] = max3(m4[((j >> 2) + 2) & 3], __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                            m4[((j >> 2) + 3) & 3] =
+                                max3(m4[((j >> 2) + 3) & 3], __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                        }
                     }
+                    mt = max3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
                 } else {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
@@ -307,30 +318,37 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
                 // P.V of the previous tile finished before this S was written
                 // x * c2 - m in pairs (fma.f32x2), 2^x on the SFU, pair sums (add.f32x2)
                 const uint64_t c22 = f2(p.c2, p.c2), nm2 = f2(-m_run, -m_run);
-                uint64_t acc2 = f2(0.f, 0.f);
+                uint64_t acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t u[32];
-                    tc::ld32(ts + c * 32, u);
+                for (int c = 0; c < 4; c += 2) {
+                    // two 32-column loads in flight; their P goes to columns
+                    // [16c, 16c + 32), all read by now (this chunk or the previous one)
+                    uint32_t u[2][32];
+                    tc::ld32(ts + c * 32, u[0]);
+                    tc::ld32(ts + c * 32 + 32, u[1]);
                     tc::wait_ld();
-                    uint32_t w[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int j = c * 32 + 2 * e;
-                        float xa, xb;
-                        unf2(ffma2(f2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), c22, nm2), xa, xb);
-                        if (!full) {
-                            xa = (j >= lo && j <= hi) ? xa : -INFINITY;
-                            xb = (j + 1 >= lo && j + 1 <= hi) ? xb : -INFINITY;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int j = (c + hh) * 32 + 2 * e;
+                            float xa, xb;
+                            unf2(ffma2(f2(__uint_as_float(u[hh][2 * e]), __uint_as_float(u[hh][2 * e + 1])), c22, nm2),
+                                 xa, xb);
+                            if (!full) {
+                                xa = (j >= lo && j <= hi) ? xa : -INFINITY;
+                                xb = (j + 1 >= lo && j + 1 <= hi) ? xb : -INFINITY;
+                            }
+                            const float a = ex2(xa), bb = ex2(xb);
+                            acc2[e & 1] = fadd2(acc2[e & 1], f2(a, bb));
+                            w[e] = tc::pack_bf16x2(a, bb);
                         }
-                        const float a = ex2(xa), bb = ex2(xb);
-                        acc2 = fadd2(acc2, f2(a, bb));
-                        w[e] = tc::pack_bf16x2(a, bb);
+                        tc::st16(ts + (c + hh) * 16, w);
                     }
-                    tc::st16(ts + c * 16, w);
                 }
                 float sa, sb;
-                unf2(acc2, sa, sb);
+                unf2(fadd2(acc2[0], acc2[1]), sa, sb);
                 const float sum = m_run == -INFINITY ? 0.f : sa + sb;
                 l_run = l_run * alpha + sum;
                 tc::wait_st();

@@ -704,7 +704,7 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
 // over the raw tokens of the k1 chunks and the tail, merging all partials.
 size_t gsa_hier_workspace_size(const gsa_hier_desc* desc) {
     if (validate_hier(desc) != GSA_OK) return 0;
-    return make_hier_plan(*desc).total;
+    return fused_hier_supported(*desc) ? make_fused_hier_plan(*desc).total : make_hier_plan(*desc).total;
 }
 
 gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void* k_g2, const void* v_g2,
@@ -720,6 +720,14 @@ gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void*
     const void* all[] = {q, k_g2, v_g2, k_g1, v_g1, k_raw, v_raw, k_tail, v_tail, idx2_out, idx1_out, out};
     for (const void* x : all)
         if (!aligned16(x)) return GSA_ERR_ALIGN;
+    if (fused_hier_supported(*desc)) {
+        // tensor-core path: level-2 gists and tail streamed, then per row the
+        // children tile (scored and attended) and the raw tile of the k1 chunks
+        const FusedPlan f = make_fused_hier_plan(*desc);
+        if (!ws || ws_bytes < f.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSA_ERR_WORKSPACE;
+        return fused_hier_launch(*desc, f, q, k_g2, v_g2, k_g1, v_g1, k_raw, v_raw, k_tail, v_tail, idx2_out,
+                                 idx1_out, out, ws, static_cast<cudaStream_t>(stream));
+    }
     const HierPlan hp = make_hier_plan(*desc);
     if (!ws || ws_bytes < hp.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSA_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);

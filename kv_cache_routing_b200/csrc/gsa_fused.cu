@@ -67,6 +67,11 @@ constexpr uint32_t SM_SCORE = SM_MISC + 1024;        // phase A: this CTA's rout
 constexpr int kScoreCap = 3072;                      // scores kept in shared memory
 constexpr uint32_t SM_SEL = SM_SCORE;                // phase B: the row's selection [kSelCap]
 constexpr uint32_t SM_ROWTAB = SM_SEL + kSelCap * 4; // phase B: source of each gathered row [kMaxTpc][128]
+// hierarchy, phase B: the level-2 selection at SM_SEL [k2 <= 512], the children
+// tile's score keys [128] and the level-1 selection [k1 <= 128] after it
+constexpr uint32_t SM_CKEY = SM_SEL + 512 * 4;
+constexpr uint32_t SM_SEL1 = SM_CKEY + TILE * 4;
+static_assert(SM_SEL1 + TILE * 4 <= SM_ROWTAB, "hierarchy tables overflow the selection buffer");
 static_assert(kSelCap * 4 + kMaxTpc * TILE * 4 <= kScoreCap * 4, "phase-B tables overflow the score buffer");
 constexpr uint32_t SM_UB = SM_SCORE + kScoreCap * 4;  // first unit of every phase-A CTA [kFusedCtas + 1]
 constexpr uint32_t SM_BAR = SM_UB + 640;
@@ -87,6 +92,7 @@ struct Unit {
     int row;
     int kind;      // 0 gist tile, 1 tail tile, 2 gathered tile (raw chunks [+ gists])
     int t;         // tile index within its kind
+    int lt;        // gathered tiles: index into the shared row table
     int nvalid;    // kinds 0/1: leading valid rows
     bool score, attn;
 };
@@ -130,17 +136,19 @@ __device__ __forceinline__ Unit unit_at(const Params& p, int u0, int row, int i)
         x.row = row;
         x.kind = 2;
         x.t = u0 + i;
+        x.lt = i;
         x.nvalid = 0;
-        x.score = false;
+        x.score = p.hier != 0 && x.t == 0;   // the hierarchy's children tile (tile 0) is scored
         x.attn = true;
     }
     return x;
 }
 
-// Is key row r of gathered tile t valid?  A row's gathered rows are packed
-// densely: the k selected chunks' raw tokens (chunk-slot major), then in
-// SELECTED_PAIRS mode the k selected gists.
-__device__ __forceinline__ bool gathered_valid(const Params& p, int t, int r) { return t * TILE + r < p.nrows_g; }
+// Is key row r of the gathered tile with row-table index lt valid?  (The
+// table marks an empty row with -1.)
+__device__ __forceinline__ bool gathered_valid(const uint8_t* base, int lt, int r) {
+    return reinterpret_cast<const int32_t*>(base + SM_ROWTAB)[lt * TILE + r] != -1;
+}
 
 // Copy 16-byte piece c16 of gathered row r into the swizzled K and V operand
 // tiles ks / vs.  e is the row's source: raw row e (e >= 0), gist row -e - 2
@@ -397,7 +405,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Ctx& cx, const Uni
     tc::wait_ld();
     tc::fence_before();
     mbar_arrive(&cx.bars->s_free[sb]);
-    const bool valid = u.kind < 2 ? (t < u.nvalid) : gathered_valid(p, u.t, t);
+    const bool valid = u.kind < 2 ? (t < u.nvalid) : gathered_valid(cx.base, u.lt, t);
     float score = 0.f;
     if (u.score) {
 #pragma unroll
@@ -463,7 +471,10 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Ctx& cx, const Uni
         cx.had_attn = 1;
     }
     // the routing score leaves after the tile is handed to the tensor core
-    if (u.score) {
+    if (u.score && u.kind == 2) {
+        // hierarchy: the level-1 scores of the children tile, as keys for the k1 selection
+        reinterpret_cast<uint32_t*>(cx.base + SM_CKEY)[t] = valid ? order_key(score) : 0u;
+    } else if (u.score) {
         if (valid) {
             p.scores[(size_t)u.row * p.NA + u.t * TILE + t] = score;
             if (cx.gtiles < kScoreCap / TILE)
@@ -646,6 +657,65 @@ __device__ __forceinline__ void gather_prologue(const Params& p, uint8_t* base, 
     for (int lt = 0; lt < npre; ++lt) cp_async_arrive_noinc(&bars->full[lt]);
 }
 
+// Hierarchy, phase B: every thread issues its share of the gathered tile
+// described by row-table entries [0, 128) into `stage`, and arrives on that
+// stage's barrier once its copies have landed.
+__device__ __forceinline__ void gather_issue(const Params& p, uint8_t* base, Bars* bars, int stage) {
+    const int32_t* tab = reinterpret_cast<const int32_t*>(base + SM_ROWTAB);
+    uint8_t* ks = base + SM_STAGE + stage * STAGE_BYTES;
+#pragma unroll 1
+    for (int q = threadIdx.x; q < TILE * 16; q += NT) gather_piece(p, ks, ks + KV_BYTES, tab[q >> 4], q >> 4, q & 15);
+    cp_async_arrive_noinc(&bars->full[stage]);
+}
+
+// Hierarchy, phase B: the row table of the children tile: the level-1 gists
+// of the k2 selected groups, group after group (a short last group leaves
+// empty rows).
+__device__ __forceinline__ void hier_children_table(const Params& p, uint8_t* base, int row) {
+    const int32_t* sel2 = reinterpret_cast<const int32_t*>(base + SM_SEL);
+    int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
+    for (int r = threadIdx.x; r < TILE; r += NT) {
+        int32_t e = -1;
+        if (r < p.K * p.group) {
+            const int child = sel2[r / p.group] * p.group + r % p.group;
+            if (child < p.N1) e = (int32_t)(-((long long)row * p.N1 + child) - 2);
+        }
+        tab[r] = e;
+    }
+    __syncthreads();
+}
+
+// Hierarchy, phase B: the exact top-k1 of the children tile's scores (ties to
+// the lower level-1 index: the tile holds the children in ascending order),
+// published as idx1 and kept in shared memory, then the row table of the
+// raw tokens of those k1 chunks.
+__device__ __forceinline__ void hier_select_children(const Params& p, uint8_t* base, int row) {
+    const uint32_t* keys = reinterpret_cast<const uint32_t*>(base + SM_CKEY);
+    const int32_t* sel2 = reinterpret_cast<const int32_t*>(base + SM_SEL);
+    int32_t* sel1 = reinterpret_cast<int32_t*>(base + SM_SEL1);
+    int32_t* res = reinterpret_cast<int32_t*>(base + SM_STAGE);   // stage 0 is free once its tile is done
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(base + SM_STAGE + 1024);
+    const int n = min(TILE, p.K * p.group);
+    select_staged(keys, n, p.K1, res, scratch);
+    for (int r = threadIdx.x; r < p.K1; r += NT) {
+        const int pos = res[r];
+        const int child = sel2[pos / p.group] * p.group + pos % p.group;
+        sel1[r] = child;
+        p.idx1[(size_t)row * p.K1 + r] = child;
+    }
+    __syncthreads();
+    int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
+    for (int r = threadIdx.x; r < TILE; r += NT) {
+        int32_t e = -1;
+        if (r < p.K1 * p.C) {
+            const int sl = r / p.C;
+            e = (int32_t)(((long long)row * p.N1 + sel1[sl]) * p.C + (r - sl * p.C));
+        }
+        tab[r] = e;
+    }
+    __syncthreads();
+}
+
 // Final log-sum-exp merge of a row: phase-A slots [0, na) and phase-B slots
 // [maxs, maxs + nb).  The partials are brought into shared memory with
 // cp.async in groups (one memory round trip per group, short rolled loops),
@@ -790,39 +860,52 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
     // that phase A left in this SM's instruction cache
     int pu0 = 0, prow = -1, pn = 0, pslot = 0;
     int row = 0, j = 0, na = 0;
-    if (p.phase == 0) {
-        pu0 = unit_begin(ub, c);
-        pn = unit_begin(ub, c + 1) - pu0;
-    } else {
-        // phase B: this CTA takes tiles [t0, t0 + ntl) of `row`
-        row = c / p.cb;
-        j = c % p.cb;
-        const int t0 = j * p.tpc, ntl = max(0, min(p.nbt, t0 + p.tpc) - t0);
-        const int ru0 = row * p.upr;
-        const int cf = p.T > 0 ? cta_of(ub, p.grid, ru0) : 0;
-        na = p.T > 0 ? cta_of(ub, p.grid, ru0 + p.upr - 1) - cf + 1 : 0;   // phase-A slots
-        if (ntl > 0) {
-            if (p.do_topk && p.sel_direct) {
-                direct_select(p, cx.base, row, j == 0);
-            } else if (p.do_topk) {
-                int n = 0;
-                for (int cc = cf; cc < cf + na; ++cc) {
-                    int a0, a1;
-                    gists_of(cc, row, a0, a1);
-                    n += min(p.K, max(0, a1 - a0));
+    // the hierarchy's phase B runs two rounds in one CTA per row: the
+    // children tile (scored and attended), then the raw tile of the k1 chunks
+    const int rounds = (p.phase == 1 && p.hier) ? (p.K1 > 0 ? 2 : 1) : 1;
+    for (int rd = 0; rd < rounds; ++rd) {
+        if (p.phase == 0) {
+            pu0 = unit_begin(ub, c);
+            pn = unit_begin(ub, c + 1) - pu0;
+        } else {
+            // phase B: this CTA takes tiles [t0, t0 + ntl) of `row`
+            row = c / p.cb;
+            j = c % p.cb;
+            const int t0 = p.hier ? rd : j * p.tpc;
+            const int ntl = p.hier ? 1 : max(0, min(p.nbt, t0 + p.tpc) - t0);
+            const int ru0 = row * p.upr;
+            const int cf = p.T > 0 ? cta_of(ub, p.grid, ru0) : 0;
+            na = p.T > 0 ? cta_of(ub, p.grid, ru0 + p.upr - 1) - cf + 1 : 0;   // phase-A slots
+            if (rd == 1) {
+                hier_select_children(p, cx.base, row);
+            } else if (ntl > 0) {
+                if (p.do_topk && p.sel_direct) {
+                    direct_select(p, cx.base, row, j == 0);
+                } else if (p.do_topk) {
+                    int n = 0;
+                    for (int cc = cf; cc < cf + na; ++cc) {
+                        int a0, a1;
+                        gists_of(cc, row, a0, a1);
+                        n += min(p.K, max(0, a1 - a0));
+                    }
+                    merge_select(p, cx.base, row, n, j == 0);
+                } else {
+                    load_selection(p, cx.base, row);
                 }
-                merge_select(p, cx.base, row, n, j == 0);
-            } else {
-                load_selection(p, cx.base, row);
+                if (p.hier) hier_children_table(p, cx.base, row);
             }
-            gather_prologue(p, cx.base, cx.bars, row, t0, ntl);
+            if (p.hier) {
+                gather_issue(p, cx.base, cx.bars, rd % NS);
+            } else if (ntl > 0) {
+                gather_prologue(p, cx.base, cx.bars, row, t0, ntl);
+            }
+            pu0 = t0;
+            prow = row;
+            pn = ntl;
+            pslot = p.maxs + (p.hier ? rd : j);
         }
-        pu0 = t0;
-        prow = row;
-        pn = ntl;
-        pslot = p.maxs + j;
+        run_pipeline<G>(p, cx, pu0, prow, pn, pslot);
     }
-    run_pipeline<G>(p, cx, pu0, prow, pn, pslot);
     if (p.phase == 0) {
         if (p.do_topk && !p.sel_direct) {
             // local top-k of every segment, from the scores this CTA kept
@@ -860,7 +943,7 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
         __syncthreads();
         if (misc[0]) {
             __threadfence();
-            merge_row<G>(p, cx.base, row, na, p.nbt > 0 ? p.cb : 0);
+            merge_row<G>(p, cx.base, row, na, p.hier ? rounds : (p.nbt > 0 ? p.cb : 0));
         }
     }
     tc::fence_before();
@@ -1061,6 +1144,116 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
         p.phase = 0;
         e = launch(f.grid);
     }
+    if (e == cudaSuccess) {
+        p.phase = 1;
+        e = launch(f.grid_b);
+    }
+    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+// --------------------------------------------------------- hierarchy ----
+bool fused_hier_supported(const gsa_hier_desc& h) {
+    const gsa_decode_desc& d = h.l1;
+    const long long rows = (long long)d.batch * d.n_kv_heads;
+    const long long units = rows * ((h.n_l2 + 127) / 128 + (d.tail_len + 127) / 128);
+    return d.dtype == GSA_BF16 && d.head_dim == 128 && (long long)h.top_k2 * h.group <= 128 &&
+           (long long)d.top_k * d.chunk <= 128 && rows * d.n_chunks * d.chunk < INT32_MAX - 2 &&
+           rows * d.n_chunks < INT32_MAX - 2 && units < (1LL << 30);
+}
+
+FusedPlan make_fused_hier_plan(const gsa_hier_desc& h) {
+    // phase A and the level-2 selection are the flat step over the level-2 gists
+    gsa_decode_desc l2 = h.l1;
+    l2.n_chunks = h.n_l2;
+    l2.top_k = h.top_k2;
+    l2.mode = GSA_ALL_GISTS;
+    FusedPlan f = make_fused_plan(l2);
+    // phase B: one CTA per row, two partial slots (children tile, raw tile)
+    f.nbt = 2;
+    f.tpc = 2;
+    f.cb = 1;
+    f.grid_b = f.rows;
+    f.slot_stride = f.maxs + 2;
+    const size_t rows = (size_t)f.rows;
+    size_t o = f.off_part;
+    o = round256(o + rows * (size_t)f.slot_stride * f.G * 128 * 4);
+    f.off_ml = o;
+    o = round256(o + rows * (size_t)f.slot_stride * f.G * 4 * 4);
+    f.off_idx1 = o;
+    o = round256(o + rows * (size_t)h.l1.top_k * 4);
+    f.total = o;
+    return f;
+}
+
+gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const void* q, const void* k_g2,
+                             const void* v_g2, const void* k_g1, const void* v_g1, const void* kr, const void* vr,
+                             const void* kt, const void* vt, int32_t* idx2_out, int32_t* idx1_out, void* out,
+                             void* ws, cudaStream_t st) {
+    using namespace fused;
+    const gsa_decode_desc& d = h.l1;
+    if (f.grid <= 0 || f.grid_b <= 0) return GSA_ERR_ARG;
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t rows = (uint64_t)f.rows;
+    bool ok = map3d(&p.tm_kg, k_g2, rows, (uint64_t)h.n_l2) && map3d(&p.tm_vg, v_g2, rows, (uint64_t)h.n_l2) &&
+              map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
+    if (!ok) return GSA_ERR_CUDA;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.q = static_cast<const uint16_t*>(q);
+    p.kr = static_cast<const uint8_t*>(kr);
+    p.vr = static_cast<const uint8_t*>(vr);
+    p.kgp = static_cast<const uint8_t*>(k_g1);   // gathered "gist" rows are the level-1 gists
+    p.vgp = static_cast<const uint8_t*>(v_g1);
+    p.out = static_cast<uint16_t*>(out);
+    p.lse = nullptr;
+    p.err = reinterpret_cast<uint32_t*>(w + kWsErrOffset);
+    p.cnt = reinterpret_cast<uint32_t*>(w + kWsCntOffset);
+    p.scores = reinterpret_cast<float*>(w + f.off_scores);
+    p.idx = idx2_out ? idx2_out : reinterpret_cast<int32_t*>(w + f.off_idx);
+    p.idx1 = idx1_out ? idx1_out : reinterpret_cast<int32_t*>(w + f.off_idx1);
+    p.cand_key = reinterpret_cast<uint32_t*>(w + f.off_cand_key);
+    p.cand_idx = reinterpret_cast<int32_t*>(w + f.off_cand_idx);
+    p.part = reinterpret_cast<float*>(w + f.off_part);
+    p.ml = reinterpret_cast<float*>(w + f.off_ml);
+    p.rows = f.rows;
+    p.Hkv = d.n_kv_heads;
+    p.G = f.G;
+    p.N = h.n_l2;
+    p.NA = h.n_l2;
+    p.C = d.chunk;
+    p.K = h.top_k2;
+    p.W = d.tail_len;
+    p.mode = GSA_ALL_GISTS;
+    p.tg = f.tg;
+    p.upr = f.upr;
+    p.T = f.T;
+    p.grid = f.grid;
+    p.slot_stride = f.slot_stride;
+    p.maxs = f.maxs;
+    p.nrows_g = 0;
+    p.nbt = f.nbt;
+    p.tpc = f.tpc;
+    p.cb = f.cb;
+    const double scale = d.scale > 0 ? (double)d.scale : 1.0 / std::sqrt(128.0);
+    p.c2 = (float)(scale * 1.4426950408889634);
+    p.do_score = 1;
+    p.do_topk = 1;
+    p.do_attn_gists = 1;
+    p.sel_direct = f.sel_direct;
+    p.hier = 1;
+    p.group = h.group;
+    p.N1 = d.n_chunks;
+    p.K1 = d.top_k;
+    auto launch = [&](int grid) {
+        switch (f.G) {
+            case 1: return launch_g<1>(p, grid, st);
+            case 2: return launch_g<2>(p, grid, st);
+            case 4: return launch_g<4>(p, grid, st);
+            default: return launch_g<8>(p, grid, st);
+        }
+    };
+    p.phase = 0;
+    cudaError_t e = launch(f.grid);
     if (e == cudaSuccess) {
         p.phase = 1;
         e = launch(f.grid_b);

@@ -20,6 +20,7 @@ struct FusedPlan {
     int slot_stride;                  // maxs + cb
     int sel_direct;                   // phase B selects from the scores (else from phase-A candidates)
     size_t off_scores, off_cand_key, off_cand_idx, off_idx, off_part, off_ml, total;
+    size_t off_idx1;                  // hierarchy: level-1 selection (when the caller passes none)
 };
 
 namespace fused {
@@ -48,10 +49,21 @@ struct Params {
     int T;                         // phase-A units in all
     float c2;
     int do_score, do_topk, do_attn_gists, sel_direct;
+    // hierarchy (phase A: level-2 gists; phase B: children tile, then raw tile)
+    int hier, group, N1, K1;       // K = k2, N = NA = n_l2; group, level-1 gists, k1
+    int32_t* idx1;                 // [rows][k1]
 };
 }  // namespace fused
 
 bool fused_supported(const gsa_decode_desc& d);
+// The hierarchy on the same kernel: the children of the selected groups must
+// fit one 128-row tile, and so must the raw tokens of the k1 chunks.
+bool fused_hier_supported(const gsa_hier_desc& h);
+FusedPlan make_fused_hier_plan(const gsa_hier_desc& h);
+gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const void* q, const void* k_g2,
+                             const void* v_g2, const void* k_g1, const void* v_g1, const void* kr, const void* vr,
+                             const void* kt, const void* vt, int32_t* idx2_out, int32_t* idx1_out, void* out,
+                             void* ws, cudaStream_t st);
 // given: the selection is supplied (gsa_unfold_attn), so nothing is scored.
 FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given = false);
 // Enqueue the fused decode step.  idx_given != null: attend over that

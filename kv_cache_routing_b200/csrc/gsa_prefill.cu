@@ -43,7 +43,12 @@
 
 namespace gsa {
 
-constexpr int PF_THREADS = 320;
+constexpr int PF_THREADS = 384;   // three warpgroups: softmax A, softmax B, loads + MMA
+// Register split (setmaxnreg): launched at 168 a thread (384 x 168 = 64,512),
+// the load/MMA warpgroup gives back down to 72 and the two softmax warpgroups
+// grow to 216: 2 x 128 x 216 + 128 x 72 = 64,512, the same total.
+constexpr uint32_t PF_REG_SOFTMAX = 216, PF_REG_OTHER = 72;
+static_assert(2 * 128 * PF_REG_SOFTMAX + 128 * PF_REG_OTHER == PF_THREADS * 168, "register split must add up");
 constexpr int PF_D = 128;
 constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
 constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, 128, 0, 1);  // P (TMEM, K-major) x V (MN-major)
@@ -106,8 +111,7 @@ struct PfBars {
     uint32_t tmem;
 };
 
-// 168 registers a thread: three warps of 10 share each scheduler's 16K registers
-__global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -152,6 +156,9 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
     const uint32_t tmem = bars.tmem;
     uint32_t* err = &g_prefill_err;   // waits below are bounded; a timeout abandons the tile
 
+    if (warp >= 8) {
+    // --------------------------------- load / MMA warpgroup (warps 8-11) ----
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PF_REG_OTHER));
     if (warp == 8) {
         if (lane == 0) {
             // --------------------------------------------------- TMA loads --
@@ -226,8 +233,10 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
                 }
             }
         }
+    }
     } else {
         // ------------------------------------------------ softmax warps ----
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(PF_REG_SOFTMAX));
         const int h = warp >> 2;                         // 0: head A, 1: head B
         if (h == 0 || hasB) {
             const int r = threadIdx.x & 127;             // query row = TMEM lane
@@ -249,44 +258,30 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
                     lo = valid ? jq * (p.C + 1) - p0 : 1;
                     hi = valid ? r : 0;
                 }
-                // pass 1: the row maximum (S stays in TMEM); the scale is applied
-                // to the maximum (it is positive), and a warp whose rows all see
-                // the whole tile takes the unmasked path (warp-uniform: the
-                // tcgen05.ld inside is .sync.aligned)
+                // the row's 128 scores in registers (all four loads in flight)
+                uint32_t uu[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tc::ld32(ts + c * 32, uu[c]);
+                tc::wait_ld();
+                uint32_t* u = &uu[0][0];
+                // the row maximum of the allowed columns; the scale is applied to
+                // the maximum (it is positive); a warp whose rows all see the
+                // whole tile takes the unmasked path
                 const bool full = __all_sync(0xFFFFFFFFu, lo == 0 && hi >= 127);
-                float mt = -INFINITY;
-                if (full) {
-                    // two 32-column loads in flight, four independent max chains
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (!full) {
 #pragma unroll
-                    for (int c = 0; c < 4; c += 2) {
-                        uint32_t u[32], v[32];
-                        tc::ld32(ts + c * 32, u);
-                        tc::ld32(ts + c * 32 + 32, v);
-                        tc::wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            m4[(j >> 2) & 3] = max3(m4[(j >> 2) & 3], __uint_as_float(u[j]), __uint_as_float(u[j + 1]));
-                            m4[((j >> 2) + 1) & 3] =
-                                max3(m4[((j >> 2) + 1) & 3], __uint_as_float(u[j + 2]), __uint_as_float(u[j + 3]));
-                            m4[((j >> 2) + 2) & 3] = max3(m4[((j >> 2) + 2) & 3], __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-                            m4[((j >> 2) + 3) & 3] =
-                                max3(m4[((j >> 2) + 3) & 3], __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-                        }
-                    }
-                    mt = max3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t u[32];
-                        tc::ld32(ts + c * 32, u);
-                        tc::wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (c * 32 + j >= lo && c * 32 + j <= hi) mt = fmaxf(mt, __uint_as_float(u[j]));
-                    }
+                    for (int jj = 0; jj < 128; ++jj)
+                        if (jj < lo || jj > hi) u[jj] = __float_as_uint(-INFINITY);
                 }
-                mt *= p.c2;
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int jj = 0; jj < 128; jj += 8) {
+                    m4[0] = max3(m4[0], __uint_as_float(u[jj]), __uint_as_float(u[jj + 1]));
+                    m4[1] = max3(m4[1], __uint_as_float(u[jj + 2]), __uint_as_float(u[jj + 3]));
+                    m4[2] = max3(m4[2], __uint_as_float(u[jj + 4]), __uint_as_float(u[jj + 5]));
+                    m4[3] = max3(m4[3], __uint_as_float(u[jj + 6]), __uint_as_float(u[jj + 7]));
+                }
+                const float mt = max3(fmaxf(m4[0], m4[1]), m4[2], m4[3]) * p.c2;
                 bool need = false;
                 float m_new = m_run;
                 if (mt > -INFINITY) {
@@ -304,48 +299,36 @@ __global__ void __maxnreg__(168) gist_prefill_kernel(const __grid_constant__ Pre
                     tc::fence_after();
 #pragma unroll 1
                     for (int c = 0; c < 8; ++c) {
-                        uint32_t u[16];
-                        tc::ld16(to + c * 16, u);
+                        uint32_t o[16];
+                        tc::ld16(to + c * 16, o);
                         tc::wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
-                        tc::st16(to + c * 16, u);
+                        for (int jj = 0; jj < 16; ++jj) o[jj] = __float_as_uint(__uint_as_float(o[jj]) * alpha);
+                        tc::st16(to + c * 16, o);
                     }
                 }
                 m_run = m_new;
-                // pass 2: P (bf16 pairs) over the first 64 columns of S, in key
-                // order, so every column it overwrites has been read already; the
-                // P.V of the previous tile finished before this S was written
-                // x * c2 - m in pairs (fma.f32x2), 2^x on the SFU, pair sums (add.f32x2)
-                const uint64_t c22 = f2(p.c2, p.c2), nm2 = f2(-m_run, -m_run);
+                // P (bf16 pairs) over the first 64 columns of S (all of S is in
+                // registers); the P.V of the previous tile finished before this S
+                // was written.  x * c2 - m in pairs (fma.f32x2), 2^x on the SFU
+                // (masked: -inf -> 0), pair sums (add.f32x2)
+                // (a row with nothing allowed yet subtracts 0: its masked -inf stay -inf)
+                const float ms = m_run == -INFINITY ? 0.f : m_run;
+                const uint64_t c22 = f2(p.c2, p.c2), nm2 = f2(-ms, -ms);
                 uint64_t acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-                for (int c = 0; c < 4; c += 2) {
-                    // two 32-column loads in flight; their P goes to columns
-                    // [16c, 16c + 32), all read by now (this chunk or the previous one)
-                    uint32_t u[2][32];
-                    tc::ld32(ts + c * 32, u[0]);
-                    tc::ld32(ts + c * 32 + 32, u[1]);
-                    tc::wait_ld();
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t w[16];
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t w[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int j = (c + hh) * 32 + 2 * e;
-                            float xa, xb;
-                            unf2(ffma2(f2(__uint_as_float(u[hh][2 * e]), __uint_as_float(u[hh][2 * e + 1])), c22, nm2),
-                                 xa, xb);
-                            if (!full) {
-                                xa = (j >= lo && j <= hi) ? xa : -INFINITY;
-                                xb = (j + 1 >= lo && j + 1 <= hi) ? xb : -INFINITY;
-                            }
-                            const float a = ex2(xa), bb = ex2(xb);
-                            acc2[e & 1] = fadd2(acc2[e & 1], f2(a, bb));
-                            w[e] = tc::pack_bf16x2(a, bb);
-                        }
-                        tc::st16(ts + (c + hh) * 16, w);
+                    for (int e = 0; e < 16; ++e) {
+                        const int jj = c * 32 + 2 * e;
+                        float xa, xb;
+                        unf2(ffma2(f2(__uint_as_float(u[jj]), __uint_as_float(u[jj + 1])), c22, nm2), xa, xb);
+                        const float a = ex2(xa), bb = ex2(xb);
+                        acc2[e & 1] = fadd2(acc2[e & 1], f2(a, bb));
+                        w[e] = tc::pack_bf16x2(a, bb);
                     }
+                    tc::st16(ts + c * 16, w);
                 }
                 float sa, sb;
                 unf2(fadd2(acc2[0], acc2[1]), sa, sb);

@@ -519,8 +519,11 @@ __device__ __forceinline__ void run_pipeline(const Params& p, Ctx& cx, int u0, i
 __device__ __noinline__ void select_staged(const uint32_t* keys, int n, int k, int32_t* res, uint32_t* scratch) {
     if (k >= n) {
         for (int i = threadIdx.x; i < n; i += NT) res[i] = i;
-    } else if (!(k <= 32 && n <= NT * 16 && threshold_topk<NT, 16>(keys, n, k, res, scratch))) {
-        smem_topk<NT>(keys, n, k, res, scratch);
+    } else {
+        bool done = false;
+        if (k <= 32 && n <= NT * 16) done = threshold_topk<NT, 16>(keys, n, k, res, scratch);
+        else if (k <= 32 && n <= NT * 32) done = threshold_topk<NT, 32>(keys, n, k, res, scratch);
+        if (!done) smem_topk<NT>(keys, n, k, res, scratch);
     }
     __syncthreads();
 }
@@ -583,13 +586,13 @@ __device__ __forceinline__ void merge_select(const Params& p, uint8_t* base, int
 
 // The row's exact top-k straight from its n = N routing scores (small N and
 // k): the scores are staged with all loads of a thread in flight at once.
-__device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, int row, bool publish) {
+template <int U>   // n <= U * NT
+__device__ __forceinline__ void direct_select_u(const Params& p, uint8_t* base, int row, bool publish) {
     const int n = p.NA, k = p.K;
     const float* sg = p.scores + (size_t)row * p.NA;
     uint32_t* keys = reinterpret_cast<uint32_t*>(base + SM_STAGE);
     int32_t* res = reinterpret_cast<int32_t*>(keys + ((n + 31) & ~31));
     uint32_t* scratch = reinterpret_cast<uint32_t*>(res + ((min(k, n) + 31) & ~31));
-    constexpr int U = 16;   // n <= U * NT
     float v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -610,6 +613,11 @@ __device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, in
         if (publish) out[r] = res[r];
     }
     __syncthreads();
+}
+
+__device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, int row, bool publish) {
+    if (p.NA <= 16 * NT) direct_select_u<16>(p, base, row, publish);
+    else direct_select_u<32>(p, base, row, publish);
 }
 
 // A given selection (gsa_unfold_attn) into sel[0..k); an index outside
@@ -718,15 +726,22 @@ __device__ __forceinline__ void hier_select_children(const Params& p, uint8_t* b
 
 // Final log-sum-exp merge of a row: phase-A slots [0, na) and phase-B slots
 // [maxs, maxs + nb).  The partials are brought into shared memory with
-// cp.async in groups (one memory round trip per group, short rolled loops),
-// and each output keeps a running (M, L, acc) over the groups.
+// cp.async in groups (one memory round trip per group).  Per group, warp h
+// finds head h's largest slot maximum M_g and each slot's weight
+// 2^(m_s - M_g) and the weighted sum L_g of the l_s; each output is then a
+// plain weighted sum over the slots (independent products, no dependent
+// rescaling chain), folded into a running (M, L, acc) once per group.
 template <int G>
 __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int row, int na, int nb) {
+    constexpr int NW = NT / 32;
     const int nsl = na + nb;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int PER = (G * D + NT - 1) / NT;          // outputs per thread
-    constexpr int GS = (int)(STAGE_BYTES * NS / ((G * D + 4 * G) * 4));   // slots per group
+    constexpr int GS = (int)((STAGE_BYTES * NS - 256) / ((G * D + 5 * G) * 4));   // slots per group
     float* so = reinterpret_cast<float*>(base + SM_STAGE);              // [GS][G][D]
     float* sml = so + GS * G * D;                                       // [GS][G][4]: (m, l, -, -)
+    float* wgt = sml + GS * G * 4;                                      // [GS][G]
+    float* gml = wgt + GS * G;                                          // [G][2]: (M_g, L_g)
     float M[PER], L[PER], acc[PER];
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
@@ -751,21 +766,48 @@ __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int ro
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncthreads();
+#pragma unroll 1
+        for (int h = warp; h < G; h += NW) {
+            float mx = -INFINITY;
+            for (int sl = lane; sl < cnt; sl += 32) mx = fmaxf(mx, sml[(sl * G + h) * 4]);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+            float ls = 0.f;
+            for (int sl = lane; sl < cnt; sl += 32) {
+                const float m = sml[(sl * G + h) * 4];
+                const float wv = m > -INFINITY ? exp2f(m - mx) : 0.f;
+                wgt[sl * G + h] = wv;
+                ls += sml[(sl * G + h) * 4 + 1] * wv;
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, o);
+            if (lane == 0) {
+                gml[h * 2] = mx;
+                gml[h * 2 + 1] = ls;
+            }
+        }
+        __syncthreads();
 #pragma unroll
         for (int q = 0; q < PER; ++q) {
             const int i = threadIdx.x + q * NT;
             if (i < G * D) {
                 const int h = i / D;
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                int sl = 0;
 #pragma unroll 1
-                for (int sl = 0; sl < cnt; ++sl) {
-                    const float m = sml[(sl * G + h) * 4];
-                    if (m > -INFINITY) {
-                        const float Mn = fmaxf(M[q], m);
-                        const float a = (M[q] == -INFINITY) ? 0.f : exp2f(M[q] - Mn), w = exp2f(m - Mn);
-                        L[q] = L[q] * a + sml[(sl * G + h) * 4 + 1] * w;
-                        acc[q] = acc[q] * a + so[sl * G * D + i] * w;
-                        M[q] = Mn;
-                    }
+                for (; sl + 4 <= cnt; sl += 4) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) a4[e] += wgt[(sl + e) * G + h] * so[(sl + e) * G * D + i];
+                }
+                for (; sl < cnt; ++sl) a4[0] += wgt[sl * G + h] * so[sl * G * D + i];
+                const float ag = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+                const float Mg = gml[h * 2], Lg = gml[h * 2 + 1];
+                if (Mg > -INFINITY) {
+                    const float Mn = fmaxf(M[q], Mg);
+                    const float a = (M[q] == -INFINITY) ? 0.f : exp2f(M[q] - Mn), wg = exp2f(Mg - Mn);
+                    L[q] = L[q] * a + Lg * wg;
+                    acc[q] = acc[q] * a + ag * wg;
+                    M[q] = Mn;
                 }
             }
         }
@@ -1045,7 +1087,7 @@ FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given) {
     f.maxs = maxs;
     // small selections are taken in phase B straight from the scores; larger
     // ones from per-CTA candidates that phase A leaves
-    f.sel_direct = (d.top_k <= 32 && d.n_chunks <= 16 * fused::NT) ? 1 : 0;
+    f.sel_direct = (d.top_k <= 32 && d.n_chunks <= 32 * fused::NT) ? 1 : 0;
     // phase B: the row's gathered rows packed into 128-row tiles, spread over
     // as many CTAs per row as fill the GPU (at most kMaxTpc tiles each)
     f.nrows_g = d.top_k * d.chunk + (pairs ? d.top_k : 0);

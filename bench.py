@@ -575,7 +575,7 @@ def run_hier(args, world, rank, local):
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": qh.numel() * qh.element_size(),
                 "d2h_bytes_per_step": oh.numel() * oh.element_size()},
-        "gpu_launches": 3 * args.steps,   # level-2 gist pass, level-1 gist pass, unfold pass
+        "gpu_launches": gsa.gsa_hier_launch_count(hd) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0:

@@ -198,6 +198,10 @@ gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, c
  * invalid.  Host only, enqueues nothing. */
 int gsa_decode_launch_count(const gsa_decode_desc* desc);
 
+/* The same for one gsa_hier_decode call: 1 on the tensor-core path, 3 on the
+ * CUDA-core passes; -1 if the descriptor is invalid.  Host only. */
+int gsa_hier_launch_count(const gsa_hier_desc* desc);
+
 /* Reads (synchronously, on `stream`) the workspace error word: 0, or an OR of
  * GSA_WS_ERR_* flags; returns GSA_ERR_TIMEOUT if a bounded wait expired,
  * GSA_ERR_ARG if an index was out of range, else GSA_OK.  flags_out nullable. */

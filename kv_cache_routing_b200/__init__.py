@@ -23,7 +23,8 @@ GSA_WS_ERR_TIMEOUT, GSA_WS_ERR_INDEX = 1, 2
 # Every function the C header declares (checked by the tests).
 EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", "gsa_topk",
            "gsa_unfold_attn", "gsa_decode_step", "gsa_hier_decode", "gsa_gist_prefill",
-           "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count")
+           "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count",
+           "gsa_hier_launch_count")
 
 
 class GsaError(RuntimeError):
@@ -70,6 +71,7 @@ def _signatures():
         "gsa_workspace_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
         "gsa_status_string": (ctypes.c_char_p, [st]),
         "gsa_decode_launch_count": (ctypes.c_int, [pd]),
+        "gsa_hier_launch_count": (ctypes.c_int, [ph]),
     }
 
 
@@ -206,6 +208,14 @@ def gsa_decode_launch_count(desc) -> int:
     n = lib().gsa_decode_launch_count(ctypes.byref(desc))
     if n < 0:
         raise GsaError(1, "gsa_decode_launch_count")
+    return int(n)
+
+
+def gsa_hier_launch_count(desc) -> int:
+    """Kernel launches one gsa_hier_decode with `desc` enqueues."""
+    n = lib().gsa_hier_launch_count(ctypes.byref(desc))
+    if n < 0:
+        raise GsaError(1, "gsa_hier_launch_count")
     return int(n)
 
 

@@ -829,9 +829,14 @@ gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, c
                            need, stream);
 }
 
+int gsa_hier_launch_count(const gsa_hier_desc* desc) {
+    if (validate_hier(desc) != GSA_OK) return -1;
+    return fused_hier_supported(*desc) ? 1 : 3;
+}
+
 int gsa_decode_launch_count(const gsa_decode_desc* desc) {
     if (validate_decode(desc) != GSA_OK) return -1;
-    if (fused_supported(*desc)) return make_fused_plan(*desc).grid > 0 ? 2 : 1;
+    if (fused_supported(*desc)) return 1;
     return (desc->n_chunks > 0 ? 1 : 0) + 1;
 }
 

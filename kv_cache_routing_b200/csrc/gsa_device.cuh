@@ -162,19 +162,30 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
 // ---------------------------------------------------------- ordering keys --
 // Monotone map fp32 -> u32 (larger score -> larger key).  -0 and +0 share a
 // key; NaN maps to 0, below every number.
+// Written with selects only, so that a key computed from a load does not
+// put a branch between that load and the next.
 __device__ __forceinline__ uint32_t order_key(float f) {
-    if (f != f) return 0u;
-    if (f == 0.0f) f = 0.0f;
-    uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const uint32_t u = f == 0.0f ? 0u : __float_as_uint(f);
+    const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return f != f ? 0u : k;
+}
+
+// ------------------------------------------------------------ thread groups --
+// The block-wide helpers below run on a group of NT threads: threads
+// [FIRST, FIRST + NT) of the block, synchronised by named barrier BAR (0: the
+// whole block, NT == blockDim.x).  FIRST is a multiple of 32.
+template <int NT, int BAR>
+__device__ __forceinline__ void group_sync() {
+    if constexpr (BAR == 0) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
 }
 
 // -------------------------------------------------------------- block scan --
-// Exclusive prefix sum over the block; returns this thread's prefix and
-// writes the block total to *total.  `sh` holds >= NT/32 + 1 words.
-template <int NT>
+// Exclusive prefix sum over the group; returns this thread's prefix and
+// writes the group total to *total.  `sh` holds >= NT/32 + 1 words.
+template <int NT, int BAR = 0, int FIRST = 0>
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* sh, uint32_t* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = (threadIdx.x - FIRST) >> 5;
     constexpr int NW = NT / 32;
     uint32_t x = v;
 #pragma unroll
@@ -183,7 +194,7 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
         if (lane >= o) x += y;
     }
     if (lane == 31) sh[warp] = x;
-    __syncthreads();
+    group_sync<NT, BAR>();
     if (warp == 0) {
         uint32_t w = lane < NW ? sh[lane] : 0u;
 #pragma unroll
@@ -193,10 +204,10 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
         }
         if (lane < NW) sh[lane] = w;  // inclusive warp totals
     }
-    __syncthreads();
+    group_sync<NT, BAR>();
     uint32_t before = (warp > 0 ? sh[warp - 1] : 0u) + x - v;
     *total = sh[NW - 1];
-    __syncthreads();
+    group_sync<NT, BAR>();
     return before;
 }
 
@@ -208,9 +219,9 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // Radix select over the 32-bit key, 8 bits per pass, then one ordered
 // compaction.  `sh` holds >= 256 + NT/32 + 8 words of shared memory.
 // All NT threads of the block must call it.
-template <int NT, class KeyF, class Emit>
+template <int NT, int BAR = 0, int FIRST = 0, class KeyF, class Emit>
 __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x - FIRST;
     if (k <= 0 || n <= 0) return;
     if (k >= n) {
         for (int i = tid; i < n; i += NT) emit(i, i);
@@ -223,7 +234,7 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
     uint32_t kk = static_cast<uint32_t>(k);
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += NT) hist[i] = 0;
-        __syncthreads();
+        group_sync<NT, BAR>();
         // warp-aggregated histogram: float keys crowd a few bins in the high
         // digits, so lanes with the same bin add once per warp instruction
         for (int i0 = tid - (tid & 31); i0 < n; i0 += NT) {
@@ -236,7 +247,7 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
             const uint32_t same = __match_any_sync(0xFFFFFFFFu, bin);
             if (bin != 0xFFFFFFFFu && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         if (tid < 32) {
             // lane l owns bins 255-8l .. 248-8l (descending)
             const int lane = tid;
@@ -262,12 +273,12 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
                 above += cnt[t];
             }
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         uint32_t digit = res[0];
         kk -= res[1];
         prefix |= digit << shift;
         pmask |= 255u << shift;
-        __syncthreads();
+        group_sync<NT, BAR>();
     }
     // threshold key T = prefix: take every key > T and the first kk keys == T.
     const uint32_t T = prefix;
@@ -276,14 +287,14 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
     uint32_t n_eq = 0;
     for (int i = lo; i < hi; ++i) n_eq += (key(i) == T);
     uint32_t tot;
-    uint32_t eq_before = block_exclusive_scan<NT>(n_eq, scan, &tot);
+    uint32_t eq_before = block_exclusive_scan<NT, BAR, FIRST>(n_eq, scan, &tot);
     uint32_t n_sel = 0, e = eq_before;
     for (int i = lo; i < hi; ++i) {
         uint32_t u = key(i);
         if (u > T) ++n_sel;
         else if (u == T) { if (e < kk) ++n_sel; ++e; }
     }
-    uint32_t sel_before = block_exclusive_scan<NT>(n_sel, scan, &tot);
+    uint32_t sel_before = block_exclusive_scan<NT, BAR, FIRST>(n_sel, scan, &tot);
     uint32_t r = sel_before;
     e = eq_before;
     for (int i = lo; i < hi; ++i) {
@@ -307,9 +318,9 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
 // Scratch `w` (shared): >= 256 + 16 + 2*NT/32 + (n+31)/32 * 2 + 2*n words
 // (histogram, control, scan, two bitmaps, two candidate lists).
 // All NT threads of the block call it.
-template <int NT>
+template <int NT, int BAR = 0, int FIRST = 0>
 __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint32_t* w) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x - FIRST, lane = tid & 31, warp = tid >> 5;
     constexpr int NW = NT / 32;
     if (k <= 0 || n <= 0) return;
     if (k >= n) {
@@ -334,7 +345,7 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += NT) hist[i] = 0;
         if (tid == 0) ctl[2] = 0;
-        __syncthreads();
+        group_sync<NT, BAR>();
         for (int i0 = tid - lane; i0 < m; i0 += NT) {
             const int i = i0 + lane;
             uint32_t bin = 0xFFFFFFFFu;
@@ -342,7 +353,7 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
             const uint32_t same = __match_any_sync(0xFFFFFFFFu, bin);
             if (bin != 0xFFFFFFFFu && lane == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         if (warp == 0) {
             // lane l owns bins 255-8l .. 248-8l (descending)
             uint32_t cnt[8], tot = 0;
@@ -367,7 +378,7 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
                 above += cnt[t];
             }
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         const uint32_t D = ctl[0], above = ctl[1];
         const bool last = shift == 0;
         // keys above the threshold digit are selected; keys on it stay
@@ -400,7 +411,7 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
                 if (eq) next[base + __popc(meq & ((1u << lane) - 1u))] = (uint32_t)pos;
             }
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         kk -= above;
         m = (int)ctl[2];
         all = false;
@@ -409,12 +420,12 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
             cand = next;
             next = t;
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         if (!last && (uint32_t)m == kk) {
             // every remaining candidate is selected
             for (int i = tid; i < m; i += NT) atomicOr(&sel[cand[i] >> 5], 1u << (cand[i] & 31));
             kk = 0;
-            __syncthreads();
+            group_sync<NT, BAR>();
             break;
         }
     }
@@ -424,7 +435,7 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
         const int per = (nw + NT - 1) / NT, lo = tid * per, hi = min(nw, lo + per);
         for (int i = lo; i < hi; ++i) c += __popc(tie[i]);
         uint32_t tot;
-        uint32_t before = block_exclusive_scan<NT>(c, scan, &tot);
+        uint32_t before = block_exclusive_scan<NT, BAR, FIRST>(c, scan, &tot);
         for (int i = lo; i < hi; ++i) {
             uint32_t bits = tie[i];
             while (bits) {
@@ -434,7 +445,7 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
                 ++before;
             }
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
     }
     // emit the selection in ascending position order
     {
@@ -442,7 +453,7 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
         const int per = (nw + NT - 1) / NT, lo = tid * per, hi = min(nw, lo + per);
         for (int i = lo; i < hi; ++i) c += __popc(sel[i]);
         uint32_t tot;
-        uint32_t r = block_exclusive_scan<NT>(c, scan, &tot);
+        uint32_t r = block_exclusive_scan<NT, BAR, FIRST>(c, scan, &tot);
         for (int i = lo; i < hi; ++i) {
             uint32_t bits = sel[i];
             while (bits) {
@@ -456,91 +467,123 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
 
 
 // --------------------------------------------------- threshold top-k --
-// Exact top-k for k <= 32 of n <= NT * M keys held in shared memory (keys[i]
-// for position i): the k largest keys, equal keys taken lowest position
-// first; out[0..k) receives the positions in ascending order.
-//  1. Thread t holds the block of positions [t*m, t*m + m), m = ceil(n / NT).
-//  2. In each warp, the k-th largest of the 32 lane maxima bounds the k-th
+// Exact top-k for k <= 32 of n <= NT * M keys: the k largest keys, equal keys
+// taken lowest position first; out[0..k) receives the positions in ascending
+// order.  Thread t holds the keys of positions lo + i * step, i < mine, in
+// registers (key[i]); the positions of the threads may interleave in any way
+// (step NT: every warp-wide load is one contiguous line).
+//  1. In each warp, the k-th largest of the 32 lane maxima bounds the k-th
 //     largest key of the whole set from below (k distinct keys reach it), so
 //     the largest such bound over the warps, tau, does as well.
-//  3. The keys >= tau (k of them at least, and rarely many more) are compacted
-//     in position order; each counts the candidates ahead of it (a larger key,
-//     or the same key at a lower position), and those with fewer than k ahead
-//     are written out in position order.
+//  2. The keys >= tau (k of them at least, and rarely many more) are appended,
+//     in any order, to a shared list as 64-bit composites (key, ~position): a
+//     larger composite is a larger key, or the same key at a lower position.
+//  3. Each candidate counts the composites above its own; those with fewer
+//     than k above are selected, and each selected one counts the selected
+//     ones at lower positions to find its place in the output.
 // Returns false without writing anything when more than NT keys reach tau
 // (a flood of equal keys): the caller then runs a general selection.
-// Scratch `w` (shared): >= 2 * NT + 2 * (NT / 32) + 8 words.
+// Scratch `w` (shared, 16-byte aligned): >= 16 + 2 * NT + 2 + NT / 4 words.
 // All NT threads call it; it ends with the block synchronised.
-template <int NT, int M>
-__device__ bool threshold_topk(const uint32_t* keys, int n, int k, int32_t* out, uint32_t* w) {
+template <int NT, int M, int BAR = 0, int FIRST = 0>
+__device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, int mine, int k, int32_t* out,
+                                    uint32_t* w) {
     constexpr int NW = NT / 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int m = (n + NT - 1) / NT;
-    const int lo = tid * m;
-    const int mine = max(0, min(m, n - lo));
-    uint32_t key[M];
+    static_assert(NW + 1 <= 16, "warp bound table overflow");
+    const int tid = threadIdx.x - FIRST, lane = tid & 31, warp = tid >> 5;
     uint32_t tmax = 0u;
 #pragma unroll
-    for (int i = 0; i < M; ++i) {
-        key[i] = i < mine ? keys[lo + i] : 0u;
-        tmax = max(tmax, key[i]);
-    }
-    // rank of this lane's maximum in its warp (equal values ordered by lane):
-    // the lane of rank k-1 holds the warp's bound (a lane without keys offers
-    // 0, the smallest key, which can only weaken the bound)
-    int ahead = 0;
+    for (int i = 0; i < M; ++i) tmax = max(tmax, i < mine ? key[i] : 0u);
+    // the k-th largest of the warp's 32 lane maxima is the warp's bound (a
+    // lane without keys offers 0, the smallest key, which can only weaken
+    // it): a bitonic sort of the lane maxima, descending, leaves it in lane k-1
+    uint32_t v = tmax;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const uint32_t v = __shfl_sync(0xFFFFFFFFu, tmax, j);
-        ahead += (v > tmax || (v == tmax && j < lane)) ? 1 : 0;
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
+            // descending runs where (lane & size) == 0, the final pass descending
+            const bool desc = ((lane & size) == 0) || size == 32;
+            const bool lower = (lane & stride) == 0;
+            v = (lower == desc) ? max(v, o) : min(v, o);
+        }
     }
-    const uint32_t at = __ballot_sync(0xFFFFFFFFu, ahead == k - 1);
-    const uint32_t tau_w = __shfl_sync(0xFFFFFFFFu, tmax, __ffs(at) - 1);
+    const uint32_t tau_w = __shfl_sync(0xFFFFFFFFu, v, k - 1);
     if (lane == 0) w[warp] = tau_w;
-    __syncthreads();
+    if (tid == 0) w[NW] = 0u;
+    group_sync<NT, BAR>();
     uint32_t tau = w[0];
 #pragma unroll
     for (int i = 1; i < NW; ++i) tau = max(tau, w[i]);
+    // append this thread's candidates: one atomic per warp
     uint32_t c = 0;
 #pragma unroll
     for (int i = 0; i < M; ++i) c += (i < mine && key[i] >= tau) ? 1u : 0u;
-    uint32_t total;
-    uint32_t off = block_exclusive_scan<NT>(c, w + NW, &total);
-    if (total > (uint32_t)NT) return false;       // the same on every thread
-    uint32_t* ckey = w + 2 * NW + 8;   // 16-byte aligned when w is
-    uint32_t* cpos = ckey + NT;
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    uint32_t base = 0;
+    if (lane == 31 && incl > 0) base = atomicAdd(&w[NW], incl);
+    base = __shfl_sync(0xFFFFFFFFu, base, 31);
+    uint32_t off = base + incl - c;
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(w + 16);
+    uint8_t* flag = reinterpret_cast<uint8_t*>(w + 16 + 2 * NT + 2);
 #pragma unroll
     for (int i = 0; i < M; ++i)
         if (i < mine && key[i] >= tau) {
-            ckey[off] = key[i];
-            cpos[off] = (uint32_t)(lo + i);
+            if (off < (uint32_t)NT)
+                cand[off] = ((unsigned long long)key[i] << 32) | (unsigned long long)(~(uint32_t)(lo + i * step));
             ++off;
         }
-    // pad the list to a multiple of 4 with key 0: a pad is never ahead of a
-    // candidate (it is not larger, and an equal one sits at a higher index)
-    if ((uint32_t)tid < ((total + 3u) & ~3u) - total) ckey[total + tid] = 0u;
-    __syncthreads();
-    uint32_t sel = 0, pos = 0;
+    group_sync<NT, BAR>();
+    const uint32_t total = w[NW];
+    if (total > (uint32_t)NT) return false;       // the same on every thread
+    unsigned long long mc = 0ull;
+    bool sel = false;
     if ((uint32_t)tid < total) {
-        const uint32_t mk = ckey[tid];
-        int a = 0;
-        const uint4* c4 = reinterpret_cast<const uint4*>(ckey);
-        for (int j = 0; j < (int)(total + 3u) / 4; ++j) {
-            const uint4 v = c4[j];
-            const int jb = 4 * j;
-            a += (v.x > mk || (v.x == mk && jb + 0 < tid)) ? 1 : 0;
-            a += (v.y > mk || (v.y == mk && jb + 1 < tid)) ? 1 : 0;
-            a += (v.z > mk || (v.z == mk && jb + 2 < tid)) ? 1 : 0;
-            a += (v.w > mk || (v.w == mk && jb + 3 < tid)) ? 1 : 0;
-        }
-        sel = a < k ? 1u : 0u;
-        pos = cpos[tid];
+        mc = cand[tid];
+        // pad to an even count with 0 (never above a candidate: keys of
+        // candidates are >= tau and positions are complemented)
+        if (tid == 0 && (total & 1)) cand[total] = 0ull;
     }
-    uint32_t nsel;
-    const uint32_t r = block_exclusive_scan<NT>(sel, w + NW, &nsel);
-    if (sel) out[r] = (int32_t)pos;
-    __syncthreads();
+    group_sync<NT, BAR>();
+    if ((uint32_t)tid < total) {
+        const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(cand);
+        int a = 0;
+#pragma unroll 4
+        for (uint32_t j = 0; j < (total + 1) / 2; ++j) {
+            const ulonglong2 v = c2[j];
+            a += (v.x > mc ? 1 : 0) + (v.y > mc ? 1 : 0);
+        }
+        sel = a < k;
+        flag[tid] = sel ? 1 : 0;
+    }
+    group_sync<NT, BAR>();
+    if (sel) {
+        const uint32_t mp = ~(uint32_t)mc;
+        int r = 0;
+#pragma unroll 4
+        for (uint32_t j = 0; j < total; ++j) r += (flag[j] && ~(uint32_t)cand[j] < mp) ? 1 : 0;
+        out[r] = (int32_t)mp;
+    }
+    group_sync<NT, BAR>();
     return true;
+}
+
+// The same selection with the keys in shared memory (keys[i] for position i).
+template <int NT, int M, int BAR = 0, int FIRST = 0>
+__device__ bool threshold_topk(const uint32_t* keys, int n, int k, int32_t* out, uint32_t* w) {
+    const int m = (n + NT - 1) / NT;
+    const int lo = (threadIdx.x - FIRST) * m;
+    const int mine = max(0, min(m, n - lo));
+    uint32_t key[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) key[i] = i < mine ? keys[lo + i] : 0u;
+    return threshold_topk_regs<NT, M, BAR, FIRST>(key, lo, 1, mine, k, out, w);
 }
 
 // ----------------------------------------------------- per-thread copies --
@@ -555,6 +598,18 @@ __device__ __forceinline__ void cp_async16_zero(void* dst, const void* any_globa
 // One arrival on `bar` once every cp.async this thread issued so far has landed.
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Hold the current phase of `bar` open until every cp.async this thread issued
+// so far has landed (the pending count is raised now and lowered on landing;
+// the phase's own expected arrivals are still needed to complete it).
+__device__ __forceinline__ void cp_async_arrive_hold(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Acquire load of a counter other CTAs publish with a release.
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 // `count` arrivals on `bar` at once.
 __device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {

@@ -1,22 +1,30 @@
 // GSA decode step on the 5th-generation tensor cores (bf16, d = 128).
 //
-// Two launches of one persistent kernel per decode step (one CTA per SM),
-// chained by programmatic dependent launch:
+// One persistent launch per decode step: at most 148 CTAs, one per SM, all
+// resident at once.  A row is one (b, kv-head).  Every CTA runs three stretches:
 //
-//  phase A  (launch 1) Stream-K over the units of all rows, a row being one
-//           (b, kv-head): 128-gist tiles (routing scores; in ALL_GISTS mode
-//           also attention) and 128-token tail tiles (attention).  Each CTA
-//           takes a contiguous range of units; a maximal run of one row's
-//           units is a segment, whose attention state leaves as one partial
-//           (M, L, O).  Each CTA then takes the exact top-k of the gists it
-//           scored, the candidates of the row's selection.
-//  phase B  (launch 2) Each row's unfolded rows (the selected chunks' raw
-//           tokens, and in SELECTED_PAIRS mode the selected gists) are packed
-//           into 128-row tiles, and the tiles are spread over CTAs.  Each CTA
-//           of a row selects the row's top-k from the candidates, gathers its
-//           tiles with every thread's cp.async, attends over them and leaves
-//           one partial; the row's last CTA (atomic ticket) merges all of the
-//           row's partials (log-sum-exp) into out.
+//  keys     Its Stream-K share of the phase-A units, a contiguous range of the
+//           units of all rows (a unit is a 128-gist tile or a 128-token tail
+//           tile of one row).  Only K is read: S = K . Q^T gives each gist's
+//           routing score (summed over the G heads of the group) and the scaled
+//           attention logits, which stay in tensor memory (TMEM).  A maximal
+//           run of one row's units is a segment; its exact per-head maximum M
+//           goes to TMEM too.  The CTA then counts itself done on every row it
+//           met.
+//  unfold   Its phase-B item(s): once every CTA that met the item's row has
+//           counted itself done (a bounded wait on the row's counter), the
+//           row's top-k is taken, the selected chunks' raw tokens (and in
+//           SELECTED_PAIRS mode the selected gists) are gathered by every
+//           thread's cp.async into 128-row tiles and attended with an online
+//           softmax, leaving one partial.  The producer warp has meanwhile
+//           issued the first V tiles of the next stretch, so the SM keeps
+//           streaming while the selection runs.
+//  values   V of the units whose logits the key stretch kept: P = 2^(x - M)
+//           against the segment's exact maximum (nothing is ever rescaled),
+//           O^T += V^T . P^T, one partial (M, L, O) per segment.
+// Every partial is counted on its row's ticket; the row's first unfold CTA
+// waits (bounded) for the full count and merges the partials (log-sum-exp)
+// into out.
 //
 // Method: gist.science explainer (EN), section 2 "Methodology": gist as
 // routing signals, selective unfolding, hybrid attention; Taki-lab slides
@@ -24,12 +32,15 @@
 //
 // Warp roles: warps 0-3 run the softmax (thread t owns key row t of a tile and,
 // for O^T, TMEM lane t = output dimension t); warp 4 issues the loads; warp 5
-// owns TMEM and issues the MMAs.  Per tile:
+// owns TMEM and issues the MMAs.  Shared memory holds a ring of six 32 KiB
+// slots; a key-stretch tile takes one (K), a value-stretch tile one (V), a
+// gathered tile two (K, V).  Per tile:
 //   S   = K_tile . Q^T     M = 128 keys, N = 16 (G heads, rest zero), K = d
 //   O^T += V_tile^T . P^T  M = 128 = d,  N = 16 heads,                K = 128 keys
 // S is double buffered in TMEM, O^T has one accumulator per segment parity,
-// P^T (bf16) and Q are double buffered in shared memory; O^T is rescaled
-// lazily (only when a head's running maximum grows by more than 2^8).
+// P^T (bf16) and Q are double buffered in shared memory.  TMEM columns:
+// S [0, 32), O^T [32, 64), then the logits of the CTA's attended units (G
+// columns each) and the maxima of its attended segments (G columns each).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -44,63 +55,85 @@
 namespace gsa {
 namespace fused {
 
-constexpr int NT = 192;
-constexpr int NS = 3;
+constexpr int NT = 192;                      // streaming warps 0-5: softmax 0-3, loads 4, MMA 5
+constexpr int NU = 128;                      // unfold warps 6-9: selection, row tables, gathers
+constexpr int UFIRST = NT;                   // first unfold thread
+constexpr int NTHR = NT + NU;
+constexpr int BAR_SOFT = 1, BAR_UNF = 2, BAR_PIPE = 3;   // named barriers (0 is the whole block)
+constexpr int NSL = 6;                       // ring slots
 constexpr int D = 128;
 constexpr int TILE = 128;
-constexpr uint32_t KV_BYTES = 32768;         // one tensor of one stage
-constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
+constexpr uint32_t SLOT_BYTES = 32768;       // one 128 x 128 bf16 tensor tile
 constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 16, 0, 0);
 constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, 16, 1, 0);
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kSelStageCap = 12288;   // keys a selection stages in shared memory (keys, result, 2 lists, bitmaps)
+constexpr uint32_t kLogitCol = 64;           // first TMEM column of the kept logits
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t SM_STAGE = 0;
-constexpr uint32_t SM_Q = NS * STAGE_BYTES;          // 2 x 4 KiB: [16 rows][128 B] x 2 K blocks
+constexpr uint32_t SM_Q = NSL * SLOT_BYTES;          // 2 x 4 KiB: [16 rows][128 B] x 2 K blocks
 constexpr uint32_t SM_P = SM_Q + 2 * 4096;           // 2 x 4 KiB: P^T [16 heads][128 keys]
 constexpr uint32_t SM_WMAX = SM_P + 2 * 4096;        // [2][4 warps][16] floats
 constexpr uint32_t SM_LRED = SM_WMAX + 2 * 4 * 16 * 4;
-constexpr uint32_t SM_TOPK = SM_LRED + 4 * 16 * 4;   // block top-k scratch
-constexpr uint32_t SM_MISC = SM_TOPK + 2048;         // finalized-row list
-constexpr uint32_t SM_SCORE = SM_MISC + 1024;        // phase A: this CTA's routing scores
+constexpr uint32_t SM_TOPK = SM_LRED + 4 * 16 * 4;   // selection scratch
+constexpr uint32_t SM_MISC = SM_TOPK + 2048;         // a threshold selection's positions [<= 32]
+constexpr uint32_t SM_SCORE = SM_MISC + 1024;        // key stretch: this CTA's routing scores
 constexpr int kScoreCap = 3072;                      // scores kept in shared memory
-constexpr uint32_t SM_SEL = SM_SCORE;                // phase B: the row's selection [kSelCap]
-constexpr uint32_t SM_ROWTAB = SM_SEL + kSelCap * 4; // phase B: source of each gathered row [kMaxTpc][128]
-// hierarchy, phase B: the level-2 selection at SM_SEL [k2 <= 512], the children
-// tile's score keys [128] and the level-1 selection [k1 <= 128] after it
+constexpr uint32_t SM_SEL = SM_SCORE;                // unfold stretch: the row's selection [kSelCap]
+constexpr uint32_t SM_ROWTAB = SM_SEL + kSelCap * 4; // unfold stretch: source of each gathered row [kMaxTpc][128]
+// hierarchy: the level-2 selection at SM_SEL [k2 <= 512], the children tile's
+// score keys [128], the level-1 selection [k1 <= 128], the children top-k's
+// result [128] and scratch after it
 constexpr uint32_t SM_CKEY = SM_SEL + 512 * 4;
 constexpr uint32_t SM_SEL1 = SM_CKEY + TILE * 4;
-static_assert(SM_SEL1 + TILE * 4 <= SM_ROWTAB, "hierarchy tables overflow the selection buffer");
-static_assert(kSelCap * 4 + kMaxTpc * TILE * 4 <= kScoreCap * 4, "phase-B tables overflow the score buffer");
-constexpr uint32_t SM_UB = SM_SCORE + kScoreCap * 4;  // first unit of every phase-A CTA [kFusedCtas + 1]
+constexpr uint32_t SM_HRES = SM_SEL1 + TILE * 4;
+constexpr uint32_t SM_HSCR = SM_HRES + TILE * 4;
+static_assert(SM_HSCR + 4608 <= SM_ROWTAB, "hierarchy tables overflow the selection buffer");
+static_assert(kSelCap * 4 + kMaxTpc * TILE * 4 <= kScoreCap * 4, "unfold tables overflow the score buffer");
+constexpr uint32_t SM_UB = SM_SCORE + kScoreCap * 4;  // first unit of every CTA [kFusedCtas + 1]
 constexpr uint32_t SM_BAR = SM_UB + 640;
 static_assert((kFusedCtas + 1) * 4 <= 640, "unit table overflow");
 constexpr uint32_t SMEM_BYTES = SM_BAR + 512 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "dynamic shared memory above the per-block limit");
 
 struct Bars {
-    uint64_t full[NS], empty[NS];
+    uint64_t full[NSL], empty[NSL];
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], o_done[2];
     uint64_t q_ready[2];
+    uint64_t gdone;              // a gathered stretch is closed (its row table and children keys are free)
     uint32_t tmem;
 };
 
-// A unit of work: 128 keys of one row.
-struct Unit {
+// A tile of work: 128 keys of one row.
+struct Tile {
     int row;
     int kind;      // 0 gist tile, 1 tail tile, 2 gathered tile (raw chunks [+ gists])
     int t;         // tile index within its kind
+    int u;         // kinds 0/1: the unit's index (its logits block)
     int lt;        // gathered tiles: index into the shared row table
     int nvalid;    // kinds 0/1: leading valid rows
     bool score, attn;
 };
 
-// Phase-A CTA c takes units [ub[c], ub[c + 1]), ub[c] = floor(c * T / grid),
-// a table every CTA builds in shared memory at start.
+// A stretch of one role loop.
+enum : int { RUN_K = 0, RUN_V = 1, RUN_G = 2 };
+struct Run {
+    int kind;
+    int u0, n;     // RUN_K / RUN_V: units [u0, u0 + n); RUN_G: n tiles of `row` from tile t0
+    int row, t0;
+    int seq0;      // slot sequence number: RUN_K unit i at seq0 + i; RUN_G tile i at seq0 + 2i (K), + 1 (V)
+    int npre;      // RUN_K: value tiles issued early; RUN_V: of those, how many; RUN_G: tiles all threads issued
+    int vseq0;     // RUN_K: sequence number of the first early value tile
+    int gap;       // RUN_V: value tile j at seq0 + j (j < npre) or seq0 + gap + j
+    int slot_b;    // RUN_G: the partial slot
+    int score;     // RUN_G: the tile is scored (the hierarchy's children tile)
+};
+
+// CTA c takes units [ub[c], ub[c + 1]), ub[c] = floor(c * T / grid), a table
+// every CTA builds in shared memory at start.
 __device__ __forceinline__ int unit_begin(const int* ub, int c) { return ub[c]; }
-// The phase-A CTA whose range holds unit u (binary search of the table).
+// The CTA whose range holds unit u (binary search of the table).
 __device__ __forceinline__ int cta_of(const int* ub, int grid, int u) {
     int lo = 0, hi = grid - 1;
     while (lo < hi) {
@@ -111,38 +144,43 @@ __device__ __forceinline__ int cta_of(const int* ub, int grid, int u) {
     return lo;
 }
 
-// Unit i of the current pipeline: phase A (row < 0) walks the CTA's unit range
-// starting at u0; phase B walks the gathered tiles of `row` from tile u0.
-__device__ __forceinline__ Unit unit_at(const Params& p, int u0, int row, int i) {
-    Unit x;
-    if (row < 0) {
-        const int u = u0 + i;
-        x.row = (int)(u / p.upr);
-        const int t = (int)(u % p.upr);
-        if (t < p.tg) {
-            x.kind = 0;
-            x.t = t;
-            x.nvalid = min(TILE, p.NA - t * TILE);
-            x.score = p.do_score != 0;
-            x.attn = p.do_attn_gists != 0;
-        } else {
-            x.kind = 1;
-            x.t = t - p.tg;
-            x.nvalid = min(TILE, p.W - x.t * TILE);
-            x.score = false;
-            x.attn = true;
-        }
+__device__ __forceinline__ Tile unit_tile(const Params& p, int u) {
+    Tile x;
+    x.u = u;
+    x.row = u / p.upr;
+    const int t = u - x.row * p.upr;
+    x.lt = 0;
+    if (t < p.tg) {
+        x.kind = 0;
+        x.t = t;
+        x.nvalid = min(TILE, p.NA - t * TILE);
+        x.score = p.do_score != 0;
+        x.attn = p.do_attn_gists != 0;
     } else {
-        x.row = row;
-        x.kind = 2;
-        x.t = u0 + i;
-        x.lt = i;
-        x.nvalid = 0;
-        x.score = p.hier != 0 && x.t == 0;   // the hierarchy's children tile (tile 0) is scored
+        x.kind = 1;
+        x.t = t - p.tg;
+        x.nvalid = min(TILE, p.W - x.t * TILE);
+        x.score = false;
         x.attn = true;
     }
     return x;
 }
+
+__device__ __forceinline__ Tile gathered_tile(int row, int t, int lt, bool score) {
+    Tile x;
+    x.row = row;
+    x.kind = 2;
+    x.t = t;
+    x.u = 0;
+    x.lt = lt;
+    x.nvalid = 0;
+    x.score = score;
+    x.attn = true;
+    return x;
+}
+
+// value tile j of a RUN_V stretch: its slot sequence number
+__device__ __forceinline__ int value_seq(const Run& r, int j) { return j < r.npre ? r.seq0 + j : r.seq0 + r.gap + j; }
 
 // Is key row r of the gathered tile with row-table index lt valid?  (The
 // table marks an empty row with -1.)
@@ -172,67 +210,106 @@ struct Ctx {
     Bars* bars;
     uint32_t tmem;
     int warp, lane;
-    // role counters (each role keeps its own copy; all roles see the same unit sequence)
-    int tiles, segs, atiles;
-    int first_attn;   // MMA role: the next attention tile starts its segment
+    // role counters (each role keeps its own copy; all roles see the same tile sequence)
+    int stiles;    // S products so far (S buffer and its barrier phases)
+    int ptiles;    // P^T tiles so far (P buffer, p_full / o_done phases)
+    int qsegs;     // segments that needed Q (Q buffer, q_ready phases)
+    int osegs;     // segments that accumulate O^T (O buffer)
     // softmax role: running state of the current segment
-    float m_run[16];
-    float l_part[16];
+    float m_run[8];
+    float l_part[8];
     int had_attn, cur_row, cur_slot;
-    int gtiles;     // softmax role: score tiles so far (index into the shared score buffer)
+    int gtiles;    // softmax role: score tiles so far (index into the shared score buffer)
+    int ai, aseg;  // softmax role: attended units / attended segments so far (TMEM columns)
+    uint32_t mcol; // first TMEM column of the segment maxima
 };
 
+// Is slot sequence number `seq` free to fill (its previous use consumed)?
+__device__ __forceinline__ bool slot_free(const Params& p, Bars* b, int seq) {
+    return seq < NSL || mbar_wait(&b->empty[seq % NSL], ((seq / NSL) - 1) & 1, p.err);
+}
+
 // ------------------------------------------------------------ producer --
-// Called by all 32 lanes of the producer warp: lane 0 issues the large boxes
-// of gist / tail tiles; the 8-row boxes of a gathered tile are spread over
-// the lanes (box lane % 16, K for lanes < 16, V above), so their issue runs
-// in parallel.
-__device__ __forceinline__ void produce(const Params& p, Ctx& cx, const Unit& u) {
-    const int gi = cx.tiles;
-    const int stage = gi % NS;
-    cx.tiles = gi + 1;
-    if (gi >= NS && !mbar_wait(&cx.bars->empty[stage], ((gi / NS) - 1) & 1, p.err)) return;
-    uint8_t* ks = cx.base + SM_STAGE + stage * STAGE_BYTES;
-    uint8_t* vs = ks + KV_BYTES;
-    uint64_t* bar = &cx.bars->full[stage];
-    if (u.kind < 2) {
-        if (cx.lane == 0) {
-            const CUtensorMap* mk = u.kind == 0 ? &p.tm_kg : &p.tm_kt;
-            const CUtensorMap* mv = u.kind == 0 ? &p.tm_vg : &p.tm_vt;
-            const int y = u.t * TILE;
-            mbar_arrive_expect_tx(bar, u.attn ? STAGE_BYTES : KV_BYTES);
-            tc::tma_load_3d(ks, mk, 0, y, u.row, bar);
-            tc::tma_load_3d(ks + 16384, mk, 64, y, u.row, bar);
-            if (u.attn) {
-                tc::tma_load_3d(vs, mv, 0, y, u.row, bar);
-                tc::tma_load_3d(vs + 16384, mv, 64, y, u.row, bar);
-            }
+// One TMA tensor (K or V) of unit tile u into slot `seq` (lane 0 of the producer warp).
+__device__ __forceinline__ void load_tensor(const Params& p, Ctx& cx, const Tile& u, int seq, bool v) {
+    const int s = seq % NSL;
+    uint8_t* dst = cx.base + SM_STAGE + s * SLOT_BYTES;
+    uint64_t* bar = &cx.bars->full[s];
+    const CUtensorMap* m = v ? (u.kind == 0 ? &p.tm_vg : &p.tm_vt) : (u.kind == 0 ? &p.tm_kg : &p.tm_kt);
+    const int y = u.t * TILE;
+    mbar_arrive_expect_tx(bar, SLOT_BYTES);
+    tc::tma_load_3d(dst, m, 0, y, u.row, bar);
+    tc::tma_load_3d(dst + 16384, m, 64, y, u.row, bar);
+}
+
+// Gathered tile i of the row table into slots k_seq and k_seq + 1 by the 32
+// lanes of the producer warp; each lane holds both phases open until its
+// copies land, lane 0 then gives the one expected arrival.
+__device__ __forceinline__ void gather_warp(const Params& p, Ctx& cx, int i, int k_seq) {
+    const int sk = k_seq % NSL, sv = (k_seq + 1) % NSL;
+    uint8_t* ks = cx.base + SM_STAGE + sk * SLOT_BYTES;
+    uint8_t* vs = cx.base + SM_STAGE + sv * SLOT_BYTES;
+    const int32_t* tab = reinterpret_cast<const int32_t*>(cx.base + SM_ROWTAB) + i * TILE;
+    for (int q = cx.lane; q < TILE * 16; q += 32) gather_piece(p, ks, vs, tab[q >> 4], q >> 4, q & 15);
+    cp_async_arrive_hold(&cx.bars->full[sk]);
+    cp_async_arrive_hold(&cx.bars->full[sv]);
+    __syncwarp();
+    if (cx.lane == 0) {
+        mbar_arrive(&cx.bars->full[sk]);
+        mbar_arrive(&cx.bars->full[sv]);
+    }
+}
+
+__device__ __forceinline__ void produce_run(const Params& p, Ctx& cx, const Run& r) {
+    if (r.kind == RUN_K) {
+        for (int i = 0; i < r.n; ++i) {
+            const int seq = r.seq0 + i;
+            if (!slot_free(p, cx.bars, seq)) return;
+            if (cx.lane == 0) load_tensor(p, cx, unit_tile(p, r.u0 + i), seq, false);
         }
-    } else if (gi >= NS) {
-        // a gathered tile beyond the ones every thread issued up front: the
-        // producer warp copies it from the shared row table; its 32 lanes'
-        // completions and one arrival for the other NT - 32 threads complete
-        // the stage's phase (the barrier counts NT in phase B)
-        const int32_t* tab = reinterpret_cast<const int32_t*>(cx.base + SM_ROWTAB) + gi * TILE;
-        for (int q = cx.lane; q < TILE * 16; q += 32) gather_piece(p, ks, vs, tab[q >> 4], q >> 4, q & 15);
-        cp_async_arrive_noinc(bar);
-        __syncwarp();
-        if (cx.lane == 0) mbar_arrive_cnt(bar, NT - 32);
+        // the first value tiles of the CTA, ahead of the unfold stretch
+        int j = 0;
+        for (int i = 0; i < r.n && j < r.npre; ++i) {
+            const Tile u = unit_tile(p, r.u0 + i);
+            if (!u.attn) continue;
+            const int seq = r.vseq0 + j;
+            ++j;
+            if (!slot_free(p, cx.bars, seq)) return;
+            if (cx.lane == 0) load_tensor(p, cx, u, seq, true);
+        }
+    } else if (r.kind == RUN_V) {
+        int j = 0;
+        for (int i = 0; i < r.n; ++i) {
+            const Tile u = unit_tile(p, r.u0 + i);
+            if (!u.attn) continue;
+            if (j >= r.npre) {
+                const int seq = value_seq(r, j);
+                if (!slot_free(p, cx.bars, seq)) return;
+                if (cx.lane == 0) load_tensor(p, cx, u, seq, true);
+            }
+            ++j;
+        }
+    } else {
+        // gathered tiles beyond the ones every thread issued up front
+        for (int i = r.npre; i < r.n; ++i) {
+            const int sk = r.seq0 + 2 * i;
+            if (!slot_free(p, cx.bars, sk) || !slot_free(p, cx.bars, sk + 1)) return;
+            gather_warp(p, cx, i, sk);
+        }
     }
 }
 
 // ----------------------------------------------------------------- MMA --
-// The MMA thread runs an event loop over its units: it issues a unit's S
-// product as soon as the unit's data, a free S buffer and (for a new segment)
-// its Q are there, and a pending P.V as soon as its P is there, whichever
-// comes first.  A stage is thus released right after its own P.V, not after
-// the next unit's data has arrived.
+// The MMA thread runs an event loop over a stretch: it issues a tile's S
+// product as soon as the tile's K, a free S buffer and (for a new segment)
+// its Q are there, and a pending P.V as soon as its P and V are there,
+// whichever comes first.
 struct PendingPV {
-    int stage, obuf, first, pj;
+    int vslot, vpar, obuf, first, pj;
 };
 
 __device__ __forceinline__ void issue_pv(Ctx& cx, const PendingPV& r) {
-    const uint32_t vs = cx.sbase + SM_STAGE + r.stage * STAGE_BYTES + KV_BYTES;
+    const uint32_t vs = cx.sbase + SM_STAGE + r.vslot * SLOT_BYTES;
     const uint32_t pt = cx.sbase + SM_P + (r.pj & 1) * 4096;
     const uint32_t dO = cx.tmem + 32 + r.obuf * 16;
 #pragma unroll
@@ -242,60 +319,80 @@ __device__ __forceinline__ void issue_pv(Ctx& cx, const PendingPV& r) {
                      (r.first && kk == 0) ? 0u : 1u);
     }
     tc::commit(&cx.bars->o_done[r.pj & 1]);
-    tc::commit(&cx.bars->empty[r.stage]);
+    tc::commit(&cx.bars->empty[r.vslot]);
 }
 
-__device__ __forceinline__ void mma_loop(const Params& p, Ctx& cx, int u0, int row, int n) {
+__device__ __forceinline__ void mma_run(const Params& p, Ctx& cx, const Run& r) {
     PendingPV ring[4];
     int head = 0, tail = 0;   // pending P.V products [head, tail)
-    int next = 0;             // next unit whose S product is due
+    int i = 0;                // next tile of the stretch
+    int j = 0;                // RUN_V: value tiles so far
     int prev_row = -1;
     uint64_t t_last = global_ns();
-    while (next < n || head != tail) {
+    for (;;) {
+        if (r.kind == RUN_V)
+            while (i < r.n && !unit_tile(p, r.u0 + i).attn) ++i;
+        if (i >= r.n && head == tail) break;
         bool prog = false;
-        if (next < n && tail - head < 4) {
-            const Unit u = unit_at(p, u0, row, next);
+        if (i < r.n && tail - head < 4) {
+            const Tile u = r.kind == RUN_G ? gathered_tile(r.row, r.t0 + i, i, false) : unit_tile(p, r.u0 + i);
             const bool ns = u.row != prev_row;
-            const int gi = cx.tiles, stage = gi % NS, sb = gi & 1;
-            const bool ready = (!ns || mbar_test(&cx.bars->q_ready[cx.segs & 1], (cx.segs >> 1) & 1)) &&
-                               mbar_test(&cx.bars->full[stage], (gi / NS) & 1) &&
-                               (gi < 2 || mbar_test(&cx.bars->s_free[sb], ((gi - 2) >> 1) & 1));
-            if (ready) {
-                tc::fence_after();
-                if (ns) {
-                    cx.segs++;
-                    cx.first_attn = 1;
-                }
-                cx.tiles = gi + 1;
-                if (u.kind == 2) tc::fence_async_smem();   // cp.async (generic proxy) writes -> tensor core reads
-                const uint32_t ks = cx.sbase + SM_STAGE + stage * STAGE_BYTES;
-                const uint32_t qb = cx.sbase + SM_Q + ((cx.segs - 1) & 1) * 4096;
-                const uint32_t dS = cx.tmem + sb * 16;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    const uint32_t qa = (kk >> 2) * 2048 + (kk & 3) * 32;
-                    tc::mma_bf16(dS, tc::sdesc_sw128(ks + ka, 16, 1024), tc::sdesc_sw128(qb + qa, 16, 1024), IDESC_S,
-                                 kk > 0 ? 1u : 0u);
-                }
-                tc::commit(&cx.bars->s_full[sb]);
-                if (!u.attn) tc::commit(&cx.bars->empty[stage]);
-                if (u.attn) {
-                    ring[tail & 3] = PendingPV{stage, (cx.segs - 1) & 1, cx.first_attn, cx.atiles};
-                    ++tail;
-                    cx.first_attn = 0;
-                    cx.atiles++;
-                }
+            if (r.kind == RUN_V) {
+                // the value tile's data is waited for with its P
+                if (ns) cx.osegs++;
+                const int seq = value_seq(r, j);
+                ring[tail & 3] = PendingPV{seq % NSL, (seq / NSL) & 1, (cx.osegs - 1) & 1, ns ? 1 : 0, cx.ptiles};
+                ++tail;
+                cx.ptiles++;
+                ++j;
                 prev_row = u.row;
-                ++next;
+                ++i;
                 prog = true;
+            } else {
+                const int kseq = r.kind == RUN_K ? r.seq0 + i : r.seq0 + 2 * i;
+                const int ks_ = kseq % NSL;
+                const int sb = cx.stiles & 1;
+                const bool ready = (!ns || mbar_test(&cx.bars->q_ready[cx.qsegs & 1], (cx.qsegs >> 1) & 1)) &&
+                                   mbar_test(&cx.bars->full[ks_], (kseq / NSL) & 1) &&
+                                   (cx.stiles < 2 || mbar_test(&cx.bars->s_free[sb], ((cx.stiles - 2) >> 1) & 1));
+                if (ready) {
+                    tc::fence_after();
+                    if (ns) cx.qsegs++;
+                    if (r.kind == RUN_G) tc::fence_async_smem();   // cp.async (generic proxy) writes -> tensor core reads
+                    const uint32_t ks = cx.sbase + SM_STAGE + ks_ * SLOT_BYTES;
+                    const uint32_t qb = cx.sbase + SM_Q + ((cx.qsegs - 1) & 1) * 4096;
+                    const uint32_t dS = cx.tmem + sb * 16;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        const uint32_t qa = (kk >> 2) * 2048 + (kk & 3) * 32;
+                        tc::mma_bf16(dS, tc::sdesc_sw128(ks + ka, 16, 1024), tc::sdesc_sw128(qb + qa, 16, 1024),
+                                     IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    tc::commit(&cx.bars->s_full[sb]);
+                    tc::commit(&cx.bars->empty[ks_]);
+                    cx.stiles++;
+                    if (r.kind == RUN_G) {
+                        if (ns) cx.osegs++;
+                        const int vseq = kseq + 1;
+                        ring[tail & 3] =
+                            PendingPV{vseq % NSL, (vseq / NSL) & 1, (cx.osegs - 1) & 1, ns ? 1 : 0, cx.ptiles};
+                        ++tail;
+                        cx.ptiles++;
+                    }
+                    prev_row = u.row;
+                    ++i;
+                    prog = true;
+                }
             }
         }
         if (head != tail) {
-            const PendingPV& r = ring[head & 3];
-            if (mbar_test(&cx.bars->p_full[r.pj & 1], (r.pj >> 1) & 1)) {
+            const PendingPV& q = ring[head & 3];
+            if (mbar_test(&cx.bars->p_full[q.pj & 1], (q.pj >> 1) & 1) &&
+                mbar_test(&cx.bars->full[q.vslot], q.vpar)) {
                 tc::fence_after();
-                issue_pv(cx, r);
+                if (r.kind == RUN_G) tc::fence_async_smem();
+                issue_pv(cx, q);
                 ++head;
                 prog = true;
             }
@@ -318,14 +415,14 @@ template <int G>
 __device__ __forceinline__ void write_q(const Params& p, Ctx& cx, int row) {
     const int t = threadIdx.x;            // 0..127: head t/16, 16-byte chunk t%16
     const int h = t >> 4, c = t & 15;
-    uint8_t* qb = cx.base + SM_Q + (cx.segs & 1) * 4096;
+    uint8_t* qb = cx.base + SM_Q + (cx.qsegs & 1) * 4096;
     if (h < G) {
         const uint4 v = *reinterpret_cast<const uint4*>(p.q + ((size_t)row * G + h) * D + c * 8);
         *reinterpret_cast<uint4*>(qb + (c >> 3) * 2048 + h * 128 + (((c & 7) ^ (h & 7)) << 4)) = v;
     }
     tc::fence_async_smem();
-    mbar_arrive(&cx.bars->q_ready[cx.segs & 1]);
-    cx.segs++;
+    mbar_arrive(&cx.bars->q_ready[cx.qsegs & 1]);
+    cx.qsegs++;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -334,14 +431,14 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Close the current segment (its O^T accumulator is `obuf`): write its
-// partial (M, L, O) to slot cur_slot of cur_row.
+// Close the current attention segment (its O^T accumulator is `obuf`): write
+// its partial (M, L, O) to slot cur_slot of cur_row.
 template <int G>
 __device__ __forceinline__ void finalize_segment(const Params& p, Ctx& cx, uint32_t obuf) {
     const int t = threadIdx.x;
     float O[G];
     if (cx.had_attn) {
-        const int pj = cx.atiles - 1;
+        const int pj = cx.ptiles - 1;
         mbar_wait(&cx.bars->o_done[pj & 1], (pj >> 1) & 1, p.err);
         tc::fence_after();
         uint32_t r[G];
@@ -359,7 +456,7 @@ __device__ __forceinline__ void finalize_segment(const Params& p, Ctx& cx, uint3
         const float s = warp_sum(cx.l_part[h]);
         if (cx.lane == 0) lred[cx.warp * 16 + h] = s;
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    group_sync<128, BAR_SOFT>();
     const size_t slot = (size_t)cx.cur_row * p.slot_stride + cx.cur_slot;
     float* part = p.part + slot * G * D;
 #pragma unroll
@@ -373,108 +470,85 @@ __device__ __forceinline__ void finalize_segment(const Params& p, Ctx& cx, uint3
         p.ml[(slot * G + t) * 4 + 0] = m;   // 16 bytes per head: (m, l, -, -)
         p.ml[(slot * G + t) * 4 + 1] = L;
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    group_sync<128, BAR_SOFT>();
 }
 
+// Close the current key-stretch segment: its exact per-head maximum of the
+// scaled logits goes to the partial's m; a segment without attention (gists
+// scored only) leaves its whole, empty partial here.
 template <int G>
-__device__ __forceinline__ void softmax_tile(const Params& p, Ctx& cx, const Unit& u, bool new_seg, int slot) {
+__device__ __forceinline__ void key_close(const Params& p, Ctx& cx) {
+    const int t = threadIdx.x;
+    float* wmax = reinterpret_cast<float*>(cx.base + SM_WMAX);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float m;
+        asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(cx.m_run[h]));
+        if (cx.lane == 0) wmax[cx.warp * 16 + h] = m;
+    }
+    group_sync<128, BAR_SOFT>();
+    if (cx.had_attn) {
+        // every lane keeps the maxima of the segment in its TMEM lane
+        uint32_t mr[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+            mr[h] = __float_as_uint(fmaxf(fmaxf(wmax[h], wmax[16 + h]), fmaxf(wmax[32 + h], wmax[48 + h])));
+        tc::stn<G>(cx.tmem + ((uint32_t)(cx.warp * 32) << 16) + cx.mcol + cx.aseg * G, mr);
+        cx.aseg++;
+    } else {
+        // scored only: the segment's partial is empty
+        const size_t slot = (size_t)cx.cur_row * p.slot_stride + cx.cur_slot;
+        if (t < G) {
+            p.ml[(slot * G + t) * 4 + 0] = -INFINITY;
+            p.ml[(slot * G + t) * 4 + 1] = 0.f;
+        }
+        float* part = p.part + slot * G * D;
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h * D + t] = 0.f;
+    }
+    group_sync<128, BAR_SOFT>();
+}
+
+// Key stretch, one unit: routing score and scaled logits of key row t.
+template <int G>
+__device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u, bool new_seg, int slot) {
     const int t = threadIdx.x;
     if (new_seg) {
-        // publish the new segment's Q first: the MMA thread issues the pending
-        // P.V of the closing segment only after the S of this tile
-        const uint32_t prev_obuf = (cx.segs - 1) & 1;
         write_q<G>(p, cx, u.row);
-        if (cx.cur_row >= 0) finalize_segment<G>(p, cx, prev_obuf);
+        if (cx.cur_row >= 0) key_close<G>(p, cx);
         cx.cur_row = u.row;
         cx.cur_slot = slot;
         cx.had_attn = 0;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            cx.m_run[h] = -INFINITY;
-            cx.l_part[h] = 0.f;
-        }
+        for (int h = 0; h < G; ++h) cx.m_run[h] = -INFINITY;
     }
-    const int gi = cx.tiles;
-    const int sb = gi & 1;
-    cx.tiles = gi + 1;
-    if (!mbar_wait(&cx.bars->s_full[sb], (gi >> 1) & 1, p.err)) return;
+    const int sb = cx.stiles & 1;
+    const bool ok = mbar_wait(&cx.bars->s_full[sb], (cx.stiles >> 1) & 1, p.err);
+    cx.stiles++;
+    if (!ok) return;
     tc::fence_after();
     uint32_t r[G];
-    const uint32_t lane_off = (uint32_t)(cx.warp * 32) << 16;
-    tc::ldn<G>(cx.tmem + sb * 16 + lane_off, r);
+    tc::ldn<G>(cx.tmem + sb * 16 + ((uint32_t)(cx.warp * 32) << 16), r);
     tc::wait_ld();
     tc::fence_before();
     mbar_arrive(&cx.bars->s_free[sb]);
-    const bool valid = u.kind < 2 ? (t < u.nvalid) : gathered_valid(cx.base, u.lt, t);
-    float score = 0.f;
-    if (u.score) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) score += __uint_as_float(r[h]);
-    }
+    const bool valid = t < u.nvalid;
     if (u.attn) {
-        const int pj = cx.atiles;
-        const int pb = pj & 1;
-        float* wmax = reinterpret_cast<float*>(cx.base + SM_WMAX) + pb * 64;
-        float x[G];
+        uint32_t xr[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            x[h] = valid ? __uint_as_float(r[h]) * p.c2 : -INFINITY;
-            float m;
-            asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(x[h]));
-            if (cx.lane == 0) wmax[cx.warp * 16 + h] = m;
+            const float x = valid ? __uint_as_float(r[h]) * p.c2 : -INFINITY;
+            xr[h] = __float_as_uint(x);
+            cx.m_run[h] = fmaxf(cx.m_run[h], x);
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        float alpha[G];
-        bool need = false;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            alpha[h] = 1.f;
-            const float mt = fmaxf(fmaxf(wmax[h], wmax[16 + h]), fmaxf(wmax[32 + h], wmax[48 + h]));
-            if (mt > -INFINITY) {
-                if (cx.m_run[h] == -INFINITY) {
-                    cx.m_run[h] = mt;   // nothing accumulated yet for this head
-                } else if (mt > cx.m_run[h] + kRescaleLog2) {
-                    alpha[h] = exp2f(cx.m_run[h] - mt);
-                    cx.m_run[h] = mt;
-                    need = true;
-                }
-            }
-        }
-        if (need && cx.had_attn) {
-            // O^T holds the P.V of this segment's earlier tiles: wait for the last, rescale columns
-            mbar_wait(&cx.bars->o_done[(pj - 1) & 1], ((pj - 1) >> 1) & 1, p.err);
-            tc::fence_after();
-            uint32_t o[G];
-            const uint32_t ta = cx.tmem + 32 + ((cx.segs - 1) & 1) * 16 + lane_off;
-            tc::ldn<G>(ta, o);
-            tc::wait_ld();
-#pragma unroll
-            for (int h = 0; h < G; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-            tc::stn<G>(ta, o);
-            tc::wait_st();
-        }
-        // P^T buffer pb was last read by the P.V of attention tile pj-2
-        if (pj >= 2) mbar_wait(&cx.bars->o_done[pb], ((pj - 2) >> 1) & 1, p.err);
-        uint8_t* pt = cx.base + SM_P + pb * 4096;
-        const int kb = t >> 6, c16 = (t & 63) >> 3, e = t & 7;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float pv = (x[h] == -INFINITY) ? 0.f : exp2f(x[h] - cx.m_run[h]);
-            cx.l_part[h] = cx.l_part[h] * alpha[h] + pv;
-            *reinterpret_cast<uint16_t*>(pt + kb * 2048 + h * 128 + ((c16 ^ (h & 7)) << 4) + e * 2) =
-                f32_to_bf16_rne(pv);
-        }
-        tc::fence_async_smem();
-        tc::fence_before();
-        mbar_arrive(&cx.bars->p_full[pb]);
-        cx.atiles = pj + 1;
+        tc::stn<G>(cx.tmem + ((uint32_t)(cx.warp * 32) << 16) + kLogitCol + cx.ai * G, xr);
+        cx.ai++;
         cx.had_attn = 1;
     }
-    // the routing score leaves after the tile is handed to the tensor core
-    if (u.score && u.kind == 2) {
-        // hierarchy: the level-1 scores of the children tile, as keys for the k1 selection
-        reinterpret_cast<uint32_t*>(cx.base + SM_CKEY)[t] = valid ? order_key(score) : 0u;
-    } else if (u.score) {
+    if (u.score) {
+        float score = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) score += __uint_as_float(r[h]);
         if (valid) {
             p.scores[(size_t)u.row * p.NA + u.t * TILE + t] = score;
             if (cx.gtiles < kScoreCap / TILE)
@@ -484,69 +558,271 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Ctx& cx, const Uni
     }
 }
 
-// Run the three roles over n units (phase A: row < 0, from unit u0; phase B:
-// the gathered tiles of `row` from tile u0).  A new segment starts where the
-// row changes; its partial goes to slot c - first CTA of the row (phase A) or
-// to slot `slot_b` (phase B).  Ends with every segment written out.
+// Value stretch, one unit: P^T = 2^(x - M) from the kept logits x (this
+// thread's key row) and the segment's exact maximum M.
 template <int G>
-__device__ __forceinline__ void run_pipeline(const Params& p, Ctx& cx, int u0, int row, int n,
-                                             int slot_b) {
-    if (cx.warp == 4) {
-        for (int i = 0; i < n; ++i) produce(p, cx, unit_at(p, u0, row, i));
-    } else if (cx.warp == 5) {
-        if (cx.lane == 0) mma_loop(p, cx, u0, row, n);
-    } else {
+__device__ __forceinline__ void value_tile(const Params& p, Ctx& cx, const Tile& u, bool new_seg, int slot,
+                                           const float (&x)[G], const float (&M)[G]) {
+    const int t = threadIdx.x;
+    if (new_seg) {
+        if (cx.cur_row >= 0) finalize_segment<G>(p, cx, (cx.osegs - 1) & 1);
+        cx.osegs++;
+        cx.cur_row = u.row;
+        cx.cur_slot = slot;
+        cx.had_attn = 1;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            cx.m_run[h] = M[h];
+            cx.l_part[h] = 0.f;
+        }
+    }
+    const int pj = cx.ptiles, pb = pj & 1;
+    // P^T buffer pb was last read by the P.V of tile pj - 2
+    if (pj >= 2) mbar_wait(&cx.bars->o_done[pb], ((pj - 2) >> 1) & 1, p.err);
+    uint8_t* pt = cx.base + SM_P + pb * 4096;
+    const int kb = t >> 6, c16 = (t & 63) >> 3, e = t & 7;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const float pv = (x[h] == -INFINITY || cx.m_run[h] == -INFINITY) ? 0.f : exp2f(x[h] - cx.m_run[h]);
+        cx.l_part[h] += pv;
+        *reinterpret_cast<uint16_t*>(pt + kb * 2048 + h * 128 + ((c16 ^ (h & 7)) << 4) + e * 2) = f32_to_bf16_rne(pv);
+    }
+    tc::fence_async_smem();
+    tc::fence_before();
+    mbar_arrive(&cx.bars->p_full[pb]);
+    cx.ptiles = pj + 1;
+}
+
+// Unfold stretch, one gathered tile: online softmax (the maximum is not
+// known ahead), O^T rescaled lazily when a head's maximum grows by more
+// than 2^8.
+template <int G>
+__device__ __forceinline__ void gathered_softmax(const Params& p, Ctx& cx, const Tile& u, bool new_seg, int slot) {
+    const int t = threadIdx.x;
+    if (new_seg) {
+        write_q<G>(p, cx, u.row);
+        if (cx.cur_row >= 0) finalize_segment<G>(p, cx, (cx.osegs - 1) & 1);
+        cx.osegs++;
+        cx.cur_row = u.row;
+        cx.cur_slot = slot;
+        cx.had_attn = 0;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            cx.m_run[h] = -INFINITY;
+            cx.l_part[h] = 0.f;
+        }
+    }
+    const int sb = cx.stiles & 1;
+    const bool ok = mbar_wait(&cx.bars->s_full[sb], (cx.stiles >> 1) & 1, p.err);
+    cx.stiles++;
+    if (!ok) return;
+    tc::fence_after();
+    uint32_t r[G];
+    const uint32_t lane_off = (uint32_t)(cx.warp * 32) << 16;
+    tc::ldn<G>(cx.tmem + sb * 16 + lane_off, r);
+    tc::wait_ld();
+    tc::fence_before();
+    mbar_arrive(&cx.bars->s_free[sb]);
+    const bool valid = gathered_valid(cx.base, u.lt, t);
+    const int pj = cx.ptiles;
+    const int pb = pj & 1;
+    float* wmax = reinterpret_cast<float*>(cx.base + SM_WMAX) + pb * 64;
+    float x[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        x[h] = valid ? __uint_as_float(r[h]) * p.c2 : -INFINITY;
+        float m;
+        asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(x[h]));
+        if (cx.lane == 0) wmax[cx.warp * 16 + h] = m;
+    }
+    group_sync<128, BAR_SOFT>();
+    float alpha[G];
+    bool need = false;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        alpha[h] = 1.f;
+        const float mt = fmaxf(fmaxf(wmax[h], wmax[16 + h]), fmaxf(wmax[32 + h], wmax[48 + h]));
+        if (mt > -INFINITY) {
+            if (cx.m_run[h] == -INFINITY) {
+                cx.m_run[h] = mt;   // nothing accumulated yet for this head
+            } else if (mt > cx.m_run[h] + kRescaleLog2) {
+                alpha[h] = exp2f(cx.m_run[h] - mt);
+                cx.m_run[h] = mt;
+                need = true;
+            }
+        }
+    }
+    if (need && cx.had_attn) {
+        // O^T holds the P.V of this segment's earlier tiles: wait for the last, rescale columns
+        mbar_wait(&cx.bars->o_done[(pj - 1) & 1], ((pj - 1) >> 1) & 1, p.err);
+        tc::fence_after();
+        uint32_t o[G];
+        const uint32_t ta = cx.tmem + 32 + ((cx.osegs - 1) & 1) * 16 + lane_off;
+        tc::ldn<G>(ta, o);
+        tc::wait_ld();
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+        tc::stn<G>(ta, o);
+        tc::wait_st();
+    }
+    if (pj >= 2) mbar_wait(&cx.bars->o_done[pb], ((pj - 2) >> 1) & 1, p.err);
+    uint8_t* pt = cx.base + SM_P + pb * 4096;
+    const int kb = t >> 6, c16 = (t & 63) >> 3, e = t & 7;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const float pv = (x[h] == -INFINITY) ? 0.f : exp2f(x[h] - cx.m_run[h]);
+        cx.l_part[h] = cx.l_part[h] * alpha[h] + pv;
+        *reinterpret_cast<uint16_t*>(pt + kb * 2048 + h * 128 + ((c16 ^ (h & 7)) << 4) + e * 2) = f32_to_bf16_rne(pv);
+    }
+    tc::fence_async_smem();
+    tc::fence_before();
+    mbar_arrive(&cx.bars->p_full[pb]);
+    cx.ptiles = pj + 1;
+    cx.had_attn = 1;
+    if (u.score) {
+        // hierarchy: the level-1 scores of the children tile, as keys for the k1 selection
+        float score = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) score += __uint_as_float(r[h]);
+        reinterpret_cast<uint32_t*>(cx.base + SM_CKEY)[t] = valid ? order_key(score) : 0u;
+    }
+}
+
+template <int G>
+__device__ __forceinline__ void softmax_run(const Params& p, Ctx& cx, const Run& r) {
+    const int* ub = reinterpret_cast<const int*>(cx.base + SM_UB);
+    const int c = blockIdx.x;
+    auto seg_slot = [&](int row) { return c - cta_of(ub, p.grid, row * p.upr); };
+    if (r.kind == RUN_K) {
         int prev_row = -1;
-        for (int i = 0; i < n; ++i) {
-            const Unit u = unit_at(p, u0, row, i);
+        for (int i = 0; i < r.n; ++i) {
+            const Tile u = unit_tile(p, r.u0 + i);
             const bool ns = u.row != prev_row;
-            const int slot =
-                row >= 0 ? slot_b
-                         : (int)blockIdx.x - cta_of(reinterpret_cast<const int*>(cx.base + SM_UB), p.grid,
-                                                    u.row * p.upr);
-            softmax_tile<G>(p, cx, u, ns, slot);
+            key_tile<G>(p, cx, u, ns, ns ? seg_slot(u.row) : cx.cur_slot);
             prev_row = u.row;
         }
-        if (cx.cur_row >= 0) finalize_segment<G>(p, cx, (cx.segs - 1) & 1);
-        cx.cur_row = -1;
+        if (cx.cur_row >= 0) key_close<G>(p, cx);
+        tc::wait_st();   // the kept logits and maxima are in TMEM before the value stretch reads them
+    } else if (r.kind == RUN_V) {
+        // the logits of value tile j and the maxima of attended segment s were
+        // kept in this thread's TMEM lane by the key stretch
+        const uint32_t lane_off = (uint32_t)(cx.warp * 32) << 16;
+        int prev_row = -1, j = 0, sg = 0;
+        float M[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) M[h] = -INFINITY;
+        for (int i = 0; i < r.n; ++i) {
+            const Tile u = unit_tile(p, r.u0 + i);
+            if (!u.attn) continue;
+            const bool ns = u.row != prev_row;
+            uint32_t xr[G], mr[G];
+            tc::ldn<G>(cx.tmem + lane_off + kLogitCol + j * G, xr);
+            if (ns) tc::ldn<G>(cx.tmem + lane_off + cx.mcol + sg * G, mr);
+            tc::wait_ld();
+            float x[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                x[h] = __uint_as_float(xr[h]);
+                if (ns) M[h] = __uint_as_float(mr[h]);
+            }
+            value_tile<G>(p, cx, u, ns, ns ? seg_slot(u.row) : cx.cur_slot, x, M);
+            sg += ns ? 1 : 0;
+            prev_row = u.row;
+            ++j;
+        }
+        if (j > 0) finalize_segment<G>(p, cx, (cx.osegs - 1) & 1);
+    } else {
+        for (int i = 0; i < r.n; ++i)
+            gathered_softmax<G>(p, cx, gathered_tile(r.row, r.t0 + i, i, r.score != 0), i == 0, r.slot_b);
+        if (r.n > 0) finalize_segment<G>(p, cx, (cx.osegs - 1) & 1);
+        mbar_arrive(&cx.bars->gdone);   // the row table (and the children keys) may be rewritten
     }
-    __syncthreads();
+    cx.cur_row = -1;
 }
 
-// Top-k of n keys in shared memory into res[0..min(k, n)) (ascending
-// positions).  One out-of-line copy serves both phases, so the code that
-// phase A runs is the code phase B finds in the instruction cache.
-__device__ __noinline__ void select_staged(const uint32_t* keys, int n, int k, int32_t* res, uint32_t* scratch) {
+// Run the three roles over one stretch.  Ends with the streaming warps
+// synchronised and every segment of the stretch closed.
+template <int G>
+__device__ __forceinline__ void run_pipeline(const Params& p, Ctx& cx, const Run& r) {
+    if (cx.warp == 4) {
+        produce_run(p, cx, r);
+    } else if (cx.warp == 5) {
+        if (cx.lane == 0) mma_run(p, cx, r);
+    } else {
+        softmax_run<G>(p, cx, r);
+    }
+    group_sync<NT, BAR_PIPE>();
+}
+
+// ----------------------------------------------------------- selection --
+// Everything from here to the merge runs on the unfold warps (threads
+// [NT, NT + NU), named barrier BAR_UNF), beside the streaming warps.
+
+__device__ __forceinline__ int utid() { return (int)threadIdx.x - UFIRST; }
+__device__ __forceinline__ void usync() { group_sync<NU, BAR_UNF>(); }
+
+// Where a selection reads its keys.
+enum : int { SRC_GSCORE = 0, SRC_SSCORE = 1, SRC_GKEY = 2, SRC_SKEY = 3 };
+
+__device__ __forceinline__ uint32_t load_key_bits(const void* src, int kind, int i) {
+    switch (kind) {
+        case SRC_GSCORE: return __float_as_uint(__ldcg(static_cast<const float*>(src) + i));
+        case SRC_SSCORE: return __float_as_uint(static_cast<const float*>(src)[i]);
+        case SRC_GKEY: return __ldcg(static_cast<const uint32_t*>(src) + i);
+        default: return static_cast<const uint32_t*>(src)[i];
+    }
+}
+// scores are mapped to orderable keys; keys pass through
+__device__ __forceinline__ uint32_t key_of_bits(uint32_t bits, int kind) {
+    return (kind == SRC_GSCORE || kind == SRC_SSCORE) ? order_key(__uint_as_float(bits)) : bits;
+}
+
+// Thread t takes positions t, t + NU, t + 2 NU, ...: every warp-wide load is
+// one contiguous line.
+template <int U>
+__device__ __forceinline__ bool threshold_u(const void* src, int kind, int n, int k, int32_t* res, uint32_t* w) {
+    const int lo = utid();
+    const int mine = lo < n ? (n - lo + NU - 1) / NU : 0;
+    uint32_t key[U];
+#pragma unroll
+    for (int i = 0; i < U; ++i) key[i] = i < mine ? load_key_bits(src, kind, lo + i * NU) : 0u;   // all loads first
+#pragma unroll
+    for (int i = 0; i < U; ++i) key[i] = i < mine ? key_of_bits(key[i], kind) : 0u;
+    return threshold_topk_regs<NU, U, BAR_UNF, UFIRST>(key, lo, NU, mine, k, res, w);
+}
+
+// Exact top-k of n keys (read from `src` as `kind` says), ties to the lower
+// position, the selected positions in ascending order: into res[0..k), or,
+// when `ck` is given, as candidates (ck[r] = key, ci[r] = pos0 + pos).  k <= 32
+// and n <= 32 NU: the threshold selection with every thread's block of keys in
+// registers; otherwise, or when equal keys flood the bound, the radix select
+// reading the keys where they are.  Neither res nor the scratch may overlap
+// the keys.  Every caller goes through this one body (the unfold path runs
+// once per launch, cold, so its code is kept small).
+__device__ __forceinline__ void unfold_topk(const void* src, int kind, int n, int k, int32_t* res, uint32_t* w,
+                                            int32_t* tmp, uint32_t* ck, int32_t* ci, int pos0) {
+    auto emit = [&](int r, int pos) {
+        if (ck != nullptr) {
+            ck[r] = key_of_bits(load_key_bits(src, kind, pos), kind);
+            ci[r] = pos0 + pos;
+        } else {
+            res[r] = pos;
+        }
+    };
     if (k >= n) {
-        for (int i = threadIdx.x; i < n; i += NT) res[i] = i;
+        for (int i = utid(); i < n; i += NU) emit(i, i);
     } else {
         bool done = false;
-        if (k <= 32 && n <= NT * 16) done = threshold_topk<NT, 16>(keys, n, k, res, scratch);
-        else if (k <= 32 && n <= NT * 32) done = threshold_topk<NT, 32>(keys, n, k, res, scratch);
-        if (!done) smem_topk<NT>(keys, n, k, res, scratch);
+        if (k <= 32 && n <= 16 * NU) done = threshold_u<16>(src, kind, n, k, tmp, w);
+        else if (k <= 32 && n <= 32 * NU) done = threshold_u<32>(src, kind, n, k, tmp, w);
+        if (done) {
+            for (int r = utid(); r < k; r += NU) emit(r, tmp[r]);
+        } else {
+            block_topk<NU, BAR_UNF, UFIRST>(
+                n, k, [&](int i) { return key_of_bits(load_key_bits(src, kind, i), kind); }, emit, w);
+        }
     }
-    __syncthreads();
-}
-
-// Top-k of n keys staged (by `key_of`) into shared memory; `emit(r, pos)` for
-// the k selected positions in ascending order.  Falls back to a radix
-// select straight from global memory when n exceeds the staging capacity.
-template <class KeyOf, class Emit>
-__device__ __forceinline__ void select_keys(uint8_t* base, int n, int k, KeyOf key_of, Emit emit) {
-    if (n <= kSelStageCap) {
-        uint32_t* keys = reinterpret_cast<uint32_t*>(base + SM_STAGE);
-        int32_t* res = reinterpret_cast<int32_t*>(keys + ((n + 31) & ~31));
-        uint32_t* scratch = reinterpret_cast<uint32_t*>(res + ((min(k, n) + 31) & ~31));
-#pragma unroll 1
-        for (int i = threadIdx.x; i < n; i += NT) keys[i] = key_of(i);
-        __syncthreads();
-        select_staged(keys, n, k, res, scratch);
-#pragma unroll 1
-        for (int r = threadIdx.x; r < min(k, n); r += NT) emit(r, res[r]);
-    } else {
-        block_topk<NT>(n, k, key_of, emit, reinterpret_cast<uint32_t*>(base + SM_TOPK));
-    }
-    __syncthreads();
+    usync();
 }
 
 // Local top-k of this CTA's gists [g0, g1) of `row` (scores in the shared
@@ -558,73 +834,44 @@ __device__ __forceinline__ void local_topk(const Params& p, uint8_t* base, int r
     const float* sg = p.scores + (size_t)row * p.NA + g0;
     uint32_t* ck = p.cand_key + (size_t)row * p.NA + off;
     int32_t* ci = p.cand_idx + (size_t)row * p.NA + off;
-    const uint32_t* keys = reinterpret_cast<const uint32_t*>(base + SM_STAGE);
-    select_keys(
-        base, g1 - g0, p.K, [&](int i) { return order_key(in_smem ? ss[i] : __ldcg(sg + i)); },
-        [&](int r, int pos) {
-            ck[r] = g1 - g0 <= kSelStageCap ? keys[pos] : order_key(__ldcg(sg + pos));
-            ci[r] = g0 + pos;
-        });
+    // the candidates go straight to global memory: nothing is written over
+    // the scores while they are read
+    unfold_topk(in_smem ? (const void*)ss : (const void*)sg, in_smem ? SRC_SSCORE : SRC_GSCORE, g1 - g0, p.K,
+                nullptr, reinterpret_cast<uint32_t*>(base + SM_TOPK), reinterpret_cast<int32_t*>(base + SM_MISC), ck,
+                ci, g0);
 }
 
-// The row's exact top-k from the candidates that every phase-A CTA meeting
-// the row left (n of them), into the shared selection sel[0..k) and, when
-// `publish`, into the row's idx output.
+// The row's exact top-k into the shared selection sel[0..k) and, when
+// `publish`, into the row's idx output: from the candidates that every CTA
+// meeting the row left (n of them), or straight from its routing scores.
 __device__ __forceinline__ void merge_select(const Params& p, uint8_t* base, int row, int n, bool publish) {
-    const uint32_t* ck = p.cand_key + (size_t)row * p.NA;
     const int32_t* ci = p.cand_idx + (size_t)row * p.NA;
     int32_t* out = p.idx + (size_t)row * p.K;
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
-    select_keys(
-        base, n, p.K, [&](int i) { return __ldcg(ck + i); },
-        [&](int r, int pos) {
-            const int32_t j = __ldcg(ci + pos);
-            sel[r] = j;
-            if (publish) out[r] = j;
-        });
-}
-
-// The row's exact top-k straight from its n = N routing scores (small N and
-// k): the scores are staged with all loads of a thread in flight at once.
-template <int U>   // n <= U * NT
-__device__ __forceinline__ void direct_select_u(const Params& p, uint8_t* base, int row, bool publish) {
-    const int n = p.NA, k = p.K;
-    const float* sg = p.scores + (size_t)row * p.NA;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(base + SM_STAGE);
-    int32_t* res = reinterpret_cast<int32_t*>(keys + ((n + 31) & ~31));
-    uint32_t* scratch = reinterpret_cast<uint32_t*>(res + ((min(k, n) + 31) & ~31));
-    float v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int i = threadIdx.x + u * NT;
-        v[u] = i < n ? __ldcg(sg + i) : 0.f;
+    unfold_topk(p.cand_key + (size_t)row * p.NA, SRC_GKEY, n, p.K, sel, reinterpret_cast<uint32_t*>(base + SM_TOPK),
+                reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
+    for (int r = utid(); r < min(p.K, n); r += NU) {
+        const int32_t j = __ldcg(ci + sel[r]);
+        sel[r] = j;
+        if (publish) out[r] = j;
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int i = threadIdx.x + u * NT;
-        if (i < n) keys[i] = order_key(v[u]);
-    }
-    __syncthreads();
-    select_staged(keys, n, k, res, scratch);
-    int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
-    int32_t* out = p.idx + (size_t)row * p.K;
-    for (int r = threadIdx.x; r < min(k, n); r += NT) {
-        sel[r] = res[r];
-        if (publish) out[r] = res[r];
-    }
-    __syncthreads();
+    usync();
 }
 
 __device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, int row, bool publish) {
-    if (p.NA <= 16 * NT) direct_select_u<16>(p, base, row, publish);
-    else direct_select_u<32>(p, base, row, publish);
+    int32_t* out = p.idx + (size_t)row * p.K;
+    int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
+    unfold_topk(p.scores + (size_t)row * p.NA, SRC_GSCORE, p.NA, p.K, sel, reinterpret_cast<uint32_t*>(base + SM_TOPK),
+                reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
+    if (publish)
+        for (int r = utid(); r < min(p.K, p.NA); r += NU) out[r] = sel[r];
 }
 
 // A given selection (gsa_unfold_attn) into sel[0..k); an index outside
 // [0, N) is clamped into range and flagged in the error word.
 __device__ __forceinline__ void load_selection(const Params& p, uint8_t* base, int row) {
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
-    for (int r = threadIdx.x; r < p.K; r += NT) {
+    for (int r = utid(); r < p.K; r += NU) {
         int32_t j = __ldcg(p.idx + (size_t)row * p.K + r);
         if (j < 0 || j >= p.N) {
             atomicOr(p.err, kErrIndex);
@@ -632,18 +879,16 @@ __device__ __forceinline__ void load_selection(const Params& p, uint8_t* base, i
         }
         sel[r] = j;
     }
-    __syncthreads();
+    usync();
 }
 
-// Phase B, before the pipeline: the source of every row of this CTA's
-// gathered tiles [t0, t0 + ntl) into the shared row table, then every thread
-// issues its share of the first min(ntl, NS) tiles' copies (stage i = tile
-// t0 + i) and arrives on each of those stages once its copies have landed.
-__device__ __forceinline__ void gather_prologue(const Params& p, uint8_t* base, Bars* bars, int row, int t0, int ntl) {
+// The source of every row of the gathered tiles [t0, t0 + ntl) of `row` into
+// the shared row table.
+__device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int row, int t0, int ntl) {
     const int32_t* sel = reinterpret_cast<const int32_t*>(base + SM_SEL);
     int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
     const int kc = p.K * p.C;
-    for (int i = threadIdx.x; i < ntl * TILE; i += NT) {
+    for (int i = utid(); i < ntl * TILE; i += NU) {
         const int gr = t0 * TILE + i;
         int32_t e = -1;
         if (gr < kc) {
@@ -654,35 +899,37 @@ __device__ __forceinline__ void gather_prologue(const Params& p, uint8_t* base, 
         }
         tab[i] = e;
     }
-    __syncthreads();
-    const int npre = min(ntl, NS);
-#pragma unroll 1
-    for (int q = threadIdx.x; q < npre * TILE * 16; q += NT) {
-        const int lt = q >> 11, r = (q >> 4) & (TILE - 1);
-        uint8_t* ks = base + SM_STAGE + lt * STAGE_BYTES;
-        gather_piece(p, ks, ks + KV_BYTES, tab[lt * TILE + r], r, q & 15);
+    usync();
+}
+
+// Tile lt of the row table into slots seq, seq + 1 (K, V) once the slots'
+// previous contents are consumed: every unfold thread issues its share and
+// holds both phases open until its copies have landed; one thread then gives
+// the one expected arrival.
+__device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars* bars, int lt, int seq) {
+    slot_free(p, bars, seq);
+    slot_free(p, bars, seq + 1);
+    const int sk = seq % NSL, sv = (seq + 1) % NSL;
+    uint8_t* ks = base + SM_STAGE + sk * SLOT_BYTES;
+    uint8_t* vs = base + SM_STAGE + sv * SLOT_BYTES;
+    const int32_t* tab = reinterpret_cast<const int32_t*>(base + SM_ROWTAB) + lt * TILE;
+#pragma unroll 4
+    for (int q = utid(); q < TILE * 16; q += NU) gather_piece(p, ks, vs, tab[q >> 4], q >> 4, q & 15);
+    cp_async_arrive_hold(&bars->full[sk]);
+    cp_async_arrive_hold(&bars->full[sv]);
+    usync();
+    if (utid() == 0) {
+        mbar_arrive(&bars->full[sk]);
+        mbar_arrive(&bars->full[sv]);
     }
-    for (int lt = 0; lt < npre; ++lt) cp_async_arrive_noinc(&bars->full[lt]);
 }
 
-// Hierarchy, phase B: every thread issues its share of the gathered tile
-// described by row-table entries [0, 128) into `stage`, and arrives on that
-// stage's barrier once its copies have landed.
-__device__ __forceinline__ void gather_issue(const Params& p, uint8_t* base, Bars* bars, int stage) {
-    const int32_t* tab = reinterpret_cast<const int32_t*>(base + SM_ROWTAB);
-    uint8_t* ks = base + SM_STAGE + stage * STAGE_BYTES;
-#pragma unroll 1
-    for (int q = threadIdx.x; q < TILE * 16; q += NT) gather_piece(p, ks, ks + KV_BYTES, tab[q >> 4], q >> 4, q & 15);
-    cp_async_arrive_noinc(&bars->full[stage]);
-}
-
-// Hierarchy, phase B: the row table of the children tile: the level-1 gists
-// of the k2 selected groups, group after group (a short last group leaves
-// empty rows).
+// Hierarchy: the row table of the children tile: the level-1 gists of the k2
+// selected groups, group after group (a short last group leaves empty rows).
 __device__ __forceinline__ void hier_children_table(const Params& p, uint8_t* base, int row) {
     const int32_t* sel2 = reinterpret_cast<const int32_t*>(base + SM_SEL);
     int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
-    for (int r = threadIdx.x; r < TILE; r += NT) {
+    for (int r = utid(); r < TILE; r += NU) {
         int32_t e = -1;
         if (r < p.K * p.group) {
             const int child = sel2[r / p.group] * p.group + r % p.group;
@@ -690,54 +937,73 @@ __device__ __forceinline__ void hier_children_table(const Params& p, uint8_t* ba
         }
         tab[r] = e;
     }
-    __syncthreads();
+    usync();
 }
 
-// Hierarchy, phase B: the exact top-k1 of the children tile's scores (ties to
-// the lower level-1 index: the tile holds the children in ascending order),
+// Hierarchy: the exact top-k1 of the children tile's scores (ties to the
+// lower level-1 index: the tile holds the children in ascending order),
 // published as idx1 and kept in shared memory, then the row table of the
 // raw tokens of those k1 chunks.
 __device__ __forceinline__ void hier_select_children(const Params& p, uint8_t* base, int row) {
     const uint32_t* keys = reinterpret_cast<const uint32_t*>(base + SM_CKEY);
     const int32_t* sel2 = reinterpret_cast<const int32_t*>(base + SM_SEL);
     int32_t* sel1 = reinterpret_cast<int32_t*>(base + SM_SEL1);
-    int32_t* res = reinterpret_cast<int32_t*>(base + SM_STAGE);   // stage 0 is free once its tile is done
-    uint32_t* scratch = reinterpret_cast<uint32_t*>(base + SM_STAGE + 1024);
+    int32_t* res = reinterpret_cast<int32_t*>(base + SM_HRES);
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(base + SM_HSCR);
     const int n = min(TILE, p.K * p.group);
-    select_staged(keys, n, p.K1, res, scratch);
-    for (int r = threadIdx.x; r < p.K1; r += NT) {
+    const int k = p.K1;
+    unfold_topk(keys, SRC_SKEY, n, k, res, scratch, reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
+    for (int r = utid(); r < k; r += NU) {
         const int pos = res[r];
         const int child = sel2[pos / p.group] * p.group + pos % p.group;
         sel1[r] = child;
         p.idx1[(size_t)row * p.K1 + r] = child;
     }
-    __syncthreads();
+    usync();
     int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
-    for (int r = threadIdx.x; r < TILE; r += NT) {
+    for (int r = utid(); r < TILE; r += NU) {
         int32_t e = -1;
-        if (r < p.K1 * p.C) {
+        if (r < k * p.C) {
             const int sl = r / p.C;
             e = (int32_t)(((long long)row * p.N1 + sel1[sl]) * p.C + (r - sl * p.C));
         }
         tab[r] = e;
     }
-    __syncthreads();
+    usync();
 }
 
-// Final log-sum-exp merge of a row: phase-A slots [0, na) and phase-B slots
-// [maxs, maxs + nb).  The partials are brought into shared memory with
-// cp.async in groups (one memory round trip per group).  Per group, warp h
-// finds head h's largest slot maximum M_g and each slot's weight
-// 2^(m_s - M_g) and the weighted sum L_g of the l_s; each output is then a
-// plain weighted sum over the slots (independent products, no dependent
-// rescaling chain), folded into a running (M, L, acc) once per group.
+// Wait (bounded) until counter `ctr` reaches `target`; the writes published
+// before it are then visible to the whole group.
+template <int GN, int GBAR>
+__device__ __forceinline__ void wait_count(const Params& p, const uint32_t* ctr, uint32_t target, bool leader) {
+    if (leader) {
+        const uint64_t t0 = global_ns();
+        while (ld_acquire_u32(ctr) < target) {
+            __nanosleep(100);
+            if (global_ns() - t0 > kWaitLimitNs) {
+                atomicOr(p.err, kErrTimeout);
+                break;
+            }
+        }
+    }
+    group_sync<GN, GBAR>();
+}
+
+// Final log-sum-exp merge of a row: slots [0, na) of the CTAs that met the
+// row and slots [maxs, maxs + nb) of its unfold partials.  The partials are
+// brought into shared memory with cp.async in groups (one memory round trip
+// per group).  Per group, warp h finds head h's largest slot maximum M_g and
+// each slot's weight 2^(m_s - M_g) and the weighted sum L_g of the l_s; each
+// output is then a plain weighted sum over the slots (independent products,
+// no dependent rescaling chain), folded into a running (M, L, acc) once per
+// group.  Leaves the row's ticket and key counter zero for the next call.
 template <int G>
 __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int row, int na, int nb) {
-    constexpr int NW = NT / 32;
+    constexpr int NW = NTHR / 32;
     const int nsl = na + nb;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int PER = (G * D + NT - 1) / NT;          // outputs per thread
-    constexpr int GS = (int)((STAGE_BYTES * NS - 256) / ((G * D + 5 * G) * 4));   // slots per group
+    constexpr int PER = (G * D + NTHR - 1) / NTHR;          // outputs per thread
+    constexpr int GS = (int)((SLOT_BYTES * NSL - 256) / ((G * D + 5 * G) * 4));   // slots per group
     float* so = reinterpret_cast<float*>(base + SM_STAGE);              // [GS][G][D]
     float* sml = so + GS * G * D;                                       // [GS][G][4]: (m, l, -, -)
     float* wgt = sml + GS * G * 4;                                      // [GS][G]
@@ -755,12 +1021,12 @@ __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int ro
         // slot s0 + i of the row lives at slot index sidx(i) of its slot array
         auto sidx = [&](int i) { const int sl = s0 + i; return row * p.slot_stride + (sl < na ? sl : p.maxs + (sl - na)); };
 #pragma unroll 1
-        for (int q = threadIdx.x; q < cnt * (G * D / 4); q += NT) {
+        for (int q = threadIdx.x; q < cnt * (G * D / 4); q += NTHR) {
             const int i = q / (G * D / 4), e4 = q - i * (G * D / 4);
             cp_async16(so + (size_t)i * G * D + e4 * 4, p.part + (size_t)sidx(i) * G * D + e4 * 4);
         }
 #pragma unroll 1
-        for (int q = threadIdx.x; q < cnt * G; q += NT) {
+        for (int q = threadIdx.x; q < cnt * G; q += NTHR) {
             const int i = q / G, h = q - i * G;
             cp_async16(sml + (i * G + h) * 4, p.ml + ((size_t)sidx(i) * G + h) * 4);
         }
@@ -789,7 +1055,7 @@ __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int ro
         __syncthreads();
 #pragma unroll
         for (int q = 0; q < PER; ++q) {
-            const int i = threadIdx.x + q * NT;
+            const int i = threadIdx.x + q * NTHR;
             if (i < G * D) {
                 const int h = i / D;
                 float a4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -815,19 +1081,22 @@ __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int ro
     }
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
-        const int i = threadIdx.x + q * NT;
+        const int i = threadIdx.x + q * NTHR;
         if (i < G * D) {
             const int h = i / D, e = i % D;
             p.out[((size_t)row * G + h) * D + e] = f32_to_bf16_rne(acc[q] / L[q]);
             if (p.lse != nullptr && e == 0) p.lse[(size_t)row * G + h] = (M[q] + log2f(L[q])) * 0.69314718055994531f;
         }
     }
-    if (threadIdx.x == 0) p.cnt[row] = 0;   // leave the ticket zero for the next call
+    if (threadIdx.x == 0) {
+        p.cnt[row] = 0;
+        p.kdone[row] = 0;
+    }
 }
 
 // ---------------------------------------------------------------- kernel --
 template <int G>
-__global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     Ctx cx;
@@ -836,24 +1105,24 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
     cx.bars = reinterpret_cast<Bars*>(cx.base + SM_BAR);
     cx.warp = threadIdx.x >> 5;
     cx.lane = threadIdx.x & 31;
-    cx.tiles = cx.segs = cx.atiles = 0;
+    cx.stiles = cx.ptiles = cx.qsegs = cx.osegs = 0;
     cx.had_attn = 0;
-    cx.first_attn = 1;
     cx.cur_row = -1;
     cx.cur_slot = 0;
     cx.gtiles = 0;
+    cx.ai = cx.aseg = 0;
 
-    // the Q and P^T rows of heads >= G must be zero (K/V stages need no
-    // clearing: TMA zero-fills past a row's end, and a gathered tile zeroes
-    // the V rows it leaves empty)
-    for (uint32_t o = SM_Q + threadIdx.x * 16; o < SM_WMAX; o += NT * 16)
+    // the Q and P^T rows of heads >= G must be zero (slots need no clearing:
+    // TMA zero-fills past a row's end, and a gathered tile zeroes the V rows
+    // it leaves empty)
+    for (uint32_t o = SM_Q + threadIdx.x * 16; o < SM_WMAX; o += NTHR * 16)
         *reinterpret_cast<uint4*>(cx.base + o) = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         Bars* b = cx.bars;
-        for (int i = 0; i < NS; ++i) {
-            // phase A: one arrival with the TMA byte count; phase B: one
-            // cp.async completion arrival per thread
-            mbar_init(&b->full[i], p.phase == 0 ? 1u : (uint32_t)NT);
+        for (int i = 0; i < NSL; ++i) {
+            // one expected arrival per fill: the TMA issuer's (with the byte
+            // count), or the gatherer's after every copier holds the phase
+            mbar_init(&b->full[i], 1);
             mbar_init(&b->empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -863,10 +1132,11 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
             mbar_init(&b->o_done[i], 1);
             mbar_init(&b->q_ready[i], 128);
         }
+        mbar_init(&b->gdone, 128);
         fence_mbar_init();
     }
     if (threadIdx.x == 32 * 4) {
-        // fetch the phase-A tensor maps' descriptors ahead of the first loads
+        // fetch the tensor maps' descriptors ahead of the first loads
         if (p.tg > 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_kg) : "memory");
         if (p.tg > 0 && p.do_attn_gists) asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_vg) : "memory");
         if (p.W > 0) {
@@ -874,12 +1144,11 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
             asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_vt) : "memory");
         }
     }
-    if (p.grid > 0)
-        for (int i = threadIdx.x; i <= p.grid; i += NT)
-            reinterpret_cast<int*>(cx.base + SM_UB)[i] = (int)((long long)i * p.T / p.grid);
+    for (int i = threadIdx.x; i <= p.grid; i += NTHR)
+        reinterpret_cast<int*>(cx.base + SM_UB)[i] = (int)((long long)i * p.T / p.grid);
     tc::fence_async_smem();
     if (cx.warp == 5) {
-        tc::tmem_alloc(&cx.bars->tmem, 64);
+        tc::tmem_alloc(&cx.bars->tmem, (uint32_t)p.tmem_cols);
         tc::tmem_relinquish();
     }
     tc::fence_before();
@@ -890,70 +1159,93 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
     pdl_launch_dependents();
 
     const int c = blockIdx.x;
-    // gists of `row` scored by phase-A CTA cc: [g0, g1)
     const int* ub = reinterpret_cast<const int*>(cx.base + SM_UB);
+    const int u0 = unit_begin(ub, c);
+    const int n1 = unit_begin(ub, c + 1) - u0;
+    // the CTAs whose ranges meet `row` (their count, the first one)
+    auto row_ctas = [&](int row, int& cf) {
+        if (p.T == 0) {
+            cf = 0;
+            return 0;
+        }
+        const int ru0 = row * p.upr;
+        cf = cta_of(ub, p.grid, ru0);
+        return cta_of(ub, p.grid, ru0 + p.upr - 1) - cf + 1;
+    };
+    // gists of `row` scored by CTA cc: [g0, g1)
     auto gists_of = [&](int cc, int row, int& g0, int& g1) {
         const int ru0 = row * p.upr;
         const int a = max(unit_begin(ub, cc), ru0), b = min(unit_begin(ub, cc + 1), ru0 + p.tg);
         g0 = (a - ru0) * TILE;
         g1 = b > a ? min((b - ru0) * TILE, p.NA) : g0;
     };
-    // the pipeline has one call site for both phases: phase B runs the code
-    // that phase A left in this SM's instruction cache
-    int pu0 = 0, prow = -1, pn = 0, pslot = 0;
-    int row = 0, j = 0, na = 0;
-    // the hierarchy's phase B runs two rounds in one CTA per row: the
-    // children tile (scored and attended), then the raw tile of the k1 chunks
-    const int rounds = (p.phase == 1 && p.hier) ? (p.K1 > 0 ? 2 : 1) : 1;
-    for (int rd = 0; rd < rounds; ++rd) {
-        if (p.phase == 0) {
-            pu0 = unit_begin(ub, c);
-            pn = unit_begin(ub, c + 1) - pu0;
-        } else {
-            // phase B: this CTA takes tiles [t0, t0 + ntl) of `row`
-            row = c / p.cb;
-            j = c % p.cb;
-            const int t0 = p.hier ? rd : j * p.tpc;
-            const int ntl = p.hier ? 1 : max(0, min(p.nbt, t0 + p.tpc) - t0);
-            const int ru0 = row * p.upr;
-            const int cf = p.T > 0 ? cta_of(ub, p.grid, ru0) : 0;
-            na = p.T > 0 ? cta_of(ub, p.grid, ru0 + p.upr - 1) - cf + 1 : 0;   // phase-A slots
-            if (rd == 1) {
-                hier_select_children(p, cx.base, row);
-            } else if (ntl > 0) {
-                if (p.do_topk && p.sel_direct) {
-                    direct_select(p, cx.base, row, j == 0);
-                } else if (p.do_topk) {
-                    int n = 0;
-                    for (int cc = cf; cc < cf + na; ++cc) {
-                        int a0, a1;
-                        gists_of(cc, row, a0, a1);
-                        n += min(p.K, max(0, a1 - a0));
-                    }
-                    merge_select(p, cx.base, row, n, j == 0);
-                } else {
-                    load_selection(p, cx.base, row);
-                }
-                if (p.hier) hier_children_table(p, cx.base, row);
-            }
-            if (p.hier) {
-                gather_issue(p, cx.base, cx.bars, rd % NS);
-            } else if (ntl > 0) {
-                gather_prologue(p, cx.base, cx.bars, row, t0, ntl);
-            }
-            pu0 = t0;
-            prow = row;
-            pn = ntl;
-            pslot = p.maxs + (p.hier ? rd : j);
+    const int rounds = p.hier ? (p.K1 > 0 ? 2 : 1) : 1;
+    // gathered tiles of unfold item `it`, round rd: [t0, t0 + ntl) of its row
+    auto item_tiles = [&](int it, int rd, int& t0) {
+        if (p.hier) {
+            t0 = rd;
+            return 1;
         }
-        run_pipeline<G>(p, cx, pu0, prow, pn, pslot);
+        t0 = (it % p.cb) * p.tpc;
+        return max(0, min(p.nbt, t0 + p.tpc) - t0);
+    };
+    int n2 = 0;   // attended units of this CTA (its value tiles)
+    for (int i = 0; i < n1; ++i) n2 += unit_tile(p, u0 + i).attn ? 1 : 0;
+    cx.mcol = kLogitCol + (uint32_t)(n2 * G);
+    const int row_first = n1 > 0 ? u0 / p.upr : 0;
+    const int row_last = n1 > 0 ? (u0 + n1 - 1) / p.upr : -1;
+    // slots: keys [0, n1), values [n1, n1 + n2), then two per gathered tile
+    const int gseq0 = n1 + n2;
+
+    // ------------------------------------------------------ key stretch --
+    if (cx.warp < 6) {
+        Run rk{};
+        rk.kind = RUN_K;
+        rk.u0 = u0;
+        rk.n = n1;
+        rk.seq0 = 0;
+        rk.npre = min(n2, NSL);   // the first value tiles follow the keys without a gap
+        rk.vseq0 = n1;
+        run_pipeline<G>(p, cx, rk);
     }
-    if (p.phase == 0) {
+    __threadfence();
+    __syncthreads();
+
+    if (cx.warp < 6) {
+        // ------------------------------------------------ value stretch --
+        Run rv{};
+        rv.kind = RUN_V;
+        rv.u0 = u0;
+        rv.n = n1;
+        rv.seq0 = n1;
+        rv.npre = min(n2, NSL);
+        rv.gap = 0;
+        run_pipeline<G>(p, cx, rv);
+        // ------------------------------------ gathered tiles, item by item --
+        int gseq = gseq0;
+        for (int it = c; it < p.items; it += p.grid) {
+            for (int rd = 0; rd < rounds; ++rd) {
+                int t0;
+                const int ntl = item_tiles(it, rd, t0);
+                if (ntl <= 0) continue;
+                Run rg{};
+                rg.kind = RUN_G;
+                rg.row = it / p.cb;
+                rg.t0 = t0;
+                rg.n = ntl;
+                rg.seq0 = gseq;
+                rg.npre = ntl;   // every tile is gathered by the unfold warps
+                rg.slot_b = p.maxs + (p.hier ? rd : it % p.cb);
+                rg.score = (p.hier && rd == 0) ? 1 : 0;
+                run_pipeline<G>(p, cx, rg);
+                gseq += 2 * ntl;
+            }
+        }
+    } else {
+        // ----------------------------------------------- unfold warps --
+        const bool lead = utid() == 0;
         if (p.do_topk && !p.sel_direct) {
             // local top-k of every segment, from the scores this CTA kept
-            const int u0 = pu0, u1 = pu0 + pn;
-            const int row_first = u0 / p.upr, row_last = (u1 - 1) / p.upr;
-            int sfirst = 0;   // score-tile offset of the segment in the shared buffer
             int ntiles = 0;
             for (int r = row_first; r <= row_last; ++r) {
                 int a0, a1;
@@ -961,11 +1253,13 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
                 ntiles += (a1 - a0 + TILE - 1) / TILE;
             }
             const bool fits = ntiles <= kScoreCap / TILE;
+            int sfirst = 0;   // score-tile offset of the segment in the shared buffer
             for (int r = row_first; r <= row_last; ++r) {
                 int g0, g1;
                 gists_of(c, r, g0, g1);
                 if (g1 <= g0) continue;
-                const int cf = cta_of(ub, p.grid, r * p.upr);
+                int cf;
+                row_ctas(r, cf);
                 int off = 0;
                 for (int cc = cf; cc < c; ++cc) {
                     int a0, a1;
@@ -975,24 +1269,82 @@ __global__ void __launch_bounds__(NT, 1) fused_decode_kernel(const __grid_consta
                 local_topk(p, cx.base, r, g0, g1, sfirst * TILE, off, fits);
                 sfirst += (g1 - g0 + TILE - 1) / TILE;
             }
-        }
-    } else {
-        // the row's last CTA merges all of its partials
-        int* misc = reinterpret_cast<int*>(cx.base + SM_MISC);
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) misc[0] = atomicAdd(&p.cnt[row], 1u) == (uint32_t)(p.cb - 1) ? 1 : 0;
-        __syncthreads();
-        if (misc[0]) {
             __threadfence();
-            merge_row<G>(p, cx.base, row, na, p.hier ? rounds : (p.nbt > 0 ? p.cb : 0));
+            usync();
         }
+        // scores (and candidates) of every row this CTA met are out
+        if (lead)
+            for (int r = row_first; r <= row_last; ++r) atomicAdd(p.kdone + r, 1u);
+        int gseq = gseq0, runs = 0;
+        for (int it = c; it < p.items; it += p.grid) {
+            const int row = it / p.cb, j = it % p.cb;
+            int cf;
+            const int na = row_ctas(row, cf);
+            if (p.do_topk) wait_count<NU, BAR_UNF>(p, p.kdone + row, (uint32_t)na, lead);
+            for (int rd = 0; rd < rounds; ++rd) {
+                int t0;
+                const int ntl = item_tiles(it, rd, t0);
+                if (ntl <= 0) continue;
+                // the previous gathered stretch is closed: its row table (and
+                // the hierarchy's children keys) are free
+                if (runs > 0) {
+                    if (lead) mbar_wait(&cx.bars->gdone, (runs - 1) & 1, p.err);
+                    usync();
+                }
+                if (rd == 1) {
+                    hier_select_children(p, cx.base, row);
+                } else {
+                    if (p.do_topk && p.sel_direct) {
+                        direct_select(p, cx.base, row, j == 0);
+                    } else if (p.do_topk) {
+                        int n = 0;
+                        for (int cc = cf; cc < cf + na; ++cc) {
+                            int a0, a1;
+                            gists_of(cc, row, a0, a1);
+                            n += min(p.K, max(0, a1 - a0));
+                        }
+                        merge_select(p, cx.base, row, n, j == 0);
+                    } else {
+                        load_selection(p, cx.base, row);
+                    }
+                    if (p.hier) hier_children_table(p, cx.base, row);
+                    else build_table(p, cx.base, row, t0, ntl);
+                }
+                for (int lt = 0; lt < ntl; ++lt) gather_tile(p, cx.base, cx.bars, lt, gseq + 2 * lt);
+                gseq += 2 * ntl;
+                ++runs;
+            }
+        }
+    }
+
+    // ---------------------------------------------------------- tickets --
+    // every partial of this CTA is out: count each on its row's ticket
+    __threadfence();
+    __syncthreads();
+    {
+        const int nA = row_last - row_first + 1;
+        const int nI = c < p.items ? (p.items - 1 - c) / p.grid + 1 : 0;
+        for (int q = threadIdx.x; q < nA + nI; q += NTHR) {
+            const int row = q < nA ? row_first + q : (c + (q - nA) * p.grid) / p.cb;
+            atomicAdd(p.cnt + row, 1u);
+        }
+    }
+    // the first unfold item's CTA of a row merges it once every partial is counted
+    const int nb = p.hier ? rounds : (p.nbt > 0 ? p.cb : 0);
+    for (int it = c; it < p.items; it += p.grid) {
+        if (it % p.cb != 0) continue;
+        const int row = it / p.cb;
+        int cf;
+        const int na = row_ctas(row, cf);
+        wait_count<NTHR, 0>(p, p.cnt + row, (uint32_t)(na + p.cb), threadIdx.x == 0);
+        merge_row<G>(p, cx.base, row, na, nb);
+        __syncthreads();
     }
     tc::fence_before();
     __syncthreads();
     if (cx.warp == 5) {
         tc::fence_after();
-        tc::tmem_dealloc(cx.tmem, 64);
+        tc::tmem_dealloc(cx.tmem, (uint32_t)p.tmem_cols);
     }
 }
 
@@ -1030,18 +1382,28 @@ static bool map3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t len)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The CTAs of one launch wait on one another (a row's unfold item waits for
+// the key stretches of the CTAs that met the row), so all of them must be
+// resident at once: the launch is refused on a device that cannot hold `grid`.
 template <int G>
 static cudaError_t launch_g(const Params& p, int grid, cudaStream_t st) {
-    static bool attr = false;
-    if (!attr) {
+    static int resident = -1;
+    if (resident < 0) {
         cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr = true;
+        int dev = 0, sms = 0, per_sm = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_decode_kernel<G>, NTHR, SMEM_BYTES)) !=
+            cudaSuccess)
+            return e;
+        resident = sms * per_sm;
     }
+    if (grid > resident) return cudaErrorCooperativeLaunchTooLarge;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(NT);
+    cfg.blockDim = dim3(NTHR);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute a[1];
@@ -1052,29 +1414,35 @@ static cudaError_t launch_g(const Params& p, int grid, cudaStream_t st) {
     return cudaLaunchKernelEx(&cfg, fused_decode_kernel<G>, p);
 }
 
+static cudaError_t launch(const Params& p, int G, int grid, cudaStream_t st) {
+    switch (G) {
+        case 1: return launch_g<1>(p, grid, st);
+        case 2: return launch_g<2>(p, grid, st);
+        case 4: return launch_g<4>(p, grid, st);
+        default: return launch_g<8>(p, grid, st);
+    }
+}
+
 }  // namespace fused
 
 bool fused_supported(const gsa_decode_desc& d) {
     // gathered rows are addressed by a 32-bit row number; the selection lives in shared memory
     const long long raw_rows = (long long)d.batch * d.n_kv_heads * d.n_chunks * d.chunk;
-    // phase-A units are counted in 32 bits
+    // units are counted in 32 bits
     const long long units = (long long)d.batch * d.n_kv_heads * ((d.n_chunks + 127) / 128 + (d.tail_len + 127) / 128);
-    return d.dtype == GSA_BF16 && d.head_dim == 128 && d.top_k <= kSelCap && raw_rows < INT32_MAX - 2 &&
-           units < (1LL << 30);
+    if (!(d.dtype == GSA_BF16 && d.head_dim == 128 && d.top_k <= kSelCap && raw_rows < INT32_MAX - 2 &&
+          units < (1LL << 30) && d.n_q_heads % d.n_kv_heads == 0))
+        return false;
+    // the kept logits and maxima of every CTA's range fit tensor memory
+    return make_fused_plan(d).tmem_cols <= 512;
 }
 
-FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given) {
-    FusedPlan f{};
-    const bool pairs = d.mode == GSA_SELECTED_PAIRS;
-    f.rows = d.batch * d.n_kv_heads;
-    f.G = d.n_q_heads / d.n_kv_heads;
-    // with a given selection in SELECTED_PAIRS mode no gist is scored or attended in phase A
-    f.tg = (given && pairs) ? 0 : (d.n_chunks + 127) / 128;
-    f.tt = (d.tail_len + 127) / 128;
-    f.upr = f.tg + f.tt;
-    f.T = f.rows * f.upr;
-    f.grid = std::min(f.T, kFusedCtas);
-    // phase-A slots of a row: the CTAs whose range meets the row
+// Grid and partial slots once the rows' unfold items (cb per row) are known:
+// every unfold item and every unit has a CTA (at most one per SM); the
+// phase-A slots of a row are the CTAs whose range meets it.
+static void place_ctas(FusedPlan& f, int nb_slots) {
+    f.items = f.rows * f.cb;
+    f.grid = std::min(kFusedCtas, std::max(f.T, f.items));
     int maxs = 0;
     if (f.T > 0) {
         for (int r = 0; r < f.rows; ++r) {
@@ -1085,25 +1453,32 @@ FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given) {
         }
     }
     f.maxs = maxs;
-    // small selections are taken in phase B straight from the scores; larger
-    // ones from per-CTA candidates that phase A leaves
-    f.sel_direct = (d.top_k <= 32 && d.n_chunks <= 32 * fused::NT) ? 1 : 0;
-    // phase B: the row's gathered rows packed into 128-row tiles, spread over
-    // as many CTAs per row as fill the GPU (at most kMaxTpc tiles each)
-    f.nrows_g = d.top_k * d.chunk + (pairs ? d.top_k : 0);
-    f.nbt = (f.nrows_g + 127) / 128;
-    if (f.nbt == 0) {
-        f.tpc = 0;
-        f.cb = 1;   // the row's merge still runs
-    } else {
-        const int cpr = std::max(1, kFusedCtas / f.rows);
-        f.tpc = std::min(kMaxTpc, (f.nbt + std::min(cpr, f.nbt) - 1) / std::min(cpr, f.nbt));
-        f.cb = (f.nbt + f.tpc - 1) / f.tpc;
+    f.slot_stride = maxs + nb_slots;
+    // TMEM: S and O^T (64 columns), then per CTA G columns for each attended
+    // unit and each attended segment of its range
+    int need = 64;
+    for (int c = 0; c < f.grid && f.T > 0; ++c) {
+        const long long u0 = (long long)c * f.T / f.grid, u1 = (long long)(c + 1) * f.T / f.grid;
+        int units = 0, segs = 0;
+        long long prev = -1;
+        for (long long u = u0; u < u1; ++u) {
+            const long long row = u / f.upr;
+            const bool attn = (u % f.upr) >= f.tg || f.attn_gists;
+            if (!attn) continue;
+            ++units;
+            if (row != prev) ++segs;
+            prev = row;
+        }
+        need = std::max(need, 64 + (units + segs) * f.G);
     }
-    f.grid_b = f.rows * f.cb;
-    f.slot_stride = maxs + f.cb;
-    const size_t rows = (size_t)f.rows, N = (size_t)d.n_chunks;
-    size_t o = round256(kWsCntOffset + rows * 4);
+    f.tmem_cols = need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : need <= 512 ? 512 : 1024;
+}
+
+// Workspace: tickets and key counters [2][rows], scores, candidates, idx,
+// partials, (m, l) (and the hierarchy's idx1).
+static void layout_ws(FusedPlan& f, size_t N, size_t top_k, size_t k1) {
+    const size_t rows = (size_t)f.rows;
+    size_t o = round256(kWsCntOffset + 2 * rows * 4);
     f.off_scores = o;
     o = round256(o + rows * N * 4);
     f.off_cand_key = o;
@@ -1111,20 +1486,81 @@ FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given) {
     f.off_cand_idx = o;
     o = round256(o + rows * N * 4);
     f.off_idx = o;
-    o = round256(o + rows * (size_t)d.top_k * 4);
+    o = round256(o + rows * top_k * 4);
     f.off_part = o;
     o = round256(o + rows * (size_t)f.slot_stride * f.G * 128 * 4);
     f.off_ml = o;
     o = round256(o + rows * (size_t)f.slot_stride * f.G * 4 * 4);
+    f.off_idx1 = o;
+    o = round256(o + rows * k1 * 4);
     f.total = o;
+}
+
+FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given) {
+    FusedPlan f{};
+    const bool pairs = d.mode == GSA_SELECTED_PAIRS;
+    f.attn_gists = pairs ? 0 : 1;
+    f.rows = d.batch * d.n_kv_heads;
+    f.G = d.n_q_heads / d.n_kv_heads;
+    // with a given selection in SELECTED_PAIRS mode no gist is scored or attended
+    f.tg = (given && pairs) ? 0 : (d.n_chunks + 127) / 128;
+    f.tt = (d.tail_len + 127) / 128;
+    f.upr = f.tg + f.tt;
+    f.T = f.rows * f.upr;
+    // small selections are taken straight from the scores; larger ones from
+    // per-CTA candidates the key stretch leaves
+    f.sel_direct = (d.top_k <= 32 && d.n_chunks <= 32 * fused::NU) ? 1 : 0;
+    // unfold: the row's gathered rows packed into 128-row tiles, spread over
+    // as many CTAs per row as fill the GPU (at most kMaxTpc tiles each)
+    f.nrows_g = d.top_k * d.chunk + (pairs ? d.top_k : 0);
+    f.nbt = (f.nrows_g + 127) / 128;
+    if (f.nbt == 0) {
+        f.tpc = 0;
+        f.cb = 1;   // the row's ticket is still taken
+    } else {
+        const int cpr = std::max(1, kFusedCtas / f.rows);
+        f.tpc = std::min(kMaxTpc, (f.nbt + std::min(cpr, f.nbt) - 1) / std::min(cpr, f.nbt));
+        f.cb = (f.nbt + f.tpc - 1) / f.tpc;
+    }
+    place_ctas(f, f.cb);
+    layout_ws(f, (size_t)d.n_chunks, (size_t)d.top_k, 0);
     return f;
+}
+
+static void fill_common(fused::Params& p, const FusedPlan& f, const gsa_decode_desc& d, uint8_t* w) {
+    p.err = reinterpret_cast<uint32_t*>(w + kWsErrOffset);
+    p.cnt = reinterpret_cast<uint32_t*>(w + kWsCntOffset);
+    p.kdone = p.cnt + f.rows;
+    p.cand_key = reinterpret_cast<uint32_t*>(w + f.off_cand_key);
+    p.cand_idx = reinterpret_cast<int32_t*>(w + f.off_cand_idx);
+    p.part = reinterpret_cast<float*>(w + f.off_part);
+    p.ml = reinterpret_cast<float*>(w + f.off_ml);
+    p.rows = f.rows;
+    p.Hkv = d.n_kv_heads;
+    p.G = f.G;
+    p.C = d.chunk;
+    p.W = d.tail_len;
+    p.tg = f.tg;
+    p.upr = f.upr;
+    p.T = f.T;
+    p.grid = f.grid;
+    p.items = f.items;
+    p.slot_stride = f.slot_stride;
+    p.maxs = f.maxs;
+    p.nbt = f.nbt;
+    p.tpc = f.tpc;
+    p.cb = f.cb;
+    p.sel_direct = f.sel_direct;
+    p.tmem_cols = f.tmem_cols;
+    const double scale = d.scale > 0 ? (double)d.scale : 1.0 / std::sqrt(128.0);
+    p.c2 = (float)(scale * 1.4426950408889634);
 }
 
 gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void* q, const void* kg, const void* vg,
                         const void* kr, const void* vr, const void* kt, const void* vt, const int32_t* idx_given,
                         int32_t* idx_out, float* scores_out, void* out, float* lse, void* ws, cudaStream_t st) {
     using namespace fused;
-    if (f.grid_b <= 0) return GSA_ERR_ARG;
+    if (f.grid <= 0) return GSA_ERR_ARG;
     Params p;
     std::memset(&p, 0, sizeof(p));
     const uint64_t rows = (uint64_t)f.rows, N = (uint64_t)d.n_chunks;
@@ -1133,6 +1569,7 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
               map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
     if (!ok) return GSA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
+    fill_common(p, f, d, w);
     p.q = static_cast<const uint16_t*>(q);
     p.kr = static_cast<const uint8_t*>(kr);
     p.vr = static_cast<const uint8_t*>(vr);
@@ -1140,57 +1577,17 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
     p.vgp = static_cast<const uint8_t*>(vg);
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
-    p.err = reinterpret_cast<uint32_t*>(w + kWsErrOffset);
-    p.cnt = reinterpret_cast<uint32_t*>(w + kWsCntOffset);
     p.scores = scores_out ? scores_out : reinterpret_cast<float*>(w + f.off_scores);
     p.idx = idx_given ? const_cast<int32_t*>(idx_given) : (idx_out ? idx_out : reinterpret_cast<int32_t*>(w + f.off_idx));
-    p.cand_key = reinterpret_cast<uint32_t*>(w + f.off_cand_key);
-    p.cand_idx = reinterpret_cast<int32_t*>(w + f.off_cand_idx);
-    p.part = reinterpret_cast<float*>(w + f.off_part);
-    p.ml = reinterpret_cast<float*>(w + f.off_ml);
-    p.rows = f.rows;
-    p.Hkv = d.n_kv_heads;
-    p.G = f.G;
     p.N = d.n_chunks;
     p.NA = d.n_chunks;
-    p.C = d.chunk;
     p.K = d.top_k;
-    p.W = d.tail_len;
     p.mode = d.mode;
-    p.tg = f.tg;
-    p.upr = f.upr;
-    p.T = f.T;
-    p.grid = f.grid;
-    p.slot_stride = f.slot_stride;
-    p.maxs = f.maxs;
     p.nrows_g = f.nrows_g;
-    p.nbt = f.nbt;
-    p.tpc = f.tpc;
-    p.cb = f.cb;
-    const double scale = d.scale > 0 ? (double)d.scale : 1.0 / std::sqrt(128.0);
-    p.c2 = (float)(scale * 1.4426950408889634);
     p.do_score = idx_given ? 0 : 1;
     p.do_topk = idx_given ? 0 : 1;
     p.do_attn_gists = pairs ? 0 : 1;
-    p.sel_direct = f.sel_direct;
-    auto launch = [&](int grid) {
-        switch (f.G) {
-            case 1: return launch_g<1>(p, grid, st);
-            case 2: return launch_g<2>(p, grid, st);
-            case 4: return launch_g<4>(p, grid, st);
-            default: return launch_g<8>(p, grid, st);
-        }
-    };
-    cudaError_t e = cudaSuccess;
-    if (f.grid > 0) {
-        p.phase = 0;
-        e = launch(f.grid);
-    }
-    if (e == cudaSuccess) {
-        p.phase = 1;
-        e = launch(f.grid_b);
-    }
-    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+    return launch(p, f.G, f.grid, st) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
 // --------------------------------------------------------- hierarchy ----
@@ -1198,32 +1595,27 @@ bool fused_hier_supported(const gsa_hier_desc& h) {
     const gsa_decode_desc& d = h.l1;
     const long long rows = (long long)d.batch * d.n_kv_heads;
     const long long units = rows * ((h.n_l2 + 127) / 128 + (d.tail_len + 127) / 128);
-    return d.dtype == GSA_BF16 && d.head_dim == 128 && (long long)h.top_k2 * h.group <= 128 &&
-           (long long)d.top_k * d.chunk <= 128 && rows * d.n_chunks * d.chunk < INT32_MAX - 2 &&
-           rows * d.n_chunks < INT32_MAX - 2 && units < (1LL << 30);
+    if (!(d.dtype == GSA_BF16 && d.head_dim == 128 && (long long)h.top_k2 * h.group <= 128 &&
+          (long long)d.top_k * d.chunk <= 128 && rows * d.n_chunks * d.chunk < INT32_MAX - 2 &&
+          rows * d.n_chunks < INT32_MAX - 2 && units < (1LL << 30) && d.n_q_heads % d.n_kv_heads == 0))
+        return false;
+    return make_fused_hier_plan(h).tmem_cols <= 512;
 }
 
 FusedPlan make_fused_hier_plan(const gsa_hier_desc& h) {
-    // phase A and the level-2 selection are the flat step over the level-2 gists
+    // the key and value stretches and the level-2 selection are the flat
+    // step over the level-2 gists
     gsa_decode_desc l2 = h.l1;
     l2.n_chunks = h.n_l2;
     l2.top_k = h.top_k2;
     l2.mode = GSA_ALL_GISTS;
     FusedPlan f = make_fused_plan(l2);
-    // phase B: one CTA per row, two partial slots (children tile, raw tile)
+    // unfold: one item per row, two partial slots (children tile, raw tile)
     f.nbt = 2;
     f.tpc = 2;
     f.cb = 1;
-    f.grid_b = f.rows;
-    f.slot_stride = f.maxs + 2;
-    const size_t rows = (size_t)f.rows;
-    size_t o = f.off_part;
-    o = round256(o + rows * (size_t)f.slot_stride * f.G * 128 * 4);
-    f.off_ml = o;
-    o = round256(o + rows * (size_t)f.slot_stride * f.G * 4 * 4);
-    f.off_idx1 = o;
-    o = round256(o + rows * (size_t)h.l1.top_k * 4);
-    f.total = o;
+    place_ctas(f, 2);
+    layout_ws(f, (size_t)h.n_l2, (size_t)h.top_k2, (size_t)h.l1.top_k);
     return f;
 }
 
@@ -1233,7 +1625,7 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
                              void* ws, cudaStream_t st) {
     using namespace fused;
     const gsa_decode_desc& d = h.l1;
-    if (f.grid <= 0 || f.grid_b <= 0) return GSA_ERR_ARG;
+    if (f.grid <= 0) return GSA_ERR_ARG;
     Params p;
     std::memset(&p, 0, sizeof(p));
     const uint64_t rows = (uint64_t)f.rows;
@@ -1241,6 +1633,7 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
               map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
     if (!ok) return GSA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
+    fill_common(p, f, d, w);
     p.q = static_cast<const uint16_t*>(q);
     p.kr = static_cast<const uint8_t*>(kr);
     p.vr = static_cast<const uint8_t*>(vr);
@@ -1248,59 +1641,22 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
     p.vgp = static_cast<const uint8_t*>(v_g1);
     p.out = static_cast<uint16_t*>(out);
     p.lse = nullptr;
-    p.err = reinterpret_cast<uint32_t*>(w + kWsErrOffset);
-    p.cnt = reinterpret_cast<uint32_t*>(w + kWsCntOffset);
     p.scores = reinterpret_cast<float*>(w + f.off_scores);
     p.idx = idx2_out ? idx2_out : reinterpret_cast<int32_t*>(w + f.off_idx);
     p.idx1 = idx1_out ? idx1_out : reinterpret_cast<int32_t*>(w + f.off_idx1);
-    p.cand_key = reinterpret_cast<uint32_t*>(w + f.off_cand_key);
-    p.cand_idx = reinterpret_cast<int32_t*>(w + f.off_cand_idx);
-    p.part = reinterpret_cast<float*>(w + f.off_part);
-    p.ml = reinterpret_cast<float*>(w + f.off_ml);
-    p.rows = f.rows;
-    p.Hkv = d.n_kv_heads;
-    p.G = f.G;
     p.N = h.n_l2;
     p.NA = h.n_l2;
-    p.C = d.chunk;
     p.K = h.top_k2;
-    p.W = d.tail_len;
     p.mode = GSA_ALL_GISTS;
-    p.tg = f.tg;
-    p.upr = f.upr;
-    p.T = f.T;
-    p.grid = f.grid;
-    p.slot_stride = f.slot_stride;
-    p.maxs = f.maxs;
     p.nrows_g = 0;
-    p.nbt = f.nbt;
-    p.tpc = f.tpc;
-    p.cb = f.cb;
-    const double scale = d.scale > 0 ? (double)d.scale : 1.0 / std::sqrt(128.0);
-    p.c2 = (float)(scale * 1.4426950408889634);
     p.do_score = 1;
     p.do_topk = 1;
     p.do_attn_gists = 1;
-    p.sel_direct = f.sel_direct;
     p.hier = 1;
     p.group = h.group;
     p.N1 = d.n_chunks;
     p.K1 = d.top_k;
-    auto launch = [&](int grid) {
-        switch (f.G) {
-            case 1: return launch_g<1>(p, grid, st);
-            case 2: return launch_g<2>(p, grid, st);
-            case 4: return launch_g<4>(p, grid, st);
-            default: return launch_g<8>(p, grid, st);
-        }
-    };
-    p.phase = 0;
-    cudaError_t e = launch(f.grid);
-    if (e == cudaSuccess) {
-        p.phase = 1;
-        e = launch(f.grid_b);
-    }
-    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+    return launch(p, f.G, f.grid, st) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
 }  // namespace gsa

@@ -8,17 +8,20 @@
 
 namespace gsa {
 
-constexpr int kFusedCtas = 148;   // one persistent CTA per B200 SM (work split is fixed by this, not the device)
+constexpr int kFusedCtas = 148;   // at most one persistent CTA per B200 SM (the work split is fixed by this, not the device)
 constexpr int kSelCap = 2048;     // largest top_k of the tensor-core path (selection kept in shared memory)
-constexpr int kMaxTpc = 8;        // largest number of gathered tiles one phase-B CTA takes
+constexpr int kMaxTpc = 8;        // largest number of gathered tiles one unfold item takes
 
 struct FusedPlan {
-    int rows, G, tg, tt, upr, grid;   // phase A: units per row, Stream-K grid
-    int T;                            // phase A: units in all
-    int maxs;                         // phase A: most CTAs meeting one row (its partial slots)
-    int nrows_g, nbt, tpc, cb, grid_b;   // phase B: gathered rows / tiles per row, tiles per CTA, CTAs per row, grid
-    int slot_stride;                  // maxs + cb
-    int sel_direct;                   // phase B selects from the scores (else from phase-A candidates)
+    int rows, G, tg, tt, upr, grid;   // units per row, Stream-K grid (one launch)
+    int T;                            // units in all
+    int maxs;                         // most CTAs meeting one row (its key/value partial slots)
+    int nrows_g, nbt, tpc, cb;        // unfold: gathered rows / tiles per row, tiles per item, items per row
+    int items;                        // unfold items in all (rows * cb)
+    int slot_stride;                  // maxs + unfold partial slots
+    int sel_direct;                   // the selection is taken from the scores (else from per-CTA candidates)
+    int attn_gists;                   // gist tiles are attended (ALL_GISTS)
+    int tmem_cols;                    // TMEM columns a CTA allocates (S, O^T, kept logits and maxima)
     size_t off_scores, off_cand_key, off_cand_idx, off_idx, off_part, off_ml, total;
     size_t off_idx1;                  // hierarchy: level-1 selection (when the caller passes none)
 };
@@ -37,19 +40,20 @@ struct Params {
     float* scores;                 // [rows][N]
     int32_t* idx;                  // [rows][K]: written by the selection, or given
     uint32_t* err;
-    uint32_t* cnt;                 // [rows] phase-B tickets
+    uint32_t* cnt;                 // [rows] tickets: partials written
+    uint32_t* kdone;               // [rows] CTAs whose key stretch over the row is done
     uint32_t* cand_key;            // [rows][N] local top-k candidates (orderable score keys)
     int32_t* cand_idx;             // [rows][N] their gist indices
     float* part;                   // [rows][slot_stride][G][d]
     float* ml;                     // [rows][slot_stride][G][4]: (m, l, unused, unused)
     int rows, Hkv, G, N, NA, C, K, W, mode;
     int tg, upr, grid, slot_stride, maxs;
-    int nrows_g, nbt, tpc, cb;
-    int phase;                     // 0: phase A (launch 1), 1: phase B (launch 2)
-    int T;                         // phase-A units in all
+    int nrows_g, nbt, tpc, cb, items;
+    int T;                         // units in all
+    int tmem_cols;                 // TMEM columns a CTA allocates
     float c2;
     int do_score, do_topk, do_attn_gists, sel_direct;
-    // hierarchy (phase A: level-2 gists; phase B: children tile, then raw tile)
+    // hierarchy (keys/values: level-2 gists; unfold: children tile, then raw tile)
     int hier, group, N1, K1;       // K = k2, N = NA = n_l2; group, level-1 gists, k1
     int32_t* idx1;                 // [rows][k1]
 };
@@ -66,9 +70,9 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
                              void* ws, cudaStream_t st);
 // given: the selection is supplied (gsa_unfold_attn), so nothing is scored.
 FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given = false);
-// Enqueue the fused decode step.  idx_given != null: attend over that
-// selection (no scores, no selection); else select and write idx_out (or the
-// workspace copy) and scores_out (or the workspace copy).
+// Enqueue the fused decode step (one launch).  idx_given != null: attend over
+// that selection (no scores, no selection); else select and write idx_out (or
+// the workspace copy) and scores_out (or the workspace copy).
 gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void* q, const void* kg, const void* vg,
                         const void* kr, const void* vr, const void* kt, const void* vt, const int32_t* idx_given,
                         int32_t* idx_out, float* scores_out, void* out, float* lse, void* ws, cudaStream_t st);

@@ -36,6 +36,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+// Raise the transaction count of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -479,11 +485,11 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
 //     in any order, to a shared list as 64-bit composites (key, ~position): a
 //     larger composite is a larger key, or the same key at a lower position.
 //  3. Each candidate counts the composites above its own; those with fewer
-//     than k above are selected, and each selected one counts the selected
-//     ones at lower positions to find its place in the output.
+//     than k above are selected, the count being the key rank.  The k
+//     selected positions, one per rank, are sorted ascending by one warp.
 // Returns false without writing anything when more than NT keys reach tau
 // (a flood of equal keys): the caller then runs a general selection.
-// Scratch `w` (shared, 16-byte aligned): >= 16 + 2 * NT + 2 + NT / 4 words.
+// Scratch `w` (shared, 16-byte aligned): >= 16 + 2 * NT + 2 + 32 words.
 // All NT threads call it; it ends with the block synchronised.
 template <int NT, int M, int BAR = 0, int FIRST = 0>
 __device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, int mine, int k, int32_t* out,
@@ -531,7 +537,6 @@ __device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, 
     base = __shfl_sync(0xFFFFFFFFu, base, 31);
     uint32_t off = base + incl - c;
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(w + 16);
-    uint8_t* flag = reinterpret_cast<uint8_t*>(w + 16 + 2 * NT + 2);
 #pragma unroll
     for (int i = 0; i < M; ++i)
         if (i < mine && key[i] >= tau) {
@@ -543,7 +548,7 @@ __device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, 
     const uint32_t total = w[NW];
     if (total > (uint32_t)NT) return false;       // the same on every thread
     unsigned long long mc = 0ull;
-    bool sel = false;
+    uint32_t* selpos = reinterpret_cast<uint32_t*>(w + 16 + 2 * NT + 2);   // [k]: position of key rank r
     if ((uint32_t)tid < total) {
         mc = cand[tid];
         // pad to an even count with 0 (never above a candidate: keys of
@@ -559,16 +564,25 @@ __device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, 
             const ulonglong2 v = c2[j];
             a += (v.x > mc ? 1 : 0) + (v.y > mc ? 1 : 0);
         }
-        sel = a < k;
-        flag[tid] = sel ? 1 : 0;
+        if (a < k) selpos[a] = ~(uint32_t)mc;   // ranks of the selected are 0..k-1, each once
     }
     group_sync<NT, BAR>();
-    if (sel) {
-        const uint32_t mp = ~(uint32_t)mc;
-        int r = 0;
-#pragma unroll 4
-        for (uint32_t j = 0; j < total; ++j) r += (flag[j] && ~(uint32_t)cand[j] < mp) ? 1 : 0;
-        out[r] = (int32_t)mp;
+    // the k selected positions, ascending: a bitonic sort in the first warp
+    if (warp == 0) {
+        // (rolled: one warp runs this once per call, and unrolled its
+        // instruction fetch, not its arithmetic, set its latency)
+        uint32_t v = lane < k ? selpos[lane] : 0xFFFFFFFFu;
+#pragma unroll 1
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll 1
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
+                const bool asc = ((lane & size) == 0) || size == 32;
+                const bool lower = (lane & stride) == 0;
+                v = (lower == asc) ? min(v, o) : max(v, o);
+            }
+        }
+        if (lane < k) out[lane] = (int32_t)v;
     }
     group_sync<NT, BAR>();
     return true;

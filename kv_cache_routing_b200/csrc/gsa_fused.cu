@@ -903,18 +903,44 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
 }
 
 // Tile lt of the row table into slots seq, seq + 1 (K, V) once the slots'
-// previous contents are consumed: every unfold thread issues its share and
-// holds both phases open until its copies have landed; one thread then gives
-// the one expected arrival.
-__device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars* bars, int lt, int seq) {
+// previous contents are consumed.  Its first tma_rows rows are runs of h
+// consecutive source rows (selected chunks, or the children of selected
+// groups) starting at multiples of h: one thread moves each run with four TMA
+// boxes (K and V, two 64-column halves each) that land in the swizzled
+// layout, h being a multiple of 8; the other rows (selected gists, empty rows)
+// are copied by every unfold thread with cp.async.  The copiers hold each
+// phase open until their copies have landed, the TMA bytes are expected on
+// it, and one thread then gives the one expected arrival.
+__device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars* bars, int lt, int seq, int row,
+                                            int tma_rows, int h, bool children) {
     slot_free(p, bars, seq);
     slot_free(p, bars, seq + 1);
     const int sk = seq % NSL, sv = (seq + 1) % NSL;
     uint8_t* ks = base + SM_STAGE + sk * SLOT_BYTES;
     uint8_t* vs = base + SM_STAGE + sv * SLOT_BYTES;
     const int32_t* tab = reinterpret_cast<const int32_t*>(base + SM_ROWTAB) + lt * TILE;
+    if (tma_rows > 0 && utid() == 0) {
+        const uint32_t bytes = (uint32_t)tma_rows * (D * 2);
+        mbar_expect_tx(&bars->full[sk], bytes);
+        mbar_expect_tx(&bars->full[sv], bytes);
+        const CUtensorMap* mk = children ? &p.tm_kc : &p.tm_kr;
+        const CUtensorMap* mv = children ? &p.tm_vc : &p.tm_vr;
+        const long long n_src = p.hier ? (long long)p.N1 : (long long)p.N;   // chunks (level-1 gists) per row
+        for (int r = 0; r < tma_rows; r += h) {
+            const long long e = tab[r];
+            // source row of the run: token (chunk * c) of the row's raw rows, or the first child
+            const int y = children ? (int)(-e - 2 - (long long)row * n_src) : (int)(e - (long long)row * n_src * p.C);
+            tc::tma_load_3d(ks + r * 128, mk, 0, y, row, &bars->full[sk]);
+            tc::tma_load_3d(ks + 16384 + r * 128, mk, 64, y, row, &bars->full[sk]);
+            tc::tma_load_3d(vs + r * 128, mv, 0, y, row, &bars->full[sv]);
+            tc::tma_load_3d(vs + 16384 + r * 128, mv, 64, y, row, &bars->full[sv]);
+        }
+    }
 #pragma unroll 4
-    for (int q = utid(); q < TILE * 16; q += NU) gather_piece(p, ks, vs, tab[q >> 4], q >> 4, q & 15);
+    for (int q = utid(); q < (TILE - tma_rows) * 16; q += NU) {
+        const int r = tma_rows + (q >> 4);
+        gather_piece(p, ks, vs, tab[r], r, q & 15);
+    }
     cp_async_arrive_hold(&bars->full[sk]);
     cp_async_arrive_hold(&bars->full[sv]);
     usync();
@@ -1310,7 +1336,22 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                     if (p.hier) hier_children_table(p, cx.base, row);
                     else build_table(p, cx.base, row, t0, ntl);
                 }
-                for (int lt = 0; lt < ntl; ++lt) gather_tile(p, cx.base, cx.bars, lt, gseq + 2 * lt);
+                for (int lt = 0; lt < ntl; ++lt) {
+                    // leading rows that are whole runs of consecutive source rows
+                    int tma_rows = 0, h = p.C;
+                    const bool children = p.hier && rd == 0;
+                    if (children) {
+                        h = p.group;
+                        tma_rows = p.tma_children ? min(TILE, p.K * p.group) : 0;
+                    } else if (p.tma_raw) {
+                        // rows of the selected chunks in this tile (the hierarchy's raw
+                        // round keeps its one tile at table index 0)
+                        const int kc = (p.hier ? p.K1 : p.K) * p.C;
+                        const int tile = p.hier ? lt : t0 + lt;
+                        tma_rows = max(0, min(TILE, kc - tile * TILE));
+                    }
+                    gather_tile(p, cx.base, cx.bars, lt, gseq + 2 * lt, row, tma_rows, h, children);
+                }
                 gseq += 2 * ntl;
                 ++runs;
             }
@@ -1363,10 +1404,11 @@ static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
     return fn;
 }
 
-// 3-D bf16 map over [rows][len][d = 128], box {64, 128, 1}, 128-byte swizzle:
-// a tile that runs past `len` is zero-filled instead of reading the next
-// (batch, kv-head) row's entries. An operand the call never reads gets a zeroed map.
-static bool map3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t len) {
+// 3-D bf16 map over [rows][len][d = 128], box {64, box_rows, 1}, 128-byte
+// swizzle: a box that runs past `len` is zero-filled instead of reading the
+// next (batch, kv-head) row's entries.  An operand the call never reads gets a
+// zeroed map.
+static bool map3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t len, uint32_t box_rows = TILE) {
     if (rows == 0 || len == 0 || base == nullptr) {
         std::memset(m, 0, sizeof(*m));
         return true;
@@ -1375,12 +1417,17 @@ static bool map3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t len)
     if (!enc) return false;
     cuuint64_t dims[3] = {D, len, rows};
     cuuint64_t strides[2] = {D * 2, len * D * 2};
-    cuuint32_t box[3] = {64, TILE, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// Runs of h consecutive source rows are gathered by TMA when each run starts
+// on a 1 KiB boundary of the swizzled tile (h a multiple of 8) and runs never
+// straddle tiles (h divides 128).
+static bool chunk_runs(int h) { return h >= 8 && h % 8 == 0 && TILE % h == 0; }
 
 // The CTAs of one launch wait on one another (a row's unfold item waits for
 // the key stretches of the CTAs that met the row), so all of them must be
@@ -1567,6 +1614,10 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
     const bool pairs = d.mode == GSA_SELECTED_PAIRS;
     bool ok = map3d(&p.tm_kg, kg, rows, N) && map3d(&p.tm_vg, pairs ? nullptr : vg, rows, N) &&
               map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
+    p.tma_raw = chunk_runs(d.chunk) && f.nbt > 0 ? 1 : 0;
+    if (p.tma_raw)
+        ok = ok && map3d(&p.tm_kr, kr, rows, N * (uint64_t)d.chunk, (uint32_t)d.chunk) &&
+             map3d(&p.tm_vr, vr, rows, N * (uint64_t)d.chunk, (uint32_t)d.chunk);
     if (!ok) return GSA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     fill_common(p, f, d, w);
@@ -1631,6 +1682,14 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
     const uint64_t rows = (uint64_t)f.rows;
     bool ok = map3d(&p.tm_kg, k_g2, rows, (uint64_t)h.n_l2) && map3d(&p.tm_vg, v_g2, rows, (uint64_t)h.n_l2) &&
               map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
+    p.tma_raw = chunk_runs(d.chunk) && d.top_k > 0 ? 1 : 0;
+    p.tma_children = chunk_runs(h.group) ? 1 : 0;
+    const uint64_t n1 = (uint64_t)d.n_chunks;
+    if (p.tma_raw)
+        ok = ok && map3d(&p.tm_kr, kr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk) &&
+             map3d(&p.tm_vr, vr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk);
+    if (p.tma_children)
+        ok = ok && map3d(&p.tm_kc, k_g1, rows, n1, (uint32_t)h.group) && map3d(&p.tm_vc, v_g1, rows, n1, (uint32_t)h.group);
     if (!ok) return GSA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     fill_common(p, f, d, w);

@@ -30,6 +30,8 @@ namespace fused {
 struct Params {
     CUtensorMap tm_kg, tm_vg;      // gists  [rows][N][d], box {64, 128, 1}
     CUtensorMap tm_kt, tm_vt;      // tail   [rows][W][d], box {64, 128, 1}
+    CUtensorMap tm_kr, tm_vr;      // raw    [rows][N c][d], box {64, c, 1} (chunk gathers by TMA)
+    CUtensorMap tm_kc, tm_vc;      // hierarchy: level-1 gists [rows][N1][d], box {64, group, 1}
     const uint16_t* q;             // [B][Hq][d]
     const uint8_t* kr;             // raw K/V and gist K/V base pointers (gathered tiles)
     const uint8_t* vr;
@@ -50,6 +52,8 @@ struct Params {
     int tg, upr, grid, slot_stride, maxs;
     int nrows_g, nbt, tpc, cb, items;
     int T;                         // units in all
+    int tma_raw;                   // chunks are gathered by TMA (c % 8 == 0 and c divides 128)
+    int tma_children;              // the children groups are gathered by TMA (same rule for group)
     int tmem_cols;                 // TMEM columns a CTA allocates
     float c2;
     int do_score, do_topk, do_attn_gists, sel_direct;

@@ -351,8 +351,9 @@ def run_ours(args, world, rank, local):
         "head_steps_per_s": round(steps_per_s * s.batch * s.n_q_heads, 1),
         "algorithmic_bytes_per_step": nbytes_step,
         "roofline": {"bound": "hbm",
-                     "kernel": f"gsa_decode_step: {launches} launches per step of one kernel "
-                               f"(per launch: half the step's algorithmic bytes in half the step's time)",
+                     "kernel": (f"gsa_decode_step: one launch of fused_decode_kernel per step" if launches == 1 else
+                                f"gsa_decode_step: {launches} launches per step (per launch: 1/{launches} of the "
+                                f"step's algorithmic bytes in 1/{launches} of its time)"),
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": nbytes_step / launches,

@@ -919,14 +919,19 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
     uint8_t* ks = base + SM_STAGE + sk * SLOT_BYTES;
     uint8_t* vs = base + SM_STAGE + sv * SLOT_BYTES;
     const int32_t* tab = reinterpret_cast<const int32_t*>(base + SM_ROWTAB) + lt * TILE;
-    if (tma_rows > 0 && utid() == 0) {
-        const uint32_t bytes = (uint32_t)tma_rows * (D * 2);
+    // lane 0 of each unfold warp issues every fourth run (TMA issue, not the
+    // copy, sets the pace: about 45 ns an instruction), expecting its own
+    // bytes first; the phase cannot complete before the final arrival below
+    const int uw = utid() >> 5;
+    if (tma_rows > 0 && (utid() & 31) == 0 && uw * h < tma_rows) {
+        const int runs = (tma_rows / h - uw + (NU / 32) - 1) / (NU / 32);
+        const uint32_t bytes = (uint32_t)(runs * h) * (D * 2);
         mbar_expect_tx(&bars->full[sk], bytes);
         mbar_expect_tx(&bars->full[sv], bytes);
         const CUtensorMap* mk = children ? &p.tm_kc : &p.tm_kr;
         const CUtensorMap* mv = children ? &p.tm_vc : &p.tm_vr;
         const long long n_src = p.hier ? (long long)p.N1 : (long long)p.N;   // chunks (level-1 gists) per row
-        for (int r = 0; r < tma_rows; r += h) {
+        for (int r = uw * h; r < tma_rows; r += (NU / 32) * h) {
             const long long e = tab[r];
             // source row of the run: token (chunk * c) of the row's raw rows, or the first child
             const int y = children ? (int)(-e - 2 - (long long)row * n_src) : (int)(e - (long long)row * n_src * p.C);
@@ -1168,6 +1173,17 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         if (p.W > 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_kt) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_vt) : "memory");
+        }
+    }
+    if (threadIdx.x == UFIRST) {
+        // and those of the gathers
+        if (p.tma_raw) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_kr) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_vr) : "memory");
+        }
+        if (p.tma_children) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_kc) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_vc) : "memory");
         }
     }
     for (int i = threadIdx.x; i <= p.grid; i += NTHR)
@@ -1502,21 +1518,20 @@ static void place_ctas(FusedPlan& f, int nb_slots) {
     f.maxs = maxs;
     f.slot_stride = maxs + nb_slots;
     // TMEM: S and O^T (64 columns), then per CTA G columns for each attended
-    // unit and each attended segment of its range
+    // unit and each attended segment of its range (its rows, few per CTA)
     int need = 64;
     for (int c = 0; c < f.grid && f.T > 0; ++c) {
         const long long u0 = (long long)c * f.T / f.grid, u1 = (long long)(c + 1) * f.T / f.grid;
-        int units = 0, segs = 0;
-        long long prev = -1;
-        for (long long u = u0; u < u1; ++u) {
-            const long long row = u / f.upr;
-            const bool attn = (u % f.upr) >= f.tg || f.attn_gists;
-            if (!attn) continue;
-            ++units;
-            if (row != prev) ++segs;
-            prev = row;
+        if (u1 <= u0) continue;
+        long long units = 0, segs = 0;
+        for (long long row = u0 / f.upr; row <= (u1 - 1) / f.upr; ++row) {
+            // the row's attended units: all of them, or its tail tiles
+            const long long a0 = row * f.upr + (f.attn_gists ? 0 : f.tg), a1 = (row + 1) * f.upr;
+            const long long n = std::max(0LL, std::min(a1, u1) - std::max(a0, u0));
+            units += n;
+            segs += n > 0 ? 1 : 0;
         }
-        need = std::max(need, 64 + (units + segs) * f.G);
+        need = (int)std::max<long long>(need, 64 + (units + segs) * f.G);
     }
     f.tmem_cols = need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : need <= 512 ? 512 : 1024;
 }

@@ -69,6 +69,12 @@ EDGE = {
     "chunk1": DecodeShape(1, 4, 1, 128, 513, 1, 40, 7, "bf16", SELECTED_PAIRS, n_needles=40),
     "chunk64": DecodeShape(1, 4, 1, 128, 100, 64, 5, 64, "bf16", ALL_GISTS, n_needles=5),
     "many_rows": DecodeShape(40, 16, 8, 64, 64, 16, 4, 16, "bf16", ALL_GISTS, n_needles=4),
+    # tensor-core path with more unfold items than CTAs: some CTAs take two or three items
+    # (row tables rewritten between gathered stretches)
+    "many_rows_tc": DecodeShape(40, 16, 8, 128, 200, 16, 8, 16, "bf16", ALL_GISTS, n_needles=8),
+    "many_rows_tc_pairs": DecodeShape(40, 16, 8, 128, 200, 8, 12, 16, "bf16", SELECTED_PAIRS, n_needles=12),
+    # ... with three gathered tiles per item and k > 32 (per-CTA candidates, radix selection)
+    "many_rows_tc_k40": DecodeShape(20, 16, 8, 128, 600, 8, 40, 8, "bf16", ALL_GISTS, n_needles=40),
     "custom_scale": dataclasses.replace(DecodeShape(1, 8, 2, 128, 256, 16, 8, 16, "f32", ALL_GISTS,
                                                     n_needles=8), scale=0.05),
 }

@@ -68,6 +68,8 @@ def test_hier_one_million_tokens():
     HierShape(DecodeShape(1, 4, 1, 64, 96, 4, 5, 8, "f32", n_needles=5, needle_alpha=30.0), 6, 16, 6),
     # group 1: level 2 mirrors level 1
     HierShape(DecodeShape(1, 8, 2, 128, 200, 8, 4, 0, "bf16", n_needles=4, needle_alpha=40.0), 200, 1, 10),
+    # more rows than CTAs: some CTAs run two items (four gathered stretches)
+    HierShape(DecodeShape(20, 8, 8, 128, 512, 16, 4, 16, "bf16", n_needles=4, needle_alpha=40.0), 32, 16, 4),
     # many candidates, small chunks, G = 8
     HierShape(DecodeShape(1, 16, 2, 128, 4096, 2, 32, 64, "bf16", n_needles=32, needle_alpha=40.0), 128, 32, 32),
 ])

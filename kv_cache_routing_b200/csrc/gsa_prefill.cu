@@ -107,10 +107,44 @@ constexpr uint32_t SM_BAR = SM_KV + 2 * 65536; // barriers and the TMEM address
 constexpr uint32_t PF_SMEM = SM_BAR + 256 + 1024;
 
 struct PfBars {
-    uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done[2];
+    uint64_t q_full, q_free, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done[2], o_free[2];
     uint32_t tmem;
 };
 
+// A work item: one query tile of one head pair.  Items are numbered heaviest
+// query tiles first (most earlier gists), then (batch, kv head, head pair).
+struct PfItem {
+    int bkv, hkv, bhA, j0, p0, n_gt, n_kv;
+    bool hasB;
+};
+
+__device__ __forceinline__ PfItem pf_item(const PrefillParams& p, int item) {
+    PfItem x;
+    const int nw = p.B * p.Hkv * p.NPAIR;
+    const int wi = item % nw;
+    const int t = p.n_qt - 1 - item / nw;
+    const int hp = wi % p.NPAIR;
+    x.bkv = wi / p.NPAIR;   // b * Hkv + kv head
+    const int b = x.bkv / p.Hkv;
+    x.hkv = x.bkv % p.Hkv;
+    const int hA = x.hkv * p.G + 2 * hp;
+    x.hasB = 2 * hp + 1 < p.G;
+    x.bhA = b * p.Hq + hA;
+    x.j0 = t * p.QC;
+    x.p0 = x.j0 * (p.C + 1);
+    const int j_last = min(x.j0 + p.QC, p.N) - 1;   // last chunk of the tile
+    x.n_gt = (j_last + 127) / 128;                  // tiles of earlier gists
+    x.n_kv = x.n_gt + 1;
+    return x;
+}
+
+// Persistent: CTA c takes items c, c + grid, ...  Every barrier's phases run
+// on across items; the K/V ring, the S / P / O hand-offs and the softmax state
+// are as for one item, and two more barriers join consecutive items: q_free
+// (the item's last S products are done with Q, so the next Q may load) and
+// o_free[h] (the epilogue has read head h's O, so the next item's first P.V
+// may overwrite it).  The next item's loads and first S products thus run
+// under the current item's epilogue.
 __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -118,31 +152,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
     const uint32_t sbase = smem_u32(base);
     PfBars& bars = *reinterpret_cast<PfBars*>(base + SM_BAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // work item: heaviest query tiles first; then (batch, kv head, head pair)
-    const int nw = p.B * p.Hkv * p.NPAIR;
-    const int bid = blockIdx.x;
-    const int wi = bid % nw;
-    const int t = p.n_qt - 1 - bid / nw;
-    const int hp = wi % p.NPAIR, bkv = wi / p.NPAIR;   // bkv = b * Hkv + kv head
-    const int b = bkv / p.Hkv, hkv = bkv % p.Hkv;
-    const int hA = hkv * p.G + 2 * hp;
-    const bool hasB = 2 * hp + 1 < p.G;
-    const int bhA = b * p.Hq + hA;
-    const int j0 = t * p.QC;
-    const int p0 = j0 * (p.C + 1);
-    const int j_last = min(j0 + p.QC, p.N) - 1;      // last chunk of the tile
-    const int n_gt = (j_last + 127) / 128;          // tiles of earlier gists
-    const int n_kv = n_gt + 1;
+    const int n_items = p.n_qt * p.B * p.Hkv * p.NPAIR;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars.q_full, 1);
+        mbar_init(&bars.q_free, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.kv_full[i], 1);
             mbar_init(&bars.kv_empty[i], 1);
             mbar_init(&bars.s_full[i], 1);
             mbar_init(&bars.p_full[i], 128);
             mbar_init(&bars.o_done[i], 1);
+            mbar_init(&bars.o_free[i], 128);
         }
         fence_mbar_init();
     }
@@ -154,7 +175,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = bars.tmem;
-    uint32_t* err = &g_prefill_err;   // waits below are bounded; a timeout abandons the tile
+    uint32_t* err = &g_prefill_err;   // waits below are bounded; a timeout abandons the item
 
     if (warp >= 8) {
     // --------------------------------- load / MMA warpgroup (warps 8-11) ----
@@ -162,34 +183,44 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
     if (warp == 8) {
         if (lane == 0) {
             // --------------------------------------------------- TMA loads --
-            mbar_arrive_expect_tx(&bars.q_full, hasB ? 65536 : 32768);
-            tc::tma_load_3d(base + SM_Q, &p.tm_q, 0, p0, bhA, &bars.q_full);
-            tc::tma_load_3d(base + SM_Q + 16384, &p.tm_q, 64, p0, bhA, &bars.q_full);
-            if (hasB) {
-                tc::tma_load_3d(base + SM_Q + 32768, &p.tm_q, 0, p0, bhA + 1, &bars.q_full);
-                tc::tma_load_3d(base + SM_Q + 49152, &p.tm_q, 64, p0, bhA + 1, &bars.q_full);
-            }
-            for (int i = 0; i < n_kv; ++i) {
-                const int s = i & 1;
-                if (i >= 2 && !mbar_wait(&bars.kv_empty[s], ((i - 2) >> 1) & 1, err)) break;
-                uint8_t* ks = base + SM_KV + s * 65536;
-                uint8_t* vs = ks + 32768;
-                mbar_arrive_expect_tx(&bars.kv_full[s], 65536);
-                const CUtensorMap* mk = i < n_gt ? &p.tm_kg : &p.tm_k;
-                const CUtensorMap* mv = i < n_gt ? &p.tm_vg : &p.tm_v;
-                const int y = i < n_gt ? i * 128 : p0;
-                tc::tma_load_3d(ks, mk, 0, y, bkv, &bars.kv_full[s]);
-                tc::tma_load_3d(ks + 16384, mk, 64, y, bkv, &bars.kv_full[s]);
-                tc::tma_load_3d(vs, mv, 0, y, bkv, &bars.kv_full[s]);
-                tc::tma_load_3d(vs + 16384, mv, 64, y, bkv, &bars.kv_full[s]);
+            int g = 0, it = 0;   // K/V tiles and items so far
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++it) {
+                const PfItem x = pf_item(p, item);
+                // the previous item's S products are done with the Q buffer
+                if (it > 0 && !mbar_wait(&bars.q_free, (it - 1) & 1, err)) break;
+                mbar_arrive_expect_tx(&bars.q_full, x.hasB ? 65536 : 32768);
+                tc::tma_load_3d(base + SM_Q, &p.tm_q, 0, x.p0, x.bhA, &bars.q_full);
+                tc::tma_load_3d(base + SM_Q + 16384, &p.tm_q, 64, x.p0, x.bhA, &bars.q_full);
+                if (x.hasB) {
+                    tc::tma_load_3d(base + SM_Q + 32768, &p.tm_q, 0, x.p0, x.bhA + 1, &bars.q_full);
+                    tc::tma_load_3d(base + SM_Q + 49152, &p.tm_q, 64, x.p0, x.bhA + 1, &bars.q_full);
+                }
+                for (int i = 0; i < x.n_kv; ++i, ++g) {
+                    const int s = g & 1;
+                    if (g >= 2 && !mbar_wait(&bars.kv_empty[s], ((g - 2) >> 1) & 1, err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* ks = base + SM_KV + s * 65536;
+                    uint8_t* vs = ks + 32768;
+                    mbar_arrive_expect_tx(&bars.kv_full[s], 65536);
+                    const CUtensorMap* mk = i < x.n_gt ? &p.tm_kg : &p.tm_k;
+                    const CUtensorMap* mv = i < x.n_gt ? &p.tm_vg : &p.tm_v;
+                    const int y = i < x.n_gt ? i * 128 : x.p0;
+                    tc::tma_load_3d(ks, mk, 0, y, x.bkv, &bars.kv_full[s]);
+                    tc::tma_load_3d(ks + 16384, mk, 64, y, x.bkv, &bars.kv_full[s]);
+                    tc::tma_load_3d(vs, mv, 0, y, x.bkv, &bars.kv_full[s]);
+                    tc::tma_load_3d(vs + 16384, mv, 64, y, x.bkv, &bars.kv_full[s]);
+                }
             }
         }
     } else if (warp == 9) {
         if (lane == 0) {
             // ----------------------------------------------------- MMA issue --
             // S_h = Q_h . K^T into TMEM columns 128 h; P_h . V into 256 + 128 h
-            auto issue_s = [&](int h, int i) {
-                const uint32_t ks = sbase + SM_KV + (i & 1) * 65536;
+            auto issue_s = [&](int h, int g) {
+                const uint32_t ks = sbase + SM_KV + (g & 1) * 65536;
                 const uint32_t qs = sbase + SM_Q + h * 32768;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -199,38 +230,54 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
                 }
                 tc::commit(&bars.s_full[h]);
             };
-            auto issue_pv = [&](int h, int i) {
-                const uint32_t vs = sbase + SM_KV + (i & 1) * 65536 + 32768;
+            auto issue_pv = [&](int h, int g, bool first) {
+                const uint32_t vs = sbase + SM_KV + (g & 1) * 65536 + 32768;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8,
-                                    tc::sdesc_sw128(vs + kk * 2048, 16384, 1024), IDESC_PV, (i > 0 || kk > 0));
+                                    tc::sdesc_sw128(vs + kk * 2048, 16384, 1024), IDESC_PV, (!first || kk > 0));
                 tc::commit(&bars.o_done[h]);
             };
-            bool ok = mbar_wait(&bars.q_full, 0, err) && mbar_wait(&bars.kv_full[0], 0, err);
-            tc::fence_after();
-            if (ok) {
-                issue_s(0, 0);
-                if (hasB) issue_s(1, 0);
-            }
-            for (int i = 0; ok && i < n_kv; ++i) {
-                const bool more = i + 1 < n_kv;
-                for (int h = 0; ok && h < (hasB ? 2 : 1); ++h) {
-                    // P_h of tile i (which also means S_h of tile i has been read)
-                    ok = mbar_wait(&bars.p_full[h], i & 1, err);
-                    if (!ok) break;
-                    tc::fence_after();
-                    issue_pv(h, i);
-                    if (h == (hasB ? 1 : 0)) tc::commit(&bars.kv_empty[i & 1]);
-                    if (more) {
-                        if (h == 0) {
-                            ok = mbar_wait(&bars.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1, err);
-                            if (!ok) break;
-                            tc::fence_after();
+            int g = 0, it = 0;
+            int pc0 = 0, pc1 = 0;   // P tiles per head so far (p_full phases)
+            int itB = 0;            // items with a head B so far (o_free[1] phases; head A: every item)
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++it) {
+                const PfItem x = pf_item(p, item);
+                const int nh = x.hasB ? 2 : 1;
+                ok = mbar_wait(&bars.q_full, it & 1, err) && mbar_wait(&bars.kv_full[g & 1], (g >> 1) & 1, err);
+                tc::fence_after();
+                if (!ok) break;
+                issue_s(0, g);
+                if (x.hasB) issue_s(1, g);
+                if (x.n_kv == 1) tc::commit(&bars.q_free);   // the item's last S products are issued
+                for (int i = 0; ok && i < x.n_kv; ++i) {
+                    const bool more = i + 1 < x.n_kv;
+                    for (int h = 0; ok && h < nh; ++h) {
+                        // P_h of tile i (which also means S_h of tile i has been read)
+                        const int pc = h == 0 ? pc0++ : pc1++;
+                        ok = mbar_wait(&bars.p_full[h], pc & 1, err);
+                        // the first P.V of an item overwrites O_h: the previous
+                        // item's epilogue must have read it
+                        const int ih = h == 0 ? it : itB;
+                        if (ok && i == 0 && ih > 0) ok = mbar_wait(&bars.o_free[h], (ih - 1) & 1, err);
+                        if (!ok) break;
+                        tc::fence_after();
+                        issue_pv(h, g + i, i == 0);
+                        if (h == nh - 1) tc::commit(&bars.kv_empty[(g + i) & 1]);
+                        if (more) {
+                            if (h == 0) {
+                                ok = mbar_wait(&bars.kv_full[(g + i + 1) & 1], ((g + i + 1) >> 1) & 1, err);
+                                if (!ok) break;
+                                tc::fence_after();
+                            }
+                            issue_s(h, g + i + 1);
+                            if (i + 2 == x.n_kv && h == nh - 1) tc::commit(&bars.q_free);
                         }
-                        issue_s(h, i + 1);
                     }
                 }
+                g += x.n_kv;
+                itB += x.hasB ? 1 : 0;
             }
         }
     }
@@ -238,24 +285,31 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
         // ------------------------------------------------ softmax warps ----
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(PF_REG_SOFTMAX));
         const int h = warp >> 2;                         // 0: head A, 1: head B
-        if (h == 0 || hasB) {
-            const int r = threadIdx.x & 127;             // query row = TMEM lane
-            const int qp = p0 + r;
+        const int r = threadIdx.x & 127;                 // query row = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t ts = tmem + h * 128 + lane_off, to = tmem + 256 + h * 128 + lane_off;
+        int sc = 0;                                      // S tiles of this head so far
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+            const PfItem x = pf_item(p, item);
+            if (h == 1 && !x.hasB) continue;             // (only with an odd group: the last pair is one head)
+            const int qp = x.p0 + r;
             const bool valid = r < p.QC * (p.C + 1) && qp < p.P;
-            const int jq = valid ? j0 + r / (p.C + 1) : -1;
-            const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-            const uint32_t ts = tmem + h * 128 + lane_off, to = tmem + 256 + h * 128 + lane_off;
+            const int jq = valid ? x.j0 + r / (p.C + 1) : -1;
             float m_run = -INFINITY, l_run = 0.f;
-            for (int i = 0; i < n_kv; ++i) {
-                if (!mbar_wait(&bars.s_full[h], i & 1, err)) break;
+            bool ok = true;
+            for (int i = 0; i < x.n_kv; ++i, ++sc) {
+                if (!mbar_wait(&bars.s_full[h], sc & 1, err)) {
+                    ok = false;
+                    break;
+                }
                 tc::fence_after();
                 // allowed key columns [lo, hi] of this row in this tile
                 int lo, hi;
-                if (i < n_gt) {
+                if (i < x.n_gt) {
                     lo = 0;
                     hi = valid ? min(127, jq - i * 128 - 1) : -1;
                 } else {
-                    lo = valid ? jq * (p.C + 1) - p0 : 1;
+                    lo = valid ? jq * (p.C + 1) - x.p0 : 1;
                     hi = valid ? r : 0;
                 }
                 // the row's 128 scores in registers (all four loads in flight)
@@ -295,7 +349,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
                 const float alpha = need ? exp2f(m_run - m_new) : 1.f;
                 if (__any_sync(0xFFFFFFFFu, need) && i > 0) {
                     // O holds P.V of tiles < i: wait for the last of them, then rescale
-                    mbar_wait(&bars.o_done[h], (i - 1) & 1, err);
+                    mbar_wait(&bars.o_done[h], (sc - 1) & 1, err);
                     tc::fence_after();
 #pragma unroll 1
                     for (int c = 0; c < 8; ++c) {
@@ -338,31 +392,36 @@ __global__ void __launch_bounds__(PF_THREADS, 1) gist_prefill_kernel(const __gri
                 tc::fence_before();
                 mbar_arrive(&bars.p_full[h]);
             }
+            if (!ok) break;
             // -------------------------------------------------- epilogue ----
-            mbar_wait(&bars.o_done[h], (n_kv - 1) & 1, err);
+            // O of the item's last tile, all 128 columns into registers; then
+            // O_h is released to the next item's first P.V
+            mbar_wait(&bars.o_done[h], (sc - 1) & 1, err);
             tc::fence_after();
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            const int bh = bhA + h;
-            uint16_t* orow = p.out + ((size_t)bh * p.P + qp) * PF_D;
+            uint32_t ov[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t u[32];
-                tc::ld32(to + c * 32, u);
-                tc::wait_ld();
-                if (valid) {
+            for (int c = 0; c < 4; ++c) tc::ld32(to + c * 32, ov[c]);
+            tc::wait_ld();
+            tc::fence_before();
+            mbar_arrive(&bars.o_free[h]);
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const int bh = x.bhA + h;
+            uint16_t* orow = p.out + ((size_t)bh * p.P + qp) * PF_D;
+            if (valid) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
                         uint4 v;
-                        v.x = tc::pack_bf16x2(__uint_as_float(u[j]) * inv, __uint_as_float(u[j + 1]) * inv);
-                        v.y = tc::pack_bf16x2(__uint_as_float(u[j + 2]) * inv, __uint_as_float(u[j + 3]) * inv);
-                        v.z = tc::pack_bf16x2(__uint_as_float(u[j + 4]) * inv, __uint_as_float(u[j + 5]) * inv);
-                        v.w = tc::pack_bf16x2(__uint_as_float(u[j + 6]) * inv, __uint_as_float(u[j + 7]) * inv);
+                        v.x = tc::pack_bf16x2(__uint_as_float(ov[c][j]) * inv, __uint_as_float(ov[c][j + 1]) * inv);
+                        v.y = tc::pack_bf16x2(__uint_as_float(ov[c][j + 2]) * inv, __uint_as_float(ov[c][j + 3]) * inv);
+                        v.z = tc::pack_bf16x2(__uint_as_float(ov[c][j + 4]) * inv, __uint_as_float(ov[c][j + 5]) * inv);
+                        v.w = tc::pack_bf16x2(__uint_as_float(ov[c][j + 6]) * inv, __uint_as_float(ov[c][j + 7]) * inv);
                         *reinterpret_cast<uint4*>(orow + c * 32 + j) = v;
                     }
                 }
+                if (p.lse != nullptr) p.lse[(size_t)bh * p.P + qp] = (m_run + log2f(l_run)) * 0.69314718055994531f;
             }
-            if (valid && p.lse != nullptr)
-                p.lse[(size_t)bh * p.P + qp] = (m_run + log2f(l_run)) * 0.69314718055994531f;
         }
     }
     tc::fence_before();
@@ -461,7 +520,16 @@ extern "C" gsa_status gsa_gist_prefill(const gsa_prefill_desc* desc, const void*
             return GSA_ERR_CUDA;
         attr = true;
     }
-    const unsigned grid = (unsigned)p.n_qt * (unsigned)(B * Hkv * p.NPAIR);
+    // persistent: one CTA per SM (the work split does not depend on the device beyond the grid)
+    static int n_sm = 0;
+    if (n_sm == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0)
+            return GSA_ERR_CUDA;
+    }
+    const long long items = (long long)p.n_qt * (B * Hkv * p.NPAIR);
+    const unsigned grid = (unsigned)std::min<long long>(items, n_sm);
     gist_prefill_kernel<<<grid, PF_THREADS, PF_SMEM, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }

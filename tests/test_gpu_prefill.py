@@ -50,6 +50,8 @@ def run_prefill(p: PrefillShape, seed: int, label: str, sample: int = 0):
     PrefillShape(1, 2, 1, 128, 5, 127),      # c = 127: one chunk per tile
     PrefillShape(1, 4, 2, 128, 300, 16),     # three gist tiles for the last query tiles
     PrefillShape(1, 8, 2, 128, 700, 7),      # ragged last tile, six gist tiles
+    PrefillShape(1, 6, 2, 128, 100, 16),     # G = 3: the last head pair has one head
+    PrefillShape(2, 8, 2, 128, 400, 16),     # 464 work items: several per persistent CTA
 ])
 def test_prefill_small_exhaustive(shape):
     run_prefill(shape, 11 + shape.n_chunks, f"prefill N={shape.n_chunks} c={shape.chunk}")

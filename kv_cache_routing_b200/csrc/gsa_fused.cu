@@ -1424,10 +1424,29 @@ static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 // swizzle: a box that runs past `len` is zero-filled instead of reading the
 // next (batch, kv-head) row's entries.  An operand the call never reads gets a
 // zeroed map.
+// The last few encoded maps are kept per host thread (a decode step encodes
+// up to six, and callers reuse the same buffers call after call).
+struct MapCacheEntry {
+    const void* base;
+    uint64_t rows, len;
+    uint32_t box_rows;
+    bool valid;
+    CUtensorMap map;
+};
 static bool map3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t len, uint32_t box_rows = TILE) {
     if (rows == 0 || len == 0 || base == nullptr) {
         std::memset(m, 0, sizeof(*m));
         return true;
+    }
+    constexpr int kMapCache = 32;
+    thread_local MapCacheEntry cache[kMapCache];
+    thread_local int next = 0;
+    for (int i = 0; i < kMapCache; ++i) {
+        const MapCacheEntry& c = cache[i];
+        if (c.valid && c.base == base && c.rows == rows && c.len == len && c.box_rows == box_rows) {
+            *m = c.map;
+            return true;
+        }
     }
     auto enc = encoder();
     if (!enc) return false;
@@ -1435,9 +1454,19 @@ static bool map3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t len,
     cuuint64_t strides[2] = {D * 2, len * D * 2};
     cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    MapCacheEntry& c = cache[next];
+    next = (next + 1) % kMapCache;
+    c.base = base;
+    c.rows = rows;
+    c.len = len;
+    c.box_rows = box_rows;
+    c.map = *m;
+    c.valid = true;
+    return true;
 }
 
 // Runs of h consecutive source rows are gathered by TMA when each run starts
@@ -1558,7 +1587,32 @@ static void layout_ws(FusedPlan& f, size_t N, size_t top_k, size_t k1) {
     f.total = o;
 }
 
+static FusedPlan build_fused_plan(const gsa_decode_desc& d, bool given);
+
+// Plans are a pure function of the descriptor; the last few are kept per host
+// thread (one decode call asks for the plan several times).
 FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given) {
+    struct Entry {
+        gsa_decode_desc d;
+        bool given, valid;
+        FusedPlan f;
+    };
+    constexpr int kPlanCache = 8;
+    thread_local Entry cache[kPlanCache];
+    thread_local int next = 0;
+    for (int i = 0; i < kPlanCache; ++i)
+        if (cache[i].valid && cache[i].given == given && std::memcmp(&cache[i].d, &d, sizeof(d)) == 0)
+            return cache[i].f;
+    Entry& e = cache[next];
+    next = (next + 1) % kPlanCache;
+    e.d = d;
+    e.given = given;
+    e.f = build_fused_plan(d, given);
+    e.valid = true;
+    return e.f;
+}
+
+static FusedPlan build_fused_plan(const gsa_decode_desc& d, bool given) {
     FusedPlan f{};
     const bool pairs = d.mode == GSA_SELECTED_PAIRS;
     f.attn_gists = pairs ? 0 : 1;

@@ -241,17 +241,11 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += NT) hist[i] = 0;
         group_sync<NT, BAR>();
-        // warp-aggregated histogram: float keys crowd a few bins in the high
-        // digits, so lanes with the same bin add once per warp instruction
-        for (int i0 = tid - (tid & 31); i0 < n; i0 += NT) {
-            const int i = i0 + (tid & 31);
-            uint32_t bin = 0xFFFFFFFFu;
-            if (i < n) {
-                const uint32_t u = key(i);
-                if ((u & pmask) == prefix) bin = (u >> shift) & 255u;
-            }
-            const uint32_t same = __match_any_sync(0xFFFFFFFFu, bin);
-            if (bin != 0xFFFFFFFFu && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+        // plain shared-memory atomics: same-bin updates serialise, but a
+        // warp-wide match of the bins costs far more
+        for (int i = tid; i < n; i += NT) {
+            const uint32_t u = key(i);
+            if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
         }
         group_sync<NT, BAR>();
         if (tid < 32) {
@@ -313,51 +307,155 @@ __device__ void block_topk(int n, int k, KeyF key, Emit emit, uint32_t* sh) {
 }
 
 
-// ------------------------------------------------- shared-memory top-k --
-// Exact top-k of n orderable keys held in shared memory (keys[i] for
-// position i): the k largest keys, equal keys taken lowest position first.
-// Writes the k selected positions to out[0..k) in ascending order.
-// Radix select, 8 bits per digit, compacting the candidates after every
-// digit (keys above the threshold digit are selected at once, keys on it
-// stay candidates), so only the first digit reads all n keys; the selection
-// is kept as a bitmap and emitted in position order by a popcount prefix.
-// Scratch `w` (shared): >= 256 + 16 + 2*NT/32 + (n+31)/32 * 2 + 2*n words
-// (histogram, control, scan, two bitmaps, two candidate lists).
-// All NT threads of the block call it.
-template <int NT, int BAR = 0, int FIRST = 0>
-__device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint32_t* w) {
-    const int tid = threadIdx.x - FIRST, lane = tid & 31, warp = tid >> 5;
+// --------------------------------------------------- threshold top-k --
+// Exact top-k for k <= 32 of n <= NT * M keys: the k largest keys, equal keys
+// taken lowest position first; out[0..k) receives the positions in ascending
+// order.  Thread t holds the keys of positions lo + i * step, i < mine, in
+// registers (key[i]); the positions of the threads may interleave in any way
+// (step NT: every warp-wide load is one contiguous line).
+//  1. In each warp, the k-th largest of the 32 lane maxima bounds the k-th
+//     largest key of the whole set from below (k distinct keys reach it), so
+//     the largest such bound over the warps, tau, does as well.
+//  2. The keys >= tau (k of them at least, and rarely many more) go to a
+//     shared list as 64-bit composites (key, ~position), each thread's after
+//     those of the lower threads (a warp scan of the counts, then the warp
+//     totals): a larger composite is a larger key, or the same key at a lower
+//     position.
+//  3. Each candidate counts the composites above its own; those with fewer
+//     than k above are selected, the count being the key rank.  Each of the
+//     k selected positions, one per rank, then counts the selected positions
+//     below it: its place in the ascending output.
+// Returns false without writing anything when more than NT keys reach tau
+// (a flood of equal keys): the caller then runs a general selection.
+// Scratch `w` (shared, 16-byte aligned): >= 16 + 2 * NT + 2 + 32 words.
+// All NT threads call it; it ends with the block synchronised.
+template <int NT, int M, int BAR = 0, int FIRST = 0>
+__device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, int mine, int k, int32_t* out,
+                                    uint32_t* w) {
     constexpr int NW = NT / 32;
-    if (k <= 0 || n <= 0) return;
-    if (k >= n) {
-        for (int i = tid; i < n; i += NT) out[i] = i;
-        return;
+    static_assert(2 * NW <= 16, "warp table overflow");
+    const int tid = threadIdx.x - FIRST, lane = tid & 31, warp = tid >> 5;
+    uint32_t tmax = 0u;
+#pragma unroll
+    for (int i = 0; i < M; ++i) tmax = max(tmax, i < mine ? key[i] : 0u);
+    // the k-th largest of the warp's 32 lane maxima is the warp's bound (a
+    // lane without keys offers 0, the smallest key, which can only weaken
+    // it): a bitonic sort of the lane maxima, descending, leaves it in lane k-1
+    uint32_t v = tmax;
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
+            // descending runs where (lane & size) == 0, the final pass descending
+            const bool desc = ((lane & size) == 0) || size == 32;
+            const bool lower = (lane & stride) == 0;
+            v = (lower == desc) ? max(v, o) : min(v, o);
+        }
     }
-    const int nw = (n + 31) >> 5;
-    uint32_t* hist = w;                   // 256
-    uint32_t* ctl = w + 256;              // [0] digit, [1] above, [2] next count, [3] done flag
-    uint32_t* scan = ctl + 16;            // 2 * NW
-    uint32_t* sel = scan + 2 * NW;        // nw words: selected positions
-    uint32_t* tie = sel + nw;             // nw words: candidates left after the last digit
-    uint32_t* cand = tie + nw;            // candidate positions (unordered), read list
-    uint32_t* next = cand + n;            // write list; the two swap after every digit
-    for (int i = tid; i < nw; i += NT) {
-        sel[i] = 0;
-        tie[i] = 0;
+    const uint32_t tau_w = __shfl_sync(0xFFFFFFFFu, v, k - 1);
+    if (lane == 0) w[warp] = tau_w;
+    group_sync<NT, BAR>();
+    uint32_t tau = w[0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) tau = max(tau, w[i]);
+    // this thread's candidates: counted, then placed after those of the lower
+    // lanes and warps (warp totals through shared memory, no atomics)
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < M; ++i) c += (i < mine && key[i] >= tau) ? 1u : 0u;
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
     }
-    uint32_t kk = (uint32_t)k;
-    int m = n;                            // candidates: all positions on the first digit
-    bool all = true;
+    if (lane == 31) w[NW + warp] = incl;
+    group_sync<NT, BAR>();
+    uint32_t base = 0, total = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+        const uint32_t x = w[NW + i];
+        base += i < warp ? x : 0u;
+        total += x;
+    }
+    if (total > (uint32_t)NT) {                   // the same on every thread
+        group_sync<NT, BAR>();                    // all have read the table before the caller reuses w
+        return false;
+    }
+    uint32_t off = base + incl - c;
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(w + 16);
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+        if (i < mine && key[i] >= tau) {
+            cand[off] = ((unsigned long long)key[i] << 32) | (unsigned long long)(~(uint32_t)(lo + i * step));
+            ++off;
+        }
+    // pad to an even count with 0 (never above a candidate: keys of
+    // candidates are >= tau and positions are complemented)
+    if (tid == 0 && (total & 1)) cand[total] = 0ull;
+    group_sync<NT, BAR>();
+    // key rank of each candidate: the composites above it; with at most NT/2
+    // candidates two neighbouring threads split the count
+    uint32_t* selpos = reinterpret_cast<uint32_t*>(w + 16 + 2 * NT + 2);   // [k]: position of key rank r
+    {
+        const bool two = total <= (uint32_t)(NT / 2);
+        const uint32_t ci = two ? (uint32_t)(tid >> 1) : (uint32_t)tid;
+        const uint32_t np = (total + 1) / 2, mid = np / 2;
+        const uint32_t j0 = (two && (tid & 1)) ? mid : 0u, j1 = (two && !(tid & 1)) ? mid : np;
+        const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(cand);
+        unsigned long long mc = 0ull;
+        int a = 0;
+        if (ci < total) {
+            mc = cand[ci];
+#pragma unroll 4
+            for (uint32_t j = j0; j < j1; ++j) {
+                const ulonglong2 v = c2[j];
+                a += (v.x > mc ? 1 : 0) + (v.y > mc ? 1 : 0);
+            }
+        }
+        if (two) a += __shfl_xor_sync(0xFFFFFFFFu, a, 1);
+        // ranks of the selected are 0..k-1, each once
+        if (ci < total && (!two || !(tid & 1)) && a < k) selpos[a] = ~(uint32_t)mc;
+    }
+    group_sync<NT, BAR>();
+    // the k selected positions, ascending: each goes to the count of selected
+    // positions below it (they are distinct)
+    if (tid < k) {
+        const uint32_t me = selpos[tid];
+        int r = 0;
+#pragma unroll 8
+        for (int j = 0; j < k; ++j) r += selpos[j] < me ? 1 : 0;
+        out[r] = (int32_t)me;
+    }
+    group_sync<NT, BAR>();
+    return true;
+}
+
+// Exact top-k (any 0 < k < n) of n keys held in registers: thread t holds
+// positions t + i * NT for i < mine (key[i]).  Radix select on 8-bit digits
+// from the top: each pass counts, in a 256-bin histogram (shared-memory
+// atomics), the keys that share the prefix found so far, and the digit on
+// which the k-th largest falls joins the prefix.  The k-th largest key T is then known; the keys above T are
+// selected, and of the keys equal to T the lowest positions (a popcount scan
+// of a bitmap in position order).  emit(r, pos) for the selected positions,
+// ascending.  Scratch: w >= 256 + 16 + NT / 32 + 1 words; bm >= 2 * ceil(n /
+// 32) words.  All NT threads of the group call it.
+template <int NT, int U, int BAR = 0, int FIRST = 0, class Emit>
+__device__ void radix_topk_regs(const uint32_t (&key)[U], int mine, int n, int k, uint32_t* w, uint32_t* bm,
+                                Emit emit) {
+    const int tid = threadIdx.x - FIRST, lane = tid & 31, warp = tid >> 5;
+    uint32_t* hist = w;          // 256
+    uint32_t* ctl = w + 256;     // [0] digit, [1] keys above it
+    uint32_t* scan = w + 272;    // NT / 32 + 1
+    uint32_t prefix = 0, pmask = 0, kk = (uint32_t)k;
+#pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += NT) hist[i] = 0;
-        if (tid == 0) ctl[2] = 0;
         group_sync<NT, BAR>();
-        for (int i0 = tid - lane; i0 < m; i0 += NT) {
-            const int i = i0 + lane;
-            uint32_t bin = 0xFFFFFFFFu;
-            if (i < m) bin = (keys[all ? i : cand[i]] >> shift) & 255u;
-            const uint32_t same = __match_any_sync(0xFFFFFFFFu, bin);
-            if (bin != 0xFFFFFFFFu && lane == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+#pragma unroll
+        for (int i = 0; i < U; ++i) {
+            if (i < mine && (key[i] & pmask) == prefix) atomicAdd(&hist[(key[i] >> shift) & 255u], 1u);
         }
         group_sync<NT, BAR>();
         if (warp == 0) {
@@ -385,65 +483,34 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
             }
         }
         group_sync<NT, BAR>();
-        const uint32_t D = ctl[0], above = ctl[1];
-        const bool last = shift == 0;
-        // keys above the threshold digit are selected; keys on it stay
-        // candidates (warp-aggregated: one atomic per warp and predicate)
-        for (int i0 = tid - lane; i0 < m; i0 += NT) {
-            const int i = i0 + lane;
-            int pos = 0;
-            uint32_t dg = 0;
-            if (i < m) {
-                pos = all ? i : (int)cand[i];
-                dg = (keys[pos] >> shift) & 255u;
-            }
-            const bool up = i < m && dg > D, eq = i < m && dg == D;
-            const uint32_t mup = __ballot_sync(0xFFFFFFFFu, up);
-            const uint32_t meq = __ballot_sync(0xFFFFFFFFu, eq);
-            if (all) {
-                // positions i0..i0+31 are exactly one bitmap word (i0 is a multiple of 32)
-                if (lane == 0) {
-                    if (mup) sel[i0 >> 5] |= mup;
-                    if (last && meq) tie[i0 >> 5] |= meq;
-                }
-            } else {
-                if (up) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
-                if (last && eq) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
-            }
-            if (!last && meq) {
-                uint32_t base = 0;
-                if (lane == 0) base = atomicAdd(&ctl[2], (uint32_t)__popc(meq));
-                base = __shfl_sync(0xFFFFFFFFu, base, 0);
-                if (eq) next[base + __popc(meq & ((1u << lane) - 1u))] = (uint32_t)pos;
-            }
-        }
+        prefix |= ctl[0] << shift;
+        pmask |= 255u << shift;
+        kk -= ctl[1];
         group_sync<NT, BAR>();
-        kk -= above;
-        m = (int)ctl[2];
-        all = false;
-        {
-            uint32_t* t = cand;
-            cand = next;
-            next = t;
-        }
-        group_sync<NT, BAR>();
-        if (!last && (uint32_t)m == kk) {
-            // every remaining candidate is selected
-            for (int i = tid; i < m; i += NT) atomicOr(&sel[cand[i] >> 5], 1u << (cand[i] & 31));
-            kk = 0;
-            group_sync<NT, BAR>();
-            break;
+    }
+    // T = prefix; take every key > T and the kk lowest positions of the keys == T
+    const int nw = (n + 31) >> 5;
+    uint32_t* sel = bm;
+    uint32_t* eq = bm + nw;
+    for (int i = tid; i < 2 * nw; i += NT) bm[i] = 0;
+    group_sync<NT, BAR>();
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+        if (i < mine) {
+            const int pos = tid + i * NT;
+            if (key[i] > prefix) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+            else if (key[i] == prefix) atomicOr(&eq[pos >> 5], 1u << (pos & 31));
         }
     }
-    // equal keys on the threshold: the kk lowest positions (tie bitmap in position order)
-    if (kk > 0) {
+    group_sync<NT, BAR>();
+    const int per = (nw + NT - 1) / NT, lo = tid * per, hi = min(nw, lo + per);
+    {
         uint32_t c = 0;
-        const int per = (nw + NT - 1) / NT, lo = tid * per, hi = min(nw, lo + per);
-        for (int i = lo; i < hi; ++i) c += __popc(tie[i]);
+        for (int i = lo; i < hi; ++i) c += __popc(eq[i]);
         uint32_t tot;
         uint32_t before = block_exclusive_scan<NT, BAR, FIRST>(c, scan, &tot);
         for (int i = lo; i < hi; ++i) {
-            uint32_t bits = tie[i];
+            uint32_t bits = eq[i];
             while (bits) {
                 const int b = __ffs(bits) - 1;
                 bits &= bits - 1;
@@ -451,12 +518,10 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
                 ++before;
             }
         }
-        group_sync<NT, BAR>();
     }
-    // emit the selection in ascending position order
+    group_sync<NT, BAR>();
     {
         uint32_t c = 0;
-        const int per = (nw + NT - 1) / NT, lo = tid * per, hi = min(nw, lo + per);
         for (int i = lo; i < hi; ++i) c += __popc(sel[i]);
         uint32_t tot;
         uint32_t r = block_exclusive_scan<NT, BAR, FIRST>(c, scan, &tot);
@@ -465,139 +530,11 @@ __device__ void smem_topk(const uint32_t* keys, int n, int k, int32_t* out, uint
             while (bits) {
                 const int b = __ffs(bits) - 1;
                 bits &= bits - 1;
-                out[r++] = i * 32 + b;
+                emit((int)r++, i * 32 + b);
             }
         }
     }
-}
-
-
-// --------------------------------------------------- threshold top-k --
-// Exact top-k for k <= 32 of n <= NT * M keys: the k largest keys, equal keys
-// taken lowest position first; out[0..k) receives the positions in ascending
-// order.  Thread t holds the keys of positions lo + i * step, i < mine, in
-// registers (key[i]); the positions of the threads may interleave in any way
-// (step NT: every warp-wide load is one contiguous line).
-//  1. In each warp, the k-th largest of the 32 lane maxima bounds the k-th
-//     largest key of the whole set from below (k distinct keys reach it), so
-//     the largest such bound over the warps, tau, does as well.
-//  2. The keys >= tau (k of them at least, and rarely many more) are appended,
-//     in any order, to a shared list as 64-bit composites (key, ~position): a
-//     larger composite is a larger key, or the same key at a lower position.
-//  3. Each candidate counts the composites above its own; those with fewer
-//     than k above are selected, the count being the key rank.  The k
-//     selected positions, one per rank, are sorted ascending by one warp.
-// Returns false without writing anything when more than NT keys reach tau
-// (a flood of equal keys): the caller then runs a general selection.
-// Scratch `w` (shared, 16-byte aligned): >= 16 + 2 * NT + 2 + 32 words.
-// All NT threads call it; it ends with the block synchronised.
-template <int NT, int M, int BAR = 0, int FIRST = 0>
-__device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, int mine, int k, int32_t* out,
-                                    uint32_t* w) {
-    constexpr int NW = NT / 32;
-    static_assert(NW + 1 <= 16, "warp bound table overflow");
-    const int tid = threadIdx.x - FIRST, lane = tid & 31, warp = tid >> 5;
-    uint32_t tmax = 0u;
-#pragma unroll
-    for (int i = 0; i < M; ++i) tmax = max(tmax, i < mine ? key[i] : 0u);
-    // the k-th largest of the warp's 32 lane maxima is the warp's bound (a
-    // lane without keys offers 0, the smallest key, which can only weaken
-    // it): a bitonic sort of the lane maxima, descending, leaves it in lane k-1
-    uint32_t v = tmax;
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
-            // descending runs where (lane & size) == 0, the final pass descending
-            const bool desc = ((lane & size) == 0) || size == 32;
-            const bool lower = (lane & stride) == 0;
-            v = (lower == desc) ? max(v, o) : min(v, o);
-        }
-    }
-    const uint32_t tau_w = __shfl_sync(0xFFFFFFFFu, v, k - 1);
-    if (lane == 0) w[warp] = tau_w;
-    if (tid == 0) w[NW] = 0u;
     group_sync<NT, BAR>();
-    uint32_t tau = w[0];
-#pragma unroll
-    for (int i = 1; i < NW; ++i) tau = max(tau, w[i]);
-    // append this thread's candidates: one atomic per warp
-    uint32_t c = 0;
-#pragma unroll
-    for (int i = 0; i < M; ++i) c += (i < mine && key[i] >= tau) ? 1u : 0u;
-    uint32_t incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    uint32_t base = 0;
-    if (lane == 31 && incl > 0) base = atomicAdd(&w[NW], incl);
-    base = __shfl_sync(0xFFFFFFFFu, base, 31);
-    uint32_t off = base + incl - c;
-    unsigned long long* cand = reinterpret_cast<unsigned long long*>(w + 16);
-#pragma unroll
-    for (int i = 0; i < M; ++i)
-        if (i < mine && key[i] >= tau) {
-            if (off < (uint32_t)NT)
-                cand[off] = ((unsigned long long)key[i] << 32) | (unsigned long long)(~(uint32_t)(lo + i * step));
-            ++off;
-        }
-    group_sync<NT, BAR>();
-    const uint32_t total = w[NW];
-    if (total > (uint32_t)NT) return false;       // the same on every thread
-    unsigned long long mc = 0ull;
-    uint32_t* selpos = reinterpret_cast<uint32_t*>(w + 16 + 2 * NT + 2);   // [k]: position of key rank r
-    if ((uint32_t)tid < total) {
-        mc = cand[tid];
-        // pad to an even count with 0 (never above a candidate: keys of
-        // candidates are >= tau and positions are complemented)
-        if (tid == 0 && (total & 1)) cand[total] = 0ull;
-    }
-    group_sync<NT, BAR>();
-    if ((uint32_t)tid < total) {
-        const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(cand);
-        int a = 0;
-#pragma unroll 4
-        for (uint32_t j = 0; j < (total + 1) / 2; ++j) {
-            const ulonglong2 v = c2[j];
-            a += (v.x > mc ? 1 : 0) + (v.y > mc ? 1 : 0);
-        }
-        if (a < k) selpos[a] = ~(uint32_t)mc;   // ranks of the selected are 0..k-1, each once
-    }
-    group_sync<NT, BAR>();
-    // the k selected positions, ascending: a bitonic sort in the first warp
-    if (warp == 0) {
-        // (rolled: one warp runs this once per call, and unrolled its
-        // instruction fetch, not its arithmetic, set its latency)
-        uint32_t v = lane < k ? selpos[lane] : 0xFFFFFFFFu;
-#pragma unroll 1
-        for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll 1
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
-                const bool asc = ((lane & size) == 0) || size == 32;
-                const bool lower = (lane & stride) == 0;
-                v = (lower == asc) ? min(v, o) : max(v, o);
-            }
-        }
-        if (lane < k) out[lane] = (int32_t)v;
-    }
-    group_sync<NT, BAR>();
-    return true;
-}
-
-// The same selection with the keys in shared memory (keys[i] for position i).
-template <int NT, int M, int BAR = 0, int FIRST = 0>
-__device__ bool threshold_topk(const uint32_t* keys, int n, int k, int32_t* out, uint32_t* w) {
-    const int m = (n + NT - 1) / NT;
-    const int lo = (threadIdx.x - FIRST) * m;
-    const int mine = max(0, min(m, n - lo));
-    uint32_t key[M];
-#pragma unroll
-    for (int i = 0; i < M; ++i) key[i] = i < mine ? keys[lo + i] : 0u;
-    return threshold_topk_regs<NT, M, BAR, FIRST>(key, lo, 1, mine, k, out, w);
 }
 
 // ----------------------------------------------------- per-thread copies --

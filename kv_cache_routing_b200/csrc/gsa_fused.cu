@@ -76,7 +76,7 @@ constexpr uint32_t SM_P = SM_Q + 2 * 4096;           // 2 x 4 KiB: P^T [16 heads
 constexpr uint32_t SM_WMAX = SM_P + 2 * 4096;        // [2][4 warps][16] floats
 constexpr uint32_t SM_LRED = SM_WMAX + 2 * 4 * 16 * 4;
 constexpr uint32_t SM_TOPK = SM_LRED + 4 * 16 * 4;   // selection scratch
-constexpr uint32_t SM_MISC = SM_TOPK + 2048;         // a threshold selection's positions [<= 32]
+constexpr uint32_t SM_MISC = SM_TOPK + 2048;         // a threshold selection's positions [<= 32], or a radix select's bitmaps [2][<= 128]
 constexpr uint32_t SM_SCORE = SM_MISC + 1024;        // key stretch: this CTA's routing scores
 constexpr int kScoreCap = 3072;                      // scores kept in shared memory
 constexpr uint32_t SM_SEL = SM_SCORE;                // unfold stretch: the row's selection [kSelCap]
@@ -778,9 +778,12 @@ __device__ __forceinline__ uint32_t key_of_bits(uint32_t bits, int kind) {
 }
 
 // Thread t takes positions t, t + NU, t + 2 NU, ...: every warp-wide load is
-// one contiguous line.
-template <int U>
-__device__ __forceinline__ bool threshold_u(const void* src, int kind, int n, int k, int32_t* res, uint32_t* w) {
+// one contiguous line.  k <= 32: the threshold selection; otherwise, or when
+// equal keys flood the threshold's bound, the radix select on the same
+// registers.
+template <int U, class Emit>
+__device__ __forceinline__ void select_regs(const void* src, int kind, int n, int k, int32_t* tmp, uint32_t* w,
+                                            uint32_t* bm, Emit emit) {
     const int lo = utid();
     const int mine = lo < n ? (n - lo + NU - 1) / NU : 0;
     uint32_t key[U];
@@ -788,17 +791,22 @@ __device__ __forceinline__ bool threshold_u(const void* src, int kind, int n, in
     for (int i = 0; i < U; ++i) key[i] = i < mine ? load_key_bits(src, kind, lo + i * NU) : 0u;   // all loads first
 #pragma unroll
     for (int i = 0; i < U; ++i) key[i] = i < mine ? key_of_bits(key[i], kind) : 0u;
-    return threshold_topk_regs<NU, U, BAR_UNF, UFIRST>(key, lo, NU, mine, k, res, w);
+    if (k <= 32 && threshold_topk_regs<NU, U, BAR_UNF, UFIRST>(key, lo, NU, mine, k, tmp, w)) {
+        for (int r = utid(); r < k; r += NU) emit(r, tmp[r]);
+        return;
+    }
+    radix_topk_regs<NU, U, BAR_UNF, UFIRST>(key, mine, n, k, w, bm, emit);
 }
 
 // Exact top-k of n keys (read from `src` as `kind` says), ties to the lower
 // position, the selected positions in ascending order: into res[0..k), or,
-// when `ck` is given, as candidates (ck[r] = key, ci[r] = pos0 + pos).  k <= 32
-// and n <= 32 NU: the threshold selection with every thread's block of keys in
-// registers; otherwise, or when equal keys flood the bound, the radix select
-// reading the keys where they are.  Neither res nor the scratch may overlap
-// the keys.  Every caller goes through this one body (the unfold path runs
-// once per launch, cold, so its code is kept small).
+// when `ck` is given, as candidates (ck[r] = key, ci[r] = pos0 + pos).  n <= 32
+// NU: every thread's keys in registers (all loaded at once), the threshold
+// selection for k <= 32, else the radix select on those registers (also when
+// equal keys flood the threshold's bound); larger n: the radix select reading
+// the keys where they are.  Neither res nor the scratch may overlap the keys.
+// Every caller goes through this one body (the unfold path runs once per
+// launch, cold, so its code is kept small).
 __device__ __forceinline__ void unfold_topk(const void* src, int kind, int n, int k, int32_t* res, uint32_t* w,
                                             int32_t* tmp, uint32_t* ck, int32_t* ci, int pos0) {
     auto emit = [&](int r, int pos) {
@@ -812,11 +820,12 @@ __device__ __forceinline__ void unfold_topk(const void* src, int kind, int n, in
     if (k >= n) {
         for (int i = utid(); i < n; i += NU) emit(i, i);
     } else {
-        bool done = false;
-        if (k <= 32 && n <= 16 * NU) done = threshold_u<16>(src, kind, n, k, tmp, w);
-        else if (k <= 32 && n <= 32 * NU) done = threshold_u<32>(src, kind, n, k, tmp, w);
-        if (done) {
-            for (int r = utid(); r < k; r += NU) emit(r, tmp[r]);
+        // the radix select's bitmaps (2 ceil(n / 32) words) share the tmp buffer
+        uint32_t* bm = reinterpret_cast<uint32_t*>(tmp);
+        if (n <= 16 * NU) {
+            select_regs<16>(src, kind, n, k, tmp, w, bm, emit);
+        } else if (n <= 32 * NU) {
+            select_regs<32>(src, kind, n, k, tmp, w, bm, emit);
         } else {
             block_topk<NU, BAR_UNF, UFIRST>(
                 n, k, [&](int i) { return key_of_bits(load_key_bits(src, kind, i), kind); }, emit, w);

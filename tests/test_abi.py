@@ -101,3 +101,20 @@ def test_prefill_validation():
     with pytest.raises(gsa.GsaError) as e:
         gsa.gsa_gist_prefill(gsa.prefill_desc(1, 8, 2, 96, 4, 16), 1 << 20, 1 << 21, 1 << 22, 1 << 23, stream=0)
     assert e.value.status == gsa.GSA_ERR_SHAPE
+
+
+def test_launch_counts_follow_the_path():
+    """One launch on the tensor-core path (bf16, d = 128); the CUDA-core path
+    runs a gist pass and an unfold pass (one when there are no gists), and its
+    hierarchy three passes; -1 for an invalid descriptor.  Host only."""
+    assert gsa.gsa_decode_launch_count(_desc()) == 1
+    assert gsa.gsa_decode_launch_count(_desc(dtype=gsa.GSA_F32)) == 2
+    assert gsa.gsa_decode_launch_count(_desc(head_dim=64)) == 2
+    assert gsa.gsa_decode_launch_count(_desc(head_dim=64, n_chunks=0, top_k=0)) == 1
+    with pytest.raises(gsa.GsaError):
+        gsa.gsa_decode_launch_count(_desc(head_dim=96))
+    l1 = _desc(n_chunks=160, top_k=8)
+    assert gsa.gsa_hier_launch_count(gsa.hier_desc(l1, 10, 16, 2)) == 1
+    assert gsa.gsa_hier_launch_count(gsa.hier_desc(_desc(n_chunks=160, top_k=8, dtype=gsa.GSA_F32), 10, 16, 2)) == 3
+    with pytest.raises(gsa.GsaError):
+        gsa.gsa_hier_launch_count(gsa.hier_desc(l1, 11, 16, 2))

@@ -95,6 +95,24 @@ def test_exact_ties_go_to_lowest_index():
     assert np.all(sc == sc[..., :1])
 
 
+@pytest.mark.parametrize("n,c,k", [(700, 4, 9), (3000, 8, 100), (4096, 8, 32), (6000, 8, 40), (16384, 8, 256)])
+def test_repeated_keys_ties_go_to_lowest_index(n, c, k):
+    """Gist keys repeat with period 7, so every score value is shared by ~n/7
+    gists and the k-th largest falls inside a run of ties: the selection is
+    the k largest with the lowest indices among equals (integer work on the
+    GPU's own scores, compared exactly), across the selection's size classes
+    (small k, large k, all keys in registers or not)."""
+    s = DecodeShape(1, 8, 2, 128, n, c, k, 16, "bf16", ALL_GISTS)
+    x = synth.decode_inputs(s, 81)
+    x.k_gist[...] = x.k_gist[:, :, np.arange(n) % 7, :]
+    idx, sc, _ = gpu_decode_step(s, upload(x))
+    rows = sc.reshape(s.rows, n)
+    for r in range(s.rows):
+        assert np.all(rows[r] == rows[r][np.arange(n) % 7])
+        want = np.sort(np.lexsort((np.arange(n), -rows[r]))[:k])
+        assert idx.reshape(s.rows, k)[r].tolist() == want.tolist()
+
+
 def test_strong_needles_always_selected():
     s = DecodeShape(4, 32, 8, 128, 4096, 16, 16, 64, "bf16", ALL_GISTS, n_needles=16,
                     needle_alpha=3 * np.sqrt(128))

@@ -433,30 +433,65 @@ __device__ bool threshold_topk_regs(const uint32_t (&key)[M], int lo, int step, 
 }
 
 // Exact top-k (any 0 < k < n) of n keys held in registers: thread t holds
-// positions t + i * NT for i < mine (key[i]).  Radix select on 8-bit digits
-// from the top: each pass counts, in a 256-bin histogram (shared-memory
-// atomics), the keys that share the prefix found so far, and the digit on
-// which the k-th largest falls joins the prefix.  The k-th largest key T is then known; the keys above T are
-// selected, and of the keys equal to T the lowest positions (a popcount scan
-// of a bitmap in position order).  emit(r, pos) for the selected positions,
-// ascending.  Scratch: w >= 256 + 16 + NT / 32 + 1 words; bm >= 2 * ceil(n /
-// 32) words.  All NT threads of the group call it.
+// positions t + i * NT for i < mine (key[i]).  Radix select on digits of up
+// to 8 bits from the top, starting below the bits every key shares: each pass
+// counts, in a 256-bin histogram (shared-memory atomics), the keys that share
+// the prefix found so far, and the digit on which the k-th largest falls
+// joins the prefix.  The k-th largest key T is then known; the keys above T
+// are selected, and of the keys equal to T the lowest positions (a popcount
+// scan of a bitmap in position order).  emit(r, pos) for the selected positions,
+// ascending.  Scratch: w >= 288 + 2 NT / 32 words; bm >= max(256, 2 ceil(n /
+// 32)) words (a histogram during the passes, then the bitmaps).  All NT
+// threads of the group call it.
 template <int NT, int U, int BAR = 0, int FIRST = 0, class Emit>
 __device__ void radix_topk_regs(const uint32_t (&key)[U], int mine, int n, int k, uint32_t* w, uint32_t* bm,
                                 Emit emit) {
     const int tid = threadIdx.x - FIRST, lane = tid & 31, warp = tid >> 5;
-    uint32_t* hist = w;          // 256
+    constexpr int NW = NT / 32;
     uint32_t* ctl = w + 256;     // [0] digit, [1] keys above it
     uint32_t* scan = w + 272;    // NT / 32 + 1
-    uint32_t prefix = 0, pmask = 0, kk = (uint32_t)k;
+    uint32_t* mm = w + 288;      // [NW] smallest, [NW] largest key of each warp
+    // the leading bits that every key shares (those of the smallest and the
+    // largest key) need no pass: score keys share their sign and most of
+    // their exponent
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+        if (i < mine) {
+            kmin = min(kmin, key[i]);
+            kmax = max(kmax, key[i]);
+        }
+    }
+    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+    if (lane == 0) {
+        mm[warp] = kmin;
+        mm[NW + warp] = kmax;
+    }
+    for (int i = tid; i < 256; i += NT) w[i] = 0;
+    group_sync<NT, BAR>();
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+        kmin = min(kmin, mm[i]);
+        kmax = max(kmax, mm[NW + i]);
+    }
+    const int common = __clz(kmin ^ kmax);   // 32 when every key is the same
+    uint32_t pmask = common > 0 ? (0xFFFFFFFFu << (32 - common)) : 0u;
+    uint32_t prefix = kmax & pmask, kk = (uint32_t)k;
+    // digits of up to 8 bits below the common prefix; the two histograms (w
+    // and bm) alternate, so the next one is cleared during this pass
+    int left = 32 - common, par = 0;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += NT) hist[i] = 0;
-        group_sync<NT, BAR>();
+    while (left > 0) {
+        const int width = min(8, left), shift = left - width;
+        const uint32_t dmask = (1u << width) - 1u;
+        uint32_t* hist = par ? bm : w;
+        uint32_t* next = par ? w : bm;
 #pragma unroll
         for (int i = 0; i < U; ++i) {
-            if (i < mine && (key[i] & pmask) == prefix) atomicAdd(&hist[(key[i] >> shift) & 255u], 1u);
+            if (i < mine && (key[i] & pmask) == prefix) atomicAdd(&hist[(key[i] >> shift) & dmask], 1u);
         }
+        for (int i = tid; i < 256; i += NT) next[i] = 0;
         group_sync<NT, BAR>();
         if (warp == 0) {
             // lane l owns bins 255-8l .. 248-8l (descending)
@@ -483,10 +518,13 @@ __device__ void radix_topk_regs(const uint32_t (&key)[U], int mine, int n, int k
             }
         }
         group_sync<NT, BAR>();
+        // (ctl is next written after the following pass's first barrier,
+        // which every thread reaches only after reading it here)
         prefix |= ctl[0] << shift;
-        pmask |= 255u << shift;
+        pmask |= dmask << shift;
         kk -= ctl[1];
-        group_sync<NT, BAR>();
+        left -= width;
+        par ^= 1;
     }
     // T = prefix; take every key > T and the kk lowest positions of the keys == T
     const int nw = (n + 31) >> 5;

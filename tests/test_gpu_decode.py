@@ -95,20 +95,22 @@ def test_exact_ties_go_to_lowest_index():
     assert np.all(sc == sc[..., :1])
 
 
-@pytest.mark.parametrize("n,c,k", [(700, 4, 9), (3000, 8, 100), (4096, 8, 32), (6000, 8, 40), (16384, 8, 256)])
-def test_repeated_keys_ties_go_to_lowest_index(n, c, k):
-    """Gist keys repeat with period 7, so every score value is shared by ~n/7
-    gists and the k-th largest falls inside a run of ties: the selection is
-    the k largest with the lowest indices among equals (integer work on the
-    GPU's own scores, compared exactly), across the selection's size classes
-    (small k, large k, all keys in registers or not)."""
+@pytest.mark.parametrize("n,c,k,period", [(700, 4, 9, 7), (3000, 8, 100, 7), (4096, 8, 32, 7), (6000, 8, 40, 7),
+                                          (16384, 8, 256, 7), (3000, 8, 100, 1), (2000, 16, 64, 2)])
+def test_repeated_keys_ties_go_to_lowest_index(n, c, k, period):
+    """Gist keys repeat with a short period, so every score value is shared by
+    ~n/period gists and the k-th largest falls inside a run of ties (period 1:
+    every score is the same): the selection is the k largest with the lowest
+    indices among equals (integer work on the GPU's own scores, compared
+    exactly), across the selection's size classes (small k, large k, all keys
+    in registers or not)."""
     s = DecodeShape(1, 8, 2, 128, n, c, k, 16, "bf16", ALL_GISTS)
     x = synth.decode_inputs(s, 81)
-    x.k_gist[...] = x.k_gist[:, :, np.arange(n) % 7, :]
+    x.k_gist[...] = x.k_gist[:, :, np.arange(n) % period, :]
     idx, sc, _ = gpu_decode_step(s, upload(x))
     rows = sc.reshape(s.rows, n)
     for r in range(s.rows):
-        assert np.all(rows[r] == rows[r][np.arange(n) % 7])
+        assert np.all(rows[r] == rows[r][np.arange(n) % period])
         want = np.sort(np.lexsort((np.arange(n), -rows[r]))[:k])
         assert idx.reshape(s.rows, k)[r].tolist() == want.tolist()
 

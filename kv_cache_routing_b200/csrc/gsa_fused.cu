@@ -60,6 +60,7 @@ constexpr int NU = 128;                      // unfold warps 6-9: selection, row
 constexpr int UFIRST = NT;                   // first unfold thread
 constexpr int NTHR = NT + NU;
 constexpr int BAR_SOFT = 1, BAR_UNF = 2, BAR_PIPE = 3;   // named barriers (0 is the whole block)
+constexpr int BAR_KEYS = 4;                  // the key stretch is done (streaming warps arrive, unfold warps wait)
 constexpr int NSL = 6;                       // ring slots
 constexpr int D = 128;
 constexpr int TILE = 128;
@@ -1258,11 +1259,9 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         rk.npre = min(n2, NSL);   // the first value tiles follow the keys without a gap
         rk.vseq0 = n1;
         run_pipeline<G>(p, cx, rk);
-    }
-    __threadfence();
-    __syncthreads();
-
-    if (cx.warp < 6) {
+        // the scores are written (global and shared memory): hand them to the
+        // unfold warps, which publish them, and go on without waiting
+        asm volatile("bar.arrive %0, %1;" ::"n"(BAR_KEYS), "n"(NTHR) : "memory");
         // ------------------------------------------------ value stretch --
         Run rv{};
         rv.kind = RUN_V;
@@ -1295,6 +1294,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
     } else {
         // ----------------------------------------------- unfold warps --
         const bool lead = utid() == 0;
+        asm volatile("bar.sync %0, %1;" ::"n"(BAR_KEYS), "n"(NTHR) : "memory");
         if (p.do_topk && !p.sel_direct) {
             // local top-k of every segment, from the scores this CTA kept
             int ntiles = 0;
@@ -1320,12 +1320,16 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                 local_topk(p, cx.base, r, g0, g1, sfirst * TILE, off, fits);
                 sfirst += (g1 - g0 + TILE - 1) / TILE;
             }
-            __threadfence();
             usync();
         }
-        // scores (and candidates) of every row this CTA met are out
-        if (lead)
+        // scores (and candidates) of every row this CTA met are out.  The
+        // lead's fence is cumulative: it orders before the counters the
+        // streaming warps' scores and the unfold warps' candidates, which the
+        // barriers above made visible to it.
+        if (lead) {
+            __threadfence();
             for (int r = row_first; r <= row_last; ++r) atomicAdd(p.kdone + r, 1u);
+        }
         int gseq = gseq0, runs = 0;
         for (int it = c; it < p.items; it += p.grid) {
             const int row = it / p.cb, j = it % p.cb;
@@ -1384,12 +1388,14 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
     }
 
     // ---------------------------------------------------------- tickets --
-    // every partial of this CTA is out: count each on its row's ticket
-    __threadfence();
+    // every partial of this CTA is out: count each on its row's ticket (each
+    // counting thread's fence is cumulative over the partials the barrier
+    // made visible to it)
     __syncthreads();
     {
         const int nA = row_last - row_first + 1;
         const int nI = c < p.items ? (p.items - 1 - c) / p.grid + 1 : 0;
+        if (threadIdx.x < nA + nI) __threadfence();
         for (int q = threadIdx.x; q < nA + nI; q += NTHR) {
             const int row = q < nA ? row_first + q : (c + (q - nA) * p.grid) / p.cb;
             atomicAdd(p.cnt + row, 1u);

@@ -1,7 +1,8 @@
 // GSA decode step on the 5th-generation tensor cores (bf16, d = 128).
 //
 // One persistent launch per decode step: at most 148 CTAs, one per SM, all
-// resident at once.  A row is one (b, kv-head).  Every CTA runs three stretches:
+// resident at once.  A row is one (b, kv-head).  Every CTA runs three stretches,
+// the last two side by side:
 //
 //  keys     Its Stream-K share of the phase-A units, a contiguous range of the
 //           units of all rows (a unit is a 128-gist tile or a 128-token tail
@@ -9,19 +10,20 @@
 //           routing score (summed over the G heads of the group) and the scaled
 //           attention logits, which stay in tensor memory (TMEM).  A maximal
 //           run of one row's units is a segment; its exact per-head maximum M
-//           goes to TMEM too.  The CTA then counts itself done on every row it
-//           met.
-//  unfold   Its phase-B item(s): once every CTA that met the item's row has
-//           counted itself done (a bounded wait on the row's counter), the
-//           row's top-k is taken, the selected chunks' raw tokens (and in
-//           SELECTED_PAIRS mode the selected gists) are gathered by every
-//           thread's cp.async into 128-row tiles and attended with an online
-//           softmax, leaving one partial.  The producer warp has meanwhile
-//           issued the first V tiles of the next stretch, so the SM keeps
-//           streaming while the selection runs.
-//  values   V of the units whose logits the key stretch kept: P = 2^(x - M)
-//           against the segment's exact maximum (nothing is ever rescaled),
-//           O^T += V^T . P^T, one partial (M, L, O) per segment.
+//           goes to TMEM too.  The streaming warps then hand the stretch to the
+//           unfold warps through a named barrier, and those count the CTA done
+//           on every row it met.
+//  values   (streaming warps) V of the units whose logits the key stretch
+//           kept: P = 2^(x - M) against the segment's exact maximum (nothing
+//           is ever rescaled), O^T += V^T . P^T, one partial (M, L, O) per
+//           segment.  Then the gathered tiles of the CTA's unfold items, with
+//           an online softmax, one partial per item.
+//  unfold   (unfold warps, beside the value stretch) Its phase-B item(s):
+//           once every CTA that met the item's row has counted itself done (a
+//           bounded wait on the row's counter), the row's top-k is taken, and
+//           the selected chunks' raw tokens (and in SELECTED_PAIRS mode the
+//           selected gists) are gathered into 128-row tiles in the ring: whole
+//           chunks by TMA boxes, other rows by cp.async.
 // Every partial is counted on its row's ticket; the row's first unfold CTA
 // waits (bounded) for the full count and merges the partials (log-sum-exp)
 // into out.
@@ -32,7 +34,8 @@
 //
 // Warp roles: warps 0-3 run the softmax (thread t owns key row t of a tile and,
 // for O^T, TMEM lane t = output dimension t); warp 4 issues the loads; warp 5
-// owns TMEM and issues the MMAs.  Shared memory holds a ring of six 32 KiB
+// owns TMEM and issues the MMAs; warps 6-9 (the unfold warps) select, build
+// the row tables and issue the gathers.  Shared memory holds a ring of six 32 KiB
 // slots; a key-stretch tile takes one (K), a value-stretch tile one (V), a
 // gathered tile two (K, V).  Per tile:
 //   S   = K_tile . Q^T     M = 128 keys, N = 16 (G heads, rest zero), K = d

@@ -29,9 +29,12 @@
  *        out      [B][Hq][d]   same dtype as q
  *  - Element type: GSA_F32 or GSA_BF16 for q and every K/V tensor alike;
  *    all accumulation is fp32; the output is rounded once (RNE).
- *  - The library allocates nothing and keeps no state between calls.  Work is
- *    enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and
- *    runs asynchronously; no entry point synchronises.
+ *  - The library allocates nothing.  Between calls it keeps only small caches
+ *    per host thread: launch plans and TMA descriptors, which are pure
+ *    functions of the descriptor and the buffer addresses.  So calls from
+ *    several host threads need no locking.  Work is enqueued on `stream` (a
+ *    cudaStream_t; NULL = legacy default stream) and runs asynchronously; no
+ *    entry point synchronises.
  *  - Workspace: entry points that take `ws` need a device buffer of at least
  *    the size the matching gsa_*_workspace_size() returns, 256-byte aligned.
  *    It must be ZERO-FILLED ONCE after allocation (e.g. cudaMemset); each call

@@ -115,6 +115,26 @@ def test_repeated_keys_ties_go_to_lowest_index(n, c, k, period):
         assert idx.reshape(s.rows, k)[r].tolist() == want.tolist()
 
 
+@pytest.mark.parametrize("n,c,k", [(3000, 8, 100), (2048, 16, 16), (6000, 8, 300)])
+def test_all_positive_scores_select_exactly(n, c, k):
+    """Non-negative queries and gist keys near 1 make every score positive and
+    close to the others: the selection's keys share their leading 12-13 bits,
+    so the radix passes start below that prefix and end on a digit narrower
+    than 8 bits.  The selection must still be the exact top-k of the GPU's own
+    scores (integer work, compared exactly)."""
+    s = DecodeShape(1, 8, 2, 128, n, c, k, 16, "bf16", ALL_GISTS)
+    x = synth.decode_inputs(s, 82)
+    # bf16 values are held as their 16-bit patterns: clearing the sign bit is |x|
+    x.q[...] = x.q & 0x7FFF
+    x.k_gist[...] = synth.round_to(1.0 + 0.05 * np.abs(synth.widen(x.k_gist, "bf16")), "bf16")
+    idx, sc, _ = gpu_decode_step(s, upload(x))
+    rows = sc.reshape(s.rows, n)
+    assert np.all(rows > 0)
+    for r in range(s.rows):
+        want = np.sort(np.lexsort((np.arange(n), -rows[r]))[:k])
+        assert idx.reshape(s.rows, k)[r].tolist() == want.tolist()
+
+
 def test_strong_needles_always_selected():
     s = DecodeShape(4, 32, 8, 128, 4096, 16, 16, 64, "bf16", ALL_GISTS, n_needles=16,
                     needle_alpha=3 * np.sqrt(128))

@@ -118,3 +118,18 @@ def test_launch_counts_follow_the_path():
     assert gsa.gsa_hier_launch_count(gsa.hier_desc(_desc(n_chunks=160, top_k=8, dtype=gsa.GSA_F32), 10, 16, 2)) == 3
     with pytest.raises(gsa.GsaError):
         gsa.gsa_hier_launch_count(gsa.hier_desc(l1, 11, 16, 2))
+
+
+def test_every_benchmark_decode_workload_takes_the_one_launch_path():
+    """The Llama-shaped step, the six compression-ratio sweeps and the
+    1M-token hierarchy all fit the tensor-core path (TMEM columns, selection
+    size, one children tile and one raw tile), so none silently falls back to
+    the CUDA-core passes.  Host only."""
+    import synth
+    from gsa_check import desc_of
+    for name, w in synth.WORKLOADS.items():
+        if isinstance(w, synth.DecodeShape) and w.dtype == "bf16" and w.head_dim == 128:
+            assert gsa.gsa_decode_launch_count(desc_of(w)) == 1, name
+        elif isinstance(w, synth.HierShape):
+            hd = gsa.hier_desc(desc_of(w.l1), w.n_l2, w.group, w.top_k2)
+            assert gsa.gsa_hier_launch_count(hd) == 1, name

@@ -68,6 +68,40 @@ def test_score_error_bound_covers_fp32_evaluation():
                 assert abs(float(acc) - s[b, hk, j]) <= eps[b, hk]
 
 
+def test_score_error_bound_closed_form_by_hand():
+    """Higham's inner-product bound gamma_n * sum |q_i k_i| evaluated by hand
+    for inputs of known sign and magnitude.
+
+    G = 1, d = 4, q = (1, -2, 3, -4); gist 0 has k = (1, 1, 1, 1) (sum of
+    |q_i k_i| = 10), gist 1 has k = (0.5, -0.5, 0.5, -0.5) (sum 5).  The row
+    bound is the larger one: n = G d = 4 products, u = 2^-24,
+        gamma_4 = 4u / (1 - 4u) = 2.384185791015625e-07 / 0.9999997615814209
+                = 2.3841863594e-07,
+        eps = 10 * gamma_4 = 2.3841863594e-06.
+    A bound built with another n, or without the absolute values, misses it."""
+    q = np.array([[[1.0, -2.0, 3.0, -4.0]]])
+    kg = np.array([[[[1.0, 1.0, 1.0, 1.0], [0.5, -0.5, 0.5, -0.5]]]])
+    eps = oracle.score_error_bound(q, kg)
+    assert eps.shape == (1, 1)
+    assert eps[0, 0] == pytest.approx(2.3841863594e-06, rel=1e-9)
+
+
+def test_score_error_bound_counts_every_product_of_the_group():
+    """The number of products in a routing score is G * d: with all entries
+    equal to 1 the bound is n * gamma_n, n = G * d, so (G = 2, d = 64) and
+    (G = 1, d = 128) give the same bound, and doubling d at G = 1 multiplies
+    it by 2 * gamma_128 / gamma_64, just above 4 (hand value 4.00001525890...)."""
+    def bound(G, d):
+        q = np.ones((1, G, d))
+        kg = np.ones((1, 1, 3, d))
+        return oracle.score_error_bound(q, kg)[0, 0]
+    assert bound(2, 64) == pytest.approx(bound(1, 128), rel=1e-12)
+    # 128 gamma_128 / (64 gamma_64) = 2 * (128u / (1 - 128u)) / (64u / (1 - 64u)) = 4 (1 - 64u) / (1 - 128u)
+    assert bound(1, 128) / bound(1, 64) == pytest.approx(4.0000152589055, rel=1e-11)
+    # n = 64: 64u = 3.814697265625e-06, gamma_64 = 3.8147118...e-06, 64 gamma_64 = 2.44141556...e-04
+    assert bound(1, 64) == pytest.approx(2.4414155633e-04, rel=1e-8)
+
+
 # ------------------------------------------------------------- selection ----
 def test_topk_worked_example(golden):
     rows = dict(r.split(None, 1) for r in golden("topk_slide10.txt"))
@@ -104,6 +138,20 @@ def test_topk_gap():
     s = np.array([[0.1, 0.8, 0.7, 0.2]])
     assert oracle.topk_gap(s, 2)[0] == pytest.approx(0.5)
     assert math.isinf(oracle.topk_gap(s, 4)[0])
+
+
+def test_topk_gap_ties_and_empty_selection():
+    """A tie across the k-th / (k+1)-th place leaves no margin (gap 0, the row
+    is undecidable at any precision); a tie inside the selected set does not
+    matter; k = 0 selects nothing and has no boundary (gap infinite)."""
+    s = np.array([[0.5, 0.2, 0.5, 0.5],        # k = 2: 0.5, 0.5 | 0.5, 0.2 -> gap 0
+                  [0.3, 0.5, 0.5, 0.1]])       # k = 2: 0.5, 0.5 | 0.3      -> gap 0.2
+    gap = oracle.topk_gap(s, 2)
+    assert gap[0] == 0.0
+    assert gap[1] == pytest.approx(0.2)
+    assert math.isinf(oracle.topk_gap(s, 0)[0]) and math.isinf(oracle.topk_gap(s, 0)[1])
+    # the tie at the boundary still resolves to the lower indices
+    assert oracle.topk(s, 2)[0].tolist() == [0, 2]
 
 
 # -------------------------------------------------------------- attention ---

@@ -47,7 +47,11 @@
  *    crosses the ABI.  Device-side anomalies (an out-of-range chunk index
  *    passed to gsa_unfold_attn, an expired bounded wait) never fault: the
  *    kernel clamps the index into range (or abandons the wait) and ORs a flag
- *    into the workspace error word, which gsa_workspace_error() reads back.
+ *    into an error word.  Entry points that take a workspace use the word at
+ *    its start, read back by gsa_workspace_error(); the others
+ *    (gsa_score, gsa_gist_prefill, gsa_decode_step_noalloc) use words of
+ *    the library, read back and cleared by gsa_device_error().  A call whose
+ *    wait expired has left unusable results in its outputs.
  */
 #ifndef GSA_H_
 #define GSA_H_
@@ -185,8 +189,12 @@ gsa_status gsa_gist_prefill(const gsa_prefill_desc* desc, const void* q, const v
  *    are rejected with GSA_ERR_WORKSPACE.
  *  - The first call on a device looks up the array's device address for that
  *    device; make that first call before any stream capture on the device.
+ *    The address is looked up again if the device's context changed (after a
+ *    device reset), so that call too must come before any capture.
  *  - Each call clears the scratch words that must start at zero
- *    (cudaMemsetAsync on `stream`), then runs the decode step in it.
+ *    (cudaMemsetAsync on `stream`), then runs the decode step in it.  The
+ *    array's error word is not cleared by the calls: it collects the flags
+ *    of every call until gsa_device_error() reads and clears it.
  *  - All calls share the one array: calls whose work overlaps on the GPU
  *    (different streams, or different host threads) race and corrupt each
  *    other's results.  Serialise them on one stream.
@@ -211,6 +219,24 @@ int gsa_hier_launch_count(const gsa_hier_desc* desc);
 #define GSA_WS_ERR_TIMEOUT 1u
 #define GSA_WS_ERR_INDEX 2u
 gsa_status gsa_workspace_error(const void* ws, uint32_t* flags_out, void* stream);
+
+/* Reads (synchronously, on `stream`) and clears the library's own error
+ * words on the current device: the one of the entry points without a
+ * workspace (gsa_score), the prefill's (gsa_gist_prefill: a work item whose
+ * bounded wait expired was abandoned and its rows of out / lse are not
+ * valid) and the scratch array's of gsa_decode_step_noalloc.  flags_out
+ * (nullable) receives the OR of the GSA_WS_ERR_* flags found; returns
+ * GSA_ERR_TIMEOUT if a bounded wait expired, GSA_ERR_ARG if an index was out
+ * of range, else GSA_OK.  Calls that overlap it on the GPU may set a flag
+ * after it was read; serialise them on `stream` to attribute the flags.   */
+gsa_status gsa_device_error(uint32_t* flags_out, void* stream);
+
+/* Diagnostics: sets the time limit (ns) of the waits in which one CTA of a
+ * decode launch waits for others (a row's key counter, its ticket), on the
+ * current device; 0 restores the default of 2 s.  When a wait runs out the
+ * kernel flags GSA_WS_ERR_TIMEOUT and finishes its launch normally.  Meant
+ * for tests of that path; synchronous; do not call while a launch runs. */
+gsa_status gsa_set_wait_limit_ns(uint64_t ns);
 
 /* Static description of a status code. */
 const char* gsa_status_string(gsa_status status);

@@ -24,7 +24,7 @@ GSA_WS_ERR_TIMEOUT, GSA_WS_ERR_INDEX = 1, 2
 EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", "gsa_topk",
            "gsa_unfold_attn", "gsa_decode_step", "gsa_hier_decode", "gsa_gist_prefill",
            "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count",
-           "gsa_hier_launch_count")
+           "gsa_hier_launch_count", "gsa_device_error", "gsa_set_wait_limit_ns")
 
 
 class GsaError(RuntimeError):
@@ -69,6 +69,8 @@ def _signatures():
         "gsa_hier_decode": (st, [ph] + [vp] * 13 + [sz, vp]),
         "gsa_gist_prefill": (st, [pp, vp, vp, vp, vp, vp, vp]),
         "gsa_workspace_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
+        "gsa_device_error": (st, [ctypes.POINTER(ctypes.c_uint32), vp]),
+        "gsa_set_wait_limit_ns": (st, [ctypes.c_uint64]),
         "gsa_status_string": (ctypes.c_char_p, [st]),
         "gsa_decode_launch_count": (ctypes.c_int, [pd]),
         "gsa_hier_launch_count": (ctypes.c_int, [ph]),
@@ -224,3 +226,19 @@ def gsa_workspace_error(ws, stream=None) -> int:
     flags = ctypes.c_uint32(0)
     lib().gsa_workspace_error(_ptr(ws), ctypes.byref(flags), _stream(stream))
     return int(flags.value)
+
+
+def gsa_device_error(stream=None) -> int:
+    """Reads and clears the library's own device error words (entry points
+    without a workspace, the prefill, the no-allocation scratch): 0 or an OR
+    of GSA_WS_ERR_* flags."""
+    flags = ctypes.c_uint32(0)
+    st = lib().gsa_device_error(ctypes.byref(flags), _stream(stream))
+    if st not in (GSA_OK, GSA_ERR_TIMEOUT, GSA_ERR_ARG):
+        raise GsaError(st, "gsa_device_error")
+    return int(flags.value)
+
+
+def gsa_set_wait_limit_ns(ns: int):
+    """Diagnostics: limit of the cross-CTA waits of a decode launch (0: default)."""
+    _check(lib().gsa_set_wait_limit_ns(int(ns)), "gsa_set_wait_limit_ns")

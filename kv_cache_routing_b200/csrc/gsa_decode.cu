@@ -16,7 +16,9 @@
 // routing signals, selective unfolding, hybrid attention; Taki-lab slides
 // page 6 (score every gist, take top-k, restore chunks with their gists) and
 // page 17 (AG+SR / SG+SR context rules).
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstring>
@@ -792,17 +794,40 @@ gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void*
 constexpr size_t kStaticWsBytes = size_t(8) << 20;   // 8 MiB
 static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
 
-// Device address of g_static_ws on each device, resolved once per device with
-// that device current.  (In host code the symbol itself is only a stand-in.)
-static void* static_ws_address(int device) {
+// The CUDA context current on this thread (driver entry point; null if none).
+static CUcontext current_context() {
+    static std::once_flag once;
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    });
+    CUcontext c = nullptr;
+    if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// Device address of g_static_ws on each device, resolved with that device
+// current the first time it is needed there.  (In host code the symbol itself
+// is only a stand-in.)  The address is kept together with the context it was
+// resolved in: after a device reset the module is loaded again, possibly
+// elsewhere, and the address is resolved anew.
+static void* static_ws_address(int device, bool resolve = true) {
     static std::mutex mu;
     static void* addr[128] = {};
+    static CUcontext ctx[128] = {};
     if (device < 0 || device >= 128) return nullptr;
+    const CUcontext cur = current_context();
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[device] == nullptr) {
+    if (addr[device] == nullptr || ctx[device] != cur) {
+        if (!resolve) return nullptr;
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess) return nullptr;
         addr[device] = p;
+        ctx[device] = cur;
     }
     return addr[device];
 }
@@ -822,9 +847,11 @@ gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, c
     void* ws = static_ws_address(device);
     if (ws == nullptr) return GSA_ERR_CUDA;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
-    // the error word and the tickets (the words before the first data region) must start at zero
+    // the tickets (the words between the error word and the first data region)
+    // must start at zero; the error word is kept until gsa_device_error reads it
     const size_t head = fused_supported(*desc) ? make_fused_plan(*desc).off_scores : make_decode_plan(*desc).off_scores;
-    if (cudaMemsetAsync(ws, 0, head, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + kWsCntOffset, 0, head - kWsCntOffset, strm) != cudaSuccess)
+        return GSA_ERR_CUDA;
     return gsa_decode_step(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, scores_out, out, ws,
                            need, stream);
 }
@@ -838,6 +865,35 @@ int gsa_decode_launch_count(const gsa_decode_desc* desc) {
     if (validate_decode(desc) != GSA_OK) return -1;
     if (fused_supported(*desc)) return 1;
     return (desc->n_chunks > 0 ? 1 : 0) + 1;
+}
+
+gsa_status gsa_device_error(uint32_t* flags_out, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess) return GSA_ERR_CUDA;
+    uint32_t* words[3] = {nullptr, nullptr, nullptr};
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&words[0]), g_err_sink) != cudaSuccess ||
+        prefill_error_word(&words[1]) != cudaSuccess)
+        return GSA_ERR_CUDA;
+    // the scratch array's word, if gsa_decode_step_noalloc has run in this context
+    words[2] = static_cast<uint32_t*>(static_ws_address(device, false));
+    uint32_t got[3] = {0u, 0u, 0u};
+    for (int i = 0; i < 3; ++i) {
+        if (words[i] == nullptr) continue;
+        if (cudaMemcpyAsync(&got[i], words[i], 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+            cudaMemsetAsync(words[i], 0, 4, st) != cudaSuccess)
+            return GSA_ERR_CUDA;
+    }
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GSA_ERR_CUDA;
+    const uint32_t f = got[0] | got[1] | got[2];
+    if (flags_out) *flags_out = f;
+    if (f & kErrTimeout) return GSA_ERR_TIMEOUT;
+    if (f & kErrIndex) return GSA_ERR_ARG;
+    return GSA_OK;
+}
+
+gsa_status gsa_set_wait_limit_ns(uint64_t ns) {
+    return set_cross_cta_wait_limit(ns) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
 gsa_status gsa_workspace_error(const void* ws, uint32_t* flags_out, void* stream) {

@@ -79,13 +79,21 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Wait for phase `parity` of `bar` to complete; after kWaitLimitNs it gives
-// up, ORs kErrTimeout into *err and returns false.
+// SM cycle counter: cheap to read (%globaltimer costs tens of nanoseconds a
+// read), so spin loops keep their time budget in cycles.  The budget of a
+// wait of kWaitLimitNs is taken at 2 cycles per ns (the clock is at most
+// 1.965 GHz), so the limit is reached after at most about that time at the
+// highest clock, and later at lower clocks.
+__device__ __forceinline__ uint64_t sm_cycles() { return (uint64_t)clock64(); }
+constexpr uint64_t kWaitLimitCycles = 2ull * kWaitLimitNs;
+
+// Wait for phase `parity` of `bar` to complete; after kWaitLimitCycles it
+// gives up, ORs kErrTimeout into *err and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
+    const uint64_t t0 = sm_cycles();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (sm_cycles() - t0 > kWaitLimitCycles) {
             atomicOr(err, kErrTimeout);
             return false;
         }

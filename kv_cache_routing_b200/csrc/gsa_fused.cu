@@ -64,7 +64,8 @@ constexpr int UFIRST = NT;                   // first unfold thread
 constexpr int NTHR = NT + NU;
 constexpr int BAR_SOFT = 1, BAR_UNF = 2, BAR_PIPE = 3;   // named barriers (0 is the whole block)
 constexpr int BAR_KEYS = 4;                  // the key stretch is done (streaming warps arrive, unfold warps wait)
-constexpr int NSL = 6;                       // ring slots
+constexpr int NSL = 4;                       // ring slots
+constexpr int PD = 4;                        // P^T buffers (the softmax runs up to PD value tiles ahead of the MMA)
 constexpr int D = 128;
 constexpr int TILE = 128;
 constexpr uint32_t SLOT_BYTES = 32768;       // one 128 x 128 bf16 tensor tile
@@ -76,8 +77,8 @@ constexpr uint32_t kLogitCol = 64;           // first TMEM column of the kept lo
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t SM_STAGE = 0;
 constexpr uint32_t SM_Q = NSL * SLOT_BYTES;          // 2 x 4 KiB: [16 rows][128 B] x 2 K blocks
-constexpr uint32_t SM_P = SM_Q + 2 * 4096;           // 2 x 4 KiB: P^T [16 heads][128 keys]
-constexpr uint32_t SM_WMAX = SM_P + 2 * 4096;        // [2][4 warps][16] floats
+constexpr uint32_t SM_P = SM_Q + 2 * 4096;           // PD x 4 KiB: P^T [16 heads][128 keys]
+constexpr uint32_t SM_WMAX = SM_P + PD * 4096;       // [2][4 warps][16] floats
 constexpr uint32_t SM_LRED = SM_WMAX + 2 * 4 * 16 * 4;
 constexpr uint32_t SM_TOPK = SM_LRED + 4 * 16 * 4;   // selection scratch
 constexpr uint32_t SM_MISC = SM_TOPK + 2048;         // a threshold selection's positions [<= 32], or a radix select's bitmaps [2][<= 128]
@@ -103,7 +104,7 @@ static_assert(SMEM_BYTES <= 227 * 1024, "dynamic shared memory above the per-blo
 struct Bars {
     uint64_t full[NSL], empty[NSL];
     uint64_t s_full[2], s_free[2];
-    uint64_t p_full[2], o_done[2];
+    uint64_t p_full[PD], o_done[PD];
     uint64_t q_ready[2];
     uint64_t gdone;              // a gathered stretch is closed (its row table and children keys are free)
     uint32_t tmem;
@@ -312,18 +313,29 @@ struct PendingPV {
     int vslot, vpar, obuf, first, pj;
 };
 
+// The descriptors of the 8 K-steps differ only in the start-address field
+// (address / 16, bits 0-13), which never carries out for addresses inside
+// shared memory: each is the first one plus a constant.
 __device__ __forceinline__ void issue_pv(Ctx& cx, const PendingPV& r) {
     const uint32_t vs = cx.sbase + SM_STAGE + r.vslot * SLOT_BYTES;
-    const uint32_t pt = cx.sbase + SM_P + (r.pj & 1) * 4096;
+    const uint32_t pt = cx.sbase + SM_P + (r.pj % PD) * 4096;
     const uint32_t dO = cx.tmem + 32 + r.obuf * 16;
+    const uint64_t a0 = tc::sdesc_sw128(vs, 16384, 1024), b0 = tc::sdesc_sw128(pt, 16, 1024);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        tc::mma_bf16(dO, tc::sdesc_sw128(vs + kk * 2048, 16384, 1024),
-                     tc::sdesc_sw128(pt + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), IDESC_PV,
-                     (r.first && kk == 0) ? 0u : 1u);
-    }
-    tc::commit(&cx.bars->o_done[r.pj & 1]);
+    for (int kk = 0; kk < 8; ++kk)
+        tc::mma_bf16(dO, a0 + (uint64_t)(kk * (2048 >> 4)), b0 + (uint64_t)((kk >> 2) * (2048 >> 4) + (kk & 3) * 2),
+                     IDESC_PV, (r.first && kk == 0) ? 0u : 1u);
+    tc::commit(&cx.bars->o_done[r.pj % PD]);
     tc::commit(&cx.bars->empty[r.vslot]);
+}
+
+// S = K_tile . Q^T into TMEM columns dS (8 K-steps of 16 over d = 128).
+__device__ __forceinline__ void issue_s(uint32_t dS, uint32_t ks, uint32_t qb) {
+    const uint64_t a0 = tc::sdesc_sw128(ks, 16, 1024), b0 = tc::sdesc_sw128(qb, 16, 1024);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        tc::mma_bf16(dS, a0 + (uint64_t)((kk >> 2) * (16384 >> 4) + (kk & 3) * 2),
+                     b0 + (uint64_t)((kk >> 2) * (2048 >> 4) + (kk & 3) * 2), IDESC_S, kk > 0 ? 1u : 0u);
 }
 
 __device__ __forceinline__ void mma_run(const Params& p, Ctx& cx, const Run& r) {
@@ -332,14 +344,27 @@ __device__ __forceinline__ void mma_run(const Params& p, Ctx& cx, const Run& r) 
     int i = 0;                // next tile of the stretch
     int j = 0;                // RUN_V: value tiles so far
     int prev_row = -1;
-    uint64_t t_last = global_ns();
+    uint64_t t_last = sm_cycles();
+    int ui = -1;              // the tile whose info `u` holds
+    Tile u{};
     for (;;) {
-        if (r.kind == RUN_V)
-            while (i < r.n && !unit_tile(p, r.u0 + i).attn) ++i;
+        if (r.kind == RUN_V) {
+            while (i < r.n) {
+                if (ui != i) {
+                    u = unit_tile(p, r.u0 + i);
+                    ui = i;
+                }
+                if (u.attn) break;
+                ++i;
+            }
+        }
         if (i >= r.n && head == tail) break;
         bool prog = false;
         if (i < r.n && tail - head < 4) {
-            const Tile u = r.kind == RUN_G ? gathered_tile(r.row, r.t0 + i, i, false) : unit_tile(p, r.u0 + i);
+            if (ui != i) {
+                u = r.kind == RUN_G ? gathered_tile(r.row, r.t0 + i, i, false) : unit_tile(p, r.u0 + i);
+                ui = i;
+            }
             const bool ns = u.row != prev_row;
             if (r.kind == RUN_V) {
                 // the value tile's data is waited for with its P
@@ -365,14 +390,7 @@ __device__ __forceinline__ void mma_run(const Params& p, Ctx& cx, const Run& r) 
                     if (r.kind == RUN_G) tc::fence_async_smem();   // cp.async (generic proxy) writes -> tensor core reads
                     const uint32_t ks = cx.sbase + SM_STAGE + ks_ * SLOT_BYTES;
                     const uint32_t qb = cx.sbase + SM_Q + ((cx.qsegs - 1) & 1) * 4096;
-                    const uint32_t dS = cx.tmem + sb * 16;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        const uint32_t qa = (kk >> 2) * 2048 + (kk & 3) * 32;
-                        tc::mma_bf16(dS, tc::sdesc_sw128(ks + ka, 16, 1024), tc::sdesc_sw128(qb + qa, 16, 1024),
-                                     IDESC_S, kk > 0 ? 1u : 0u);
-                    }
+                    issue_s(cx.tmem + sb * 16, ks, qb);
                     tc::commit(&cx.bars->s_full[sb]);
                     tc::commit(&cx.bars->empty[ks_]);
                     cx.stiles++;
@@ -392,7 +410,7 @@ __device__ __forceinline__ void mma_run(const Params& p, Ctx& cx, const Run& r) 
         }
         if (head != tail) {
             const PendingPV& q = ring[head & 3];
-            if (mbar_test(&cx.bars->p_full[q.pj & 1], (q.pj >> 1) & 1) &&
+            if (mbar_test(&cx.bars->p_full[q.pj % PD], (q.pj / PD) & 1) &&
                 mbar_test(&cx.bars->full[q.vslot], q.vpar)) {
                 tc::fence_after();
                 if (r.kind == RUN_G) tc::fence_async_smem();
@@ -402,10 +420,10 @@ __device__ __forceinline__ void mma_run(const Params& p, Ctx& cx, const Run& r) 
             }
         }
         if (prog) {
-            t_last = global_ns();
+            t_last = sm_cycles();
         } else {
             __nanosleep(20);   // leave the issue slots to the softmax warp sharing this scheduler
-            if (global_ns() - t_last > kWaitLimitNs) {
+            if (sm_cycles() - t_last > kWaitLimitCycles) {
                 atomicOr(p.err, kErrTimeout);
                 return;
             }
@@ -443,7 +461,7 @@ __device__ __forceinline__ void finalize_segment(const Params& p, Ctx& cx, uint3
     float O[G];
     if (cx.had_attn) {
         const int pj = cx.ptiles - 1;
-        mbar_wait(&cx.bars->o_done[pj & 1], (pj >> 1) & 1, p.err);
+        mbar_wait(&cx.bars->o_done[pj % PD], (pj / PD) & 1, p.err);
         tc::fence_after();
         uint32_t r[G];
         tc::ldn<G>(cx.tmem + 32 + obuf * 16 + ((uint32_t)(cx.warp * 32) << 16), r);
@@ -580,9 +598,9 @@ __device__ __forceinline__ void value_tile(const Params& p, Ctx& cx, const Tile&
             cx.l_part[h] = 0.f;
         }
     }
-    const int pj = cx.ptiles, pb = pj & 1;
-    // P^T buffer pb was last read by the P.V of tile pj - 2
-    if (pj >= 2) mbar_wait(&cx.bars->o_done[pb], ((pj - 2) >> 1) & 1, p.err);
+    const int pj = cx.ptiles, pb = pj % PD;
+    // P^T buffer pb was last read by the P.V of tile pj - PD
+    if (pj >= PD) mbar_wait(&cx.bars->o_done[pb], ((pj - PD) / PD) & 1, p.err);
     uint8_t* pt = cx.base + SM_P + pb * 4096;
     const int kb = t >> 6, c16 = (t & 63) >> 3, e = t & 7;
 #pragma unroll
@@ -629,8 +647,8 @@ __device__ __forceinline__ void gathered_softmax(const Params& p, Ctx& cx, const
     mbar_arrive(&cx.bars->s_free[sb]);
     const bool valid = gathered_valid(cx.base, u.lt, t);
     const int pj = cx.ptiles;
-    const int pb = pj & 1;
-    float* wmax = reinterpret_cast<float*>(cx.base + SM_WMAX) + pb * 64;
+    const int pb = pj % PD;
+    float* wmax = reinterpret_cast<float*>(cx.base + SM_WMAX) + (pj & 1) * 64;
     float x[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -658,7 +676,7 @@ __device__ __forceinline__ void gathered_softmax(const Params& p, Ctx& cx, const
     }
     if (need && cx.had_attn) {
         // O^T holds the P.V of this segment's earlier tiles: wait for the last, rescale columns
-        mbar_wait(&cx.bars->o_done[(pj - 1) & 1], ((pj - 1) >> 1) & 1, p.err);
+        mbar_wait(&cx.bars->o_done[(pj - 1) % PD], ((pj - 1) / PD) & 1, p.err);
         tc::fence_after();
         uint32_t o[G];
         const uint32_t ta = cx.tmem + 32 + ((cx.osegs - 1) & 1) * 16 + lane_off;
@@ -669,7 +687,7 @@ __device__ __forceinline__ void gathered_softmax(const Params& p, Ctx& cx, const
         tc::stn<G>(ta, o);
         tc::wait_st();
     }
-    if (pj >= 2) mbar_wait(&cx.bars->o_done[pb], ((pj - 2) >> 1) & 1, p.err);
+    if (pj >= PD) mbar_wait(&cx.bars->o_done[pb], ((pj - PD) / PD) & 1, p.err);
     uint8_t* pt = cx.base + SM_P + pb * 4096;
     const int kb = t >> 6, c16 = (t & 63) >> 3, e = t & 7;
 #pragma unroll
@@ -1016,15 +1034,23 @@ __device__ __forceinline__ void hier_select_children(const Params& p, uint8_t* b
     usync();
 }
 
+// Limit of the cross-CTA waits below (default kWaitLimitNs; a diagnostics
+// setter shortens it so that tests can make such a wait run out).
+__device__ unsigned long long g_cross_wait_ns = kWaitLimitNs;
+
 // Wait (bounded) until counter `ctr` reaches `target`; the writes published
-// before it are then visible to the whole group.
+// before it are then visible to the whole group.  The comparison is
+// wrap-aware (the signed difference), so a counter word that holds a value
+// half the 32-bit range away never reaches the target: the wait then runs
+// out, flags kErrTimeout and the kernel carries on to its normal end.
 template <int GN, int GBAR>
 __device__ __forceinline__ void wait_count(const Params& p, const uint32_t* ctr, uint32_t target, bool leader) {
     if (leader) {
         const uint64_t t0 = global_ns();
-        while (ld_acquire_u32(ctr) < target) {
+        const uint64_t limit = g_cross_wait_ns;
+        while ((int32_t)(ld_acquire_u32(ctr) - target) < 0) {
             __nanosleep(100);
-            if (global_ns() - t0 > kWaitLimitNs) {
+            if (global_ns() - t0 > limit) {
                 atomicOr(p.err, kErrTimeout);
                 break;
             }
@@ -1172,9 +1198,11 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         for (int i = 0; i < 2; ++i) {
             mbar_init(&b->s_full[i], 1);
             mbar_init(&b->s_free[i], 128);
+            mbar_init(&b->q_ready[i], 128);
+        }
+        for (int i = 0; i < PD; ++i) {
             mbar_init(&b->p_full[i], 128);
             mbar_init(&b->o_done[i], 1);
-            mbar_init(&b->q_ready[i], 128);
         }
         mbar_init(&b->gdone, 128);
         fence_mbar_init();
@@ -1534,6 +1562,11 @@ static cudaError_t launch(const Params& p, int G, int grid, cudaStream_t st) {
 }
 
 }  // namespace fused
+
+cudaError_t set_cross_cta_wait_limit(uint64_t ns) {
+    const unsigned long long v = ns ? (unsigned long long)ns : (unsigned long long)kWaitLimitNs;
+    return cudaMemcpyToSymbol(fused::g_cross_wait_ns, &v, sizeof(v));
+}
 
 bool fused_supported(const gsa_decode_desc& d) {
     // gathered rows are addressed by a 32-bit row number; the selection lives in shared memory

@@ -8,6 +8,8 @@
 
 #include <algorithm>
 
+#include <cuda_runtime.h>
+
 #include "gsa.h"
 
 namespace gsa {
@@ -17,6 +19,10 @@ constexpr size_t kWsCntOffset = 64;         // u32 tickets [2][rows]
 constexpr int kTargetGistCtas = 296;        // 2 resident gist-pass CTAs per SM on 148 SMs
 constexpr int kTargetUnfoldCtas = 444;      // 3 resident unfold-pass CTAs per SM
 constexpr int kMaxSplits = 256;
+
+// Library-wide device state shared between the source files (host side).
+cudaError_t prefill_error_word(uint32_t** addr);        // gsa_prefill.cu
+cudaError_t set_cross_cta_wait_limit(uint64_t ns);      // gsa_fused.cu (0 restores the default)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -473,6 +473,12 @@ static gsa_status validate_prefill(const gsa_prefill_desc* d) {
     return GSA_OK;
 }
 
+// Device address of the prefill's error word on the current device (read and
+// cleared by gsa_device_error).
+cudaError_t prefill_error_word(uint32_t** addr) {
+    return cudaGetSymbolAddress(reinterpret_cast<void**>(addr), g_prefill_err);
+}
+
 }  // namespace gsa
 
 using namespace gsa;

@@ -60,6 +60,92 @@ def algorithmic_bytes(s: synth.DecodeShape) -> int:
     return s.rows * per_kv + 2 * s.batch * s.n_q_heads * row            # + q and out
 
 
+def _dev(a: np.ndarray):
+    """Host array -> device tensor (bf16 bit patterns become torch.bfloat16)."""
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def _tdtype(dt: str):
+    import torch
+    return torch.float32 if dt == "f32" else torch.bfloat16
+
+
+def _desc_of(s):
+    import kv_cache_routing_b200 as gsa
+    return gsa.decode_desc(s.batch, s.n_q_heads, s.n_kv_heads, s.head_dim, s.n_chunks, s.chunk, s.top_k,
+                           s.tail_len, gsa.GSA_F32 if s.dtype == "f32" else gsa.GSA_BF16, s.mode, s.scale)
+
+
+B200_L2_BYTES = 132644864   # reported by the device; used for the replica count when no GPU is visible
+
+
+def l2_bytes(local: int = 0) -> int:
+    try:
+        import torch
+        if torch.cuda.is_available():
+            return int(torch.cuda.get_device_properties(local).L2_cache_size)
+    except Exception:
+        pass
+    return B200_L2_BYTES
+
+
+def replicas_for(nbytes_step: int, l2: int, override: int = 0) -> int:
+    """Layer replicas to rotate over so that one rotation touches >= 4x L2."""
+    return override if override else max(2, -(-4 * l2 // nbytes_step))
+
+
+def decode_config(s, workload: str, world: int, L: int, nbytes_step: int, l2: int) -> dict:
+    """The `config` of a flat decode line (both arms print the same one)."""
+    return {"workload": workload, "batch": s.batch, "n_q_heads": s.n_q_heads, "n_kv_heads": s.n_kv_heads,
+            "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk, "chunk": s.chunk, "n_gists": s.n_chunks,
+            "top_k": s.top_k, "tail": s.tail_len,
+            "mode": "ALL_GISTS" if s.mode == synth.ALL_GISTS else "SELECTED_PAIRS",
+            "parallelism": f"replicas x{world}",
+            "l2": f"rotating {L} layer replicas, {L * nbytes_step / 1e6:.0f} MB touched per rotation "
+                  f"(L2 {l2 / 1e6:.0f} MB)"}
+
+
+def hier_config(h, workload: str, world: int, L: int, nbytes: int, l2: int) -> dict:
+    s = h.l1
+    return {"workload": workload, "batch": s.batch, "n_q_heads": s.n_q_heads, "n_kv_heads": s.n_kv_heads,
+            "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk, "chunk": s.chunk, "n_l2": h.n_l2,
+            "group": h.group, "top_k2": h.top_k2, "top_k1": s.top_k, "tail": s.tail_len,
+            "parallelism": f"replicas x{world}",
+            "l2": f"rotating {L} replicas (own level-2 gists and query), {L * nbytes / 1e6:.0f} MB touched "
+                  f"per rotation (L2 {l2 / 1e6:.0f} MB)"}
+
+
+def prefill_config(p, workload: str, world: int, l2: int) -> dict:
+    qkv = (p.batch * p.n_q_heads + 2 * p.batch * p.n_kv_heads) * p.positions * p.head_dim * 2
+    return {"workload": workload, "batch": p.batch, "n_q_heads": p.n_q_heads, "n_kv_heads": p.n_kv_heads,
+            "head_dim": p.head_dim, "n_chunks": p.n_chunks, "chunk": p.chunk, "positions": p.positions,
+            "parallelism": f"replicas x{world}",
+            "l2": f"q, k, v of {qkv / 1e6:.0f} MB per step (L2 {l2 / 1e6:.0f} MB)"}
+
+
+REPLAYS = 10
+
+
+def timed_replays(run, stream, n: int = REPLAYS):
+    """Device time (ms) of `run()` on `stream`, once per replay, CUDA events
+    on the launching stream, synchronised on both sides of every replay."""
+    import torch
+    ms = []
+    for _ in range(n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            run()
+            e1.record(stream)
+        stream.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return ms
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -110,9 +196,20 @@ KERNEL_SOURCES = ("gsa_fused.cu", "gsa_fused.h", "gsa_device.cuh", "gsa_tc.cuh")
 
 
 def measured_traffic(workload: str):
-    """DRAM bytes per launch of the decode step from a committed ncu summary
-    under profiles/, or None when none covers this workload or the kernel
-    sources have changed since the counters were taken."""
+    """DRAM bytes per launch of the decode step stored in a committed ncu
+    summary under profiles/ (it is not measured by this run), or None when
+    none covers this workload or the kernel sources have changed since the
+    counters were taken.  See traffic_source() for the file it came from."""
+    return _stored_traffic(workload)[0]
+
+
+def traffic_source(workload: str) -> str:
+    """Where roofline.traffic comes from: the stored profile's file name."""
+    path = _stored_traffic(workload)[1]
+    return f"stored ncu profile {os.path.relpath(path, ROOT)}" if path else "none (no profile of these sources)"
+
+
+def _stored_traffic(workload: str):
     import glob
     import hashlib
     h = hashlib.sha256()
@@ -128,10 +225,10 @@ def measured_traffic(workload: str):
                 kv[k.strip()] = v.strip()
         if kv.get("workload") == workload and kv.get("sources_sha256") == digest:
             try:
-                return int(kv["dram_bytes_per_step"]) / int(kv["launches_per_step"])
+                return int(kv["dram_bytes_per_step"]) / int(kv["launches_per_step"]), path
             except (KeyError, ValueError):
-                return None
-    return None
+                return None, None
+    return None, None
 
 
 class ClockSampler:
@@ -236,31 +333,26 @@ def run_ours(args, world, rank, local):
     import torch
 
     import kv_cache_routing_b200 as gsa
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from gsa_check import desc_of, dev, tdtype
 
     s = synth.WORKLOADS[args.workload]
     torch.cuda.set_device(local)
-    dev_props = torch.cuda.get_device_properties(local)
-    l2 = dev_props.L2_cache_size
+    l2 = l2_bytes(local)
     nbytes_step = algorithmic_bytes(s)
-    L = max(2, -(-4 * l2 // nbytes_step))                 # replicas: touched bytes per rotation >= 4 x L2
-    if args.replicas:
-        L = args.replicas
+    L = replicas_for(nbytes_step, l2, args.replicas)
     x = synth.decode_inputs(s, synth.seed_for(args.workload) + 17 * rank)
-    base = {k: dev(v) for k, v in x.tensors().items()}
+    base = {k: _dev(v) for k, v in x.tensors().items()}
     reps = []
     for r in range(L):
         t = {k: (v if r == 0 else v.clone()) for k, v in base.items()}
         if r:
             # a distinct query per replica (distinct selections); caches are separate copies
             qn = synth.normal(synth.seed_for(args.workload) + 1000 * r + rank, synth.S_Q, x.q.shape, s.dtype)
-            t["q"] = dev(qn)
+            t["q"] = _dev(qn)
         reps.append(t)
-    desc = desc_of(s)
+    desc = _desc_of(s)
     wsz = gsa.gsa_decode_workspace_size(desc)
     launches = gsa.gsa_decode_launch_count(desc)
-    outs = [torch.empty((s.batch, s.n_q_heads, s.head_dim), dtype=tdtype(s.dtype), device="cuda") for _ in range(L)]
+    outs = [torch.empty((s.batch, s.n_q_heads, s.head_dim), dtype=_tdtype(s.dtype), device="cuda") for _ in range(L)]
     idxs = [torch.empty((s.batch, s.n_kv_heads, s.top_k), dtype=torch.int32, device="cuda") for _ in range(L)]
     ws = torch.zeros(wsz, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.Stream()
@@ -274,7 +366,7 @@ def run_ours(args, world, rank, local):
         for i in range(args.warmup):
             step(i, stream)
     stream.synchronize()
-    # K timed steps captured as one graph
+    # K timed steps captured as one graph, replayed REPLAYS times
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g, stream=stream):
@@ -285,20 +377,14 @@ def run_ours(args, world, rank, local):
     stream.synchronize()
     assert gsa.gsa_workspace_error(ws, stream=stream) == 0
 
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-        stream.synchronize()
-        torch.cuda.synchronize()
+        reps_ms = timed_replays(g.replay, stream)
         barrier(world)
-    ms = e0.elapsed_time(e1)
+    ms = statistics.median(reps_ms)
     ms_max = max_over_ranks(ms, world)
     clocks = clk.summary()
+    assert gsa.gsa_workspace_error(ws, stream=stream) == 0
 
     # e2e through the C ABI: per step, H2D of the query from pinned memory,
     # the decode step, D2H of the output and the selection.
@@ -308,11 +394,8 @@ def run_ours(args, world, rank, local):
     out_host = torch.empty_like(outs[0], device="cpu").pin_memory()
     idx_host = torch.empty_like(idxs[0], device="cpu").pin_memory()
     q_dev = [reps[r]["q"] for r in range(L)]
-    barrier(world)
-    torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        f0.record(stream)
+
+    def e2e_run():
         for i in range(args.steps):
             r = i % L
             q_dev[r].copy_(q_host[r], non_blocking=True)
@@ -320,9 +403,9 @@ def run_ours(args, world, rank, local):
             out_host.copy_(outs[r], non_blocking=True)
             idx_host.copy_(idxs[r], non_blocking=True)
             stream.synchronize()                     # the host reads the step's result
-        f1.record(stream)
-    stream.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+
+    barrier(world)
+    e2e_ms = max_over_ranks(statistics.median(timed_replays(e2e_run, stream, 3)), world)
 
     per_step_ms = ms_max / args.steps
     steps_per_s = whole_job_rate(args.steps, world, ms_max)
@@ -341,13 +424,10 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": s.dtype,
         "data": "synthetic",
-        "config": {"workload": args.workload, "batch": s.batch, "n_q_heads": s.n_q_heads,
-                   "n_kv_heads": s.n_kv_heads, "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk,
-                   "chunk": s.chunk, "n_gists": s.n_chunks, "top_k": s.top_k, "tail": s.tail_len,
-                   "mode": "ALL_GISTS" if s.mode == synth.ALL_GISTS else "SELECTED_PAIRS",
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"rotating {L} layer replicas, {L * nbytes_step / 1e6:.0f} MB touched per rotation "
-                         f"(L2 {l2 / 1e6:.0f} MB)"},
+        "config": decode_config(s, args.workload, world, L, nbytes_step, l2),
+        "timing": {"replays": len(reps_ms), "statistic": "median over replays of the K-step graph",
+                   "ms_per_step_min": round(min(reps_ms) / args.steps, 5),
+                   "ms_per_step_max": round(max(reps_ms) / args.steps, 5)},
         "head_steps_per_s": round(steps_per_s * s.batch * s.n_q_heads, 1),
         "algorithmic_bytes_per_step": nbytes_step,
         "roofline": {"bound": "hbm",
@@ -357,7 +437,8 @@ def run_ours(args, world, rank, local):
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": nbytes_step / launches,
-                     "traffic": measured_traffic(args.workload)},
+                     "traffic": measured_traffic(args.workload),
+                     "traffic_source": traffic_source(args.workload)},
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()
@@ -375,39 +456,37 @@ def run_ours(args, world, rank, local):
 # ------------------------------------------------------------- prefill ----
 def run_prefill(args, world, rank, local):
     """The gist-causal prefill: K launches back to back (each reads its q, k,
-    v, together far larger than L2), timed with CUDA events on the stream."""
+    v, together far larger than L2), timed with CUDA events on the stream,
+    median over REPLAYS replays of the K launches."""
     import torch
 
     import kv_cache_routing_b200 as gsa
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from gsa_check import dev
 
     p = synth.WORKLOADS[args.workload]
     torch.cuda.set_device(local)
     x = synth.prefill_inputs(p, synth.seed_for(args.workload) + 17 * rank)
-    d = {k: dev(v) for k, v in x.tensors().items()}
+    d = {k: _dev(v) for k, v in x.tensors().items()}
     P = p.positions
     desc = gsa.prefill_desc(p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.n_chunks, p.chunk, gsa.GSA_BF16,
                             p.scale)
     out = torch.empty((p.batch, p.n_q_heads, P, p.head_dim), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.Stream()
     step = lambda: gsa.gsa_gist_prefill(desc, d["q"], d["k"], d["v"], out, None, stream=stream)
+
+    def run_k():
+        for _ in range(args.steps):
+            step()
+
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
     stream.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.steps):
-                step()
-            e1.record(stream)
-        stream.synchronize()
+        reps_ms = timed_replays(run_k, stream)
         barrier(world)
-    ms_max = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_max = max_over_ranks(statistics.median(reps_ms), world)
+    assert gsa.gsa_device_error() == 0
     flops = 4.0 * p.head_dim * prefill_pairs(p.n_chunks, p.chunk) * p.batch * p.n_q_heads
     per_ms = ms_max / args.steps
     tflops = world * flops / (per_ms / 1e3) / 1e12
@@ -417,33 +496,31 @@ def run_prefill(args, world, rank, local):
         hq[k].copy_(d[k].cpu())
     ho = torch.empty_like(out, device="cpu").pin_memory()
     steps_e2e = max(1, min(args.steps, 5))
-    barrier(world)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        f0.record(stream)
+
+    def e2e_run():
         for _ in range(steps_e2e):
             for k in d:
                 d[k].copy_(hq[k], non_blocking=True)
             step()
             ho.copy_(out, non_blocking=True)
             stream.synchronize()
-        f1.record(stream)
-    stream.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world) / steps_e2e
+
+    barrier(world)
+    e2e_ms = max_over_ranks(statistics.median(timed_replays(e2e_run, stream, 3)), world) / steps_e2e
     peak, peak_kind = tensor_peak()
     line = {
         "metric": PREFILL_METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_ms, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": p.batch, "n_q_heads": p.n_q_heads,
-                   "n_kv_heads": p.n_kv_heads, "head_dim": p.head_dim, "n_chunks": p.n_chunks, "chunk": p.chunk,
-                   "positions": P, "parallelism": f"replicas x{world}",
-                   "l2": f"q, k, v of {sum(v.numel() * v.element_size() for v in d.values()) / 1e6:.0f} MB "
-                         f"per step (L2 {torch.cuda.get_device_properties(local).L2_cache_size / 1e6:.0f} MB)"},
+        "config": prefill_config(p, args.workload, world, l2_bytes(local)),
+        "timing": {"replays": len(reps_ms), "statistic": "median over replays of K back-to-back launches",
+                   "ms_per_step_min": round(min(reps_ms) / args.steps, 5),
+                   "ms_per_step_max": round(max(reps_ms) / args.steps, 5)},
         "algorithmic_flop_per_step": flops,
         "roofline": {"bound": "tensor", "kernel": "gist_prefill_kernel (one launch per step)",
                      "achieved": round(tflops / world, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(tflops / world / peak, 4), "peak_kind": peak_kind, "traffic": None},
+                     "frac": round(tflops / world / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                     "traffic_source": "none"},
         "e2e": {"value": round(world * flops / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in d.values()),
                 "d2h_bytes_per_step": out.numel() * out.element_size()},
@@ -483,33 +560,31 @@ def run_hier(args, world, rank, local):
     """The two-level descent: K steps captured as one graph rotating over L
     replicas (own level-2 gists and query each; level-1 gists and raw chunks
     shared, distinct queries select distinct children) so that the bytes a
-    rotation touches exceed 4x L2."""
+    rotation touches exceed 4x L2; median over REPLAYS replays."""
     import torch
 
     import kv_cache_routing_b200 as gsa
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from gsa_check import desc_of, dev, tdtype
 
     h = synth.WORKLOADS[args.workload]
     s = h.l1
     torch.cuda.set_device(local)
-    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    l2 = l2_bytes(local)
     nbytes = hier_bytes(h)
-    L = max(2, -(-4 * l2 // nbytes)) if not args.replicas else args.replicas
+    L = replicas_for(nbytes, l2, args.replicas)
     seed = synth.seed_for(args.workload) + 17 * rank
     x = synth.hier_inputs(h, seed)
-    base = {k: dev(v) for k, v in x.tensors().items()}
+    base = {k: _dev(v) for k, v in x.tensors().items()}
     reps = []
     for r in range(L):
         t = dict(base)
         if r:
-            t["q"] = dev(synth.normal(seed + 1000 * r, synth.S_Q, x.q.shape, s.dtype))
+            t["q"] = _dev(synth.normal(seed + 1000 * r, synth.S_Q, x.q.shape, s.dtype))
             t["k_g2"] = base["k_g2"].clone()
             t["v_g2"] = base["v_g2"].clone()
         reps.append(t)
-    hd = gsa.hier_desc(desc_of(s), h.n_l2, h.group, h.top_k2)
+    hd = gsa.hier_desc(_desc_of(s), h.n_l2, h.group, h.top_k2)
     ws = torch.zeros(max(256, gsa.gsa_hier_workspace_size(hd)), dtype=torch.uint8, device="cuda")
-    outs = [torch.empty((s.batch, s.n_q_heads, s.head_dim), dtype=tdtype(s.dtype), device="cuda") for _ in range(L)]
+    outs = [torch.empty((s.batch, s.n_q_heads, s.head_dim), dtype=_tdtype(s.dtype), device="cuda") for _ in range(L)]
     i2 = torch.empty((s.batch, s.n_kv_heads, h.top_k2), dtype=torch.int32, device="cuda")
     i1 = torch.empty((s.batch, s.n_kv_heads, s.top_k), dtype=torch.int32, device="cuda")
     stream = torch.cuda.Stream()
@@ -530,55 +605,48 @@ def run_hier(args, world, rank, local):
                 step(i, stream)
         g.replay()
     stream.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-        stream.synchronize()
+        reps_ms = timed_replays(g.replay, stream)
         barrier(world)
-    ms_max = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_max = max_over_ranks(statistics.median(reps_ms), world)
+    assert gsa.gsa_workspace_error(ws, stream=stream) == 0
     per_ms = ms_max / args.steps
     gbs = nbytes / (per_ms / 1e3) / 1e9
     qh = torch.empty_like(reps[0]["q"], device="cpu").pin_memory()
     qh.copy_(reps[0]["q"].cpu())
     oh = torch.empty_like(outs[0], device="cpu").pin_memory()
-    barrier(world)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        f0.record(stream)
+
+    def e2e_run():
         for i in range(args.steps):
             reps[i % L]["q"].copy_(qh, non_blocking=True)
             step(i, stream)
             oh.copy_(outs[i % L], non_blocking=True)
             stream.synchronize()
-        f1.record(stream)
-    stream.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+
+    barrier(world)
+    e2e_ms = max_over_ranks(statistics.median(timed_replays(e2e_run, stream, 3)), world)
     peak, peak_kind = peaks()
     line = {
         "metric": HIER_METRIC, "value": round(whole_job_rate(args.steps, world, ms_max), 2), "unit": "steps/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
-        "config": {"workload": args.workload, "batch": s.batch, "n_q_heads": s.n_q_heads,
-                   "n_kv_heads": s.n_kv_heads, "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk,
-                   "chunk": s.chunk, "n_l2": h.n_l2, "group": h.group, "top_k2": h.top_k2, "top_k1": s.top_k,
-                   "tail": s.tail_len, "parallelism": f"replicas x{world}",
-                   "l2": f"rotating {L} replicas (own level-2 gists and query), {L * nbytes / 1e6:.0f} MB touched "
-                         f"per rotation (L2 {l2 / 1e6:.0f} MB)"},
+        "config": hier_config(h, args.workload, world, L, nbytes, l2),
+        "timing": {"replays": len(reps_ms), "statistic": "median over replays of the K-step graph",
+                   "ms_per_step_min": round(min(reps_ms) / args.steps, 5),
+                   "ms_per_step_max": round(max(reps_ms) / args.steps, 5)},
         "algorithmic_bytes_per_step": nbytes,
         "roofline": {"bound": "hbm", "kernel": f"gsa_hier_decode (whole step)", "achieved": round(gbs, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
-                     "traffic": None},
+                     "traffic": None, "traffic_source": "none"},
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": qh.numel() * qh.element_size(),
                 "d2h_bytes_per_step": oh.numel() * oh.element_size()},
         "gpu_launches": gsa.gsa_hier_launch_count(hd) * args.steps,
         "clocks": clk.summary(),
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_hier(h, x, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g
@@ -604,34 +672,88 @@ def cpu_baseline(s, x, budget_s: float):
                       f"fp64, OpenMP over rows, {el:.1f} s"}
 
 
-def run_reference(args, world, rank):
-    if rank != 0:
-        return
-    s = synth.WORKLOADS[args.workload]
-    x = synth.decode_inputs(s, synth.seed_for(args.workload))
+def cpu_baseline_hier(h, x, budget_s: float):
+    """The fp64 oracle of the two-level descent, as it stands, on the host
+    cores: whole steps until the time budget is spent (at least one).  A step
+    has batch x kv-heads rows (8 for the 1M-token workload), so OpenMP over
+    rows uses at most that many threads."""
     import oracle
     t = x.tensors()
-    oracle.decode(t, s.top_k, s.mode)
-    times = []
+    s = h.l1
+    oracle.hier_decode(t, h.group, h.top_k2, s.top_k)   # load + warm
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.hier_decode(t, h.group, h.top_k2, s.top_k)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 1000:
+            break
+    cores = min(s.rows, int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
+    return {"value": round(n / el, 4), "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} full hierarchical steps of the workload ({s.rows} (batch, kv-head) rows each, so at "
+                      f"most {s.rows} OpenMP threads), fp64, {el:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle as it stands, on the host cores, on
+    the same workload, metric, unit and config as the GPU arm; each step is
+    a bounded sample of the workload (whole decode steps; for the prefill,
+    random query rows).  Under torchrun only rank 0 runs it."""
+    if rank != 0:
+        return
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    l2 = l2_bytes(0)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    seed = synth.seed_for(args.workload)
+    if isinstance(w, synth.PrefillShape):
+        x = synth.prefill_inputs(w, seed)
+        t = x.tensors()
+        rng = np.random.default_rng(7)
+        rows = np.stack([rng.integers(w.batch, size=512), rng.integers(w.n_q_heads, size=512),
+                         rng.integers(w.positions, size=512)], axis=1).astype(np.int64)
+        flop = sum(4.0 * w.head_dim * prefill_row_pairs(int(r[2]), w.chunk) for r in rows)
+        run = lambda: oracle.prefill_rows(t, w.n_chunks, w.chunk, rows, w.scale)
+        metric, unit, dtype = PREFILL_METRIC, "TFLOP/s", "f64"
+        config = prefill_config(w, args.workload, world, l2)
+        sample = f"512 random query rows of the workload per step ({flop / 1e9:.2f} GFLOP algorithmic), fp64"
+        rate = lambda sec: flop / sec / 1e12
+    elif isinstance(w, synth.HierShape):
+        x = synth.hier_inputs(w, seed)
+        t = x.tensors()
+        run = lambda: oracle.hier_decode(t, w.group, w.top_k2, w.l1.top_k)
+        metric, unit, dtype = HIER_METRIC, "steps/s", "f64"
+        nb = hier_bytes(w)
+        config = hier_config(w, args.workload, world, replicas_for(nb, l2, args.replicas), nb, l2)
+        sample = f"one full hierarchical step per step ({w.l1.rows} rows, OpenMP over rows), fp64"
+        cores = min(cores, w.l1.rows)
+        rate = lambda sec: 1.0 / sec
+    else:
+        x = synth.decode_inputs(w, seed)
+        t = x.tensors()
+        run = lambda: oracle.decode(t, w.top_k, w.mode)
+        metric, unit, dtype = METRIC, "steps/s", "f64"
+        nb = algorithmic_bytes(w)
+        config = decode_config(w, args.workload, world, replicas_for(nb, l2, args.replicas), nb, l2)
+        sample = f"one full decode step per step ({w.rows} rows, OpenMP over rows), fp64"
+        rate = lambda sec: 1.0 / sec
+    run()
     for _ in range(args.warmup):
-        oracle.decode(t, s.top_k, s.mode)
+        run()
+    times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.decode(t, s.top_k, s.mode)
+        run()
         times.append(time.perf_counter() - t0)
     total = sum(times)
-    v = args.steps / total
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "steps/s", "n_gpus": world,
+    v = rate(total / args.steps)
+    line = {"impl": "reference", "metric": metric, "value": round(v, 6), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "batch": s.batch, "n_q_heads": s.n_q_heads,
-                       "n_kv_heads": s.n_kv_heads, "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk,
-                       "top_k": s.top_k, "parallelism": "host cores"},
-            "cpu_baseline": {"value": round(v, 4), "unit": "steps/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{args.steps} full decode steps, fp64 oracle, OpenMP over "
-                                       f"{s.rows} rows"},
-            "e2e": {"value": round(v, 4), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+            "config": config,
+            "cpu_baseline": {"value": round(v, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} steps; {sample}"},
+            "e2e": {"value": round(v, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -650,8 +772,6 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
-        if not isinstance(synth.WORKLOADS[args.workload], synth.DecodeShape):
-            ap.error("--impl reference times the decode workloads")
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, world, rank)

@@ -21,7 +21,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 F32, BF16, F64 = 0, 1, 2
-ALL_GISTS, SELECTED_PAIRS = 0, 1
+ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS = 0, 1, 2, 3
 _DT = {"f32": F32, "bf16": BF16, "f64": F64}
 
 

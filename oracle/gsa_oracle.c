@@ -32,7 +32,7 @@
 #include <string.h>
 
 enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
-enum { OR_ALL_GISTS = 0, OR_SELECTED_PAIRS = 1 };
+enum { OR_ALL_GISTS = 0, OR_SELECTED_PAIRS = 1, OR_SR_ONLY = 2, OR_UNSELECTED_GISTS = 3 };
 
 /* Exact widening of one stored element to double. */
 static double ld(const void* p, int dt, int64_t i) {
@@ -193,6 +193,11 @@ static void attend(int d, int dt, double scale, const void* q, int64_t q_off, in
  * tokens of the selected chunks ([SL-17] "AG+SR").
  * [SL-6] / [SL-17] "SG+SR": only the selected chunks' gists and raw tokens
  * -> SELECTED_PAIRS.
+ * [SL-17] "SR-only": the selected chunks' raw tokens, no gist at all
+ * -> SR_ONLY.
+ * [DE-M] "Hybride Attention": the selected raw tokens and the gists of the
+ * chunks that were NOT selected (a selected chunk is represented by its raw
+ * tokens instead of its gist) -> UNSELECTED_GISTS.
  * In both modes the W uncompressed tail tokens after the last chunk are
  * always attended ([SL-9]: the generation suffix attends directly).          */
 static int flat_context(int Hkv, int d, int N, int c, int W, int mode, int b, int hk, int k,
@@ -202,9 +207,15 @@ static int flat_context(int Hkv, int d, int N, int c, int W, int mode, int b, in
     int64_t row = (int64_t)b * Hkv + hk;
     if (mode == OR_ALL_GISTS) {
         for (int j = 0; j < N; ++j) keys[n++] = (key_ref){kg, vg, (row * N + j) * d};
-    } else {
+    } else if (mode == OR_SELECTED_PAIRS) {
         for (int t = 0; t < k; ++t) keys[n++] = (key_ref){kg, vg, (row * N + sel[t]) * d};
-    }
+    } else if (mode == OR_UNSELECTED_GISTS) {
+        for (int j = 0; j < N; ++j) {
+            int selected = 0;
+            for (int t = 0; t < k; ++t) selected |= sel[t] == j;
+            if (!selected) keys[n++] = (key_ref){kg, vg, (row * N + j) * d};
+        }
+    }   /* OR_SR_ONLY: no gist */
     for (int t = 0; t < k; ++t)
         for (int u = 0; u < c; ++u)
             keys[n++] = (key_ref){kraw, vraw, ((row * N + sel[t]) * c + u) * d};

@@ -106,7 +106,7 @@ def widen(a: np.ndarray, dtype: str) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Workload shapes
 # ---------------------------------------------------------------------------
-ALL_GISTS, SELECTED_PAIRS = 0, 1
+ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS = 0, 1, 2, 3
 
 # stream ids, one per generated tensor
 S_Q, S_KG, S_VG, S_KR, S_VR, S_KT, S_VT, S_NEEDLE_IDX, S_NEEDLE_NOISE = range(1, 10)

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 import synth
-from synth import DecodeShape, HierShape, ALL_GISTS, SELECTED_PAIRS
+from synth import DecodeShape, HierShape, ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS
 
 
 def sdpa(qv, K, V, scale, mask=None, causal=False):
@@ -184,11 +184,13 @@ def test_full_selection_is_full_attention(mode, dtype):
                                        rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode", [ALL_GISTS, SELECTED_PAIRS])
+@pytest.mark.parametrize("mode", [ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS])
 def test_partial_selection_is_masked_attention(mode):
     """k < N: the gathered context equals full attention under a boolean mask
-    that keeps the selected chunks' raw tokens (and, for SELECTED_PAIRS, only
-    the selected gists); the selection itself equals a lexsort top-k."""
+    that keeps the selected chunks' raw tokens and the tail, and of the gists:
+    all (ALL_GISTS), the selected ones (SELECTED_PAIRS), none (SR_ONLY) or
+    the unselected ones (UNSELECTED_GISTS); the selection itself equals a
+    lexsort top-k."""
     sh = small_shape(n_chunks=9, chunk=4, top_k=3, tail_len=3, mode=mode)
     x = synth.decode_inputs(sh, 33)
     s, idx, out = oracle.decode(x.tensors(), sh.top_k, mode, scale=0.3)
@@ -199,12 +201,52 @@ def test_partial_selection_is_masked_attention(mode):
             assert idx[b, hk].tolist() == sorted(order[:3].tolist())
             sel = np.zeros(N, bool)
             sel[idx[b, hk]] = True
-            gist_keep = np.ones(N, bool) if mode == ALL_GISTS else sel
+            gist_keep = {ALL_GISTS: np.ones(N, bool), SELECTED_PAIRS: sel, SR_ONLY: np.zeros(N, bool),
+                         UNSELECTED_GISTS: ~sel}[mode]
             mask = np.concatenate([gist_keep, np.repeat(sel, c), np.ones(sh.tail_len, bool)])
             K, V = _all_keys(x, b, hk)
             qv = synth.widen(x.q[b, hk * G:(hk + 1) * G], "f32")
             want = sdpa(qv, K, V, 0.3, mask=np.broadcast_to(mask, (G, mask.size)))
             np.testing.assert_allclose(out[b, hk * G:(hk + 1) * G], want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", [SR_ONLY, UNSELECTED_GISTS])
+def test_full_selection_without_gists_is_raw_and_tail_attention(mode):
+    """k = N: SR_ONLY keeps no gist and UNSELECTED_GISTS has no unselected
+    chunk left, so both reduce to softmax attention over every raw token and
+    the tail (library SDPA over that key list)."""
+    sh = small_shape(top_k=6, mode=mode)
+    x = synth.decode_inputs(sh, 23)
+    _, idx, out = oracle.decode(x.tensors(), sh.top_k, mode)
+    N, c, d, G = sh.n_chunks, sh.chunk, sh.head_dim, sh.group
+    for b in range(sh.batch):
+        for hk in range(sh.n_kv_heads):
+            K = np.concatenate([synth.widen(x.k_raw[b, hk], "f32").reshape(N * c, d),
+                                synth.widen(x.k_tail[b, hk], "f32")])
+            V = np.concatenate([synth.widen(x.v_raw[b, hk], "f32").reshape(N * c, d),
+                                synth.widen(x.v_tail[b, hk], "f32")])
+            qv = synth.widen(x.q[b, hk * G:(hk + 1) * G], "f32")
+            np.testing.assert_allclose(out[b, hk * G:(hk + 1) * G], sdpa(qv, K, V, 1 / math.sqrt(d)),
+                                       rtol=0, atol=1e-12)
+
+
+def test_empty_selection_of_the_gist_rules():
+    """k = 0: UNSELECTED_GISTS keeps every gist and equals ALL_GISTS (both are
+    every gist plus the tail); SR_ONLY keeps the tail alone."""
+    sh = small_shape(top_k=0, tail_len=3)
+    x = synth.decode_inputs(sh, 25)
+    t = x.tensors()
+    _, _, a = oracle.decode(t, 0, ALL_GISTS)
+    _, _, u = oracle.decode(t, 0, UNSELECTED_GISTS)
+    np.testing.assert_array_equal(a, u)
+    _, _, r = oracle.decode(t, 0, SR_ONLY)
+    G, d = sh.group, sh.head_dim
+    for b in range(sh.batch):
+        for hk in range(sh.n_kv_heads):
+            qv = synth.widen(x.q[b, hk * G:(hk + 1) * G], "f32")
+            want = sdpa(qv, synth.widen(x.k_tail[b, hk], "f32"), synth.widen(x.v_tail[b, hk], "f32"),
+                        1 / math.sqrt(d))
+            np.testing.assert_allclose(r[b, hk * G:(hk + 1) * G], want, rtol=0, atol=1e-12)
 
 
 def test_unfold_attn_lse_is_library_logsumexp():

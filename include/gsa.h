@@ -77,11 +77,25 @@ typedef enum {
 typedef enum { GSA_F32 = 0, GSA_BF16 = 1 } gsa_dtype;
 
 /* Context rule of the hybrid attention.
- * GSA_ALL_GISTS      every gist once + raw tokens of the k selected chunks +
- *                    tail ([EN-2] "Hybrid Attention"; [SL-17] "AG+SR").
- * GSA_SELECTED_PAIRS gists and raw tokens of the k selected chunks only +
- *                    tail ([SL-6]; [SL-17] "SG+SR").                       */
-typedef enum { GSA_ALL_GISTS = 0, GSA_SELECTED_PAIRS = 1 } gsa_mode;
+ * GSA_ALL_GISTS        every gist once + raw tokens of the k selected chunks
+ *                      + tail ([EN-2] "Hybrid Attention"; [SL-17] "AG+SR").
+ * GSA_SELECTED_PAIRS   gists and raw tokens of the k selected chunks only +
+ *                      tail ([SL-6]; [SL-17] "SG+SR").
+ * GSA_SR_ONLY          raw tokens of the k selected chunks + tail, no gist
+ *                      ([SL-17] "SR-only").
+ * GSA_UNSELECTED_GISTS raw tokens of the k selected chunks + the gists of
+ *                      the N - k chunks not selected + tail ([DE-M]
+ *                      "Hybride Attention": a selected chunk is represented
+ *                      by its raw tokens instead of its gist).
+ * In GSA_UNSELECTED_GISTS mode gsa_decode_step enqueues gsa_score, gsa_topk
+ * and gsa_unfold_attn (the gist attention needs the selection first); the
+ * other modes are one launch on the tensor-core path.                     */
+typedef enum {
+    GSA_ALL_GISTS = 0,
+    GSA_SELECTED_PAIRS = 1,
+    GSA_SR_ONLY = 2,
+    GSA_UNSELECTED_GISTS = 3
+} gsa_mode;
 
 typedef struct {
     int32_t batch, n_q_heads, n_kv_heads, head_dim;

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libgsa.so")
 GSA_OK, GSA_ERR_ARG, GSA_ERR_SHAPE, GSA_ERR_DTYPE, GSA_ERR_ALIGN, GSA_ERR_WORKSPACE, GSA_ERR_CUDA, \
     GSA_ERR_TIMEOUT = range(8)
 GSA_F32, GSA_BF16 = 0, 1
-GSA_ALL_GISTS, GSA_SELECTED_PAIRS = 0, 1
+GSA_ALL_GISTS, GSA_SELECTED_PAIRS, GSA_SR_ONLY, GSA_UNSELECTED_GISTS = 0, 1, 2, 3
 GSA_WS_ERR_TIMEOUT, GSA_WS_ERR_INDEX = 1, 2
 
 # Every function the C header declares (checked by the tests).

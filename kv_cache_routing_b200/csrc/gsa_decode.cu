@@ -61,6 +61,7 @@ struct PassParams {
     int SB, tprB, KB, U;              // unfold pass: splits, stages, keys per row, keys per unit
     int64_t candA;
     int do_score, do_attn, do_topk;   // gist pass work
+    int mask_sel;                     // do_attn with a given selection (idx_in) whose gists leave the context
     int local_topk;                   // 1: per-split candidates then merge; 0: last CTA selects from all scores
     int merge_a;                      // unfold pass merges the gist-pass partials
     // gist-pass source: the virtual gist list of a row has Nv entries.  Flat:
@@ -196,6 +197,19 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
                 if (p.do_score) {
                     const float sc = wa.score(ws, lane);
                     if (lane < nv) p.scores[score_row + g0 + warp * C::TW + lane] = sc;
+                }
+                if (p.mask_sel) {
+                    // UNSELECTED_GISTS with a given selection: its gists get no weight
+                    if (lane < nv) {
+                        const int j = gist_of(p, row, g0 + warp * C::TW + lane);
+                        bool hit = false;
+                        for (int u = 0; u < p.K && !hit; ++u) hit = __ldg(p.idx_in + (size_t)row * p.K + u) == j;
+                        if (hit) {
+#pragma unroll
+                            for (int h = 0; h < G; ++h) ws.lg[lane * G + h] = kNegInf;
+                        }
+                    }
+                    __syncwarp();
                 }
                 if (attn) wa.softmax_pv(sm.stage[slot][1] + warp * C::TW * C::ROWB, ws, nv, p.c2, lane);
             }
@@ -584,6 +598,21 @@ static size_t decode_ws_bytes(const gsa_decode_desc& d) {
                               : make_decode_plan(d).total;
 }
 
+// UNSELECTED_GISTS decode step: where the scores and the selection go when the
+// caller passes no buffers for them.  Both plans keep score and selection
+// regions that the given-selection pass does not use.
+static void unselected_scratch(const gsa_decode_desc& d, size_t& off_scores, size_t& off_idx) {
+    if (fused_supported(d)) {
+        const FusedPlan f = make_fused_plan(d, true);
+        off_scores = f.off_scores;
+        off_idx = f.off_idx;
+    } else {
+        const DecodePlan pl = make_decode_plan(d);
+        off_scores = pl.off_scores;
+        off_idx = pl.off_idx;
+    }
+}
+
 }  // namespace gsa
 
 // ================================================================ C ABI ====
@@ -633,7 +662,8 @@ static gsa_status check_tensors(const gsa_decode_desc* d, const void* q, const v
     const bool raw_needed = d->top_k > 0;
     const bool tail_needed = d->tail_len > 0;
     if (!q || !out) return GSA_ERR_ARG;
-    if (gists_needed && (!kg || (d->mode == GSA_ALL_GISTS && !vg))) return GSA_ERR_ARG;
+    const bool gist_attn = d->mode == GSA_ALL_GISTS || d->mode == GSA_UNSELECTED_GISTS;
+    if (gists_needed && (!kg || (gist_attn && !vg))) return GSA_ERR_ARG;
     if (raw_needed && (!kr || !vr || (d->mode == GSA_SELECTED_PAIRS && (!kg || !vg)))) return GSA_ERR_ARG;
     if (tail_needed && (!kt || !vt)) return GSA_ERR_ARG;
     const void* all[] = {q, kg, vg, kr, vr, kt, vt, out};
@@ -665,7 +695,8 @@ gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const voi
     p.idx_in = idx;
     p.out = static_cast<uint8_t*>(out);
     p.lse = lse;
-    p.do_attn = (desc->mode == GSA_ALL_GISTS);
+    p.do_attn = (desc->mode == GSA_ALL_GISTS || desc->mode == GSA_UNSELECTED_GISTS);
+    p.mask_sel = (desc->mode == GSA_UNSELECTED_GISTS);
     p.merge_a = p.do_attn && desc->n_chunks > 0;
     cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, desc->n_q_heads / desc->n_kv_heads, p.merge_a != 0,
                                true, static_cast<cudaStream_t>(stream));
@@ -681,6 +712,21 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
     if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
     if (!aligned16(idx_out) || !aligned16(scores_out)) return GSA_ERR_ALIGN;
     if ((st = check_ws(decode_ws_bytes(*desc), ws, ws_bytes)) != GSA_OK) return st;
+    if (desc->mode == GSA_UNSELECTED_GISTS && desc->top_k > 0) {
+        // the gist attention needs the selection first: score, select, then
+        // attend with the selection given (its gists masked out).  The scores
+        // and the selection go to the caller's buffers or to workspace
+        // regions the given-selection pass leaves unused.
+        uint8_t* w = static_cast<uint8_t*>(ws);
+        size_t off_s, off_i;
+        unselected_scratch(*desc, off_s, off_i);
+        float* sc = scores_out ? scores_out : reinterpret_cast<float*>(w + off_s);
+        int32_t* ix = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + off_i);
+        if ((st = gsa_score(desc, q, k_gist, sc, stream)) != GSA_OK) return st;
+        if ((st = gsa_topk(desc, sc, ix, stream)) != GSA_OK) return st;
+        return gsa_unfold_attn(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ix, out, nullptr, ws, ws_bytes,
+                               stream);
+    }
     if (fused_supported(*desc))
         return fused_launch(*desc, make_fused_plan(*desc), q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, nullptr,
                             idx_out, scores_out, out, nullptr, ws, static_cast<cudaStream_t>(stream));
@@ -692,7 +738,7 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
     p.out = static_cast<uint8_t*>(out);
     p.do_score = 1;
     p.do_topk = 1;
-    p.do_attn = (desc->mode == GSA_ALL_GISTS);
+    p.do_attn = (desc->mode == GSA_ALL_GISTS || desc->mode == GSA_UNSELECTED_GISTS);   // (k = 0 here: nothing to mask)
     p.merge_a = p.do_attn && desc->n_chunks > 0;
     cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, desc->n_q_heads / desc->n_kv_heads,
                                desc->n_chunks > 0, true, static_cast<cudaStream_t>(stream));
@@ -863,8 +909,12 @@ int gsa_hier_launch_count(const gsa_hier_desc* desc) {
 
 int gsa_decode_launch_count(const gsa_decode_desc* desc) {
     if (validate_decode(desc) != GSA_OK) return -1;
-    if (fused_supported(*desc)) return 1;
-    return (desc->n_chunks > 0 ? 1 : 0) + 1;
+    // the attention pass: one fused launch, or the gist pass (if any gists) and the unfold pass
+    const bool gist_attn = desc->mode == GSA_ALL_GISTS || desc->mode == GSA_UNSELECTED_GISTS;
+    const int attn = fused_supported(*desc) ? 1 : (desc->n_chunks > 0 ? 1 : 0) + 1;
+    if (desc->mode == GSA_UNSELECTED_GISTS && desc->top_k > 0)
+        return 2 + (fused_supported(*desc) ? 1 : (gist_attn && desc->n_chunks > 0 ? 1 : 0) + 1);
+    return attn;
 }
 
 gsa_status gsa_device_error(uint32_t* flags_out, void* stream) {

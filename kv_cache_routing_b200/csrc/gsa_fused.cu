@@ -58,6 +58,10 @@
 namespace gsa {
 namespace fused {
 
+// Limit of the waits of one CTA on others (default kWaitLimitNs; a
+// diagnostics setter shortens it so that tests can make such a wait run out).
+__device__ unsigned long long g_cross_wait_ns = kWaitLimitNs;
+
 constexpr int NT = 192;                      // streaming warps 0-5: softmax 0-3, loads 4, MMA 5
 constexpr int NU = 128;                      // unfold warps 6-9: selection, row tables, gathers
 constexpr int UFIRST = NT;                   // first unfold thread
@@ -96,7 +100,10 @@ constexpr uint32_t SM_HSCR = SM_HRES + TILE * 4;
 static_assert(SM_HSCR + 4608 <= SM_ROWTAB, "hierarchy tables overflow the selection buffer");
 static_assert(kSelCap * 4 + kMaxTpc * TILE * 4 <= kScoreCap * 4, "unfold tables overflow the score buffer");
 constexpr uint32_t SM_UB = SM_SCORE + kScoreCap * 4;  // first unit of every CTA [kFusedCtas + 1]
-constexpr uint32_t SM_BAR = SM_UB + 640;
+constexpr uint32_t SM_SEGC = SM_UB + 640;              // key stretch, k <= 32: the kept top-k of each score tile [24][32] u64
+constexpr uint32_t SM_CAND = SM_SEGC + (kScoreCap / TILE) * 32 * 8;   // a score tile, packed [NU] u64; the row's candidates [2 NU] u64
+constexpr uint32_t SM_TMASK = SM_CAND + 2 * NU * 8;   // key stretch: the tile's gists of a given selection (UNSELECTED_GISTS) [4] u32
+constexpr uint32_t SM_BAR = SM_TMASK + 16;
 static_assert((kFusedCtas + 1) * 4 <= 640, "unit table overflow");
 constexpr uint32_t SMEM_BYTES = SM_BAR + 512 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "dynamic shared memory above the per-block limit");
@@ -107,6 +114,8 @@ struct Bars {
     uint64_t p_full[PD], o_done[PD];
     uint64_t q_ready[2];
     uint64_t gdone;              // a gathered stretch is closed (its row table and children keys are free)
+    uint64_t gready;             // the first NSL gathered slots are free (their key / value tiles consumed)
+    uint64_t sc_full[kScoreCap / 128];   // k <= 32: score tile i of this CTA is in shared memory (used once)
     uint32_t tmem;
 };
 
@@ -133,6 +142,8 @@ struct Run {
     int gap;       // RUN_V: value tile j at seq0 + j (j < npre) or seq0 + gap + j
     int slot_b;    // RUN_G: the partial slot
     int score;     // RUN_G: the tile is scored (the hierarchy's children tile)
+    int gfirst;    // RUN_V: the first gathered tile's slot sequence number
+    int gwait;     // RUN_V: slots from gfirst the producer waits free for the unfold warps
 };
 
 // CTA c takes units [ub[c], ub[c + 1]), ub[c] = floor(c * T / grid), a table
@@ -147,6 +158,26 @@ __device__ __forceinline__ int cta_of(const int* ub, int grid, int u) {
         else hi = mid - 1;
     }
     return lo;
+}
+
+// Gists [g0, g1) of `row` that CTA cc scores (an empty range if none).
+__device__ __forceinline__ void cta_gists(const Params& p, const int* ub, int cc, int row, int& g0, int& g1) {
+    const int ru0 = row * p.upr;
+    const int a = max(ub[cc], ru0), b = min(ub[cc + 1], ru0 + p.tg);
+    g0 = (a - ru0) * TILE;
+    g1 = b > a ? min((b - ru0) * TILE, p.NA) : g0;
+}
+
+// First candidate slot of CTA c for `row`: the CTAs meeting the row before
+// it publish min(k, gists they score) candidates each.
+__device__ __forceinline__ int cand_offset(const Params& p, const int* ub, int c, int row) {
+    int off = 0;
+    for (int cc = cta_of(ub, p.grid, row * p.upr); cc < c; ++cc) {
+        int g0, g1;
+        cta_gists(p, ub, cc, row, g0, g1);
+        off += min(p.K, g1 - g0);
+    }
+    return off;
 }
 
 __device__ __forceinline__ Tile unit_tile(const Params& p, int u) {
@@ -229,6 +260,21 @@ struct Ctx {
     uint32_t mcol; // first TMEM column of the segment maxima
 };
 
+// Packed candidate: orderable score key, then the complemented gist index,
+// so that comparing the packed values compares (score, then lower index).
+__device__ __forceinline__ uint64_t pack_cand(uint32_t key, int pos) {
+    return ((uint64_t)key << 32) | (uint64_t)(uint32_t)~(uint32_t)pos;
+}
+__device__ __forceinline__ int cand_pos(uint64_t c) { return (int)~(uint32_t)c; }
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* a, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* a) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
+    return v;
+}
+
 // Is slot sequence number `seq` free to fill (its previous use consumed)?
 __device__ __forceinline__ bool slot_free(const Params& p, Bars* b, int seq) {
     return seq < NSL || mbar_wait(&b->empty[seq % NSL], ((seq / NSL) - 1) & 1, p.err);
@@ -293,6 +339,16 @@ __device__ __forceinline__ void produce_run(const Params& p, Ctx& cx, const Run&
                 if (cx.lane == 0) load_tensor(p, cx, u, seq, true);
             }
             ++j;
+        }
+        // The first gathered tiles take slots whose previous use was a key or
+        // value tile many ring turns back, too far for a parity wait by the
+        // unfold warps (a phase parity names only the current or the
+        // previous phase).  The producer, which walks the ring in order, waits
+        // them free and hands them over through one mbarrier.
+        if (r.gwait > 0) {
+            for (int q = 0; q < r.gwait; ++q)
+                if (!slot_free(p, cx.bars, r.gfirst + q)) return;
+            if (cx.lane == 0) mbar_arrive(&cx.bars->gready);
         }
     } else {
         // gathered tiles beyond the ones every thread issued up front
@@ -554,7 +610,21 @@ __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u
     tc::wait_ld();
     tc::fence_before();
     mbar_arrive(&cx.bars->s_free[sb]);
-    const bool valid = t < u.nvalid;
+    bool valid = t < u.nvalid;
+    if (p.mask_sel && u.kind == 0) {
+        // the given selection's gists are not in the context: a 128-bit mask
+        // of the tile's selected gists (every thread reads the selection)
+        uint32_t* tm = reinterpret_cast<uint32_t*>(cx.base + SM_TMASK);
+        if (t < 4) tm[t] = 0u;
+        group_sync<128, BAR_SOFT>();
+        for (int j = t; j < p.K; j += 128) {
+            const int o = __ldg(p.idx + (size_t)u.row * p.K + j) - u.t * TILE;
+            if (o >= 0 && o < TILE) atomicOr(&tm[o >> 5], 1u << (o & 31));
+        }
+        group_sync<128, BAR_SOFT>();
+        valid = valid && !((tm[t >> 5] >> (t & 31)) & 1u);
+        group_sync<128, BAR_SOFT>();
+    }
     if (u.attn) {
         uint32_t xr[G];
 #pragma unroll
@@ -576,6 +646,8 @@ __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u
             if (cx.gtiles < kScoreCap / TILE)
                 reinterpret_cast<float*>(cx.base + SM_SCORE)[cx.gtiles * TILE + t] = score;
         }
+        // k <= 32: the unfold warps fold this tile of scores into their running top-k lists
+        if (p.inc_sel && cx.gtiles < kScoreCap / TILE) mbar_arrive(&cx.bars->sc_full[cx.gtiles]);
         cx.gtiles++;
     }
 }
@@ -889,6 +961,130 @@ __device__ __forceinline__ void merge_select(const Params& p, uint8_t* base, int
     usync();
 }
 
+// k <= 32, during the key stretch (unfold warps, beside the streaming): a
+// running top-k list of the row segment's gists, sorted descending, is kept
+// in shared memory.  As each score tile arrives, the scores that beat the
+// list's k-th entry are collected (warp ballots, then the four warp counts)
+// and ranked together with the list: each element of the union counts the
+// larger ones, and those of rank < k form the new list.  Packed scores
+// compare as (score, then lower index), so ranks are exact and distinct.
+// After the first tile of a segment few scores pass the k-th entry.  At the
+// segment's end the list is the CTA's top-k of the segment and goes to the
+// row's candidate slots.  Score tile st of this CTA is announced by mbarrier
+// sc_full[st].
+__device__ __forceinline__ void fold_scores(const Params& p, uint8_t* base, Bars* bars, int c, int row_first,
+                                            int row_last) {
+    const int* ub = reinterpret_cast<const int*>(base + SM_UB);
+    const float* sc = reinterpret_cast<const float*>(base + SM_SCORE);
+    uint64_t* uni = reinterpret_cast<uint64_t*>(base + SM_CAND);    // [2 NU] the list, then the passing scores
+    uint64_t* nl = reinterpret_cast<uint64_t*>(base + SM_SEGC);     // [32] the new list
+    uint32_t* wc = reinterpret_cast<uint32_t*>(base + SM_SEGC + 32 * 8);   // [4] passing scores per warp
+    const int i = utid(), lane = i & 31, uw = i >> 5;
+    const int K = p.K;
+    int st = 0;
+    for (int r = row_first; r <= row_last; ++r) {
+        int g0, g1;
+        cta_gists(p, ub, c, r, g0, g1);
+        if (g1 <= g0) continue;
+        if (i < K) uni[i] = 0ull;
+        usync();
+        for (int g = g0; g < g1; g += TILE, ++st) {
+            mbar_wait(&bars->sc_full[st], 0, p.err);
+            const uint64_t me = g + i < g1 ? pack_cand(order_key(sc[st * TILE + i]), g + i) : 0ull;
+            const uint64_t kth = uni[K - 1];
+            const bool pass = me > kth;
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
+            if (lane == 0) wc[uw] = __popc(m);
+            usync();
+            int before = 0, total = 0;
+#pragma unroll
+            for (int w = 0; w < NU / 32; ++w) {
+                const int x = (int)wc[w];
+                before += w < uw ? x : 0;
+                total += x;
+            }
+            if (pass) uni[K + before + __popc(m & ((1u << lane) - 1u))] = me;
+            if (i < K) nl[i] = 0ull;   // empty entries (all 0) share one rank: the places after the real ones stay 0
+            usync();
+            if (total > 0) {
+                const int n = K + total;   // up to K + NU entries
+                for (int q = i; q < n; q += NU) {
+                    const uint64_t e = uni[q];
+                    int rank = 0;
+                    for (int j = 0; j < n; ++j) rank += uni[j] > e ? 1 : 0;
+                    if (rank < K) nl[rank] = e;
+                }
+                usync();
+                if (i < K) uni[i] = nl[i];
+                usync();
+            }
+        }
+        // the list holds min(k, gists of this CTA in the row) entries
+        if (i < K && uni[i] != 0ull) st_relaxed_u64(p.cand64 + (size_t)r * p.NA + cand_offset(p, ub, c, r) + i, uni[i]);
+        usync();
+    }
+}
+
+// k <= 32: the row's exact top-k from the n <= 2 NU candidates the CTAs
+// meeting the row published in the key stretch (each CTA's top-k of the
+// gists it scored, so their union holds the row's top-k).  A slot reads 0
+// until its value lands; the wait on it is bounded.  Ranks come from
+// counting the larger packed candidates (ties of score go to the lower
+// index), then the k positions are put in ascending order.
+__device__ __forceinline__ void inc_select(const Params& p, uint8_t* base, int row, int n, bool publish) {
+    const uint64_t* slots = p.cand64 + (size_t)row * p.NA;
+    uint64_t* cs = reinterpret_cast<uint64_t*>(base + SM_CAND);
+    int32_t* byrank = reinterpret_cast<int32_t*>(base + SM_MISC);
+    const uint64_t limit = 2ull * g_cross_wait_ns;
+    for (int i = utid(); i < p.K; i += NU) byrank[i] = i;   // stays in range if a slot never lands
+    if (utid() < 32) {
+        // one warp polls, all of its loads in flight at once (a pause between
+        // rounds), so that the waiting CTAs do not flood L2 with loads
+        const int lane = utid();
+        const uint64_t t0 = sm_cycles();
+        uint64_t v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = q * 32 + lane < n ? ld_relaxed_u64(slots + q * 32 + lane) : 1ull;
+        bool late = false;
+        for (;;) {
+            bool have = true;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) have = have && v[q] != 0ull;
+            if (__all_sync(0xFFFFFFFFu, have) || late) break;
+            __nanosleep(200);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (v[q] == 0ull) v[q] = ld_relaxed_u64(slots + q * 32 + lane);
+            late = sm_cycles() - t0 > limit;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (q * 32 + lane < n) cs[q * 32 + lane] = v[q];
+        if (late && lane == 0) atomicOr(p.err, kErrTimeout);
+    }
+    usync();
+    for (int i = utid(); i < n; i += NU) {
+        const uint64_t me = cs[i];
+        if (me == 0ull) continue;
+        int rank = 0;
+        for (int j = 0; j < n; ++j) rank += cs[j] > me ? 1 : 0;
+        if (rank < p.K) byrank[rank] = cand_pos(me);
+    }
+    usync();
+    int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
+    if (utid() < p.K) {
+        // place in ascending order (equal entries, possible only after a
+        // timed-out slot, still take distinct places)
+        const int me = utid();
+        const int32_t v = byrank[me];
+        int r = 0;
+        for (int j = 0; j < p.K; ++j) r += (byrank[j] < v || (byrank[j] == v && j < me)) ? 1 : 0;
+        sel[r] = v;
+        if (publish) p.idx[(size_t)row * p.K + r] = v;
+    }
+    usync();
+}
+
 __device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, int row, bool publish) {
     int32_t* out = p.idx + (size_t)row * p.K;
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
@@ -943,9 +1139,16 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
 // phase open until their copies have landed, the TMA bytes are expected on
 // it, and one thread then gives the one expected arrival.
 __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars* bars, int lt, int seq, int row,
-                                            int tma_rows, int h, bool children) {
-    slot_free(p, bars, seq);
-    slot_free(p, bars, seq + 1);
+                                            int tma_rows, int h, bool children, int gfirst) {
+    if (seq < gfirst + NSL) {
+        // handed over by the producer (see the value stretch)
+        mbar_wait(&bars->gready, 0, p.err);
+    } else {
+        // the previous use of these slots is this CTA's own gathered tile
+        // NSL / 2 tiles back: one phase behind, so a parity wait is exact
+        slot_free(p, bars, seq);
+        slot_free(p, bars, seq + 1);
+    }
     const int sk = seq % NSL, sv = (seq + 1) % NSL;
     uint8_t* ks = base + SM_STAGE + sk * SLOT_BYTES;
     uint8_t* vs = base + SM_STAGE + sv * SLOT_BYTES;
@@ -1034,10 +1237,6 @@ __device__ __forceinline__ void hier_select_children(const Params& p, uint8_t* b
     usync();
 }
 
-// Limit of the cross-CTA waits below (default kWaitLimitNs; a diagnostics
-// setter shortens it so that tests can make such a wait run out).
-__device__ unsigned long long g_cross_wait_ns = kWaitLimitNs;
-
 // Wait (bounded) until counter `ctr` reaches `target`; the writes published
 // before it are then visible to the whole group.  The comparison is
 // wrap-aware (the signed difference), so a counter word that holds a value
@@ -1068,7 +1267,7 @@ __device__ __forceinline__ void wait_count(const Params& p, const uint32_t* ctr,
 // no dependent rescaling chain), folded into a running (M, L, acc) once per
 // group.  Leaves the row's ticket and key counter zero for the next call.
 template <int G>
-__device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int row, int na, int nb) {
+__device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int row, int na, int nb, int ncand) {
     constexpr int NW = NTHR / 32;
     const int nsl = na + nb;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1162,6 +1361,8 @@ __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int ro
         p.cnt[row] = 0;
         p.kdone[row] = 0;
     }
+    // every reader of the row's candidate slots is done (its partial is counted)
+    for (int i = threadIdx.x; i < ncand; i += NTHR) p.cand64[(size_t)row * p.NA + i] = 0ull;
 }
 
 // ---------------------------------------------------------------- kernel --
@@ -1205,6 +1406,8 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
             mbar_init(&b->o_done[i], 1);
         }
         mbar_init(&b->gdone, 128);
+        mbar_init(&b->gready, 1);
+        for (int i = 0; i < kScoreCap / TILE; ++i) mbar_init(&b->sc_full[i], 128);
         fence_mbar_init();
     }
     if (threadIdx.x == 32 * 4) {
@@ -1279,6 +1482,12 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
     const int row_last = n1 > 0 ? (u0 + n1 - 1) / p.upr : -1;
     // slots: keys [0, n1), values [n1, n1 + n2), then two per gathered tile
     const int gseq0 = n1 + n2;
+    int gtiles_total = 0;   // gathered tiles of this CTA's unfold items
+    for (int it = c; it < p.items; it += p.grid)
+        for (int rd = 0; rd < rounds; ++rd) {
+            int t0;
+            gtiles_total += max(0, item_tiles(it, rd, t0));
+        }
 
     // ------------------------------------------------------ key stretch --
     if (cx.warp < 6) {
@@ -1301,6 +1510,8 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         rv.seq0 = n1;
         rv.npre = min(n2, NSL);
         rv.gap = 0;
+        rv.gfirst = gseq0;
+        rv.gwait = min(NSL, 2 * gtiles_total);
         run_pipeline<G>(p, cx, rv);
         // ------------------------------------ gathered tiles, item by item --
         int gseq = gseq0;
@@ -1325,8 +1536,9 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
     } else {
         // ----------------------------------------------- unfold warps --
         const bool lead = utid() == 0;
+        if (p.inc_sel) fold_scores(p, cx.base, cx.bars, c, row_first, row_last);
         asm volatile("bar.sync %0, %1;" ::"n"(BAR_KEYS), "n"(NTHR) : "memory");
-        if (p.do_topk && !p.sel_direct) {
+        if (p.do_topk && !p.sel_direct && !p.inc_sel) {
             // local top-k of every segment, from the scores this CTA kept
             int ntiles = 0;
             for (int r = row_first; r <= row_last; ++r) {
@@ -1357,7 +1569,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         // lead's fence is cumulative: it orders before the counters the
         // streaming warps' scores and the unfold warps' candidates, which the
         // barriers above made visible to it.
-        if (lead) {
+        if (lead && !p.inc_sel) {
             __threadfence();
             for (int r = row_first; r <= row_last; ++r) atomicAdd(p.kdone + r, 1u);
         }
@@ -1366,7 +1578,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
             const int row = it / p.cb, j = it % p.cb;
             int cf;
             const int na = row_ctas(row, cf);
-            if (p.do_topk) wait_count<NU, BAR_UNF>(p, p.kdone + row, (uint32_t)na, lead);
+            if (p.do_topk && !p.inc_sel) wait_count<NU, BAR_UNF>(p, p.kdone + row, (uint32_t)na, lead);
             for (int rd = 0; rd < rounds; ++rd) {
                 int t0;
                 const int ntl = item_tiles(it, rd, t0);
@@ -1380,7 +1592,15 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                 if (rd == 1) {
                     hier_select_children(p, cx.base, row);
                 } else {
-                    if (p.do_topk && p.sel_direct) {
+                    if (p.do_topk && p.inc_sel) {
+                        int n = 0;
+                        for (int cc = cf; cc < cf + na; ++cc) {
+                            int a0, a1;
+                            gists_of(cc, row, a0, a1);
+                            n += min(p.K, max(0, a1 - a0));
+                        }
+                        inc_select(p, cx.base, row, n, j == 0);
+                    } else if (p.do_topk && p.sel_direct) {
                         direct_select(p, cx.base, row, j == 0);
                     } else if (p.do_topk) {
                         int n = 0;
@@ -1410,7 +1630,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                         const int tile = p.hier ? lt : t0 + lt;
                         tma_rows = max(0, min(TILE, kc - tile * TILE));
                     }
-                    gather_tile(p, cx.base, cx.bars, lt, gseq + 2 * lt, row, tma_rows, h, children);
+                    gather_tile(p, cx.base, cx.bars, lt, gseq + 2 * lt, row, tma_rows, h, children, gseq0);
                 }
                 gseq += 2 * ntl;
                 ++runs;
@@ -1440,7 +1660,14 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         int cf;
         const int na = row_ctas(row, cf);
         wait_count<NTHR, 0>(p, p.cnt + row, (uint32_t)(na + p.cb), threadIdx.x == 0);
-        merge_row<G>(p, cx.base, row, na, nb);
+        int ncand = 0;
+        if (p.inc_sel)
+            for (int cc = cf; cc < cf + na; ++cc) {
+                int a0, a1;
+                gists_of(cc, row, a0, a1);
+                ncand += min(p.K, max(0, a1 - a0));
+            }
+        merge_row<G>(p, cx.base, row, na, nb, ncand);
         __syncthreads();
     }
     tc::fence_before();
@@ -1635,6 +1862,8 @@ static void layout_ws(FusedPlan& f, size_t N, size_t top_k, size_t k1) {
     o = round256(o + rows * (size_t)f.slot_stride * f.G * 4 * 4);
     f.off_idx1 = o;
     o = round256(o + rows * k1 * 4);
+    f.off_cand64 = o;
+    if (f.inc_sel) o = round256(o + rows * N * 8);
     f.total = o;
 }
 
@@ -1666,17 +1895,21 @@ FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given) {
 static FusedPlan build_fused_plan(const gsa_decode_desc& d, bool given) {
     FusedPlan f{};
     const bool pairs = d.mode == GSA_SELECTED_PAIRS;
-    f.attn_gists = pairs ? 0 : 1;
+    // gists attended by the stream: all of them, or all but the given
+    // selection (UNSELECTED_GISTS, masked in the key stretch); SELECTED_PAIRS
+    // gathers its gists with the raw rows and SR_ONLY attends none
+    f.attn_gists = (d.mode == GSA_ALL_GISTS || d.mode == GSA_UNSELECTED_GISTS) ? 1 : 0;
     f.rows = d.batch * d.n_kv_heads;
     f.G = d.n_q_heads / d.n_kv_heads;
     // with a given selection in SELECTED_PAIRS mode no gist is scored or attended
-    f.tg = (given && pairs) ? 0 : (d.n_chunks + 127) / 128;
+    f.tg = (given && !f.attn_gists) ? 0 : (d.n_chunks + 127) / 128;
     f.tt = (d.tail_len + 127) / 128;
     f.upr = f.tg + f.tt;
     f.T = f.rows * f.upr;
     // small selections are taken straight from the scores; larger ones from
     // per-CTA candidates the key stretch leaves
     f.sel_direct = (d.top_k <= 32 && d.n_chunks <= 32 * fused::NU) ? 1 : 0;
+    f.inc_sel = 0;
     // unfold: the row's gathered rows packed into 128-row tiles, spread over
     // as many CTAs per row as fill the GPU (at most kMaxTpc tiles each)
     f.nrows_g = d.top_k * d.chunk + (pairs ? d.top_k : 0);
@@ -1690,6 +1923,13 @@ static FusedPlan build_fused_plan(const gsa_decode_desc& d, bool given) {
         f.cb = (f.nbt + f.tpc - 1) / f.tpc;
     }
     place_ctas(f, f.cb);
+    // k <= 32 and at most 2 NU candidates per row: the key stretch keeps
+    // running top-k lists and publishes each CTA's candidates
+    if (!given && d.top_k >= 1 && d.top_k <= 32 && f.maxs * d.top_k <= 2 * fused::NU &&
+        (f.T + f.grid - 1) / f.grid <= fused::kScoreCap / 128) {
+        f.inc_sel = 1;
+        f.sel_direct = 0;
+    }
     layout_ws(f, (size_t)d.n_chunks, (size_t)d.top_k, 0);
     return f;
 }
@@ -1718,6 +1958,8 @@ static void fill_common(fused::Params& p, const FusedPlan& f, const gsa_decode_d
     p.tpc = f.tpc;
     p.cb = f.cb;
     p.sel_direct = f.sel_direct;
+    p.inc_sel = f.inc_sel;
+    p.cand64 = reinterpret_cast<uint64_t*>(w + f.off_cand64);
     p.tmem_cols = f.tmem_cols;
     const double scale = d.scale > 0 ? (double)d.scale : 1.0 / std::sqrt(128.0);
     p.c2 = (float)(scale * 1.4426950408889634);
@@ -1731,8 +1973,7 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
     Params p;
     std::memset(&p, 0, sizeof(p));
     const uint64_t rows = (uint64_t)f.rows, N = (uint64_t)d.n_chunks;
-    const bool pairs = d.mode == GSA_SELECTED_PAIRS;
-    bool ok = map3d(&p.tm_kg, kg, rows, N) && map3d(&p.tm_vg, pairs ? nullptr : vg, rows, N) &&
+    bool ok = map3d(&p.tm_kg, kg, rows, N) && map3d(&p.tm_vg, f.attn_gists ? vg : nullptr, rows, N) &&
               map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
     p.tma_raw = chunk_runs(d.chunk) && f.nbt > 0 ? 1 : 0;
     if (p.tma_raw)
@@ -1757,7 +1998,9 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
     p.nrows_g = f.nrows_g;
     p.do_score = idx_given ? 0 : 1;
     p.do_topk = idx_given ? 0 : 1;
-    p.do_attn_gists = pairs ? 0 : 1;
+    p.do_attn_gists = f.attn_gists;
+    // a given selection in UNSELECTED_GISTS mode: its gists leave the context
+    p.mask_sel = (idx_given != nullptr && d.mode == GSA_UNSELECTED_GISTS) ? 1 : 0;
     return launch(p, f.G, f.grid, st) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
@@ -1786,6 +2029,10 @@ FusedPlan make_fused_hier_plan(const gsa_hier_desc& h) {
     f.tpc = 2;
     f.cb = 1;
     place_ctas(f, 2);
+    f.inc_sel = (h.top_k2 >= 1 && h.top_k2 <= 32 && f.maxs * h.top_k2 <= 2 * fused::NU &&
+                 (f.T + f.grid - 1) / f.grid <= fused::kScoreCap / 128) ? 1 : 0;
+    if (f.inc_sel) f.sel_direct = 0;
+    else f.sel_direct = (h.top_k2 <= 32 && h.n_l2 <= 32 * fused::NU) ? 1 : 0;
     layout_ws(f, (size_t)h.n_l2, (size_t)h.top_k2, (size_t)h.l1.top_k);
     return f;
 }

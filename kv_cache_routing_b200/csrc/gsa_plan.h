@@ -34,7 +34,9 @@ inline int stage_keys(int dtype, int head_dim) { return 16384 / (head_dim * elem
 inline gsa_status validate_decode(const gsa_decode_desc* d) {
     if (!d) return GSA_ERR_ARG;
     if (d->dtype != GSA_F32 && d->dtype != GSA_BF16) return GSA_ERR_DTYPE;
-    if (d->mode != GSA_ALL_GISTS && d->mode != GSA_SELECTED_PAIRS) return GSA_ERR_ARG;
+    if (d->mode != GSA_ALL_GISTS && d->mode != GSA_SELECTED_PAIRS && d->mode != GSA_SR_ONLY &&
+        d->mode != GSA_UNSELECTED_GISTS)
+        return GSA_ERR_ARG;
     if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1) return GSA_ERR_SHAPE;
     if (d->n_q_heads % d->n_kv_heads != 0) return GSA_ERR_SHAPE;
     const int G = d->n_q_heads / d->n_kv_heads;
@@ -48,7 +50,10 @@ inline gsa_status validate_decode(const gsa_decode_desc* d) {
     // element counts must fit the kernels' 32-bit per-row key arithmetic
     if (kb > INT32_MAX / 2 || (int64_t)d->n_chunks * d->chunk > INT32_MAX / 2) return GSA_ERR_SHAPE;
     if (rows > 65535) return GSA_ERR_SHAPE;   // grid.y
-    const int64_t ctx = (d->mode == GSA_ALL_GISTS ? d->n_chunks : 0) + kb;
+    // gists in the context: all, the selected ones (counted in kb), none, or the unselected ones
+    const int64_t gists = d->mode == GSA_ALL_GISTS ? d->n_chunks
+                        : d->mode == GSA_UNSELECTED_GISTS ? (int64_t)d->n_chunks - d->top_k : 0;
+    const int64_t ctx = gists + kb;
     if (ctx <= 0) return GSA_ERR_ARG;         // empty attention context
     return GSA_OK;
 }

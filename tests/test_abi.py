@@ -50,6 +50,8 @@ def _desc(**kw):
     (dict(dtype=7), gsa.GSA_ERR_DTYPE),
     (dict(mode=5), gsa.GSA_ERR_ARG),
     (dict(mode=gsa.GSA_SELECTED_PAIRS, top_k=0, tail_len=0), gsa.GSA_ERR_ARG),   # empty context
+    (dict(mode=gsa.GSA_SR_ONLY, top_k=0, tail_len=0), gsa.GSA_ERR_ARG),          # empty context
+    (dict(mode=4), gsa.GSA_ERR_ARG),
     (dict(batch=0), gsa.GSA_ERR_SHAPE),
 ])
 def test_descriptor_validation(kw, code):
@@ -111,6 +113,11 @@ def test_launch_counts_follow_the_path():
     assert gsa.gsa_decode_launch_count(_desc(dtype=gsa.GSA_F32)) == 2
     assert gsa.gsa_decode_launch_count(_desc(head_dim=64)) == 2
     assert gsa.gsa_decode_launch_count(_desc(head_dim=64, n_chunks=0, top_k=0)) == 1
+    # SR-only is one step; the unselected-gists step scores, selects, then attends
+    assert gsa.gsa_decode_launch_count(_desc(mode=gsa.GSA_SR_ONLY)) == 1
+    assert gsa.gsa_decode_launch_count(_desc(mode=gsa.GSA_UNSELECTED_GISTS)) == 3
+    assert gsa.gsa_decode_launch_count(_desc(mode=gsa.GSA_UNSELECTED_GISTS, dtype=gsa.GSA_F32)) == 4
+    assert gsa.gsa_decode_launch_count(_desc(mode=gsa.GSA_UNSELECTED_GISTS, top_k=0)) == 1
     with pytest.raises(gsa.GsaError):
         gsa.gsa_decode_launch_count(_desc(head_dim=96))
     l1 = _desc(n_chunks=160, top_k=8)

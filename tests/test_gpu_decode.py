@@ -9,7 +9,7 @@ import torch
 import kv_cache_routing_b200 as gsa
 import oracle
 import synth
-from synth import ALL_GISTS, SELECTED_PAIRS, DecodeShape
+from synth import ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS, DecodeShape
 
 from gsa_check import (check_out, check_selection, desc_of, dev, gpu_decode_step, host, tdtype, upload,
                        workspace)
@@ -50,6 +50,62 @@ def test_decode_configs_full(name):
 def test_decode_compression_sweep_full(name):
     s = synth.WORKLOADS[name]
     _run_and_check(s, synth.seed_for(name), name)
+
+
+@pytest.mark.parametrize("name", ["sweep_c16_all", "sweep_c8_all"])
+@pytest.mark.parametrize("mode", [SR_ONLY, UNSELECTED_GISTS])
+def test_decode_gist_rules_full(name, mode):
+    """The two further context rules at full compression-sweep size (k > 32)."""
+    s = dataclasses.replace(synth.WORKLOADS[name], mode=mode)
+    _run_and_check(s, synth.seed_for(name), f"{name} mode {mode}")
+
+
+GIST_RULE_EDGE = {
+    # k <= 32 (running top-k lists in the key stretch), tensor-core path
+    "llama_rows": DecodeShape(2, 32, 8, 128, 2048, 16, 16, 64, "bf16", ALL_GISTS, n_needles=16),
+    # fp32 / d = 64: the CUDA-core passes
+    "f32_d64": DecodeShape(2, 8, 2, 64, 300, 8, 6, 10, "f32", ALL_GISTS, n_needles=6),
+    # k = N and k = 0
+    "k_all": DecodeShape(1, 8, 2, 128, 40, 8, 40, 12, "bf16", ALL_GISTS),
+    "k_none": DecodeShape(1, 8, 2, 128, 300, 16, 0, 12, "bf16", ALL_GISTS),
+    "k_all_f32": DecodeShape(1, 4, 1, 64, 37, 4, 37, 3, "f32", ALL_GISTS),
+    "ragged": DecodeShape(2, 8, 2, 128, 1000, 3, 7, 5, "bf16", ALL_GISTS, n_needles=7),
+}
+
+
+@pytest.mark.parametrize("name", sorted(GIST_RULE_EDGE))
+@pytest.mark.parametrize("mode", [SR_ONLY, UNSELECTED_GISTS])
+def test_decode_gist_rules_edge(name, mode):
+    s = dataclasses.replace(GIST_RULE_EDGE[name], mode=mode)
+    if s.top_k == 0 and s.tail_len == 0 and mode == SR_ONLY:
+        pytest.skip("empty context")
+    _run_and_check(s, 2000 + sorted(GIST_RULE_EDGE).index(name), f"{name} mode {mode}")
+
+
+@pytest.mark.parametrize("dt,d", [("bf16", 128), ("f32", 64)])
+def test_unfold_attn_given_selection_gist_rules(dt, d):
+    """gsa_unfold_attn with a given (unsorted) selection in the two further
+    rules: the tensor-core step masks the selected gists in its key stretch,
+    the CUDA-core gist pass in its logits."""
+    s = DecodeShape(2, 8, 2, d, 700, 8, 11, 20, dt, ALL_GISTS, n_needles=11)
+    x = synth.decode_inputs(s, 90)
+    t = x.tensors()
+    dd = upload(x)
+    rng = np.random.default_rng(5)
+    idx = np.stack([np.stack([rng.permutation(700)[:11] for _ in range(2)]) for _ in range(2)]).astype(np.int32)
+    for mode in (SR_ONLY, UNSELECTED_GISTS):
+        sm = dataclasses.replace(s, mode=mode)
+        dm = desc_of(sm)
+        ws = workspace(gsa.gsa_decode_workspace_size(dm))
+        out = torch.empty((2, 8, d), dtype=tdtype(dt), device="cuda")
+        lse = torch.empty((2, 8), dtype=torch.float32, device="cuda")
+        gsa.gsa_unfold_attn(dm, dd["q"], dd["k_gist"], dd["v_gist"], dd["k_raw"], dd["v_raw"], dd["k_tail"],
+                            dd["v_tail"], dev(idx), out, lse, ws)
+        torch.cuda.synchronize()
+        assert gsa.gsa_workspace_error(ws) == 0
+        o_ex, l_ex = oracle.unfold_attn(t, idx, mode, with_lse=True)
+        check_out(host(out), o_ex, dt, f"unfold {dt} mode {mode}")
+        assert np.max(np.abs(lse.cpu().numpy() - l_ex)) < (1e-5 if dt == "f32" else 1e-3)
 
 
 EDGE = {

@@ -44,6 +44,7 @@ def _load():
         "oracle_gist_scores": [i, i, i, i, i, i, vp, vp, vp],
         "oracle_topk": [i, i, i, vp, vp],
         "oracle_topk_gap": [i, i, i, vp, vp],
+        "oracle_topp": [i, i, i, d, d, vp, vp, vp],
         "oracle_score_error_bound": [i, i, i, i, i, i, vp, vp, vp],
         "oracle_decode": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
         "oracle_unfold_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
@@ -98,6 +99,19 @@ def topk(scores: np.ndarray, k: int) -> np.ndarray:
     idx = np.empty(s.shape[:-1] + (k,), np.int32)
     _load().oracle_topk(rows, N, k, _p(s), _p(idx))
     return idx
+
+
+def topp(scores: np.ndarray, p: float, kmax: int, scale: float):
+    """Top-p selection of each row of scores [..., N] (fp64): the shortest
+    prefix of the top-k order whose softmax(scale * s) mass reaches p, cut at
+    kmax.  Returns (idx [..., kmax] int32 ascending then -1, count [...])."""
+    s = np.ascontiguousarray(scores, np.float64)
+    N = s.shape[-1]
+    rows = int(np.prod(s.shape[:-1])) if s.ndim > 1 else 1
+    idx = np.empty(s.shape[:-1] + (kmax,), np.int32)
+    cnt = np.empty(s.shape[:-1], np.int32)
+    _load().oracle_topp(rows, N, kmax, float(p), float(scale), _p(s), _p(idx), _p(cnt))
+    return idx, cnt
 
 
 def topk_gap(scores: np.ndarray, k: int) -> np.ndarray:

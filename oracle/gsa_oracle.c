@@ -19,7 +19,10 @@
  *   [SL-10]  slide deck, page 10 "Training, Stage 2" — top-k worked example;
  *   [SL-11]  slide deck, page 11 "Hierarchical Gist-of-Gist Compression";
  *   [SL-17]  slide deck, page 17 "Selective Rules Comparison" — SR-only,
- *            AG+SR, SG+SR.
+ *            AG+SR, SG+SR;
+ *   [SL-18]  slide deck, page 18 "Top-k vs. Top-p";
+ *   [DE-E]   gist.science explainer (DE), section "Ergebnisse" (top-p /
+ *            nucleus selection).
  *
  * Every floating-point value is widened exactly to double before use; all
  * arithmetic is in double.  Softmax is the two-pass textbook form.
@@ -133,6 +136,47 @@ void oracle_topk_gap(int rows, int N, int k, const double* s, double* gap) {
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Top-p (nucleus) chunk selection.  [SL-18] "Top-k vs. Top-p" and [DE-E]     */
+/* "Ergebnisse" compare a fixed top-p selection with top-k; the pages give no */
+/* formula.  Reading taken: the routing distribution of a row is the softmax  */
+/* of the scaled routing scores, pi_j = exp(scale s_j) / sum_i exp(scale s_i);*/
+/* the chunks are taken in the top-k order (higher score first, the lower     */
+/* index on ties), and the selection is the shortest prefix of that order     */
+/* whose mass reaches p (at least one chunk), cut at kmax.  Output: the       */
+/* selected indices ascending, then -1 up to kmax; count[r] = their number.   */
+/* ------------------------------------------------------------------------ */
+void oracle_topp(int rows, int N, int kmax, double p, double scale, const double* s, int32_t* idx,
+                 int32_t* count) {
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        const double* sr = s + (int64_t)r * N;
+        scored_t* all = (scored_t*)malloc(sizeof(scored_t) * (size_t)(N > 0 ? N : 1));
+        double mx = -INFINITY;
+        for (int t = 0; t < N; ++t) {
+            all[t].s = sr[t];
+            all[t].j = t;
+            if (sr[t] > mx) mx = sr[t];
+        }
+        qsort(all, (size_t)N, sizeof(scored_t), by_score_desc_then_index);
+        double z = 0.0;
+        for (int t = 0; t < N; ++t) z += exp(scale * (sr[t] - mx));
+        int m = 0;
+        double acc = 0.0;
+        while (m < N && m < kmax) {
+            acc += exp(scale * (all[m].s - mx)) / z;
+            ++m;
+            if (acc >= p) break;
+        }
+        int32_t* out = idx + (int64_t)r * kmax;
+        for (int t = 0; t < m; ++t) out[t] = all[t].j;
+        qsort(out, (size_t)m, sizeof(int32_t), by_index);
+        for (int t = m; t < kmax; ++t) out[t] = -1;
+        count[r] = m;
+        free(all);
+    }
+}
+
 /* Rounding-error bound of an fp32 evaluation of each score, any summation   */
 /* order (Higham, "Accuracy and Stability of Numerical Algorithms", 2nd ed., */
 /* eq. 3.5, inner products):  |fl(s) - s| <= gamma_n * sum |q_i k_i|,        */
@@ -208,7 +252,8 @@ static int flat_context(int Hkv, int d, int N, int c, int W, int mode, int b, in
     if (mode == OR_ALL_GISTS) {
         for (int j = 0; j < N; ++j) keys[n++] = (key_ref){kg, vg, (row * N + j) * d};
     } else if (mode == OR_SELECTED_PAIRS) {
-        for (int t = 0; t < k; ++t) keys[n++] = (key_ref){kg, vg, (row * N + sel[t]) * d};
+        for (int t = 0; t < k; ++t)
+            if (sel[t] >= 0) keys[n++] = (key_ref){kg, vg, (row * N + sel[t]) * d};
     } else if (mode == OR_UNSELECTED_GISTS) {
         for (int j = 0; j < N; ++j) {
             int selected = 0;
@@ -217,8 +262,9 @@ static int flat_context(int Hkv, int d, int N, int c, int W, int mode, int b, in
         }
     }   /* OR_SR_ONLY: no gist */
     for (int t = 0; t < k; ++t)
-        for (int u = 0; u < c; ++u)
-            keys[n++] = (key_ref){kraw, vraw, ((row * N + sel[t]) * c + u) * d};
+        if (sel[t] >= 0)   /* -1: an empty place of a variable-size (top-p) selection */
+            for (int u = 0; u < c; ++u)
+                keys[n++] = (key_ref){kraw, vraw, ((row * N + sel[t]) * c + u) * d};
     for (int u = 0; u < W; ++u) keys[n++] = (key_ref){ktail, vtail, (row * W + u) * d};
     return n;
 }

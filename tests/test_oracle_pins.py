@@ -7,6 +7,7 @@ assembled key list or a boolean mask, selection against ``numpy.lexsort``,
 scores against one-hot closed forms, the prefill mask against the slide's
 table and a pair-count closed form.
 """
+import dataclasses
 import math
 
 import numpy as np
@@ -465,3 +466,74 @@ def test_hier_given_selection_reproduces_own_selection():
     idx2, idx1, out = oracle.hier_decode(t, h.group, h.top_k2, h.l1.top_k)
     _, _, out2 = oracle.hier_decode(t, h.group, h.top_k2, h.l1.top_k, given=(idx2, idx1))
     np.testing.assert_array_equal(out, out2)
+
+
+# ------------------------------------------------------------------ top-p ----
+def test_topp_slide10_scores_by_hand():
+    """Slide 10's scores 0.1 / 0.8 / 0.7 / 0.2 under softmax with scale 1.
+    By hand: e^0.1 = 1.1051709, e^0.8 = 2.2255409, e^0.7 = 2.0137527,
+    e^0.2 = 1.2214028, sum 6.5658673, so the masses are 0.168321, 0.338957,
+    0.306700, 0.186022.  In score order (g2, g3, g4, g1) they accumulate to
+    0.338957, 0.645657, 0.831679, 1."""
+    s = np.array([[0.1, 0.8, 0.7, 0.2]])
+    cases = [(0.30, [1]), (0.60, [1, 2]), (0.65, [1, 2, 3]), (0.83, [1, 2, 3]), (0.84, [0, 1, 2, 3])]
+    for p, want in cases:
+        idx, cnt = oracle.topp(s, p, 4, 1.0)
+        assert cnt[0] == len(want), p
+        assert idx[0, :cnt[0]].tolist() == want, p
+        assert (idx[0, cnt[0]:] == -1).all()
+    # cut at kmax: p = 0.9 would need all four
+    idx, cnt = oracle.topp(s, 0.9, 2, 1.0)
+    assert cnt[0] == 2 and idx[0].tolist() == [1, 2]
+
+
+def test_topp_uniform_mass_closed_form():
+    """scale 0 makes every chunk weigh 1/N: the count is ceil(p N), taken in
+    the top-k order (lexsort)."""
+    rng = np.random.default_rng(3)
+    s = rng.standard_normal((4, 10))
+    for p, m in [(0.35, 4), (0.05, 1), (0.5, 5), (0.91, 10)]:
+        idx, cnt = oracle.topp(s, p, 10, 0.0)
+        assert (cnt == m).all(), p
+        for r in range(4):
+            want = np.sort(np.lexsort((np.arange(10), -s[r]))[:m])
+            assert idx[r, :m].tolist() == want.tolist()
+
+
+def test_topp_is_the_shortest_prefix_reaching_p():
+    """Invariants on random rows against library routines (softmax of the
+    scaled scores, lexsort order): the selected mass reaches p, the mass
+    without the last chunk of the prefix does not, and the set is that prefix."""
+    rng = np.random.default_rng(11)
+    s = rng.standard_normal((50, 64)) * 3.0
+    s[::7, 5] = s[::7, 9]                      # ties
+    scale = 0.7
+    for p in (0.2, 0.5, 0.9, 0.99):
+        idx, cnt = oracle.topp(s, p, 64, scale)
+        for r in range(50):
+            w = np.exp(scale * (s[r] - s[r].max()))
+            w /= w.sum()
+            order = np.lexsort((np.arange(64), -s[r]))
+            m = int(cnt[r])
+            assert w[order[:m]].sum() >= p - 1e-12
+            assert m == 1 or w[order[:m - 1]].sum() < p
+            assert idx[r, :m].tolist() == np.sort(order[:m]).tolist()
+
+
+def test_padded_selection_equals_the_compacted_one():
+    """A selection padded with -1 (variable size, as top-p returns it) attends
+    exactly the context of its non-negative entries."""
+    sh = small_shape(n_chunks=9, chunk=4, top_k=4, tail_len=3)
+    x = synth.decode_inputs(sh, 47)
+    t = x.tensors()
+    full = np.array([[[1, 4, 6, 8], [0, 2, 3, 7]], [[2, 5, -1, -1], [8, -1, -1, -1]]], np.int32)
+    for mode in (ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS):
+        out = oracle.unfold_attn(t, full, mode, 0.4)
+        for b in range(2):
+            for hk in range(2):
+                kept = full[b, hk][full[b, hk] >= 0]
+                one = {k: v[b:b + 1, hk:hk + 1].copy() for k, v in t.items()}
+                one["q"] = t["q"][b:b + 1, hk * sh.group:(hk + 1) * sh.group].copy()
+                sub = dataclasses.replace(sh, top_k=len(kept))
+                want = oracle.unfold_attn(one, kept.reshape(1, 1, -1), mode, 0.4)
+                np.testing.assert_array_equal(out[b, hk * sh.group:(hk + 1) * sh.group], want[0])

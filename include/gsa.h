@@ -9,9 +9,10 @@
  *           Attention" (interleaved gist tokens; gist as routing signals;
  *           selective unfolding; hybrid attention; hierarchical extension);
  *   [DE-M]  gist.science explainer (DE), section "Methodik";
+ *   [DE-E]  gist.science explainer (DE), section "Ergebnisse";
  *   [SL-n]  Taki-lab slide deck (docswell), page n: 6 "GSA とは", 7 "Gist
  *           token", 9/10 "Training", 11 "H-GSA", 17 "Selective Rules
- *           Comparison".
+ *           Comparison", 18 "Top-k vs. Top-p".
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -146,13 +147,27 @@ gsa_status gsa_score(const gsa_decode_desc* desc, const void* q, const void* k_g
  * idx [B][Hkv][k].                                                         */
 gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* idx, void* stream);
 
+/* Top-p (nucleus) chunk selection ([SL-18] "Top-k vs. Top-p"; [DE-E]
+ * "Ergebnisse": a fixed top-p selection is compared with top-k).  The pages
+ * give no formula; the reading taken: per (b, hk) the routing distribution
+ * is the softmax of scale * scores (scale as in the descriptor), the chunks
+ * are taken in the top-k order (higher score first, the lower index on
+ * ties), and the selection is the shortest prefix of that order whose mass
+ * reaches top_p, at least one chunk and at most kmax = desc->top_k chunks.
+ * Weights and sums are fp32.  Reads scores [B][Hkv][N]; writes idx
+ * [B][Hkv][kmax] (the selected chunks ascending, then -1) and count [B][Hkv]
+ * (nullable).  0 < top_p <= 1, 1 <= kmax <= 2048; scores must be finite.   */
+gsa_status gsa_topp(const gsa_decode_desc* desc, float top_p, const float* scores, int32_t* idx,
+                    int32_t* count, void* stream);
+
 /* Selective unfolding + hybrid attention ([EN-2] "Selective Unfolding",
  * "Hybrid Attention"; [DE-M] "Selektive Entfaltung", "Hybride Attention";
  * [SL-17]).  For every query head h of KV head hk the softmax of
  * scale * q_h . K over the context of desc->mode, times V, where the selected
- * chunks are idx[b][hk][0..k) (distinct, in [0, N); an index out of range is
- * clamped into range and flagged).  lse (nullable) [B][Hq] receives the natural-log
- * sum of exp(scale * q.K) over the context.                               */
+ * chunks are idx[b][hk][0..k) (distinct, in [0, N); -1 marks an empty place
+ * of a variable-size selection such as gsa_topp's and adds nothing; any other
+ * index out of range is clamped into range and flagged).  lse (nullable)
+ * [B][Hq] receives the natural-log sum of exp(scale * q.K) over the context. */
 gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist,
                            const void* v_gist, const void* k_raw, const void* v_raw,
                            const void* k_tail, const void* v_tail, const int32_t* idx, void* out,
@@ -166,6 +181,18 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
                            const void* v_gist, const void* k_raw, const void* v_raw,
                            const void* k_tail, const void* v_tail, int32_t* idx_out,
                            float* scores_out, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* One decode step with top-p selection: gsa_score -> gsa_topp ->
+ * gsa_unfold_attn (three launches on the tensor-core path).  desc->top_k is
+ * kmax; idx_out [B][Hkv][kmax] receives the selection padded with -1,
+ * count_out [B][Hkv] its size, scores_out the routing scores (all three
+ * nullable; the workspace holds them otherwise).  Other arguments as for
+ * gsa_decode_step.                                                          */
+gsa_status gsa_decode_step_topp(const gsa_decode_desc* desc, float top_p, const void* q, const void* k_gist,
+                                const void* v_gist, const void* k_raw, const void* v_raw,
+                                const void* k_tail, const void* v_tail, int32_t* idx_out,
+                                int32_t* count_out, float* scores_out, void* out, void* ws,
+                                size_t ws_bytes, void* stream);
 
 /* Hierarchical decode: level-2 scores over every meta-gist -> top-k2 groups;
  * level-1 scores over the gists of those groups -> top-k1 chunks among them;

@@ -24,7 +24,8 @@ GSA_WS_ERR_TIMEOUT, GSA_WS_ERR_INDEX = 1, 2
 EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", "gsa_topk",
            "gsa_unfold_attn", "gsa_decode_step", "gsa_hier_decode", "gsa_gist_prefill",
            "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count",
-           "gsa_hier_launch_count", "gsa_device_error", "gsa_set_wait_limit_ns")
+           "gsa_hier_launch_count", "gsa_device_error", "gsa_set_wait_limit_ns", "gsa_topp",
+           "gsa_decode_step_topp")
 
 
 class GsaError(RuntimeError):
@@ -70,6 +71,8 @@ def _signatures():
         "gsa_gist_prefill": (st, [pp, vp, vp, vp, vp, vp, vp]),
         "gsa_workspace_error": (st, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
         "gsa_device_error": (st, [ctypes.POINTER(ctypes.c_uint32), vp]),
+        "gsa_topp": (st, [pd, ctypes.c_float, vp, vp, vp, vp]),
+        "gsa_decode_step_topp": (st, [pd, ctypes.c_float] + [vp] * 11 + [sz, vp]),
         "gsa_set_wait_limit_ns": (st, [ctypes.c_uint64]),
         "gsa_status_string": (ctypes.c_char_p, [st]),
         "gsa_decode_launch_count": (ctypes.c_int, [pd]),
@@ -242,3 +245,17 @@ def gsa_device_error(stream=None) -> int:
 def gsa_set_wait_limit_ns(ns: int):
     """Diagnostics: limit of the cross-CTA waits of a decode launch (0: default)."""
     _check(lib().gsa_set_wait_limit_ns(int(ns)), "gsa_set_wait_limit_ns")
+
+
+def gsa_topp(desc, top_p, scores, idx, count=None, stream=None):
+    _check(lib().gsa_topp(ctypes.byref(desc), float(top_p), _ptr(scores), _ptr(idx), _ptr(count), _stream(stream)),
+           "gsa_topp")
+
+
+def gsa_decode_step_topp(desc, top_p, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, count_out,
+                         scores_out, out, ws, stream=None, ws_bytes=None):
+    nb = _nbytes(ws) if ws_bytes is None else ws_bytes
+    _check(lib().gsa_decode_step_topp(ctypes.byref(desc), float(top_p), _ptr(q), _ptr(k_gist), _ptr(v_gist),
+                                      _ptr(k_raw), _ptr(v_raw), _ptr(k_tail), _ptr(v_tail), _ptr(idx_out),
+                                      _ptr(count_out), _ptr(scores_out), _ptr(out), _ptr(ws), nb, _stream(stream)),
+           "gsa_decode_step_topp")

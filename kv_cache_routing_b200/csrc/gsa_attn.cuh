@@ -166,8 +166,10 @@ struct WarpAttn {
     }
 
     // Online softmax over the warp tile (first nv keys valid) and P.V.
+    // (vmask: keys of the tile that take part; a key outside it gets no weight)
     __device__ __forceinline__ void softmax_pv(const uint8_t* vt /* warp tile V rows */,
-                                               WarpScratch<G, C::TW>& ws, int nv, float c2, int lane) {
+                                               WarpScratch<G, C::TW>& ws, int nv, float c2, int lane,
+                                               uint32_t vmask = 0xFFFFFFFFu) {
         const int sub = lane & (C::LPK - 1);
         const int hf = lane >> C::LOG_LPK;
         const int hl = lane / C::LPH;                     // this lane's head (softmax phase)
@@ -177,7 +179,7 @@ struct WarpAttn {
         for (int u = 0; u < C::PPL; ++u) {
             const int pi = lane * C::PPL + u;             // head-major pair index
             const int key = pi % C::TW;
-            x[u] = (lane < C::ACT && key < nv) ? ws.lg[key * G + hl] * c2 : kNegInf;
+            x[u] = (lane < C::ACT && key < nv && ((vmask >> key) & 1u)) ? ws.lg[key * G + hl] * c2 : kNegInf;
             mt = fmaxf(mt, x[u]);
         }
 #pragma unroll

@@ -292,7 +292,9 @@ __device__ __forceinline__ void unfold_issue(const PassParams& p, int row, int x
         if (x < kU) {
             const int u = x / p.U, r = x % p.U;
             int j = __ldcg(p.idx_in + (size_t)row * p.K + u);
-            if (j < 0 || j >= p.N) {
+            if (j == -1) {
+                j = 0;   // an empty place of a variable-size selection: copied, then masked
+            } else if (j < 0 || j >= p.N) {
                 atomicOr(p.err, kErrIndex);
                 j = j < 0 ? 0 : p.N - 1;
             }
@@ -373,8 +375,12 @@ __global__ void __launch_bounds__(NTHREADS, 3) unfold_pass_kernel(const __grid_c
             const int nk = min(C::TILE, x1 - xa);
             const int nv = min(C::TW, nk - warp * C::TW);
             if (nv > 0) {
+                // keys of an empty place (-1) of the selection take no part
+                const int x = xa + warp * C::TW + lane;
+                const bool gone = lane < nv && x < p.K * p.U && __ldcg(p.idx_in + (size_t)row * p.K + x / p.U) == -1;
+                const uint32_t vmask = ~__ballot_sync(0xFFFFFFFFu, gone);
                 wa.qk(sm.stage[slot][0] + warp * C::TW * C::ROWB, ws, lane);
-                wa.softmax_pv(sm.stage[slot][1] + warp * C::TW * C::ROWB, ws, nv, p.c2, lane);
+                wa.softmax_pv(sm.stage[slot][1] + warp * C::TW * C::ROWB, ws, nv, p.c2, lane, vmask);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[slot]);
@@ -463,6 +469,100 @@ __global__ void __launch_bounds__(NTHREADS) topk_kernel(const float* __restrict_
     pdl_wait();
     block_topk<NTHREADS>(
         N, K, [&](int i) { return order_key(sc[i]); }, [&](int r, int i) { out[r] = i; }, sh);
+}
+
+// =============================================================== top-p =====
+// Top-p selection, one CTA per row: the row's softmax weights w = 2^((s -
+// max) c2) and their sum Z; the exact top-kmax by the block radix select (in
+// index order); each of those ranked in score order (higher score, then the
+// lower index) by counting; the weights placed in rank order and prefix-summed
+// (a block scan over contiguous segments); the cut is the first rank at which
+// the prefix reaches p Z.  The selected positions are written ascending, then
+// -1 up to kmax, and their number to count.  NaN scores weigh nothing.
+constexpr int kToppMax = 2048;   // largest kmax of gsa_topp
+__global__ void __launch_bounds__(NTHREADS) topp_kernel(const float* __restrict__ scores, int N, int kmax, float p,
+                                                        float c2, int32_t* __restrict__ idx, int32_t* count) {
+    extern __shared__ __align__(16) uint32_t dyn[];   // pos, key, rank [kmax] and weights in rank order [kmax]
+    __shared__ uint32_t sh[256 + 8 + NTHREADS / 32 + 8];
+    __shared__ float red[NTHREADS / 32];
+    __shared__ int cut;
+    const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = NTHREADS / 32;
+    const float* sc = scores + (size_t)row * N;
+    int32_t* pos = reinterpret_cast<int32_t*>(dyn);
+    uint32_t* key = dyn + kmax;
+    int32_t* rnk = reinterpret_cast<int32_t*>(dyn + 2 * kmax);
+    float* wr = reinterpret_cast<float*>(dyn + 3 * kmax);
+    pdl_wait();
+    const int kk = min(kmax, N);
+    // the row's maximum and the softmax normaliser
+    float mx = kNegInf;
+    for (int i = tid; i < N; i += NTHREADS) mx = fmaxf(mx, sc[i]);
+    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    mx = red[0];
+    for (int w = 1; w < NW; ++w) mx = fmaxf(mx, red[w]);
+    __syncthreads();
+    auto weight = [&](float x) { return x == x ? exp2f((x - mx) * c2) : 0.f; };
+    float z = 0.f;
+    for (int i = tid; i < N; i += NTHREADS) z += weight(sc[i]);
+    for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+    if (lane == 0) red[warp] = z;
+    __syncthreads();
+    z = 0.f;
+    for (int w = 0; w < NW; ++w) z += red[w];
+    const float target = p * z;
+    // the top-kmax, in index order
+    block_topk<NTHREADS>(
+        N, kk, [&](int i) { return order_key(sc[i]); }, [&](int r, int i) { pos[r] = i; }, sh);
+    __syncthreads();
+    for (int r = tid; r < kk; r += NTHREADS) key[r] = order_key(sc[pos[r]]);
+    __syncthreads();
+    // rank in score order (pos is ascending, so r' < r means a lower index)
+    for (int r = tid; r < kk; r += NTHREADS) {
+        const uint32_t kr = key[r];
+        int rank = 0;
+        for (int q = 0; q < kk; ++q) rank += (key[q] > kr || (key[q] == kr && q < r)) ? 1 : 0;
+        rnk[r] = rank;
+        wr[rank] = weight(sc[pos[r]]);
+    }
+    if (tid == 0) cut = kk;
+    __syncthreads();
+    // prefix sums of the weights in rank order: contiguous segments, then a scan of their totals
+    const int seg = (kk + NTHREADS - 1) / NTHREADS;
+    const int lo = min(kk, tid * seg), hi = min(kk, lo + seg);
+    float part = 0.f;
+    for (int t = lo; t < hi; ++t) part += wr[t];
+    float incl = part;
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    float before = incl - part;
+    for (int w = 0; w < warp; ++w) before += red[w];
+    float acc = before;
+    for (int t = lo; t < hi; ++t) {
+        acc += wr[t];
+        if (acc >= target) {
+            atomicMin(&cut, t + 1);
+            break;
+        }
+    }
+    __syncthreads();
+    const int m = max(1, cut);
+    // the selected positions (rank < m), ascending, then -1
+    uint32_t n_sel = 0;
+    for (int t = lo; t < hi; ++t) n_sel += rnk[t] < m ? 1u : 0u;
+    uint32_t tot;
+    uint32_t at = block_exclusive_scan<NTHREADS>(n_sel, sh, &tot);
+    int32_t* out = idx + (size_t)row * kmax;
+    for (int t = lo; t < hi; ++t)
+        if (rnk[t] < m) out[at++] = pos[t];
+    for (int t = m + tid; t < kmax; t += NTHREADS) out[t] = -1;
+    if (count != nullptr && tid == 0) count[row] = m;
 }
 
 // ============================================================ host side ====
@@ -601,6 +701,7 @@ static size_t decode_ws_bytes(const gsa_decode_desc& d) {
 // UNSELECTED_GISTS decode step: where the scores and the selection go when the
 // caller passes no buffers for them.  Both plans keep score and selection
 // regions that the given-selection pass does not use.
+// (also the top-p step's, which runs the same three kernels)
 static void unselected_scratch(const gsa_decode_desc& d, size_t& off_scores, size_t& off_idx) {
     if (fused_supported(d)) {
         const FusedPlan f = make_fused_plan(d, true);
@@ -653,6 +754,22 @@ gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* i
     const int rows = desc->batch * desc->n_kv_heads;
     topk_kernel<<<rows, NTHREADS, 0, static_cast<cudaStream_t>(stream)>>>(scores, desc->n_chunks, desc->top_k,
                                                                          idx);
+    return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+gsa_status gsa_topp(const gsa_decode_desc* desc, float top_p, const float* scores, int32_t* idx, int32_t* count,
+                    void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if (!(top_p > 0.f && top_p <= 1.f) || desc->top_k < 1) return GSA_ERR_ARG;
+    if (desc->top_k > kToppMax) return GSA_ERR_SHAPE;
+    if (!scores || !idx) return GSA_ERR_ARG;
+    if (!aligned16(scores) || !aligned16(idx) || (reinterpret_cast<uintptr_t>(count) & 3u)) return GSA_ERR_ALIGN;
+    const int rows = desc->batch * desc->n_kv_heads;
+    const double scale = desc->scale > 0 ? (double)desc->scale : 1.0 / std::sqrt((double)desc->head_dim);
+    const size_t smem = (size_t)desc->top_k * 16;
+    topp_kernel<<<rows, NTHREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+        scores, desc->n_chunks, desc->top_k, top_p, (float)(scale * 1.4426950408889634), idx, count);
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
@@ -745,6 +862,29 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
     return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
+
+gsa_status gsa_decode_step_topp(const gsa_decode_desc* desc, float top_p, const void* q, const void* k_gist,
+                                const void* v_gist, const void* k_raw, const void* v_raw, const void* k_tail,
+                                const void* v_tail, int32_t* idx_out, int32_t* count_out, float* scores_out,
+                                void* out, void* ws, size_t ws_bytes, void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if (!(top_p > 0.f && top_p <= 1.f) || desc->top_k < 1) return GSA_ERR_ARG;
+    if (desc->top_k > kToppMax) return GSA_ERR_SHAPE;
+    if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
+    if (!aligned16(idx_out) || !aligned16(scores_out) || (reinterpret_cast<uintptr_t>(count_out) & 3u))
+        return GSA_ERR_ALIGN;
+    if ((st = check_ws(decode_ws_bytes(*desc), ws, ws_bytes)) != GSA_OK) return st;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    size_t off_s, off_i;
+    unselected_scratch(*desc, off_s, off_i);
+    float* sc = scores_out ? scores_out : reinterpret_cast<float*>(w + off_s);
+    int32_t* ix = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + off_i);
+    if ((st = gsa_score(desc, q, k_gist, sc, stream)) != GSA_OK) return st;
+    if ((st = gsa_topp(desc, top_p, sc, ix, count_out, stream)) != GSA_OK) return st;
+    return gsa_unfold_attn(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ix, out, nullptr, ws, ws_bytes,
+                           stream);
+}
 
 // Hierarchical decode ([EN-2] "Hierarchical Extension (H-GSA)"; slide page 11):
 // gist pass over the level-2 gists (scores, attention, top-k2), gist pass over

@@ -100,9 +100,7 @@ constexpr uint32_t SM_HSCR = SM_HRES + TILE * 4;
 static_assert(SM_HSCR + 4608 <= SM_ROWTAB, "hierarchy tables overflow the selection buffer");
 static_assert(kSelCap * 4 + kMaxTpc * TILE * 4 <= kScoreCap * 4, "unfold tables overflow the score buffer");
 constexpr uint32_t SM_UB = SM_SCORE + kScoreCap * 4;  // first unit of every CTA [kFusedCtas + 1]
-constexpr uint32_t SM_SEGC = SM_UB + 640;              // key stretch, k <= 32: the kept top-k of each score tile [24][32] u64
-constexpr uint32_t SM_CAND = SM_SEGC + (kScoreCap / TILE) * 32 * 8;   // a score tile, packed [NU] u64; the row's candidates [2 NU] u64
-constexpr uint32_t SM_TMASK = SM_CAND + 2 * NU * 8;   // key stretch: the tile's gists of a given selection (UNSELECTED_GISTS) [4] u32
+constexpr uint32_t SM_TMASK = SM_UB + 640;             // key stretch: the tile's gists of a given selection (UNSELECTED_GISTS) [4] u32
 constexpr uint32_t SM_BAR = SM_TMASK + 16;
 static_assert((kFusedCtas + 1) * 4 <= 640, "unit table overflow");
 constexpr uint32_t SMEM_BYTES = SM_BAR + 512 + 1024;
@@ -115,7 +113,6 @@ struct Bars {
     uint64_t q_ready[2];
     uint64_t gdone;              // a gathered stretch is closed (its row table and children keys are free)
     uint64_t gready;             // the first NSL gathered slots are free (their key / value tiles consumed)
-    uint64_t sc_full[kScoreCap / 128];   // k <= 32: score tile i of this CTA is in shared memory (used once)
     uint32_t tmem;
 };
 
@@ -158,26 +155,6 @@ __device__ __forceinline__ int cta_of(const int* ub, int grid, int u) {
         else hi = mid - 1;
     }
     return lo;
-}
-
-// Gists [g0, g1) of `row` that CTA cc scores (an empty range if none).
-__device__ __forceinline__ void cta_gists(const Params& p, const int* ub, int cc, int row, int& g0, int& g1) {
-    const int ru0 = row * p.upr;
-    const int a = max(ub[cc], ru0), b = min(ub[cc + 1], ru0 + p.tg);
-    g0 = (a - ru0) * TILE;
-    g1 = b > a ? min((b - ru0) * TILE, p.NA) : g0;
-}
-
-// First candidate slot of CTA c for `row`: the CTAs meeting the row before
-// it publish min(k, gists they score) candidates each.
-__device__ __forceinline__ int cand_offset(const Params& p, const int* ub, int c, int row) {
-    int off = 0;
-    for (int cc = cta_of(ub, p.grid, row * p.upr); cc < c; ++cc) {
-        int g0, g1;
-        cta_gists(p, ub, cc, row, g0, g1);
-        off += min(p.K, g1 - g0);
-    }
-    return off;
 }
 
 __device__ __forceinline__ Tile unit_tile(const Params& p, int u) {
@@ -259,21 +236,6 @@ struct Ctx {
     int ai, aseg;  // softmax role: attended units / attended segments so far (TMEM columns)
     uint32_t mcol; // first TMEM column of the segment maxima
 };
-
-// Packed candidate: orderable score key, then the complemented gist index,
-// so that comparing the packed values compares (score, then lower index).
-__device__ __forceinline__ uint64_t pack_cand(uint32_t key, int pos) {
-    return ((uint64_t)key << 32) | (uint64_t)(uint32_t)~(uint32_t)pos;
-}
-__device__ __forceinline__ int cand_pos(uint64_t c) { return (int)~(uint32_t)c; }
-__device__ __forceinline__ void st_relaxed_u64(uint64_t* a, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* a) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
-    return v;
-}
 
 // Is slot sequence number `seq` free to fill (its previous use consumed)?
 __device__ __forceinline__ bool slot_free(const Params& p, Bars* b, int seq) {
@@ -646,8 +608,6 @@ __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u
             if (cx.gtiles < kScoreCap / TILE)
                 reinterpret_cast<float*>(cx.base + SM_SCORE)[cx.gtiles * TILE + t] = score;
         }
-        // k <= 32: the unfold warps fold this tile of scores into their running top-k lists
-        if (p.inc_sel && cx.gtiles < kScoreCap / TILE) mbar_arrive(&cx.bars->sc_full[cx.gtiles]);
         cx.gtiles++;
     }
 }
@@ -961,130 +921,6 @@ __device__ __forceinline__ void merge_select(const Params& p, uint8_t* base, int
     usync();
 }
 
-// k <= 32, during the key stretch (unfold warps, beside the streaming): a
-// running top-k list of the row segment's gists, sorted descending, is kept
-// in shared memory.  As each score tile arrives, the scores that beat the
-// list's k-th entry are collected (warp ballots, then the four warp counts)
-// and ranked together with the list: each element of the union counts the
-// larger ones, and those of rank < k form the new list.  Packed scores
-// compare as (score, then lower index), so ranks are exact and distinct.
-// After the first tile of a segment few scores pass the k-th entry.  At the
-// segment's end the list is the CTA's top-k of the segment and goes to the
-// row's candidate slots.  Score tile st of this CTA is announced by mbarrier
-// sc_full[st].
-__device__ __forceinline__ void fold_scores(const Params& p, uint8_t* base, Bars* bars, int c, int row_first,
-                                            int row_last) {
-    const int* ub = reinterpret_cast<const int*>(base + SM_UB);
-    const float* sc = reinterpret_cast<const float*>(base + SM_SCORE);
-    uint64_t* uni = reinterpret_cast<uint64_t*>(base + SM_CAND);    // [2 NU] the list, then the passing scores
-    uint64_t* nl = reinterpret_cast<uint64_t*>(base + SM_SEGC);     // [32] the new list
-    uint32_t* wc = reinterpret_cast<uint32_t*>(base + SM_SEGC + 32 * 8);   // [4] passing scores per warp
-    const int i = utid(), lane = i & 31, uw = i >> 5;
-    const int K = p.K;
-    int st = 0;
-    for (int r = row_first; r <= row_last; ++r) {
-        int g0, g1;
-        cta_gists(p, ub, c, r, g0, g1);
-        if (g1 <= g0) continue;
-        if (i < K) uni[i] = 0ull;
-        usync();
-        for (int g = g0; g < g1; g += TILE, ++st) {
-            mbar_wait(&bars->sc_full[st], 0, p.err);
-            const uint64_t me = g + i < g1 ? pack_cand(order_key(sc[st * TILE + i]), g + i) : 0ull;
-            const uint64_t kth = uni[K - 1];
-            const bool pass = me > kth;
-            const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
-            if (lane == 0) wc[uw] = __popc(m);
-            usync();
-            int before = 0, total = 0;
-#pragma unroll
-            for (int w = 0; w < NU / 32; ++w) {
-                const int x = (int)wc[w];
-                before += w < uw ? x : 0;
-                total += x;
-            }
-            if (pass) uni[K + before + __popc(m & ((1u << lane) - 1u))] = me;
-            if (i < K) nl[i] = 0ull;   // empty entries (all 0) share one rank: the places after the real ones stay 0
-            usync();
-            if (total > 0) {
-                const int n = K + total;   // up to K + NU entries
-                for (int q = i; q < n; q += NU) {
-                    const uint64_t e = uni[q];
-                    int rank = 0;
-                    for (int j = 0; j < n; ++j) rank += uni[j] > e ? 1 : 0;
-                    if (rank < K) nl[rank] = e;
-                }
-                usync();
-                if (i < K) uni[i] = nl[i];
-                usync();
-            }
-        }
-        // the list holds min(k, gists of this CTA in the row) entries
-        if (i < K && uni[i] != 0ull) st_relaxed_u64(p.cand64 + (size_t)r * p.NA + cand_offset(p, ub, c, r) + i, uni[i]);
-        usync();
-    }
-}
-
-// k <= 32: the row's exact top-k from the n <= 2 NU candidates the CTAs
-// meeting the row published in the key stretch (each CTA's top-k of the
-// gists it scored, so their union holds the row's top-k).  A slot reads 0
-// until its value lands; the wait on it is bounded.  Ranks come from
-// counting the larger packed candidates (ties of score go to the lower
-// index), then the k positions are put in ascending order.
-__device__ __forceinline__ void inc_select(const Params& p, uint8_t* base, int row, int n, bool publish) {
-    const uint64_t* slots = p.cand64 + (size_t)row * p.NA;
-    uint64_t* cs = reinterpret_cast<uint64_t*>(base + SM_CAND);
-    int32_t* byrank = reinterpret_cast<int32_t*>(base + SM_MISC);
-    const uint64_t limit = 2ull * g_cross_wait_ns;
-    for (int i = utid(); i < p.K; i += NU) byrank[i] = i;   // stays in range if a slot never lands
-    if (utid() < 32) {
-        // one warp polls, all of its loads in flight at once (a pause between
-        // rounds), so that the waiting CTAs do not flood L2 with loads
-        const int lane = utid();
-        const uint64_t t0 = sm_cycles();
-        uint64_t v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = q * 32 + lane < n ? ld_relaxed_u64(slots + q * 32 + lane) : 1ull;
-        bool late = false;
-        for (;;) {
-            bool have = true;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) have = have && v[q] != 0ull;
-            if (__all_sync(0xFFFFFFFFu, have) || late) break;
-            __nanosleep(200);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (v[q] == 0ull) v[q] = ld_relaxed_u64(slots + q * 32 + lane);
-            late = sm_cycles() - t0 > limit;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (q * 32 + lane < n) cs[q * 32 + lane] = v[q];
-        if (late && lane == 0) atomicOr(p.err, kErrTimeout);
-    }
-    usync();
-    for (int i = utid(); i < n; i += NU) {
-        const uint64_t me = cs[i];
-        if (me == 0ull) continue;
-        int rank = 0;
-        for (int j = 0; j < n; ++j) rank += cs[j] > me ? 1 : 0;
-        if (rank < p.K) byrank[rank] = cand_pos(me);
-    }
-    usync();
-    int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
-    if (utid() < p.K) {
-        // place in ascending order (equal entries, possible only after a
-        // timed-out slot, still take distinct places)
-        const int me = utid();
-        const int32_t v = byrank[me];
-        int r = 0;
-        for (int j = 0; j < p.K; ++j) r += (byrank[j] < v || (byrank[j] == v && j < me)) ? 1 : 0;
-        sel[r] = v;
-        if (publish) p.idx[(size_t)row * p.K + r] = v;
-    }
-    usync();
-}
-
 __device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, int row, bool publish) {
     int32_t* out = p.idx + (size_t)row * p.K;
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
@@ -1094,13 +930,14 @@ __device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, in
         for (int r = utid(); r < min(p.K, p.NA); r += NU) out[r] = sel[r];
 }
 
-// A given selection (gsa_unfold_attn) into sel[0..k); an index outside
+// A given selection (gsa_unfold_attn) into sel[0..k); -1 is an empty place
+// (a variable-size selection such as top-p's), any other index outside
 // [0, N) is clamped into range and flagged in the error word.
 __device__ __forceinline__ void load_selection(const Params& p, uint8_t* base, int row) {
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
     for (int r = utid(); r < p.K; r += NU) {
         int32_t j = __ldcg(p.idx + (size_t)row * p.K + r);
-        if (j < 0 || j >= p.N) {
+        if (j != -1 && (j < 0 || j >= p.N)) {
             atomicOr(p.err, kErrIndex);
             j = j < 0 ? 0 : p.N - 1;
         }
@@ -1120,9 +957,9 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
         int32_t e = -1;
         if (gr < kc) {
             const int sidx = gr / p.C, tok = gr - sidx * p.C;
-            e = (int32_t)(((long long)row * p.N + sel[sidx]) * p.C + tok);
+            if (sel[sidx] >= 0) e = (int32_t)(((long long)row * p.N + sel[sidx]) * p.C + tok);
         } else if (gr < p.nrows_g) {
-            e = (int32_t)(-((long long)row * p.N + sel[gr - kc]) - 2);
+            if (sel[gr - kc] >= 0) e = (int32_t)(-((long long)row * p.N + sel[gr - kc]) - 2);
         }
         tab[i] = e;
     }
@@ -1158,7 +995,10 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
     // bytes first; the phase cannot complete before the final arrival below
     const int uw = utid() >> 5;
     if (tma_rows > 0 && (utid() & 31) == 0 && uw * h < tma_rows) {
-        const int runs = (tma_rows / h - uw + (NU / 32) - 1) / (NU / 32);
+        // runs of empty places (-1 in the table) are not loaded: their V rows
+        // are zeroed below with the other rows that are not whole runs
+        int runs = 0;
+        for (int r = uw * h; r < tma_rows; r += (NU / 32) * h) runs += tab[r] != -1 ? 1 : 0;
         const uint32_t bytes = (uint32_t)(runs * h) * (D * 2);
         mbar_expect_tx(&bars->full[sk], bytes);
         mbar_expect_tx(&bars->full[sv], bytes);
@@ -1167,6 +1007,7 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
         const long long n_src = p.hier ? (long long)p.N1 : (long long)p.N;   // chunks (level-1 gists) per row
         for (int r = uw * h; r < tma_rows; r += (NU / 32) * h) {
             const long long e = tab[r];
+            if (e == -1) continue;
             // source row of the run: token (chunk * c) of the row's raw rows, or the first child
             const int y = children ? (int)(-e - 2 - (long long)row * n_src) : (int)(e - (long long)row * n_src * p.C);
             tc::tma_load_3d(ks + r * 128, mk, 0, y, row, &bars->full[sk]);
@@ -1180,6 +1021,9 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
         const int r = tma_rows + (q >> 4);
         gather_piece(p, ks, vs, tab[r], r, q & 15);
     }
+    // runs skipped above (an empty place of a variable-size selection): V rows zeroed
+    for (int q = utid(); q < tma_rows * 16; q += NU)
+        if (tab[((q >> 4) / h) * h] == -1) gather_piece(p, ks, vs, -1, q >> 4, q & 15);
     cp_async_arrive_hold(&bars->full[sk]);
     cp_async_arrive_hold(&bars->full[sv]);
     usync();
@@ -1267,7 +1111,7 @@ __device__ __forceinline__ void wait_count(const Params& p, const uint32_t* ctr,
 // no dependent rescaling chain), folded into a running (M, L, acc) once per
 // group.  Leaves the row's ticket and key counter zero for the next call.
 template <int G>
-__device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int row, int na, int nb, int ncand) {
+__device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int row, int na, int nb) {
     constexpr int NW = NTHR / 32;
     const int nsl = na + nb;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1361,8 +1205,6 @@ __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int ro
         p.cnt[row] = 0;
         p.kdone[row] = 0;
     }
-    // every reader of the row's candidate slots is done (its partial is counted)
-    for (int i = threadIdx.x; i < ncand; i += NTHR) p.cand64[(size_t)row * p.NA + i] = 0ull;
 }
 
 // ---------------------------------------------------------------- kernel --
@@ -1407,7 +1249,6 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         }
         mbar_init(&b->gdone, 128);
         mbar_init(&b->gready, 1);
-        for (int i = 0; i < kScoreCap / TILE; ++i) mbar_init(&b->sc_full[i], 128);
         fence_mbar_init();
     }
     if (threadIdx.x == 32 * 4) {
@@ -1536,9 +1377,8 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
     } else {
         // ----------------------------------------------- unfold warps --
         const bool lead = utid() == 0;
-        if (p.inc_sel) fold_scores(p, cx.base, cx.bars, c, row_first, row_last);
         asm volatile("bar.sync %0, %1;" ::"n"(BAR_KEYS), "n"(NTHR) : "memory");
-        if (p.do_topk && !p.sel_direct && !p.inc_sel) {
+        if (p.do_topk && !p.sel_direct) {
             // local top-k of every segment, from the scores this CTA kept
             int ntiles = 0;
             for (int r = row_first; r <= row_last; ++r) {
@@ -1569,7 +1409,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         // lead's fence is cumulative: it orders before the counters the
         // streaming warps' scores and the unfold warps' candidates, which the
         // barriers above made visible to it.
-        if (lead && !p.inc_sel) {
+        if (lead) {
             __threadfence();
             for (int r = row_first; r <= row_last; ++r) atomicAdd(p.kdone + r, 1u);
         }
@@ -1578,7 +1418,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
             const int row = it / p.cb, j = it % p.cb;
             int cf;
             const int na = row_ctas(row, cf);
-            if (p.do_topk && !p.inc_sel) wait_count<NU, BAR_UNF>(p, p.kdone + row, (uint32_t)na, lead);
+            if (p.do_topk) wait_count<NU, BAR_UNF>(p, p.kdone + row, (uint32_t)na, lead);
             for (int rd = 0; rd < rounds; ++rd) {
                 int t0;
                 const int ntl = item_tiles(it, rd, t0);
@@ -1592,15 +1432,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                 if (rd == 1) {
                     hier_select_children(p, cx.base, row);
                 } else {
-                    if (p.do_topk && p.inc_sel) {
-                        int n = 0;
-                        for (int cc = cf; cc < cf + na; ++cc) {
-                            int a0, a1;
-                            gists_of(cc, row, a0, a1);
-                            n += min(p.K, max(0, a1 - a0));
-                        }
-                        inc_select(p, cx.base, row, n, j == 0);
-                    } else if (p.do_topk && p.sel_direct) {
+                    if (p.do_topk && p.sel_direct) {
                         direct_select(p, cx.base, row, j == 0);
                     } else if (p.do_topk) {
                         int n = 0;
@@ -1660,14 +1492,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         int cf;
         const int na = row_ctas(row, cf);
         wait_count<NTHR, 0>(p, p.cnt + row, (uint32_t)(na + p.cb), threadIdx.x == 0);
-        int ncand = 0;
-        if (p.inc_sel)
-            for (int cc = cf; cc < cf + na; ++cc) {
-                int a0, a1;
-                gists_of(cc, row, a0, a1);
-                ncand += min(p.K, max(0, a1 - a0));
-            }
-        merge_row<G>(p, cx.base, row, na, nb, ncand);
+        merge_row<G>(p, cx.base, row, na, nb);
         __syncthreads();
     }
     tc::fence_before();
@@ -1862,8 +1687,6 @@ static void layout_ws(FusedPlan& f, size_t N, size_t top_k, size_t k1) {
     o = round256(o + rows * (size_t)f.slot_stride * f.G * 4 * 4);
     f.off_idx1 = o;
     o = round256(o + rows * k1 * 4);
-    f.off_cand64 = o;
-    if (f.inc_sel) o = round256(o + rows * N * 8);
     f.total = o;
 }
 
@@ -1909,7 +1732,6 @@ static FusedPlan build_fused_plan(const gsa_decode_desc& d, bool given) {
     // small selections are taken straight from the scores; larger ones from
     // per-CTA candidates the key stretch leaves
     f.sel_direct = (d.top_k <= 32 && d.n_chunks <= 32 * fused::NU) ? 1 : 0;
-    f.inc_sel = 0;
     // unfold: the row's gathered rows packed into 128-row tiles, spread over
     // as many CTAs per row as fill the GPU (at most kMaxTpc tiles each)
     f.nrows_g = d.top_k * d.chunk + (pairs ? d.top_k : 0);
@@ -1923,13 +1745,6 @@ static FusedPlan build_fused_plan(const gsa_decode_desc& d, bool given) {
         f.cb = (f.nbt + f.tpc - 1) / f.tpc;
     }
     place_ctas(f, f.cb);
-    // k <= 32 and at most 2 NU candidates per row: the key stretch keeps
-    // running top-k lists and publishes each CTA's candidates
-    if (!given && d.top_k >= 1 && d.top_k <= 32 && f.maxs * d.top_k <= 2 * fused::NU &&
-        (f.T + f.grid - 1) / f.grid <= fused::kScoreCap / 128) {
-        f.inc_sel = 1;
-        f.sel_direct = 0;
-    }
     layout_ws(f, (size_t)d.n_chunks, (size_t)d.top_k, 0);
     return f;
 }
@@ -1958,8 +1773,6 @@ static void fill_common(fused::Params& p, const FusedPlan& f, const gsa_decode_d
     p.tpc = f.tpc;
     p.cb = f.cb;
     p.sel_direct = f.sel_direct;
-    p.inc_sel = f.inc_sel;
-    p.cand64 = reinterpret_cast<uint64_t*>(w + f.off_cand64);
     p.tmem_cols = f.tmem_cols;
     const double scale = d.scale > 0 ? (double)d.scale : 1.0 / std::sqrt(128.0);
     p.c2 = (float)(scale * 1.4426950408889634);
@@ -2029,10 +1842,6 @@ FusedPlan make_fused_hier_plan(const gsa_hier_desc& h) {
     f.tpc = 2;
     f.cb = 1;
     place_ctas(f, 2);
-    f.inc_sel = (h.top_k2 >= 1 && h.top_k2 <= 32 && f.maxs * h.top_k2 <= 2 * fused::NU &&
-                 (f.T + f.grid - 1) / f.grid <= fused::kScoreCap / 128) ? 1 : 0;
-    if (f.inc_sel) f.sel_direct = 0;
-    else f.sel_direct = (h.top_k2 <= 32 && h.n_l2 <= 32 * fused::NU) ? 1 : 0;
     layout_ws(f, (size_t)h.n_l2, (size_t)h.top_k2, (size_t)h.l1.top_k);
     return f;
 }

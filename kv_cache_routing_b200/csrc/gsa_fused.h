@@ -20,12 +20,10 @@ struct FusedPlan {
     int items;                        // unfold items in all (rows * cb)
     int slot_stride;                  // maxs + unfold partial slots
     int sel_direct;                   // the selection is taken from the scores (else from per-CTA candidates)
-    int inc_sel;                      // k <= 32: running top-k lists in the key stretch, published candidate slots
     int attn_gists;                   // gist tiles are attended (ALL_GISTS)
     int tmem_cols;                    // TMEM columns a CTA allocates (S, O^T, kept logits and maxima)
     size_t off_scores, off_cand_key, off_cand_idx, off_idx, off_part, off_ml, total;
     size_t off_idx1;                  // hierarchy: level-1 selection (when the caller passes none)
-    size_t off_cand64;                // inc_sel: candidate slots [rows][N] u64 (0 = not yet published)
 };
 
 namespace fused {
@@ -59,9 +57,7 @@ struct Params {
     int tmem_cols;                 // TMEM columns a CTA allocates
     float c2;
     int do_score, do_topk, do_attn_gists, sel_direct;
-    int inc_sel;                   // k <= 32: candidates from the key stretch's running lists
     int mask_sel;                  // given selection, UNSELECTED_GISTS: its gists are masked in the key stretch
-    uint64_t* cand64;              // [rows][N] published candidates (key << 32 | ~gist), 0 = empty
     // hierarchy (keys/values: level-2 gists; unfold: children tile, then raw tile)
     int hier, group, N1, K1;       // K = k2, N = NA = n_l2; group, level-1 gists, k1
     int32_t* idx1;                 // [rows][k1]

@@ -118,6 +118,20 @@ def test_launch_counts_follow_the_path():
     assert gsa.gsa_decode_launch_count(_desc(mode=gsa.GSA_UNSELECTED_GISTS)) == 3
     assert gsa.gsa_decode_launch_count(_desc(mode=gsa.GSA_UNSELECTED_GISTS, dtype=gsa.GSA_F32)) == 4
     assert gsa.gsa_decode_launch_count(_desc(mode=gsa.GSA_UNSELECTED_GISTS, top_k=0)) == 1
+
+
+def test_topp_arguments_are_checked_before_launch():
+    d = _desc(top_k=8)
+    for p, code in [(0.0, gsa.GSA_ERR_ARG), (1.5, gsa.GSA_ERR_ARG), (float("nan"), gsa.GSA_ERR_ARG)]:
+        with pytest.raises(gsa.GsaError) as e:
+            gsa.gsa_topp(d, p, 1 << 20, 1 << 21, None, stream=0)
+        assert e.value.status == code
+    with pytest.raises(gsa.GsaError) as e:
+        gsa.gsa_topp(_desc(n_chunks=4000, top_k=3000), 0.5, 1 << 20, 1 << 21, None, stream=0)
+    assert e.value.status == gsa.GSA_ERR_SHAPE
+    with pytest.raises(gsa.GsaError) as e:
+        gsa.gsa_topp(d, 0.5, (1 << 20) + 4, 1 << 21, None, stream=0)
+    assert e.value.status == gsa.GSA_ERR_ALIGN
     with pytest.raises(gsa.GsaError):
         gsa.gsa_decode_launch_count(_desc(head_dim=96))
     l1 = _desc(n_chunks=160, top_k=8)

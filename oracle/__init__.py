@@ -48,6 +48,7 @@ def _load():
         "oracle_score_error_bound": [i, i, i, i, i, i, vp, vp, vp],
         "oracle_decode": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
         "oracle_unfold_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
+        "oracle_decode_paged": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12,
         "oracle_hier_decode": [i, i, i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12 + [i],
         "oracle_gist_mask": [i64, i64, i],
         "oracle_prefill_pair_count": [i, i],
@@ -146,6 +147,28 @@ def decode(t: dict, top_k: int, mode: int = ALL_GISTS, scale: float = 0.0):
     _load().oracle_decode(B, Hq, Hkv, d, N, c, top_k, W, mode, scale, _dtcode(q), _p(q), _p(kg),
                           _p(t["v_gist"]), _p(t["k_raw"]), _p(t["v_raw"]), _p(t["k_tail"]),
                           _p(t["v_tail"]), _p(s), _p(idx), _p(out))
+    return s, idx, out
+
+
+def decode_paged(t: dict, k_pages: np.ndarray, v_pages: np.ndarray, table: np.ndarray, top_k: int,
+                 mode: int = ALL_GISTS, scale: float = 0.0, seq_chunks=None):
+    """Flat decode step over a paged raw cache.  t holds q, k_gist, v_gist
+    [B,Hkv,N,d], k_tail, v_tail; chunk j of sequence b is page table[b, j] of
+    the pools k_pages / v_pages [pages, Hkv, c, d]; seq_chunks [B] (or None)
+    gives the chunks of each sequence.  Returns (scores, idx, out)."""
+    q, kg = t["q"], t["k_gist"]
+    B, Hq, d = q.shape
+    _, Hkv, N, _ = kg.shape
+    c = k_pages.shape[2]
+    W = t["k_tail"].shape[2]
+    table = np.ascontiguousarray(table, np.int32)
+    nch = None if seq_chunks is None else np.ascontiguousarray(seq_chunks, np.int32)
+    s = np.empty((B, Hkv, N), np.float64)
+    idx = np.empty((B, Hkv, top_k), np.int32)
+    out = np.empty((B, Hq, d), np.float64)
+    _load().oracle_decode_paged(B, Hq, Hkv, d, N, c, top_k, W, mode, scale, _dtcode(q), _p(q), _p(kg),
+                                _p(t["v_gist"]), _p(k_pages), _p(v_pages), _p(table), _p(nch),
+                                _p(t["k_tail"]), _p(t["v_tail"]), _p(s), _p(idx), _p(out))
     return s, idx, out
 
 

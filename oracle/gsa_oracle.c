@@ -12,6 +12,8 @@
  *            Attention" — interleaved gist tokens, gist as routing signals,
  *            selective unfolding, hybrid attention, hierarchical extension;
  *   [DE-M]   gist.science explainer (DE), section "Methodik";
+ *   [EN-4]   gist.science explainer (EN), section 4 "Experimental Results"
+ *            (KV-cache reuse: precomputed document caches);
  *   [SL-6]   Taki-lab slide deck (docswell), page 6 "GSA とは" — query scores
  *            every gist, takes top-k, restores the chunks with their gists;
  *   [SL-7]   slide deck, page 7 "Gist token" — gist causal mask example;
@@ -244,18 +246,35 @@ static void attend(int d, int dt, double scale, const void* q, int64_t q_off, in
  * tokens instead of its gist) -> UNSELECTED_GISTS.
  * In both modes the W uncompressed tail tokens after the last chunk are
  * always attended ([SL-9]: the generation suffix attends directly).          */
-static int flat_context(int Hkv, int d, int N, int c, int W, int mode, int b, int hk, int k,
+/* Raw token u of chunk j of row `row`: in the dense cache [rows][N][c][d], or,  */
+/* when a block table is given, in page table[row][j] of a page pool            */
+/* [pages][c][d] ([EN-4] "KV-Cache Reuse": precomputed document caches routed   */
+/* through their gists; a page may belong to several rows).                     */
+/* Element offset of raw token u of chunk j of (b, hk).  Dense: raw [B][Hkv][N][c][d].
+ * Paged ([EN-4] "KV-Cache Reuse": precomputed document caches are shared, not
+ * copied): chunk j of sequence b is page table[b*N + j] of a pool
+ * [pages][Hkv][c][d]; one page holds one chunk of every KV head, so the
+ * sequences whose contexts hold the same document point at the same pages. */
+static int64_t raw_off(int Hkv, int N, int c, int d, const int32_t* table, int b, int hk, int j, int u) {
+    if (table) return (((int64_t)table[(int64_t)b * N + j] * Hkv + hk) * c + u) * d;
+    return ((((int64_t)b * Hkv + hk) * N + j) * c + u) * d;
+}
+
+/* The context of (b, hk): gists as the mode says (of the sequence's nb <= N
+ * chunks), raw tokens of the selected chunks, tail.                         */
+static int flat_context(int Hkv, int d, int N, int nb, int c, int W, int mode, int b, int hk, int k,
                         const int32_t* sel, const void* kg, const void* vg, const void* kraw,
-                        const void* vraw, const void* ktail, const void* vtail, key_ref* keys) {
+                        const void* vraw, const void* ktail, const void* vtail, const int32_t* table,
+                        key_ref* keys) {
     int n = 0;
     int64_t row = (int64_t)b * Hkv + hk;
     if (mode == OR_ALL_GISTS) {
-        for (int j = 0; j < N; ++j) keys[n++] = (key_ref){kg, vg, (row * N + j) * d};
+        for (int j = 0; j < nb; ++j) keys[n++] = (key_ref){kg, vg, (row * N + j) * d};
     } else if (mode == OR_SELECTED_PAIRS) {
         for (int t = 0; t < k; ++t)
             if (sel[t] >= 0) keys[n++] = (key_ref){kg, vg, (row * N + sel[t]) * d};
     } else if (mode == OR_UNSELECTED_GISTS) {
-        for (int j = 0; j < N; ++j) {
+        for (int j = 0; j < nb; ++j) {
             int selected = 0;
             for (int t = 0; t < k; ++t) selected |= sel[t] == j;
             if (!selected) keys[n++] = (key_ref){kg, vg, (row * N + j) * d};
@@ -264,33 +283,40 @@ static int flat_context(int Hkv, int d, int N, int c, int W, int mode, int b, in
     for (int t = 0; t < k; ++t)
         if (sel[t] >= 0)   /* -1: an empty place of a variable-size (top-p) selection */
             for (int u = 0; u < c; ++u)
-                keys[n++] = (key_ref){kraw, vraw, ((row * N + sel[t]) * c + u) * d};
+                keys[n++] = (key_ref){kraw, vraw, raw_off(Hkv, N, c, d, table, b, hk, sel[t], u)};
     for (int u = 0; u < W; ++u) keys[n++] = (key_ref){ktail, vtail, (row * W + u) * d};
     return n;
 }
 
 /* Full flat decode step: scores (step 1), selection (step 2), hybrid
  * attention (steps 3-4).  Outputs: scores [B*Hkv*N] (may be NULL), selected
- * indices [B*Hkv*k] ascending, out [B*Hq*d].                                */
-void oracle_decode(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode, double scale,
-                   int dt, const void* q, const void* kg, const void* vg, const void* kraw,
-                   const void* vraw, const void* ktail, const void* vtail, double* scores_out,
-                   int32_t* idx_out, double* out) {
+ * indices [B*Hkv*k] ascending, out [B*Hq*d].
+ * nch (may be NULL: every sequence has N chunks) gives sequence b nb =
+ * nch[b] <= N chunks: its gists j >= nb do not exist, so they score -inf,
+ * are never selected and are not in the context; with nb < k the selection
+ * holds all nb chunks and its other places are empty (-1).                 */
+static void decode_impl(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode, double scale,
+                        int dt, const void* q, const void* kg, const void* vg, const void* kraw,
+                        const void* vraw, const int32_t* table, const int32_t* nch, const void* ktail,
+                        const void* vtail, double* scores_out, int32_t* idx_out, double* out) {
     int G = Hq / Hkv;
     double sc = default_scale(scale, d);
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < B; ++b)
         for (int hk = 0; hk < Hkv; ++hk) {
             int64_t row = (int64_t)b * Hkv + hk;
+            int nb = nch ? nch[b] : N;
             double* s = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
-            for (int j = 0; j < N; ++j) s[j] = gist_score(Hq, Hkv, d, N, dt, q, kg, b, hk, j);
+            for (int j = 0; j < nb; ++j) s[j] = gist_score(Hq, Hkv, d, N, dt, q, kg, b, hk, j);
             if (scores_out)
-                for (int j = 0; j < N; ++j) scores_out[row * N + j] = s[j];
+                for (int j = 0; j < N; ++j) scores_out[row * N + j] = j < nb ? s[j] : -INFINITY;
             int32_t* sel = idx_out + row * k;
-            topk_list(N, s, NULL, k, sel);
+            int kk = k < nb ? k : nb;
+            topk_list(nb, s, NULL, kk, sel);
+            for (int t = kk; t < k; ++t) sel[t] = -1;
             key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(N + (int64_t)k * c + W + 1));
-            int nk = flat_context(Hkv, d, N, c, W, mode, b, hk, k, sel, kg, vg, kraw, vraw, ktail,
-                                  vtail, keys);
+            int nk = flat_context(Hkv, d, N, nb, c, W, mode, b, hk, k, sel, kg, vg, kraw, vraw, ktail,
+                                  vtail, table, keys);
             for (int g = 0; g < G; ++g) {
                 int h = hk * G + g;
                 attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
@@ -304,10 +330,10 @@ void oracle_decode(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, in
 /* Hybrid attention alone, for a given selection idx [B*Hkv*k] (the unfolding
  * + attention step without routing).  lse (may be NULL) [B*Hq] receives the
  * natural log of sum_x exp(scale * q_h . K_x) over the context.              */
-void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode,
+static void unfold_impl(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode,
                         double scale, int dt, const void* q, const void* kg, const void* vg,
-                        const void* kraw, const void* vraw, const void* ktail, const void* vtail,
-                        const int32_t* idx, double* out, double* lse) {
+                        const void* kraw, const void* vraw, const int32_t* table, const void* ktail,
+                        const void* vtail, const int32_t* idx, double* out, double* lse) {
     int G = Hq / Hkv;
     double sc = default_scale(scale, d);
 #pragma omp parallel for collapse(2) schedule(dynamic)
@@ -315,8 +341,8 @@ void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int 
         for (int hk = 0; hk < Hkv; ++hk) {
             int64_t row = (int64_t)b * Hkv + hk;
             key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(N + (int64_t)k * c + W + 1));
-            int nk = flat_context(Hkv, d, N, c, W, mode, b, hk, k, idx + row * k, kg, vg, kraw, vraw,
-                                  ktail, vtail, keys);
+            int nk = flat_context(Hkv, d, N, N, c, W, mode, b, hk, k, idx + row * k, kg, vg, kraw, vraw,
+                                  ktail, vtail, table, keys);
             for (int g = 0; g < G; ++g) {
                 int h = hk * G + g;
                 attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys,
@@ -324,6 +350,32 @@ void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int 
             }
             free(keys);
         }
+}
+
+void oracle_decode(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode, double scale,
+                   int dt, const void* q, const void* kg, const void* vg, const void* kraw,
+                   const void* vraw, const void* ktail, const void* vtail, double* scores_out,
+                   int32_t* idx_out, double* out) {
+    decode_impl(B, Hq, Hkv, d, N, c, k, W, mode, scale, dt, q, kg, vg, kraw, vraw, NULL, NULL, ktail, vtail,
+                scores_out, idx_out, out);
+}
+
+void oracle_unfold_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode,
+                        double scale, int dt, const void* q, const void* kg, const void* vg,
+                        const void* kraw, const void* vraw, const void* ktail, const void* vtail,
+                        const int32_t* idx, double* out, double* lse) {
+    unfold_impl(B, Hq, Hkv, d, N, c, k, W, mode, scale, dt, q, kg, vg, kraw, vraw, NULL, ktail, vtail,
+                idx, out, lse);
+}
+
+/* Decode over a paged raw cache (pools k_pages / v_pages [pages][Hkv][c][d],
+ * table [B][N]) with nch[b] chunks in sequence b (nch may be NULL).        */
+void oracle_decode_paged(int B, int Hq, int Hkv, int d, int N, int c, int k, int W, int mode, double scale,
+                         int dt, const void* q, const void* kg, const void* vg, const void* kpages,
+                         const void* vpages, const int32_t* table, const int32_t* nch, const void* ktail,
+                         const void* vtail, double* scores_out, int32_t* idx_out, double* out) {
+    decode_impl(B, Hq, Hkv, d, N, c, k, W, mode, scale, dt, q, kg, vg, kpages, vpages, table, nch, ktail,
+                vtail, scores_out, idx_out, out);
 }
 
 /* ------------------------------------------------------------------------ */

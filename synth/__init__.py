@@ -112,6 +112,7 @@ ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS = 0, 1, 2, 3
 S_Q, S_KG, S_VG, S_KR, S_VR, S_KT, S_VT, S_NEEDLE_IDX, S_NEEDLE_NOISE = range(1, 10)
 S_KG2, S_VG2, S_NEEDLE2_NOISE = 10, 11, 12
 S_PQ, S_PK, S_PV = 20, 21, 22
+S_PAGE_K, S_PAGE_V, S_PAGE_ORDER, S_DOC, S_SEQ_LEN = 30, 31, 32, 33, 34
 
 
 @dataclass(frozen=True)
@@ -161,6 +162,21 @@ class PrefillShape:
     @property
     def positions(self) -> int:
         return self.n_chunks * (self.chunk + 1)
+
+
+@dataclass(frozen=True)
+class PagedShape:
+    """A batch of sequences whose raw chunks live in a shared page pool.
+
+    The pool holds n_docs documents of doc_min..doc_max chunks each (one page
+    per chunk, all KV heads in the page) in a scrambled page order; each
+    sequence is a run of documents drawn from the pool (so sequences share
+    pages) cut to its chunk count, between 3/4 N and N unless given."""
+    base: DecodeShape      # n_chunks = N, the most chunks a sequence has
+    n_docs: int
+    doc_min: int
+    doc_max: int
+    spare_pages: int = 0   # pool pages that no document uses
 
 
 # The five workloads (shapes, dtypes, needles).
@@ -317,3 +333,79 @@ def prefill_inputs(p: PrefillShape, seed: int) -> PrefillInputs:
     k = normal(seed, S_PK, (p.batch, p.n_kv_heads, P, p.head_dim), p.dtype)
     v = normal(seed, S_PV, (p.batch, p.n_kv_heads, P, p.head_dim), p.dtype)
     return PrefillInputs(p, q, k, v)
+
+
+@dataclass
+class PagedInputs:
+    shape: PagedShape
+    q: np.ndarray
+    k_gist: np.ndarray       # [B, Hkv, N, d]; entries past a sequence's chunk count are decoys
+    v_gist: np.ndarray
+    k_pages: np.ndarray      # [pages, Hkv, c, d]
+    v_pages: np.ndarray
+    table: np.ndarray        # [B, N] int32 page of chunk j of sequence b; -1 past its chunk count
+    seq_chunks: np.ndarray   # [B] int32
+    k_tail: np.ndarray
+    v_tail: np.ndarray
+
+    def tensors(self):
+        return dict(q=self.q, k_gist=self.k_gist, v_gist=self.v_gist, k_tail=self.k_tail, v_tail=self.v_tail)
+
+    def dense_raw(self):
+        """The raw cache gathered per sequence, [B, Hkv, N, c, d] (zeros past
+        each sequence's chunk count)."""
+        B, N = self.table.shape
+        P, Hkv, c, d = self.k_pages.shape
+        kr = np.zeros((B, Hkv, N, c, d), self.k_pages.dtype)
+        vr = np.zeros_like(kr)
+        for b in range(B):
+            n = int(self.seq_chunks[b])
+            kr[b, :, :n] = self.k_pages[self.table[b, :n]].transpose(1, 0, 2, 3)
+            vr[b, :, :n] = self.v_pages[self.table[b, :n]].transpose(1, 0, 2, 3)
+        return kr, vr
+
+
+def paged_inputs(ps: PagedShape, seed: int, seq_chunks=None) -> PagedInputs:
+    s = ps.base
+    B, Hq, Hkv, d, N, c, W, dt = (s.batch, s.n_q_heads, s.n_kv_heads, s.head_dim, s.n_chunks, s.chunk,
+                                  s.tail_len, s.dtype)
+    span = ps.doc_max - ps.doc_min + 1
+    doc_len = [ps.doc_min + u64(seed, S_DOC, i) % span for i in range(ps.n_docs)]
+    P = sum(doc_len) + ps.spare_pages
+    order = np.argsort(np.array([u64(seed, S_PAGE_ORDER, i) for i in range(P)], np.uint64), kind="stable")
+    starts = np.concatenate([[0], np.cumsum(doc_len)])
+    if seq_chunks is None:
+        seq_chunks = [N - u64(seed, S_SEQ_LEN, b) % (N // 4 + 1) for b in range(B)]
+    seq_chunks = np.asarray(seq_chunks, np.int32)
+    assert seq_chunks.shape == (B,) and np.all((seq_chunks >= 0) & (seq_chunks <= N))
+    table = np.full((B, N), -1, np.int32)
+    for b in range(B):
+        pages, t = [], 0
+        while len(pages) < seq_chunks[b]:
+            doc = u64(seed, S_DOC, 1_000_003 * (b + 1) + t) % ps.n_docs
+            t += 1
+            pages.extend(order[starts[doc]:starts[doc] + doc_len[doc]].tolist())
+        table[b, :seq_chunks[b]] = pages[:seq_chunks[b]]
+    q = normal(seed, S_Q, (B, Hq, d), dt)
+    kg = normal(seed, S_KG, (B, Hkv, N, d), dt)
+    vg = normal(seed, S_VG, (B, Hkv, N, d), dt)
+    kp = normal(seed, S_PAGE_K, (P, Hkv, c, d), dt)
+    vp = normal(seed, S_PAGE_V, (P, Hkv, c, d), dt)
+    kt = normal(seed, S_KT, (B, Hkv, W, d), dt)
+    vt = normal(seed, S_VT, (B, Hkv, W, d), dt)
+    qw = widen(q, dt)
+    G = s.group
+    for b in range(B):
+        n = int(seq_chunks[b])
+        for hk in range(Hkv):
+            row = b * Hkv + hk
+            # needles among the sequence's chunks; every gist past its end is a
+            # decoy that would win the routing if it were scored
+            m = min(s.n_needles, n)
+            ids = _distinct_draws(seed, S_NEEDLE_IDX, row * 1_000_003, m, n) if m else []
+            noise = normal(seed, S_NEEDLE_NOISE, (max(m, 1) + N - n, d), "f64", offset=row * (N + 1) * d)
+            for t, j in enumerate(ids):
+                kg[b, hk, j] = round_to(_needle_keys(qw, b, hk, G, s.needle_alpha, noise[t]), dt)
+            for t, j in enumerate(range(n, N)):
+                kg[b, hk, j] = round_to(_needle_keys(qw, b, hk, G, 2 * s.needle_alpha, noise[max(m, 1) + t]), dt)
+    return PagedInputs(ps, q, kg, vg, kp, vp, table, seq_chunks, kt, vt)

@@ -537,3 +537,71 @@ def test_padded_selection_equals_the_compacted_one():
                 sub = dataclasses.replace(sh, top_k=len(kept))
                 want = oracle.unfold_attn(one, kept.reshape(1, 1, -1), mode, 0.4)
                 np.testing.assert_array_equal(out[b, hk * sh.group:(hk + 1) * sh.group], want[0])
+
+
+# ------------------------------------------------------------ paged cache ----
+def _paged_small(seq_chunks=None, mode=ALL_GISTS, k=3, dt="f32", seed=71):
+    base = small_shape(n_chunks=10, top_k=k, mode=mode, dtype=dt, n_needles=2)
+    ps = synth.PagedShape(base, n_docs=4, doc_min=2, doc_max=5, spare_pages=2)
+    return ps, synth.paged_inputs(ps, seed, seq_chunks)
+
+
+@pytest.mark.parametrize("mode", [ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS])
+def test_paged_full_sequences_equal_the_gathered_dense_cache(mode):
+    """Every sequence N chunks long: decoding over the page pool equals
+    decoding over the raw cache gathered through the table by numpy
+    indexing (bit for bit: the same keys in the same order)."""
+    ps, x = _paged_small([10, 10], mode)
+    kr, vr = x.dense_raw()
+    t = dict(x.tensors(), k_raw=kr, v_raw=vr)
+    s0, i0, o0 = oracle.decode(t, 3, mode)
+    s1, i1, o1 = oracle.decode_paged(x.tensors(), x.k_pages, x.v_pages, x.table, 3, mode,
+                                     seq_chunks=x.seq_chunks)
+    np.testing.assert_array_equal(s0, s1)
+    np.testing.assert_array_equal(i0, i1)
+    np.testing.assert_array_equal(o0, o1)
+
+
+@pytest.mark.parametrize("mode", [ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS])
+@pytest.mark.parametrize("chunks", [(7, 10), (2, 0), (1, 5)])
+def test_paged_short_sequence_is_the_truncated_problem(mode, chunks):
+    """Sequence b with nb < N chunks: its scores, selection and output are
+    those of a one-sequence dense problem with N = nb and k = min(k, nb)
+    (sliced arrays), its scores past nb are -inf and its selection is padded
+    with -1; the decoy gists past nb (needles twice as strong) are ignored."""
+    ps, x = _paged_small(list(chunks), mode)
+    kr, vr = x.dense_raw()
+    s1, i1, o1 = oracle.decode_paged(x.tensors(), x.k_pages, x.v_pages, x.table, 3, mode,
+                                     seq_chunks=x.seq_chunks)
+    G = ps.base.group
+    for b, n in enumerate(chunks):
+        kk = min(3, n)
+        sl = lambda a: np.ascontiguousarray(a[b:b + 1, :, :n])
+        t = dict(q=np.ascontiguousarray(x.q[b:b + 1]), k_gist=sl(x.k_gist), v_gist=sl(x.v_gist),
+                 k_raw=sl(kr), v_raw=sl(vr), k_tail=np.ascontiguousarray(x.k_tail[b:b + 1]),
+                 v_tail=np.ascontiguousarray(x.v_tail[b:b + 1]))
+        s0, i0, o0 = oracle.decode(t, kk, mode)
+        np.testing.assert_array_equal(s1[b, :, :n], s0[0])
+        assert np.all(s1[b, :, n:] == -np.inf)
+        np.testing.assert_array_equal(i1[b, :, :kk], i0[0])
+        assert np.all(i1[b, :, kk:] == -1)
+        np.testing.assert_array_equal(o1[b], o0[0])
+
+
+def test_paged_sequences_sharing_a_document_see_the_same_raw_keys():
+    """Two sequences whose tables name the same page read the same bytes: a
+    pool page changed in place changes the output of both and nothing else."""
+    ps, x = _paged_small([10, 10], SR_ONLY, k=10)
+    common = sorted(set(x.table[0].tolist()) & set(x.table[1].tolist()))
+    assert common, "the draw gives the two sequences a shared document"
+    _, _, o0 = oracle.decode_paged(x.tensors(), x.k_pages, x.v_pages, x.table, 10, SR_ONLY)
+    vp = x.v_pages.copy()
+    vp[common[0]] += 1.0
+    _, _, o1 = oracle.decode_paged(x.tensors(), x.k_pages, vp, x.table, 10, SR_ONLY)
+    assert np.all(np.abs(o1 - o0).max(axis=(1, 2)) > 0)
+    unused = sorted(set(range(x.k_pages.shape[0])) - set(x.table[x.table >= 0].tolist()))
+    assert unused
+    vp = x.v_pages.copy()
+    vp[unused] += 1.0
+    _, _, o2 = oracle.decode_paged(x.tensors(), x.k_pages, vp, x.table, 10, SR_ONLY)
+    np.testing.assert_array_equal(o2, o0)

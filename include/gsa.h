@@ -8,6 +8,8 @@
  *   [EN-2]  gist.science explainer (EN), section 2 "Methodology: Gist Sparse
  *           Attention" (interleaved gist tokens; gist as routing signals;
  *           selective unfolding; hybrid attention; hierarchical extension);
+ *   [EN-4]  gist.science explainer (EN), section 4 "Experimental Results"
+ *           (KV-cache reuse);
  *   [DE-M]  gist.science explainer (DE), section "Methodik";
  *   [DE-E]  gist.science explainer (DE), section "Ergebnisse";
  *   [SL-n]  Taki-lab slide deck (docswell), page n: 6 "GSA とは", 7 "Gist
@@ -193,6 +195,30 @@ gsa_status gsa_decode_step_topp(const gsa_decode_desc* desc, float top_p, const 
                                 const void* k_tail, const void* v_tail, int32_t* idx_out,
                                 int32_t* count_out, float* scores_out, void* out, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/* One decode step over a paged, multi-document raw cache ([EN-4] "KV-Cache
+ * Reuse": the caches of documents are computed once and reused, and the
+ * gists route the query to the relevant documents without a scan of their
+ * raw caches).  The raw K/V live in page pools k_pages / v_pages
+ * [n_pages][Hkv][c][d], one page per chunk holding that chunk for every KV
+ * head; chunk j of sequence b is page block_table[b][j] (int32 [B][N]), so
+ * sequences that hold the same document name the same pages.  seq_chunks
+ * (int32 [B], nullable: every sequence has N chunks) gives each sequence's
+ * chunk count nb <= N: its gists j >= nb (of k_gist / v_gist [B][Hkv][N][d],
+ * which stay dense per sequence) do not exist, score -inf, are never
+ * selected and are not in the context, and with nb < k the selection holds
+ * all nb chunks and its other places are -1.  Table entries past nb are not
+ * read.  A page index outside [0, n_pages) or a chunk count outside [0, N]
+ * is clamped into range and flagged in the workspace error word
+ * (GSA_WS_ERR_INDEX).  With seq_chunks given, tail_len >= 1 (a sequence
+ * with no chunk keeps its tail as context).  Other arguments, the workspace
+ * size and the outputs as for gsa_decode_step; n_pages * Hkv * c <= 2^30.  */
+gsa_status gsa_decode_step_paged(const gsa_decode_desc* desc, const void* q, const void* k_gist,
+                                 const void* v_gist, const void* k_pages, const void* v_pages,
+                                 int32_t n_pages, const int32_t* block_table,
+                                 const int32_t* seq_chunks, const void* k_tail, const void* v_tail,
+                                 int32_t* idx_out, float* scores_out, void* out, void* ws,
+                                 size_t ws_bytes, void* stream);
 
 /* Hierarchical decode: level-2 scores over every meta-gist -> top-k2 groups;
  * level-1 scores over the gists of those groups -> top-k1 chunks among them;

@@ -25,7 +25,7 @@ EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", 
            "gsa_unfold_attn", "gsa_decode_step", "gsa_hier_decode", "gsa_gist_prefill",
            "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count",
            "gsa_hier_launch_count", "gsa_device_error", "gsa_set_wait_limit_ns", "gsa_topp",
-           "gsa_decode_step_topp")
+           "gsa_decode_step_topp", "gsa_decode_step_paged")
 
 
 class GsaError(RuntimeError):
@@ -73,6 +73,7 @@ def _signatures():
         "gsa_device_error": (st, [ctypes.POINTER(ctypes.c_uint32), vp]),
         "gsa_topp": (st, [pd, ctypes.c_float, vp, vp, vp, vp]),
         "gsa_decode_step_topp": (st, [pd, ctypes.c_float] + [vp] * 11 + [sz, vp]),
+        "gsa_decode_step_paged": (st, [pd] + [vp] * 5 + [ctypes.c_int32] + [vp] * 8 + [sz, vp]),
         "gsa_set_wait_limit_ns": (st, [ctypes.c_uint64]),
         "gsa_status_string": (ctypes.c_char_p, [st]),
         "gsa_decode_launch_count": (ctypes.c_int, [pd]),
@@ -259,3 +260,14 @@ def gsa_decode_step_topp(desc, top_p, q, k_gist, v_gist, k_raw, v_raw, k_tail, v
                                       _ptr(k_raw), _ptr(v_raw), _ptr(k_tail), _ptr(v_tail), _ptr(idx_out),
                                       _ptr(count_out), _ptr(scores_out), _ptr(out), _ptr(ws), nb, _stream(stream)),
            "gsa_decode_step_topp")
+
+
+def gsa_decode_step_paged(desc, q, k_gist, v_gist, k_pages, v_pages, n_pages, block_table, seq_chunks, k_tail,
+                          v_tail, idx_out, scores_out, out, ws, stream=None, ws_bytes=None):
+    """Decode step over a paged raw cache: k_pages / v_pages [n_pages, Hkv, c, d],
+    block_table int32 [B, N], seq_chunks int32 [B] or None."""
+    nb = _nbytes(ws) if ws_bytes is None else ws_bytes
+    _check(lib().gsa_decode_step_paged(ctypes.byref(desc), _ptr(q), _ptr(k_gist), _ptr(v_gist), _ptr(k_pages),
+                                       _ptr(v_pages), int(n_pages), _ptr(block_table), _ptr(seq_chunks),
+                                       _ptr(k_tail), _ptr(v_tail), _ptr(idx_out), _ptr(scores_out), _ptr(out),
+                                       _ptr(ws), nb, _stream(stream)), "gsa_decode_step_paged")

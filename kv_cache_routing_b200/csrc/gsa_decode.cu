@@ -72,6 +72,11 @@ struct PassParams {
     const int32_t* parent_idx;        // [rows][parent_k]
     int parent_k, group;
     int slot_base, slot_stride;       // gist-pass partial slots: [rows][slot_stride], this pass at slot_base + s
+    // paged raw cache (table != null): chunk j of sequence b is page table[b N + j] of the
+    // pools kr / vr [n_pages][Hkv][c][d]; nch (may be null) holds each sequence's chunk count
+    const int32_t* table;
+    const int32_t* nch;
+    int n_pages;
 };
 
 // --------------------------------------------------------- shared memory --
@@ -113,9 +118,21 @@ __device__ __forceinline__ int gist_of(const PassParams& p, int row, int v) {
     return __ldcg(p.parent_idx + (size_t)row * p.parent_k + u) * p.group + (v - u * p.group);
 }
 
+// Chunks of sequence b: nch[b] clamped into [0, N] (a value outside is
+// flagged when err is given), or N.
+__device__ __forceinline__ int seq_chunks(const int32_t* nch, uint32_t* err, int b, int N) {
+    if (nch == nullptr) return N;
+    const int n = __ldg(nch + b);
+    if (n < 0 || n > N) {
+        if (err != nullptr) atomicOr(err, kErrIndex);
+        return n < 0 ? 0 : N;
+    }
+    return n;
+}
+
 // Valid entries of a row's virtual gist list.
 __device__ __forceinline__ int valid_entries(const PassParams& p, int row) {
-    if (p.parent_idx == nullptr) return p.Nv;
+    if (p.parent_idx == nullptr) return seq_chunks(p.nch, p.err, row / p.Hkv, p.Nv);
     if (p.parent_k == 0) return 0;
     const int last = __ldcg(p.parent_idx + (size_t)row * p.parent_k + p.parent_k - 1);
     return (p.parent_k - 1) * p.group + min(p.group, p.N - last * p.group);
@@ -224,6 +241,11 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
         }
     }
     __syncthreads();
+    if (p.do_score && p.nch != nullptr) {
+        // gists past the sequence's chunk count do not exist: score -inf
+        for (int j = max(j0, nvalid) + threadIdx.x; j < min(t1 * C::TILE, p.Nv); j += NTHREADS)
+            p.scores[score_row + j] = kNegInf;
+    }
 
     if (attn) {
         CombineView<D, G> cv(&sm.stage[0][0][0]);
@@ -239,7 +261,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
         for (int s2 = 0; s2 < s; ++s2) {
             int a0, a1;
             split_range(s2, p.SA, p.tprA, a0, a1);
-            const int len = min(a1 * C::TILE, p.Nv) - a0 * C::TILE;
+            const int len = max(0, min(a1 * C::TILE, nvalid) - a0 * C::TILE);
             off += min(p.K, len);
         }
         const float* sc = p.scores + score_row + j0;
@@ -267,9 +289,18 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
     if (p.local_topk) {
         const uint32_t* ck = p.cand_key + (size_t)row * p.candA;
         const int32_t* ci = p.cand_idx + (size_t)row * p.candA;
+        // candidates the splits left (all of candA unless the sequence is short)
+        int ncand = 0;
+        for (int s2 = 0; s2 < p.SA; ++s2) {
+            int a0, a1;
+            split_range(s2, p.SA, p.tprA, a0, a1);
+            ncand += min(p.K, max(0, min(a1 * C::TILE, nvalid) - a0 * C::TILE));
+        }
         block_topk<NTHREADS>(
-            (int)p.candA, p.K, [&](int i) { return __ldcg(ck + i); },
+            ncand, p.K, [&](int i) { return __ldcg(ck + i); },
             [&](int r, int i) { out[r] = gist_of(p, row, __ldcg(ci + i)); }, sm.topk);
+        // a sequence shorter than k: its other places are empty
+        for (int r = min(p.K, ncand) + threadIdx.x; r < p.K; r += NTHREADS) out[r] = -1;
     } else {
         const float* sc = p.scores + score_row;
         block_topk<NTHREADS>(
@@ -280,6 +311,23 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
 }
 
 // ========================================================== unfold pass ====
+// First raw row of chunk j of `row`: in the dense cache [rows][N][c], or in
+// the page pool [n_pages][Hkv][c] (a page outside the pool is clamped into it
+// and flagged).  An empty place reads page 0, which always exists.
+__device__ __forceinline__ size_t raw_first_row(const PassParams& p, int row, int j, bool empty) {
+    if (p.table == nullptr) return ((size_t)row * p.N + j) * p.C;
+    const int b = row / p.Hkv, hk = row - b * p.Hkv;
+    int pg = 0;
+    if (!empty) {
+        pg = __ldg(p.table + (size_t)b * p.N + j);
+        if (pg < 0 || pg >= p.n_pages) {
+            atomicOr(p.err, kErrIndex);
+            pg = pg < 0 ? 0 : p.n_pages - 1;
+        }
+    }
+    return ((size_t)pg * p.Hkv + hk) * p.C;
+}
+
 // Unfolded keys of a row, in order: for each selected chunk u (idx order) its
 // c raw tokens (then its gist in SELECTED_PAIRS mode), then the W tail tokens.
 template <int ROWB>
@@ -292,7 +340,8 @@ __device__ __forceinline__ void unfold_issue(const PassParams& p, int row, int x
         if (x < kU) {
             const int u = x / p.U, r = x % p.U;
             int j = __ldcg(p.idx_in + (size_t)row * p.K + u);
-            if (j == -1) {
+            const bool empty = j == -1;
+            if (empty) {
                 j = 0;   // an empty place of a variable-size selection: copied, then masked
             } else if (j < 0 || j >= p.N) {
                 atomicOr(p.err, kErrIndex);
@@ -300,7 +349,7 @@ __device__ __forceinline__ void unfold_issue(const PassParams& p, int row, int x
             }
             if (r < p.C) {
                 run = min(p.C - r, xe - x);
-                const size_t o = (((size_t)row * p.N + j) * p.C + r) * ROWB;
+                const size_t o = (raw_first_row(p, row, j, empty) + r) * ROWB;
                 sk = p.kr + o;
                 sv = p.vr + o;
             } else {
@@ -459,16 +508,20 @@ __global__ void __launch_bounds__(NTHREADS, 3) unfold_pass_kernel(const __grid_c
 }
 
 // =============================================================== top-k =====
-// Standalone selection: one CTA per row over the row's N scores.
+// Standalone selection: one CTA per row over the row's N scores, or over the
+// first nch[b] of them (nch may be null) with the places past those empty (-1).
 __global__ void __launch_bounds__(NTHREADS) topk_kernel(const float* __restrict__ scores, int N, int K,
-                                                        int32_t* __restrict__ idx) {
+                                                        int32_t* __restrict__ idx, const int32_t* __restrict__ nch,
+                                                        int Hkv) {
     __shared__ uint32_t sh[256 + 8 + NTHREADS / 32 + 8];
     const int row = blockIdx.x;
     const float* sc = scores + (size_t)row * N;
     int32_t* out = idx + (size_t)row * K;
     pdl_wait();
+    const int n = seq_chunks(nch, nullptr, row / Hkv, N);
     block_topk<NTHREADS>(
-        N, K, [&](int i) { return order_key(sc[i]); }, [&](int r, int i) { out[r] = i; }, sh);
+        n, K, [&](int i) { return order_key(sc[i]); }, [&](int r, int i) { out[r] = i; }, sh);
+    for (int r = min(K, n) + threadIdx.x; r < K; r += NTHREADS) out[r] = -1;
 }
 
 // =============================================================== top-p =====
@@ -692,6 +745,13 @@ static PassParams make_params(const DecodePlan& pl, const gsa_decode_desc& d, co
     return p;
 }
 
+static void set_paging(PassParams& p, const Paging* pg) {
+    if (pg == nullptr) return;
+    p.table = pg->table;
+    p.nch = pg->nch;
+    p.n_pages = pg->n_pages;
+}
+
 // Workspace bytes of a flat decode descriptor on the path it will take.
 static size_t decode_ws_bytes(const gsa_decode_desc& d) {
     return fused_supported(d) ? std::max(make_fused_plan(d).total, make_fused_plan(d, true).total)
@@ -726,8 +786,8 @@ size_t gsa_decode_workspace_size(const gsa_decode_desc* desc) {
     return decode_ws_bytes(*desc);
 }
 
-gsa_status gsa_score(const gsa_decode_desc* desc, const void* q, const void* k_gist, float* scores,
-                     void* stream) {
+static gsa_status score_impl(const gsa_decode_desc* desc, const void* q, const void* k_gist, float* scores,
+                             void* stream, const Paging* pg) {
     gsa_status st = validate_decode(desc);
     if (st != GSA_OK) return st;
     if (!q || (desc->n_chunks > 0 && (!k_gist || !scores))) return GSA_ERR_ARG;
@@ -740,12 +800,19 @@ gsa_status gsa_score(const gsa_decode_desc* desc, const void* q, const void* k_g
     p.err = sink;
     p.scores = scores;
     p.do_score = 1;
+    if (pg != nullptr) p.nch = pg->nch;
     cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, desc->n_q_heads / desc->n_kv_heads, true, false,
                                static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
-gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* idx, void* stream) {
+gsa_status gsa_score(const gsa_decode_desc* desc, const void* q, const void* k_gist, float* scores,
+                     void* stream) {
+    return score_impl(desc, q, k_gist, scores, stream, nullptr);
+}
+
+static gsa_status topk_impl(const gsa_decode_desc* desc, const float* scores, int32_t* idx, void* stream,
+                            const int32_t* nch) {
     gsa_status st = validate_decode(desc);
     if (st != GSA_OK) return st;
     if (desc->top_k == 0) return GSA_OK;
@@ -753,8 +820,12 @@ gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* i
     if (!aligned16(scores) || !aligned16(idx)) return GSA_ERR_ALIGN;
     const int rows = desc->batch * desc->n_kv_heads;
     topk_kernel<<<rows, NTHREADS, 0, static_cast<cudaStream_t>(stream)>>>(scores, desc->n_chunks, desc->top_k,
-                                                                         idx);
+                                                                         idx, nch, desc->n_kv_heads);
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+gsa_status gsa_topk(const gsa_decode_desc* desc, const float* scores, int32_t* idx, void* stream) {
+    return topk_impl(desc, scores, idx, stream, nullptr);
 }
 
 gsa_status gsa_topp(const gsa_decode_desc* desc, float top_p, const float* scores, int32_t* idx, int32_t* count,
@@ -795,9 +866,10 @@ static gsa_status check_ws(size_t need, const void* ws, size_t ws_bytes) {
     return GSA_OK;
 }
 
-gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
-                           const void* k_raw, const void* v_raw, const void* k_tail, const void* v_tail,
-                           const int32_t* idx, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+static gsa_status unfold_impl(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+                              const void* k_raw, const void* v_raw, const void* k_tail, const void* v_tail,
+                              const int32_t* idx, void* out, float* lse, void* ws, size_t ws_bytes, void* stream,
+                              const Paging* pg) {
     gsa_status st = validate_decode(desc);
     if (st != GSA_OK) return st;
     if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
@@ -806,9 +878,10 @@ gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const voi
     if ((st = check_ws(decode_ws_bytes(*desc), ws, ws_bytes)) != GSA_OK) return st;
     if (fused_supported(*desc))
         return fused_launch(*desc, make_fused_plan(*desc, true), q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx,
-                            nullptr, nullptr, out, lse, ws, static_cast<cudaStream_t>(stream));
+                            nullptr, nullptr, out, lse, ws, static_cast<cudaStream_t>(stream), pg);
     DecodePlan pl = make_decode_plan(*desc);
     PassParams p = make_params(pl, *desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ws);
+    set_paging(p, pg);
     p.idx_in = idx;
     p.out = static_cast<uint8_t*>(out);
     p.lse = lse;
@@ -820,10 +893,17 @@ gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const voi
     return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
-gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+gsa_status gsa_unfold_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
                            const void* k_raw, const void* v_raw, const void* k_tail, const void* v_tail,
-                           int32_t* idx_out, float* scores_out, void* out, void* ws, size_t ws_bytes,
-                           void* stream) {
+                           const int32_t* idx, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    return unfold_impl(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx, out, lse, ws, ws_bytes, stream,
+                       nullptr);
+}
+
+static gsa_status step_impl(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+                            const void* k_raw, const void* v_raw, const void* k_tail, const void* v_tail,
+                            int32_t* idx_out, float* scores_out, void* out, void* ws, size_t ws_bytes, void* stream,
+                            const Paging* pg) {
     gsa_status st = validate_decode(desc);
     if (st != GSA_OK) return st;
     if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
@@ -839,16 +919,17 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
         unselected_scratch(*desc, off_s, off_i);
         float* sc = scores_out ? scores_out : reinterpret_cast<float*>(w + off_s);
         int32_t* ix = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + off_i);
-        if ((st = gsa_score(desc, q, k_gist, sc, stream)) != GSA_OK) return st;
-        if ((st = gsa_topk(desc, sc, ix, stream)) != GSA_OK) return st;
-        return gsa_unfold_attn(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ix, out, nullptr, ws, ws_bytes,
-                               stream);
+        if ((st = score_impl(desc, q, k_gist, sc, stream, pg)) != GSA_OK) return st;
+        if ((st = topk_impl(desc, sc, ix, stream, pg ? pg->nch : nullptr)) != GSA_OK) return st;
+        return unfold_impl(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ix, out, nullptr, ws, ws_bytes,
+                           stream, pg);
     }
     if (fused_supported(*desc))
         return fused_launch(*desc, make_fused_plan(*desc), q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, nullptr,
-                            idx_out, scores_out, out, nullptr, ws, static_cast<cudaStream_t>(stream));
+                            idx_out, scores_out, out, nullptr, ws, static_cast<cudaStream_t>(stream), pg);
     DecodePlan pl = make_decode_plan(*desc);
     PassParams p = make_params(pl, *desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, ws);
+    set_paging(p, pg);
     if (scores_out) p.scores = scores_out;
     if (idx_out) p.idx_out = idx_out;
     p.idx_in = p.idx_out;
@@ -860,6 +941,33 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
     cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, desc->n_q_heads / desc->n_kv_heads,
                                desc->n_chunks > 0, true, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+                           const void* k_raw, const void* v_raw, const void* k_tail, const void* v_tail,
+                           int32_t* idx_out, float* scores_out, void* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+    return step_impl(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, scores_out, out, ws, ws_bytes,
+                     stream, nullptr);
+}
+
+gsa_status gsa_decode_step_paged(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+                                 const void* k_pages, const void* v_pages, int32_t n_pages,
+                                 const int32_t* block_table, const int32_t* seq_chunks, const void* k_tail,
+                                 const void* v_tail, int32_t* idx_out, float* scores_out, void* out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if (n_pages < 1 || !block_table) return GSA_ERR_ARG;
+    // a short sequence keeps the tail as its context, so the tail may not be empty
+    if (seq_chunks && desc->tail_len < 1) return GSA_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_chunks) & 3u))
+        return GSA_ERR_ALIGN;
+    // pool rows are addressed with 32-bit arithmetic
+    if ((int64_t)n_pages * desc->n_kv_heads * desc->chunk > INT32_MAX / 2) return GSA_ERR_SHAPE;
+    const Paging pg{block_table, seq_chunks, n_pages};
+    return step_impl(desc, q, k_gist, v_gist, k_pages, v_pages, k_tail, v_tail, idx_out, scores_out, out, ws,
+                     ws_bytes, stream, &pg);
 }
 
 

@@ -549,6 +549,32 @@ __device__ __forceinline__ void key_close(const Params& p, Ctx& cx) {
     group_sync<128, BAR_SOFT>();
 }
 
+// Chunks of the sequence of `row`: nch[b] clamped into [0, N] (a value
+// outside is flagged), or N.
+__device__ __forceinline__ int seq_chunks(const Params& p, int row) {
+    if (p.nch == nullptr) return p.N;
+    const int n = __ldg(p.nch + row / p.Hkv);
+    if (n < 0 || n > p.N) {
+        atomicOr(p.err, kErrIndex);
+        return n < 0 ? 0 : p.N;
+    }
+    return n;
+}
+
+// First raw row of chunk j of `row`: in the dense cache [rows][N][c], or in
+// the page pool [n_pages][Hkv][c] (a page outside the pool is clamped into
+// it and flagged).
+__device__ __forceinline__ long long raw_first(const Params& p, int row, int j) {
+    if (p.table == nullptr) return ((long long)row * p.N + j) * p.C;
+    const int b = row / p.Hkv, hk = row - b * p.Hkv;
+    int pg = __ldg(p.table + (size_t)b * p.N + j);
+    if (pg < 0 || pg >= p.n_pages) {
+        atomicOr(p.err, kErrIndex);
+        pg = pg < 0 ? 0 : p.n_pages - 1;
+    }
+    return ((long long)pg * p.Hkv + hk) * p.C;
+}
+
 // Key stretch, one unit: routing score and scaled logits of key row t.
 template <int G>
 __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u, bool new_seg, int slot) {
@@ -572,7 +598,10 @@ __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u
     tc::wait_ld();
     tc::fence_before();
     mbar_arrive(&cx.bars->s_free[sb]);
-    bool valid = t < u.nvalid;
+    const bool in_row = t < u.nvalid;
+    // gists past the sequence's chunk count do not exist: no weight, score -inf
+    const bool exists = in_row && (p.nch == nullptr || u.kind != 0 || u.t * TILE + t < seq_chunks(p, u.row));
+    bool valid = exists;
     if (p.mask_sel && u.kind == 0) {
         // the given selection's gists are not in the context: a 128-bit mask
         // of the tile's selected gists (every thread reads the selection)
@@ -603,7 +632,8 @@ __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u
         float score = 0.f;
 #pragma unroll
         for (int h = 0; h < G; ++h) score += __uint_as_float(r[h]);
-        if (valid) {
+        if (in_row) {
+            if (!exists) score = -INFINITY;
             p.scores[(size_t)u.row * p.NA + u.t * TILE + t] = score;
             if (cx.gtiles < kScoreCap / TILE)
                 reinterpret_cast<float*>(cx.base + SM_SCORE)[cx.gtiles * TILE + t] = score;
@@ -913,8 +943,10 @@ __device__ __forceinline__ void merge_select(const Params& p, uint8_t* base, int
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
     unfold_topk(p.cand_key + (size_t)row * p.NA, SRC_GKEY, n, p.K, sel, reinterpret_cast<uint32_t*>(base + SM_TOPK),
                 reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
+    const int nb = seq_chunks(p, row);
     for (int r = utid(); r < min(p.K, n); r += NU) {
-        const int32_t j = __ldcg(ci + sel[r]);
+        int32_t j = __ldcg(ci + sel[r]);
+        if (j >= nb) j = -1;   // a sequence shorter than k: the place is empty
         sel[r] = j;
         if (publish) out[r] = j;
     }
@@ -926,6 +958,12 @@ __device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, in
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
     unfold_topk(p.scores + (size_t)row * p.NA, SRC_GSCORE, p.NA, p.K, sel, reinterpret_cast<uint32_t*>(base + SM_TOPK),
                 reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
+    if (p.nch != nullptr) {
+        const int nb = seq_chunks(p, row);
+        for (int r = utid(); r < p.K; r += NU)
+            if (sel[r] >= nb) sel[r] = -1;   // a sequence shorter than k: the place is empty
+        usync();
+    }
     if (publish)
         for (int r = utid(); r < min(p.K, p.NA); r += NU) out[r] = sel[r];
 }
@@ -957,7 +995,7 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
         int32_t e = -1;
         if (gr < kc) {
             const int sidx = gr / p.C, tok = gr - sidx * p.C;
-            if (sel[sidx] >= 0) e = (int32_t)(((long long)row * p.N + sel[sidx]) * p.C + tok);
+            if (sel[sidx] >= 0) e = (int32_t)(raw_first(p, row, sel[sidx]) + tok);
         } else if (gr < p.nrows_g) {
             if (sel[gr - kc] >= 0) e = (int32_t)(-((long long)row * p.N + sel[gr - kc]) - 2);
         }
@@ -1004,16 +1042,23 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
         mbar_expect_tx(&bars->full[sv], bytes);
         const CUtensorMap* mk = children ? &p.tm_kc : &p.tm_kr;
         const CUtensorMap* mv = children ? &p.tm_vc : &p.tm_vr;
-        const long long n_src = p.hier ? (long long)p.N1 : (long long)p.N;   // chunks (level-1 gists) per row
         for (int r = uw * h; r < tma_rows; r += (NU / 32) * h) {
             const long long e = tab[r];
             if (e == -1) continue;
-            // source row of the run: token (chunk * c) of the row's raw rows, or the first child
-            const int y = children ? (int)(-e - 2 - (long long)row * n_src) : (int)(e - (long long)row * n_src * p.C);
-            tc::tma_load_3d(ks + r * 128, mk, 0, y, row, &bars->full[sk]);
-            tc::tma_load_3d(ks + 16384 + r * 128, mk, 64, y, row, &bars->full[sk]);
-            tc::tma_load_3d(vs + r * 128, mv, 0, y, row, &bars->full[sv]);
-            tc::tma_load_3d(vs + 16384 + r * 128, mv, 64, y, row, &bars->full[sv]);
+            // the run's source: a whole chunk (box {64, c, 1} at chunk e / c of
+            // the raw map), or the first child of a group in the row's level-1 gists
+            int y, z;
+            if (children) {
+                y = (int)(-e - 2 - (long long)row * p.N1);
+                z = row;
+            } else {
+                z = (int)(e / p.C);
+                y = (int)(e - (long long)z * p.C);
+            }
+            tc::tma_load_3d(ks + r * 128, mk, 0, y, z, &bars->full[sk]);
+            tc::tma_load_3d(ks + 16384 + r * 128, mk, 64, y, z, &bars->full[sk]);
+            tc::tma_load_3d(vs + r * 128, mv, 0, y, z, &bars->full[sv]);
+            tc::tma_load_3d(vs + 16384 + r * 128, mv, 64, y, z, &bars->full[sv]);
         }
     }
 #pragma unroll 4
@@ -1780,7 +1825,8 @@ static void fill_common(fused::Params& p, const FusedPlan& f, const gsa_decode_d
 
 gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void* q, const void* kg, const void* vg,
                         const void* kr, const void* vr, const void* kt, const void* vt, const int32_t* idx_given,
-                        int32_t* idx_out, float* scores_out, void* out, float* lse, void* ws, cudaStream_t st) {
+                        int32_t* idx_out, float* scores_out, void* out, float* lse, void* ws, cudaStream_t st,
+                        const Paging* pg) {
     using namespace fused;
     if (f.grid <= 0) return GSA_ERR_ARG;
     Params p;
@@ -1789,9 +1835,11 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
     bool ok = map3d(&p.tm_kg, kg, rows, N) && map3d(&p.tm_vg, f.attn_gists ? vg : nullptr, rows, N) &&
               map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
     p.tma_raw = chunk_runs(d.chunk) && f.nbt > 0 ? 1 : 0;
+    // the raw cache as chunks: [rows N][c][d] dense, [n_pages Hkv][c][d] paged
+    const uint64_t nchunk = pg ? (uint64_t)pg->n_pages * (uint64_t)d.n_kv_heads : rows * N;
     if (p.tma_raw)
-        ok = ok && map3d(&p.tm_kr, kr, rows, N * (uint64_t)d.chunk, (uint32_t)d.chunk) &&
-             map3d(&p.tm_vr, vr, rows, N * (uint64_t)d.chunk, (uint32_t)d.chunk);
+        ok = ok && map3d(&p.tm_kr, kr, nchunk, (uint64_t)d.chunk, (uint32_t)d.chunk) &&
+             map3d(&p.tm_vr, vr, nchunk, (uint64_t)d.chunk, (uint32_t)d.chunk);
     if (!ok) return GSA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     fill_common(p, f, d, w);
@@ -1814,6 +1862,11 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
     p.do_attn_gists = f.attn_gists;
     // a given selection in UNSELECTED_GISTS mode: its gists leave the context
     p.mask_sel = (idx_given != nullptr && d.mode == GSA_UNSELECTED_GISTS) ? 1 : 0;
+    if (pg != nullptr) {
+        p.table = pg->table;
+        p.nch = pg->nch;
+        p.n_pages = pg->n_pages;
+    }
     return launch(p, f.G, f.grid, st) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
@@ -1862,8 +1915,8 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
     p.tma_children = chunk_runs(h.group) ? 1 : 0;
     const uint64_t n1 = (uint64_t)d.n_chunks;
     if (p.tma_raw)
-        ok = ok && map3d(&p.tm_kr, kr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk) &&
-             map3d(&p.tm_vr, vr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk);
+        ok = ok && map3d(&p.tm_kr, kr, rows * n1, (uint64_t)d.chunk, (uint32_t)d.chunk) &&
+             map3d(&p.tm_vr, vr, rows * n1, (uint64_t)d.chunk, (uint32_t)d.chunk);
     if (p.tma_children)
         ok = ok && map3d(&p.tm_kc, k_g1, rows, n1, (uint32_t)h.group) && map3d(&p.tm_vc, v_g1, rows, n1, (uint32_t)h.group);
     if (!ok) return GSA_ERR_CUDA;

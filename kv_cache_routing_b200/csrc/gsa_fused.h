@@ -30,7 +30,7 @@ namespace fused {
 struct Params {
     CUtensorMap tm_kg, tm_vg;      // gists  [rows][N][d], box {64, 128, 1}
     CUtensorMap tm_kt, tm_vt;      // tail   [rows][W][d], box {64, 128, 1}
-    CUtensorMap tm_kr, tm_vr;      // raw    [rows][N c][d], box {64, c, 1} (chunk gathers by TMA)
+    CUtensorMap tm_kr, tm_vr;      // raw as chunks [rows N | pages Hkv][c][d], box {64, c, 1} (chunk gathers by TMA)
     CUtensorMap tm_kc, tm_vc;      // hierarchy: level-1 gists [rows][N1][d], box {64, group, 1}
     const uint16_t* q;             // [B][Hq][d]
     const uint8_t* kr;             // raw K/V and gist K/V base pointers (gathered tiles)
@@ -58,6 +58,11 @@ struct Params {
     float c2;
     int do_score, do_topk, do_attn_gists, sel_direct;
     int mask_sel;                  // given selection, UNSELECTED_GISTS: its gists are masked in the key stretch
+    // paged raw cache (table != null): chunk j of sequence b is page table[b N + j] of the
+    // pools [n_pages][Hkv][c][d]; nch (may be null) holds each sequence's chunk count
+    const int32_t* table;
+    const int32_t* nch;
+    int n_pages;
     // hierarchy (keys/values: level-2 gists; unfold: children tile, then raw tile)
     int hier, group, N1, K1;       // K = k2, N = NA = n_l2; group, level-1 gists, k1
     int32_t* idx1;                 // [rows][k1]
@@ -78,8 +83,10 @@ FusedPlan make_fused_plan(const gsa_decode_desc& d, bool given = false);
 // Enqueue the fused decode step (one launch).  idx_given != null: attend over
 // that selection (no scores, no selection); else select and write idx_out (or
 // the workspace copy) and scores_out (or the workspace copy).
+// pg (may be null): kr / vr are page pools and the chunks are found through pg's table.
 gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void* q, const void* kg, const void* vg,
                         const void* kr, const void* vr, const void* kt, const void* vt, const int32_t* idx_given,
-                        int32_t* idx_out, float* scores_out, void* out, float* lse, void* ws, cudaStream_t st);
+                        int32_t* idx_out, float* scores_out, void* out, float* lse, void* ws, cudaStream_t st,
+                        const Paging* pg = nullptr);
 
 }  // namespace gsa

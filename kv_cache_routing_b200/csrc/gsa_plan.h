@@ -24,6 +24,16 @@ constexpr int kMaxSplits = 256;
 cudaError_t prefill_error_word(uint32_t** addr);        // gsa_prefill.cu
 cudaError_t set_cross_cta_wait_limit(uint64_t ns);      // gsa_fused.cu (0 restores the default)
 
+// A paged raw cache: chunk j of sequence b is page table[b * N + j] of the
+// pools k_pages / v_pages [n_pages][Hkv][c][d] (one page: one chunk of every
+// KV head); sequence b has nch[b] chunks (nch null: all N).  Dense callers
+// pass no Paging.
+struct Paging {
+    const int32_t* table;
+    const int32_t* nch;
+    int n_pages;
+};
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 

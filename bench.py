@@ -23,9 +23,10 @@ by the slowest rank's time.
 cores on a bounded sample of the same workload.
 
 Other workloads: --workload NAME for every decode shape of synth.WORKLOADS
-(the sweeps), hier_1m (two-level descent, steps/s against the HBM roofline)
-and gist_prefill (the gist-causal prefill, algorithmic TFLOP/s against the
-bf16 tensor roofline).
+(the sweeps), llama8b_paged (the same step over a shared page pool of
+documents through gsa_decode_step_paged), hier_1m (two-level descent, steps/s
+against the HBM roofline) and gist_prefill (the gist-causal prefill,
+algorithmic TFLOP/s against the bf16 tensor roofline).
 """
 from __future__ import annotations
 
@@ -58,6 +59,24 @@ def algorithmic_bytes(s: synth.DecodeShape) -> int:
     per_kv += 2 * s.top_k * s.chunk * row                               # unfolded raw K, V
     per_kv += 2 * s.tail_len * row                                      # tail K, V
     return s.rows * per_kv + 2 * s.batch * s.n_q_heads * row            # + q and out
+
+
+def paged_bytes(ps: synth.PagedShape, seq_chunks: np.ndarray) -> int:
+    """algorithmic_bytes with each sequence's own chunk count nb: nb gist
+    keys (and values), the raw K/V of min(k, nb) chunks, the tail."""
+    s = ps.base
+    e = 4 if s.dtype == "f32" else 2
+    row = s.head_dim * e
+    total = 2 * s.batch * s.n_q_heads * row
+    for nb in seq_chunks.tolist():
+        kk = min(s.top_k, nb)
+        per_kv = nb * row + (nb if s.mode == synth.ALL_GISTS else kk) * row + 2 * kk * s.chunk * row
+        total += s.n_kv_heads * (per_kv + 2 * s.tail_len * row)
+    return total
+
+
+MODE_NAMES = {synth.ALL_GISTS: "ALL_GISTS", synth.SELECTED_PAIRS: "SELECTED_PAIRS", synth.SR_ONLY: "SR_ONLY",
+              synth.UNSELECTED_GISTS: "UNSELECTED_GISTS"}
 
 
 def _dev(a: np.ndarray):
@@ -101,11 +120,19 @@ def decode_config(s, workload: str, world: int, L: int, nbytes_step: int, l2: in
     """The `config` of a flat decode line (both arms print the same one)."""
     return {"workload": workload, "batch": s.batch, "n_q_heads": s.n_q_heads, "n_kv_heads": s.n_kv_heads,
             "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk, "chunk": s.chunk, "n_gists": s.n_chunks,
-            "top_k": s.top_k, "tail": s.tail_len,
-            "mode": "ALL_GISTS" if s.mode == synth.ALL_GISTS else "SELECTED_PAIRS",
+            "top_k": s.top_k, "tail": s.tail_len, "mode": MODE_NAMES[s.mode],
             "parallelism": f"replicas x{world}",
             "l2": f"rotating {L} layer replicas, {L * nbytes_step / 1e6:.0f} MB touched per rotation "
                   f"(L2 {l2 / 1e6:.0f} MB)"}
+
+
+def paged_config(ps, x, workload: str, world: int, L: int, nbytes_step: int, l2: int) -> dict:
+    c = decode_config(ps.base, workload, world, L, nbytes_step, l2)
+    c.update({"n_pages": int(x.k_pages.shape[0]), "n_docs": ps.n_docs,
+              "doc_chunks": f"{ps.doc_min}..{ps.doc_max}",
+              "seq_chunks_mean": round(float(np.mean(x.seq_chunks)), 1),
+              "pages_shared": int(x.table[x.table >= 0].size - np.unique(x.table[x.table >= 0]).size)})
+    return c
 
 
 def hier_config(h, workload: str, world: int, L: int, nbytes: int, l2: int) -> dict:
@@ -334,13 +361,25 @@ def run_ours(args, world, rank, local):
 
     import kv_cache_routing_b200 as gsa
 
-    s = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[args.workload]
+    paged = isinstance(w, synth.PagedShape)
+    s = w.base if paged else w
     torch.cuda.set_device(local)
     l2 = l2_bytes(local)
-    nbytes_step = algorithmic_bytes(s)
+    if paged:
+        x = synth.paged_inputs(w, synth.seed_for(args.workload) + 17 * rank)
+        nbytes_step = paged_bytes(w, x.seq_chunks)
+    else:
+        x = synth.decode_inputs(s, synth.seed_for(args.workload) + 17 * rank)
+        nbytes_step = algorithmic_bytes(s)
     L = replicas_for(nbytes_step, l2, args.replicas)
-    x = synth.decode_inputs(s, synth.seed_for(args.workload) + 17 * rank)
     base = {k: _dev(v) for k, v in x.tensors().items()}
+    if paged:
+        # every replica has its own pool (its own layer's caches); the table is shared
+        base["k_pages"], base["v_pages"] = _dev(x.k_pages), _dev(x.v_pages)
+        table = torch.from_numpy(x.table).cuda()
+        nch = torch.from_numpy(x.seq_chunks).cuda()
+        n_pages = int(x.k_pages.shape[0])
     reps = []
     for r in range(L):
         t = {k: (v if r == 0 else v.clone()) for k, v in base.items()}
@@ -359,8 +398,13 @@ def run_ours(args, world, rank, local):
 
     def step(i, st):
         t = reps[i % L]
-        gsa.gsa_decode_step(desc, t["q"], t["k_gist"], t["v_gist"], t["k_raw"], t["v_raw"], t["k_tail"],
-                            t["v_tail"], idxs[i % L], None, outs[i % L], ws, stream=st)
+        if paged:
+            gsa.gsa_decode_step_paged(desc, t["q"], t["k_gist"], t["v_gist"], t["k_pages"], t["v_pages"], n_pages,
+                                      table, nch, t["k_tail"], t["v_tail"], idxs[i % L], None, outs[i % L], ws,
+                                      stream=st)
+        else:
+            gsa.gsa_decode_step(desc, t["q"], t["k_gist"], t["v_gist"], t["k_raw"], t["v_raw"], t["k_tail"],
+                                t["v_tail"], idxs[i % L], None, outs[i % L], ws, stream=st)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -411,6 +455,7 @@ def run_ours(args, world, rank, local):
     steps_per_s = whole_job_rate(args.steps, world, ms_max)
     gbs = nbytes_step / (per_step_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
+    entry = "gsa_decode_step_paged" if paged else "gsa_decode_step"
     line = {
         "metric": METRIC,
         "value": round(steps_per_s, 2),
@@ -424,15 +469,16 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": s.dtype,
         "data": "synthetic",
-        "config": decode_config(s, args.workload, world, L, nbytes_step, l2),
+        "config": (paged_config(w, x, args.workload, world, L, nbytes_step, l2) if paged else
+                   decode_config(s, args.workload, world, L, nbytes_step, l2)),
         "timing": {"replays": len(reps_ms), "statistic": "median over replays of the K-step graph",
                    "ms_per_step_min": round(min(reps_ms) / args.steps, 5),
                    "ms_per_step_max": round(max(reps_ms) / args.steps, 5)},
         "head_steps_per_s": round(steps_per_s * s.batch * s.n_q_heads, 1),
         "algorithmic_bytes_per_step": nbytes_step,
         "roofline": {"bound": "hbm",
-                     "kernel": (f"gsa_decode_step: one launch of fused_decode_kernel per step" if launches == 1 else
-                                f"gsa_decode_step: {launches} launches per step (per launch: 1/{launches} of the "
+                     "kernel": (f"{entry}: one launch of fused_decode_kernel per step" if launches == 1 else
+                                f"{entry}: {launches} launches per step (per launch: 1/{launches} of the "
                                 f"step's algorithmic bytes in 1/{launches} of its time)"),
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                      "peak_kind": peak_kind,
@@ -447,7 +493,7 @@ def run_ours(args, world, rank, local):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(s, x, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(s, x, args.cpu_seconds, w if paged else None)
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g
@@ -653,15 +699,24 @@ def run_hier(args, world, rank, local):
 
 
 # ------------------------------------------------------------ CPU oracle ----
-def cpu_baseline(s, x, budget_s: float):
-    """The fp64 oracle, as it stands, on the host cores: whole decode steps of
-    the same workload until the time budget is spent (at least one)."""
+def _oracle_step(s, x, ps=None):
+    """One whole decode step of the oracle on the workload's inputs."""
     import oracle
     t = x.tensors()
-    oracle.decode(t, s.top_k, s.mode)  # load + warm
+    if ps is not None:
+        return lambda: oracle.decode_paged(t, x.k_pages, x.v_pages, x.table, s.top_k, s.mode,
+                                           seq_chunks=x.seq_chunks)
+    return lambda: oracle.decode(t, s.top_k, s.mode)
+
+
+def cpu_baseline(s, x, budget_s: float, ps=None):
+    """The fp64 oracle, as it stands, on the host cores: whole decode steps of
+    the same workload until the time budget is spent (at least one)."""
+    run = _oracle_step(s, x, ps)
+    run()  # load + warm
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.decode(t, s.top_k, s.mode)
+        run()
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 1000:
@@ -727,6 +782,14 @@ def run_reference(args, world, rank):
         config = hier_config(w, args.workload, world, replicas_for(nb, l2, args.replicas), nb, l2)
         sample = f"one full hierarchical step per step ({w.l1.rows} rows, OpenMP over rows), fp64"
         cores = min(cores, w.l1.rows)
+        rate = lambda sec: 1.0 / sec
+    elif isinstance(w, synth.PagedShape):
+        x = synth.paged_inputs(w, seed)
+        run = _oracle_step(w.base, x, w)
+        metric, unit, dtype = METRIC, "steps/s", "f64"
+        nb = paged_bytes(w, x.seq_chunks)
+        config = paged_config(w, x, args.workload, world, replicas_for(nb, l2, args.replicas), nb, l2)
+        sample = f"one full decode step per step ({w.base.rows} rows, OpenMP over rows), fp64"
         rate = lambda sec: 1.0 / sec
     else:
         x = synth.decode_inputs(w, seed)

@@ -576,7 +576,7 @@ __device__ __forceinline__ long long raw_first(const Params& p, int row, int j) 
 }
 
 // Key stretch, one unit: routing score and scaled logits of key row t.
-template <int G>
+template <int G, bool PG>
 __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u, bool new_seg, int slot) {
     const int t = threadIdx.x;
     if (new_seg) {
@@ -600,7 +600,8 @@ __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u
     mbar_arrive(&cx.bars->s_free[sb]);
     const bool in_row = t < u.nvalid;
     // gists past the sequence's chunk count do not exist: no weight, score -inf
-    const bool exists = in_row && (p.nch == nullptr || u.kind != 0 || u.t * TILE + t < seq_chunks(p, u.row));
+    bool exists = in_row;
+    if constexpr (PG) exists = exists && (p.nch == nullptr || u.kind != 0 || u.t * TILE + t < seq_chunks(p, u.row));
     bool valid = exists;
     if (p.mask_sel && u.kind == 0) {
         // the given selection's gists are not in the context: a 128-bit mask
@@ -633,7 +634,9 @@ __device__ __forceinline__ void key_tile(const Params& p, Ctx& cx, const Tile& u
 #pragma unroll
         for (int h = 0; h < G; ++h) score += __uint_as_float(r[h]);
         if (in_row) {
-            if (!exists) score = -INFINITY;
+            if constexpr (PG) {
+                if (!exists) score = -INFINITY;
+            }
             p.scores[(size_t)u.row * p.NA + u.t * TILE + t] = score;
             if (cx.gtiles < kScoreCap / TILE)
                 reinterpret_cast<float*>(cx.base + SM_SCORE)[cx.gtiles * TILE + t] = score;
@@ -772,7 +775,7 @@ __device__ __forceinline__ void gathered_softmax(const Params& p, Ctx& cx, const
     }
 }
 
-template <int G>
+template <int G, bool PG>
 __device__ __forceinline__ void softmax_run(const Params& p, Ctx& cx, const Run& r) {
     const int* ub = reinterpret_cast<const int*>(cx.base + SM_UB);
     const int c = blockIdx.x;
@@ -782,7 +785,7 @@ __device__ __forceinline__ void softmax_run(const Params& p, Ctx& cx, const Run&
         for (int i = 0; i < r.n; ++i) {
             const Tile u = unit_tile(p, r.u0 + i);
             const bool ns = u.row != prev_row;
-            key_tile<G>(p, cx, u, ns, ns ? seg_slot(u.row) : cx.cur_slot);
+            key_tile<G, PG>(p, cx, u, ns, ns ? seg_slot(u.row) : cx.cur_slot);
             prev_row = u.row;
         }
         if (cx.cur_row >= 0) key_close<G>(p, cx);
@@ -826,14 +829,14 @@ __device__ __forceinline__ void softmax_run(const Params& p, Ctx& cx, const Run&
 
 // Run the three roles over one stretch.  Ends with the streaming warps
 // synchronised and every segment of the stretch closed.
-template <int G>
+template <int G, bool PG>
 __device__ __forceinline__ void run_pipeline(const Params& p, Ctx& cx, const Run& r) {
     if (cx.warp == 4) {
         produce_run(p, cx, r);
     } else if (cx.warp == 5) {
         if (cx.lane == 0) mma_run(p, cx, r);
     } else {
-        softmax_run<G>(p, cx, r);
+        softmax_run<G, PG>(p, cx, r);
     }
     group_sync<NT, BAR_PIPE>();
 }
@@ -937,28 +940,30 @@ __device__ __forceinline__ void local_topk(const Params& p, uint8_t* base, int r
 // The row's exact top-k into the shared selection sel[0..k) and, when
 // `publish`, into the row's idx output: from the candidates that every CTA
 // meeting the row left (n of them), or straight from its routing scores.
+template <bool PG>
 __device__ __forceinline__ void merge_select(const Params& p, uint8_t* base, int row, int n, bool publish) {
     const int32_t* ci = p.cand_idx + (size_t)row * p.NA;
     int32_t* out = p.idx + (size_t)row * p.K;
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
     unfold_topk(p.cand_key + (size_t)row * p.NA, SRC_GKEY, n, p.K, sel, reinterpret_cast<uint32_t*>(base + SM_TOPK),
                 reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
-    const int nb = seq_chunks(p, row);
+    const int nb = PG ? seq_chunks(p, row) : p.N;
     for (int r = utid(); r < min(p.K, n); r += NU) {
         int32_t j = __ldcg(ci + sel[r]);
-        if (j >= nb) j = -1;   // a sequence shorter than k: the place is empty
+        if (PG && j >= nb) j = -1;   // a sequence shorter than k: the place is empty
         sel[r] = j;
         if (publish) out[r] = j;
     }
     usync();
 }
 
+template <bool PG>
 __device__ __forceinline__ void direct_select(const Params& p, uint8_t* base, int row, bool publish) {
     int32_t* out = p.idx + (size_t)row * p.K;
     int32_t* sel = reinterpret_cast<int32_t*>(base + SM_SEL);
     unfold_topk(p.scores + (size_t)row * p.NA, SRC_GSCORE, p.NA, p.K, sel, reinterpret_cast<uint32_t*>(base + SM_TOPK),
                 reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
-    if (p.nch != nullptr) {
+    if (PG && p.nch != nullptr) {
         const int nb = seq_chunks(p, row);
         for (int r = utid(); r < p.K; r += NU)
             if (sel[r] >= nb) sel[r] = -1;   // a sequence shorter than k: the place is empty
@@ -986,6 +991,7 @@ __device__ __forceinline__ void load_selection(const Params& p, uint8_t* base, i
 
 // The source of every row of the gathered tiles [t0, t0 + ntl) of `row` into
 // the shared row table.
+template <bool PG>
 __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int row, int t0, int ntl) {
     const int32_t* sel = reinterpret_cast<const int32_t*>(base + SM_SEL);
     int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
@@ -995,7 +1001,8 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
         int32_t e = -1;
         if (gr < kc) {
             const int sidx = gr / p.C, tok = gr - sidx * p.C;
-            if (sel[sidx] >= 0) e = (int32_t)(raw_first(p, row, sel[sidx]) + tok);
+            if (sel[sidx] >= 0)
+                e = (int32_t)((PG ? raw_first(p, row, sel[sidx]) : ((long long)row * p.N + sel[sidx]) * p.C) + tok);
         } else if (gr < p.nrows_g) {
             if (sel[gr - kc] >= 0) e = (int32_t)(-((long long)row * p.N + sel[gr - kc]) - 2);
         }
@@ -1013,6 +1020,7 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
 // are copied by every unfold thread with cp.async.  The copiers hold each
 // phase open until their copies have landed, the TMA bytes are expected on
 // it, and one thread then gives the one expected arrival.
+template <bool PG>
 __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars* bars, int lt, int seq, int row,
                                             int tma_rows, int h, bool children, int gfirst) {
     if (seq < gfirst + NSL) {
@@ -1051,9 +1059,14 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
             if (children) {
                 y = (int)(-e - 2 - (long long)row * p.N1);
                 z = row;
+            } else if (PG && p.table != nullptr) {
+                // pool rows are below 2^31 (checked on the host): 32-bit division
+                z = (int)((uint32_t)e / (uint32_t)p.C);
+                y = (int)e - z * p.C;
             } else {
-                z = (int)(e / p.C);
-                y = (int)(e - (long long)z * p.C);
+                // dense: token chunk * c of the row's raw rows
+                z = row;
+                y = (int)(e - (long long)row * (p.hier ? p.N1 : p.N) * p.C);
             }
             tc::tma_load_3d(ks + r * 128, mk, 0, y, z, &bars->full[sk]);
             tc::tma_load_3d(ks + 16384 + r * 128, mk, 64, y, z, &bars->full[sk]);
@@ -1253,7 +1266,8 @@ __device__ __forceinline__ void merge_row(const Params& p, uint8_t* base, int ro
 }
 
 // ---------------------------------------------------------------- kernel --
-template <int G>
+// PG: the raw cache is paged or the sequences have their own chunk counts
+template <int G, bool PG>
 __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -1384,7 +1398,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         rk.seq0 = 0;
         rk.npre = min(n2, NSL);   // the first value tiles follow the keys without a gap
         rk.vseq0 = n1;
-        run_pipeline<G>(p, cx, rk);
+        run_pipeline<G, PG>(p, cx, rk);
         // the scores are written (global and shared memory): hand them to the
         // unfold warps, which publish them, and go on without waiting
         asm volatile("bar.arrive %0, %1;" ::"n"(BAR_KEYS), "n"(NTHR) : "memory");
@@ -1398,7 +1412,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         rv.gap = 0;
         rv.gfirst = gseq0;
         rv.gwait = min(NSL, 2 * gtiles_total);
-        run_pipeline<G>(p, cx, rv);
+        run_pipeline<G, PG>(p, cx, rv);
         // ------------------------------------ gathered tiles, item by item --
         int gseq = gseq0;
         for (int it = c; it < p.items; it += p.grid) {
@@ -1415,7 +1429,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                 rg.npre = ntl;   // every tile is gathered by the unfold warps
                 rg.slot_b = p.maxs + (p.hier ? rd : it % p.cb);
                 rg.score = (p.hier && rd == 0) ? 1 : 0;
-                run_pipeline<G>(p, cx, rg);
+                run_pipeline<G, PG>(p, cx, rg);
                 gseq += 2 * ntl;
             }
         }
@@ -1478,7 +1492,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                     hier_select_children(p, cx.base, row);
                 } else {
                     if (p.do_topk && p.sel_direct) {
-                        direct_select(p, cx.base, row, j == 0);
+                        direct_select<PG>(p, cx.base, row, j == 0);
                     } else if (p.do_topk) {
                         int n = 0;
                         for (int cc = cf; cc < cf + na; ++cc) {
@@ -1486,12 +1500,12 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                             gists_of(cc, row, a0, a1);
                             n += min(p.K, max(0, a1 - a0));
                         }
-                        merge_select(p, cx.base, row, n, j == 0);
+                        merge_select<PG>(p, cx.base, row, n, j == 0);
                     } else {
                         load_selection(p, cx.base, row);
                     }
                     if (p.hier) hier_children_table(p, cx.base, row);
-                    else build_table(p, cx.base, row, t0, ntl);
+                    else build_table<PG>(p, cx.base, row, t0, ntl);
                 }
                 for (int lt = 0; lt < ntl; ++lt) {
                     // leading rows that are whole runs of consecutive source rows
@@ -1507,7 +1521,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                         const int tile = p.hier ? lt : t0 + lt;
                         tma_rows = max(0, min(TILE, kc - tile * TILE));
                     }
-                    gather_tile(p, cx.base, cx.bars, lt, gseq + 2 * lt, row, tma_rows, h, children, gseq0);
+                    gather_tile<PG>(p, cx.base, cx.bars, lt, gseq + 2 * lt, row, tma_rows, h, children, gseq0);
                 }
                 gseq += 2 * ntl;
                 ++runs;
@@ -1620,17 +1634,17 @@ static bool chunk_runs(int h) { return h >= 8 && h % 8 == 0 && TILE % h == 0; }
 // The CTAs of one launch wait on one another (a row's unfold item waits for
 // the key stretches of the CTAs that met the row), so all of them must be
 // resident at once: the launch is refused on a device that cannot hold `grid`.
-template <int G>
+template <int G, bool PG>
 static cudaError_t launch_g(const Params& p, int grid, cudaStream_t st) {
     static int resident = -1;
     if (resident < 0) {
-        cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel<G, PG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
         int dev = 0, sms = 0, per_sm = 0;
         if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
         if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_decode_kernel<G>, NTHR, SMEM_BYTES)) !=
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_decode_kernel<G, PG>, NTHR, SMEM_BYTES)) !=
             cudaSuccess)
             return e;
         resident = sms * per_sm;
@@ -1646,15 +1660,23 @@ static cudaError_t launch_g(const Params& p, int grid, cudaStream_t st) {
     a[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = a;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fused_decode_kernel<G>, p);
+    return cudaLaunchKernelEx(&cfg, fused_decode_kernel<G, PG>, p);
 }
 
 static cudaError_t launch(const Params& p, int G, int grid, cudaStream_t st) {
+    if (p.table != nullptr || p.nch != nullptr) {
+        switch (G) {
+            case 1: return launch_g<1, true>(p, grid, st);
+            case 2: return launch_g<2, true>(p, grid, st);
+            case 4: return launch_g<4, true>(p, grid, st);
+            default: return launch_g<8, true>(p, grid, st);
+        }
+    }
     switch (G) {
-        case 1: return launch_g<1>(p, grid, st);
-        case 2: return launch_g<2>(p, grid, st);
-        case 4: return launch_g<4>(p, grid, st);
-        default: return launch_g<8>(p, grid, st);
+        case 1: return launch_g<1, false>(p, grid, st);
+        case 2: return launch_g<2, false>(p, grid, st);
+        case 4: return launch_g<4, false>(p, grid, st);
+        default: return launch_g<8, false>(p, grid, st);
     }
 }
 
@@ -1835,11 +1857,12 @@ gsa_status fused_launch(const gsa_decode_desc& d, const FusedPlan& f, const void
     bool ok = map3d(&p.tm_kg, kg, rows, N) && map3d(&p.tm_vg, f.attn_gists ? vg : nullptr, rows, N) &&
               map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
     p.tma_raw = chunk_runs(d.chunk) && f.nbt > 0 ? 1 : 0;
-    // the raw cache as chunks: [rows N][c][d] dense, [n_pages Hkv][c][d] paged
-    const uint64_t nchunk = pg ? (uint64_t)pg->n_pages * (uint64_t)d.n_kv_heads : rows * N;
+    // the raw cache: [rows][N c][d] dense; [n_pages Hkv][c][d] (pages as rows) paged
+    const uint64_t mrows = pg && pg->table ? (uint64_t)pg->n_pages * (uint64_t)d.n_kv_heads : rows;
+    const uint64_t mlen = pg && pg->table ? (uint64_t)d.chunk : N * (uint64_t)d.chunk;
     if (p.tma_raw)
-        ok = ok && map3d(&p.tm_kr, kr, nchunk, (uint64_t)d.chunk, (uint32_t)d.chunk) &&
-             map3d(&p.tm_vr, vr, nchunk, (uint64_t)d.chunk, (uint32_t)d.chunk);
+        ok = ok && map3d(&p.tm_kr, kr, mrows, mlen, (uint32_t)d.chunk) &&
+             map3d(&p.tm_vr, vr, mrows, mlen, (uint32_t)d.chunk);
     if (!ok) return GSA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     fill_common(p, f, d, w);
@@ -1915,8 +1938,8 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
     p.tma_children = chunk_runs(h.group) ? 1 : 0;
     const uint64_t n1 = (uint64_t)d.n_chunks;
     if (p.tma_raw)
-        ok = ok && map3d(&p.tm_kr, kr, rows * n1, (uint64_t)d.chunk, (uint32_t)d.chunk) &&
-             map3d(&p.tm_vr, vr, rows * n1, (uint64_t)d.chunk, (uint32_t)d.chunk);
+        ok = ok && map3d(&p.tm_kr, kr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk) &&
+             map3d(&p.tm_vr, vr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk);
     if (p.tma_children)
         ok = ok && map3d(&p.tm_kc, k_g1, rows, n1, (uint32_t)h.group) && map3d(&p.tm_vc, v_g1, rows, n1, (uint32_t)h.group);
     if (!ok) return GSA_ERR_CUDA;

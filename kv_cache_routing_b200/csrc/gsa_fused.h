@@ -30,7 +30,7 @@ namespace fused {
 struct Params {
     CUtensorMap tm_kg, tm_vg;      // gists  [rows][N][d], box {64, 128, 1}
     CUtensorMap tm_kt, tm_vt;      // tail   [rows][W][d], box {64, 128, 1}
-    CUtensorMap tm_kr, tm_vr;      // raw as chunks [rows N | pages Hkv][c][d], box {64, c, 1} (chunk gathers by TMA)
+    CUtensorMap tm_kr, tm_vr;      // raw [rows][N c][d], or pages [n_pages Hkv][c][d]; box {64, c, 1} (chunk gathers by TMA)
     CUtensorMap tm_kc, tm_vc;      // hierarchy: level-1 gists [rows][N1][d], box {64, group, 1}
     const uint16_t* q;             // [B][Hq][d]
     const uint8_t* kr;             // raw K/V and gist K/V base pointers (gathered tiles)

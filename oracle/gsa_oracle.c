@@ -441,6 +441,75 @@ void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, in
 }
 
 /* ------------------------------------------------------------------------ */
+/* Hierarchy of any depth L >= 2 ([EN-2] "Hierarchical Extension (H-GSA)":   */
+/* gists are compressed again into higher-level gists and the query descends */
+/* coarse to fine; [SL-11] shows the level-2 to level-1 step).  Level 1 has  */
+/* one gist per chunk (n[0] = N1); gist J of level l+1 summarises the level-l */
+/* gists [J*g, (J+1)*g), g = group[l-1], so n[l] = ceil(n[l-1] / g).  Step:   */
+/* every top-level gist is scored and the top k[L-1] taken; at each lower    */
+/* level the candidates are the children of the level above's selection (in  */
+/* parent order, then child order), scored and cut to the top k[l-1]; the     */
+/* raw tokens of the level-1 selection are unfolded.  The context: every     */
+/* top-level gist, every candidate of every lower level, the raw tokens of   */
+/* the selected chunks, the tail (the two-level step above, one level at a   */
+/* time).  kg[l-1], vg[l-1]: the level-l gists [B][Hkv][n[l-1]][d], level 1  */
+/* first; idx[l-1] [B][Hkv][k[l-1]] receives level l's selection.            */
+/* ------------------------------------------------------------------------ */
+void oracle_hier_levels(int B, int Hq, int Hkv, int d, int c, int W, int L, const int* n, const int* group,
+                        const int* k, double scale, int dt, const void* q, const void* const* kg,
+                        const void* const* vg, const void* kraw, const void* vraw, const void* ktail,
+                        const void* vtail, int32_t* const* idx, double* out) {
+    int G = Hq / Hkv;
+    double sc = default_scale(scale, d);
+    int64_t cap = 0;   /* context keys: bounded by all gists of all levels + raw + tail */
+    for (int l = 0; l < L; ++l) cap += n[l];
+    cap += (int64_t)k[0] * c + W + 1;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk) {
+            int64_t row = (int64_t)b * Hkv + hk;
+            key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)cap);
+            int nk = 0;
+            /* top level: every gist is a candidate */
+            int top = L - 1;
+            int nc = n[top];
+            int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nc > 0 ? nc : 1));
+            for (int J = 0; J < nc; ++J) cand[J] = J;
+            for (int l = top; l >= 0; --l) {
+                /* the candidates of level l+1 (index l) are in the context */
+                for (int t = 0; t < nc; ++t) keys[nk++] = (key_ref){kg[l], vg[l], (row * n[l] + cand[t]) * d};
+                double* s = (double*)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
+                for (int t = 0; t < nc; ++t) s[t] = gist_score(Hq, Hkv, d, n[l], dt, q, kg[l], b, hk, cand[t]);
+                int32_t* S = idx[l] + row * k[l];
+                topk_list(nc, s, cand, k[l], S);
+                free(s);
+                if (l == 0) break;
+                /* children of the selection, parent by parent */
+                int32_t* next = (int32_t*)malloc(sizeof(int32_t) * ((size_t)k[l] * group[l - 1] + 1));
+                int m = 0;
+                for (int t = 0; t < k[l]; ++t)
+                    for (int u = 0; u < group[l - 1]; ++u) {
+                        int j = S[t] * group[l - 1] + u;
+                        if (j < n[l - 1]) next[m++] = j;
+                    }
+                free(cand);
+                cand = next;
+                nc = m;
+            }
+            for (int t = 0; t < k[0]; ++t)
+                for (int u = 0; u < c; ++u)
+                    keys[nk++] = (key_ref){kraw, vraw, ((row * n[0] + idx[0][row * k[0] + t]) * c + u) * d};
+            for (int u = 0; u < W; ++u) keys[nk++] = (key_ref){ktail, vtail, (row * W + u) * d};
+            for (int g = 0; g < G; ++g) {
+                int h = hk * G + g;
+                attend(d, dt, sc, q, ((int64_t)b * Hq + h) * d, nk, keys, out + ((int64_t)b * Hq + h) * d, NULL);
+            }
+            free(cand);
+            free(keys);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Gist-causal prefill.  [EN-2] "Interleaved Gist Tokens": the sequence is   */
 /* cut into chunks of c tokens and a gist token follows every chunk; a       */
 /* gist attends only to its own chunk and to earlier gists.  [SL-7]:         */

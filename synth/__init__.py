@@ -113,6 +113,7 @@ S_Q, S_KG, S_VG, S_KR, S_VR, S_KT, S_VT, S_NEEDLE_IDX, S_NEEDLE_NOISE = range(1,
 S_KG2, S_VG2, S_NEEDLE2_NOISE = 10, 11, 12
 S_PQ, S_PK, S_PV = 20, 21, 22
 S_PAGE_K, S_PAGE_V, S_PAGE_ORDER, S_DOC, S_SEQ_LEN = 30, 31, 32, 33, 34
+S_LEVEL_K, S_LEVEL_V, S_LEVEL_NOISE = 40, 50, 60   # + level
 
 
 @dataclass(frozen=True)
@@ -162,6 +163,23 @@ class PrefillShape:
     @property
     def positions(self) -> int:
         return self.n_chunks * (self.chunk + 1)
+
+
+@dataclass(frozen=True)
+class LevelsShape:
+    """A gist hierarchy of depth L = len(groups) + 1: level 1 is l1's gists
+    (one per chunk); groups[i] level-(i+1) gists make one level-(i+2) gist;
+    top_ks[i] is the selection size at level i + 2 (l1.top_k at level 1)."""
+    l1: DecodeShape
+    groups: tuple
+    top_ks: tuple
+
+    @property
+    def counts(self) -> list:
+        n = [self.l1.n_chunks]
+        for g in self.groups:
+            n.append(-(-n[-1] // g))
+        return n
 
 
 @dataclass(frozen=True)
@@ -413,3 +431,54 @@ def paged_inputs(ps: PagedShape, seed: int, seq_chunks=None) -> PagedInputs:
             for t, j in enumerate(range(n, N)):
                 kg[b, hk, j] = round_to(_needle_keys(qw, b, hk, G, 2 * s.needle_alpha, noise[max(m, 1) + t]), dt)
     return PagedInputs(ps, q, kg, vg, kp, vp, table, seq_chunks, kt, vt)
+
+
+@dataclass
+class LevelsInputs:
+    shape: LevelsShape
+    q: np.ndarray
+    k_g: list            # level 1 first, [B, Hkv, n_l, d]
+    v_g: list
+    k_raw: np.ndarray
+    v_raw: np.ndarray
+    k_tail: np.ndarray
+    v_tail: np.ndarray
+    needles: np.ndarray  # [rows, n_needles] level-1 chunk of each needle chain
+
+
+def levels_inputs(h: LevelsShape, seed: int) -> LevelsInputs:
+    """Level-1 tensors as for flat decode, upper-level gists drawn per level.
+    Each needle is a chain: a level-1 chunk and every ancestor of it get a
+    needle key, the chains in distinct top-level gists, so the descent can
+    follow each chain to its chunk."""
+    s = h.l1
+    base = decode_inputs(replace(s, n_needles=0), seed)
+    B, Hkv, d, dt = s.batch, s.n_kv_heads, s.head_dim, s.dtype
+    n = h.counts
+    L = len(n)
+    kg, vg = [base.k_gist], [base.v_gist]
+    for lv in range(1, L):
+        kg.append(normal(seed, S_LEVEL_K + lv, (B, Hkv, n[lv], d), dt))
+        vg.append(normal(seed, S_LEVEL_V + lv, (B, Hkv, n[lv], d), dt))
+    needles = np.zeros((B * Hkv, s.n_needles), np.int64)
+    if s.n_needles:
+        qw = widen(base.q, dt)
+        G = s.group
+        for b in range(B):
+            for hk in range(Hkv):
+                row = b * Hkv + hk
+                tops = _distinct_draws(seed, S_NEEDLE_IDX, row * 1_000_003, s.n_needles, n[-1])
+                for t, top in enumerate(tops):
+                    node = top
+                    for lv in range(L - 1, -1, -1):
+                        noise = normal(seed, S_LEVEL_NOISE + lv, (d,), "f64",
+                                       offset=(row * s.n_needles + t) * d)
+                        kg[lv][b, hk, node] = round_to(_needle_keys(qw, b, hk, G, s.needle_alpha, noise), dt)
+                        if lv == 0:
+                            break
+                        g = h.groups[lv - 1]
+                        lo = node * g
+                        width = min(g, n[lv - 1] - lo)
+                        node = lo + u64(seed, S_NEEDLE_IDX, 5_555_555 + (row * s.n_needles + t) * L + lv) % width
+                    needles[row, t] = node
+    return LevelsInputs(h, base.q, kg, vg, base.k_raw, base.v_raw, base.k_tail, base.v_tail, needles)

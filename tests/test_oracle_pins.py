@@ -605,3 +605,88 @@ def test_paged_sequences_sharing_a_document_see_the_same_raw_keys():
     vp[unused] += 1.0
     _, _, o2 = oracle.decode_paged(x.tensors(), x.k_pages, vp, x.table, 10, SR_ONLY)
     np.testing.assert_array_equal(o2, o0)
+
+
+# ---------------------------------------------------- deeper hierarchy -----
+def _levels(x, h):
+    return oracle.hier_levels(x.q, x.k_g, x.v_g, x.k_raw, x.v_raw, x.k_tail, x.v_tail, h.groups,
+                              (h.l1.top_k,) + tuple(h.top_ks))
+
+
+def test_levels_depth_two_is_the_two_level_hierarchy():
+    """L = 2 is the two-level step (pinned above) bit for bit."""
+    h2, x2 = _hier_small(n1=41, group=4, k2=3, k1=4)
+    hl = synth.LevelsShape(h2.l1, (4,), (3,))
+    idx, out = oracle.hier_levels(x2.q, [x2.k_g1, x2.k_g2], [x2.v_g1, x2.v_g2], x2.k_raw, x2.v_raw, x2.k_tail,
+                                  x2.v_tail, hl.groups, (4, 3))
+    i2, i1, o = oracle.hier_decode(x2.tensors(), 4, 3, 4)
+    np.testing.assert_array_equal(idx[1], i2)
+    np.testing.assert_array_equal(idx[0], i1)
+    np.testing.assert_array_equal(out, o)
+
+
+def test_levels_three_worked_example_by_hand():
+    """Eight chunks, groups of two at both levels (n = 8, 4, 2), k = 1 at
+    every level, q = e0 so a score is the key's first coordinate.  Level 3
+    scores (1, 5) pick gist 1, whose children are level-2 gists 2, 3; these
+    score (2, 3) and 3 wins although gists 0, 1 score 9 (they are not
+    candidates); its children, chunks 6 and 7, score (1, 4): chunk 7.  The
+    context is level-3 {0, 1}, level-2 {2, 3}, level-1 {6, 7}, chunk 7's raw
+    token and the tail, listed here by hand for library SDPA."""
+    d = 4
+    h = synth.LevelsShape(DecodeShape(1, 1, 1, d, 8, 1, 1, 1, "f32"), (2, 2), (1, 1))
+    x = synth.levels_inputs(h, 83)
+    x.q[...] = np.float32([1, 0, 0, 0])
+    for lv, first in ((0, [8, 8, 8, 8, 8, 8, 1, 4]), (1, [9, 9, 2, 3]), (2, [1, 5])):
+        x.k_g[lv][0, 0, :, 0] = np.float32(first)
+    idx, out = _levels(x, h)
+    assert [i[0, 0].tolist() for i in idx] == [[7], [3], [1]]
+    K = np.concatenate([x.k_g[2][0, 0, [0, 1]], x.k_g[1][0, 0, [2, 3]], x.k_g[0][0, 0, [6, 7]], x.k_raw[0, 0, 7],
+                        x.k_tail[0, 0]])
+    V = np.concatenate([x.v_g[2][0, 0, [0, 1]], x.v_g[1][0, 0, [2, 3]], x.v_g[0][0, 0, [6, 7]], x.v_raw[0, 0, 7],
+                        x.v_tail[0, 0]])
+    want = sdpa(x.q[0].astype(np.float64), K.astype(np.float64), V.astype(np.float64), 0.5)
+    np.testing.assert_allclose(out[0], want, rtol=0, atol=1e-12)
+
+
+def test_levels_with_every_upper_group_selected_and_silent_is_flat_decode():
+    """Depth 4, every upper level selects all of its candidates and its gist
+    keys point against the query (logits near -1e4: weight exactly 0 in
+    fp64): the candidates of level 1 are all gists, so the step is the flat
+    decode step (pinned above) over the level-1 gists."""
+    d, n1 = 8, 50
+    h = synth.LevelsShape(DecodeShape(2, 2, 2, d, n1, 3, 5, 2, "f32", n_needles=0), (4, 3, 2), (13, 5, 3))
+    assert h.counts == [50, 13, 5, 3]
+    x = synth.levels_inputs(h, 84)
+    qw = x.q.astype(np.float64)
+    for lv in (1, 2, 3):
+        for b in range(2):
+            for hk in range(2):
+                x.k_g[lv][b, hk, :] = (-1e4 * qw[b, hk] / np.linalg.norm(qw[b, hk])).astype(np.float32)
+    idx, out = _levels(x, h)
+    for lv, cnt in ((1, 13), (2, 5), (3, 3)):
+        assert np.all(idx[lv] == np.arange(cnt))
+    t = dict(q=x.q, k_gist=x.k_g[0], v_gist=x.v_g[0], k_raw=x.k_raw, v_raw=x.v_raw, k_tail=x.k_tail,
+             v_tail=x.v_tail)
+    _, i_flat, o_flat = oracle.decode(t, 5, ALL_GISTS)
+    np.testing.assert_array_equal(idx[0], i_flat)
+    np.testing.assert_allclose(out, o_flat, rtol=0, atol=1e-13)
+
+
+def test_levels_selection_follows_the_tree_and_finds_needle_chains():
+    """Each level's selection lies among the children of the level above's,
+    ascending and distinct; the planted needle chains are found at every
+    level (one needle chunk per selected top-level gist)."""
+    h = synth.LevelsShape(DecodeShape(2, 4, 2, 16, 300, 2, 4, 3, "f32", n_needles=3), (5, 4), (6, 3))
+    x = synth.levels_inputs(h, 85)
+    idx, _ = _levels(x, h)
+    for lv in (0, 1):
+        g = h.groups[lv]
+        for r in range(4):
+            b, hk = divmod(r, 2)
+            sel, par = idx[lv][b, hk], idx[lv + 1][b, hk]
+            assert np.all(np.diff(sel) > 0)
+            assert set((sel // g).tolist()) <= set(par.tolist())
+    for r in range(4):
+        b, hk = divmod(r, 2)
+        assert set(x.needles[r].tolist()) <= set(idx[0][b, hk].tolist())

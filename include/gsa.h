@@ -120,6 +120,22 @@ typedef struct {
     int32_t n_l2, group, top_k2;
 } gsa_hier_desc;
 
+/* A gist hierarchy of any depth L = levels, 2 <= L <= GSA_MAX_LEVELS ([EN-2]
+ * "Hierarchical Extension (H-GSA)": gists compressed again, coarse-to-fine
+ * descent; [SL-11]).  l1 describes the level-1 gists (one per chunk), raw
+ * chunks and tail as for the two-level hierarchy (l1.top_k = k1, l1.mode
+ * GSA_ALL_GISTS).  For i = 0 .. L-2: group[i] level-(i+1) gists make one
+ * level-(i+2) gist, so level i+2 has n = ceil(n_{i+1} / group[i]) gists,
+ * and top_k[i] is the selection size at level i+2.  Each level's top_k may
+ * not exceed the fewest candidates the level above can yield.              */
+#define GSA_MAX_LEVELS 8
+typedef struct {
+    gsa_decode_desc l1;
+    int32_t levels;
+    int32_t group[GSA_MAX_LEVELS - 1];
+    int32_t top_k[GSA_MAX_LEVELS - 1];
+} gsa_levels_desc;
+
 /* Gist-causal prefill over P = N*(c+1) interleaved positions (a gist after
  * every chunk of c raw tokens). */
 typedef struct {
@@ -133,6 +149,8 @@ typedef struct {
 size_t gsa_decode_workspace_size(const gsa_decode_desc* desc);
 /* Bytes of workspace gsa_hier_decode needs (0 if invalid). */
 size_t gsa_hier_workspace_size(const gsa_hier_desc* desc);
+/* Bytes of workspace gsa_levels_decode needs (0 if invalid). */
+size_t gsa_levels_workspace_size(const gsa_levels_desc* desc);
 
 /* Routing scores ([EN-2] "Gist as Routing Signals"; [DE-M]
  * "Relevanz-Scoring"): the decoding query is scored against every gist key
@@ -233,6 +251,22 @@ gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void*
                            const void* v_tail, int32_t* idx2_out, int32_t* idx1_out, void* out,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Hierarchical decode of any depth: every level-L gist is scored and the
+ * top k_L taken; at each lower level the candidates are the children of the
+ * level above's selection, scored and cut to that level's top-k; the raw
+ * tokens of the level-1 selection are unfolded.  Attention over every
+ * level-L gist, every candidate of every lower level, the raw tokens of the
+ * k1 chunks and the tail (for L = 2: gsa_hier_decode's step).
+ *   k_gists, v_gists: HOST arrays of L device pointers, level 1 first, level
+ *   l's gists [B][Hkv][n_l][d]; raw and tail as for gsa_decode_step;
+ *   idx_out: NULL or a HOST array of L nullable device pointers, level l's
+ *   selection [B][Hkv][k_l] (ascending).  Runs as L + 1 launches of the
+ *   CUDA-core passes (bf16 or fp32, d = 64 or 128).                        */
+gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const void* const* k_gists,
+                             const void* const* v_gists, const void* k_raw, const void* v_raw,
+                             const void* k_tail, const void* v_tail, int32_t* const* idx_out,
+                             void* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Gist-causal prefill ([EN-2] "Interleaved Gist Tokens"; [SL-7] gist causal
  * mask g1 -> x1,x2; g2 -> g1,x3,x4; g3 -> g1,g2,x5,x6,g3; [SL-9]).  Position p
  * is in chunk p / (c+1) and is a gist iff p % (c+1) == c.  Query p attends key
@@ -279,6 +313,8 @@ int gsa_decode_launch_count(const gsa_decode_desc* desc);
 /* The same for one gsa_hier_decode call: 1 on the tensor-core path, 3 on the
  * CUDA-core passes; -1 if the descriptor is invalid.  Host only. */
 int gsa_hier_launch_count(const gsa_hier_desc* desc);
+/* The same for one gsa_levels_decode call (L + 1), -1 if invalid. */
+int gsa_levels_launch_count(const gsa_levels_desc* desc);
 
 /* Reads (synchronously, on `stream`) the workspace error word: 0, or an OR of
  * GSA_WS_ERR_* flags; returns GSA_ERR_TIMEOUT if a bounded wait expired,

@@ -25,7 +25,8 @@ EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", 
            "gsa_unfold_attn", "gsa_decode_step", "gsa_hier_decode", "gsa_gist_prefill",
            "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count",
            "gsa_hier_launch_count", "gsa_device_error", "gsa_set_wait_limit_ns", "gsa_topp",
-           "gsa_decode_step_topp", "gsa_decode_step_paged")
+           "gsa_decode_step_topp", "gsa_decode_step_paged",
+           "gsa_levels_workspace_size", "gsa_levels_decode", "gsa_levels_launch_count")
 
 
 class GsaError(RuntimeError):
@@ -44,6 +45,14 @@ class DecodeDesc(ctypes.Structure):
 class HierDesc(ctypes.Structure):
     _fields_ = [("l1", DecodeDesc), ("n_l2", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("top_k2", ctypes.c_int32)]
+
+
+GSA_MAX_LEVELS = 8
+
+
+class LevelsDesc(ctypes.Structure):
+    _fields_ = [("l1", DecodeDesc), ("levels", ctypes.c_int32),
+                ("group", ctypes.c_int32 * (GSA_MAX_LEVELS - 1)), ("top_k", ctypes.c_int32 * (GSA_MAX_LEVELS - 1))]
 
 
 class PrefillDesc(ctypes.Structure):
@@ -77,6 +86,9 @@ def _signatures():
         "gsa_set_wait_limit_ns": (st, [ctypes.c_uint64]),
         "gsa_status_string": (ctypes.c_char_p, [st]),
         "gsa_decode_launch_count": (ctypes.c_int, [pd]),
+        "gsa_levels_workspace_size": (sz, [ctypes.POINTER(LevelsDesc)]),
+        "gsa_levels_decode": (st, [ctypes.POINTER(LevelsDesc)] + [vp] * 10 + [sz, vp]),
+        "gsa_levels_launch_count": (ctypes.c_int, [ctypes.POINTER(LevelsDesc)]),
         "gsa_hier_launch_count": (ctypes.c_int, [ph]),
     }
 
@@ -147,6 +159,15 @@ def decode_desc(batch, n_q_heads, n_kv_heads, head_dim, n_chunks, chunk, top_k, 
 
 def hier_desc(l1: DecodeDesc, n_l2, group, top_k2) -> HierDesc:
     return HierDesc(l1, n_l2, group, top_k2)
+
+
+def levels_desc(l1: DecodeDesc, groups, top_ks) -> LevelsDesc:
+    """groups[i]: level-(i+1) gists per level-(i+2) gist; top_ks[i]: the
+    selection size at level i + 2 (level 1: l1.top_k)."""
+    assert len(groups) == len(top_ks) and 1 <= len(groups) < GSA_MAX_LEVELS
+    g = (ctypes.c_int32 * (GSA_MAX_LEVELS - 1))(*groups)
+    k = (ctypes.c_int32 * (GSA_MAX_LEVELS - 1))(*top_ks)
+    return LevelsDesc(l1, len(groups) + 1, g, k)
 
 
 def prefill_desc(batch, n_q_heads, n_kv_heads, head_dim, n_chunks, chunk, dtype=GSA_BF16,
@@ -271,3 +292,27 @@ def gsa_decode_step_paged(desc, q, k_gist, v_gist, k_pages, v_pages, n_pages, bl
                                        _ptr(v_pages), int(n_pages), _ptr(block_table), _ptr(seq_chunks),
                                        _ptr(k_tail), _ptr(v_tail), _ptr(idx_out), _ptr(scores_out), _ptr(out),
                                        _ptr(ws), nb, _stream(stream)), "gsa_decode_step_paged")
+
+
+def gsa_levels_workspace_size(desc: LevelsDesc) -> int:
+    return int(lib().gsa_levels_workspace_size(ctypes.byref(desc)))
+
+
+def gsa_levels_launch_count(desc: LevelsDesc) -> int:
+    n = lib().gsa_levels_launch_count(ctypes.byref(desc))
+    if n < 0:
+        raise GsaError(1, "gsa_levels_launch_count")
+    return int(n)
+
+
+def gsa_levels_decode(desc, q, k_gists, v_gists, k_raw, v_raw, k_tail, v_tail, idx_out, out, ws, stream=None,
+                      ws_bytes=None):
+    """Hierarchy of any depth.  k_gists / v_gists: sequences of the L levels'
+    gist tensors, level 1 first; idx_out: None or a sequence of L nullable
+    selection tensors."""
+    L = len(k_gists)
+    arr = lambda xs: (ctypes.c_void_p * L)(*[_ptr(x) for x in xs])
+    nb = _nbytes(ws) if ws_bytes is None else ws_bytes
+    _check(lib().gsa_levels_decode(ctypes.byref(desc), _ptr(q), arr(k_gists), arr(v_gists), _ptr(k_raw), _ptr(v_raw),
+                                   _ptr(k_tail), _ptr(v_tail), None if idx_out is None else arr(idx_out), _ptr(out),
+                                   _ptr(ws), nb, _stream(stream)), "gsa_levels_decode")

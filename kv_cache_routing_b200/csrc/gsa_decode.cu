@@ -1150,6 +1150,104 @@ gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, c
                            need, stream);
 }
 
+// Hierarchy of any depth ([EN-2] "Hierarchical Extension (H-GSA)"): the
+// top-level gist pass, one gathered gist pass per lower level (the children
+// of the selection above: scores, attention, top-k), then the unfold pass
+// over the raw tokens of the level-1 selection and the tail, merging the
+// partials of every pass.
+size_t gsa_levels_workspace_size(const gsa_levels_desc* desc) {
+    if (validate_levels(desc) != GSA_OK) return 0;
+    return make_levels_plan(*desc).total;
+}
+
+gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const void* const* k_gists,
+                             const void* const* v_gists, const void* k_raw, const void* v_raw, const void* k_tail,
+                             const void* v_tail, int32_t* const* idx_out, void* out, void* ws, size_t ws_bytes,
+                             void* stream) {
+    gsa_status st = validate_levels(desc);
+    if (st != GSA_OK) return st;
+    const gsa_decode_desc& d = desc->l1;
+    const int L = desc->levels;
+    if (!q || !k_gists || !v_gists || !out) return GSA_ERR_ARG;
+    if (d.top_k > 0 && (!k_raw || !v_raw)) return GSA_ERR_ARG;
+    if (d.tail_len > 0 && (!k_tail || !v_tail)) return GSA_ERR_ARG;
+    for (int lv = 0; lv < L; ++lv) {
+        if (!k_gists[lv] || !v_gists[lv]) return GSA_ERR_ARG;
+        if (!aligned16(k_gists[lv]) || !aligned16(v_gists[lv])) return GSA_ERR_ALIGN;
+        if (idx_out && !aligned16(idx_out[lv])) return GSA_ERR_ALIGN;
+    }
+    const void* all[] = {q, k_raw, v_raw, k_tail, v_tail, out};
+    for (const void* x : all)
+        if (!aligned16(x)) return GSA_ERR_ALIGN;
+    const LevelsPlan lp = make_levels_plan(*desc);
+    if (!ws || ws_bytes < lp.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSA_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    const int G = d.n_q_heads / d.n_kv_heads;
+    int32_t* idx[GSA_MAX_LEVELS];
+    for (int lv = 0; lv < L; ++lv)
+        idx[lv] = (idx_out && idx_out[lv]) ? idx_out[lv] : reinterpret_cast<int32_t*>(w + lp.off_idx[lv]);
+    Kernels kern = pick_kernels(d.dtype, d.head_dim, G);
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(w + kWsCntOffset);
+    float* partA = reinterpret_cast<float*>(w + lp.off_partA);
+    float* mlA = reinterpret_cast<float*>(w + lp.off_mlA);
+
+    // pass 0: every top-level gist
+    const int top = L - 1;
+    PassParams p = make_params(lp.top, lp.topdesc, q, k_gists[top], v_gists[top], nullptr, nullptr, nullptr,
+                               nullptr, ws);
+    p.cntA = cnt;
+    p.scores = reinterpret_cast<float*>(w + lp.off_scores[top]);
+    p.cand_key = reinterpret_cast<uint32_t*>(w + lp.off_cand_key);
+    p.cand_idx = reinterpret_cast<int32_t*>(w + lp.off_cand_idx);
+    p.idx_out = idx[top];
+    p.partA = partA;
+    p.mlA = mlA;
+    p.slot_base = lp.slot_base[top];
+    p.slot_stride = lp.slots;
+    p.do_score = p.do_attn = p.do_topk = 1;
+    if (kern.gist(p, strm) != cudaSuccess) return GSA_ERR_CUDA;
+
+    // passes 1 .. L-1: the children of the selection one level up
+    for (int lv = top - 1; lv >= 0; --lv) {
+        PassParams c = p;
+        c.N = lp.n[lv];
+        c.K = level_k(*desc, lv);
+        c.kg = static_cast<const uint8_t*>(k_gists[lv]);
+        c.vg = static_cast<const uint8_t*>(v_gists[lv]);
+        c.Nv = lp.Nv[lv];
+        c.parent_idx = idx[lv + 1];
+        c.parent_k = level_k(*desc, lv + 1);
+        c.group = desc->group[lv];
+        c.SA = lp.SA[lv];
+        c.tprA = lp.tpr[lv];
+        c.scores = reinterpret_cast<float*>(w + lp.off_scores[lv]);
+        c.idx_out = idx[lv];
+        c.local_topk = 0;
+        c.slot_base = lp.slot_base[lv];
+        if (kern.gist(c, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    }
+
+    // raw tokens of the level-1 selection + tail, final merge of every partial
+    PassParams u = make_params(lp.l1, d, q, k_gists[0], v_gists[0], k_raw, v_raw, k_tail, v_tail, ws);
+    u.cntB = cnt + lp.l1.rows;
+    u.partA = partA;
+    u.mlA = mlA;
+    u.partB = reinterpret_cast<float*>(w + lp.off_partB);
+    u.mlB = reinterpret_cast<float*>(w + lp.off_mlB);
+    u.idx_in = idx[0];
+    u.out = static_cast<uint8_t*>(out);
+    u.merge_a = 1;
+    u.slot_stride = lp.slots;
+    if (kern.unfold(u, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    return GSA_OK;
+}
+
+int gsa_levels_launch_count(const gsa_levels_desc* desc) {
+    if (validate_levels(desc) != GSA_OK) return -1;
+    return desc->levels + 1;
+}
+
 int gsa_hier_launch_count(const gsa_hier_desc* desc) {
     if (validate_hier(desc) != GSA_OK) return -1;
     return fused_hier_supported(*desc) ? 1 : 3;

@@ -189,3 +189,99 @@ inline HierPlan make_hier_plan(const gsa_hier_desc& h) {
 }
 
 }  // namespace gsa
+
+namespace gsa {
+
+// Gists per level of a hierarchy of any depth: n[0] = N, n[i+1] = ceil(n[i] / group[i]).
+inline void level_counts(const gsa_levels_desc& h, int* n) {
+    n[0] = h.l1.n_chunks;
+    for (int i = 0; i + 1 < h.levels; ++i) n[i + 1] = (n[i] + h.group[i] - 1) / h.group[i];
+}
+// Selection size at level lv + 1 (lv = 0: level 1).
+inline int level_k(const gsa_levels_desc& h, int lv) { return lv == 0 ? h.l1.top_k : h.top_k[lv - 1]; }
+
+inline gsa_status validate_levels(const gsa_levels_desc* h) {
+    if (!h) return GSA_ERR_ARG;
+    gsa_status st = validate_decode(&h->l1);
+    if (st != GSA_OK) return st;
+    if (h->l1.mode != GSA_ALL_GISTS || h->l1.n_chunks < 1) return GSA_ERR_ARG;
+    if (h->levels < 2 || h->levels > GSA_MAX_LEVELS) return GSA_ERR_ARG;
+    for (int i = 0; i + 1 < h->levels; ++i)
+        if (h->group[i] < 1 || h->top_k[i] < 1) return GSA_ERR_ARG;
+    int n[GSA_MAX_LEVELS];
+    level_counts(*h, n);
+    const int L = h->levels;
+    if (level_k(*h, L - 1) > n[L - 1]) return GSA_ERR_ARG;
+    for (int lv = L - 2; lv >= 0; --lv) {
+        // fewest candidates: k full groups of the level above but the shortest (its last) one
+        const int g = h->group[lv], kp = level_k(*h, lv + 1);
+        const int64_t last = n[lv] - (int64_t)(n[lv + 1] - 1) * g;
+        if ((int64_t)kp * g > INT32_MAX / 2) return GSA_ERR_SHAPE;
+        if (level_k(*h, lv) > (int64_t)(kp - 1) * g + last) return GSA_ERR_ARG;
+    }
+    return GSA_OK;
+}
+
+// Passes: the top level flat (pass 0), each lower level over the children
+// of the selection above (passes 1 .. L-1, level L-1 down to 1), then the
+// unfold pass of the level-1 descriptor.
+struct LevelsPlan {
+    int L, n[GSA_MAX_LEVELS];
+    gsa_decode_desc topdesc;       // the top level as a flat descriptor
+    DecodePlan top, l1;            // pass 0; the unfold pass
+    int Nv[GSA_MAX_LEVELS], tpr[GSA_MAX_LEVELS], SA[GSA_MAX_LEVELS];   // by level index (0 = level 1)
+    int slot_base[GSA_MAX_LEVELS], slots;
+    size_t off_scores[GSA_MAX_LEVELS], off_idx[GSA_MAX_LEVELS];
+    size_t off_cand_key, off_cand_idx, off_partA, off_mlA, off_partB, off_mlB, total;
+};
+
+inline LevelsPlan make_levels_plan(const gsa_levels_desc& h) {
+    LevelsPlan p{};
+    const gsa_decode_desc& d = h.l1;
+    p.L = h.levels;
+    level_counts(h, p.n);
+    const int top = p.L - 1;
+    p.topdesc = d;
+    p.topdesc.n_chunks = p.n[top];
+    p.topdesc.top_k = level_k(h, top);
+    p.top = make_decode_plan(p.topdesc);
+    p.l1 = make_decode_plan(d);
+    const int rows = p.l1.rows, tile = p.l1.tile;
+    p.Nv[top] = p.n[top];
+    p.tpr[top] = p.top.tprA;
+    p.SA[top] = p.top.SA;
+    p.slot_base[top] = 0;
+    p.slots = p.SA[top];
+    for (int lv = top - 1; lv >= 0; --lv) {
+        p.Nv[lv] = level_k(h, lv + 1) * h.group[lv];
+        p.tpr[lv] = (p.Nv[lv] + tile - 1) / tile;
+        p.SA[lv] = std::min({p.tpr[lv], std::max(1, kTargetGistCtas / rows), kMaxSplits});
+        p.slot_base[lv] = p.slots;
+        p.slots += p.SA[lv];
+    }
+    const size_t R = (size_t)rows;
+    const int G = p.l1.G, D = d.head_dim;
+    size_t o = round256(kWsCntOffset + 2 * R * 4);
+    for (int lv = 0; lv < p.L; ++lv) {
+        p.off_scores[lv] = o;
+        o = round256(o + R * (size_t)p.Nv[lv] * 4);
+        p.off_idx[lv] = o;
+        o = round256(o + R * (size_t)level_k(h, lv) * 4);
+    }
+    p.off_cand_key = o;
+    o = round256(o + R * (size_t)p.top.candA * 4);
+    p.off_cand_idx = o;
+    o = round256(o + R * (size_t)p.top.candA * 4);
+    p.off_partA = o;
+    o = round256(o + R * (size_t)p.slots * G * D * 4);
+    p.off_mlA = o;
+    o = round256(o + R * (size_t)p.slots * G * 2 * 4);
+    p.off_partB = o;
+    o = round256(o + R * (size_t)p.l1.SB * G * D * 4);
+    p.off_mlB = o;
+    o = round256(o + R * (size_t)p.l1.SB * G * 2 * 4);
+    p.total = o;
+    return p;
+}
+
+}  // namespace gsa

@@ -25,7 +25,8 @@ cores on a bounded sample of the same workload.
 Other workloads: --workload NAME for every decode shape of synth.WORKLOADS
 (the sweeps), llama8b_paged (the same step over a shared page pool of
 documents through gsa_decode_step_paged), hier_1m (two-level descent, steps/s
-against the HBM roofline) and gist_prefill (the gist-causal prefill,
+against the HBM roofline), hier3_1m (three-level descent through
+gsa_levels_decode) and gist_prefill (the gist-causal prefill,
 algorithmic TFLOP/s against the bf16 tensor roofline).
 """
 from __future__ import annotations
@@ -145,6 +146,17 @@ def hier_config(h, workload: str, world: int, L: int, nbytes: int, l2: int) -> d
                   f"per rotation (L2 {l2 / 1e6:.0f} MB)"}
 
 
+def levels_config(h, workload: str, world: int, L: int, nbytes: int, l2: int) -> dict:
+    s = h.l1
+    return {"workload": workload, "batch": s.batch, "n_q_heads": s.n_q_heads, "n_kv_heads": s.n_kv_heads,
+            "head_dim": s.head_dim, "raw_tokens": s.n_chunks * s.chunk, "chunk": s.chunk,
+            "levels": len(h.counts), "gists_per_level": h.counts, "groups": list(h.groups),
+            "top_k_per_level": [s.top_k] + list(h.top_ks), "tail": s.tail_len,
+            "parallelism": f"replicas x{world}",
+            "l2": f"rotating {L} replicas (own top-level gists and query), {L * nbytes / 1e6:.0f} MB touched "
+                  f"per rotation (L2 {l2 / 1e6:.0f} MB)"}
+
+
 def prefill_config(p, workload: str, world: int, l2: int) -> dict:
     qkv = (p.batch * p.n_q_heads + 2 * p.batch * p.n_kv_heads) * p.positions * p.head_dim * 2
     return {"workload": workload, "batch": p.batch, "n_q_heads": p.n_q_heads, "n_kv_heads": p.n_kv_heads,
@@ -216,6 +228,21 @@ def hier_bytes(h) -> int:
     s = h.l1
     row = s.head_dim * (4 if s.dtype == "f32" else 2)
     per_kv = 2 * h.n_l2 * row + 2 * h.top_k2 * h.group * row + 2 * s.top_k * s.chunk * row + 2 * s.tail_len * row
+    return s.rows * per_kv + 2 * s.batch * s.n_q_heads * row
+
+
+def levels_bytes(h) -> int:
+    """Bytes a descent of any depth must move: q, every top-level gist K and
+    V, the K and V of every lower level's candidates, the raw K/V of the k1
+    chunks, the tail K/V, out."""
+    s = h.l1
+    row = s.head_dim * (4 if s.dtype == "f32" else 2)
+    n = h.counts
+    ks = (s.top_k,) + tuple(h.top_ks)
+    per_kv = 2 * n[-1] * row
+    for lv in range(len(n) - 1):
+        per_kv += 2 * min(ks[lv + 1] * h.groups[lv], n[lv]) * row
+    per_kv += 2 * s.top_k * s.chunk * row + 2 * s.tail_len * row
     return s.rows * per_kv + 2 * s.batch * s.n_q_heads * row
 
 
@@ -698,6 +725,99 @@ def run_hier(args, world, rank, local):
     del g
 
 
+def run_levels(args, world, rank, local):
+    """The descent of any depth through gsa_levels_decode, timed like the
+    two-level one: K steps as one graph rotating over L replicas (own
+    top-level gists and query each)."""
+    import torch
+
+    import kv_cache_routing_b200 as gsa
+
+    h = synth.WORKLOADS[args.workload]
+    s = h.l1
+    torch.cuda.set_device(local)
+    l2 = l2_bytes(local)
+    nbytes = levels_bytes(h)
+    L = replicas_for(nbytes, l2, args.replicas)
+    seed = synth.seed_for(args.workload) + 17 * rank
+    x = synth.levels_inputs(h, seed)
+    kg = [_dev(a) for a in x.k_g]
+    vg = [_dev(a) for a in x.v_g]
+    raw = [_dev(a) for a in (x.k_raw, x.v_raw, x.k_tail, x.v_tail)]
+    q0 = _dev(x.q)
+    reps = []
+    for r in range(L):
+        q = q0 if r == 0 else _dev(synth.normal(seed + 1000 * r, synth.S_Q, x.q.shape, s.dtype))
+        top_k, top_v = (kg[-1], vg[-1]) if r == 0 else (kg[-1].clone(), vg[-1].clone())
+        reps.append((q, kg[:-1] + [top_k], vg[:-1] + [top_v]))
+    desc = gsa.levels_desc(_desc_of(s), h.groups, h.top_ks)
+    ws = torch.zeros(max(256, gsa.gsa_levels_workspace_size(desc)), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((s.batch, s.n_q_heads, s.head_dim), dtype=_tdtype(s.dtype), device="cuda") for _ in range(L)]
+    stream = torch.cuda.Stream()
+
+    def step(i, st):
+        q, kl, vl = reps[i % L]
+        gsa.gsa_levels_decode(desc, q, kl, vl, *raw, None, outs[i % L], ws, stream=st)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(args.steps):
+                step(i, stream)
+        g.replay()
+    stream.synchronize()
+    with ClockSampler(local) as clk:
+        barrier(world)
+        reps_ms = timed_replays(g.replay, stream)
+        barrier(world)
+    ms_max = max_over_ranks(statistics.median(reps_ms), world)
+    assert gsa.gsa_workspace_error(ws, stream=stream) == 0
+    per_ms = ms_max / args.steps
+    gbs = nbytes / (per_ms / 1e3) / 1e9
+    qh = torch.empty_like(q0, device="cpu").pin_memory()
+    qh.copy_(q0.cpu())
+    oh = torch.empty_like(outs[0], device="cpu").pin_memory()
+
+    def e2e_run():
+        for i in range(args.steps):
+            reps[i % L][0].copy_(qh, non_blocking=True)
+            step(i, stream)
+            oh.copy_(outs[i % L], non_blocking=True)
+            stream.synchronize()
+
+    barrier(world)
+    e2e_ms = max_over_ranks(statistics.median(timed_replays(e2e_run, stream, 3)), world)
+    peak, peak_kind = peaks()
+    launches = gsa.gsa_levels_launch_count(desc)
+    line = {
+        "metric": HIER_METRIC, "value": round(whole_job_rate(args.steps, world, ms_max), 2), "unit": "steps/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+        "config": levels_config(h, args.workload, world, L, nbytes, l2),
+        "timing": {"replays": len(reps_ms), "statistic": "median over replays of the K-step graph",
+                   "ms_per_step_min": round(min(reps_ms) / args.steps, 5),
+                   "ms_per_step_max": round(max(reps_ms) / args.steps, 5)},
+        "algorithmic_bytes_per_step": nbytes,
+        "roofline": {"bound": "hbm", "kernel": f"gsa_levels_decode (whole step, {launches} launches)",
+                     "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                     "peak_kind": peak_kind, "traffic": None, "traffic_source": "none"},
+        "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
+                "h2d_bytes_per_step": qh.numel() * qh.element_size(),
+                "d2h_bytes_per_step": oh.numel() * oh.element_size()},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_levels(h, x, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+
+
 # ------------------------------------------------------------ CPU oracle ----
 def _oracle_step(s, x, ps=None):
     """One whole decode step of the oracle on the workload's inputs."""
@@ -749,6 +869,31 @@ def cpu_baseline_hier(h, x, budget_s: float):
                       f"most {s.rows} OpenMP threads), fp64, {el:.1f} s"}
 
 
+def _oracle_levels(h, x):
+    import oracle
+    ks = (h.l1.top_k,) + tuple(h.top_ks)
+    return lambda: oracle.hier_levels(x.q, x.k_g, x.v_g, x.k_raw, x.v_raw, x.k_tail, x.v_tail, h.groups, ks)
+
+
+def cpu_baseline_levels(h, x, budget_s: float):
+    """The fp64 oracle of the descent of any depth, as it stands, on the host
+    cores: whole steps until the time budget is spent (at least one)."""
+    run = _oracle_levels(h, x)
+    s = h.l1
+    run()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 1000:
+            break
+    cores = min(s.rows, int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
+    return {"value": round(n / el, 4), "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} full {len(h.counts)}-level steps of the workload ({s.rows} (batch, kv-head) rows each, "
+                      f"so at most {s.rows} OpenMP threads), fp64, {el:.1f} s"}
+
+
 def run_reference(args, world, rank):
     """The reference arm: the fp64 oracle as it stands, on the host cores, on
     the same workload, metric, unit and config as the GPU arm; each step is
@@ -781,6 +926,15 @@ def run_reference(args, world, rank):
         nb = hier_bytes(w)
         config = hier_config(w, args.workload, world, replicas_for(nb, l2, args.replicas), nb, l2)
         sample = f"one full hierarchical step per step ({w.l1.rows} rows, OpenMP over rows), fp64"
+        cores = min(cores, w.l1.rows)
+        rate = lambda sec: 1.0 / sec
+    elif isinstance(w, synth.LevelsShape):
+        x = synth.levels_inputs(w, seed)
+        run = _oracle_levels(w, x)
+        metric, unit, dtype = HIER_METRIC, "steps/s", "f64"
+        nb = levels_bytes(w)
+        config = levels_config(w, args.workload, world, replicas_for(nb, l2, args.replicas), nb, l2)
+        sample = f"one full {len(w.counts)}-level step per step ({w.l1.rows} rows, OpenMP over rows), fp64"
         cores = min(cores, w.l1.rows)
         rate = lambda sec: 1.0 / sec
     elif isinstance(w, synth.PagedShape):
@@ -846,6 +1000,8 @@ def main():
             run_prefill(args, world, rank, local)
         elif isinstance(w, synth.HierShape):
             run_hier(args, world, rank, local)
+        elif isinstance(w, synth.LevelsShape):
+            run_levels(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

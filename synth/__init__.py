@@ -211,6 +211,9 @@ WORKLOADS = {
     "hier_1m": HierShape(DecodeShape(1, 32, 8, 128, 65536, 16, 8, 128, "bf16", ALL_GISTS, n_needles=8),
                          n_l2=4096, group=16, top_k2=8),
     "gist_prefill": PrefillShape(2, 32, 8, 128, 1024, 16, "bf16"),
+    # three levels over 1M raw tokens: 65536 -> 4096 -> 256 gists, k = 8 at every level
+    "hier3_1m": LevelsShape(DecodeShape(1, 32, 8, 128, 65536, 16, 8, 128, "bf16", ALL_GISTS, n_needles=8),
+                            groups=(16, 16), top_ks=(8, 8)),
     # the Llama-shaped step over a shared page pool of 32..160-chunk documents
     # (KV-cache reuse), sequences of 1536..2048 chunks
     "llama8b_paged": PagedShape(DecodeShape(8, 32, 8, 128, 2048, 16, 16, 64, "bf16", ALL_GISTS, n_needles=16),
@@ -220,7 +223,8 @@ WORKLOADS = {
 # workload -> index in the published config list (seeds 20260422 + 100*cfg + rep)
 CONFIG_INDEX = {"tiny_f32": 1, "llama8b_decode": 2, "sweep_c8_all": 3, "sweep_c16_all": 3,
                 "sweep_c32_all": 3, "sweep_c8_pairs": 3, "sweep_c16_pairs": 3,
-                "sweep_c32_pairs": 3, "hier_1m": 4, "gist_prefill": 5, "llama8b_paged": 6}
+                "sweep_c32_pairs": 3, "hier_1m": 4, "gist_prefill": 5, "llama8b_paged": 6,
+                "hier3_1m": 7}
 
 
 def seed_for(workload: str, rep: int = 0) -> int:

@@ -50,7 +50,8 @@ def _load():
         "oracle_unfold_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
         "oracle_decode_paged": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12,
         "oracle_hier_decode": [i, i, i, i, i, i, i, i, i, i, i, d, i] + [vp] * 12 + [i],
-        "oracle_hier_levels": [i, i, i, i, i, i, i, vp, vp, vp, d, i, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "oracle_hier_levels": [i, i, i, i, i, i, i, vp, vp, vp, d, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i],
+        "oracle_suffix_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
         "oracle_gist_mask": [i64, i64, i],
         "oracle_prefill_pair_count": [i, i],
         "oracle_prefill_rows": [i, i, i, i, i, i, d, i, vp, vp, vp, i64, vp, vp],
@@ -212,11 +213,26 @@ def hier_decode(t: dict, group: int, top_k2: int, top_k1: int, scale: float = 0.
     return idx2, idx1, out
 
 
-def hier_levels(q, k_g, v_g, k_raw, v_raw, k_tail, v_tail, groups, top_ks, scale: float = 0.0):
+def suffix_attn(q, k_gist, v_gist, k_raw, v_raw, k_suf, v_suf, top_k: int, mode: int = ALL_GISTS,
+                scale: float = 0.0):
+    """Stage-2 forward: q [B,S,Hq,d] (position-major), k_suf / v_suf
+    [B,Hkv,S,d].  Returns (scores [B,Hkv,S,N], idx [B,Hkv,S,k], out [B,S,Hq,d])."""
+    B, S, Hq, d = q.shape
+    _, Hkv, N, c, _ = k_raw.shape
+    sc = np.empty((B, Hkv, S, N), np.float64)
+    idx = np.empty((B, Hkv, S, top_k), np.int32)
+    out = np.empty((B, S, Hq, d), np.float64)
+    _load().oracle_suffix_attn(B, Hq, Hkv, d, N, c, top_k, S, mode, scale, _dtcode(q), _p(q), _p(k_gist),
+                               _p(v_gist), _p(k_raw), _p(v_raw), _p(k_suf), _p(v_suf), _p(sc), _p(idx), _p(out))
+    return sc, idx, out
+
+
+def hier_levels(q, k_g, v_g, k_raw, v_raw, k_tail, v_tail, groups, top_ks, scale: float = 0.0, given=None):
     """Hierarchy of any depth: k_g / v_g are lists of the gist tensors of
     levels 1..L ([B,Hkv,n_l,d], level 1 one gist per chunk), groups[l-1] the
     level-l gists per level-(l+1) gist (L-1 values), top_ks[l-1] the
-    selection size at level l (L values).  Returns ([idx_l], out)."""
+    selection size at level l (L values).  Returns ([idx_l], out).  given: a
+    list of L selections to evaluate the step for instead of selecting."""
     B, Hq, d = q.shape
     Hkv = k_raw.shape[1]
     c = k_raw.shape[3]
@@ -226,14 +242,17 @@ def hier_levels(q, k_g, v_g, k_raw, v_raw, k_tail, v_tail, groups, top_ks, scale
     n = np.array([g.shape[2] for g in k_g], np.int32)
     grp = np.array(list(groups) + [0], np.int32)
     kk = np.array(top_ks, np.int32)
-    idx = [np.empty((B, Hkv, int(t)), np.int32) for t in top_ks]
+    if given is None:
+        idx = [np.empty((B, Hkv, int(t)), np.int32) for t in top_ks]
+    else:
+        idx = [np.ascontiguousarray(g, np.int32).copy() for g in given]
     out = np.empty((B, Hq, d), np.float64)
     arr = lambda xs: (ctypes.c_void_p * len(xs))(*[x.ctypes.data for x in xs])
     for x in list(k_g) + list(v_g):
         assert x.flags["C_CONTIGUOUS"]
     _load().oracle_hier_levels(B, Hq, Hkv, d, c, W, L, _p(n), _p(grp), _p(kk), scale, _dtcode(q), _p(q),
                                arr(k_g), arr(v_g), _p(k_raw), _p(v_raw), _p(k_tail), _p(v_tail), arr(idx),
-                               _p(out))
+                               _p(out), 0 if given is None else 1)
     return idx, out
 
 

@@ -60,17 +60,22 @@ static double default_scale(double scale, int d) { return scale > 0 ? scale : 1.
 /*        s[b,hk,j] = sum_{h in group(hk)} sum_i q[b,h,i] * Kg[b,hk,j,i].    */
 /* (No softmax scale: a positive scale does not change the ranking.)         */
 /* ------------------------------------------------------------------------ */
-static double gist_score(int Hq, int Hkv, int d, int N, int dt, const void* q, const void* kg,
-                         int b, int hk, int j) {
+/* qb: the query's batch index in q [..][Hq][d] (b for a decode step).      */
+static double gist_score_q(int Hq, int Hkv, int d, int N, int dt, const void* q, int64_t qb, const void* kg,
+                           int b, int hk, int j) {
     int G = Hq / Hkv;
     double acc = 0.0;
     for (int g = 0; g < G; ++g) {
         int h = hk * G + g;
         for (int i = 0; i < d; ++i)
-            acc += ld(q, dt, ((int64_t)b * Hq + h) * d + i) *
-                   ld(kg, dt, (((int64_t)b * Hkv + hk) * N + j) * d + i);
+            acc += ld(q, dt, (qb * Hq + h) * d + i) * ld(kg, dt, (((int64_t)b * Hkv + hk) * N + j) * d + i);
     }
     return acc;
+}
+
+static double gist_score(int Hq, int Hkv, int d, int N, int dt, const void* q, const void* kg,
+                         int b, int hk, int j) {
+    return gist_score_q(Hq, Hkv, d, N, dt, q, b, kg, b, hk, j);
 }
 
 void oracle_gist_scores(int B, int Hq, int Hkv, int d, int N, int dt, const void* q, const void* kg,
@@ -244,12 +249,8 @@ static void attend(int d, int dt, double scale, const void* q, int64_t q_off, in
  * [DE-M] "Hybride Attention": the selected raw tokens and the gists of the
  * chunks that were NOT selected (a selected chunk is represented by its raw
  * tokens instead of its gist) -> UNSELECTED_GISTS.
- * In both modes the W uncompressed tail tokens after the last chunk are
+ * In every mode the W uncompressed tail tokens after the last chunk are
  * always attended ([SL-9]: the generation suffix attends directly).          */
-/* Raw token u of chunk j of row `row`: in the dense cache [rows][N][c][d], or,  */
-/* when a block table is given, in page table[row][j] of a page pool            */
-/* [pages][c][d] ([EN-4] "KV-Cache Reuse": precomputed document caches routed   */
-/* through their gists; a page may belong to several rows).                     */
 /* Element offset of raw token u of chunk j of (b, hk).  Dense: raw [B][Hkv][N][c][d].
  * Paged ([EN-4] "KV-Cache Reuse": precomputed document caches are shared, not
  * copied): chunk j of sequence b is page table[b*N + j] of a pool
@@ -441,6 +442,49 @@ void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, in
 }
 
 /* ------------------------------------------------------------------------ */
+/* Stage-2 selective finetuning, forward pass.  [EN-2] "Training Procedure": */
+/* selective finetuning changes the attention mask so that attention goes    */
+/* only to the top-k selected chunks and their raw tokens; [SL-10]: the      */
+/* suffix token's attention to the gists gives the scores, the top-k picks   */
+/* the chunks to unfold.  Reading taken: every suffix position p selects its */
+/* own chunks exactly as a decode query does (the G heads of a KV head share */
+/* one selection, summed logits), and attends to the decode context of the   */
+/* mode with the suffix tokens 0..p as its tail (causal).                    */
+/*   q, out [B][S][Hq][d] (position-major); gists and raw as for decode;     */
+/*   ksuf, vsuf [B][Hkv][S][d]; idx_out [B][Hkv][S][k]; scores_out           */
+/*   [B][Hkv][S][N] (may be NULL).                                           */
+/* ------------------------------------------------------------------------ */
+void oracle_suffix_attn(int B, int Hq, int Hkv, int d, int N, int c, int k, int S, int mode, double scale,
+                        int dt, const void* q, const void* kg, const void* vg, const void* kraw,
+                        const void* vraw, const void* ksuf, const void* vsuf, double* scores_out,
+                        int32_t* idx_out, double* out) {
+    int G = Hq / Hkv;
+    double sc = default_scale(scale, d);
+#pragma omp parallel for collapse(3) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk)
+            for (int p = 0; p < S; ++p) {
+                int64_t row = (int64_t)b * Hkv + hk, qb = (int64_t)b * S + p, yrow = row * S + p;
+                double* s = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+                for (int j = 0; j < N; ++j) s[j] = gist_score_q(Hq, Hkv, d, N, dt, q, qb, kg, b, hk, j);
+                if (scores_out)
+                    for (int j = 0; j < N; ++j) scores_out[yrow * N + j] = s[j];
+                int32_t* sel = idx_out + yrow * k;
+                topk_list(N, s, NULL, k, sel);
+                key_ref* keys = (key_ref*)malloc(sizeof(key_ref) * (size_t)(N + (int64_t)k * c + S + 1));
+                int nk = flat_context(Hkv, d, N, N, c, 0, mode, b, hk, k, sel, kg, vg, kraw, vraw, NULL, NULL,
+                                      NULL, keys);
+                for (int u = 0; u <= p; ++u) keys[nk++] = (key_ref){ksuf, vsuf, (row * S + u) * d};
+                for (int g = 0; g < G; ++g) {
+                    int h = hk * G + g;
+                    attend(d, dt, sc, q, (qb * Hq + h) * d, nk, keys, out + (qb * Hq + h) * d, NULL);
+                }
+                free(keys);
+                free(s);
+            }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Hierarchy of any depth L >= 2 ([EN-2] "Hierarchical Extension (H-GSA)":   */
 /* gists are compressed again into higher-level gists and the query descends */
 /* coarse to fine; [SL-11] shows the level-2 to level-1 step).  Level 1 has  */
@@ -453,12 +497,13 @@ void oracle_hier_decode(int B, int Hq, int Hkv, int d, int N1, int c, int k1, in
 /* top-level gist, every candidate of every lower level, the raw tokens of   */
 /* the selected chunks, the tail (the two-level step above, one level at a   */
 /* time).  kg[l-1], vg[l-1]: the level-l gists [B][Hkv][n[l-1]][d], level 1  */
-/* first; idx[l-1] [B][Hkv][k[l-1]] receives level l's selection.            */
+/* first; idx[l-1] [B][Hkv][k[l-1]] receives level l's selection (given != 0:  */
+/* holds it, and the step is evaluated for that selection).                 */
 /* ------------------------------------------------------------------------ */
 void oracle_hier_levels(int B, int Hq, int Hkv, int d, int c, int W, int L, const int* n, const int* group,
                         const int* k, double scale, int dt, const void* q, const void* const* kg,
                         const void* const* vg, const void* kraw, const void* vraw, const void* ktail,
-                        const void* vtail, int32_t* const* idx, double* out) {
+                        const void* vtail, int32_t* const* idx, double* out, int given) {
     int G = Hq / Hkv;
     double sc = default_scale(scale, d);
     int64_t cap = 0;   /* context keys: bounded by all gists of all levels + raw + tail */
@@ -481,7 +526,7 @@ void oracle_hier_levels(int B, int Hq, int Hkv, int d, int c, int W, int L, cons
                 double* s = (double*)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
                 for (int t = 0; t < nc; ++t) s[t] = gist_score(Hq, Hkv, d, n[l], dt, q, kg[l], b, hk, cand[t]);
                 int32_t* S = idx[l] + row * k[l];
-                topk_list(nc, s, cand, k[l], S);
+                if (!given) topk_list(nc, s, cand, k[l], S);
                 free(s);
                 if (l == 0) break;
                 /* children of the selection, parent by parent */

@@ -114,6 +114,7 @@ S_KG2, S_VG2, S_NEEDLE2_NOISE = 10, 11, 12
 S_PQ, S_PK, S_PV = 20, 21, 22
 S_PAGE_K, S_PAGE_V, S_PAGE_ORDER, S_DOC, S_SEQ_LEN = 30, 31, 32, 33, 34
 S_LEVEL_K, S_LEVEL_V, S_LEVEL_NOISE = 40, 50, 60   # + level
+S_SUF_Q, S_SUF_K, S_SUF_V = 70, 71, 72
 
 
 @dataclass(frozen=True)
@@ -180,6 +181,14 @@ class LevelsShape:
         for g in self.groups:
             n.append(-(-n[-1] // g))
         return n
+
+
+@dataclass(frozen=True)
+class SuffixShape:
+    """The forward pass of a suffix of S = base.tail_len tokens after N
+    compressed chunks (stage-2 selective finetuning): every suffix position
+    selects its own chunks; the suffix attends causally to itself."""
+    base: DecodeShape
 
 
 @dataclass(frozen=True)
@@ -486,3 +495,30 @@ def levels_inputs(h: LevelsShape, seed: int) -> LevelsInputs:
                         node = lo + u64(seed, S_NEEDLE_IDX, 5_555_555 + (row * s.n_needles + t) * L + lv) % width
                     needles[row, t] = node
     return LevelsInputs(h, base.q, kg, vg, base.k_raw, base.v_raw, base.k_tail, base.v_tail, needles)
+
+
+@dataclass
+class SuffixInputs:
+    shape: SuffixShape
+    q: np.ndarray        # [B, S, Hq, d]
+    k_gist: np.ndarray
+    v_gist: np.ndarray
+    k_raw: np.ndarray
+    v_raw: np.ndarray
+    k_suf: np.ndarray    # [B, Hkv, S, d]
+    v_suf: np.ndarray
+
+
+def suffix_inputs(ss: SuffixShape, seed: int) -> SuffixInputs:
+    """Gists and raw chunks as for decode (needles along each sequence's
+    common query direction); the suffix queries of a sequence share that
+    direction: q[b, p, h] = q0[b, h] + 0.5 * noise[b, p, h]."""
+    s = ss.base
+    B, Hq, Hkv, d, S, dt = s.batch, s.n_q_heads, s.n_kv_heads, s.head_dim, s.tail_len, s.dtype
+    base = decode_inputs(replace(s, tail_len=0), seed)
+    q0 = widen(base.q, dt)
+    noise = normal(seed, S_SUF_Q, (B, S, Hq, d), "f64")
+    q = round_to(q0[:, None] + 0.5 * noise, dt)
+    ks = normal(seed, S_SUF_K, (B, Hkv, S, d), dt)
+    vs = normal(seed, S_SUF_V, (B, Hkv, S, d), dt)
+    return SuffixInputs(ss, q, base.k_gist, base.v_gist, base.k_raw, base.v_raw, ks, vs)

@@ -690,3 +690,69 @@ def test_levels_selection_follows_the_tree_and_finds_needle_chains():
     for r in range(4):
         b, hk = divmod(r, 2)
         assert set(x.needles[r].tolist()) <= set(idx[0][b, hk].tolist())
+
+
+def test_levels_given_selection_reproduces_own_selection():
+    h = synth.LevelsShape(DecodeShape(1, 4, 2, 16, 120, 2, 4, 3, "f32", n_needles=2), (4, 3), (5, 3))
+    x = synth.levels_inputs(h, 86)
+    idx, out = _levels(x, h)
+    idx2, out2 = oracle.hier_levels(x.q, x.k_g, x.v_g, x.k_raw, x.v_raw, x.k_tail, x.v_tail, h.groups,
+                                    (h.l1.top_k,) + tuple(h.top_ks), given=idx)
+    np.testing.assert_array_equal(out, out2)
+
+
+# ------------------------------------------- stage-2 suffix forward --------
+def _suffix_small(mode=ALL_GISTS, S=5, k=2, seed=91, dt="f32"):
+    ss = synth.SuffixShape(small_shape(n_chunks=7, top_k=k, tail_len=S, mode=mode, dtype=dt, n_needles=1))
+    return ss, synth.suffix_inputs(ss, seed)
+
+
+@pytest.mark.parametrize("mode", [ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS])
+def test_suffix_position_is_a_decode_step_with_the_causal_tail(mode):
+    """Suffix position p is the decode step (pinned above) of query q[:, p]
+    with the suffix tokens 0..p as the tail: scores, selection and output
+    bit for bit."""
+    ss, x = _suffix_small(mode)
+    sc, idx, out = oracle.suffix_attn(x.q, x.k_gist, x.v_gist, x.k_raw, x.v_raw, x.k_suf, x.v_suf, 2, mode)
+    for p in range(ss.base.tail_len):
+        t = dict(q=np.ascontiguousarray(x.q[:, p]), k_gist=x.k_gist, v_gist=x.v_gist, k_raw=x.k_raw,
+                 v_raw=x.v_raw, k_tail=np.ascontiguousarray(x.k_suf[:, :, :p + 1]),
+                 v_tail=np.ascontiguousarray(x.v_suf[:, :, :p + 1]))
+        s0, i0, o0 = oracle.decode(t, 2, mode)
+        np.testing.assert_array_equal(sc[:, :, p], s0)
+        np.testing.assert_array_equal(idx[:, :, p], i0)
+        np.testing.assert_array_equal(out[:, p], o0)
+
+
+def test_suffix_slide10_worked_example():
+    """Slide 10: four chunks whose gists score 0.1, 0.8, 0.7, 0.2 against the
+    suffix token; top-2 unfolds chunks 2 and 3 (0-based 1, 2).  The context
+    (every gist, the raw tokens of chunks 1 and 2, the suffix so far) is
+    listed here by hand for library SDPA."""
+    d, c = 4, 2
+    ss = synth.SuffixShape(DecodeShape(1, 1, 1, d, 4, c, 2, 2, "f32"))
+    x = synth.suffix_inputs(ss, 92)
+    x.q[...] = np.float32([1, 0, 0, 0])
+    x.k_gist[0, 0, :, 0] = np.float32([0.1, 0.8, 0.7, 0.2])
+    x.k_gist[0, 0, :, 1:] = 0
+    sc, idx, out = oracle.suffix_attn(x.q, x.k_gist, x.v_gist, x.k_raw, x.v_raw, x.k_suf, x.v_suf, 2)
+    np.testing.assert_allclose(sc[0, 0, 0], np.float32([0.1, 0.8, 0.7, 0.2]), rtol=0, atol=0)
+    assert idx[0, 0].tolist() == [[1, 2], [1, 2]]
+    for p in range(2):
+        K = np.concatenate([x.k_gist[0, 0], x.k_raw[0, 0, [1, 2]].reshape(-1, d), x.k_suf[0, 0, :p + 1]])
+        V = np.concatenate([x.v_gist[0, 0], x.v_raw[0, 0, [1, 2]].reshape(-1, d), x.v_suf[0, 0, :p + 1]])
+        want = sdpa(x.q[0, p].astype(np.float64), K.astype(np.float64), V.astype(np.float64), 0.5)
+        np.testing.assert_allclose(out[0, p], want, rtol=0, atol=1e-12)
+
+
+def test_suffix_is_causal():
+    """Changing suffix token t's key and value changes the outputs of
+    positions >= t and leaves the earlier ones bit for bit."""
+    ss, x = _suffix_small(S=6)
+    _, _, o0 = oracle.suffix_attn(x.q, x.k_gist, x.v_gist, x.k_raw, x.v_raw, x.k_suf, x.v_suf, 2)
+    ks, vs = x.k_suf.copy(), x.v_suf.copy()
+    ks[:, :, 3] += 1.0
+    vs[:, :, 3] -= 2.0
+    _, _, o1 = oracle.suffix_attn(x.q, x.k_gist, x.v_gist, x.k_raw, x.v_raw, ks, vs, 2)
+    np.testing.assert_array_equal(o1[:, :3], o0[:, :3])
+    assert np.all(np.abs(o1[:, 3:] - o0[:, 3:]).max(axis=(2, 3)) > 0)

@@ -13,7 +13,7 @@
  *   [DE-M]  gist.science explainer (DE), section "Methodik";
  *   [DE-E]  gist.science explainer (DE), section "Ergebnisse";
  *   [SL-n]  Taki-lab slide deck (docswell), page n: 6 "GSA とは", 7 "Gist
- *           token", 9/10 "Training", 11 "H-GSA", 17 "Selective Rules
+ *           token", 9/10 "Training" (stage 1 / stage 2), 11 "H-GSA", 17 "Selective Rules
  *           Comparison", 18 "Top-k vs. Top-p".
  *
  * Conventions shared by every entry point
@@ -266,6 +266,27 @@ gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const v
                              const void* const* v_gists, const void* k_raw, const void* v_raw,
                              const void* k_tail, const void* v_tail, int32_t* const* idx_out,
                              void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Stage-2 selective-finetuning forward pass ([EN-2] "Training Procedure":
+ * in selective finetuning the attention mask is changed so that attention
+ * goes only to the top-k selected chunks and their raw tokens; [SL-10]: the
+ * suffix token's attention to the gists gives the scores, top-k picks the
+ * chunks to unfold).  Reading taken: every position p of a suffix of
+ * S = desc->tail_len tokens selects its own chunks exactly as a decode query
+ * does (gsa_score summed over the G heads of a KV head, top-k ascending,
+ * ties to the lower index) and attends to the decode context of desc->mode
+ * with the suffix tokens 0..p as its tail (causal).
+ *   q, out [B][S][Hq][d] (position-major, so a position's heads are
+ *   contiguous); k_gist, v_gist, k_raw, v_raw as for gsa_decode_step;
+ *   k_suffix, v_suffix [B][Hkv][S][d]; idx_out [B][Hkv][S][k] and
+ *   scores_out [B][Hkv][S][N] nullable.  B * S * Hkv <= 65535.  Runs on the
+ *   CUDA-core passes: 2 launches (3 in GSA_UNSELECTED_GISTS mode).         */
+size_t gsa_suffix_workspace_size(const gsa_decode_desc* desc);
+int gsa_suffix_launch_count(const gsa_decode_desc* desc);
+gsa_status gsa_suffix_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist,
+                           const void* v_gist, const void* k_raw, const void* v_raw,
+                           const void* k_suffix, const void* v_suffix, int32_t* idx_out,
+                           float* scores_out, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Gist-causal prefill ([EN-2] "Interleaved Gist Tokens"; [SL-7] gist causal
  * mask g1 -> x1,x2; g2 -> g1,x3,x4; g3 -> g1,g2,x5,x6,g3; [SL-9]).  Position p

@@ -26,7 +26,8 @@ EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", 
            "gsa_workspace_error", "gsa_status_string", "gsa_decode_step_noalloc", "gsa_decode_launch_count",
            "gsa_hier_launch_count", "gsa_device_error", "gsa_set_wait_limit_ns", "gsa_topp",
            "gsa_decode_step_topp", "gsa_decode_step_paged",
-           "gsa_levels_workspace_size", "gsa_levels_decode", "gsa_levels_launch_count")
+           "gsa_levels_workspace_size", "gsa_levels_decode", "gsa_levels_launch_count",
+           "gsa_suffix_workspace_size", "gsa_suffix_launch_count", "gsa_suffix_attn")
 
 
 class GsaError(RuntimeError):
@@ -89,6 +90,9 @@ def _signatures():
         "gsa_levels_workspace_size": (sz, [ctypes.POINTER(LevelsDesc)]),
         "gsa_levels_decode": (st, [ctypes.POINTER(LevelsDesc)] + [vp] * 10 + [sz, vp]),
         "gsa_levels_launch_count": (ctypes.c_int, [ctypes.POINTER(LevelsDesc)]),
+        "gsa_suffix_workspace_size": (sz, [pd]),
+        "gsa_suffix_launch_count": (ctypes.c_int, [pd]),
+        "gsa_suffix_attn": (st, [pd] + [vp] * 10 + [vp, sz, vp]),
         "gsa_hier_launch_count": (ctypes.c_int, [ph]),
     }
 
@@ -316,3 +320,24 @@ def gsa_levels_decode(desc, q, k_gists, v_gists, k_raw, v_raw, k_tail, v_tail, i
     _check(lib().gsa_levels_decode(ctypes.byref(desc), _ptr(q), arr(k_gists), arr(v_gists), _ptr(k_raw), _ptr(v_raw),
                                    _ptr(k_tail), _ptr(v_tail), None if idx_out is None else arr(idx_out), _ptr(out),
                                    _ptr(ws), nb, _stream(stream)), "gsa_levels_decode")
+
+
+def gsa_suffix_workspace_size(desc) -> int:
+    return int(lib().gsa_suffix_workspace_size(ctypes.byref(desc)))
+
+
+def gsa_suffix_launch_count(desc) -> int:
+    n = lib().gsa_suffix_launch_count(ctypes.byref(desc))
+    if n < 0:
+        raise GsaError(1, "gsa_suffix_launch_count")
+    return int(n)
+
+
+def gsa_suffix_attn(desc, q, k_gist, v_gist, k_raw, v_raw, k_suffix, v_suffix, idx_out, scores_out, out, ws,
+                    stream=None, ws_bytes=None):
+    """Stage-2 forward over a suffix of desc.tail_len tokens: q / out
+    [B, S, Hq, d], k_suffix / v_suffix [B, Hkv, S, d]."""
+    nb = _nbytes(ws) if ws_bytes is None else ws_bytes
+    _check(lib().gsa_suffix_attn(ctypes.byref(desc), _ptr(q), _ptr(k_gist), _ptr(v_gist), _ptr(k_raw), _ptr(v_raw),
+                                 _ptr(k_suffix), _ptr(v_suffix), _ptr(idx_out), _ptr(scores_out), _ptr(out), _ptr(ws),
+                                 nb, _stream(stream)), "gsa_suffix_attn")

@@ -77,6 +77,10 @@ struct PassParams {
     const int32_t* table;
     const int32_t* nch;
     int n_pages;
+    // selection rows: blockIdx.y = kv row * S + position (S = 1 for a decode step).  causal: the
+    // tail of position p is its first p + 1 tokens (a suffix attending to itself); q / out are
+    // [B][S][Hq][d]
+    int S, causal;
 };
 
 // --------------------------------------------------------- shared memory --
@@ -131,8 +135,8 @@ __device__ __forceinline__ int seq_chunks(const int32_t* nch, uint32_t* err, int
 }
 
 // Valid entries of a row's virtual gist list.
-__device__ __forceinline__ int valid_entries(const PassParams& p, int row) {
-    if (p.parent_idx == nullptr) return seq_chunks(p.nch, p.err, row / p.Hkv, p.Nv);
+__device__ __forceinline__ int valid_entries(const PassParams& p, int row, int b) {
+    if (p.parent_idx == nullptr) return seq_chunks(p.nch, p.err, b, p.Nv);
     if (p.parent_k == 0) return 0;
     const int last = __ldcg(p.parent_idx + (size_t)row * p.parent_k + p.parent_k - 1);
     return (p.parent_k - 1) * p.group + min(p.group, p.N - last * p.group);
@@ -145,8 +149,9 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     auto& sm = *reinterpret_cast<Smem<T, D, G, NS>*>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int s = blockIdx.x, row = blockIdx.y;
-    const int b = row / p.Hkv, hk = row % p.Hkv;
+    const int s = blockIdx.x, row = blockIdx.y;        // row: the selection row
+    const int kv = row / p.S, pos = row - kv * p.S;    // its K/V row and query position
+    const int b = kv / p.Hkv, hk = kv % p.Hkv;
     const bool attn = p.do_attn != 0;
 
     if (threadIdx.x == 0) {
@@ -162,11 +167,11 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
 
     int t0, t1;
     split_range(s, p.SA, p.tprA, t0, t1);
-    const int nvalid = valid_entries(p, row);
+    const int nvalid = valid_entries(p, row, b);
     const int j0 = t0 * C::TILE;
     const int j1 = min(t1 * C::TILE, nvalid);
     const int ntiles = j1 > j0 ? (j1 - j0 + C::TILE - 1) / C::TILE : 0;
-    const size_t gist_row = (size_t)row * p.N;      // physical gist rows of this (b, hk)
+    const size_t gist_row = (size_t)kv * p.N;       // physical gist rows of this (b, hk)
     const size_t score_row = (size_t)row * p.Nv;     // virtual score entries
 
     if (warp == NCW) {
@@ -200,7 +205,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) gist_pass_kernel(const __grid_con
     } else {
         // ------------------------------------------------------ consumers --
         WarpAttn<T, D, G> wa;
-        wa.load_q(reinterpret_cast<const T*>(p.q + ((size_t)b * p.Hkv * G + (size_t)hk * G) * C::ROWB), lane);
+        wa.load_q(reinterpret_cast<const T*>(p.q + (((size_t)b * p.S + pos) * p.Hkv * G + (size_t)hk * G) * C::ROWB),
+                  lane);
         auto& ws = sm.warp[warp];
         for (int t = 0; t < ntiles; ++t) {
             const int slot = t % NS;
@@ -331,7 +337,7 @@ __device__ __forceinline__ size_t raw_first_row(const PassParams& p, int row, in
 // Unfolded keys of a row, in order: for each selected chunk u (idx order) its
 // c raw tokens (then its gist in SELECTED_PAIRS mode), then the W tail tokens.
 template <int ROWB>
-__device__ __forceinline__ void unfold_issue(const PassParams& p, int row, int x, int xe, uint8_t* dk,
+__device__ __forceinline__ void unfold_issue(const PassParams& p, int row, int kv, int x, int xe, uint8_t* dk,
                                              uint8_t* dv, uint64_t* bar, uint64_t pol) {
     const int kU = p.K * p.U;
     while (x < xe) {
@@ -349,19 +355,19 @@ __device__ __forceinline__ void unfold_issue(const PassParams& p, int row, int x
             }
             if (r < p.C) {
                 run = min(p.C - r, xe - x);
-                const size_t o = (raw_first_row(p, row, j, empty) + r) * ROWB;
+                const size_t o = (raw_first_row(p, kv, j, empty) + r) * ROWB;
                 sk = p.kr + o;
                 sv = p.vr + o;
             } else {
                 run = 1;
-                const size_t o = ((size_t)row * p.N + j) * ROWB;
+                const size_t o = ((size_t)kv * p.N + j) * ROWB;
                 sk = p.kg + o;
                 sv = p.vg + o;
             }
         } else {
             const int tt = x - kU;
             run = min(p.W - tt, xe - x);
-            const size_t o = ((size_t)row * p.W + tt) * ROWB;
+            const size_t o = ((size_t)kv * p.W + tt) * ROWB;
             sk = p.kt + o;
             sv = p.vt + o;
         }
@@ -380,13 +386,16 @@ __global__ void __launch_bounds__(NTHREADS, 3) unfold_pass_kernel(const __grid_c
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     auto& sm = *reinterpret_cast<Smem<T, D, G, NS>*>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int s = blockIdx.x, row = blockIdx.y;
-    const int b = row / p.Hkv, hk = row % p.Hkv;
+    const int s = blockIdx.x, row = blockIdx.y;        // row: the selection row
+    const int kv = row / p.S, pos = row - kv * p.S;    // its K/V row and query position
+    const int b = kv / p.Hkv, hk = kv % p.Hkv;
+    // keys of this row: the unfolded units, then its tail (causal: tokens 0..pos)
+    const int KB = p.causal ? p.K * p.U + pos + 1 : p.KB;
     int t0, t1;
     split_range(s, p.SB, p.tprB, t0, t1);
     const int x0 = t0 * C::TILE;
-    const int x1 = min(t1 * C::TILE, p.KB);
-    const int ntiles = t1 - t0;
+    const int x1 = min(t1 * C::TILE, KB);
+    const int ntiles = x1 > x0 ? (x1 - x0 + C::TILE - 1) / C::TILE : 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
@@ -408,14 +417,15 @@ __global__ void __launch_bounds__(NTHREADS, 3) unfold_pass_kernel(const __grid_c
                 const int xa = x0 + t * C::TILE;
                 const int nk = min(C::TILE, x1 - xa);
                 mbar_arrive_expect_tx(&sm.full[slot], 2u * nk * C::ROWB);
-                unfold_issue<C::ROWB>(p, row, xa, xa + nk, sm.stage[slot][0], sm.stage[slot][1], &sm.full[slot],
-                                      pol);
+                unfold_issue<C::ROWB>(p, row, kv, xa, xa + nk, sm.stage[slot][0], sm.stage[slot][1],
+                                      &sm.full[slot], pol);
             }
             for (int t = max(0, ntiles - NS); t < ntiles; ++t) mbar_wait(&sm.full[t % NS], (t / NS) & 1, p.err);
         }
     } else {
         WarpAttn<T, D, G> wa;
-        wa.load_q(reinterpret_cast<const T*>(p.q + ((size_t)b * p.Hkv * G + (size_t)hk * G) * C::ROWB), lane);
+        wa.load_q(reinterpret_cast<const T*>(p.q + (((size_t)b * p.S + pos) * p.Hkv * G + (size_t)hk * G) * C::ROWB),
+                  lane);
         auto& ws = sm.warp[warp];
         for (int t = 0; t < ntiles; ++t) {
             const int slot = t % NS;
@@ -493,7 +503,7 @@ __global__ void __launch_bounds__(NTHREADS, 3) unfold_pass_kernel(const __grid_c
             acc = fmaf(w, v, acc);
         }
         const float r = acc / fin[h * 2 + 1];
-        const size_t oi = ((size_t)b * p.Hkv * G + (size_t)hk * G + h) * D + e;
+        const size_t oi = ((((size_t)b * p.S + pos) * p.Hkv + hk) * G + h) * D + e;
         if constexpr (sizeof(T) == 4) {
             reinterpret_cast<float*>(p.out)[oi] = r;
         } else {
@@ -502,7 +512,7 @@ __global__ void __launch_bounds__(NTHREADS, 3) unfold_pass_kernel(const __grid_c
     }
     if (p.lse != nullptr && threadIdx.x < G) {
         const int h = threadIdx.x;
-        p.lse[(size_t)b * p.Hkv * G + (size_t)hk * G + h] = (fin[h * 2] + log2f(fin[h * 2 + 1])) * 0.69314718055994531f;
+        p.lse[(((size_t)b * p.S + pos) * p.Hkv + hk) * G + h] = (fin[h * 2] + log2f(fin[h * 2 + 1])) * 0.69314718055994531f;
     }
     if (threadIdx.x == 0) p.cntB[row] = 0;
 }
@@ -742,6 +752,8 @@ static PassParams make_params(const DecodePlan& pl, const gsa_decode_desc& d, co
     p.Nv = d.n_chunks;
     p.slot_base = 0;
     p.slot_stride = pl.SA;
+    p.S = 1;
+    p.causal = 0;
     return p;
 }
 
@@ -1246,6 +1258,74 @@ gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const v
 int gsa_levels_launch_count(const gsa_levels_desc* desc) {
     if (validate_levels(desc) != GSA_OK) return -1;
     return desc->levels + 1;
+}
+
+// Stage-2 selective-finetuning forward ([EN-2] "Training Procedure";
+// slide page 10): every suffix position is a selection row of the CUDA-core
+// passes (its own scores and top-k, shared by the G heads of a KV head), the
+// suffix tokens 0..p its causal tail.  The plan is the decode plan of a
+// batch of B * S rows.
+static gsa_decode_desc suffix_rows_desc(const gsa_decode_desc& d) {
+    gsa_decode_desc v = d;
+    v.batch = d.batch * d.tail_len;
+    return v;
+}
+
+static gsa_status validate_suffix(const gsa_decode_desc* desc) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if (desc->tail_len < 1) return GSA_ERR_ARG;
+    if ((int64_t)desc->batch * desc->tail_len * desc->n_kv_heads > 65535) return GSA_ERR_SHAPE;   // grid.y
+    return GSA_OK;
+}
+
+size_t gsa_suffix_workspace_size(const gsa_decode_desc* desc) {
+    if (validate_suffix(desc) != GSA_OK) return 0;
+    return make_decode_plan(suffix_rows_desc(*desc)).total;
+}
+
+int gsa_suffix_launch_count(const gsa_decode_desc* desc) {
+    if (validate_suffix(desc) != GSA_OK) return -1;
+    return desc->mode == GSA_UNSELECTED_GISTS && desc->top_k > 0 ? 3 : 2;
+}
+
+gsa_status gsa_suffix_attn(const gsa_decode_desc* desc, const void* q, const void* k_gist, const void* v_gist,
+                           const void* k_raw, const void* v_raw, const void* k_suffix, const void* v_suffix,
+                           int32_t* idx_out, float* scores_out, void* out, void* ws, size_t ws_bytes, void* stream) {
+    gsa_status st = validate_suffix(desc);
+    if (st != GSA_OK) return st;
+    if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_suffix, v_suffix, out)) != GSA_OK) return st;
+    if (!aligned16(idx_out) || !aligned16(scores_out)) return GSA_ERR_ALIGN;
+    const gsa_decode_desc v = suffix_rows_desc(*desc);
+    const DecodePlan pl = make_decode_plan(v);
+    if ((st = check_ws(pl.total, ws, ws_bytes)) != GSA_OK) return st;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    PassParams p = make_params(pl, v, q, k_gist, v_gist, k_raw, v_raw, k_suffix, v_suffix, ws);
+    p.S = desc->tail_len;
+    p.causal = 1;
+    if (scores_out) p.scores = scores_out;
+    if (idx_out) p.idx_out = idx_out;
+    p.idx_in = p.idx_out;
+    p.out = static_cast<uint8_t*>(out);
+    p.do_score = 1;
+    p.do_topk = 1;
+    const int G = desc->n_q_heads / desc->n_kv_heads;
+    const bool gists = desc->mode == GSA_ALL_GISTS || desc->mode == GSA_UNSELECTED_GISTS;
+    Kernels kern = pick_kernels(desc->dtype, desc->head_dim, G);
+    if (desc->mode == GSA_UNSELECTED_GISTS && desc->top_k > 0) {
+        // the gist attention needs the selection first: select, then attend
+        // with the selection's gists masked out
+        if (kern.gist(p, strm) != cudaSuccess) return GSA_ERR_CUDA;
+        p.do_score = 0;
+        p.do_topk = 0;
+        p.do_attn = 1;
+        p.mask_sel = 1;
+    } else {
+        p.do_attn = gists ? 1 : 0;
+    }
+    p.merge_a = p.do_attn && desc->n_chunks > 0;
+    cudaError_t e = run_passes(p, desc->dtype, desc->head_dim, G, desc->n_chunks > 0, true, strm);
+    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
 int gsa_hier_launch_count(const gsa_hier_desc* desc) {

@@ -26,7 +26,8 @@ Other workloads: --workload NAME for every decode shape of synth.WORKLOADS
 (the sweeps), llama8b_paged (the same step over a shared page pool of
 documents through gsa_decode_step_paged), hier_1m (two-level descent, steps/s
 against the HBM roofline), hier3_1m (three-level descent through
-gsa_levels_decode) and gist_prefill (the gist-causal prefill,
+gsa_levels_decode) and suffix_stage2 (the stage-2 selective-finetuning
+forward over a 512-token suffix, positions/s and algorithmic TFLOP/s) and gist_prefill (the gist-causal prefill,
 algorithmic TFLOP/s against the bf16 tensor roofline).
 """
 from __future__ import annotations
@@ -144,6 +145,35 @@ def hier_config(h, workload: str, world: int, L: int, nbytes: int, l2: int) -> d
             "parallelism": f"replicas x{world}",
             "l2": f"rotating {L} replicas (own level-2 gists and query), {L * nbytes / 1e6:.0f} MB touched "
                   f"per rotation (L2 {l2 / 1e6:.0f} MB)"}
+
+
+def suffix_flops(ss) -> float:
+    """Algorithmic FLOPs of a suffix forward: per selection row (b, hk, p)
+    the routing scores (2 G N d) and the attention over the position's
+    context (4 G n_ctx d: QK and PV), n_ctx = the mode's gists + k c + p + 1."""
+    s = ss.base
+    gists = {synth.ALL_GISTS: s.n_chunks, synth.SELECTED_PAIRS: s.top_k, synth.SR_ONLY: 0,
+             synth.UNSELECTED_GISTS: s.n_chunks - s.top_k}[s.mode]
+    G, d, S = s.group, s.head_dim, s.tail_len
+    ctx_sum = S * (gists + s.top_k * s.chunk) + S * (S + 1) / 2
+    return float(s.rows * (S * 2 * G * s.n_chunks * d + 4 * G * d * ctx_sum))
+
+
+def suffix_replicas(ss, l2: int, override: int = 0) -> int:
+    """Replicas of the per-step tensors (queries, gists, suffix K/V) to
+    rotate over so that one rotation touches >= 4x L2."""
+    s = ss.base
+    e = 4 if s.dtype == "f32" else 2
+    per_rep = e * s.head_dim * (s.batch * s.tail_len * s.n_q_heads + 2 * s.rows * (s.n_chunks + s.tail_len))
+    return override if override else max(2, -(-4 * l2 // per_rep))
+
+
+def suffix_config(ss, workload: str, world: int, L: int, l2: int) -> dict:
+    c = decode_config(ss.base, workload, world, L, 0, l2)
+    c.pop("tail")
+    c["suffix_len"] = ss.base.tail_len
+    c["l2"] = f"rotating {L} replicas (own queries, gists and suffix K/V); raw chunks shared (L2 {l2 / 1e6:.0f} MB)"
+    return c
 
 
 def levels_config(h, workload: str, world: int, L: int, nbytes: int, l2: int) -> dict:
@@ -725,6 +755,99 @@ def run_hier(args, world, rank, local):
     del g
 
 
+SUFFIX_METRIC = "GSA stage-2 suffix forward positions/s and achieved TFLOP/s against the B200 bf16 peak"
+
+
+def run_suffix(args, world, rank, local):
+    """The stage-2 forward: K steps (each the whole suffix of every sequence)
+    as one graph rotating over L replicas, median over REPLAYS replays."""
+    import torch
+
+    import kv_cache_routing_b200 as gsa
+
+    ss = synth.WORKLOADS[args.workload]
+    s = ss.base
+    torch.cuda.set_device(local)
+    l2 = l2_bytes(local)
+    seed = synth.seed_for(args.workload) + 17 * rank
+    x = synth.suffix_inputs(ss, seed)
+    shared = {k: _dev(v) for k, v in (("k_raw", x.k_raw), ("v_raw", x.v_raw))}
+    own = {k: _dev(getattr(x, k)) for k in ("q", "k_gist", "v_gist", "k_suf", "v_suf")}
+    L = suffix_replicas(ss, l2, args.replicas)
+    reps = [own] + [{k: v.clone() for k, v in own.items()} for _ in range(L - 1)]
+    desc = _desc_of(s)
+    ws = torch.zeros(max(256, gsa.gsa_suffix_workspace_size(desc)), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((s.batch, s.tail_len, s.n_q_heads, s.head_dim), dtype=_tdtype(s.dtype), device="cuda")
+            for _ in range(L)]
+    stream = torch.cuda.Stream()
+
+    def step(i, st):
+        t = reps[i % L]
+        gsa.gsa_suffix_attn(desc, t["q"], t["k_gist"], t["v_gist"], shared["k_raw"], shared["v_raw"], t["k_suf"],
+                            t["v_suf"], None, None, outs[i % L], ws, stream=st)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(args.steps):
+                step(i, stream)
+        g.replay()
+    stream.synchronize()
+    with ClockSampler(local) as clk:
+        barrier(world)
+        reps_ms = timed_replays(g.replay, stream)
+        barrier(world)
+    ms_max = max_over_ranks(statistics.median(reps_ms), world)
+    assert gsa.gsa_workspace_error(ws, stream=stream) == 0
+    per_ms = ms_max / args.steps
+    flops = suffix_flops(ss)
+    tflops = flops / (per_ms / 1e3) / 1e12
+    positions = s.batch * s.tail_len
+    qh = torch.empty_like(own["q"], device="cpu").pin_memory()
+    qh.copy_(own["q"].cpu())
+    oh = torch.empty_like(outs[0], device="cpu").pin_memory()
+    steps_e2e = max(1, min(args.steps, 20))
+
+    def e2e_run():
+        for i in range(steps_e2e):
+            reps[i % L]["q"].copy_(qh, non_blocking=True)
+            step(i, stream)
+            oh.copy_(outs[i % L], non_blocking=True)
+            stream.synchronize()
+
+    barrier(world)
+    e2e_ms = max_over_ranks(statistics.median(timed_replays(e2e_run, stream, 3)), world) / steps_e2e
+    peak, peak_kind = tensor_peak()
+    launches = gsa.gsa_suffix_launch_count(desc)
+    line = {
+        "metric": SUFFIX_METRIC, "value": round(whole_job_rate(args.steps, world, ms_max) * positions, 1),
+        "unit": "positions/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per_ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": s.dtype, "data": "synthetic", "config": suffix_config(ss, args.workload, world, L, l2),
+        "timing": {"replays": len(reps_ms), "statistic": "median over replays of the K-step graph",
+                   "ms_per_step_min": round(min(reps_ms) / args.steps, 5),
+                   "ms_per_step_max": round(max(reps_ms) / args.steps, 5)},
+        "algorithmic_flop_per_step": flops,
+        "roofline": {"bound": "tensor", "kernel": f"gsa_suffix_attn (whole step, {launches} launches, CUDA cores)",
+                     "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                     "peak_kind": peak_kind, "traffic": None, "traffic_source": "none"},
+        "e2e": {"value": round(positions * 1e3 / e2e_ms, 1), "unit": "positions/s",
+                "h2d_bytes_per_step": qh.numel() * qh.element_size(),
+                "d2h_bytes_per_step": oh.numel() * oh.element_size()},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_suffix(ss, x, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+
+
 def run_levels(args, world, rank, local):
     """The descent of any depth through gsa_levels_decode, timed like the
     two-level one: K steps as one graph rotating over L replicas (own
@@ -894,6 +1017,33 @@ def cpu_baseline_levels(h, x, budget_s: float):
                       f"so at most {s.rows} OpenMP threads), fp64, {el:.1f} s"}
 
 
+def _oracle_suffix_sample(ss, x, n_pos: int):
+    """The oracle on the first n_pos suffix positions of every sequence (a
+    causal prefix of the suffix is a complete problem of its own)."""
+    import oracle
+    s = ss.base
+    q = np.ascontiguousarray(x.q[:, :n_pos])
+    ks, vs = np.ascontiguousarray(x.k_suf[:, :, :n_pos]), np.ascontiguousarray(x.v_suf[:, :, :n_pos])
+    return lambda: oracle.suffix_attn(q, x.k_gist, x.v_gist, x.k_raw, x.v_raw, ks, vs, s.top_k, s.mode)
+
+
+def cpu_baseline_suffix(ss, x, budget_s: float):
+    s = ss.base
+    n_pos = min(s.tail_len, 16)
+    run = _oracle_suffix_sample(ss, x, n_pos)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 1000:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(n * s.batch * n_pos / el, 3), "unit": "positions/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} runs of the first {n_pos} suffix positions of each of the {s.batch} sequences, fp64, "
+                      f"OpenMP over (b, kv head, position), {el:.1f} s"}
+
+
 def run_reference(args, world, rank):
     """The reference arm: the fp64 oracle as it stands, on the host cores, on
     the same workload, metric, unit and config as the GPU arm; each step is
@@ -928,6 +1078,14 @@ def run_reference(args, world, rank):
         sample = f"one full hierarchical step per step ({w.l1.rows} rows, OpenMP over rows), fp64"
         cores = min(cores, w.l1.rows)
         rate = lambda sec: 1.0 / sec
+    elif isinstance(w, synth.SuffixShape):
+        x = synth.suffix_inputs(w, seed)
+        n_pos = min(w.base.tail_len, 16)
+        run = _oracle_suffix_sample(w, x, n_pos)
+        metric, unit, dtype = SUFFIX_METRIC, "positions/s", "f64"
+        config = suffix_config(w, args.workload, world, suffix_replicas(w, l2, args.replicas), l2)
+        sample = f"the first {n_pos} suffix positions of each of the {w.base.batch} sequences per step, fp64"
+        rate = lambda sec: w.base.batch * n_pos / sec
     elif isinstance(w, synth.LevelsShape):
         x = synth.levels_inputs(w, seed)
         run = _oracle_levels(w, x)
@@ -974,6 +1132,20 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def _with_chunks(w, n: int):
+    """The workload with n level-1 chunks (profiling captures of a smaller case)."""
+    import dataclasses
+    if isinstance(w, synth.DecodeShape):
+        return dataclasses.replace(w, n_chunks=n, n_needles=min(w.n_needles, n))
+    if isinstance(w, synth.HierShape):
+        return dataclasses.replace(w, l1=_with_chunks(w.l1, n), n_l2=-(-n // w.group))
+    if isinstance(w, (synth.LevelsShape,)):
+        return dataclasses.replace(w, l1=_with_chunks(w.l1, n))
+    if isinstance(w, (synth.SuffixShape, synth.PagedShape)):
+        return dataclasses.replace(w, base=_with_chunks(w.base, n))
+    raise SystemExit("--n-chunks applies to decode-shaped workloads")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -983,11 +1155,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--n-chunks", type=int, default=0,
+                    help="profiling captures only: a smaller case of the same kernel (level-1 chunks of a decode "
+                         "or hierarchical workload; the upper levels shrink with it)")
     ap.add_argument("--replicas", type=int, default=0,
                     help="layer replicas to rotate over (default: enough to exceed 4x L2); 1 for profiling captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.n_chunks:
+        synth.WORKLOADS[args.workload] = _with_chunks(synth.WORKLOADS[args.workload], args.n_chunks)
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
@@ -1002,6 +1179,8 @@ def main():
             run_hier(args, world, rank, local)
         elif isinstance(w, synth.LevelsShape):
             run_levels(args, world, rank, local)
+        elif isinstance(w, synth.SuffixShape):
+            run_suffix(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

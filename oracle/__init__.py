@@ -54,7 +54,7 @@ def _load():
         "oracle_suffix_attn": [i, i, i, i, i, i, i, i, i, d, i] + [vp] * 10,
         "oracle_gist_mask": [i64, i64, i],
         "oracle_prefill_pair_count": [i, i],
-        "oracle_prefill_rows": [i, i, i, i, i, i, d, i, vp, vp, vp, i64, vp, vp],
+        "oracle_prefill_rows": [i, i, i, i, i, i, d, i, vp, vp, vp, i64, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -265,14 +265,16 @@ def prefill_pair_count(n_chunks: int, chunk: int) -> int:
     return int(_load().oracle_prefill_pair_count(n_chunks, chunk))
 
 
-def prefill_rows(t: dict, n_chunks: int, chunk: int, rows: np.ndarray, scale: float = 0.0) -> np.ndarray:
-    """rows: int64 [n, 3] of (b, h, p).  Returns [n, d] fp64."""
+def prefill_rows(t: dict, n_chunks: int, chunk: int, rows: np.ndarray, scale: float = 0.0, with_lse: bool = False):
+    """rows: int64 [n, 3] of (b, h, p).  Returns out [n, d] fp64 (and the
+    natural-log normaliser lse [n] of each row's softmax)."""
     q, k, v = t["q"], t["k"], t["v"]
     B, Hq, P, d = q.shape
     Hkv = k.shape[1]
     assert P == n_chunks * (chunk + 1)
     rows = np.ascontiguousarray(rows, np.int64)
     out = np.empty((rows.shape[0], d), np.float64)
+    lse = np.empty(rows.shape[0], np.float64) if with_lse else None
     _load().oracle_prefill_rows(B, Hq, Hkv, d, n_chunks, chunk, scale, _dtcode(q), _p(q), _p(k),
-                                _p(v), rows.shape[0], _p(rows), _p(out))
-    return out
+                                _p(v), rows.shape[0], _p(rows), _p(out), _p(lse))
+    return (out, lse) if with_lse else out

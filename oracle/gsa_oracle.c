@@ -586,7 +586,7 @@ int64_t oracle_prefill_pair_count(int N, int c) {
  * out: n_rows * d.  q [B][Hq][P][d], k, v [B][Hkv][P][d].                     */
 void oracle_prefill_rows(int B, int Hq, int Hkv, int d, int N, int c, double scale, int dt,
                          const void* q, const void* k, const void* v, int64_t n_rows,
-                         const int64_t* rows, double* out) {
+                         const int64_t* rows, double* out, double* lse) {
     int G = Hq / Hkv;
     int64_t P = (int64_t)N * (c + 1);
     double sc = default_scale(scale, d);
@@ -599,7 +599,7 @@ void oracle_prefill_rows(int B, int Hq, int Hkv, int d, int N, int c, double sca
         int nk = 0;
         for (int64_t t = 0; t <= p; ++t)
             if (oracle_gist_mask(p, t, c)) keys[nk++] = (key_ref){k, v, ((b * Hkv + hk) * P + t) * d};
-        attend(d, dt, sc, q, ((b * Hq + h) * P + p) * d, nk, keys, out + r * d, NULL);
+        attend(d, dt, sc, q, ((b * Hq + h) * P + p) * d, nk, keys, out + r * d, lse ? lse + r : NULL);
         free(keys);
     }
 }

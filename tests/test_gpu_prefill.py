@@ -62,6 +62,36 @@ def test_prefill_full_size_sampled():
     run_prefill(synth.WORKLOADS[name], synth.seed_for(name), name, sample=768)
 
 
+def test_prefill_full_size_exhaustive_with_lse():
+    """Every query row of the full-size prefill (2 x 32 heads x 17408
+    positions) against the oracle, output and log-normaliser, one head at a
+    time.  lse is fp32 from an fp32 logit sum: within 1e-3."""
+    name = "gist_prefill"
+    p = synth.WORKLOADS[name]
+    x = synth.prefill_inputs(p, synth.seed_for(name))
+    d = upload(x)
+    P = p.positions
+    desc = gsa.prefill_desc(p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.n_chunks, p.chunk, gsa.GSA_BF16,
+                            p.scale)
+    out = torch.full((p.batch, p.n_q_heads, P, p.head_dim), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((p.batch, p.n_q_heads, P), float("nan"), dtype=torch.float32, device="cuda")
+    gsa.gsa_gist_prefill(desc, d["q"], d["k"], d["v"], out, lse)
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0
+    got_o, got_l = host(out), lse.cpu().numpy().astype(np.float64)
+    worst_o = worst_l = 0.0
+    t = x.tensors()
+    for b in range(p.batch):
+        for h in range(p.n_q_heads):
+            rows = np.stack([np.full(P, b), np.full(P, h), np.arange(P)], axis=1).astype(np.int64)
+            want_o, want_l = oracle.prefill_rows(t, p.n_chunks, p.chunk, rows, p.scale, with_lse=True)
+            worst_o = max(worst_o, float(np.max(np.abs(got_o[b, h] - want_o))))
+            worst_l = max(worst_l, float(np.max(np.abs(got_l[b, h] - want_l))))
+    print(f"{name}: every row, max |out err| {worst_o:.3e}, max |lse err| {worst_l:.3e}")
+    assert worst_o <= TOL["bf16"]
+    assert worst_l <= 1e-3
+
+
 def test_prefill_lse_matches_oracle_normaliser():
     """lse[p] = log sum_t exp(scale q.k_t) over the allowed keys: with V = 1 the
     output is 1 everywhere, and lse equals the oracle's log-normaliser."""

@@ -756,3 +756,24 @@ def test_suffix_is_causal():
     _, _, o1 = oracle.suffix_attn(x.q, x.k_gist, x.v_gist, x.k_raw, x.v_raw, ks, vs, 2)
     np.testing.assert_array_equal(o1[:, :3], o0[:, :3])
     assert np.all(np.abs(o1[:, 3:] - o0[:, 3:]).max(axis=(2, 3)) > 0)
+
+
+def test_prefill_lse_is_library_logsumexp():
+    """The prefill rows' log-normaliser is torch.logsumexp of the scaled
+    logits over the keys the slide-7 mask allows (mask from the slide's
+    table, not from the oracle)."""
+    c, n = 2, 3
+    p = synth.PrefillShape(1, 2, 1, 8, n, c, "f32", 0.3)
+    x = synth.prefill_inputs(p, 93)
+    P = p.positions
+    rows = np.array([(0, h, t) for h in range(2) for t in range(P)], np.int64)
+    _, lse = oracle.prefill_rows(x.tensors(), n, c, rows, 0.3, with_lse=True)
+    names = _slide7_names(c, n)
+    allowed = {"x1": ["x1"], "x2": ["x1", "x2"], "g1": ["x1", "x2", "g1"], "x3": ["g1", "x3"],
+               "x4": ["g1", "x3", "x4"], "g2": ["g1", "x3", "x4", "g2"], "x5": ["g1", "g2", "x5"],
+               "x6": ["g1", "g2", "x5", "x6"], "g3": ["g1", "g2", "x5", "x6", "g3"]}
+    k = torch.from_numpy(x.k[0, 0].astype(np.float64))
+    for i, (_, h, t) in enumerate(rows):
+        keys = [names.index(nm) for nm in allowed[names[t]]]
+        logits = 0.3 * (k[keys] @ torch.from_numpy(x.q[0, h, t].astype(np.float64)))
+        assert lse[i] == pytest.approx(torch.logsumexp(logits, 0).item(), abs=1e-12)

@@ -540,8 +540,8 @@ def run_ours(args, world, rank, local):
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": nbytes_step / launches,
-                     "traffic": measured_traffic(args.workload),
-                     "traffic_source": traffic_source(args.workload)},
+                     "traffic": measured_traffic(args.workload) if not args.n_chunks else None,
+                     "traffic_source": traffic_source(args.workload) if not args.n_chunks else "none"},
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()
@@ -741,7 +741,8 @@ def run_hier(args, world, rank, local):
         "algorithmic_bytes_per_step": nbytes,
         "roofline": {"bound": "hbm", "kernel": f"gsa_hier_decode (whole step)", "achieved": round(gbs, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
-                     "traffic": None, "traffic_source": "none"},
+                     "traffic": measured_traffic(args.workload) if not args.n_chunks else None,
+                     "traffic_source": traffic_source(args.workload) if not args.n_chunks else "none"},
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
                 "h2d_bytes_per_step": qh.numel() * qh.element_size(),
                 "d2h_bytes_per_step": oh.numel() * oh.element_size()},

@@ -115,6 +115,10 @@ struct Bars {
     uint64_t gready;             // the first NSL gathered slots are free (their key / value tiles consumed)
     uint32_t tmem;
 };
+static_assert(sizeof(Bars) <= 512, "mbarriers overflow their shared-memory region");
+// a gathered tile takes two consecutive slots from the CTA's first gathered
+// one, so with an even ring a tile's slots are both handed over or neither
+static_assert(NSL % 2 == 0, "the gathered slots' hand-over assumes an even ring");
 
 // A tile of work: 128 keys of one row.
 struct Tile {

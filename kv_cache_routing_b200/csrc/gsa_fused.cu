@@ -1083,9 +1083,13 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
         const int r = tma_rows + (q >> 4);
         gather_piece(p, ks, vs, tab[r], r, q & 15);
     }
-    // runs skipped above (an empty place of a variable-size selection): V rows zeroed
-    for (int q = utid(); q < tma_rows * 16; q += NU)
-        if (tab[((q >> 4) / h) * h] == -1) gather_piece(p, ks, vs, -1, q >> 4, q & 15);
+    // runs skipped above (an empty place of a variable-size selection): their
+    // V rows zeroed.  One table read per run (a broadcast), so a tile with no
+    // empty place costs a handful of loads, not a pass over its pieces
+    for (int r0 = 0; r0 < tma_rows; r0 += h) {
+        if (tab[r0] != -1) continue;
+        for (int q = utid(); q < h * 16; q += NU) gather_piece(p, ks, vs, -1, r0 + (q >> 4), q & 15);
+    }
     cp_async_arrive_hold(&bars->full[sk]);
     cp_async_arrive_hold(&bars->full[sv]);
     usync();

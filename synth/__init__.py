@@ -223,6 +223,8 @@ WORKLOADS = {
     # three levels over 1M raw tokens: 65536 -> 4096 -> 256 gists, k = 8 at every level
     "hier3_1m": LevelsShape(DecodeShape(1, 32, 8, 128, 65536, 16, 8, 128, "bf16", ALL_GISTS, n_needles=8),
                             groups=(16, 16), top_ks=(8, 8)),
+    # the fixed latency of the one-launch step: a 2048-token context (8 rows, 128 gists), about 1 MB
+    "decode_floor": DecodeShape(1, 32, 8, 128, 128, 16, 4, 64, "bf16", ALL_GISTS, n_needles=4),
     # stage-2 forward: a 512-token suffix after 2048 chunks of 16 (Llama-style heads)
     "suffix_stage2": SuffixShape(DecodeShape(2, 32, 8, 128, 2048, 16, 16, 512, "bf16", ALL_GISTS, n_needles=16)),
     # the Llama-shaped step over a shared page pool of 32..160-chunk documents
@@ -235,7 +237,8 @@ WORKLOADS = {
 CONFIG_INDEX = {"tiny_f32": 1, "llama8b_decode": 2, "sweep_c8_all": 3, "sweep_c16_all": 3,
                 "sweep_c32_all": 3, "sweep_c8_pairs": 3, "sweep_c16_pairs": 3,
                 "sweep_c32_pairs": 3, "hier_1m": 4, "gist_prefill": 5, "llama8b_paged": 6,
-                "hier3_1m": 7, "suffix_stage2": 8}
+                "hier3_1m": 7, "suffix_stage2": 8,
+                "decode_floor": 9}
 
 
 def seed_for(workload: str, rep: int = 0) -> int:

@@ -75,3 +75,70 @@ def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(tmp_path, m
 def test_tensor_peak_prefers_the_sustained_measurement():
     v, kind = bench.tensor_peak()
     assert v > 0 and "sustained" in kind
+
+
+def test_paged_bytes_full_sequences_equal_the_dense_step():
+    ps = synth.WORKLOADS["llama8b_paged"]
+    s = ps.base
+    assert bench.paged_bytes(ps, np.full(s.batch, s.n_chunks)) == bench.algorithmic_bytes(s)
+
+
+def test_paged_bytes_are_the_sum_of_one_sequence_problems():
+    """A short sequence counts as the dense one-sequence problem with N = nb
+    and k = min(k, nb)."""
+    import dataclasses
+    ps = synth.WORKLOADS["llama8b_paged"]
+    s = dataclasses.replace(ps.base, batch=4)
+    ps = dataclasses.replace(ps, base=s)
+    counts = [0, 5, 700, s.n_chunks]
+    want = sum(bench.algorithmic_bytes(dataclasses.replace(s, batch=1, n_chunks=n, top_k=min(s.top_k, n)))
+               for n in counts)
+    assert bench.paged_bytes(ps, np.array(counts)) == want
+
+
+def test_levels_bytes_at_depth_two_are_the_two_level_bytes():
+    h = synth.WORKLOADS["hier_1m"]
+    hl = synth.LevelsShape(h.l1, (h.group,), (h.top_k2,))
+    assert hl.counts == [h.l1.n_chunks, h.n_l2]
+    assert bench.levels_bytes(hl) == bench.hier_bytes(h)
+
+
+def test_suffix_flops_by_position():
+    """Per selection row (b, hk, p): scores 2 G N d, attention 4 G d over the
+    mode's gists + k c raw tokens + the p + 1 suffix tokens."""
+    import dataclasses
+    base = synth.WORKLOADS["suffix_stage2"].base
+    for mode, gists in ((synth.ALL_GISTS, base.n_chunks), (synth.SELECTED_PAIRS, base.top_k),
+                        (synth.SR_ONLY, 0), (synth.UNSELECTED_GISTS, base.n_chunks - base.top_k)):
+        s = dataclasses.replace(base, tail_len=3, mode=mode)
+        G, d = s.group, s.head_dim
+        want = s.rows * sum(2 * G * s.n_chunks * d + 4 * G * d * (gists + s.top_k * s.chunk + p + 1)
+                            for p in range(3))
+        assert bench.suffix_flops(synth.SuffixShape(s)) == want
+
+
+def test_suffix_workspace_is_the_decode_plan_of_its_selection_rows():
+    """On the CUDA-core passes (fp32, d = 64) the suffix forward's workspace
+    is the decode workspace of a batch of B * S rows."""
+    import kv_cache_routing_b200 as gsa
+    for B, S in ((1, 5), (2, 64), (3, 1)):
+        d = gsa.decode_desc(B, 8, 2, 64, 300, 8, 12, S, gsa.GSA_F32)
+        rows = gsa.decode_desc(B * S, 8, 2, 64, 300, 8, 12, S, gsa.GSA_F32)
+        assert gsa.gsa_suffix_workspace_size(d) == gsa.gsa_decode_workspace_size(rows) > 0
+
+
+def test_levels_workspace_holds_every_level():
+    """The workspace holds every level's scores (top level: all its gists;
+    lower levels: the children of the selection above), selection and the
+    partials of every pass: at least the score and selection regions."""
+    import kv_cache_routing_b200 as gsa
+    l1 = gsa.decode_desc(2, 8, 2, 128, 4096, 16, 8, 64, gsa.GSA_BF16)
+    rows = 2 * 2
+    for g, k in (((8,), (16,)), ((8, 8), (16, 4)), ((8, 8, 4), (16, 8, 2))):
+        n = [4096]
+        for gg in g:
+            n.append(-(-n[-1] // gg))
+        ks = (8,) + k
+        nv = [ks[i + 1] * g[i] for i in range(len(g))] + [n[-1]]
+        floor = rows * 4 * (sum(nv) + sum(ks))
+        assert gsa.gsa_levels_workspace_size(gsa.levels_desc(l1, g, k)) >= floor

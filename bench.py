@@ -11,8 +11,9 @@ bf16).  Inputs are synthetic (seeded normals with planted needle chunks).
 Device timing: the K timed steps are one CUDA graph that rotates over L
 layer replicas whose bytes touched per rotation exceed 4x the L2 size, timed
 with CUDA events on the launching stream, max over ranks.  e2e: the same K
-steps through the C ABI from Python with the step's query copied host->device
-from pinned memory and the result copied back every step.
+steps through the C ABI from Python, each one gsa_decode_step_host call (the
+query copied host->device from pinned memory, the step, the output and the
+selection copied back) followed by a wait for the result.
 
 With --gpus N > 1 (torchrun, one process per GPU) every rank runs its own
 replica set (the path shards by independent sequences; no collective on the
@@ -499,10 +500,17 @@ def run_ours(args, world, rank, local):
     def e2e_run():
         for i in range(args.steps):
             r = i % L
-            q_dev[r].copy_(q_host[r], non_blocking=True)
-            step(i, stream)
-            out_host.copy_(outs[r], non_blocking=True)
-            idx_host.copy_(idxs[r], non_blocking=True)
+            if paged:
+                q_dev[r].copy_(q_host[r], non_blocking=True)
+                step(i, stream)
+                out_host.copy_(outs[r], non_blocking=True)
+                idx_host.copy_(idxs[r], non_blocking=True)
+            else:
+                # one C-ABI call: the query in, the step, the output and the selection out
+                t = reps[r]
+                gsa.gsa_decode_step_host(desc, q_host[r], t["q"], t["k_gist"], t["v_gist"], t["k_raw"], t["v_raw"],
+                                         t["k_tail"], t["v_tail"], idxs[r], idx_host, outs[r], out_host, ws,
+                                         stream=stream)
             stream.synchronize()                     # the host reads the step's result
 
     barrier(world)

@@ -202,6 +202,20 @@ gsa_status gsa_decode_step(const gsa_decode_desc* desc, const void* q, const voi
                            const void* k_tail, const void* v_tail, int32_t* idx_out,
                            float* scores_out, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* gsa_decode_step with the query and the result in HOST memory, for a
+ * caller whose decode loop lives on the host: copies q_host [B][Hq][d] into
+ * the device buffer q, runs the step, and copies out back to out_host (and
+ * the selection idx_out to idx_host, when given), all enqueued on `stream`
+ * in this one call; nothing synchronises, so the caller waits on the stream
+ * before reading out_host.  Host buffers should be page-locked for the
+ * copies to be asynchronous.  Other arguments as for gsa_decode_step (no
+ * scores output).                                                           */
+gsa_status gsa_decode_step_host(const gsa_decode_desc* desc, const void* q_host, void* q,
+                                const void* k_gist, const void* v_gist, const void* k_raw,
+                                const void* v_raw, const void* k_tail, const void* v_tail,
+                                int32_t* idx_out, int32_t* idx_host, void* out, void* out_host,
+                                void* ws, size_t ws_bytes, void* stream);
+
 /* One decode step with top-p selection: gsa_score -> gsa_topp ->
  * gsa_unfold_attn (three launches on the tensor-core path).  desc->top_k is
  * kmax; idx_out [B][Hkv][kmax] receives the selection padded with -1,

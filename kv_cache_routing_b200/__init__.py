@@ -27,7 +27,7 @@ EXPORTS = ("gsa_decode_workspace_size", "gsa_hier_workspace_size", "gsa_score", 
            "gsa_hier_launch_count", "gsa_device_error", "gsa_set_wait_limit_ns", "gsa_topp",
            "gsa_decode_step_topp", "gsa_decode_step_paged",
            "gsa_levels_workspace_size", "gsa_levels_decode", "gsa_levels_launch_count",
-           "gsa_suffix_workspace_size", "gsa_suffix_launch_count", "gsa_suffix_attn")
+           "gsa_suffix_workspace_size", "gsa_suffix_launch_count", "gsa_suffix_attn", "gsa_decode_step_host")
 
 
 class GsaError(RuntimeError):
@@ -93,6 +93,7 @@ def _signatures():
         "gsa_suffix_workspace_size": (sz, [pd]),
         "gsa_suffix_launch_count": (ctypes.c_int, [pd]),
         "gsa_suffix_attn": (st, [pd] + [vp] * 10 + [vp, sz, vp]),
+        "gsa_decode_step_host": (st, [pd] + [vp] * 13 + [sz, vp]),
         "gsa_hier_launch_count": (ctypes.c_int, [ph]),
     }
 
@@ -341,3 +342,14 @@ def gsa_suffix_attn(desc, q, k_gist, v_gist, k_raw, v_raw, k_suffix, v_suffix, i
     _check(lib().gsa_suffix_attn(ctypes.byref(desc), _ptr(q), _ptr(k_gist), _ptr(v_gist), _ptr(k_raw), _ptr(v_raw),
                                  _ptr(k_suffix), _ptr(v_suffix), _ptr(idx_out), _ptr(scores_out), _ptr(out), _ptr(ws),
                                  nb, _stream(stream)), "gsa_suffix_attn")
+
+
+def gsa_decode_step_host(desc, q_host, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, idx_host, out,
+                         out_host, ws, stream=None, ws_bytes=None):
+    """gsa_decode_step with q_host / out_host (and idx_host) in host memory
+    (page-locked tensors or raw addresses): copy in, step, copy out, one call."""
+    nb = _nbytes(ws) if ws_bytes is None else ws_bytes
+    _check(lib().gsa_decode_step_host(ctypes.byref(desc), _ptr(q_host), _ptr(q), _ptr(k_gist), _ptr(v_gist),
+                                      _ptr(k_raw), _ptr(v_raw), _ptr(k_tail), _ptr(v_tail), _ptr(idx_out),
+                                      _ptr(idx_host), _ptr(out), _ptr(out_host), _ptr(ws), nb, _stream(stream)),
+           "gsa_decode_step_host")

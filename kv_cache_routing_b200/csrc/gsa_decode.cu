@@ -1162,6 +1162,33 @@ gsa_status gsa_decode_step_noalloc(const gsa_decode_desc* desc, const void* q, c
                            need, stream);
 }
 
+// One decode step with host-side query and output: the query is copied to
+// the device, the step runs, and the output (and the selection, when asked)
+// is copied back, all enqueued on `stream` in one call.
+gsa_status gsa_decode_step_host(const gsa_decode_desc* desc, const void* q_host, void* q, const void* k_gist,
+                                const void* v_gist, const void* k_raw, const void* v_raw, const void* k_tail,
+                                const void* v_tail, int32_t* idx_out, int32_t* idx_host, void* out, void* out_host,
+                                void* ws, size_t ws_bytes, void* stream) {
+    gsa_status st = validate_decode(desc);
+    if (st != GSA_OK) return st;
+    if (!q_host || !out_host || (idx_host && !idx_out)) return GSA_ERR_ARG;
+    const size_t qn = (size_t)desc->batch * desc->n_q_heads * desc->head_dim * elem_bytes(desc->dtype);
+    const size_t in = (size_t)desc->batch * desc->n_kv_heads * desc->top_k * sizeof(int32_t);
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    // the device-side arguments are checked by the step before anything is enqueued
+    if ((st = check_tensors(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, out)) != GSA_OK) return st;
+    if (!aligned16(idx_out)) return GSA_ERR_ALIGN;
+    if ((st = check_ws(decode_ws_bytes(*desc), ws, ws_bytes)) != GSA_OK) return st;
+    if (cudaMemcpyAsync(q, q_host, qn, cudaMemcpyHostToDevice, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    if ((st = gsa_decode_step(desc, q, k_gist, v_gist, k_raw, v_raw, k_tail, v_tail, idx_out, nullptr, out, ws,
+                              ws_bytes, stream)) != GSA_OK)
+        return st;
+    if (cudaMemcpyAsync(out_host, out, qn, cudaMemcpyDeviceToHost, strm) != cudaSuccess) return GSA_ERR_CUDA;
+    if (idx_host && in > 0 && cudaMemcpyAsync(idx_host, idx_out, in, cudaMemcpyDeviceToHost, strm) != cudaSuccess)
+        return GSA_ERR_CUDA;
+    return GSA_OK;
+}
+
 // Hierarchy of any depth ([EN-2] "Hierarchical Extension (H-GSA)"): the
 // top-level gist pass, one gathered gist pass per lower level (the children
 // of the selection above: scores, attention, top-k), then the unfold pass

@@ -154,3 +154,16 @@ def test_every_benchmark_decode_workload_takes_the_one_launch_path():
         elif isinstance(w, synth.HierShape):
             hd = gsa.hier_desc(desc_of(w.l1), w.n_l2, w.group, w.top_k2)
             assert gsa.gsa_hier_launch_count(hd) == 1, name
+
+
+def test_host_buffer_step_argument_checks():
+    """Missing host buffers, or a host selection without a device one, are
+    refused before anything is enqueued."""
+    desc = gsa.decode_desc(1, 4, 1, 64, 8, 4, 2, 2, gsa.GSA_F32)
+    dev_args = [1 << 20] * 7
+    for q_host, idx_out, idx_host, out_host in ((None, None, None, 1 << 20), (1 << 20, None, None, None),
+                                                (1 << 20, None, 1 << 20, 1 << 20)):
+        with pytest.raises(gsa.GsaError) as e:
+            gsa.gsa_decode_step_host(desc, q_host, *dev_args, idx_out, idx_host, 1 << 20, out_host, 1 << 20,
+                                     stream=0, ws_bytes=1 << 30)
+        assert e.value.status == gsa.GSA_ERR_ARG

@@ -299,3 +299,31 @@ def test_cuda_graph_capture_replays_identically():
         g.replay()
     torch.cuda.synchronize()
     assert torch.equal(idx, ref[0]) and torch.equal(out, ref[1])
+
+
+def test_host_buffer_step_equals_the_device_step():
+    """gsa_decode_step_host (query and result in pinned host memory) gives
+    the device-buffer step's selection and output bit for bit."""
+    s = dataclasses.replace(synth.WORKLOADS["llama8b_decode"], batch=2)
+    x = synth.decode_inputs(s, 83)
+    d = upload(x)
+    desc = desc_of(s)
+    ws = workspace(gsa.gsa_decode_workspace_size(desc))
+    idx = torch.empty((2, 8, 16), dtype=torch.int32, device="cuda")
+    out = torch.empty((2, 32, 128), dtype=torch.bfloat16, device="cuda")
+    gsa.gsa_decode_step(desc, d["q"], d["k_gist"], d["v_gist"], d["k_raw"], d["v_raw"], d["k_tail"], d["v_tail"],
+                        idx, None, out, ws)
+    torch.cuda.synchronize()
+    q_host = d["q"].cpu().pin_memory()
+    q_dev = torch.zeros_like(d["q"])
+    out_host = torch.empty((2, 32, 128), dtype=torch.bfloat16).pin_memory()
+    idx_host = torch.empty((2, 8, 16), dtype=torch.int32).pin_memory()
+    idx2 = torch.empty_like(idx)
+    out2 = torch.empty_like(out)
+    stream = torch.cuda.Stream()
+    gsa.gsa_decode_step_host(desc, q_host, q_dev, d["k_gist"], d["v_gist"], d["k_raw"], d["v_raw"], d["k_tail"],
+                             d["v_tail"], idx2, idx_host, out2, out_host, ws, stream=stream)
+    stream.synchronize()
+    assert gsa.gsa_workspace_error(ws) == 0
+    np.testing.assert_array_equal(idx_host.numpy(), idx.cpu().numpy())
+    np.testing.assert_array_equal(out_host.float().numpy(), out.float().cpu().numpy())

@@ -8,7 +8,6 @@ finish its launch normally and flag GSA_WS_ERR_TIMEOUT in the workspace
 error word; a fresh zero-filled workspace then gives oracle-exact results.
 The library's own error words (prefill, workspace-less calls) read 0 after
 normal calls."""
-import numpy as np
 import pytest
 import torch
 

@@ -16,7 +16,7 @@ import oracle
 import synth
 from synth import DecodeShape, LevelsShape
 
-from gsa_check import TOL, check_out, desc_of, dev, host, tdtype, workspace
+from gsa_check import check_out, desc_of, dev, host, tdtype, workspace
 
 SHAPES = {
     # 65536 raw tokens, 4096 -> 512 -> 64 gists, k = 8 / 16 / 4

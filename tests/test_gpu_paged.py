@@ -18,7 +18,7 @@ import oracle
 import synth
 from synth import ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS, DecodeShape, PagedShape
 
-from gsa_check import TOL, check_out, desc_of, dev, host, tdtype, workspace
+from gsa_check import check_out, desc_of, dev, host, tdtype, workspace
 
 MODES = [ALL_GISTS, SELECTED_PAIRS, SR_ONLY, UNSELECTED_GISTS]
 

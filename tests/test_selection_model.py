@@ -15,7 +15,6 @@ chunks), with the tie rule and output order the library documents: ties to
 the lowest index, indices ascending.
 """
 import numpy as np
-import pytest
 
 NT = 128          # threads of the unfold warp group
 WARP = 32

@@ -777,3 +777,16 @@ def test_prefill_lse_is_library_logsumexp():
         keys = [names.index(nm) for nm in allowed[names[t]]]
         logits = 0.3 * (k[keys] @ torch.from_numpy(x.q[0, h, t].astype(np.float64)))
         assert lse[i] == pytest.approx(torch.logsumexp(logits, 0).item(), abs=1e-12)
+
+
+def test_topp_ties_take_the_lower_index_first():
+    """Equal scores enter the prefix lowest index first: scores (1, 3, 1, 3, 1)
+    with scale ln 2 give weights (2, 8, 2, 8, 2) / 22.  In order 1, 3, 0, 2, 4
+    the masses accumulate to 8/22, 16/22, 18/22, 20/22, 1, so p = 0.8 stops at
+    the third chunk (index 0, the lowest of the tied ones), p = 0.85 at the
+    fourth (index 2)."""
+    s = np.array([[1.0, 3.0, 1.0, 3.0, 1.0]])
+    for p, want in ((0.30, [1]), (0.70, [1, 3]), (0.80, [0, 1, 3]), (0.85, [0, 1, 2, 3]), (0.95, [0, 1, 2, 3, 4])):
+        idx, cnt = oracle.topp(s, p, 5, math.log(2.0))
+        assert idx[0, :cnt[0]].tolist() == want, p
+        assert (idx[0, cnt[0]:] == -1).all()

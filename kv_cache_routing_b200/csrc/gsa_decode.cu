@@ -1196,7 +1196,7 @@ gsa_status gsa_decode_step_host(const gsa_decode_desc* desc, const void* q_host,
 // partials of every pass.
 size_t gsa_levels_workspace_size(const gsa_levels_desc* desc) {
     if (validate_levels(desc) != GSA_OK) return 0;
-    return make_levels_plan(*desc).total;
+    return fused_levels_supported(*desc) ? make_fused_levels_plan(*desc).total : make_levels_plan(*desc).total;
 }
 
 gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const void* const* k_gists,
@@ -1218,6 +1218,14 @@ gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const v
     const void* all[] = {q, k_raw, v_raw, k_tail, v_tail, out};
     for (const void* x : all)
         if (!aligned16(x)) return GSA_ERR_ALIGN;
+    if (fused_levels_supported(*desc)) {
+        // tensor-core path: the top level and the tail streamed, then per row one
+        // children tile per lower level and the raw tile, in one launch
+        const FusedPlan f = make_fused_levels_plan(*desc);
+        if (!ws || ws_bytes < f.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSA_ERR_WORKSPACE;
+        return fused_levels_launch(*desc, f, q, k_gists, v_gists, k_raw, v_raw, k_tail, v_tail, idx_out, out, ws,
+                                   static_cast<cudaStream_t>(stream));
+    }
     const LevelsPlan lp = make_levels_plan(*desc);
     if (!ws || ws_bytes < lp.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSA_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
@@ -1284,7 +1292,7 @@ gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const v
 
 int gsa_levels_launch_count(const gsa_levels_desc* desc) {
     if (validate_levels(desc) != GSA_OK) return -1;
-    return desc->levels + 1;
+    return fused_levels_supported(*desc) ? 1 : desc->levels + 1;
 }
 
 // Stage-2 selective-finetuning forward ([EN-2] "Training Procedure";

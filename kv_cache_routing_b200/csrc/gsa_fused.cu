@@ -1015,6 +1015,17 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
     usync();
 }
 
+// Hierarchy levels (1-based: level 1 has one gist per chunk, level L is the
+// top): gist count, selection size and selection output of level l.
+__device__ __forceinline__ int lvl_n(const Params& p, int l) {
+    return l == 1 ? p.N1 : l == p.levels ? p.N : p.midN[l - 2];
+}
+__device__ __forceinline__ int lvl_k(const Params& p, int l) {
+    return l == 1 ? p.K1 : l == p.levels ? p.K : p.midK[l - 2];
+}
+__device__ __forceinline__ int32_t* lvl_idx(const Params& p, int l) {
+    return l == 1 ? p.idx1 : l == p.levels ? p.idx : p.midIdx[l - 2];
+}
 // Tile lt of the row table into slots seq, seq + 1 (K, V) once the slots'
 // previous contents are consumed.  Its first tma_rows rows are runs of h
 // consecutive source rows (selected chunks, or the children of selected
@@ -1026,7 +1037,7 @@ __device__ __forceinline__ void build_table(const Params& p, uint8_t* base, int 
 // it, and one thread then gives the one expected arrival.
 template <bool PG>
 __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars* bars, int lt, int seq, int row,
-                                            int tma_rows, int h, bool children, int gfirst) {
+                                            int tma_rows, int h, bool children, int gfirst, int cl) {
     if (seq < gfirst + NSL) {
         // handed over by the producer (see the value stretch)
         mbar_wait(&bars->gready, 0, p.err);
@@ -1052,8 +1063,10 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
         const uint32_t bytes = (uint32_t)(runs * h) * (D * 2);
         mbar_expect_tx(&bars->full[sk], bytes);
         mbar_expect_tx(&bars->full[sv], bytes);
-        const CUtensorMap* mk = children ? &p.tm_kc : &p.tm_kr;
-        const CUtensorMap* mv = children ? &p.tm_vc : &p.tm_vr;
+        // children of level cl: level 1's own maps, the middle levels' from their arrays
+        const CUtensorMap* mk = children ? (cl == 1 ? &p.tm_kc : &p.tm_kcm[cl - 2]) : &p.tm_kr;
+        const CUtensorMap* mv = children ? (cl == 1 ? &p.tm_vc : &p.tm_vcm[cl - 2]) : &p.tm_vr;
+        const long long nch = children ? (long long)lvl_n(p, cl) : 0;
         for (int r = uw * h; r < tma_rows; r += (NU / 32) * h) {
             const long long e = tab[r];
             if (e == -1) continue;
@@ -1061,7 +1074,7 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
             // the raw map), or the first child of a group in the row's level-1 gists
             int y, z;
             if (children) {
-                y = (int)(-e - 2 - (long long)row * p.N1);
+                y = (int)(-e - 2 - (long long)row * nch);
                 z = row;
             } else if (PG && p.table != nullptr) {
                 // pool rows are below 2^31 (checked on the host): 32-bit division
@@ -1099,42 +1112,60 @@ __device__ __forceinline__ void gather_tile(const Params& p, uint8_t* base, Bars
     }
 }
 
-// Hierarchy: the row table of the children tile: the level-1 gists of the k2
-// selected groups, group after group (a short last group leaves empty rows).
-__device__ __forceinline__ void hier_children_table(const Params& p, uint8_t* base, int row) {
-    const int32_t* sel2 = reinterpret_cast<const int32_t*>(base + SM_SEL);
+// The selection made at the start of unfold round rd (round 0: the top
+// level's), kept in shared memory; consecutive rounds alternate buffers, so a
+// round's selection never overwrites the parents it is read against.
+__device__ __forceinline__ int32_t* round_sel(uint8_t* base, int rd) {
+    return reinterpret_cast<int32_t*>(base + ((rd & 1) ? SM_SEL1 : SM_SEL));
+}
+
+// Hierarchy, round rd < L - 1: the row table of the children tile, the
+// level-(L-1-rd) gists of the groups that round rd's selection (one level up)
+// picked, group after group (a short last group leaves empty rows).
+__device__ __forceinline__ void hier_children_table(const Params& p, uint8_t* base, int row, int rd) {
+    const int cl = p.levels - 1 - rd;                 // the children's level
+    const int32_t* par = round_sel(base, rd);
+    const int kp = lvl_k(p, cl + 1), g = p.grp[cl - 1], nch = lvl_n(p, cl);
     int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
     for (int r = utid(); r < TILE; r += NU) {
         int32_t e = -1;
-        if (r < p.K * p.group) {
-            const int child = sel2[r / p.group] * p.group + r % p.group;
-            if (child < p.N1) e = (int32_t)(-((long long)row * p.N1 + child) - 2);
+        if (r < kp * g) {
+            const int child = par[r / g] * g + r % g;
+            if (child < nch) e = (int32_t)(-((long long)row * nch + child) - 2);
         }
         tab[r] = e;
     }
     usync();
 }
 
-// Hierarchy: the exact top-k1 of the children tile's scores (ties to the
-// lower level-1 index: the tile holds the children in ascending order),
-// published as idx1 and kept in shared memory, then the row table of the
-// raw tokens of those k1 chunks.
-__device__ __forceinline__ void hier_select_children(const Params& p, uint8_t* base, int row) {
+// Hierarchy, round rd >= 1: the exact top-k of the children tile that round
+// rd - 1 attended and scored (level L - rd; ties to the lower index: the tile
+// holds the children in ascending order), published and kept as round rd's
+// selection; then the next table: that level's children, or at level 1 the
+// raw tokens of the selected chunks.
+__device__ __forceinline__ void hier_select_children(const Params& p, uint8_t* base, int row, int rd) {
+    const int lv = p.levels - rd;                     // the level selected here
     const uint32_t* keys = reinterpret_cast<const uint32_t*>(base + SM_CKEY);
-    const int32_t* sel2 = reinterpret_cast<const int32_t*>(base + SM_SEL);
-    int32_t* sel1 = reinterpret_cast<int32_t*>(base + SM_SEL1);
+    const int32_t* par = round_sel(base, rd - 1);
+    int32_t* sel1 = round_sel(base, rd);
     int32_t* res = reinterpret_cast<int32_t*>(base + SM_HRES);
     uint32_t* scratch = reinterpret_cast<uint32_t*>(base + SM_HSCR);
-    const int n = min(TILE, p.K * p.group);
-    const int k = p.K1;
+    const int g = p.grp[lv - 1];
+    const int n = min(TILE, lvl_k(p, lv + 1) * g);
+    const int k = lvl_k(p, lv);
+    int32_t* out = lvl_idx(p, lv);
     unfold_topk(keys, SRC_SKEY, n, k, res, scratch, reinterpret_cast<int32_t*>(base + SM_MISC), nullptr, nullptr, 0);
     for (int r = utid(); r < k; r += NU) {
         const int pos = res[r];
-        const int child = sel2[pos / p.group] * p.group + pos % p.group;
+        const int child = par[pos / g] * g + pos % g;
         sel1[r] = child;
-        p.idx1[(size_t)row * p.K1 + r] = child;
+        out[(size_t)row * k + r] = child;
     }
     usync();
+    if (lv > 1) {
+        hier_children_table(p, base, row, rd);
+        return;
+    }
     int32_t* tab = reinterpret_cast<int32_t*>(base + SM_ROWTAB);
     for (int r = utid(); r < TILE; r += NU) {
         int32_t e = -1;
@@ -1373,7 +1404,9 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
         g0 = (a - ru0) * TILE;
         g1 = b > a ? min((b - ru0) * TILE, p.NA) : g0;
     };
-    const int rounds = p.hier ? (p.K1 > 0 ? 2 : 1) : 1;
+    // the hierarchy's rounds: one children tile per level below the top, then
+    // the raw tile of the level-1 selection (none when k1 = 0)
+    const int rounds = p.hier ? (p.K1 > 0 ? p.levels : p.levels - 1) : 1;
     // gathered tiles of unfold item `it`, round rd: [t0, t0 + ntl) of its row
     auto item_tiles = [&](int it, int rd, int& t0) {
         if (p.hier) {
@@ -1436,7 +1469,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                 rg.seq0 = gseq;
                 rg.npre = ntl;   // every tile is gathered by the unfold warps
                 rg.slot_b = p.maxs + (p.hier ? rd : it % p.cb);
-                rg.score = (p.hier && rd == 0) ? 1 : 0;
+                rg.score = (p.hier && rd < p.levels - 1) ? 1 : 0;   // children tiles are scored
                 run_pipeline<G, PG>(p, cx, rg);
                 gseq += 2 * ntl;
             }
@@ -1496,8 +1529,8 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                     if (lead) mbar_wait(&cx.bars->gdone, (runs - 1) & 1, p.err);
                     usync();
                 }
-                if (rd == 1) {
-                    hier_select_children(p, cx.base, row);
+                if (rd >= 1) {
+                    hier_select_children(p, cx.base, row, rd);
                 } else {
                     if (p.do_topk && p.sel_direct) {
                         direct_select<PG>(p, cx.base, row, j == 0);
@@ -1512,16 +1545,17 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                     } else {
                         load_selection(p, cx.base, row);
                     }
-                    if (p.hier) hier_children_table(p, cx.base, row);
+                    if (p.hier) hier_children_table(p, cx.base, row, 0);
                     else build_table<PG>(p, cx.base, row, t0, ntl);
                 }
                 for (int lt = 0; lt < ntl; ++lt) {
                     // leading rows that are whole runs of consecutive source rows
                     int tma_rows = 0, h = p.C;
-                    const bool children = p.hier && rd == 0;
+                    const bool children = p.hier && rd < p.levels - 1;
+                    const int cl = children ? p.levels - 1 - rd : 0;   // the children's level
                     if (children) {
-                        h = p.group;
-                        tma_rows = p.tma_children ? min(TILE, p.K * p.group) : 0;
+                        h = p.grp[cl - 1];
+                        tma_rows = p.tma_children ? min(TILE, lvl_k(p, cl + 1) * h) : 0;
                     } else if (p.tma_raw) {
                         // rows of the selected chunks in this tile (the hierarchy's raw
                         // round keeps its one tile at table index 0)
@@ -1529,7 +1563,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_decode_kernel(const __grid_cons
                         const int tile = p.hier ? lt : t0 + lt;
                         tma_rows = max(0, min(TILE, kc - tile * TILE));
                     }
-                    gather_tile<PG>(p, cx.base, cx.bars, lt, gseq + 2 * lt, row, tma_rows, h, children, gseq0);
+                    gather_tile<PG>(p, cx.base, cx.bars, lt, gseq + 2 * lt, row, tma_rows, h, children, gseq0, cl);
                 }
                 gseq += 2 * ntl;
                 ++runs;
@@ -1975,6 +2009,128 @@ gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const v
     p.group = h.group;
     p.N1 = d.n_chunks;
     p.K1 = d.top_k;
+    p.levels = 2;
+    p.grp[0] = h.group;
+    return launch(p, f.G, f.grid, st) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+// --------------------------------------------------- hierarchy, any depth ----
+constexpr int kFusedMaxLevels = 4;   // the middle levels' maps in Params (levels 2 .. L-1)
+
+bool fused_levels_supported(const gsa_levels_desc& h) {
+    using namespace fused;
+    const gsa_decode_desc& d = h.l1;
+    const int L = h.levels;
+    if (L < 2 || L > kFusedMaxLevels) return false;
+    if (L > 2 && h.l1.top_k < 1) return false;   // (no raw round: the CUDA-core passes)
+    int n[GSA_MAX_LEVELS];
+    level_counts(h, n);
+    const long long rows = (long long)d.batch * d.n_kv_heads;
+    const long long units = rows * ((n[L - 1] + 127) / 128 + (d.tail_len + 127) / 128);
+    if (!(d.dtype == GSA_BF16 && d.head_dim == 128 && (long long)d.top_k * d.chunk <= 128 &&
+          rows * d.n_chunks * d.chunk < INT32_MAX - 2 && rows * d.n_chunks < INT32_MAX - 2 && units < (1LL << 30) &&
+          d.n_q_heads % d.n_kv_heads == 0))
+        return false;
+    // every level's children of the selection above: one tile, gathered in whole
+    // groups by TMA (the two-level step also takes other groups, by cp.async)
+    for (int l = 1; l < L; ++l) {
+        const int g = h.group[l - 1];
+        if ((long long)level_k(h, l) * g > 128 || (L > 2 && !chunk_runs(g))) return false;
+    }
+    return make_fused_levels_plan(h).tmem_cols <= 512;
+}
+
+FusedPlan make_fused_levels_plan(const gsa_levels_desc& h) {
+    const int L = h.levels;
+    int n[GSA_MAX_LEVELS];
+    level_counts(h, n);
+    // the key and value stretches and the top selection are the flat step
+    // over the top level's gists
+    gsa_decode_desc top = h.l1;
+    top.n_chunks = n[L - 1];
+    top.top_k = level_k(h, L - 1);
+    top.mode = GSA_ALL_GISTS;
+    FusedPlan f = make_fused_plan(top);
+    // unfold: one item per row, a partial slot per round (a children tile per
+    // level below the top, the raw tile)
+    f.nbt = L;
+    f.tpc = L;
+    f.cb = 1;
+    place_ctas(f, L);
+    // the lower levels' selections when the caller passes none: level 1, then 2 .. L-1
+    size_t lower = 0;
+    for (int l = 0; l < L - 1; ++l) lower += (size_t)level_k(h, l);
+    layout_ws(f, (size_t)n[L - 1], (size_t)top.top_k, lower);
+    return f;
+}
+
+gsa_status fused_levels_launch(const gsa_levels_desc& h, const FusedPlan& f, const void* q, const void* const* kg,
+                               const void* const* vg, const void* kr, const void* vr, const void* kt, const void* vt,
+                               int32_t* const* idx_out, void* out, void* ws, cudaStream_t st) {
+    using namespace fused;
+    const gsa_decode_desc& d = h.l1;
+    const int L = h.levels;
+    if (f.grid <= 0 || L > kFusedMaxLevels) return GSA_ERR_ARG;
+    int n[GSA_MAX_LEVELS];
+    level_counts(h, n);
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t rows = (uint64_t)f.rows;
+    bool ok = map3d(&p.tm_kg, kg[L - 1], rows, (uint64_t)n[L - 1]) &&
+              map3d(&p.tm_vg, vg[L - 1], rows, (uint64_t)n[L - 1]) &&
+              map3d(&p.tm_kt, kt, rows, (uint64_t)d.tail_len) && map3d(&p.tm_vt, vt, rows, (uint64_t)d.tail_len);
+    p.tma_raw = chunk_runs(d.chunk) && d.top_k > 0 ? 1 : 0;
+    p.tma_children = chunk_runs(h.group[0]) ? 1 : 0;   // (every group, from three levels on)
+    const uint64_t n1 = (uint64_t)d.n_chunks;
+    if (p.tma_raw)
+        ok = ok && map3d(&p.tm_kr, kr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk) &&
+             map3d(&p.tm_vr, vr, rows, n1 * (uint64_t)d.chunk, (uint32_t)d.chunk);
+    if (p.tma_children)
+        ok = ok && map3d(&p.tm_kc, kg[0], rows, n1, (uint32_t)h.group[0]) &&
+             map3d(&p.tm_vc, vg[0], rows, n1, (uint32_t)h.group[0]);
+    for (int l = 2; l < L; ++l)
+        ok = ok && map3d(&p.tm_kcm[l - 2], kg[l - 1], rows, (uint64_t)n[l - 1], (uint32_t)h.group[l - 1]) &&
+             map3d(&p.tm_vcm[l - 2], vg[l - 1], rows, (uint64_t)n[l - 1], (uint32_t)h.group[l - 1]);
+    if (!ok) return GSA_ERR_CUDA;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    fill_common(p, f, d, w);
+    p.q = static_cast<const uint16_t*>(q);
+    p.kr = static_cast<const uint8_t*>(kr);
+    p.vr = static_cast<const uint8_t*>(vr);
+    p.kgp = static_cast<const uint8_t*>(kg[0]);   // gathered "gist" rows are level-1 gists (two levels, cp.async)
+    p.vgp = static_cast<const uint8_t*>(vg[0]);
+    p.out = static_cast<uint16_t*>(out);
+    p.lse = nullptr;
+    p.scores = reinterpret_cast<float*>(w + f.off_scores);
+    // selections: the caller's, else workspace (level 1, then 2 .. L-1, after the top level's)
+    auto sel_of = [&](int l, size_t& off) -> int32_t* {
+        int32_t* given = idx_out ? idx_out[l - 1] : nullptr;
+        int32_t* mine = reinterpret_cast<int32_t*>(w + f.off_idx1 + off);
+        off += (size_t)f.rows * level_k(h, l - 1) * 4;
+        return given ? given : mine;
+    };
+    size_t off = 0;
+    p.idx1 = sel_of(1, off);
+    for (int l = 2; l < L; ++l) p.midIdx[l - 2] = sel_of(l, off);
+    p.idx = (idx_out && idx_out[L - 1]) ? idx_out[L - 1] : reinterpret_cast<int32_t*>(w + f.off_idx);
+    p.N = n[L - 1];
+    p.NA = n[L - 1];
+    p.K = level_k(h, L - 1);
+    p.mode = GSA_ALL_GISTS;
+    p.nrows_g = 0;
+    p.do_score = 1;
+    p.do_topk = 1;
+    p.do_attn_gists = 1;
+    p.hier = 1;
+    p.group = h.group[0];
+    p.N1 = d.n_chunks;
+    p.K1 = d.top_k;
+    p.levels = L;
+    for (int l = 1; l < L; ++l) p.grp[l - 1] = h.group[l - 1];
+    for (int l = 2; l < L; ++l) {
+        p.midN[l - 2] = n[l - 1];
+        p.midK[l - 2] = level_k(h, l - 1);
+    }
     return launch(p, f.G, f.grid, st) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 

@@ -66,6 +66,14 @@ struct Params {
     // hierarchy (keys/values: level-2 gists; unfold: children tile, then raw tile)
     int hier, group, N1, K1;       // K = k2, N = NA = n_l2; group, level-1 gists, k1
     int32_t* idx1;                 // [rows][k1]
+    // any depth: L = levels (2 for the two-level step; K, N are the top level's);
+    // grp[l - 1] level-l gists per level-(l + 1) gist; the middle levels 2 .. L-1:
+    // gist counts, selection sizes, selection outputs, gist maps (box {64, grp[l - 1], 1})
+    int levels;
+    int grp[3];
+    int midN[2], midK[2];
+    int32_t* midIdx[2];
+    CUtensorMap tm_kcm[2], tm_vcm[2];
 };
 }  // namespace fused
 
@@ -74,6 +82,16 @@ bool fused_supported(const gsa_decode_desc& d);
 // fit one 128-row tile, and so must the raw tokens of the k1 chunks.
 bool fused_hier_supported(const gsa_hier_desc& h);
 FusedPlan make_fused_hier_plan(const gsa_hier_desc& h);
+// Any depth on the same kernel (up to 4 levels): each level's children of the
+// selection above must fit one 128-row tile (by TMA: the groups are whole
+// 16-byte-aligned runs), and so must the raw tokens of the level-1 selection.
+bool fused_levels_supported(const gsa_levels_desc& h);
+FusedPlan make_fused_levels_plan(const gsa_levels_desc& h);
+// kg / vg: host arrays of the L levels' gist tensors, level 1 first; idx_out:
+// null or a host array of L nullable selection outputs.
+gsa_status fused_levels_launch(const gsa_levels_desc& h, const FusedPlan& f, const void* q, const void* const* kg,
+                               const void* const* vg, const void* kr, const void* vr, const void* kt, const void* vt,
+                               int32_t* const* idx_out, void* out, void* ws, cudaStream_t st);
 gsa_status fused_hier_launch(const gsa_hier_desc& h, const FusedPlan& f, const void* q, const void* k_g2,
                              const void* v_g2, const void* k_g1, const void* v_g1, const void* kr, const void* vr,
                              const void* kt, const void* vt, int32_t* idx2_out, int32_t* idx1_out, void* out,

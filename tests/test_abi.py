@@ -154,6 +154,9 @@ def test_every_benchmark_decode_workload_takes_the_one_launch_path():
         elif isinstance(w, synth.HierShape):
             hd = gsa.hier_desc(desc_of(w.l1), w.n_l2, w.group, w.top_k2)
             assert gsa.gsa_hier_launch_count(hd) == 1, name
+        elif isinstance(w, synth.LevelsShape):
+            ld = gsa.levels_desc(desc_of(w.l1), w.groups, w.top_ks)
+            assert gsa.gsa_levels_launch_count(ld) == 1, name
 
 
 def test_host_buffer_step_argument_checks():

@@ -21,6 +21,8 @@ from gsa_check import check_out, desc_of, dev, host, tdtype, workspace
 SHAPES = {
     # 65536 raw tokens, 4096 -> 512 -> 64 gists, k = 8 / 16 / 4
     "l3_bf16": LevelsShape(DecodeShape(2, 32, 8, 128, 4096, 16, 8, 64, "bf16", n_needles=4), (8, 8), (16, 4)),
+    # four levels on the tensor-core path: 8192 -> 1024 -> 128 -> 16 gists, k = 8 / 16 / 8 / 4
+    "l4_bf16": LevelsShape(DecodeShape(1, 32, 8, 128, 8192, 16, 8, 64, "bf16", n_needles=4), (8, 8, 8), (16, 8, 4)),
     # 2000 chunks, 2000 -> 400 -> 100 -> 25 gists, k = 6 / 12 / 6 / 3
     "l4_f32": LevelsShape(DecodeShape(2, 4, 2, 64, 2000, 8, 6, 16, "f32", n_needles=3), (5, 4, 4), (12, 6, 3)),
 }
@@ -112,6 +114,15 @@ def test_levels_depth_two_matches_the_two_level_oracle():
     _, _, want = oracle.hier_decode(t, 16, 8, 8, given=(idx[1], idx[0]))
     check_out(out, want, "bf16", "depth 2")
     assert h2.group == 16
+
+
+def test_levels_paths():
+    """bf16 with d = 128 and every level's children within one tile: one
+    tensor-core launch (up to four levels); otherwise the CUDA-core passes."""
+    for name, launches in (("l3_bf16", 1), ("l4_bf16", 1), ("l4_f32", 5)):
+        assert gsa.gsa_levels_launch_count(_desc(SHAPES[name])) == launches, name
+    five = LevelsShape(DecodeShape(1, 32, 8, 128, 65536, 16, 8, 64, "bf16"), (8, 8, 8, 8), (8, 8, 8, 4))
+    assert gsa.gsa_levels_launch_count(_desc(five)) == 6
 
 
 def test_levels_descriptor_checks():

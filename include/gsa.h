@@ -274,7 +274,10 @@ gsa_status gsa_hier_decode(const gsa_hier_desc* desc, const void* q, const void*
  *   k_gists, v_gists: HOST arrays of L device pointers, level 1 first, level
  *   l's gists [B][Hkv][n_l][d]; raw and tail as for gsa_decode_step;
  *   idx_out: NULL or a HOST array of L nullable device pointers, level l's
- *   selection [B][Hkv][k_l] (ascending).  Runs as L + 1 launches of the
+ *   selection [B][Hkv][k_l] (ascending).  One launch of the tensor-core
+ *   step (bf16, d = 128, up to four levels, each level's children of the
+ *   selection above within 128 rows and, beyond two levels, in groups of a
+ *   multiple of 8 dividing 128; k1 c <= 128); otherwise L + 1 launches of the
  *   CUDA-core passes (bf16 or fp32, d = 64 or 128).                        */
 gsa_status gsa_levels_decode(const gsa_levels_desc* desc, const void* q, const void* const* k_gists,
                              const void* const* v_gists, const void* k_raw, const void* v_raw,

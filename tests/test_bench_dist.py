@@ -1,11 +1,13 @@
 """The multi-rank host logic of bench.py on CPU: two gloo ranks, one process
 each (the GPU runs use the same code with NCCL).  Checks the max-over-ranks
-timing reduction, the whole-job rate, and that only rank 0 prints."""
+timing reduction, the whole-job rate, that only rank 0 prints, and the keys of
+the reference arm's line."""
 import os
 import socket
 import subprocess
 import sys
 
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -55,3 +57,34 @@ def test_reference_arm_prints_only_on_rank_zero():
                           "--warmup", "3", "--workload", "tiny_f32"], env=env, capture_output=True, text=True,
                          timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("workload", ["tiny_f32", "suffix_stage2"])
+def test_reference_arm_line_carries_the_contract_keys(workload):
+    """Rank 0 of the reference arm prints one JSON line with the contract's
+    keys, its cpu_baseline and e2e repeating the line's own value, and the
+    same config keys as the GPU arm's line for that workload."""
+    import json
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "3", "--workload", workload], env=env, capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["config"]["workload"] == workload
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    w = synth.WORKLOADS[workload]
+    if isinstance(w, synth.SuffixShape):
+        gpu_cfg = bench.suffix_config(w, workload, 1, 2, bench.l2_bytes())
+    else:
+        gpu_cfg = bench.decode_config(w, workload, 1, 2, bench.algorithmic_bytes(w), bench.l2_bytes())
+    assert set(d["config"]) == set(gpu_cfg)

@@ -790,3 +790,25 @@ def test_topp_ties_take_the_lower_index_first():
         idx, cnt = oracle.topp(s, p, 5, math.log(2.0))
         assert idx[0, :cnt[0]].tolist() == want, p
         assert (idx[0, cnt[0]:] == -1).all()
+
+
+def test_levels_ragged_groups_reduce_to_the_two_level_step():
+    """Ragged groups at every level (301 -> 61 -> 16 gists: the last groups
+    hold 1 and 1 children).  With every level-3 gist selected and its keys
+    silenced (weight exactly 0 in fp64), the three-level step is the
+    two-level step (pinned above) over levels 2 and 1, bit for bit."""
+    d = 8
+    h = synth.LevelsShape(DecodeShape(1, 2, 2, d, 301, 2, 4, 3, "f32", n_needles=0), (5, 4), (6, 16))
+    assert h.counts == [301, 61, 16]
+    x = synth.levels_inputs(h, 87)
+    qw = x.q.astype(np.float64)
+    for hk in range(2):
+        x.k_g[2][0, hk, :] = (-1e4 * qw[0, hk] / np.linalg.norm(qw[0, hk])).astype(np.float32)
+    idx, out = _levels(x, h)
+    assert np.all(idx[2] == np.arange(16))
+    t = dict(q=x.q, k_g2=x.k_g[1], v_g2=x.v_g[1], k_g1=x.k_g[0], v_g1=x.v_g[0], k_raw=x.k_raw, v_raw=x.v_raw,
+             k_tail=x.k_tail, v_tail=x.v_tail)
+    i2, i1, o = oracle.hier_decode(t, 5, 6, 4)
+    np.testing.assert_array_equal(idx[1], i2)
+    np.testing.assert_array_equal(idx[0], i1)
+    np.testing.assert_allclose(out, o, rtol=0, atol=1e-13)

@@ -90,9 +90,10 @@ constexpr uint32_t SM_SCORE = SM_MISC + 1024;        // key stretch: this CTA's 
 constexpr int kScoreCap = 3072;                      // scores kept in shared memory
 constexpr uint32_t SM_SEL = SM_SCORE;                // unfold stretch: the row's selection [kSelCap]
 constexpr uint32_t SM_ROWTAB = SM_SEL + kSelCap * 4; // unfold stretch: source of each gathered row [kMaxTpc][128]
-// hierarchy: the level-2 selection at SM_SEL [k2 <= 512], the children tile's
-// score keys [128], the level-1 selection [k1 <= 128], the children top-k's
-// result [128] and scratch after it
+// hierarchy: the top level's selection at SM_SEL [<= 512], the children tile's
+// score keys [128], a lower level's selection [<= 128] (rounds alternate
+// between SM_SEL1 and SM_SEL), the children top-k's result [128] and scratch
+// after it
 constexpr uint32_t SM_CKEY = SM_SEL + 512 * 4;
 constexpr uint32_t SM_SEL1 = SM_CKEY + TILE * 4;
 constexpr uint32_t SM_HRES = SM_SEL1 + TILE * 4;
@@ -771,7 +772,7 @@ __device__ __forceinline__ void gathered_softmax(const Params& p, Ctx& cx, const
     cx.ptiles = pj + 1;
     cx.had_attn = 1;
     if (u.score) {
-        // hierarchy: the level-1 scores of the children tile, as keys for the k1 selection
+        // hierarchy: the scores of the children tile, as keys for the next level's selection
         float score = 0.f;
 #pragma unroll
         for (int h = 0; h < G; ++h) score += __uint_as_float(r[h]);
@@ -1778,7 +1779,7 @@ static void place_ctas(FusedPlan& f, int nb_slots) {
 }
 
 // Workspace: tickets and key counters [2][rows], scores, candidates, idx,
-// partials, (m, l) (and the hierarchy's idx1).
+// partials, (m, l) (and the hierarchy's lower-level selections).
 static void layout_ws(FusedPlan& f, size_t N, size_t top_k, size_t k1) {
     const size_t rows = (size_t)f.rows;
     size_t o = round256(kWsCntOffset + 2 * rows * 4);

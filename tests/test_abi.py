@@ -170,3 +170,21 @@ def test_host_buffer_step_argument_checks():
             gsa.gsa_decode_step_host(desc, q_host, *dev_args, idx_out, idx_host, 1 << 20, out_host, 1 << 20,
                                      stream=0, ws_bytes=1 << 30)
         assert e.value.status == gsa.GSA_ERR_ARG
+
+
+def test_levels_path_choice():
+    """The any-depth hierarchy takes the one-launch tensor-core step only for
+    bf16, d = 128, at most four levels, every children tile within 128 rows
+    (and, beyond two levels, groups that are whole TMA runs), k1 c <= 128."""
+    bf = lambda N, c, k1: gsa.decode_desc(1, 32, 8, 128, N, c, k1, 64, gsa.GSA_BF16)
+    cases = [
+        (bf(4096, 16, 8), (8, 8), (16, 4), 1),
+        (bf(4096, 16, 8), (16,), (8,), 1),                  # two levels through the same entry point
+        (bf(4096, 16, 8), (5, 8), (16, 4), 4),              # a group of 5 is not a whole TMA run
+        (bf(4096, 16, 8), (8, 8), (32, 4), 4),              # 32 x 8 = 256 children at level 1
+        (bf(4096, 16, 16), (8, 8), (16, 4), 4),             # 16 x 16 = 256 raw rows
+        (bf(65536, 16, 8), (8, 8, 8, 8), (8, 8, 8, 4), 6),  # five levels
+        (gsa.decode_desc(1, 8, 2, 64, 4096, 16, 8, 64, gsa.GSA_F32), (8, 8), (16, 4), 4),
+    ]
+    for l1, groups, ks, launches in cases:
+        assert gsa.gsa_levels_launch_count(gsa.levels_desc(l1, groups, ks)) == launches, (groups, ks)

@@ -61,10 +61,16 @@ def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(tmp_path, m
     for f in os.listdir(os.path.join(ROOT, "profiles")):
         shutil.copy(os.path.join(ROOT, "profiles", f), tmp_path / "profiles" / f)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    t = bench.measured_traffic("llama8b_decode")
-    if t is None:
-        pytest.skip("the committed decode profile predates the current kernel sources")
-    assert t > 0
+    # a profile stating these sources' digest (as a fresh capture would)
+    import hashlib
+    h = hashlib.sha256()
+    for f in bench.KERNEL_SOURCES:
+        h.update((csrc / f).read_bytes())
+    (tmp_path / "profiles" / "fresh_capture.md").write_text(
+        "# capture\n\nworkload: llama8b_decode\ndram_bytes_per_step: 80000000\nlaunches_per_step: 2\n"
+        f"sources_sha256: {h.hexdigest()}\n")
+    assert bench.measured_traffic("llama8b_decode") == 40_000_000    # per launch
+    assert bench.traffic_source("llama8b_decode").endswith("fresh_capture.md")
     assert bench.measured_traffic("no_such_workload") is None
     # any edit of a kernel source voids the figure
     with open(csrc / bench.KERNEL_SOURCES[0], "a") as fh:

@@ -19,7 +19,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Tensors are dense, row-major, caller-owned DEVICE pointers (16-byte
- *    aligned).  Shapes use B batch, Hq query heads, Hkv KV heads
+ *    aligned), except where a declaration says HOST (gsa_decode_step_host's
+ *    query and result buffers; gsa_levels_decode's arrays of pointers).  Shapes use B batch, Hq query heads, Hkv KV heads
  *    (G = Hq / Hkv query heads share one KV head: head h reads KV head h / G),
  *    d head_dim, N chunks (= gists), c raw tokens per chunk, k top-k,
  *    W uncompressed tail tokens:
@@ -48,9 +49,10 @@
  *    a failing check returns an error code and enqueues nothing.  A CUDA
  *    launch failure returns GSA_ERR_CUDA.  Nothing is printed, no exception
  *    crosses the ABI.  Device-side anomalies (an out-of-range chunk index
- *    passed to gsa_unfold_attn, an expired bounded wait) never fault: the
- *    kernel clamps the index into range (or abandons the wait) and ORs a flag
- *    into an error word.  Entry points that take a workspace use the word at
+ *    passed to gsa_unfold_attn, a page index or a chunk count out of range
+ *    in gsa_decode_step_paged, an expired bounded wait) never fault: the
+ *    kernel clamps the value into range (or abandons the wait) and ORs a
+ *    flag into an error word.  Entry points that take a workspace use the word at
  *    its start, read back by gsa_workspace_error(); the others
  *    (gsa_score, gsa_gist_prefill, gsa_decode_step_noalloc) use words of
  *    the library, read back and cleared by gsa_device_error().  A call whose

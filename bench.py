@@ -934,7 +934,9 @@ def run_levels(args, world, rank, local):
                    "ms_per_step_min": round(min(reps_ms) / args.steps, 5),
                    "ms_per_step_max": round(max(reps_ms) / args.steps, 5)},
         "algorithmic_bytes_per_step": nbytes,
-        "roofline": {"bound": "hbm", "kernel": f"gsa_levels_decode (whole step, {launches} launches)",
+        "roofline": {"bound": "hbm",
+                     "kernel": (f"gsa_levels_decode: one launch of fused_decode_kernel per step" if launches == 1 else
+                                f"gsa_levels_decode (whole step, {launches} launches)"),
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                      "peak_kind": peak_kind, "traffic": None, "traffic_source": "none"},
         "e2e": {"value": round(whole_job_rate(args.steps, world, e2e_ms), 2), "unit": "steps/s",
